@@ -1,0 +1,265 @@
+"""Pins for the fp64 HLA oracle (CPU only).
+
+Each test pins the oracle to something other than itself: the plain token-by-token
+gated delta rule, exact rational brute force with explicit per-token matrices,
+closed forms, special cases and invariants that the definition fixes.  Source
+passages: HLA summary page, "Methodology in Plain English" (affine per-token rule;
+exact chunk summaries; weight 1 keeps the transition, weight 0 leaves the state
+untouched; current chunk weight one, future masked; threshold skip is exact) and
+"Key Contributions" 2-3.
+"""
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+from oracle import hla_oracle as ho
+from oracle import brute
+from oracle import routing_recipe as rr
+
+
+def _head(rng, T, dk, dv=None, bf16_like=False):
+    dv = dk if dv is None else dv
+    q = rng.standard_normal((T, dk))
+    k = rng.standard_normal((T, dk))
+    q /= np.linalg.norm(q, axis=1, keepdims=True)
+    k /= np.linalg.norm(k, axis=1, keepdims=True)
+    v = rng.standard_normal((T, dv))
+    alpha = np.exp(-np.log1p(np.exp(rng.standard_normal(T) - 3.0)))
+    beta = 1.0 / (1.0 + np.exp(-rng.standard_normal(T)))
+    if bf16_like:
+        q, k, v = (x.astype(np.float32) for x in (q, k, v))
+    return q, k, v, alpha, beta
+
+
+# ---- chunk transitions ------------------------------------------------------------
+
+@pytest.mark.parametrize("n,d,dv", [(8, 5, 6), (16, 12, 12), (64, 128, 128)])
+def test_wy_form_equals_literal_transition(n, d, dv):
+    rng = np.random.default_rng(n + d)
+    _, k, v, a, b = _head(rng, n, d, dv)
+    A, B = ho.chunk_transition(k, v, a, b)
+    A2, B2, Wb, Ub, ell = ho.chunk_transition_wy(k, v, a, b)
+    assert np.abs(A - A2).max() <= 1e-12
+    assert np.abs(B - B2).max() <= 1e-12
+
+
+def test_composition_law_two_chunks():
+    rng = np.random.default_rng(11)
+    _, k, v, a, b = _head(rng, 16, 6)
+    A1, B1 = ho.chunk_transition(k[:8], v[:8], a[:8], b[:8])
+    A2, B2 = ho.chunk_transition(k[8:], v[8:], a[8:], b[8:])
+    A, B = ho.chunk_transition(k, v, a, b)
+    assert np.abs(A - A1 @ A2).max() <= 1e-13
+    assert np.abs(B - (B1 @ A2 + B2)).max() <= 1e-13
+
+
+def test_transition_contraction():
+    # eigenvalues of I - beta k k^T lie in [1 - beta, 1] for unit k, so ||A_c||_2 <= gamma_C
+    rng = np.random.default_rng(12)
+    for _ in range(5):
+        _, k, v, a, b = _head(rng, 64, 32)
+        A, _ = ho.chunk_transition(k, v, a, b)
+        gamma = np.prod(a)
+        assert np.linalg.norm(A, 2) <= gamma * (1 + 1e-12)
+
+
+def test_identity_transition_alpha1_beta0():
+    rng = np.random.default_rng(13)
+    q, k, v, _, _ = _head(rng, 24, 8)
+    a = np.ones(24)
+    b = np.zeros(24)
+    A, B = ho.chunk_transition(k[:8], v[:8], a[:8], b[:8])
+    assert np.array_equal(A, np.eye(8)) and np.array_equal(B, np.zeros((8, 8)))
+    r = ho.hla_prefill_head(q, k, v, a, b, 8, bias=1.0)
+    assert np.array_equal(r.o, np.zeros_like(r.o))
+
+
+# ---- prefill reductions ----------------------------------------------------------
+
+def test_T1_closed_form():
+    rng = np.random.default_rng(14)
+    q, k, v, a, b = _head(rng, 1, 16)
+    r = ho.hla_prefill_head(q, k, v, a, b, 64)
+    np.testing.assert_allclose(r.o[0], b[0] * (k[0] @ q[0]) * v[0], rtol=1e-14, atol=1e-15)
+
+
+def test_single_chunk_equals_gdn():
+    rng = np.random.default_rng(15)
+    q, k, v, a, b = _head(rng, 50, 16)
+    r = ho.hla_prefill_head(q, k, v, a, b, 64, bias=-3.0)
+    o, _ = ho.gdn_recurrent(q, k, v, a, b)
+    assert np.abs(r.o - o).max() <= 1e-13
+
+
+@pytest.mark.parametrize("T", [64, 70])
+def test_gates_one_is_native_gdn(T):
+    rng = np.random.default_rng(16 + T)
+    q, k, v, a, b = _head(rng, T, 12)
+    r = ho.hla_prefill_head(q, k, v, a, b, 8, gate_mode=ho.GATES_ONE)
+    o, _ = ho.gdn_recurrent(q, k, v, a, b)
+    assert np.abs(r.o - o).max() <= 1e-12
+
+
+def test_gates_zero_leaves_intra_chunk_only():
+    rng = np.random.default_rng(17)
+    q, k, v, a, b = _head(rng, 40, 12)
+    r = ho.hla_prefill_head(q, k, v, a, b, 8, gate_mode=ho.GATES_ZERO)
+    for c in range(5):
+        sl = slice(8 * c, 8 * c + 8)
+        o, _ = ho.gdn_recurrent(q[sl], k[sl], v[sl], a[sl], b[sl])
+        assert np.abs(r.o[sl] - o).max() <= 1e-14
+
+
+def test_two_chunks_output_affine_in_gate():
+    rng = np.random.default_rng(18)
+    q, k, v, a, b = _head(rng, 16, 6)
+    outs = []
+    for g in (0.0, 0.3, 1.0):
+        ug = np.zeros((2, 2))
+        ug[1, 0] = g
+        outs.append(ho.hla_prefill_head(q, k, v, a, b, 8, gate_mode=ho.GATES_USER, user_gates=ug).o)
+    # S_in(1) = g B_0, chunk 1 output is affine in g (gates are binary32 values)
+    interp = outs[0] + float(np.float32(0.3)) * (outs[2] - outs[0])
+    assert np.abs(outs[1] - interp).max() <= 1e-13
+    # chunk 0 never sees the gate
+    assert np.array_equal(outs[0][:8], outs[2][:8])
+    # with g = 1 the state entering chunk 1 is B_0: compare against the token rule
+    o, S8 = ho.gdn_recurrent(q[:8], k[:8], v[:8], a[:8], b[:8])
+    o2, _ = ho.gdn_recurrent(q[8:], k[8:], v[8:], a[8:], b[8:], S0=S8)
+    assert np.abs(outs[2][8:] - o2).max() <= 1e-13
+
+
+def test_skip_is_exactly_identity():
+    rng = np.random.default_rng(19)
+    T, d, C = 96, 8, 8
+    q, k, v, a, b = _head(rng, T, d)
+    qr = rng.standard_normal((T, d)) * 2
+    kr = rng.standard_normal((T, d)) * 2
+    r0 = ho.hla_prefill_head(q, k, v, a, b, C, bias=-1.0, q_route=qr, k_route=kr)
+    thr = float(np.median(r0.gates[np.tril_indices(T // C, -1)]))
+    r = ho.hla_prefill_head(q, k, v, a, b, C, bias=-1.0, thr=thr, q_route=qr, k_route=kr)
+    skipped = sum(i - len(x) for i, x in enumerate(r.active))
+    assert skipped > 10
+    ug = np.where(r.gates >= np.float32(thr), r.gates, 0).astype(np.float64)
+    r2 = ho.hla_prefill_head(q, k, v, a, b, C, gate_mode=ho.GATES_USER, user_gates=ug, thr=0.0)
+    assert np.array_equal(r.o, r2.o)
+
+
+def test_future_chunks_do_not_change_past_outputs():
+    rng = np.random.default_rng(20)
+    q, k, v, a, b = _head(rng, 64, 8)
+    r1 = ho.hla_prefill_head(q, k, v, a, b, 8, bias=0.5)
+    q2, k2, v2 = q.copy(), k.copy(), v.copy()
+    v2[40:] += 3.0
+    k2[40:] = np.roll(k2[40:], 1, axis=1)
+    r2 = ho.hla_prefill_head(q2, k2, v2, a, b, 8, bias=0.5)
+    assert np.array_equal(r1.o[:40], r2.o[:40])
+
+
+# ---- brute force ----------------------------------------------------------------
+
+def _frac(x):
+    return Fraction(float(x))
+
+
+@pytest.mark.parametrize("T,C,d", [(8, 2, 2), (8, 4, 3), (7, 4, 2), (6, 2, 4)])
+def test_exact_rational_brute_force(T, C, d):
+    rng = np.random.default_rng(100 + T * C * d)
+    q, k, v, a, b = _head(rng, T, d)
+    N = (T + C - 1) // C
+    ug = np.tril(rng.uniform(0, 1, (N, N)), -1).astype(np.float32)   # gates are binary32
+    r = ho.hla_prefill_head(q, k, v, a, b, C, gate_mode=ho.GATES_USER, user_gates=ug)
+    F = lambda M: [[_frac(x) for x in row] for row in np.atleast_2d(M)]
+    ob = brute.hla_brute(F(q), F(k), F(v), [_frac(x) for x in a], [_frac(x) for x in b], C,
+                         [[_frac(x) for x in row] for row in ug], zero=Fraction(0), one=Fraction(1))
+    exact = np.array([[float(x) for x in row] for row in ob])
+    assert np.abs(r.o - exact).max() <= 1e-13
+
+
+def test_brute_force_with_routed_thresholded_gates():
+    rng = np.random.default_rng(21)
+    T, C, d = 8, 2, 4
+    q, k, v, a, b = _head(rng, T, d)
+    qr = (rng.standard_normal((T, d)) * 3).astype(np.float32)
+    kr = (rng.standard_normal((T, d)) * 3).astype(np.float32)
+    r = ho.hla_prefill_head(q, k, v, a, b, C, bias=-0.5, thr=0.4, q_route=qr, k_route=kr)
+    assert any(len(x) < i for i, x in enumerate(r.active))
+    gates = [[float(g) for g in row] for row in r.gates]
+    ob = brute.hla_brute(q.tolist(), k.tolist(), v.tolist(), a.tolist(), b.tolist(), C, gates,
+                         active=[list(x) for x in r.active])
+    assert np.abs(r.o - np.array(ob)).max() <= 1e-13
+    # gates come from pools of the route tokens of each chunk
+    rq = np.stack([rr.lme_pool32(qr[c * C:(c + 1) * C], 1.0) for c in range(4)])
+    assert np.array_equal(r.rq, rq)
+
+
+# ---- decode -----------------------------------------------------------------------
+
+def _steps(rng, n, d):
+    out = []
+    for _ in range(n):
+        q, k, v, a, b = _head(rng, 1, d)
+        out.append((q[0], k[0], v[0], a[0], b[0]))
+    return out
+
+
+@pytest.mark.parametrize("T0", [16, 21])
+def test_decode_matches_prefill_of_extended_sequence(T0):
+    rng = np.random.default_rng(22 + T0)
+    C, d = 8, 6
+    q, k, v, a, b = _head(rng, T0, d)
+    qr = rng.standard_normal((T0, d)) * 2
+    kr = rng.standard_normal((T0, d)) * 2
+    st = ho.HlaDecodeHead.from_prefill(q, k, v, a, b, C, bias=-0.5, thr=0.3,
+                                       q_route=qr, k_route=kr)
+    toks = _steps(rng, 12, d)   # crosses a chunk boundary
+    for s, (tq, tk, tv, ta, tb) in enumerate(toks):
+        tqr = rng.standard_normal(d) * 2
+        tkr = rng.standard_normal(d) * 2
+        o = st.step(tq, tk, tv, ta, tb, tqr, tkr)
+        q = np.vstack([q, tq]); k = np.vstack([k, tk]); v = np.vstack([v, tv])
+        a = np.append(a, ta); b = np.append(b, tb)
+        qr = np.vstack([qr, tqr]); kr = np.vstack([kr, tkr])
+        ref = ho.hla_prefill_head(q, k, v, a, b, C, bias=-0.5, thr=0.3, q_route=qr,
+                                  k_route=kr, query_chunks=[(len(a) - 1) // C])
+        assert np.abs(o - ref.o[-1]).max() <= 1e-12
+    # closed chunks in the cache equal the literal transitions and pools
+    n = len(a) // C
+    assert len(st.trans) == n
+    A, B = ho.chunk_transition(k[(n - 1) * C:n * C], v[(n - 1) * C:n * C], a[(n - 1) * C:n * C],
+                               b[(n - 1) * C:n * C])
+    assert np.abs(st.trans[-1][0] - A).max() <= 1e-14
+    assert np.array_equal(st.rk[-1], rr.lme_pool32(kr[(n - 1) * C:n * C].astype(np.float32), 1.0))
+
+
+def test_decode_backward_chain_equals_forward_composition():
+    rng = np.random.default_rng(23)
+    C, d, T = 8, 6, 64
+    q, k, v, a, b = _head(rng, T, d)
+    trans = [ho.chunk_transition(k[c * C:(c + 1) * C], v[c * C:(c + 1) * C], a[c * C:(c + 1) * C],
+                                 b[c * C:(c + 1) * C]) for c in range(8)]
+    g = rng.uniform(0, 1, 8)
+    active = [0, 2, 3, 6, 7]
+    x = rng.standard_normal(d)
+    S = np.zeros((d, d))
+    for j in active:
+        S = S + g[j] * ((S @ trans[j][0] + trans[j][1]) - S)
+    y = ho.decode_output_backward(trans, g, active, x, np.zeros(d))
+    assert np.abs(y - S @ x).max() <= 1e-13
+
+
+def test_decode_partial_chunk_sweep_closed_form():
+    # right-to-left sweep over buffered tokens gives A_p q and B_p q
+    rng = np.random.default_rng(24)
+    d, m = 6, 5
+    _, k, v, a, b = _head(rng, m, d)
+    qv = rng.standard_normal(d)
+    Ap, Bp = ho.chunk_transition(k, v, a, b)
+    x = qv.copy()
+    y0 = np.zeros(d)
+    for t in reversed(range(m)):
+        y0 += b[t] * v[t] * (k[t] @ x)
+        x = a[t] * (x - b[t] * k[t] * (k[t] @ x))
+    assert np.abs(x - Ap @ qv).max() <= 1e-14
+    assert np.abs(y0 - Bp @ qv).max() <= 1e-14
