@@ -1,0 +1,300 @@
+// Decode step kernels (one new token per sequence) and the prefill -> cache hand-off.
+//
+// HLA summary page, "Key Contributions" 3 (dynamic autoregressive decoding) and
+// "Methodology in Plain English" paras. 3-4.  For the open chunk holding m tokens
+// (the new one included), the output is o = S_t q with
+//   S_t = S_in A_p + B_p,  S_in = gated composition over the active closed chunks,
+// where (A_p, B_p) is the open chunk's own transition.  It is evaluated without
+// forming any d x d product:
+//   (1) right-to-left sweep over the open chunk's tokens gives x = A_p q and
+//       y0 = B_p q:  c = k_t . x;  y0 += beta_t c v_t;  x <- alpha_t (x - beta_t c k_t);
+//   (2) S_in x = sum_j g_j B_j prod_{l>j} ((1-g_l) I + g_l A_l) x, evaluated for the
+//       active j in descending order:  y += g_j B_j x;  x <- (1-g_j) x + g_j A_j x;
+//   (3) o = y + y0.
+// Each active chunk's A_j and B_j are read exactly once; skipped chunks are not read.
+#include "common.cuh"
+#include "kernels.cuh"
+#include "routing_recipe.cuh"
+
+namespace hla {
+
+HLA_DEFINE_ERROR_WORD(decode)
+
+template <int D>
+__device__ __forceinline__ float block_sum(float v, float* red) {
+  // D threads, D/32 warps
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  const int w = threadIdx.x >> 5;
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red[w] = v;
+  __syncthreads();
+  float s = 0.0f;
+#pragma unroll
+  for (int k = 0; k < D / 32; ++k) s += red[k];
+  return s;
+}
+
+// grid B*H, block D.  Thread = channel / row.
+template <int D, typename Tio>
+__global__ void __launch_bounds__(128) decode_main_kernel(DecodeArgs a) {
+  __shared__ float rq[D];
+  __shared__ float xs[2][D];
+  __shared__ float red[D / 32];
+  __shared__ int wcount[D / 32];
+  const int bh = blockIdx.x;
+  const int b = bh / a.H;
+  const int tid = threadIdx.x;
+  const int C = a.C;
+  const int n = a.n_chunks[b];
+  const int m = a.m_partial[b];
+  const int mp = m + 1;
+  const long tok = (long)bh * D + tid;
+  // (0) append the token to the open chunk
+  const long bslot = ((long)bh * C + m) * D + tid;
+  const Tio* qr_in = (const Tio*)(a.q_route ? a.q_route : a.q);
+  const Tio* kr_in = (const Tio*)(a.k_route ? a.k_route : a.k);
+  ((Tio*)a.buf_k)[bslot] = ((const Tio*)a.k)[tok];
+  ((Tio*)a.buf_v)[bslot] = ((const Tio*)a.v)[tok];
+  ((Tio*)a.buf_qr)[bslot] = qr_in[tok];
+  ((Tio*)a.buf_kr)[bslot] = kr_in[tok];
+  if (tid == 0) {
+    a.buf_alpha[(long)bh * C + m] = a.alpha[bh];
+    a.buf_beta[(long)bh * C + m] = a.beta[bh];
+  }
+  __syncthreads();
+  const Tio* bk = (const Tio*)a.buf_k + (long)bh * C * D;
+  const Tio* bv = (const Tio*)a.buf_v + (long)bh * C * D;
+  // (1) open-chunk sweep
+  float x = ldf((const Tio*)a.q + tok);
+  float y0 = 0.0f;
+  for (int t = mp - 1; t >= 0; --t) {
+    const float kt = ldf(bk + (long)t * D + tid);
+    const float c = block_sum<D>(kt * x, red);
+    const float bt = a.buf_beta[(long)bh * C + t];
+    const float at = a.buf_alpha[(long)bh * C + t];
+    y0 = fmaf(bt * c, ldf(bv + (long)t * D + tid), y0);
+    x = at * (x - bt * c * kt);
+  }
+  // (2) gates against every closed chunk, compacted ascending into the workspace
+  int32_t* act_idx = a.act_idx + (long)bh * a.max_chunks;
+  float* act_g = a.act_g + (long)bh * a.max_chunks;
+  int cnt = 0;
+  if (a.mode != HLA_GATES_ZERO && n > 0) {
+    const route::Consts K = route::make_consts();
+    if (a.mode == HLA_GATES_ROUTED) {
+      // query pool over the open chunk's mp route tokens (channel = tid)
+      const Tio* bq = (const Tio*)a.buf_qr + (long)bh * C * D + tid;
+      const float inv_tau = __fdiv_rn(1.0f, a.tau);
+      float mx = __fmul_rn(ldf(bq), inv_tau);
+      for (int t = 1; t < mp; ++t) mx = fmaxf(mx, __fmul_rn(ldf(bq + (long)t * D), inv_tau));
+      float s = 0.0f;
+      for (int t = 0; t < mp; ++t)
+        s = __fadd_rn(s, route::rexp(__fsub_rn(__fmul_rn(ldf(bq + (long)t * D), inv_tau), mx), K));
+      rq[tid] = __fmul_rn(a.tau, __fadd_rn(mx, route::rlog(__fdiv_rn(s, (float)mp), K)));
+      __syncthreads();
+    }
+    const float* rk = a.rk + (long)bh * a.max_chunks * D;
+    for (int jb = 0; jb < n; jb += D) {
+      const int j = jb + tid;
+      float g = 1.0f;
+      bool keep = false;
+      if (j < n) {
+        if (a.mode == HLA_GATES_ROUTED) {
+          const float* rkj = rk + (long)j * D;
+          float dot = 0.0f;
+          for (int c = 0; c < D; ++c) dot = __fadd_rn(dot, __fmul_rn(rq[c], rkj[c]));
+          g = route::gate_from_dot(dot, a.c_d, a.bias, K);
+        }
+        keep = a.thr <= 0.0f || g >= a.thr;
+      }
+      const unsigned int bal = __ballot_sync(0xFFFFFFFFu, keep);
+      const int w = tid >> 5;
+      if ((tid & 31) == 0) wcount[w] = __popc(bal);
+      __syncthreads();
+      int before = 0, total = 0;
+      for (int k2 = 0; k2 < D / 32; ++k2) {
+        if (k2 < w) before += wcount[k2];
+        total += wcount[k2];
+      }
+      if (keep) {
+        const int pos = cnt + before + __popc(bal & ((1u << (tid & 31)) - 1u));
+        act_idx[pos] = j;
+        act_g[pos] = g;
+      }
+      cnt += total;
+      __syncthreads();
+    }
+  }
+  // (3) backward chain over active chunks, descending j
+  float y = 0.0f;
+  int cur = 0;
+  xs[0][tid] = x;
+  __syncthreads();
+  for (int p = cnt - 1; p >= 0; --p) {
+    const int j = act_idx[p];
+    const float g = act_g[p];
+    const Tio* A = (const Tio*)a.A + ((long)bh * a.max_chunks + j) * (long)D * D + (long)tid * D;
+    const Tio* Bm = (const Tio*)a.Bm + ((long)bh * a.max_chunks + j) * (long)D * D + (long)tid * D;
+    float ax = 0.0f, bx = 0.0f;
+#pragma unroll 8
+    for (int c = 0; c < D; ++c) {
+      const float xc = xs[cur][c];
+      ax = fmaf(ldf(A + c), xc, ax);
+      bx = fmaf(ldf(Bm + c), xc, bx);
+    }
+    y = fmaf(g, bx, y);
+    xs[cur ^ 1][tid] = (1.0f - g) * xs[cur][tid] + g * ax;
+    cur ^= 1;
+    __syncthreads();
+  }
+  stf((Tio*)a.o + tok, y + y0);
+}
+
+// Key pool of the closing chunk into the cache (only sequences whose open chunk
+// becomes full this step).  grid B*H, block D.
+template <int D, typename Tio>
+__global__ void decode_close_pool_kernel(DecodeArgs a) {
+  const int bh = blockIdx.x;
+  const int b = bh / a.H;
+  const int tid = threadIdx.x;
+  if (a.m_partial[b] + 1 != a.C) return;
+  const int n = a.n_chunks[b];
+  if (n >= a.max_chunks) {
+    if (tid == 0) report_device_error(kErrCacheFull);
+    return;
+  }
+  const route::Consts K = route::make_consts();
+  const Tio* bk = (const Tio*)a.buf_kr + (long)bh * a.C * D + tid;
+  const float inv_tau = __fdiv_rn(1.0f, a.tau);
+  float mx = __fmul_rn(ldf(bk), inv_tau);
+  for (int t = 1; t < a.C; ++t) mx = fmaxf(mx, __fmul_rn(ldf(bk + (long)t * D), inv_tau));
+  float s = 0.0f;
+  for (int t = 0; t < a.C; ++t)
+    s = __fadd_rn(s, route::rexp(__fsub_rn(__fmul_rn(ldf(bk + (long)t * D), inv_tau), mx), K));
+  a.rk[((long)bh * a.max_chunks + n) * D + tid] =
+      __fmul_rn(a.tau, __fadd_rn(mx, route::rlog(__fdiv_rn(s, (float)a.C), K)));
+}
+
+__global__ void decode_counters_kernel(int B, int C, int max_chunks, int32_t* n_chunks, int32_t* m_partial) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= B) return;
+  const int m = m_partial[b] + 1;
+  if (m == C) {
+    if (n_chunks[b] < max_chunks) n_chunks[b] += 1;
+    m_partial[b] = 0;
+  } else {
+    m_partial[b] = m;
+  }
+}
+
+// Prefill -> cache hand-off: copies the closed chunks' key pools (computed into the
+// prefill workspace with chunk stride N) and the final partial chunk's tokens, and
+// sets the counters.  grid B*H, block 128.
+struct FillArgs {
+  int B, H, T, C, d, N, max_chunks;
+  const float* rk_ws;  // [B,H,N,d]
+  const void *qr, *kr, *k, *v;  // [B,T,H,d]
+  const float *alpha, *beta;    // [B,T,H]
+};
+
+template <typename Tio>
+__global__ void cache_fill_kernel(DecodeArgs c, FillArgs f) {
+  const int bh = blockIdx.x;
+  const int b = bh / f.H, h = bh % f.H;
+  const int nc = f.T / f.C;
+  const int m = f.T - nc * f.C;
+  for (long idx = threadIdx.x; idx < (long)nc * f.d; idx += blockDim.x)
+    c.rk[(long)bh * f.max_chunks * f.d + idx] = f.rk_ws[(long)bh * f.N * f.d + idx];
+  const long HD = (long)f.H * f.d;
+  for (long idx = threadIdx.x; idx < (long)m * f.d; idx += blockDim.x) {
+    const int t = (int)(idx / f.d), ch = (int)(idx - (long)t * f.d);
+    const long src = ((long)b * f.T + nc * f.C + t) * HD + (long)h * f.d + ch;
+    const long dst = ((long)bh * f.C + t) * f.d + ch;
+    ((Tio*)c.buf_k)[dst] = ((const Tio*)f.k)[src];
+    ((Tio*)c.buf_v)[dst] = ((const Tio*)f.v)[src];
+    ((Tio*)c.buf_qr)[dst] = ((const Tio*)f.qr)[src];
+    ((Tio*)c.buf_kr)[dst] = ((const Tio*)f.kr)[src];
+  }
+  for (int t = threadIdx.x; t < m; t += blockDim.x) {
+    const long src = ((long)b * f.T + nc * f.C + t) * f.H + h;
+    c.buf_alpha[(long)bh * f.C + t] = f.alpha[src];
+    c.buf_beta[(long)bh * f.C + t] = f.beta[src];
+  }
+  if (h == 0 && threadIdx.x == 0) {
+    c.n_chunks[b] = nc;
+    c.m_partial[b] = m;
+  }
+}
+
+template <int D, typename Tio>
+static cudaError_t launch_d(const DecodeArgs& a, cudaStream_t s) {
+  decode_main_kernel<D, Tio><<<a.B * a.H, D, 0, s>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // close full chunks: transition into the cache, then the key pool
+  TransArgs t{};
+  t.B = a.B;
+  t.H = a.H;
+  t.T = a.C;
+  t.C = a.C;
+  t.d = D;
+  t.dtype = a.dtype;
+  t.in.k = a.buf_k;
+  t.in.v = a.buf_v;
+  t.in.alpha = a.buf_alpha;
+  t.in.beta = a.buf_beta;
+  t.in.sb = (long)a.H * a.C * D;
+  t.in.sh = (long)a.C * D;
+  t.in.st = D;
+  t.in.ab = (long)a.H * a.C;
+  t.in.ah = a.C;
+  t.in.at = 1;
+  t.n_chunks = 1;
+  t.A = const_cast<void*>(a.A);
+  t.Bm = const_cast<void*>(a.Bm);
+  t.ab_chunk_stride = a.max_chunks;
+  t.ab_chunk_offset = 0;
+  t.close_m = a.m_partial;
+  t.close_n = a.n_chunks;
+  // the transition kernel never writes past max_chunks; the pool kernel flags it
+  e = launch_transitions(t, s);
+  if (e != cudaSuccess) return e;
+  decode_close_pool_kernel<D, Tio><<<a.B * a.H, D, 0, s>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  decode_counters_kernel<<<(a.B + 127) / 128, 128, 0, s>>>(a.B, a.C, a.max_chunks, a.n_chunks, a.m_partial);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
+  if (a.d == 128) return a.dtype == HLA_BF16 ? launch_d<128, __nv_bfloat16>(a, s) : launch_d<128, float>(a, s);
+  return a.dtype == HLA_BF16 ? launch_d<64, __nv_bfloat16>(a, s) : launch_d<64, float>(a, s);
+}
+
+cudaError_t launch_cache_fill(const DecodeArgs& c, const float* rk_ws, const void* q_route, const void* k_route,
+                              const void* k, const void* v, const float* alpha, const float* beta, int T,
+                              cudaStream_t s) {
+  FillArgs f{};
+  f.B = c.B;
+  f.H = c.H;
+  f.T = T;
+  f.C = c.C;
+  f.d = c.d;
+  f.N = (T + c.C - 1) / c.C;
+  f.max_chunks = c.max_chunks;
+  f.rk_ws = rk_ws;
+  f.qr = q_route;
+  f.kr = k_route;
+  f.k = k;
+  f.v = v;
+  f.alpha = alpha;
+  f.beta = beta;
+  if (c.dtype == HLA_BF16)
+    cache_fill_kernel<__nv_bfloat16><<<c.B * c.H, 128, 0, s>>>(c, f);
+  else
+    cache_fill_kernel<float><<<c.B * c.H, 128, 0, s>>>(c, f);
+  return cudaGetLastError();
+}
+
+}  // namespace hla

@@ -1,0 +1,485 @@
+// C ABI of libhla: argument checks, workspace and cache layout, launch sequence.
+// Every entry point validates on the host first and launches nothing on error.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace {
+
+thread_local char g_msg[512] = "";
+
+hla_status fail(hla_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+hla_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(HLA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+size_t esize(int dtype) { return dtype == HLA_BF16 ? 2 : 4; }
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+// Shape/dtype checks common to every entry point.  need_T: T must be >= 1.
+hla_status check_cfg(const hla_config* c, bool need_T) {
+  if (c == nullptr) return fail(HLA_ERR_INVALID_ARG, "cfg is NULL");
+  if (c->B <= 0 || c->H <= 0) return fail(HLA_ERR_INVALID_ARG, "B and H must be positive (B=%d H=%d)", c->B, c->H);
+  if (need_T && c->T <= 0) return fail(HLA_ERR_INVALID_ARG, "T must be positive (T=%d)", c->T);
+  if (c->C != 64) return fail(HLA_ERR_UNSUPPORTED, "chunk size C=%d unsupported (64 only)", c->C);
+  if (c->dk != c->dv) return fail(HLA_ERR_UNSUPPORTED, "dk != dv (%d, %d) unsupported", c->dk, c->dv);
+  if (c->dk != 64 && c->dk != 128) return fail(HLA_ERR_UNSUPPORTED, "head dim %d unsupported (64, 128)", c->dk);
+  if (c->dtype != HLA_F32 && c->dtype != HLA_BF16) return fail(HLA_ERR_UNSUPPORTED, "dtype %d unsupported", c->dtype);
+  if (c->gate_mode < HLA_GATES_ROUTED || c->gate_mode > HLA_GATES_USER)
+    return fail(HLA_ERR_INVALID_ARG, "gate_mode %d invalid", c->gate_mode);
+  if (!(c->tau > 0.0f) || !std::isfinite(c->tau)) return fail(HLA_ERR_INVALID_ARG, "tau must be finite and > 0");
+  if (!std::isfinite(c->bias) || !std::isfinite(c->skip_threshold))
+    return fail(HLA_ERR_INVALID_ARG, "bias and skip_threshold must be finite");
+  const double elems = (double)c->B * (need_T ? c->T : 1) * c->H * c->dk;
+  if (elems > 9.0e15) return fail(HLA_ERR_UNSUPPORTED, "problem too large");
+  return HLA_OK;
+}
+
+hla_status need_ptr(const void* p, const char* name) {
+  if (p == nullptr) return fail(HLA_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned16(p)) return fail(HLA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  return HLA_OK;
+}
+
+hla_status opt_ptr(const void* p, const char* name) {
+  if (p != nullptr && !aligned16(p)) return fail(HLA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  return HLA_OK;
+}
+
+#define HLA_TRY(expr)                \
+  do {                               \
+    hla_status _s = (expr);          \
+    if (_s != HLA_OK) return _s;     \
+  } while (0)
+
+#define HLA_CUDA(expr, where)                   \
+  do {                                          \
+    cudaError_t _e = (expr);                    \
+    if (_e != cudaSuccess) return cuda_fail(_e, where); \
+  } while (0)
+
+float gate_scale(int d) { return (float)(1.0 / std::sqrt((double)d)); }
+
+// Prefill workspace layout.
+struct PrefillWs {
+  size_t rq, rk, act_idx, act_g, act_cnt, A, Bm, Wb, Ub, ell, S_in, total;
+};
+
+PrefillWs prefill_layout(const hla_config* c) {
+  PrefillWs w{};
+  const size_t B = c->B, H = c->H, d = c->dk, C = c->C;
+  const size_t N = (c->T + C - 1) / C;
+  const size_t Nc = c->T / C;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  w.rq = take(B * H * N * d * 4);
+  w.rk = take(B * H * N * d * 4);
+  w.act_idx = take(B * H * N * N * 4);
+  w.act_g = take(B * H * N * N * 4);
+  w.act_cnt = take(B * H * N * 4);
+  w.A = take(B * H * Nc * d * d * esize(c->dtype));
+  w.Bm = take(B * H * Nc * d * d * esize(c->dtype));
+  w.Wb = take(B * H * N * C * d * 4);
+  w.Ub = take(B * H * N * C * d * 4);
+  w.ell = take(B * H * N * C * 4);
+  w.S_in = take(B * H * N * d * d * 4);
+  w.total = off;
+  return w;
+}
+
+struct CacheLayout {
+  size_t A, Bm, rk, bk, bv, bqr, bkr, balpha, bbeta, n, m, total;
+};
+
+CacheLayout cache_layout(const hla_config* c, int32_t maxc) {
+  CacheLayout L{};
+  const size_t B = c->B, H = c->H, d = c->dk, C = c->C, es = esize(c->dtype);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  L.A = take(B * H * (size_t)maxc * d * d * es);
+  L.Bm = take(B * H * (size_t)maxc * d * d * es);
+  L.rk = take(B * H * (size_t)maxc * d * 4);
+  L.bk = take(B * H * C * d * es);
+  L.bv = take(B * H * C * d * es);
+  L.bqr = take(B * H * C * d * es);
+  L.bkr = take(B * H * C * d * es);
+  L.balpha = take(B * H * C * 4);
+  L.bbeta = take(B * H * C * 4);
+  L.n = take(B * 4);
+  L.m = take(B * 4);
+  L.total = off;
+  return L;
+}
+
+hla_status check_cache(const hla_config* c, const hla_cache* k) {
+  if (k == nullptr) return fail(HLA_ERR_INVALID_ARG, "cache is NULL");
+  if (k->B != c->B || k->H != c->H || k->C != c->C || k->d != c->dk || k->dtype != c->dtype)
+    return fail(HLA_ERR_INVALID_ARG, "cache was initialised for a different config");
+  if (k->max_chunks <= 0) return fail(HLA_ERR_INVALID_ARG, "cache max_chunks must be positive");
+  const void* ps[] = {k->A, k->Bm, k->rk, k->buf_k, k->buf_v, k->buf_qr, k->buf_kr,
+                      k->buf_alpha, k->buf_beta, k->n_chunks, k->m_partial};
+  for (const void* p : ps) HLA_TRY(need_ptr(p, "cache buffer"));
+  return HLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* hla_last_error(void) { return g_msg; }
+
+size_t hla_cache_bytes(const hla_config* cfg, int32_t max_chunks) {
+  if (check_cfg(cfg, false) != HLA_OK || max_chunks <= 0) return 0;
+  return cache_layout(cfg, max_chunks).total;
+}
+
+hla_status hla_cache_init(const hla_config* cfg, int32_t max_chunks, void* mem, size_t bytes, hla_cache* out,
+                          hla_stream_t stream) {
+  g_msg[0] = 0;
+  HLA_TRY(check_cfg(cfg, false));
+  if (out == nullptr) return fail(HLA_ERR_INVALID_ARG, "out is NULL");
+  if (max_chunks <= 0) return fail(HLA_ERR_INVALID_ARG, "max_chunks must be positive");
+  HLA_TRY(need_ptr(mem, "mem"));
+  if (((uintptr_t)mem & 255u) != 0) return fail(HLA_ERR_INVALID_ARG, "cache memory must be 256-byte aligned");
+  const CacheLayout L = cache_layout(cfg, max_chunks);
+  if (bytes < L.total) return fail(HLA_ERR_WORKSPACE, "cache block too small: %zu < %zu", bytes, L.total);
+  char* base = (char*)mem;
+  hla_cache c{};
+  c.max_chunks = max_chunks;
+  c.B = cfg->B;
+  c.H = cfg->H;
+  c.C = cfg->C;
+  c.d = cfg->dk;
+  c.dtype = cfg->dtype;
+  c.A = base + L.A;
+  c.Bm = base + L.Bm;
+  c.rk = (float*)(base + L.rk);
+  c.buf_k = base + L.bk;
+  c.buf_v = base + L.bv;
+  c.buf_qr = base + L.bqr;
+  c.buf_kr = base + L.bkr;
+  c.buf_alpha = (float*)(base + L.balpha);
+  c.buf_beta = (float*)(base + L.bbeta);
+  c.n_chunks = (int32_t*)(base + L.n);
+  c.m_partial = (int32_t*)(base + L.m);
+  HLA_CUDA(cudaMemsetAsync(base + L.n, 0, L.total - L.n, (cudaStream_t)stream), "hla_cache_init memset");
+  *out = c;
+  return HLA_OK;
+}
+
+size_t hla_prefill_workspace_bytes(const hla_config* cfg) {
+  if (check_cfg(cfg, true) != HLA_OK) return 0;
+  return prefill_layout(cfg).total;
+}
+
+size_t hla_decode_workspace_bytes(const hla_config* cfg, int32_t max_chunks) {
+  if (check_cfg(cfg, false) != HLA_OK || max_chunks <= 0) return 0;
+  const size_t n = (size_t)cfg->B * cfg->H * max_chunks;
+  return align256(n * 4) + align256(n * 4);
+}
+
+hla_status gdn_chunk_transitions(const hla_config* cfg, const void* k, const void* v, const float* alpha,
+                                 const float* beta, void* A_out, void* B_out, hla_stream_t stream) {
+  g_msg[0] = 0;
+  HLA_TRY(check_cfg(cfg, true));
+  HLA_TRY(need_ptr(k, "k"));
+  HLA_TRY(need_ptr(v, "v"));
+  HLA_TRY(need_ptr(alpha, "alpha"));
+  HLA_TRY(need_ptr(beta, "beta"));
+  HLA_TRY(need_ptr(A_out, "A_out"));
+  HLA_TRY(need_ptr(B_out, "B_out"));
+  const int Nc = cfg->T / cfg->C;
+  if (Nc == 0) return HLA_OK;
+  hla::TransArgs t{};
+  t.B = cfg->B;
+  t.H = cfg->H;
+  t.T = Nc * cfg->C;
+  t.C = cfg->C;
+  t.d = cfg->dk;
+  t.dtype = cfg->dtype;
+  t.in = {k, v, alpha, beta, (long)cfg->T * cfg->H * cfg->dk, cfg->dk, (long)cfg->H * cfg->dk,
+          (long)cfg->T * cfg->H, 1, cfg->H};
+  t.n_chunks = Nc;
+  t.A = A_out;
+  t.Bm = B_out;
+  t.ab_chunk_stride = Nc;
+  HLA_CUDA(hla::launch_transitions(t, (cudaStream_t)stream), "gdn_chunk_transitions launch");
+  return HLA_OK;
+}
+
+static hla_status routing_impl(const hla_config* cfg, const void* q_route, const void* k_route, float* rq,
+                               float* rk, const float* user_gates, int32_t* act_idx, float* act_g,
+                               int32_t* act_cnt, float* gates_out, int32_t* active_idx_out,
+                               int32_t* active_cnt_out, cudaStream_t s) {
+  const int N = (cfg->T + cfg->C - 1) / cfg->C;
+  if (cfg->gate_mode == HLA_GATES_ROUTED || rk != nullptr) {
+    HLA_CUDA(hla::launch_pools(cfg->gate_mode == HLA_GATES_ROUTED ? q_route : nullptr, k_route,
+                               cfg->gate_mode == HLA_GATES_ROUTED ? rq : nullptr, rk, cfg->B, cfg->T, cfg->H,
+                               cfg->dk, cfg->C, N, cfg->tau, cfg->dtype, s),
+             "pool launch");
+  }
+  hla::GatesArgs g{};
+  g.B = cfg->B;
+  g.H = cfg->H;
+  g.N = N;
+  g.d = cfg->dk;
+  g.mode = cfg->gate_mode;
+  g.c_d = gate_scale(cfg->dk);
+  g.bias = cfg->bias;
+  g.thr = cfg->skip_threshold;
+  g.rq = rq;
+  g.rk = rk;
+  g.user_gates = user_gates;
+  g.act_idx = act_idx;
+  g.act_g = act_g;
+  g.act_cnt = act_cnt;
+  g.gates_out = gates_out;
+  g.active_idx_out = active_idx_out;
+  g.active_cnt_out = active_cnt_out;
+  HLA_CUDA(hla::launch_gates(g, s), "gates launch");
+  return HLA_OK;
+}
+
+hla_status hla_routing(const hla_config* cfg, const void* q_route, const void* k_route, float* rq_out,
+                       float* rk_out, float* gates_out, int32_t* active_idx_out, int32_t* active_cnt_out,
+                       hla_stream_t stream) {
+  g_msg[0] = 0;
+  HLA_TRY(check_cfg(cfg, true));
+  if (cfg->gate_mode == HLA_GATES_USER) return fail(HLA_ERR_UNSUPPORTED, "hla_routing does not take user gates");
+  HLA_TRY(need_ptr(q_route, "q_route"));
+  HLA_TRY(need_ptr(k_route, "k_route"));
+  HLA_TRY(need_ptr(rq_out, "rq_out"));
+  HLA_TRY(need_ptr(rk_out, "rk_out"));
+  HLA_TRY(opt_ptr(gates_out, "gates_out"));
+  HLA_TRY(opt_ptr(active_idx_out, "active_idx_out"));
+  HLA_TRY(opt_ptr(active_cnt_out, "active_cnt_out"));
+  if ((active_idx_out == nullptr) != (active_cnt_out == nullptr))
+    return fail(HLA_ERR_INVALID_ARG, "active_idx_out and active_cnt_out go together");
+  const int N = (cfg->T + cfg->C - 1) / cfg->C;
+  cudaStream_t s = (cudaStream_t)stream;
+  HLA_CUDA(hla::launch_pools(q_route, k_route, rq_out, rk_out, cfg->B, cfg->T, cfg->H, cfg->dk, cfg->C, N,
+                             cfg->tau, cfg->dtype, s),
+           "pool launch");
+  hla::GatesArgs g{};
+  g.B = cfg->B;
+  g.H = cfg->H;
+  g.N = N;
+  g.d = cfg->dk;
+  g.mode = cfg->gate_mode;
+  g.c_d = gate_scale(cfg->dk);
+  g.bias = cfg->bias;
+  g.thr = cfg->skip_threshold;
+  g.rq = rq_out;
+  g.rk = rk_out;
+  g.act_idx = active_idx_out;
+  g.act_cnt = active_cnt_out;
+  g.pad_act_idx = true;
+  g.gates_out = gates_out;
+  HLA_CUDA(hla::launch_gates(g, s), "gates launch");
+  return HLA_OK;
+}
+
+hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, const void* v, const float* alpha,
+                       const float* beta, const void* q_route, const void* k_route, const float* user_gates,
+                       void* o, float* gates_out, int32_t* active_idx_out, int32_t* active_cnt_out,
+                       hla_cache* cache_out, void* workspace, size_t workspace_bytes, hla_stream_t stream) {
+  g_msg[0] = 0;
+  HLA_TRY(check_cfg(cfg, true));
+  HLA_TRY(need_ptr(q, "q"));
+  HLA_TRY(need_ptr(k, "k"));
+  HLA_TRY(need_ptr(v, "v"));
+  HLA_TRY(need_ptr(alpha, "alpha"));
+  HLA_TRY(need_ptr(beta, "beta"));
+  HLA_TRY(need_ptr(o, "o"));
+  HLA_TRY(opt_ptr(q_route, "q_route"));
+  HLA_TRY(opt_ptr(k_route, "k_route"));
+  HLA_TRY(opt_ptr(gates_out, "gates_out"));
+  HLA_TRY(opt_ptr(active_idx_out, "active_idx_out"));
+  HLA_TRY(opt_ptr(active_cnt_out, "active_cnt_out"));
+  if (cfg->gate_mode == HLA_GATES_USER) HLA_TRY(need_ptr(user_gates, "user_gates"));
+  const int N = (cfg->T + cfg->C - 1) / cfg->C;
+  const int Nc = cfg->T / cfg->C;
+  if (cache_out != nullptr) {
+    HLA_TRY(check_cache(cfg, cache_out));
+    if (cache_out->max_chunks < Nc)
+      return fail(HLA_ERR_WORKSPACE, "cache holds %d chunks, prompt has %d", cache_out->max_chunks, Nc);
+  }
+  const PrefillWs w = prefill_layout(cfg);
+  HLA_TRY(need_ptr(workspace, "workspace"));
+  if (((uintptr_t)workspace & 255u) != 0) return fail(HLA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (workspace_bytes < w.total)
+    return fail(HLA_ERR_WORKSPACE, "workspace too small: %zu < %zu", workspace_bytes, w.total);
+  char* ws = (char*)workspace;
+  cudaStream_t s = (cudaStream_t)stream;
+  const void* qr = q_route ? q_route : q;
+  const void* kr = k_route ? k_route : k;
+  float* rq = (float*)(ws + w.rq);
+  float* rk = (float*)(ws + w.rk);
+  int32_t* act_idx = (int32_t*)(ws + w.act_idx);
+  float* act_g = (float*)(ws + w.act_g);
+  int32_t* act_cnt = (int32_t*)(ws + w.act_cnt);
+  HLA_TRY(routing_impl(cfg, qr, kr, rq, (cfg->gate_mode == HLA_GATES_ROUTED || cache_out) ? rk : nullptr,
+                       user_gates, act_idx, act_g, act_cnt, gates_out, active_idx_out, active_cnt_out, s));
+  // transitions of every chunk (A/B of complete chunks into the cache or workspace)
+  hla::TransArgs t{};
+  t.B = cfg->B;
+  t.H = cfg->H;
+  t.T = cfg->T;
+  t.C = cfg->C;
+  t.d = cfg->dk;
+  t.dtype = cfg->dtype;
+  t.in = {k, v, alpha, beta, (long)cfg->T * cfg->H * cfg->dk, cfg->dk, (long)cfg->H * cfg->dk,
+          (long)cfg->T * cfg->H, 1, cfg->H};
+  t.n_chunks = N;
+  t.A = cache_out ? cache_out->A : (void*)(ws + w.A);
+  t.Bm = cache_out ? cache_out->Bm : (void*)(ws + w.Bm);
+  t.ab_chunk_stride = cache_out ? cache_out->max_chunks : Nc;
+  t.Wb = (float*)(ws + w.Wb);
+  t.Ub = (float*)(ws + w.Ub);
+  t.ell = (float*)(ws + w.ell);
+  HLA_CUDA(hla::launch_transitions(t, s), "transitions launch");
+  hla::ComposeArgs c{};
+  c.B = cfg->B;
+  c.H = cfg->H;
+  c.N = N;
+  c.d = cfg->dk;
+  c.dtype = cfg->dtype;
+  c.A = t.A;
+  c.Bm = t.Bm;
+  c.ab_chunk_stride = t.ab_chunk_stride;
+  c.act_idx = act_idx;
+  c.act_g = act_g;
+  c.act_cnt = act_cnt;
+  c.S_in = (float*)(ws + w.S_in);
+  HLA_CUDA(hla::launch_compose(c, s), "compose launch");
+  hla::ReadoutArgs r{};
+  r.B = cfg->B;
+  r.H = cfg->H;
+  r.T = cfg->T;
+  r.C = cfg->C;
+  r.N = N;
+  r.d = cfg->dk;
+  r.dtype = cfg->dtype;
+  r.q = q;
+  r.k = k;
+  r.S_in = c.S_in;
+  r.Wb = t.Wb;
+  r.Ub = t.Ub;
+  r.ell = t.ell;
+  r.o = o;
+  HLA_CUDA(hla::launch_readout(r, s), "readout launch");
+  if (cache_out) {
+    hla::DecodeArgs dc{};
+    dc.B = cfg->B;
+    dc.H = cfg->H;
+    dc.C = cfg->C;
+    dc.d = cfg->dk;
+    dc.dtype = cfg->dtype;
+    dc.max_chunks = cache_out->max_chunks;
+    dc.rk = cache_out->rk;
+    dc.buf_k = cache_out->buf_k;
+    dc.buf_v = cache_out->buf_v;
+    dc.buf_qr = cache_out->buf_qr;
+    dc.buf_kr = cache_out->buf_kr;
+    dc.buf_alpha = cache_out->buf_alpha;
+    dc.buf_beta = cache_out->buf_beta;
+    dc.n_chunks = cache_out->n_chunks;
+    dc.m_partial = cache_out->m_partial;
+    HLA_CUDA(hla::launch_cache_fill(dc, rk, qr, kr, k, v, alpha, beta, cfg->T, s), "cache fill launch");
+  }
+  return HLA_OK;
+}
+
+hla_status hla_decode_step(const hla_config* cfg, hla_cache* cache, const void* q, const void* k, const void* v,
+                           const float* alpha, const float* beta, const void* q_route, const void* k_route,
+                           void* o, void* workspace, size_t workspace_bytes, hla_stream_t stream) {
+  g_msg[0] = 0;
+  HLA_TRY(check_cfg(cfg, false));
+  if (cfg->gate_mode == HLA_GATES_USER) return fail(HLA_ERR_UNSUPPORTED, "decode does not take user gates");
+  HLA_TRY(check_cache(cfg, cache));
+  HLA_TRY(need_ptr(q, "q"));
+  HLA_TRY(need_ptr(k, "k"));
+  HLA_TRY(need_ptr(v, "v"));
+  HLA_TRY(need_ptr(alpha, "alpha"));
+  HLA_TRY(need_ptr(beta, "beta"));
+  HLA_TRY(need_ptr(o, "o"));
+  HLA_TRY(opt_ptr(q_route, "q_route"));
+  HLA_TRY(opt_ptr(k_route, "k_route"));
+  const size_t need = hla_decode_workspace_bytes(cfg, cache->max_chunks);
+  HLA_TRY(need_ptr(workspace, "workspace"));
+  if (((uintptr_t)workspace & 255u) != 0) return fail(HLA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (workspace_bytes < need) return fail(HLA_ERR_WORKSPACE, "workspace too small: %zu < %zu", workspace_bytes, need);
+  hla::DecodeArgs a{};
+  a.B = cfg->B;
+  a.H = cfg->H;
+  a.C = cfg->C;
+  a.d = cfg->dk;
+  a.dtype = cfg->dtype;
+  a.mode = cfg->gate_mode;
+  a.max_chunks = cache->max_chunks;
+  a.tau = cfg->tau;
+  a.c_d = gate_scale(cfg->dk);
+  a.bias = cfg->bias;
+  a.thr = cfg->skip_threshold;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.alpha = alpha;
+  a.beta = beta;
+  a.q_route = q_route;
+  a.k_route = k_route;
+  a.o = o;
+  a.A = cache->A;
+  a.Bm = cache->Bm;
+  a.rk = cache->rk;
+  a.buf_k = cache->buf_k;
+  a.buf_v = cache->buf_v;
+  a.buf_qr = cache->buf_qr;
+  a.buf_kr = cache->buf_kr;
+  a.buf_alpha = cache->buf_alpha;
+  a.buf_beta = cache->buf_beta;
+  a.n_chunks = cache->n_chunks;
+  a.m_partial = cache->m_partial;
+  const size_t n = (size_t)cfg->B * cfg->H * cache->max_chunks;
+  a.act_idx = (int32_t*)workspace;
+  a.act_g = (float*)((char*)workspace + align256(n * 4));
+  HLA_CUDA(hla::launch_decode(a, (cudaStream_t)stream), "decode launch");
+  return HLA_OK;
+}
+
+hla_status hla_device_status(int32_t clear, uint32_t* code_out) {
+  g_msg[0] = 0;
+  HLA_CUDA(cudaDeviceSynchronize(), "hla_device_status synchronize");
+  unsigned int word = 0, w = 0;
+  HLA_CUDA(hla::read_error_word_decode(&w, clear != 0), "hla_device_status read");
+  word |= w;
+  if (code_out) *code_out = word;
+  if (word & (hla::kErrMbarTimeout | hla::kErrTmemAlloc))
+    return fail(HLA_ERR_TIMEOUT, "a bounded device wait expired (code 0x%x)", word);
+  if (word & hla::kErrCacheFull) return fail(HLA_ERR_WORKSPACE, "a decode step found the cache full (code 0x%x)", word);
+  return HLA_OK;
+}
+
+}  // extern "C"

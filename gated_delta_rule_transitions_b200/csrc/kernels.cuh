@@ -1,0 +1,113 @@
+// Internal launch interfaces between hla_api.cu and the kernel translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace hla {
+
+struct GatesArgs {
+  int B, H, N, d, mode;
+  float c_d, bias, thr;
+  const float* rq;          // [B,H,N,d]
+  const float* rk;          // [B,H,N,d]
+  const float* user_gates;  // [B,H,N,N] (mode USER)
+  int32_t* act_idx;         // [B,H,N,N] compacted ascending j
+  float* act_g;             // [B,H,N,N] matching gates
+  int32_t* act_cnt;         // [B,H,N]
+  float* gates_out;         // optional [B,H,N,N]
+  int32_t* active_idx_out;  // optional [B,H,N,N]
+  int32_t* active_cnt_out;  // optional [B,H,N]
+  bool pad_act_idx;         // pad act_idx rows beyond the count with -1
+};
+
+// Token-major input view of k/v/alpha/beta used by the transition kernels:
+// element (b, h, t, c) of k is at k[b*sb + h*sh + t*st + c]; alpha at
+// alpha[b*ab + h*ah + t*at].
+struct TokenView {
+  const void* k;
+  const void* v;
+  const float* alpha;
+  const float* beta;
+  long sb, sh, st;   // k/v strides (elements)
+  long ab, ah, at;   // alpha/beta strides (elements)
+};
+
+struct TransArgs {
+  int B, H, T, C, d, dtype;
+  TokenView in;
+  int n_chunks;          // chunks to process per (b,h) (complete + optional partial)
+  void* A;               // [B,H,chunk_stride,d,d] (dtype) or null
+  void* Bm;              // same
+  long ab_chunk_stride;  // chunk stride of A/B (in chunks)
+  long ab_chunk_offset;  // first chunk index written (decode close)
+  float* Wb;             // [B,H,N,C,d] fp32 or null
+  float* Ub;             // [B,H,N,C,d] fp32 or null
+  float* ell;            // [B,H,N,C] fp32 or null
+  const int32_t* close_m;   // decode close: per-b m_partial (before the step) or null
+  const int32_t* close_n;   // decode close: per-b n_chunks or null
+};
+
+struct ComposeArgs {
+  int B, H, N, d, dtype;
+  const void* A;          // [B,H,ab_stride,d,d]
+  const void* Bm;
+  long ab_chunk_stride;
+  const int32_t* act_idx; // [B,H,N,N]
+  const float* act_g;
+  const int32_t* act_cnt; // [B,H,N]
+  float* S_in;            // [B,H,N,d,d] fp32
+};
+
+struct ReadoutArgs {
+  int B, H, T, C, N, d, dtype;
+  const void* q;          // [B,T,H,d]
+  const void* k;
+  const float* S_in;      // [B,H,N,d,d]
+  const float* Wb;        // [B,H,N,C,d]
+  const float* Ub;
+  const float* ell;       // [B,H,N,C]
+  void* o;                // [B,T,H,d]
+};
+
+struct DecodeArgs {
+  int B, H, C, d, dtype, mode, max_chunks;
+  float tau, c_d, bias, thr;
+  const void* q;   // [B,H,d]
+  const void* k;
+  const void* v;
+  const float* alpha;  // [B,H]
+  const float* beta;
+  const void* q_route;
+  const void* k_route;
+  void* o;
+  // cache
+  const void* A;
+  const void* Bm;
+  float* rk;
+  void* buf_k;
+  void* buf_v;
+  void* buf_qr;
+  void* buf_kr;
+  float* buf_alpha;
+  float* buf_beta;
+  int32_t* n_chunks;
+  int32_t* m_partial;
+  // workspace
+  int32_t* act_idx;  // [B,H,max_chunks]
+  float* act_g;      // [B,H,max_chunks]
+};
+
+cudaError_t launch_pools(const void* x0, const void* x1, float* r0, float* r1, int B, int T, int H, int d,
+                         int C, int out_chunk_stride, float tau, int dtype, cudaStream_t s);
+cudaError_t launch_gates(const GatesArgs& a, cudaStream_t s);
+cudaError_t launch_transitions(const TransArgs& a, cudaStream_t s);
+cudaError_t launch_compose(const ComposeArgs& a, cudaStream_t s);
+cudaError_t launch_readout(const ReadoutArgs& a, cudaStream_t s);
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_cache_fill(const DecodeArgs& c, const float* rk_ws, const void* q_route, const void* k_route,
+                              const void* k, const void* v, const float* alpha, const float* beta, int T,
+                              cudaStream_t s);
+cudaError_t read_error_word_decode(unsigned int* out, bool clear);
+
+}  // namespace hla

@@ -1,0 +1,225 @@
+/*
+ * hla.h -- C ABI of libhla.so: Hybrid Linear Attention (HLA) over Gated DeltaNet,
+ * prefill and decode hot path on one NVIDIA B200 (sm_100a).
+ *
+ * Source passages (HLA: Expressive Hybrid Linear Attention via Chunk-Wise Dynamic
+ * Mixing, ai.info AI summary page):
+ *   - "Methodology in Plain English", para. 1: per-token affine rule of Gated
+ *     DeltaNet; a whole chunk is summarised exactly by one (matrix, additive term)
+ *     pair because affine maps compose.
+ *   - same section, para. 2: each chunk gets a pooled representative; a query's
+ *     score against it is squashed through a sigmoid into a weight in (0, 1).
+ *   - same section, para. 3: the weight interpolates the chunk's full transition
+ *     with the identity; the current chunk has weight one; future chunks are masked.
+ *   - same section, para. 4: weights below an inference threshold are set to zero
+ *     without renormalisation, which makes skipping that chunk exact.
+ *   - "Key Contributions" 3: training/prefill and dynamic autoregressive decoding.
+ *   - "Overview": log-mean-exp pooled routing gates.
+ *
+ * Definitions used throughout (per sequence b and head h; d_k = d_v = d):
+ *   token rule   S_t = S_{t-1} alpha_t (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
+ *                o_t = S_t q_t            (S is d_v x d_k; no scaling of q)
+ *   chunk c      tokens cC .. cC+C-1 act as S -> S A_c + B_c (exact)
+ *   pools        r_c = tau * log(mean_t exp(x_t / tau)) per channel over chunk c's
+ *                route tokens (route inputs default to q for r^q and k for r^k)
+ *   gates        g_ij = sigmoid(<r^q_i, r^k_j> / sqrt(d) + bias), j < i, computed by
+ *                a fixed binary32 recipe (no fused multiply-add, exp/log evaluated by
+ *                a fixed polynomial scheme) so that gates and skip decisions are
+ *                reproducible bit for bit
+ *   skip         j is skipped for query chunk i iff skip_threshold > 0 and
+ *                g_ij < skip_threshold (equality is kept)
+ *   composition  S <- 0; for active j ascending: S <- S + g_ij ((S A_j + B_j) - S)
+ *   read-out     the token rule runs from that S over chunk i's tokens.
+ *
+ * Conventions
+ *   - Every pointer argument named as device memory is a CUDA device pointer owned
+ *     by the caller.  The library never allocates device memory: callers query
+ *     the workspace and cache sizes and pass buffers in.
+ *   - Every device pointer must be 16-byte aligned (HLA_ERR_INVALID_ARG otherwise).
+ *   - Layouts are dense row-major:
+ *       q, k, v, q_route, k_route, o : [B, T, H, d]      (dtype)
+ *       alpha, beta                   : [B, T, H]         float32, alpha in (0,1], beta in [0,1]
+ *       A_c                           : [d_k][d_k]; entry (r, c) multiplies column r
+ *                                       of S into column c of S A
+ *       B_c                           : [d_v][d_k]
+ *   - q, k, v, the route inputs, o and cached A/B share the config's dtype.  Gates,
+ *     pools and the composed state are float32.  Arithmetic is float32 (bf16
+ *     tensor-core products accumulate in float32).
+ *   - Calls are asynchronous on the given stream.  Argument checks run on the host
+ *     before any launch; on error nothing is launched and hla_last_error() returns a
+ *     message (thread-local).
+ *   - Supported: C = 64; d_k = d_v in {64, 128}; dtype float32 or bf16; any T >= 1
+ *     in prefill (a final partial chunk is read out and, with a cache, buffered).
+ */
+#ifndef HLA_H_
+#define HLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same underlying type as cudaStream_t (NULL = legacy default stream). */
+typedef struct CUstream_st* hla_stream_t;
+
+typedef enum {
+  HLA_OK = 0,
+  HLA_ERR_INVALID_ARG = 1, /* NULL/misaligned pointer, inconsistent sizes      */
+  HLA_ERR_UNSUPPORTED = 2, /* shape or dtype outside the supported set          */
+  HLA_ERR_WORKSPACE = 3,   /* workspace or cache buffer too small              */
+  HLA_ERR_CUDA = 4,        /* a CUDA runtime call failed (message has details) */
+  HLA_ERR_TIMEOUT = 5      /* a bounded device-side wait expired (see below)   */
+} hla_status;
+
+typedef enum { HLA_F32 = 0, HLA_BF16 = 1 } hla_dtype;
+
+typedef enum {
+  HLA_GATES_ROUTED = 0, /* gates from the pools (the method)                        */
+  HLA_GATES_ONE = 1,    /* every earlier chunk weight 1: native Gated DeltaNet      */
+  HLA_GATES_ZERO = 2,   /* every earlier chunk weight 0: intra-chunk term only      */
+  HLA_GATES_USER = 3    /* caller-given input-independent weights [B,H,N,N] (prefill) */
+} hla_gate_mode;
+
+typedef struct hla_config {
+  int32_t B;              /* sequences                                          */
+  int32_t H;              /* heads                                              */
+  int32_t T;              /* tokens per sequence (prefill, transitions)         */
+  int32_t C;              /* chunk size (64)                                    */
+  int32_t dk, dv;         /* head dims, equal, 64 or 128                        */
+  int32_t dtype;          /* hla_dtype                                          */
+  int32_t gate_mode;      /* hla_gate_mode                                      */
+  float tau;              /* pooling temperature, > 0                           */
+  float bias;             /* gate bias b                                        */
+  float skip_threshold;   /* <= 0: nothing skipped                              */
+} hla_config;
+
+/*
+ * Decode cache of B sequences (all pointers are device memory carved out of one
+ * caller-owned block by hla_cache_init):
+ *   A, Bm        [B, H, max_chunks, d, d]  dtype  -- transitions of closed chunks
+ *   rk           [B, H, max_chunks, d]     float32 -- key pools of closed chunks
+ *   buf_k, buf_v, buf_qr, buf_kr  [B, H, C, d] dtype -- tokens of the open chunk
+ *   buf_alpha, buf_beta           [B, H, C]  float32
+ *   n_chunks     [B] int32 -- closed chunks per sequence
+ *   m_partial    [B] int32 -- tokens in the open chunk (0 .. C-1 between calls)
+ * The cache is the resumable decode state ("Main Findings": per-chunk affine
+ * states replace the KV cache): A/B take 2 d^2 elements per closed chunk.
+ */
+typedef struct hla_cache {
+  int32_t max_chunks;
+  int32_t B, H, C, d, dtype;
+  void* A;
+  void* Bm;
+  float* rk;
+  void* buf_k;
+  void* buf_v;
+  void* buf_qr;
+  void* buf_kr;
+  float* buf_alpha;
+  float* buf_beta;
+  int32_t* n_chunks;
+  int32_t* m_partial;
+} hla_cache;
+
+/* Message for the last non-OK status returned on this thread ("" if none). */
+const char* hla_last_error(void);
+
+/* Bytes of the single device block that hla_cache_init carves (256-byte aligned
+ * sub-buffers).  Returns 0 for an unsupported config. */
+size_t hla_cache_bytes(const hla_config* cfg, int32_t max_chunks);
+
+/* Fill *out with pointers into mem (device, >= hla_cache_bytes) and enqueue the
+ * zeroing of the counters on stream.  Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE,
+ * CUDA. */
+hla_status hla_cache_init(const hla_config* cfg, int32_t max_chunks, void* mem, size_t bytes,
+                          hla_cache* out, hla_stream_t stream);
+
+/* Workspace bytes that hla_prefill needs for cfg (0 for an unsupported config). */
+size_t hla_prefill_workspace_bytes(const hla_config* cfg);
+
+/* Workspace bytes that hla_decode_step needs for a cache of max_chunks chunks. */
+size_t hla_decode_workspace_bytes(const hla_config* cfg, int32_t max_chunks);
+
+/*
+ * gdn_chunk_transitions -- the exact affine transition of every complete chunk
+ * (Methodology para. 1), built through the chunkwise WY/UT form:
+ *   l_t = sum_{s<=t} log alpha_s, gamma_t = exp(l_t), Gamma_ts = exp(l_t - l_s)
+ *   L = strictly-lower(diag(beta) (Gamma o K K^T)), T = (I + L)^{-1} diag(beta)
+ *   Wb = T diag(gamma) K, Ub = T V, D = diag(gamma_C / gamma_t)
+ *   A_c = gamma_C I - Wb^T D K,  B_c = Ub^T D K.
+ * In:  k, v [B,T,H,d] dtype; alpha, beta [B,T,H] float32 (device).
+ * Out: A_out [B,H,T/C,d,d], B_out [B,H,T/C,d,d] dtype (device); a final partial
+ *      chunk has no output.  Errors: INVALID_ARG, UNSUPPORTED, CUDA.
+ */
+hla_status gdn_chunk_transitions(const hla_config* cfg, const void* k, const void* v,
+                                 const float* alpha, const float* beta, void* A_out,
+                                 void* B_out, hla_stream_t stream);
+
+/*
+ * hla_routing -- pools and gates only (Overview; Methodology paras. 2 and 4).
+ * In:  q_route, k_route [B,T,H,d] dtype (device; NULL is not allowed here).
+ * Out: rq_out, rk_out [B,H,N,d] float32 (required), N = ceil(T/C);
+ *      gates_out [B,H,N,N] float32 raw gates for j < i, 0 elsewhere (may be NULL);
+ *      active_idx_out [B,H,N,N] int32: entries 0..cnt-1 of row i are the active j
+ *      in ascending order, the rest are -1 (may be NULL together with cnt);
+ *      active_cnt_out [B,H,N] int32.
+ * Honours gate_mode (ONE/ZERO give 1/0 gates; USER is not accepted here).
+ */
+hla_status hla_routing(const hla_config* cfg, const void* q_route, const void* k_route,
+                       float* rq_out, float* rk_out, float* gates_out,
+                       int32_t* active_idx_out, int32_t* active_cnt_out, hla_stream_t stream);
+
+/*
+ * hla_prefill -- HLA over a whole prompt (Key Contributions 3; Methodology paras. 1-4).
+ * In:  q, k, v [B,T,H,d] dtype; alpha, beta [B,T,H] float32;
+ *      q_route, k_route [B,T,H,d] dtype or NULL (NULL: q, k);
+ *      user_gates [B,H,N,N] float32 (HLA_GATES_USER only, else ignored).
+ * Out: o [B,T,H,d] dtype.  Optional (NULL to skip): gates_out, active_idx_out,
+ *      active_cnt_out as in hla_routing; cache_out -- an initialised cache with
+ *      max_chunks >= T/C, filled with A/B/rk of every complete chunk, the final
+ *      partial chunk's tokens and the counters.
+ * workspace: device, >= hla_prefill_workspace_bytes(cfg), 256-byte aligned.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
+ */
+hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, const void* v,
+                       const float* alpha, const float* beta, const void* q_route,
+                       const void* k_route, const float* user_gates, void* o,
+                       float* gates_out, int32_t* active_idx_out, int32_t* active_cnt_out,
+                       hla_cache* cache_out, void* workspace, size_t workspace_bytes,
+                       hla_stream_t stream);
+
+/*
+ * hla_decode_step -- one new token per sequence (Key Contributions 3: dynamic
+ * autoregressive decoding; Methodology para. 4: skipped chunks are not read).
+ * In:  q, k, v [B,H,d] dtype; alpha, beta [B,H] float32; q_route, k_route [B,H,d]
+ *      or NULL (q, k).  cache: initialised (by hla_prefill or empty).
+ * Out: o [B,H,d] dtype.  The token is appended to the open chunk; the query pool
+ *      runs over the open chunk's m tokens so far; gates against every closed
+ *      chunk's key pool; active chunks are applied by the equivalent right-to-left
+ *      form  y += g_j B_j x; x <- (1-g_j) x + g_j A_j x  (j descending), which reads
+ *      each active A_j/B_j once; when the open chunk reaches C tokens it is closed
+ *      (its A/B/rk are appended).  Gate modes ROUTED, ONE and ZERO.
+ * workspace: device, >= hla_decode_workspace_bytes(cfg, cache->max_chunks).
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE (also: cache full), CUDA.
+ */
+hla_status hla_decode_step(const hla_config* cfg, hla_cache* cache, const void* q,
+                           const void* k, const void* v, const float* alpha,
+                           const float* beta, const void* q_route, const void* k_route,
+                           void* o, void* workspace, size_t workspace_bytes,
+                           hla_stream_t stream);
+
+/*
+ * Bounded device waits.  Kernels that wait on an mbarrier or a flag give up after
+ * a fixed number of polls, record a code in a device-side error word and return.
+ * hla_device_status synchronises the device, reads and (if clear != 0) resets that
+ * word; it returns HLA_ERR_TIMEOUT if a wait expired since the last reset, else
+ * HLA_OK (or HLA_ERR_CUDA).  *code_out (may be NULL) receives the raw word.
+ */
+hla_status hla_device_status(int32_t clear, uint32_t* code_out);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HLA_H_ */

@@ -1,0 +1,145 @@
+"""C ABI checks that need no GPU: the library loads, exports every symbol that
+include/hla.h declares, sizes its cache and workspaces by the stated arithmetic,
+and rejects bad arguments on the host before any launch."""
+import ctypes
+import json
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hla.h")
+
+
+@pytest.fixture(scope="module")
+def hla():
+    from gated_delta_rule_transitions_b200 import _hla
+    from gated_delta_rule_transitions_b200 import build as b
+    b.build()
+    return _hla
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^[A-Za-z_][\w\s\*]*?\b([a-z_][a-z0-9_]*)\s*\(", src, flags=re.M)
+    return sorted(set(n for n in names if n not in ("defined",)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("gdn_chunk_transitions", "hla_prefill", "hla_decode_step", "hla_routing",
+              "hla_prefill_workspace_bytes", "hla_cache_bytes", "hla_cache_init",
+              "hla_decode_workspace_bytes", "hla_last_error", "hla_device_status"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(hla):
+    L = hla.lib()
+    for n in declared_functions():
+        assert hasattr(L, n), n
+    assert set(hla.EXPORTS) <= set(declared_functions())
+
+
+def cfg(hla, **kw):
+    base = dict(B=1, H=1, T=4096, C=64, d=128, dtype="bf16")
+    base.update(kw)
+    return hla.make_config(**base)
+
+
+def test_cache_bytes_match_affine_state_arithmetic(hla):
+    """Main Findings (affine-state memory): the per-chunk A and B, d x d each at 2
+    bytes, reproduce the page's 2 MiB KV figure and its 100/50/25/12.5% table."""
+    gold = json.load(open(os.path.join(ROOT, "tests", "golden", "affine_state_memory.json")))
+    d = gold["head_dim"]
+    c = cfg(hla, d=d)
+    per_chunk = hla.cache_bytes(c, 101) - hla.cache_bytes(c, 100)
+    rk_bytes = d * 4  # float32 key pool per chunk (routing only)
+    ab_bytes = per_chunk - rk_bytes
+    assert ab_bytes == 2 * d * d * 2
+    kv = gold["context_tokens"] * 2 * d * 2
+    assert kv == gold["kv_cache_bytes_per_layer_head"]
+    for C, frac in gold["affine_state_fraction_of_kv"].items():
+        chunks = gold["context_tokens"] // int(C)
+        assert chunks * ab_bytes / kv == pytest.approx(frac, abs=0)
+    # float32 storage doubles the A/B part
+    c32 = cfg(hla, d=d, dtype="f32")
+    assert hla.cache_bytes(c32, 101) - hla.cache_bytes(c32, 100) - rk_bytes == 2 * d * d * 4
+
+
+def test_decode_workspace_and_cache_sizes(hla):
+    c = hla.make_config(64, 16, 1, 64, 128, "bf16")
+    # config of a 64-sequence, 512-chunk decode: 32 GiB of A/B
+    nb = hla.cache_bytes(c, 512)
+    assert nb >= 64 * 16 * 512 * 2 * 128 * 128 * 2
+    assert nb < 64 * 16 * 512 * 2 * 128 * 128 * 2 * 1.02
+    assert hla.decode_workspace_bytes(c, 512) == 2 * 64 * 16 * 512 * 4
+
+
+def test_prefill_workspace_grows_with_T(hla):
+    a = hla.prefill_workspace_bytes(cfg(hla, T=1024))
+    b = hla.prefill_workspace_bytes(cfg(hla, T=2048))
+    assert 0 < a < b
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(C=32), 2), (dict(d=96), 2), (dict(T=0), 1), (dict(B=0), 1), (dict(tau=0.0), 1),
+])
+def test_bad_config_rejected_on_host(hla, kw, status):
+    c = cfg(hla, **kw)
+    P = ctypes.c_void_p(0x100000)
+    st = hla.lib().gdn_chunk_transitions(ctypes.byref(c), P, P, P, P, P, P, None)
+    assert st == status
+    assert hla.last_error() != ""
+    assert hla.prefill_workspace_bytes(c) == 0
+
+
+def test_null_and_misaligned_pointers_rejected(hla):
+    c = cfg(hla, T=256)
+    P = ctypes.c_void_p(0x100000)
+    L = hla.lib()
+    assert L.gdn_chunk_transitions(ctypes.byref(c), None, P, P, P, P, P, None) == hla.HLA_ERR_INVALID_ARG
+    assert "k is NULL" in hla.last_error()
+    bad = ctypes.c_void_p(0x100008)
+    assert L.gdn_chunk_transitions(ctypes.byref(c), P, bad, P, P, P, P, None) == hla.HLA_ERR_INVALID_ARG
+    assert "aligned" in hla.last_error()
+
+
+def test_small_workspace_rejected_before_launch(hla):
+    c = cfg(hla, T=256)
+    P = ctypes.c_void_p(0x100000)
+    need = hla.prefill_workspace_bytes(c)
+    st = hla.lib().hla_prefill(ctypes.byref(c), P, P, P, P, P, None, None, None, P, None, None, None, None,
+                               P, need - 256, None)
+    assert st == hla.HLA_ERR_WORKSPACE
+    assert "workspace too small" in hla.last_error()
+
+
+def test_user_gates_required_in_user_mode(hla):
+    c = cfg(hla, T=256, gate_mode="user")
+    P = ctypes.c_void_p(0x100000)
+    st = hla.lib().hla_prefill(ctypes.byref(c), P, P, P, P, P, None, None, None, P, None, None, None, None,
+                               P, 1 << 40, None)
+    assert st == hla.HLA_ERR_INVALID_ARG and "user_gates" in hla.last_error()
+
+
+def test_decode_rejects_user_gates_and_foreign_cache(hla):
+    c = cfg(hla, T=1, gate_mode="user")
+    P = ctypes.c_void_p(0x100000)
+    cache = hla.HlaCache()
+    st = hla.lib().hla_decode_step(ctypes.byref(c), ctypes.byref(cache), P, P, P, P, P, None, None, P, P, 1 << 30,
+                                   None)
+    assert st == hla.HLA_ERR_UNSUPPORTED
+    c = cfg(hla, T=1)
+    st = hla.lib().hla_decode_step(ctypes.byref(c), ctypes.byref(cache), P, P, P, P, P, None, None, P, P, 1 << 30,
+                                   None)
+    assert st == hla.HLA_ERR_INVALID_ARG and "different config" in hla.last_error()
+
+
+def test_python_binding_refuses_cpu_tensors(hla):
+    import torch
+    c = cfg(hla, T=64, d=64, dtype="f32")
+    x = torch.zeros(1, 64, 1, 64)
+    with pytest.raises(ValueError, match="CUDA"):
+        hla.gdn_chunk_transitions(c, x, x, x[..., 0], x[..., 0], x, x)

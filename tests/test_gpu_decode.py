@@ -1,0 +1,110 @@
+"""GPU parity of the decode step against the oracle (through the C ABI).
+
+A prefill writes the cache; chained decode steps (crossing a chunk boundary, so a
+chunk is closed into the cache) are compared token by token with the oracle's
+decode state, which follows the definition (forward composition of S_in, then the
+token rule over the open chunk).  Cached key pools must be bit-exact."""
+import numpy as np
+import pytest
+import torch
+
+import hla_synth as syn
+from oracle import hla_oracle as ho
+from tests import _parity as P
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def hla():
+    import gated_delta_rule_transitions_b200 as m
+    m.lib()
+    return m._hla
+
+
+def _route_tokens(B, H, d, steps, seed, dtype):
+    g = torch.Generator().manual_seed(seed)
+    out = []
+    for _ in range(steps):
+        mu = torch.randn((B, H, d), generator=g) * 1.4
+        out.append((mu.to(dtype), (mu + 0.3 * torch.randn((B, H, d), generator=g)).to(dtype)))
+    return out
+
+
+@pytest.mark.parametrize("dtype,d,mode,thr,route", [
+    ("f32", 64, "routed", 0.05, False),
+    ("f32", 64, "routed", 0.4, True),
+    ("bf16", 128, "routed", 0.05, False),
+    ("bf16", 128, "routed", 0.4, True),
+    ("bf16", 128, "one", 0.0, False),
+    ("f32", 64, "zero", 0.0, False),
+])
+def test_decode_chain_matches_oracle(hla, dtype, d, mode, thr, route):
+    T0 = 64 * 3 + 58
+    steps = 9  # closes chunk 3 after 6 steps, then opens chunk 4
+    w = syn.DECODE_32K.with_(B=2, H=2, T=T0, dtype=dtype, d=d, gate_mode=mode, thr=thr,
+                             route="spread" if route else "default", bias=-0.5 if route else -2.0)
+    inp = P.gpu_inputs(w)
+    cfg = hla.make_config(w.B, w.H, T0, 64, d, dtype, mode, w.tau, w.bias, w.thr)
+    cache = hla.Cache(cfg, max_chunks=8)
+    P.run_prefill(hla, w, inp, cache=cache)
+    toks = syn.make_decode_tokens(w, steps)
+    tdt = syn.torch_dtype(w)
+    routes = _route_tokens(w.B, w.H, d, steps, 77, tdt) if route else [(None, None)] * steps
+    heads = {}
+    for b in range(w.B):
+        for h in range(w.H):
+            f = lambda n: None if inp.get(n) is None else inp[n][b, :, h]
+            heads[(b, h)] = ho.HlaDecodeHead.from_prefill(
+                P.np64(f("q")), P.np64(f("k")), P.np64(f("v")), P.np64(f("alpha")), P.np64(f("beta")), 64,
+                w.tau, w.bias, w.thr, mode,
+                None if f("q_route") is None else P.np32(f("q_route")),
+                None if f("k_route") is None else P.np32(f("k_route")))
+    dcfg = hla.make_config(w.B, w.H, 1, 64, d, dtype, mode, w.tau, w.bias, w.thr)
+    errs = []
+    for s, tk in enumerate(toks):
+        g = {k: v.cuda().contiguous() for k, v in tk.items()}
+        qr, kr = routes[s]
+        o = torch.empty_like(g["q"])
+        hla.hla_decode_step(dcfg, cache, g["q"], g["k"], g["v"], g["alpha"], g["beta"], o,
+                            q_route=None if qr is None else qr.cuda(), k_route=None if kr is None else kr.cuda())
+        torch.cuda.synchronize()
+        o = P.np64(o)
+        for (b, h), st in heads.items():
+            ref = st.step(P.np64(tk["q"][b, h]), P.np64(tk["k"][b, h]), P.np64(tk["v"][b, h]),
+                          float(tk["alpha"][b, h]), float(tk["beta"][b, h]),
+                          None if qr is None else P.np32(qr[b, h]), None if kr is None else P.np32(kr[b, h]))
+            errs.append((o[b, h], ref))
+    got = np.stack([e[0] for e in errs])
+    ref = np.stack([e[1] for e in errs])
+    if dtype == "f32":
+        assert np.abs(got - ref).max() <= P.TOL_F32_MAXABS
+    else:
+        assert P.rel_l2(got, ref) <= P.TOL_BF16_RELL2
+    st, code = hla.hla_device_status()
+    assert st == 0 and code == 0
+    # counters and the closed chunk's key pool
+    n = cache.view("n_chunks", (w.B,), torch.int32).cpu()
+    m = cache.view("m_partial", (w.B,), torch.int32).cpu()
+    assert n.tolist() == [4] * w.B and m.tolist() == [(T0 + steps) % 64] * w.B
+    rk = cache.view("rk", (w.B, w.H, 8, d), torch.float32).cpu().numpy()
+    for (b, h), st_ in heads.items():
+        for j in range(4):
+            assert np.array_equal(rk[b, h, j].view(np.uint32), st_.rk[j].view(np.uint32))
+
+
+def test_decode_cache_full_is_reported(hla):
+    w = syn.DECODE_32K.with_(B=1, H=1, T=64 * 2 + 63, dtype="f32", d=64)
+    inp = P.gpu_inputs(w)
+    cfg = hla.make_config(1, 1, w.T, 64, 64, "f32", "routed", 1.0, -2.0, 0.05)
+    cache = hla.Cache(cfg, max_chunks=2)
+    P.run_prefill(hla, w, inp, cache=cache)
+    tk = syn.make_decode_tokens(w, 1)[0]
+    g = {k: v.cuda().contiguous() for k, v in tk.items()}
+    o = torch.empty_like(g["q"])
+    hla.hla_decode_step(hla.make_config(1, 1, 1, 64, 64, "f32", "routed", 1.0, -2.0, 0.05), cache,
+                        g["q"], g["k"], g["v"], g["alpha"], g["beta"], o)
+    st, code = hla.hla_device_status(clear=True)
+    assert st == hla.HLA_ERR_WORKSPACE and code & 4
+    st, code = hla.hla_device_status(clear=True)
+    assert st == 0 and code == 0

@@ -1,0 +1,202 @@
+"""GPU parity of the prefill path against the oracle (through the C ABI).
+
+Bars: gates and active lists bit-exact; outputs max-abs <= 1e-4 on the float32 path
+and relative L2 <= 2e-2 on the bf16 path (over the whole output tensor)."""
+import numpy as np
+import pytest
+import torch
+
+import hla_synth as syn
+from oracle import hla_oracle as ho
+from oracle import routing_recipe as rr
+from tests import _parity as P
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def hla():
+    import gated_delta_rule_transitions_b200 as m
+    m.lib()
+    return m._hla
+
+
+def _oracle_all(w, inp, user_gates=None):
+    B, T, H, _ = inp["q"].shape
+    o = np.zeros(tuple(inp["v"].shape), np.float64)
+    res = {}
+    for b in range(B):
+        for h in range(H):
+            r = P.oracle_prefill_head(w, inp, b, h, user_gates)
+            o[b, :, h] = r.o
+            res[(b, h)] = r
+    return o, res
+
+
+def test_tiny_f32_prefill(hla):
+    w = syn.TINY_F32
+    inp = P.gpu_inputs(w)
+    o, gates, aidx, acnt = P.run_prefill(hla, w, inp)
+    ref, res = _oracle_all(w, inp)
+    assert np.abs(P.np64(o) - ref).max() <= P.TOL_F32_MAXABS
+    for (b, h), r in res.items():
+        P.check_routing_exact(r, gates, aidx, acnt, b, h)
+
+
+@pytest.mark.parametrize("T", [64 * 5, 64 * 5 + 17, 40])
+def test_bf16_spread_gates_ragged(hla, T):
+    w = syn.PREFILL_0P8B.with_(B=2, H=2, T=T)
+    inp = P.gpu_inputs(w)
+    o, gates, aidx, acnt = P.run_prefill(hla, w, inp)
+    ref, res = _oracle_all(w, inp)
+    assert P.rel_l2(P.np64(o), ref) <= P.TOL_BF16_RELL2
+    for (b, h), r in res.items():
+        P.check_routing_exact(r, gates, aidx, acnt, b, h)
+    g = np.concatenate([r.gates[np.tril_indices(r.gates.shape[0], -1)] for r in res.values()])
+    if g.size > 10:
+        assert g.min() < 0.2 and g.max() > 0.5  # spread over (0, 1)
+
+
+def test_f32_routed_thresholded(hla):
+    w = syn.SPARSE_LONG.with_(B=1, H=2, T=64 * 12, dtype="f32", d=64, topics=3)
+    inp = P.gpu_inputs(w)
+    o, gates, aidx, acnt = P.run_prefill(hla, w, inp)
+    ref, res = _oracle_all(w, inp)
+    assert np.abs(P.np64(o) - ref).max() <= P.TOL_F32_MAXABS
+    skipped = 0
+    for (b, h), r in res.items():
+        P.check_routing_exact(r, gates, aidx, acnt, b, h)
+        skipped += sum(i - len(a) for i, a in enumerate(r.active))
+    assert skipped > 0
+
+
+def test_bf16_planted_sparse(hla):
+    w = syn.SPARSE_LONG.with_(B=1, H=2, T=64 * 20, topics=4)
+    inp = P.gpu_inputs(w)
+    o, gates, aidx, acnt = P.run_prefill(hla, w, inp)
+    ref, res = _oracle_all(w, inp)
+    assert P.rel_l2(P.np64(o), ref) <= P.TOL_BF16_RELL2
+    for (b, h), r in res.items():
+        P.check_routing_exact(r, gates, aidx, acnt, b, h)
+        kept = [len(a) for a in r.active]
+        assert 0 < sum(kept) < sum(range(len(kept)))
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_gates_one_is_native_gdn(hla, dtype):
+    w = syn.GDN_REDUCTION.with_(B=2, H=2, T=64 * 4 + 9, dtype=dtype, d=64 if dtype == "f32" else 128)
+    inp = P.gpu_inputs(w)
+    o, gates, aidx, acnt = P.run_prefill(hla, w, inp)
+    for b in range(2):
+        for h in range(2):
+            ref, _ = ho.gdn_recurrent(P.np64(inp["q"][b, :, h]), P.np64(inp["k"][b, :, h]),
+                                      P.np64(inp["v"][b, :, h]), P.np64(inp["alpha"][b, :, h]),
+                                      P.np64(inp["beta"][b, :, h]))
+            got = P.np64(o[b, :, h])
+            if dtype == "f32":
+                assert np.abs(got - ref).max() <= P.TOL_F32_MAXABS
+            else:
+                assert P.rel_l2(got, ref) <= P.TOL_BF16_RELL2
+
+
+def test_gates_zero_is_intra_chunk_only(hla):
+    w = syn.TINY_F32.with_(gate_mode="zero", T=64 * 3 + 5)
+    inp = P.gpu_inputs(w)
+    o, *_ = P.run_prefill(hla, w, inp)
+    for h in range(2):
+        for c in range(4):
+            sl = slice(64 * c, min(64 * c + 64, w.T))
+            ref, _ = ho.gdn_recurrent(P.np64(inp["q"][0, sl, h]), P.np64(inp["k"][0, sl, h]),
+                                      P.np64(inp["v"][0, sl, h]), P.np64(inp["alpha"][0, sl, h]),
+                                      P.np64(inp["beta"][0, sl, h]))
+            assert np.abs(P.np64(o[0, sl, h]) - ref).max() <= P.TOL_F32_MAXABS
+
+
+def test_identity_tokens_give_zero_output(hla):
+    w = syn.TINY_F32
+    inp = P.gpu_inputs(w)
+    inp["alpha"] = torch.ones_like(inp["alpha"])
+    inp["beta"] = torch.zeros_like(inp["beta"])
+    o, *_ = P.run_prefill(hla, w, inp)
+    assert torch.count_nonzero(o) == 0
+
+
+def test_user_gates(hla):
+    w = syn.TINY_F32.with_(gate_mode="user", thr=0.3)
+    inp = P.gpu_inputs(w)
+    ug = syn.make_user_gates(w)
+    o, gates, aidx, acnt = P.run_prefill(hla, w, inp, user_gates=ug)
+    ref, res = _oracle_all(w, inp, user_gates=ug)
+    assert np.abs(P.np64(o) - ref).max() <= P.TOL_F32_MAXABS
+    for (b, h), r in res.items():
+        P.check_routing_exact(r, gates, aidx, acnt, b, h)
+
+
+@pytest.mark.parametrize("dtype,d", [("f32", 64), ("f32", 128), ("bf16", 128), ("bf16", 64)])
+def test_gdn_chunk_transitions(hla, dtype, d):
+    w = syn.TINY_F32.with_(dtype=dtype, d=d, B=2, H=3, T=64 * 3 + 11)
+    inp = P.gpu_inputs(w)
+    B, T, H = 2, w.T, 3
+    cfg = hla.make_config(B, H, T, 64, d, dtype)
+    g = P.to_cuda(inp)
+    tdt = torch.float32 if dtype == "f32" else torch.bfloat16
+    A = torch.empty((B, H, T // 64, d, d), dtype=tdt, device="cuda")
+    Bm = torch.empty_like(A)
+    hla.gdn_chunk_transitions(cfg, g["k"], g["v"], g["alpha"], g["beta"], A, Bm)
+    torch.cuda.synchronize()
+    A, Bm = P.np64(A), P.np64(Bm)
+    for b in range(B):
+        for h in range(H):
+            for c in range(T // 64):
+                sl = slice(64 * c, 64 * c + 64)
+                Ar, Br = ho.chunk_transition(P.np64(inp["k"][b, sl, h]), P.np64(inp["v"][b, sl, h]),
+                                             P.np64(inp["alpha"][b, sl, h]), P.np64(inp["beta"][b, sl, h]))
+                if dtype == "f32":
+                    assert np.abs(A[b, h, c] - Ar).max() <= P.TOL_F32_MAXABS
+                    assert np.abs(Bm[b, h, c] - Br).max() <= P.TOL_F32_MAXABS
+                else:
+                    # bf16 storage: every entry within half an ulp of bf16 plus fp32 error
+                    assert np.all(np.abs(A[b, h, c] - Ar) <= np.abs(Ar) * 2 ** -8 + 1e-4)
+                    assert np.all(np.abs(Bm[b, h, c] - Br) <= np.abs(Br) * 2 ** -8 + 1e-4)
+
+
+@pytest.mark.parametrize("dtype,d,T", [("f32", 64, 64 * 7 + 3), ("bf16", 128, 64 * 9)])
+def test_routing_bit_exact(hla, dtype, d, T):
+    w = syn.PREFILL_0P8B.with_(B=2, H=3, T=T, dtype=dtype, d=d, thr=0.3)
+    inp = P.gpu_inputs(w)
+    B, H, N = 2, 3, (T + 63) // 64
+    cfg = hla.make_config(B, H, T, 64, d, dtype, "routed", w.tau, w.bias, w.thr)
+    g = P.to_cuda(inp)
+    rq = torch.empty((B, H, N, d), device="cuda")
+    rk = torch.empty_like(rq)
+    gates = torch.empty((B, H, N, N), device="cuda")
+    aidx = torch.empty((B, H, N, N), dtype=torch.int32, device="cuda")
+    acnt = torch.empty((B, H, N), dtype=torch.int32, device="cuda")
+    hla.hla_routing(cfg, g["q_route"], g["k_route"], rq, rk, gates, aidx, acnt)
+    torch.cuda.synchronize()
+    for b in range(B):
+        for h in range(H):
+            qr = P.np32(inp["q_route"][b, :, h])
+            kr = P.np32(inp["k_route"][b, :, h])
+            rq_ref = ho.route_pools(qr, 64, w.tau)
+            rk_ref = ho.route_pools(kr, 64, w.tau)
+            assert np.array_equal(rq[b, h].cpu().numpy().view(np.uint32), rq_ref.view(np.uint32))
+            assert np.array_equal(rk[b, h].cpu().numpy().view(np.uint32), rk_ref.view(np.uint32))
+            G = ho.gate_matrix(rq_ref, rk_ref, d, w.bias)
+            act = ho.active_lists(G, w.thr)
+            res = ho.HeadResult(o=None, gates=G, active=act, rq=rq_ref, rk=rk_ref)
+            P.check_routing_exact(res, gates.cpu(), aidx.cpu(), acnt.cpu(), b, h)
+
+
+def test_full_size_prefill_sampled(hla):
+    """Dense 0.8B-like layer (T=16384, H=16, d=128, bf16): all gates bit-exact on
+    two heads; sampled query chunks against the oracle."""
+    w = syn.PREFILL_0P8B
+    inp = P.gpu_inputs(w)
+    o, gates, aidx, acnt = P.run_prefill(hla, w, inp)
+    for h in (0, 9):
+        sample = [0, 1, 37, 128, 255]
+        r = P.oracle_prefill_head(w, inp, 0, h, query_chunks=sample)
+        P.check_routing_exact(r, gates, aidx, acnt, 0, h)
+        rows = np.concatenate([np.arange(64 * i, 64 * i + 64) for i in sample])
+        assert P.rel_l2(P.np64(o[0, rows, h]), r.o[rows]) <= P.TOL_BF16_RELL2
