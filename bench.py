@@ -1,0 +1,456 @@
+#!/usr/bin/env python
+"""HLA prefill and decode benchmark on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one pass of the hot path over synthetic inputs already resident in HBM:
+  * prefill of the dense 0.8B-like layer (B=1, H=16, T=16384, C=64, d=128, bf16,
+    bias -2 with spread route inputs, no skipping): pools, gates, chunk
+    transitions, gated composition, read-out;
+  * one decode step of 64 sequences with 32768-token contexts (512 cached A_j/B_j
+    per head, H=16, d=128, bf16, bias -2, threshold 0.05: every chunk active).
+The L2 cache is flushed (256 MiB write, untimed) before each timed phase.  Each
+phase is timed with CUDA events on the launching stream; per-stage times come from
+the library's own event pairs (hla_profile_*), on the same stream.
+
+``value`` is prefill tokens/s (whole job: every rank runs an independent replica,
+weak scaling, max time over ranks); the decode numbers are in ``decode``.  The
+``reference`` arm times the CPU oracle on a bounded sample of the same workloads.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "HLA prefill tokens/s (% bf16 tensor peak); decode tokens/s at 32K (% HBM BW)"
+L2_FLUSH_BYTES = 256 << 20
+# algorithmic flops per chunk at C=64, d=128 (see the kernel headers):
+#   transition: K K^T 2C^2d + Wb, Ub 2*2C^2d + A, B 2*2Cd^2  (triangular solve ignored)
+#   read-out:   Q S^T, Wb S^T 2*2Cd^2 + Q K^T 2C^2d + P X 2C^2d
+FLOP_TRANSITION = 3 * 2 * 64 * 64 * 128 + 2 * 2 * 64 * 128 * 128
+FLOP_READOUT = 2 * 2 * 64 * 128 * 128 + 2 * 2 * 64 * 64 * 128
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.samples = []
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                out = subprocess.run(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                      "--format=csv,noheader,nounits"], capture_output=True, text=True,
+                                     timeout=5).stdout.strip()
+                if out:
+                    self.samples.append([x.strip() for x in out.split(",")])
+            except Exception:
+                pass
+            self._stop.wait(0.2)
+
+    def __enter__(self):
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        self._t.join(timeout=10)
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        mx = [float(s[2]) for s in self.samples if s[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in self.samples for i in range(4) if len(s) > 5 + i and s[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------------
+
+def build_decode_cache(hla, syn, torch, w, max_chunks, group=8):
+    """Fill a decode cache for w.B sequences of w.T-token contexts through the public
+    API: hla_prefill with every earlier-chunk weight 0 writes the cache (A/B/key pools
+    do not depend on gates) without the quadratic composition."""
+    cfg = hla.make_config(w.B, w.H, w.T, w.C, w.d, w.dtype, "routed", w.tau, w.bias, w.thr)
+    cache = hla.Cache(cfg, max_chunks)
+    gcfg = hla.make_config(group, w.H, w.T, w.C, w.d, w.dtype, "zero", w.tau, w.bias, w.thr)
+    ws = torch.empty(hla.prefill_workspace_bytes(gcfg), dtype=torch.uint8, device="cuda")
+    es = 2 if w.dtype == "bf16" else 4
+    per_b = {  # bytes per sequence of each buffer
+        "A": w.H * max_chunks * w.d * w.d * es, "Bm": w.H * max_chunks * w.d * w.d * es,
+        "rk": w.H * max_chunks * w.d * 4, "buf_k": w.H * w.C * w.d * es, "buf_v": w.H * w.C * w.d * es,
+        "buf_qr": w.H * w.C * w.d * es, "buf_kr": w.H * w.C * w.d * es, "buf_alpha": w.H * w.C * 4,
+        "buf_beta": w.H * w.C * 4, "n_chunks": 4, "m_partial": 4}
+    first_ctx = None
+    for b0 in range(0, w.B, group):
+        ctx = syn.make_context_group(w, b0, group, device="cuda")
+        if b0 == 0:
+            first_ctx = {k: v[:2].clone() for k, v in ctx.items()}
+        sub = hla.HlaCache()
+        ctypes_fields = [f[0] for f in hla.HlaCache._fields_]
+        for f in ctypes_fields:
+            setattr(sub, f, getattr(cache.struct, f))
+        sub.B = group
+        for f, nb in per_b.items():
+            setattr(sub, f, getattr(cache.struct, f) + b0 * nb)
+        holder = type("SubCache", (), {})()
+        holder.struct = sub
+        o = torch.empty_like(ctx["q"])
+        hla.hla_prefill(gcfg, ctx["q"], ctx["k"], ctx["v"], ctx["alpha"], ctx["beta"], o, cache=holder,
+                        workspace=ws)
+        del ctx, o
+    torch.cuda.synchronize()
+    del ws
+    return cache, first_ctx
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import gated_delta_rule_transitions_b200 as pkg
+    import hla_synth as syn
+
+    hla = pkg._hla
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    hbm_gbs, bf16_tf, bf16_tf_sus, peak_src = _peaks()
+    stream = torch.cuda.current_stream()
+
+    # ---- prefill workload (inputs resident in HBM) ----
+    wp = syn.PREFILL_0P8B
+    inp = syn.make_gdn_inputs(wp)
+    qr, kr = syn.make_route_inputs(wp)
+    inp["q_route"], inp["k_route"] = qr, kr
+    host = {k: v.contiguous().pin_memory() for k, v in inp.items()}
+    dev = {k: v.cuda() for k, v in host.items()}
+    pcfg = hla.make_config(wp.B, wp.H, wp.T, wp.C, wp.d, wp.dtype, wp.gate_mode, wp.tau, wp.bias, wp.thr)
+    pws = torch.empty(hla.prefill_workspace_bytes(pcfg), dtype=torch.uint8, device="cuda")
+    o = torch.empty_like(dev["q"])
+    o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    N = wp.N
+    acnt = torch.empty((wp.B, wp.H, N), dtype=torch.int32, device="cuda")
+
+    def prefill():
+        hla.hla_prefill(pcfg, dev["q"], dev["k"], dev["v"], dev["alpha"], dev["beta"], o,
+                        q_route=dev["q_route"], k_route=dev["k_route"], workspace=pws)
+
+    # ---- decode workload ----
+    wd = syn.DECODE_32K
+    max_chunks = wd.T // wd.C + 1
+    cache, ctx0 = build_decode_cache(hla, syn, torch, wd, max_chunks)
+    dcfg = hla.make_config(wd.B, wd.H, 1, wd.C, wd.d, wd.dtype, wd.gate_mode, wd.tau, wd.bias, wd.thr)
+    dws = torch.empty(hla.decode_workspace_bytes(dcfg, max_chunks), dtype=torch.uint8, device="cuda")
+    ntok = args.warmup + args.steps + 1
+    toks_host = [{k: v.contiguous().pin_memory() for k, v in t.items()} for t in syn.make_decode_tokens(wd, ntok)]
+    toks = [{k: v.cuda() for k, v in t.items()} for t in toks_host]
+    od = torch.empty_like(toks[0]["q"])
+    od_host = torch.empty(od.shape, dtype=od.dtype).pin_memory()
+    step_idx = [0]
+
+    def decode():
+        t = toks[step_idx[0]]
+        step_idx[0] += 1
+        hla.hla_decode_step(dcfg, cache, t["q"], t["k"], t["v"], t["alpha"], t["beta"], od, workspace=dws)
+
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+
+    def l2_flush():
+        flush.zero_()
+
+    for _ in range(max(args.warmup, 0)):
+        prefill()
+        l2_flush()
+        decode()
+        l2_flush()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+    # active pairs of the prefill (for the algorithmic flop count)
+    hla.hla_prefill(pcfg, dev["q"], dev["k"], dev["v"], dev["alpha"], dev["beta"], o,
+                    q_route=dev["q_route"], k_route=dev["k_route"], workspace=pws, active_cnt_out=acnt,
+                    active_idx_out=torch.empty((wp.B, wp.H, N, N), dtype=torch.int32, device="cuda"))
+    torch.cuda.synchronize()
+    active_pairs = int(acnt.sum().item())
+
+    hla.hla_profile_read(reset=True)
+    hla.hla_profile_enable(True)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(4 * args.steps)]
+    with ClockSampler(local) as clocks:
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        for s in range(args.steps):
+            e = ev[2 * s]
+            e[0].record(stream)
+            prefill()
+            e[1].record(stream)
+            l2_flush()
+            e = ev[2 * s + 1]
+            e[0].record(stream)
+            decode()
+            e[1].record(stream)
+            l2_flush()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+    hla.hla_profile_enable(False)
+    stages = hla.hla_profile_read(reset=True)
+    pre_ms = sum(ev[2 * s][0].elapsed_time(ev[2 * s][1]) for s in range(args.steps)) / args.steps
+    dec_ms = sum(ev[2 * s + 1][0].elapsed_time(ev[2 * s + 1][1]) for s in range(args.steps)) / args.steps
+    t = torch.tensor([pre_ms, dec_ms], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    pre_ms, dec_ms = float(t[0]), float(t[1])
+
+    # ---- end to end through the public API with host buffers ----
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(2)]
+    reps = max(1, min(args.steps, 5))
+    e2e_pre = e2e_dec = 0.0
+    for _ in range(reps):
+        l2_flush()
+        e2e_ev[0][0].record(stream)
+        for k in dev:
+            dev[k].copy_(host[k], non_blocking=True)
+        prefill()
+        o_host.copy_(o, non_blocking=True)
+        e2e_ev[0][1].record(stream)
+        l2_flush()
+        e2e_ev[1][0].record(stream)
+        t_ = toks[step_idx[0] % len(toks)]
+        th = toks_host[step_idx[0] % len(toks)]
+        for k in t_:
+            t_[k].copy_(th[k], non_blocking=True)
+        decode_idx = step_idx[0] % len(toks)
+        step_idx[0] = decode_idx
+        decode()
+        od_host.copy_(od, non_blocking=True)
+        e2e_ev[1][1].record(stream)
+        torch.cuda.synchronize()
+        e2e_pre += e2e_ev[0][0].elapsed_time(e2e_ev[0][1]) / reps
+        e2e_dec += e2e_ev[1][0].elapsed_time(e2e_ev[1][1]) / reps
+    t = torch.tensor([e2e_pre, e2e_dec], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    e2e_pre, e2e_dec = float(t[0]), float(t[1])
+    h2d_pre = sum(v.numel() * v.element_size() for v in host.values())
+    d2h_pre = o.numel() * o.element_size()
+    h2d_dec = sum(v.numel() * v.element_size() for v in toks_host[0].values())
+    d2h_dec = od.numel() * od.element_size()
+
+    # ---- roofline of the dominant kernels ----
+    d = wp.d
+    flops_compose = active_pairs * 2.0 * d ** 3
+    comp_ms, comp_n = stages["compose"]
+    comp_avg = comp_ms / max(comp_n, 1)
+    comp_tf = flops_compose / (comp_avg * 1e-3) / 1e12 if comp_avg > 0 else None
+    n_ctx = wd.T // wd.C
+    bytes_decode = wd.B * wd.H * (n_ctx * (2 * wd.d * wd.d * 2 + wd.d * 4))
+    dmain_ms, dmain_n = stages["decode"]
+    dmain_avg = dmain_ms / max(dmain_n, 1)
+    dec_gbs = bytes_decode / (dmain_avg * 1e-3) / 1e9 if dmain_avg > 0 else None
+    launches = sum(n for (_, n) in stages.values())
+
+    tokens_pre = wp.B * wp.T * world
+    tokens_dec = wd.B * world
+    out = {
+        "metric": METRIC,
+        "value": tokens_pre / (pre_ms * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": pre_ms + dec_ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded; shapes and distributions of the HLA workloads; no dataset)",
+        "config": {"workload": wp.name, "decode_workload": wd.name, "prefill_ms": pre_ms, "decode_ms": dec_ms,
+                   "active_pairs": active_pairs, "parallelism": f"replicas x{world} (no data-path collective)",
+                   "l2": "flushed before every timed phase (256 MiB write, untimed)"},
+        "roofline": {"kernel": "compose", "bound": "tensor", "achieved": comp_tf, "peak": bf16_tf,
+                     "unit": "TFLOP/s", "frac": (comp_tf / bf16_tf) if comp_tf else None, "traffic": None,
+                     "peak_source": f"{peak_src} bf16 dense (burst)",
+                     "algorithmic": f"{active_pairs} active pairs x 2 d^3 = {flops_compose:.4g} flop per launch",
+                     "prefill_frac_of_peak": (flops_compose + N * wp.H * (FLOP_TRANSITION + FLOP_READOUT))
+                     / (pre_ms * 1e-3) / 1e12 / bf16_tf},
+        "decode": {"value": tokens_dec / (dec_ms * 1e-3), "unit": "tokens/s", "ms_per_step": dec_ms,
+                   "roofline": {"kernel": "decode_main", "bound": "hbm", "achieved": dec_gbs, "peak": hbm_gbs,
+                                "unit": "GB/s", "frac": (dec_gbs / hbm_gbs) if dec_gbs else None,
+                                "traffic": None, "peak_source": f"{peak_src} HBM copy",
+                                "algorithmic": f"{bytes_decode:.4g} bytes per launch (512 active A_j/B_j bf16 + "
+                                               "key pools per sequence and head)"},
+                   "e2e": {"value": tokens_dec / (e2e_dec * 1e-3), "unit": "tokens/s",
+                           "h2d_bytes_per_step": h2d_dec, "d2h_bytes_per_step": d2h_dec}},
+        "stages_ms_per_step": {k: v[0] / args.steps for k, v in stages.items() if v[1]},
+        "e2e": {"value": tokens_pre / (e2e_pre * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d_pre,
+                "d2h_bytes_per_step": d2h_pre},
+        "gpu_launches": launches,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(inp, wp, wd, ctx0, toks_host, torch)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+# ----------------------------------------------------------------------------------
+# CPU oracle (baseline and reference arm)
+# ----------------------------------------------------------------------------------
+
+def _oracle_prefill_sample(inp, wp, heads):
+    from oracle import hla_oracle as ho
+    t0 = time.perf_counter()
+    for h in heads:
+        f = lambda n: None if inp.get(n) is None else inp[n][0, :, h].float().numpy()
+        ho.hla_prefill_head(f("q").astype(np.float64), f("k").astype(np.float64), f("v").astype(np.float64),
+                            f("alpha").astype(np.float64), f("beta").astype(np.float64), wp.C, wp.tau, wp.bias,
+                            wp.thr, wp.gate_mode, f("q_route"), f("k_route"))
+    return time.perf_counter() - t0
+
+
+def _oracle_decode_sample(ctx, wd, toks, pairs):
+    """Time one decode step (definition form) for `pairs` (seq, head) pairs whose
+    oracle caches are built (untimed) from the same context."""
+    from oracle import hla_oracle as ho
+    states = []
+    for (b, h) in pairs:
+        f = lambda n: ctx[n][b, :, h].float().cpu().numpy().astype(np.float64)
+        states.append(((b, h), ho.HlaDecodeHead.from_prefill(f("q"), f("k"), f("v"), f("alpha"), f("beta"), wd.C,
+                                                             wd.tau, wd.bias, wd.thr, wd.gate_mode)))
+    tk = toks[0]
+    t0 = time.perf_counter()
+    for (b, h), st in states:
+        st.step(tk["q"][b, h].double().numpy(), tk["k"][b, h].double().numpy(), tk["v"][b, h].double().numpy(),
+                float(tk["alpha"][b, h]), float(tk["beta"][b, h]))
+    return time.perf_counter() - t0
+
+
+def _blas_one_thread():
+    try:
+        from threadpoolctl import threadpool_limits
+        return threadpool_limits(1)
+    except Exception:
+        return None
+
+
+def cpu_baseline(inp, wp, wd, ctx0, toks_host, torch):
+    lim = _blas_one_thread()
+    heads = [0]
+    tp = _oracle_prefill_sample(inp, wp, heads)
+    pairs = [(0, 0), (1, 5)]
+    td = _oracle_decode_sample(ctx0, wd, toks_host, pairs)
+    del lim
+    return {"value": wp.T * len(heads) / wp.H / tp, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"prefill: {len(heads)} of {wp.H} heads of the full T={wp.T} prompt ({tp:.1f} s), tokens/s "
+                      f"scaled by heads; decode: {len(pairs)} of {wd.B * wd.H} (sequence, head) pairs, one step "
+                      f"({td:.2f} s)",
+            "decode": {"value": len(pairs) / wd.H / td, "unit": "tokens/s"}}
+
+
+def run_reference(args):
+    """The oracle as it stands, on the host cores, on bounded samples of the same
+    workloads; rank 0 only."""
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    import torch
+    import hla_synth as syn
+    lim = _blas_one_thread()
+    wp = syn.PREFILL_0P8B
+    wd = syn.DECODE_32K
+    inp = syn.make_gdn_inputs(wp)
+    inp["q_route"], inp["k_route"] = syn.make_route_inputs(wp)
+    # decode context of 1 sequence (CPU generator; same shapes and distributions)
+    ctx = syn.make_gdn_inputs(wd.with_(B=1), device="cpu")
+    toks = syn.make_decode_tokens(wd.with_(B=1), 1)
+    times_p, times_d = [], []
+    for s in range(args.warmup + args.steps):
+        h = s % wp.H
+        tp = _oracle_prefill_sample(inp, wp, [h])
+        td = _oracle_decode_sample(ctx, wd.with_(B=1), toks, [(0, h)]) if s < 2 or s >= args.warmup else 0
+        if s >= args.warmup:
+            times_p.append(tp)
+            times_d.append(td)
+    del lim
+    tp = statistics.mean(times_p)
+    td = statistics.mean(times_d)
+    val = wp.T / wp.H / tp
+    out = {"impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": (tp + td) * 1e3, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": wp.name, "decode_workload": wd.name},
+           "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                            "sample": "each step: one of 16 heads of the full T=16384 prefill, plus one decode "
+                                      "step of one (sequence, head) pair; tokens/s scaled by heads"},
+           "decode": {"value": 1.0 / wd.H / td, "unit": "tokens/s"},
+           "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

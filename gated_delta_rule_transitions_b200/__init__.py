@@ -14,6 +14,8 @@ from ._hla import (  # noqa: F401
     hla_decode_step,
     hla_device_status,
     hla_prefill,
+    hla_profile_enable,
+    hla_profile_read,
     hla_routing,
     lib,
     make_config,

@@ -67,7 +67,11 @@ _SIGS = {
     "hla_decode_step": ([ctypes.POINTER(HlaConfig), ctypes.POINTER(HlaCache), _P, _P, _P, _P, _P, _P, _P, _P, _P,
                          ctypes.c_size_t, _P], ctypes.c_int),
     "hla_device_status": ([ctypes.c_int32, ctypes.POINTER(ctypes.c_uint32)], ctypes.c_int),
+    "hla_profile_enable": ([ctypes.c_int32], ctypes.c_int),
+    "hla_profile_read": ([_P, _P, ctypes.c_int32], ctypes.c_int),
 }
+
+STAGES = ("pools", "gates", "transitions", "compose", "readout", "cache", "decode", "decode_close")
 
 # Every symbol that include/hla.h declares (checked by the CPU tests).
 EXPORTS = tuple(_SIGS)
@@ -198,3 +202,17 @@ def hla_device_status(clear: bool = True):
     code = ctypes.c_uint32(0)
     st = lib().hla_device_status(1 if clear else 0, ctypes.byref(code))
     return st, int(code.value)
+
+
+def hla_profile_enable(on: bool = True):
+    _check(lib().hla_profile_enable(1 if on else 0))
+
+
+def hla_profile_read(reset: bool = True):
+    """Accumulated per-stage device milliseconds and kernel launches since the last reset."""
+    n = len(STAGES)
+    ms = (ctypes.c_float * n)()
+    la = (ctypes.c_int32 * n)()
+    _check(lib().hla_profile_read(ctypes.cast(ms, ctypes.c_void_p), ctypes.cast(la, ctypes.c_void_p),
+                                  1 if reset else 0))
+    return {STAGES[i]: (float(ms[i]), int(la[i])) for i in range(n)}

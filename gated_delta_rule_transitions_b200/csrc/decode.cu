@@ -228,11 +228,14 @@ __global__ void cache_fill_kernel(DecodeArgs c, FillArgs f) {
 }
 
 template <int D, typename Tio>
-static cudaError_t launch_d(const DecodeArgs& a, cudaStream_t s) {
+static cudaError_t launch_main(const DecodeArgs& a, cudaStream_t s) {
   decode_main_kernel<D, Tio><<<a.B * a.H, D, 0, s>>>(a);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  // close full chunks: transition into the cache, then the key pool
+  return cudaGetLastError();
+}
+
+template <int D, typename Tio>
+static cudaError_t launch_close(const DecodeArgs& a, cudaStream_t s) {
+  // close full chunks: transition into the cache, then the key pool, then counters
   TransArgs t{};
   t.B = a.B;
   t.H = a.H;
@@ -258,7 +261,7 @@ static cudaError_t launch_d(const DecodeArgs& a, cudaStream_t s) {
   t.close_m = a.m_partial;
   t.close_n = a.n_chunks;
   // the transition kernel never writes past max_chunks; the pool kernel flags it
-  e = launch_transitions(t, s);
+  cudaError_t e = launch_transitions(t, s);
   if (e != cudaSuccess) return e;
   decode_close_pool_kernel<D, Tio><<<a.B * a.H, D, 0, s>>>(a);
   e = cudaGetLastError();
@@ -267,9 +270,15 @@ static cudaError_t launch_d(const DecodeArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
-  if (a.d == 128) return a.dtype == HLA_BF16 ? launch_d<128, __nv_bfloat16>(a, s) : launch_d<128, float>(a, s);
-  return a.dtype == HLA_BF16 ? launch_d<64, __nv_bfloat16>(a, s) : launch_d<64, float>(a, s);
+cudaError_t launch_decode_main(const DecodeArgs& a, cudaStream_t s) {
+  if (a.d == 128) return a.dtype == HLA_BF16 ? launch_main<128, __nv_bfloat16>(a, s) : launch_main<128, float>(a, s);
+  return a.dtype == HLA_BF16 ? launch_main<64, __nv_bfloat16>(a, s) : launch_main<64, float>(a, s);
+}
+
+cudaError_t launch_decode_close(const DecodeArgs& a, cudaStream_t s) {
+  if (a.d == 128)
+    return a.dtype == HLA_BF16 ? launch_close<128, __nv_bfloat16>(a, s) : launch_close<128, float>(a, s);
+  return a.dtype == HLA_BF16 ? launch_close<64, __nv_bfloat16>(a, s) : launch_close<64, float>(a, s);
 }
 
 cudaError_t launch_cache_fill(const DecodeArgs& c, const float* rk_ws, const void* q_route, const void* k_route,

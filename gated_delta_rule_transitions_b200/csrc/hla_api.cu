@@ -4,6 +4,8 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
+#include <vector>
 
 #include "common.cuh"
 #include "kernels.cuh"
@@ -144,6 +146,42 @@ hla_status check_cache(const hla_config* c, const hla_cache* k) {
   return HLA_OK;
 }
 
+// ---- stage timing ------------------------------------------------------------
+struct StagePair {
+  cudaEvent_t a, b;
+  int stage;
+};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<StagePair> g_prof_pending;
+double g_prof_ms[HLA_STAGE_COUNT] = {};
+long g_prof_launches[HLA_STAGE_COUNT] = {};
+
+// Records events around one stage on `stream` while profiling is on.
+class StageScope {
+ public:
+  StageScope(int stage, cudaStream_t s, int launches) : stage_(stage), s_(s) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    if (!g_prof_on) return;
+    if (cudaEventCreate(&a_) != cudaSuccess || cudaEventCreate(&b_) != cudaSuccess) return;
+    cudaEventRecord(a_, s_);
+    g_prof_launches[stage] += launches;
+    on_ = true;
+  }
+  ~StageScope() {
+    if (!on_) return;
+    cudaEventRecord(b_, s_);
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof_pending.push_back({a_, b_, stage_});
+  }
+
+ private:
+  int stage_;
+  cudaStream_t s_;
+  cudaEvent_t a_ = nullptr, b_ = nullptr;
+  bool on_ = false;
+};
+
 }  // namespace
 
 extern "C" {
@@ -235,6 +273,7 @@ static hla_status routing_impl(const hla_config* cfg, const void* q_route, const
                                int32_t* active_cnt_out, cudaStream_t s) {
   const int N = (cfg->T + cfg->C - 1) / cfg->C;
   if (cfg->gate_mode == HLA_GATES_ROUTED || rk != nullptr) {
+    StageScope _sc(HLA_STAGE_POOLS, s, 1);
     HLA_CUDA(hla::launch_pools(cfg->gate_mode == HLA_GATES_ROUTED ? q_route : nullptr, k_route,
                                cfg->gate_mode == HLA_GATES_ROUTED ? rq : nullptr, rk, cfg->B, cfg->T, cfg->H,
                                cfg->dk, cfg->C, N, cfg->tau, cfg->dtype, s),
@@ -258,7 +297,10 @@ static hla_status routing_impl(const hla_config* cfg, const void* q_route, const
   g.gates_out = gates_out;
   g.active_idx_out = active_idx_out;
   g.active_cnt_out = active_cnt_out;
-  HLA_CUDA(hla::launch_gates(g, s), "gates launch");
+  {
+    StageScope _sc(HLA_STAGE_GATES, s, 1);
+    HLA_CUDA(hla::launch_gates(g, s), "gates launch");
+  }
   return HLA_OK;
 }
 
@@ -359,7 +401,10 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
   t.Wb = (float*)(ws + w.Wb);
   t.Ub = (float*)(ws + w.Ub);
   t.ell = (float*)(ws + w.ell);
-  HLA_CUDA(hla::launch_transitions(t, s), "transitions launch");
+  {
+    StageScope _sc(HLA_STAGE_TRANSITIONS, s, 1);
+    HLA_CUDA(hla::launch_transitions(t, s), "transitions launch");
+  }
   hla::ComposeArgs c{};
   c.B = cfg->B;
   c.H = cfg->H;
@@ -373,7 +418,10 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
   c.act_g = act_g;
   c.act_cnt = act_cnt;
   c.S_in = (float*)(ws + w.S_in);
-  HLA_CUDA(hla::launch_compose(c, s), "compose launch");
+  {
+    StageScope _sc(HLA_STAGE_COMPOSE, s, 1);
+    HLA_CUDA(hla::launch_compose(c, s), "compose launch");
+  }
   hla::ReadoutArgs r{};
   r.B = cfg->B;
   r.H = cfg->H;
@@ -389,7 +437,10 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
   r.Ub = t.Ub;
   r.ell = t.ell;
   r.o = o;
-  HLA_CUDA(hla::launch_readout(r, s), "readout launch");
+  {
+    StageScope _sc(HLA_STAGE_READOUT, s, 1);
+    HLA_CUDA(hla::launch_readout(r, s), "readout launch");
+  }
   if (cache_out) {
     hla::DecodeArgs dc{};
     dc.B = cfg->B;
@@ -407,6 +458,7 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
     dc.buf_beta = cache_out->buf_beta;
     dc.n_chunks = cache_out->n_chunks;
     dc.m_partial = cache_out->m_partial;
+    StageScope _sc(HLA_STAGE_CACHE, s, 1);
     HLA_CUDA(hla::launch_cache_fill(dc, rk, qr, kr, k, v, alpha, beta, cfg->T, s), "cache fill launch");
   }
   return HLA_OK;
@@ -465,7 +517,44 @@ hla_status hla_decode_step(const hla_config* cfg, hla_cache* cache, const void* 
   const size_t n = (size_t)cfg->B * cfg->H * cache->max_chunks;
   a.act_idx = (int32_t*)workspace;
   a.act_g = (float*)((char*)workspace + align256(n * 4));
-  HLA_CUDA(hla::launch_decode(a, (cudaStream_t)stream), "decode launch");
+  cudaStream_t s = (cudaStream_t)stream;
+  {
+    StageScope _sc(HLA_STAGE_DECODE, s, 1);
+    HLA_CUDA(hla::launch_decode_main(a, s), "decode launch");
+  }
+  {
+    StageScope _sc(HLA_STAGE_DECODE_CLOSE, s, 3);
+    HLA_CUDA(hla::launch_decode_close(a, s), "decode close launch");
+  }
+  return HLA_OK;
+}
+
+hla_status hla_profile_enable(int32_t on) {
+  g_msg[0] = 0;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_prof_on = on != 0;
+  return HLA_OK;
+}
+
+hla_status hla_profile_read(float* ms_out, int32_t* launches_out, int32_t reset) {
+  g_msg[0] = 0;
+  HLA_CUDA(cudaDeviceSynchronize(), "hla_profile_read synchronize");
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  for (const StagePair& p : g_prof_pending) {
+    float ms = 0.0f;
+    if (cudaEventElapsedTime(&ms, p.a, p.b) == cudaSuccess) g_prof_ms[p.stage] += ms;
+    cudaEventDestroy(p.a);
+    cudaEventDestroy(p.b);
+  }
+  g_prof_pending.clear();
+  for (int i = 0; i < HLA_STAGE_COUNT; ++i) {
+    if (ms_out) ms_out[i] = (float)g_prof_ms[i];
+    if (launches_out) launches_out[i] = (int32_t)g_prof_launches[i];
+    if (reset) {
+      g_prof_ms[i] = 0.0;
+      g_prof_launches[i] = 0;
+    }
+  }
   return HLA_OK;
 }
 

@@ -104,7 +104,8 @@ cudaError_t launch_gates(const GatesArgs& a, cudaStream_t s);
 cudaError_t launch_transitions(const TransArgs& a, cudaStream_t s);
 cudaError_t launch_compose(const ComposeArgs& a, cudaStream_t s);
 cudaError_t launch_readout(const ReadoutArgs& a, cudaStream_t s);
-cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_decode_main(const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_decode_close(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_cache_fill(const DecodeArgs& c, const float* rk_ws, const void* q_route, const void* k_route,
                               const void* k, const void* v, const float* alpha, const float* beta, int T,
                               cudaStream_t s);

@@ -156,3 +156,21 @@ def make_decode_tokens(w: Workload, steps: int, device="cpu", seed: int | None =
         b = torch.sigmoid(torch.randn((w.B, w.H), generator=g, device=device)).float()
         out.append(dict(q=q.to(dt), k=k.to(dt), v=v.to(dt), alpha=a, beta=b))
     return out
+
+
+def make_context_group(w: Workload, b0: int, nb: int, device="cuda"):
+    """Decode context (prompt) of sequences b0 .. b0+nb-1, generated on ``device``
+    with a generator seeded by (seed, b0): q, k, v [nb, T, H, d], alpha, beta
+    [nb, T, H].  Used to build large decode caches group by group."""
+    g = torch.Generator(device=device)
+    g.manual_seed(w.seed * 1000003 + b0)
+    shape = (nb, w.T, w.H, w.d)
+    dt = torch_dtype(w)
+    q = _l2n(torch.randn(shape, generator=g, device=device)).to(dt)
+    k = _l2n(torch.randn(shape, generator=g, device=device)).to(dt)
+    v = torch.randn(shape, generator=g, device=device).to(dt)
+    a_raw = torch.randn((nb, w.T, w.H), generator=g, device=device)
+    b_raw = torch.randn((nb, w.T, w.H), generator=g, device=device)
+    alpha = torch.exp(-torch.nn.functional.softplus(a_raw - 3.0)).float()
+    beta = torch.sigmoid(b_raw).float()
+    return dict(q=q, k=k, v=v, alpha=alpha, beta=beta)

@@ -219,6 +219,29 @@ hla_status hla_decode_step(const hla_config* cfg, hla_cache* cache, const void* 
  */
 hla_status hla_device_status(int32_t clear, uint32_t* code_out);
 
+/*
+ * Stage timing (tracing).  While enabled, hla_prefill and hla_decode_step record a
+ * pair of CUDA events on the caller's stream around each stage below and count the
+ * kernels each stage launches.  hla_profile_read synchronises the device, writes
+ * the accumulated milliseconds and launch counts per stage into ms_out[] and
+ * launches_out[] (HLA_STAGE_COUNT entries each; either may be NULL) and, if
+ * reset != 0, clears them.  Errors: CUDA.
+ */
+typedef enum {
+  HLA_STAGE_POOLS = 0,        /* log-mean-exp pools                        */
+  HLA_STAGE_GATES = 1,        /* gates + active lists                      */
+  HLA_STAGE_TRANSITIONS = 2,  /* chunk transitions (A, B) and WY factors   */
+  HLA_STAGE_COMPOSE = 3,      /* gated composition of S_in                 */
+  HLA_STAGE_READOUT = 4,      /* intra-chunk read-out                      */
+  HLA_STAGE_CACHE = 5,        /* prefill -> decode cache hand-off          */
+  HLA_STAGE_DECODE = 6,       /* decode: sweep, gates, active chain        */
+  HLA_STAGE_DECODE_CLOSE = 7, /* decode: closing full chunks, counters     */
+  HLA_STAGE_COUNT = 8
+} hla_stage;
+
+hla_status hla_profile_enable(int32_t on);
+hla_status hla_profile_read(float* ms_out, int32_t* launches_out, int32_t reset);
+
 #ifdef __cplusplus
 }
 #endif
