@@ -158,6 +158,8 @@ def run_ours(args):
 
     # ---- prefill workload (inputs resident in HBM) ----
     wp = syn.PREFILL_0P8B
+    if args.prefill_T:
+        wp = wp.with_(T=args.prefill_T, name=wp.name.replace("T16384", f"T{args.prefill_T}"))
     inp = syn.make_gdn_inputs(wp)
     qr, kr = syn.make_route_inputs(wp)
     inp["q_route"], inp["k_route"] = qr, kr
@@ -176,8 +178,15 @@ def run_ours(args):
 
     # ---- decode workload ----
     wd = syn.DECODE_32K
+    if args.decode_B or args.decode_ctx:
+        B_ = args.decode_B or wd.B
+        T_ = args.decode_ctx or wd.T
+        wd = wd.with_(B=B_, T=T_, name=f"decode_bf16_{B_}seq_ctx{T_}_H16_C64_d128_thr0.05")
+    if args.skip_decode:
+        wd = wd.with_(B=8, T=64 * 4, name="decode_skipped")
     max_chunks = wd.T // wd.C + 1
-    cache, ctx0 = build_decode_cache(hla, syn, torch, wd, max_chunks)
+    cache, ctx0 = build_decode_cache(hla, syn, torch, wd, max_chunks, group=min(8, wd.B))
+    torch.cuda.empty_cache()
     dcfg = hla.make_config(wd.B, wd.H, 1, wd.C, wd.d, wd.dtype, wd.gate_mode, wd.tau, wd.bias, wd.thr)
     dws = torch.empty(hla.decode_workspace_bytes(dcfg, max_chunks), dtype=torch.uint8, device="cuda")
     ntok = args.warmup + args.steps + 1
@@ -260,13 +269,10 @@ def run_ours(args):
         e2e_ev[0][1].record(stream)
         l2_flush()
         e2e_ev[1][0].record(stream)
-        t_ = toks[step_idx[0] % len(toks)]
-        th = toks_host[step_idx[0] % len(toks)]
+        t_, th = toks[-1], toks_host[-1]
         for k in t_:
             t_[k].copy_(th[k], non_blocking=True)
-        decode_idx = step_idx[0] % len(toks)
-        step_idx[0] = decode_idx
-        decode()
+        hla.hla_decode_step(dcfg, cache, t_["q"], t_["k"], t_["v"], t_["alpha"], t_["beta"], od, workspace=dws)
         od_host.copy_(od, non_blocking=True)
         e2e_ev[1][1].record(stream)
         torch.cuda.synchronize()
@@ -443,6 +449,11 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    # smaller variants for profiling captures (the default is the full workload)
+    ap.add_argument("--prefill-T", type=int, default=None, help="prefill tokens (default 16384)")
+    ap.add_argument("--decode-B", type=int, default=None, help="decode sequences (default 64)")
+    ap.add_argument("--decode-ctx", type=int, default=None, help="decode context tokens (default 32768)")
+    ap.add_argument("--skip-decode", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

@@ -1,0 +1,356 @@
+// Gated composition on the 5th-generation tensor cores (tcgen05 + TMEM + TMA),
+// bf16 operands, float32 state.  d = 128, C = 64.
+//
+// HLA summary page, "Methodology in Plain English" paras. 3-4: for query chunk i,
+//   S <- 0;  for j in active(i), ascending:  S <- S + g_ij ((S A_j + B_j) - S)
+// and a chunk below the threshold is skipped (it is not in active(i)).
+//
+// One CTA runs two query chunks ("chains") of one head.  Per step j of the merged
+// active lists, TMA brings A_j and B_j (bf16, 128-byte swizzle) into a 3-stage ring;
+// for each chain active at j the MMA warp issues
+//     D_k += Aop_k x A_j     (M = 128 rows v, N = 128 columns c, K = 128)
+// where the float32 master state lives in tensor memory pre-scaled, D_k = (1-g) S,
+// and the MMA operand Aop_k = bf16(g S) also lives in tensor memory.  The epilogue
+// warps then add g B_j[v][c], giving S_new, and prepare the next active step of that
+// chain: D_k <- (1 - g_next) S_new, Aop_k <- bf16(g_next S_new).  After a chain's
+// last active step S_new is written to S_in (float32, [v][c]).
+//
+// Warp roles: warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer, warps 2-9
+// epilogue (lane quarter = warp % 4, column half = (warp - 2) / 4).  All waits are
+// bounded (about 2 s, then a device error word is set and the CTA exits cleanly).
+#include "common.cuh"
+#include "kernels.cuh"
+#include "tc_common.cuh"
+
+namespace hla {
+
+HLA_DEFINE_ERROR_WORD(compose_tc)
+
+namespace {
+
+constexpr int kD = 128;
+constexpr int kStages = 3;
+constexpr int kStageBytes = 2 * kD * kD * 2;     // A_j + B_j, bf16
+constexpr int kHalfBytes = kD * 64 * 2;          // one 64-column box
+constexpr int kThreads = 320;
+constexpr uint32_t kIdesc = tc::idesc_bf16_f32(128, 128, /*a_mn=*/0, /*b_mn=*/1);
+
+struct ComposeTcArgs {
+  int BH, N;
+  long ab_chunk_stride;
+  const int32_t* act_idx;
+  const float* act_g;
+  const int32_t* act_cnt;
+  float* S_in;
+};
+
+// Walks the merged ascending active lists of the two chains.
+struct Sched {
+  const int32_t* idx[2];
+  const float* g[2];
+  int cnt[2];
+  int p[2];
+  int j;
+  bool act[2];
+  bool first[2];
+  float gate[2];
+  float gnext[2];
+  bool last[2];
+
+  __device__ void init(const ComposeTcArgs& a, int bh, const int i[2]) {
+    for (int k = 0; k < 2; ++k) {
+      p[k] = 0;
+      if (i[k] >= 0) {
+        const long row = (long)bh * a.N + i[k];
+        idx[k] = a.act_idx + row * a.N;
+        g[k] = a.act_g + row * a.N;
+        cnt[k] = a.act_cnt[row];
+      } else {
+        idx[k] = nullptr;
+        g[k] = nullptr;
+        cnt[k] = 0;
+      }
+    }
+  }
+  // Loads the next step; false when both lists are exhausted.
+  __device__ bool next() {
+    int j0 = p[0] < cnt[0] ? idx[0][p[0]] : 0x7FFFFFFF;
+    int j1 = p[1] < cnt[1] ? idx[1][p[1]] : 0x7FFFFFFF;
+    j = min(j0, j1);
+    if (j == 0x7FFFFFFF) return false;
+    const int jj[2] = {j0, j1};
+    for (int k = 0; k < 2; ++k) {
+      act[k] = jj[k] == j;
+      first[k] = act[k] && p[k] == 0;
+      gate[k] = act[k] ? g[k][p[k]] : 0.0f;
+      last[k] = act[k] && p[k] + 1 == cnt[k];
+      gnext[k] = (act[k] && !last[k]) ? g[k][p[k] + 1] : 0.0f;
+    }
+    return true;
+  }
+  __device__ void advance() {
+    for (int k = 0; k < 2; ++k)
+      if (act[k]) ++p[k];
+  }
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    compose_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                      ComposeTcArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* ring = smem;  // kStages x [A half0 | A half1 | B half0 | B half1]
+  uint64_t* bars = (uint64_t*)(smem + kStages * kStageBytes);
+  uint64_t* full = bars;                 // [kStages]
+  uint64_t* empty = bars + kStages;      // [kStages]
+  uint64_t* mma_done = bars + 2 * kStages;  // [2]
+  uint64_t* op_ready = mma_done + 2;        // [2]
+  uint64_t* final_bar = op_ready + 2;       // [1]
+  uint32_t* tmem_base_s = (uint32_t*)(final_bar + 1);
+  volatile int* abort_s = (volatile int*)(tmem_base_s + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int pair = blockIdx.x / a.BH;
+  const int bh = blockIdx.x % a.BH;
+  const int chains[2] = {a.N - 1 - 2 * pair, a.N - 2 - 2 * pair};
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 2);
+    }
+    for (int k = 0; k < 2; ++k) {
+      tc::mbar_init(&mma_done[k], 1);
+      tc::mbar_init(&op_ready[k], 1);
+    }
+    tc::mbar_init(final_bar, 1);
+    *abort_s = 0;
+    tc::mbar_fence_init();
+    tc::fence_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    tc::tma_prefetch_desc(&tmA);
+    tc::tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) tc::tmem_alloc(tmem_base_s, 512);
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tbase = *tmem_base_s;
+
+  Sched sc;
+  sc.init(a, bh, chains);
+
+  if (warp == 0) {
+    // ---------------- TMA producer (lane 0) ----------------
+    if (lane == 0) {
+      int s = 0;
+      while (sc.next()) {
+        const int st = s % kStages;
+        if (s >= kStages && !tc::mbar_wait(&empty[st], ((s / kStages) - 1) & 1, abort_s)) break;
+        tc::mbar_arrive_expect_tx(&full[st], kStageBytes);
+        const int row = (int)(((long)bh * a.ab_chunk_stride + sc.j) * kD);
+        uint8_t* dst = ring + st * kStageBytes;
+        tc::tma_load_2d(dst, &tmA, 0, row, &full[st]);
+        tc::tma_load_2d(dst + kHalfBytes, &tmA, 64, row, &full[st]);
+        tc::tma_load_2d(dst + 2 * kHalfBytes, &tmB, 0, row, &full[st]);
+        tc::tma_load_2d(dst + 3 * kHalfBytes, &tmB, 64, row, &full[st]);
+        sc.advance();
+        ++s;
+      }
+      if (*abort_s) {
+        // never leave the CTA with copies in flight
+        for (int t = max(0, s - kStages); t < s; ++t)
+          tc::mbar_wait(&full[t % kStages], (t / kStages) & 1, nullptr, 200000000ull);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (lane 0) ----------------
+    if (lane == 0) {
+      int s = 0;
+      bool ok = true;
+      while (ok && sc.next()) {
+        const int st = s % kStages;
+        if (!tc::mbar_wait(&full[st], (s / kStages) & 1, abort_s)) break;
+        tc::tc_fence_after();
+        const uint32_t b_base = tc::smem_u32(ring + st * kStageBytes);
+        for (int k = 0; k < 2; ++k) {
+          if (!sc.act[k] || sc.first[k]) continue;
+          if (!tc::mbar_wait(&op_ready[k], (sc.p[k] - 1) & 1, abort_s)) {
+            ok = false;
+            break;
+          }
+          tc::tc_fence_after();
+          const uint32_t d_t = tbase + 128u * k;
+          const uint32_t a_t = tbase + 256u + 64u * k;
+#pragma unroll
+          for (int ks = 0; ks < kD / 16; ++ks) {
+            const uint64_t bd = tc::sdesc_sw128(b_base + ks * 2048, kHalfBytes, 1024);
+            tc::mma_ts(d_t, a_t + 8u * ks, bd, kIdesc, 1u);
+          }
+          tc::mma_commit(&mma_done[k]);
+        }
+        if (!ok) break;
+        tc::mma_commit(&empty[st]);
+        sc.advance();
+        ++s;
+      }
+      // all MMAs issued by this thread complete before the CTA frees tensor memory
+      tc::mma_commit(final_bar);
+      tc::mbar_wait(final_bar, 0, nullptr, 200000000ull);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue (8 warps, 256 threads, named barrier 1) ----------------
+    const int q = warp & 3;
+    const int h = (warp - 2) >> 2;
+    const int v = 32 * q + lane;
+    const int col0 = 64 * h;
+    const uint32_t lane_off = (uint32_t)(32 * q) << 16;
+    // chains with nothing active have S_in = 0
+    for (int k = 0; k < 2; ++k) {
+      if (chains[k] >= 0 && sc.cnt[k] == 0) {
+        float4* out = (float4*)(a.S_in + ((long)bh * a.N + chains[k]) * kD * kD + (long)v * kD + col0);
+        for (int e = 0; e < 16; ++e) out[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    int s = 0;
+    bool ok = true;
+    while (ok && sc.next()) {
+      const int st = s % kStages;
+      ok = tc::bar_all(1, 256, tc::mbar_wait(&full[st], (s / kStages) & 1, abort_s));
+      if (!ok) break;
+      // B_j[v][col0 .. col0+64) from the swizzled box
+      const uint8_t* brow = ring + st * kStageBytes + 2 * kHalfBytes + h * kHalfBytes + v * 128;
+      uint32_t bw[32];
+#pragma unroll
+      for (int c8 = 0; c8 < 8; ++c8) {
+        const uint4 w = *(const uint4*)(brow + ((c8 ^ (v & 7)) << 4));
+        bw[4 * c8 + 0] = w.x;
+        bw[4 * c8 + 1] = w.y;
+        bw[4 * c8 + 2] = w.z;
+        bw[4 * c8 + 3] = w.w;
+      }
+      for (int k = 0; k < 2; ++k) {
+        if (!sc.act[k]) continue;
+        const bool first = sc.first[k];
+        const float g = sc.gate[k];
+        const float gn = sc.gnext[k];
+        const float keep = 1.0f - gn;
+        if (!first) {
+          ok = tc::bar_all(1, 256, tc::mbar_wait(&mma_done[k], (sc.p[k] - 1) & 1, abort_s));
+          if (!ok) break;
+          tc::tc_fence_after();
+        }
+#pragma unroll
+        for (int cc = 0; cc < 64; cc += 32) {
+          const uint32_t d_addr = tbase + lane_off + 128u * k + col0 + cc;
+          uint32_t d[32];
+          if (!first) {
+            tc::tmem_ld32(d_addr, d);
+            tc::tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) d[e] = 0u;
+          }
+          float x[32];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const uint32_t w = bw[cc / 2 + e];
+            x[2 * e] = fmaf(g, tc::bf16lo(w), __uint_as_float(d[2 * e]));
+            x[2 * e + 1] = fmaf(g, tc::bf16hi(w), __uint_as_float(d[2 * e + 1]));
+          }
+          if (sc.last[k]) {
+            float4* out =
+                (float4*)(a.S_in + ((long)bh * a.N + chains[k]) * kD * kD + (long)v * kD + col0 + cc);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) out[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
+          } else {
+            uint32_t dn[32];
+            uint32_t op[16];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) dn[e] = __float_as_uint(keep * x[e]);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) op[e] = tc::pack_bf16x2(gn * x[2 * e], gn * x[2 * e + 1]);
+            tc::tmem_st32(d_addr, dn);
+            tc::tmem_st16(tbase + lane_off + 256u + 64u * k + (col0 + cc) / 2, op);
+          }
+        }
+        tc::tmem_wait_st();
+        tc::tc_fence_before();
+        tc::bar_sync(1, 256);
+        if (threadIdx.x == 64 && !sc.last[k]) tc::mbar_arrive(&op_ready[k]);
+      }
+      if (!ok) break;
+      tc::bar_sync(1, 256);
+      if (threadIdx.x == 64) tc::mbar_arrive(&empty[st]);
+      sc.advance();
+      ++s;
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  if (warp == 1) tc::tmem_dealloc(tbase, 512);
+  if (threadIdx.x == 0 && *abort_s) report_device_error(kErrMbarTimeout);
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+  }
+  return fn;
+}
+
+}  // namespace
+
+// 2-D bf16 tensor map over `rows` rows of 128 elements, box 64 x 128, 128-byte swizzle.
+cudaError_t make_tmap_rows128(CUtensorMap* m, const void* base, long rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return cudaErrorNotSupported;
+  cuuint64_t dims[2] = {128, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {128 * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t launch_compose_tc(const ComposeArgs& c, cudaStream_t s) {
+  if (c.N <= 0) return cudaSuccess;
+  const long rows = (long)c.B * c.H * c.ab_chunk_stride * kD;
+  CUtensorMap tmA, tmB;
+  cudaError_t e = make_tmap_rows128(&tmA, c.A, rows);
+  if (e != cudaSuccess) return e;
+  e = make_tmap_rows128(&tmB, c.Bm, rows);
+  if (e != cudaSuccess) return e;
+  ComposeTcArgs a;
+  a.BH = c.B * c.H;
+  a.N = c.N;
+  a.ab_chunk_stride = c.ab_chunk_stride;
+  a.act_idx = c.act_idx;
+  a.act_g = c.act_g;
+  a.act_cnt = c.act_cnt;
+  a.S_in = c.S_in;
+  const size_t smem = 1024 + kStages * kStageBytes + 256;
+  e = cudaFuncSetAttribute(compose_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int pairs = (c.N + 1) / 2;
+  compose_tc_kernel<<<pairs * a.BH, kThreads, smem, s>>>(tmA, tmB, a);
+  return cudaGetLastError();
+}
+
+}  // namespace hla

@@ -271,6 +271,7 @@ static cudaError_t launch_close(const DecodeArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_decode_main(const DecodeArgs& a, cudaStream_t s) {
+  if (a.d == 128 && a.dtype == HLA_BF16) return launch_decode_stream(a, s);
   if (a.d == 128) return a.dtype == HLA_BF16 ? launch_main<128, __nv_bfloat16>(a, s) : launch_main<128, float>(a, s);
   return a.dtype == HLA_BF16 ? launch_main<64, __nv_bfloat16>(a, s) : launch_main<64, float>(a, s);
 }

@@ -1,0 +1,259 @@
+// Decode step for bf16 caches with d = 128: the active-chunk chain streams A_j and B_j
+// from HBM through a TMA-fed shared-memory ring.
+//
+// HLA summary page, "Key Contributions" 3 (dynamic autoregressive decoding) and
+// "Methodology in Plain English" paras. 3-4 (gated transitions; chunks below the
+// threshold are skipped, so they are never read).  Same steps as the portable decode
+// kernel: append the token, sweep the open chunk right to left (x = A_p q,
+// y0 = B_p q), pool the open chunk's route queries, gate every closed chunk, then
+//   for active j descending:  y += g_j B_j x;  x <- (1-g_j) x + g_j A_j x
+// and o = y + y0.  The chain is bound by HBM: each active chunk costs 64 KiB of bf16
+// and 4 d^2 flops.  One CTA per (sequence, head): warps 0-3 compute (thread = row r),
+// warp 4 issues TMA loads of A_j and B_j (128-byte swizzle, 64-column boxes) into a
+// 3-stage ring, so about two chunks are in flight per SM while one is consumed.
+#include "common.cuh"
+#include "kernels.cuh"
+#include "routing_recipe.cuh"
+#include "tc_common.cuh"
+
+namespace hla {
+
+HLA_DEFINE_ERROR_WORD(decode_stream)
+
+cudaError_t make_tmap_rows128(CUtensorMap* m, const void* base, long rows);
+
+namespace {
+
+constexpr int kD = 128;
+constexpr int kStages = 3;
+constexpr int kHalf = kD * 64 * 2;       // 16 KiB: one 64-column box of a 128x128 bf16 matrix
+constexpr int kStageBytes = 4 * kHalf;   // A_j and B_j
+constexpr int kCompute = 128;
+constexpr int kThreads = kCompute + 32;
+
+__device__ __forceinline__ float blk_sum(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  tc::bar_sync(1, kCompute);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  tc::bar_sync(1, kCompute);
+  return red[0] + red[1] + red[2] + red[3];
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_stream_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                         DecodeArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* ring = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint64_t* full = (uint64_t*)(ring + kStages * kStageBytes);
+  uint64_t* empty = full + kStages;
+  float* xs = (float*)(empty + kStages);     // [2][kD]
+  float* rq = xs + 2 * kD;                   // [kD]
+  float* red = rq + kD;                      // [4]
+  int* wcount = (int*)(red + 4);             // [4]
+  int* cnt_s = wcount + 4;                   // [1]
+  volatile int* abort_s = (volatile int*)(cnt_s + 1);
+
+  const int bh = blockIdx.x;
+  const int b = bh / a.H;
+  const int tid = threadIdx.x;
+  const int C = a.C;
+  const int n = a.n_chunks[b];
+  const int m = a.m_partial[b];
+  const int mp = m + 1;
+  int32_t* act_idx = a.act_idx + (long)bh * a.max_chunks;
+  float* act_g = a.act_g + (long)bh * a.max_chunks;
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);
+    }
+    *abort_s = 0;
+    tc::mbar_fence_init();
+    tc::fence_async_smem();
+  }
+  __syncthreads();
+
+  if (tid >= kCompute) {
+    // ---------------- TMA producer (warp 4, lane 0) ----------------
+    // waits for the active list, then streams A_j / B_j for j descending
+    tc::bar_sync(2, kThreads);
+    if (tid == kCompute) {
+      tc::tma_prefetch_desc(&tmA);
+      tc::tma_prefetch_desc(&tmB);
+      const int cnt = *cnt_s;
+      int s = 0;
+      for (int p = cnt - 1; p >= 0; --p, ++s) {
+        const int st = s % kStages;
+        if (s >= kStages && !tc::mbar_wait(&empty[st], ((s / kStages) - 1) & 1, abort_s)) break;
+        const int j = act_idx[p];
+        const int row = (int)(((long)bh * a.max_chunks + j) * kD);
+        tc::mbar_arrive_expect_tx(&full[st], kStageBytes);
+        uint8_t* dst = ring + st * kStageBytes;
+        tc::tma_load_2d(dst, &tmA, 0, row, &full[st]);
+        tc::tma_load_2d(dst + kHalf, &tmA, 64, row, &full[st]);
+        tc::tma_load_2d(dst + 2 * kHalf, &tmB, 0, row, &full[st]);
+        tc::tma_load_2d(dst + 3 * kHalf, &tmB, 64, row, &full[st]);
+      }
+      if (*abort_s)
+        for (int t = max(0, s - kStages); t < s; ++t)
+          tc::mbar_wait(&full[t % kStages], (t / kStages) & 1, nullptr, 200000000ull);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- compute (warps 0-3), thread = channel / row ----------------
+    const long tok = (long)bh * kD + tid;
+    const long bslot = ((long)bh * C + m) * kD + tid;
+    const __nv_bfloat16* qr_in = (const __nv_bfloat16*)(a.q_route ? a.q_route : a.q);
+    const __nv_bfloat16* kr_in = (const __nv_bfloat16*)(a.k_route ? a.k_route : a.k);
+    ((__nv_bfloat16*)a.buf_k)[bslot] = ((const __nv_bfloat16*)a.k)[tok];
+    ((__nv_bfloat16*)a.buf_v)[bslot] = ((const __nv_bfloat16*)a.v)[tok];
+    ((__nv_bfloat16*)a.buf_qr)[bslot] = qr_in[tok];
+    ((__nv_bfloat16*)a.buf_kr)[bslot] = kr_in[tok];
+    if (tid == 0) {
+      a.buf_alpha[(long)bh * C + m] = a.alpha[bh];
+      a.buf_beta[(long)bh * C + m] = a.beta[bh];
+    }
+    tc::bar_sync(1, kCompute);
+    __threadfence_block();
+    const __nv_bfloat16* bk = (const __nv_bfloat16*)a.buf_k + (long)bh * C * kD;
+    const __nv_bfloat16* bv = (const __nv_bfloat16*)a.buf_v + (long)bh * C * kD;
+    // (1) open-chunk sweep
+    float x = ldf((const __nv_bfloat16*)a.q + tok);
+    float y0 = 0.0f;
+    for (int t = mp - 1; t >= 0; --t) {
+      const float kt = ldf(bk + (long)t * kD + tid);
+      const float c = blk_sum(kt * x, red);
+      const float bt = a.buf_beta[(long)bh * C + t];
+      const float at = a.buf_alpha[(long)bh * C + t];
+      y0 = fmaf(bt * c, ldf(bv + (long)t * kD + tid), y0);
+      x = at * (x - bt * c * kt);
+    }
+    // (2) gates and the ascending active list
+    int cnt = 0;
+    if (a.mode != HLA_GATES_ZERO && n > 0) {
+      const route::Consts K = route::make_consts();
+      if (a.mode == HLA_GATES_ROUTED) {
+        const __nv_bfloat16* bq = (const __nv_bfloat16*)a.buf_qr + (long)bh * C * kD + tid;
+        const float inv_tau = __fdiv_rn(1.0f, a.tau);
+        float mx = __fmul_rn(ldf(bq), inv_tau);
+        for (int t = 1; t < mp; ++t) mx = fmaxf(mx, __fmul_rn(ldf(bq + (long)t * kD), inv_tau));
+        float s = 0.0f;
+        for (int t = 0; t < mp; ++t)
+          s = __fadd_rn(s, route::rexp(__fsub_rn(__fmul_rn(ldf(bq + (long)t * kD), inv_tau), mx), K));
+        rq[tid] = __fmul_rn(a.tau, __fadd_rn(mx, route::rlog(__fdiv_rn(s, (float)mp), K)));
+        tc::bar_sync(1, kCompute);
+      }
+      const float* rk = a.rk + (long)bh * a.max_chunks * kD;
+      for (int jb = 0; jb < n; jb += kCompute) {
+        const int j = jb + tid;
+        float g = 1.0f;
+        bool keep = false;
+        if (j < n) {
+          if (a.mode == HLA_GATES_ROUTED) {
+            const float4* rkj = (const float4*)(rk + (long)j * kD);
+            float dot = 0.0f;
+            for (int c4 = 0; c4 < kD / 4; ++c4) {
+              const float4 r4 = rkj[c4];
+              dot = __fadd_rn(dot, __fmul_rn(rq[4 * c4 + 0], r4.x));
+              dot = __fadd_rn(dot, __fmul_rn(rq[4 * c4 + 1], r4.y));
+              dot = __fadd_rn(dot, __fmul_rn(rq[4 * c4 + 2], r4.z));
+              dot = __fadd_rn(dot, __fmul_rn(rq[4 * c4 + 3], r4.w));
+            }
+            g = route::gate_from_dot(dot, a.c_d, a.bias, K);
+          }
+          keep = a.thr <= 0.0f || g >= a.thr;
+        }
+        const unsigned int bal = __ballot_sync(0xFFFFFFFFu, keep);
+        const int w = tid >> 5;
+        if ((tid & 31) == 0) wcount[w] = __popc(bal);
+        tc::bar_sync(1, kCompute);
+        int before = 0, total = 0;
+#pragma unroll
+        for (int k2 = 0; k2 < 4; ++k2) {
+          if (k2 < w) before += wcount[k2];
+          total += wcount[k2];
+        }
+        if (keep) {
+          const int pos = cnt + before + __popc(bal & ((1u << (tid & 31)) - 1u));
+          act_idx[pos] = j;
+          act_g[pos] = g;
+        }
+        cnt += total;
+        tc::bar_sync(1, kCompute);
+      }
+    }
+    if (tid == 0) *cnt_s = cnt;
+    xs[tid] = x;
+    __threadfence_block();
+    tc::bar_sync(2, kThreads);  // releases the producer
+    // (3) active chain, descending j
+    float y = 0.0f;
+    int cur = 0;
+    bool ok = true;
+    for (int p = cnt - 1, s = 0; p >= 0; --p, ++s) {
+      const int st = s % kStages;
+      ok = tc::bar_all(1, kCompute, tc::mbar_wait(&full[st], (s / kStages) & 1, abort_s));
+      if (!ok) break;
+      const uint8_t* stA = ring + st * kStageBytes;
+      const uint8_t* stB = stA + 2 * kHalf;
+      const float* xc = xs + cur * kD;
+      float ax0 = 0.f, ax1 = 0.f, bx0 = 0.f, bx1 = 0.f;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8) {
+          const int off = hh * kHalf + tid * 128 + ((c8 ^ (tid & 7)) << 4);
+          const uint4 wa = *(const uint4*)(stA + off);
+          const uint4 wb = *(const uint4*)(stB + off);
+          const float4 x0 = *(const float4*)(xc + hh * 64 + c8 * 8);
+          const float4 x1 = *(const float4*)(xc + hh * 64 + c8 * 8 + 4);
+          ax0 = fmaf(tc::bf16lo(wa.x), x0.x, ax0);
+          ax1 = fmaf(tc::bf16hi(wa.x), x0.y, ax1);
+          ax0 = fmaf(tc::bf16lo(wa.y), x0.z, ax0);
+          ax1 = fmaf(tc::bf16hi(wa.y), x0.w, ax1);
+          ax0 = fmaf(tc::bf16lo(wa.z), x1.x, ax0);
+          ax1 = fmaf(tc::bf16hi(wa.z), x1.y, ax1);
+          ax0 = fmaf(tc::bf16lo(wa.w), x1.z, ax0);
+          ax1 = fmaf(tc::bf16hi(wa.w), x1.w, ax1);
+          bx0 = fmaf(tc::bf16lo(wb.x), x0.x, bx0);
+          bx1 = fmaf(tc::bf16hi(wb.x), x0.y, bx1);
+          bx0 = fmaf(tc::bf16lo(wb.y), x0.z, bx0);
+          bx1 = fmaf(tc::bf16hi(wb.y), x0.w, bx1);
+          bx0 = fmaf(tc::bf16lo(wb.z), x1.x, bx0);
+          bx1 = fmaf(tc::bf16hi(wb.z), x1.y, bx1);
+          bx0 = fmaf(tc::bf16lo(wb.w), x1.z, bx0);
+          bx1 = fmaf(tc::bf16hi(wb.w), x1.w, bx1);
+        }
+      }
+      const float g = act_g[p];
+      y = fmaf(g, bx0 + bx1, y);
+      xs[(cur ^ 1) * kD + tid] = (1.0f - g) * xc[tid] + g * (ax0 + ax1);
+      cur ^= 1;
+      tc::bar_sync(1, kCompute);
+      if (tid == 0) tc::mbar_arrive(&empty[st]);
+    }
+    stf((__nv_bfloat16*)a.o + tok, y + y0);
+  }
+  __syncthreads();
+  if (tid == 0 && *abort_s) report_device_error(kErrMbarTimeout);
+}
+
+}  // namespace
+
+cudaError_t launch_decode_stream(const DecodeArgs& a, cudaStream_t s) {
+  const long rows = (long)a.B * a.H * a.max_chunks * kD;
+  CUtensorMap tmA, tmB;
+  cudaError_t e = make_tmap_rows128(&tmA, a.A, rows);
+  if (e != cudaSuccess) return e;
+  e = make_tmap_rows128(&tmB, a.Bm, rows);
+  if (e != cudaSuccess) return e;
+  const size_t smem = 1024 + kStages * kStageBytes + 2 * kStages * 8 + (4 * kD + 16) * 4;
+  e = cudaFuncSetAttribute(decode_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  decode_stream_kernel<<<a.B * a.H, kThreads, smem, s>>>(tmA, tmB, a);
+  return cudaGetLastError();
+}
+
+}  // namespace hla

@@ -420,7 +420,10 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
   c.S_in = (float*)(ws + w.S_in);
   {
     StageScope _sc(HLA_STAGE_COMPOSE, s, 1);
-    HLA_CUDA(hla::launch_compose(c, s), "compose launch");
+    if (cfg->dtype == HLA_BF16 && cfg->dk == 128)
+      HLA_CUDA(hla::launch_compose_tc(c, s), "compose (tensor core) launch");
+    else
+      HLA_CUDA(hla::launch_compose(c, s), "compose launch");
   }
   hla::ReadoutArgs r{};
   r.B = cfg->B;
@@ -563,6 +566,10 @@ hla_status hla_device_status(int32_t clear, uint32_t* code_out) {
   HLA_CUDA(cudaDeviceSynchronize(), "hla_device_status synchronize");
   unsigned int word = 0, w = 0;
   HLA_CUDA(hla::read_error_word_decode(&w, clear != 0), "hla_device_status read");
+  word |= w;
+  HLA_CUDA(hla::read_error_word_compose_tc(&w, clear != 0), "hla_device_status read");
+  word |= w;
+  HLA_CUDA(hla::read_error_word_decode_stream(&w, clear != 0), "hla_device_status read");
   word |= w;
   if (code_out) *code_out = word;
   if (word & (hla::kErrMbarTimeout | hla::kErrTmemAlloc))

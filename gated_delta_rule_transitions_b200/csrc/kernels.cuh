@@ -110,5 +110,9 @@ cudaError_t launch_cache_fill(const DecodeArgs& c, const float* rk_ws, const voi
                               const void* k, const void* v, const float* alpha, const float* beta, int T,
                               cudaStream_t s);
 cudaError_t read_error_word_decode(unsigned int* out, bool clear);
+cudaError_t read_error_word_compose_tc(unsigned int* out, bool clear);
+cudaError_t launch_compose_tc(const ComposeArgs& a, cudaStream_t s);
+cudaError_t launch_decode_stream(const DecodeArgs& a, cudaStream_t s);
+cudaError_t read_error_word_decode_stream(unsigned int* out, bool clear);
 
 }  // namespace hla
