@@ -331,6 +331,8 @@ cudaError_t make_tmap_rows128(CUtensorMap* m, const void* base, long rows) {
 
 cudaError_t launch_compose_tc(const ComposeArgs& c, cudaStream_t s) {
   if (c.N <= 0) return cudaSuccess;
+  if (c.ab_chunk_stride <= 0)  // no complete chunk: every composed state is zero
+    return cudaMemsetAsync(c.S_in, 0, (size_t)c.B * c.H * c.N * kD * kD * sizeof(float), s);
   const long rows = (long)c.B * c.H * c.ab_chunk_stride * kD;
   CUtensorMap tmA, tmB;
   cudaError_t e = make_tmap_rows128(&tmA, c.A, rows);
