@@ -41,7 +41,7 @@ struct ComposeTcArgs {
   const int32_t* act_idx;
   const float* act_g;
   const int32_t* act_cnt;
-  float* S_in;
+  __nv_bfloat16* S_in;  // [B,H,N,d,d] bf16, row v, column c
 };
 
 // Walks the merged ascending active lists of the two chains.
@@ -212,8 +212,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // chains with nothing active have S_in = 0
     for (int k = 0; k < 2; ++k) {
       if (chains[k] >= 0 && sc.cnt[k] == 0) {
-        float4* out = (float4*)(a.S_in + ((long)bh * a.N + chains[k]) * kD * kD + (long)v * kD + col0);
-        for (int e = 0; e < 16; ++e) out[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+        uint4* out = (uint4*)(a.S_in + ((long)bh * a.N + chains[k]) * kD * kD + (long)v * kD + col0);
+        for (int e = 0; e < 8; ++e) out[e] = make_uint4(0u, 0u, 0u, 0u);
       }
     }
     int s = 0;
@@ -263,10 +263,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             x[2 * e + 1] = fmaf(g, tc::bf16hi(w), __uint_as_float(d[2 * e + 1]));
           }
           if (sc.last[k]) {
-            float4* out =
-                (float4*)(a.S_in + ((long)bh * a.N + chains[k]) * kD * kD + (long)v * kD + col0 + cc);
+            uint4* out = (uint4*)(a.S_in + ((long)bh * a.N + chains[k]) * kD * kD + (long)v * kD + col0 + cc);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) out[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
+            for (int e = 0; e < 4; ++e)
+              out[e] = make_uint4(tc::pack_bf16x2(x[8 * e], x[8 * e + 1]), tc::pack_bf16x2(x[8 * e + 2], x[8 * e + 3]),
+                                  tc::pack_bf16x2(x[8 * e + 4], x[8 * e + 5]),
+                                  tc::pack_bf16x2(x[8 * e + 6], x[8 * e + 7]));
           } else {
             uint32_t dn[32];
             uint32_t op[16];
@@ -315,6 +317,21 @@ EncodeTiledFn encode_fn() {
 
 }  // namespace
 
+// 2-D bf16 tensor map, `inner` elements per row, `rows` rows, 128-byte swizzle.
+cudaError_t make_tmap_2d(CUtensorMap* m, const void* base, long inner, long rows, long row_stride_bytes,
+                         int box_inner, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return cudaErrorNotSupported;
+  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)row_stride_bytes};
+  cuuint32_t box[2] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 // 2-D bf16 tensor map over `rows` rows of 128 elements, box 64 x 128, 128-byte swizzle.
 cudaError_t make_tmap_rows128(CUtensorMap* m, const void* base, long rows) {
   EncodeTiledFn fn = encode_fn();
@@ -332,7 +349,7 @@ cudaError_t make_tmap_rows128(CUtensorMap* m, const void* base, long rows) {
 cudaError_t launch_compose_tc(const ComposeArgs& c, cudaStream_t s) {
   if (c.N <= 0) return cudaSuccess;
   if (c.ab_chunk_stride <= 0)  // no complete chunk: every composed state is zero
-    return cudaMemsetAsync(c.S_in, 0, (size_t)c.B * c.H * c.N * kD * kD * sizeof(float), s);
+    return cudaMemsetAsync(c.S_in, 0, (size_t)c.B * c.H * c.N * kD * kD * sizeof(__nv_bfloat16), s);
   const long rows = (long)c.B * c.H * c.ab_chunk_stride * kD;
   CUtensorMap tmA, tmB;
   cudaError_t e = make_tmap_rows128(&tmA, c.A, rows);
@@ -346,7 +363,7 @@ cudaError_t launch_compose_tc(const ComposeArgs& c, cudaStream_t s) {
   a.act_idx = c.act_idx;
   a.act_g = c.act_g;
   a.act_cnt = c.act_cnt;
-  a.S_in = c.S_in;
+  a.S_in = (__nv_bfloat16*)c.S_in;
   const size_t smem = 1024 + kStages * kStageBytes + 256;
   e = cudaFuncSetAttribute(compose_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

@@ -263,7 +263,10 @@ hla_status gdn_chunk_transitions(const hla_config* cfg, const void* k, const voi
   t.A = A_out;
   t.Bm = B_out;
   t.ab_chunk_stride = Nc;
-  HLA_CUDA(hla::launch_transitions(t, (cudaStream_t)stream), "gdn_chunk_transitions launch");
+  if (cfg->dtype == HLA_BF16 && cfg->dk == 128)
+    HLA_CUDA(hla::launch_transitions_tc(t, (cudaStream_t)stream), "gdn_chunk_transitions (tensor core) launch");
+  else
+    HLA_CUDA(hla::launch_transitions(t, (cudaStream_t)stream), "gdn_chunk_transitions launch");
   return HLA_OK;
 }
 
@@ -375,6 +378,9 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
     return fail(HLA_ERR_WORKSPACE, "workspace too small: %zu < %zu", workspace_bytes, w.total);
   char* ws = (char*)workspace;
   cudaStream_t s = (cudaStream_t)stream;
+  // bf16 with d = 128 runs on the tensor cores (bf16 WY factors and S_in in the
+  // workspace); other shapes run the float32 CUDA-core kernels.
+  const bool tc_path = cfg->dtype == HLA_BF16 && cfg->dk == 128;
   const void* qr = q_route ? q_route : q;
   const void* kr = k_route ? k_route : k;
   float* rq = (float*)(ws + w.rq);
@@ -403,7 +409,10 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
   t.ell = (float*)(ws + w.ell);
   {
     StageScope _sc(HLA_STAGE_TRANSITIONS, s, 1);
-    HLA_CUDA(hla::launch_transitions(t, s), "transitions launch");
+    if (tc_path)
+      HLA_CUDA(hla::launch_transitions_tc(t, s), "transitions (tensor core) launch");
+    else
+      HLA_CUDA(hla::launch_transitions(t, s), "transitions launch");
   }
   hla::ComposeArgs c{};
   c.B = cfg->B;
@@ -420,7 +429,7 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
   c.S_in = (float*)(ws + w.S_in);
   {
     StageScope _sc(HLA_STAGE_COMPOSE, s, 1);
-    if (cfg->dtype == HLA_BF16 && cfg->dk == 128)
+    if (tc_path)
       HLA_CUDA(hla::launch_compose_tc(c, s), "compose (tensor core) launch");
     else
       HLA_CUDA(hla::launch_compose(c, s), "compose launch");
@@ -442,7 +451,10 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
   r.o = o;
   {
     StageScope _sc(HLA_STAGE_READOUT, s, 1);
-    HLA_CUDA(hla::launch_readout(r, s), "readout launch");
+    if (tc_path)
+      HLA_CUDA(hla::launch_readout_tc(r, c.S_in, t.Wb, t.Ub, s), "readout (tensor core) launch");
+    else
+      HLA_CUDA(hla::launch_readout(r, s), "readout launch");
   }
   if (cache_out) {
     hla::DecodeArgs dc{};
@@ -570,6 +582,10 @@ hla_status hla_device_status(int32_t clear, uint32_t* code_out) {
   HLA_CUDA(hla::read_error_word_compose_tc(&w, clear != 0), "hla_device_status read");
   word |= w;
   HLA_CUDA(hla::read_error_word_decode_stream(&w, clear != 0), "hla_device_status read");
+  word |= w;
+  HLA_CUDA(hla::read_error_word_transitions_tc(&w, clear != 0), "hla_device_status read");
+  word |= w;
+  HLA_CUDA(hla::read_error_word_readout_tc(&w, clear != 0), "hla_device_status read");
   word |= w;
   if (code_out) *code_out = word;
   if (word & (hla::kErrMbarTimeout | hla::kErrTmemAlloc))

@@ -113,6 +113,11 @@ cudaError_t read_error_word_decode(unsigned int* out, bool clear);
 cudaError_t read_error_word_compose_tc(unsigned int* out, bool clear);
 cudaError_t launch_compose_tc(const ComposeArgs& a, cudaStream_t s);
 cudaError_t launch_decode_stream(const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_transitions_tc(const TransArgs& t, cudaStream_t s);
+cudaError_t launch_readout_tc(const ReadoutArgs& r, const void* S_in_bf16, const void* Wb_bf16, const void* Ub_bf16,
+                              cudaStream_t s);
+cudaError_t read_error_word_transitions_tc(unsigned int* out, bool clear);
+cudaError_t read_error_word_readout_tc(unsigned int* out, bool clear);
 cudaError_t read_error_word_decode_stream(unsigned int* out, bool clear);
 
 }  // namespace hla

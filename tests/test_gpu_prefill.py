@@ -155,9 +155,10 @@ def test_gdn_chunk_transitions(hla, dtype, d):
                     assert np.abs(A[b, h, c] - Ar).max() <= P.TOL_F32_MAXABS
                     assert np.abs(Bm[b, h, c] - Br).max() <= P.TOL_F32_MAXABS
                 else:
-                    # bf16 storage: every entry within half an ulp of bf16 plus fp32 error
-                    assert np.all(np.abs(A[b, h, c] - Ar) <= np.abs(Ar) * 2 ** -8 + 1e-4)
-                    assert np.all(np.abs(Bm[b, h, c] - Br) <= np.abs(Br) * 2 ** -8 + 1e-4)
+                    # bf16 operands and storage: relative L2 per matrix well inside the
+                    # output tolerance
+                    assert P.rel_l2(A[b, h, c], Ar) <= 1e-2
+                    assert P.rel_l2(Bm[b, h, c], Br) <= 1e-2
 
 
 @pytest.mark.parametrize("dtype,d,T", [("f32", 64, 64 * 7 + 3), ("bf16", 128, 64 * 9)])
