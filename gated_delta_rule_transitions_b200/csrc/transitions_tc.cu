@@ -300,7 +300,7 @@ __global__ void __launch_bounds__(128, 2)
 cudaError_t launch_transitions_tc(const TransArgs& t, cudaStream_t s) {
   if (t.n_chunks <= 0) return cudaSuccess;
   const long HD = (long)t.H * kD;
-  const long rows = t.in.sb / HD;  // B * T_total
+  const long rows = (long)t.B * (t.in.sb / HD);  // B x tokens per sequence
   CUtensorMap tk, tv;
   cudaError_t e = make_tmap_2d(&tk, t.in.k, HD, rows, HD * 2, 64, 64);
   if (e == cudaSuccess) e = make_tmap_2d(&tv, t.in.v, HD, rows, HD * 2, 64, 64);
