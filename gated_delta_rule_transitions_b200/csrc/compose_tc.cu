@@ -16,8 +16,10 @@
 // last active step S_new is written to S_in (float32, [v][c]).
 //
 // Warp roles: warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer, warps 2-9
-// epilogue (lane quarter = warp % 4, column half = (warp - 2) / 4).  All waits are
-// bounded (about 2 s, then a device error word is set and the CTA exits cleanly).
+// epilogue of chain 0 and warps 10-17 epilogue of chain 1 (lane quarter = warp % 4,
+// column half = ((warp - 2) % 8) / 4), so each chain's epilogue overlaps the other
+// chain's MMA.  Elementwise math uses packed float32 pairs.  All waits are bounded
+// (about 2 s, then a device error word is set and the CTA exits cleanly).
 #include "common.cuh"
 #include "kernels.cuh"
 #include "tc_common.cuh"
@@ -32,7 +34,7 @@ constexpr int kD = 128;
 constexpr int kStages = 3;
 constexpr int kStageBytes = 2 * kD * kD * 2;     // A_j + B_j, bf16
 constexpr int kHalfBytes = kD * 64 * 2;          // one 64-column box
-constexpr int kThreads = 320;
+constexpr int kThreads = 576;  // producer, MMA, 2 x 8 epilogue warps
 constexpr uint32_t kIdesc = tc::idesc_bf16_f32(128, 128, /*a_mn=*/0, /*b_mn=*/1);
 
 struct ComposeTcArgs {
@@ -118,7 +120,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       tc::mbar_init(&full[s], 1);
-      tc::mbar_init(&empty[s], 2);
+      tc::mbar_init(&empty[s], 3);  // MMA commit + one arrival per epilogue group
     }
     for (int k = 0; k < 2; ++k) {
       tc::mbar_init(&mma_done[k], 1);
@@ -203,44 +205,47 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else {
-    // ---------------- epilogue (8 warps, 256 threads, named barrier 1) ----------------
+    // ------------- epilogue: group k (8 warps, 256 threads, named barrier 1 + k) -------------
+    const int k = (warp - 2) >> 3;
+    const int bar_id = 1 + k;
+    const int leader = (2 + 8 * k) * 32;
     const int q = warp & 3;
-    const int h = (warp - 2) >> 2;
+    const int h = ((warp - 2) & 7) >> 2;
     const int v = 32 * q + lane;
     const int col0 = 64 * h;
     const uint32_t lane_off = (uint32_t)(32 * q) << 16;
-    // chains with nothing active have S_in = 0
-    for (int k = 0; k < 2; ++k) {
-      if (chains[k] >= 0 && sc.cnt[k] == 0) {
-        uint4* out = (uint4*)(a.S_in + ((long)bh * a.N + chains[k]) * kD * kD + (long)v * kD + col0);
-        for (int e = 0; e < 8; ++e) out[e] = make_uint4(0u, 0u, 0u, 0u);
-      }
-    }
+    const int chain = k ? chains[1] : chains[0];
+    __nv_bfloat16* out_row =
+        chain >= 0 ? a.S_in + ((long)bh * a.N + chain) * kD * kD + (long)v * kD + col0 : nullptr;
+    // a chain with nothing active has S_in = 0
+    if (chain >= 0 && (k ? sc.cnt[1] : sc.cnt[0]) == 0)
+      for (int e = 0; e < 8; ++e) ((uint4*)out_row)[e] = make_uint4(0u, 0u, 0u, 0u);
     int s = 0;
     bool ok = true;
     while (ok && sc.next()) {
       const int st = s % kStages;
-      ok = tc::bar_all(1, 256, tc::mbar_wait(&full[st], (s / kStages) & 1, abort_s));
+      ok = tc::bar_all(bar_id, 256, tc::mbar_wait(&full[st], (s / kStages) & 1, abort_s));
       if (!ok) break;
-      // B_j[v][col0 .. col0+64) from the swizzled box
-      const uint8_t* brow = ring + st * kStageBytes + 2 * kHalfBytes + h * kHalfBytes + v * 128;
-      uint32_t bw[32];
+      if (k ? sc.act[1] : sc.act[0]) {
+        // B_j[v][col0 .. col0+64) from the swizzled box
+        const uint8_t* brow = ring + st * kStageBytes + 2 * kHalfBytes + h * kHalfBytes + v * 128;
+        uint32_t bw[32];
 #pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) {
-        const uint4 w = *(const uint4*)(brow + ((c8 ^ (v & 7)) << 4));
-        bw[4 * c8 + 0] = w.x;
-        bw[4 * c8 + 1] = w.y;
-        bw[4 * c8 + 2] = w.z;
-        bw[4 * c8 + 3] = w.w;
-      }
-      for (int k = 0; k < 2; ++k) {
-        if (!sc.act[k]) continue;
-        const bool first = sc.first[k];
-        const float g = sc.gate[k];
-        const float gn = sc.gnext[k];
+        for (int c8 = 0; c8 < 8; ++c8) {
+          const uint4 w = *(const uint4*)(brow + ((c8 ^ (v & 7)) << 4));
+          bw[4 * c8 + 0] = w.x;
+          bw[4 * c8 + 1] = w.y;
+          bw[4 * c8 + 2] = w.z;
+          bw[4 * c8 + 3] = w.w;
+        }
+        const bool first = k ? sc.first[1] : sc.first[0];
+        const bool last = k ? sc.last[1] : sc.last[0];
+        const float g = k ? sc.gate[1] : sc.gate[0];
+        const float gn = k ? sc.gnext[1] : sc.gnext[0];
+        const int pk = k ? sc.p[1] : sc.p[0];
         const float keep = 1.0f - gn;
         if (!first) {
-          ok = tc::bar_all(1, 256, tc::mbar_wait(&mma_done[k], (sc.p[k] - 1) & 1, abort_s));
+          ok = tc::bar_all(bar_id, 256, tc::mbar_wait(&mma_done[k], (pk - 1) & 1, abort_s));
           if (!ok) break;
           tc::tc_fence_after();
         }
@@ -259,35 +264,41 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const uint32_t w = bw[cc / 2 + e];
-            x[2 * e] = fmaf(g, tc::bf16lo(w), __uint_as_float(d[2 * e]));
-            x[2 * e + 1] = fmaf(g, tc::bf16hi(w), __uint_as_float(d[2 * e + 1]));
+            tc::fma2(x[2 * e], x[2 * e + 1], g, g, tc::bf16lo(w), tc::bf16hi(w), __uint_as_float(d[2 * e]),
+                     __uint_as_float(d[2 * e + 1]));
           }
-          if (sc.last[k]) {
-            uint4* out = (uint4*)(a.S_in + ((long)bh * a.N + chains[k]) * kD * kD + (long)v * kD + col0 + cc);
+          if (last) {
+            uint4* out = (uint4*)(out_row + cc);
 #pragma unroll
             for (int e = 0; e < 4; ++e)
               out[e] = make_uint4(tc::pack_bf16x2(x[8 * e], x[8 * e + 1]), tc::pack_bf16x2(x[8 * e + 2], x[8 * e + 3]),
                                   tc::pack_bf16x2(x[8 * e + 4], x[8 * e + 5]),
                                   tc::pack_bf16x2(x[8 * e + 6], x[8 * e + 7]));
           } else {
-            uint32_t dn[32];
             uint32_t op[16];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) dn[e] = __float_as_uint(keep * x[e]);
-#pragma unroll
-            for (int e = 0; e < 16; ++e) op[e] = tc::pack_bf16x2(gn * x[2 * e], gn * x[2 * e + 1]);
-            tc::tmem_st32(d_addr, dn);
+            for (int e = 0; e < 16; ++e) {
+              float o0, o1, n0, n1;
+              tc::mul2(o0, o1, gn, gn, x[2 * e], x[2 * e + 1]);
+              tc::mul2(n0, n1, keep, keep, x[2 * e], x[2 * e + 1]);
+              op[e] = tc::pack_bf16x2(o0, o1);
+              d[2 * e] = __float_as_uint(n0);
+              d[2 * e + 1] = __float_as_uint(n1);
+            }
+            tc::tmem_st32(d_addr, d);
             tc::tmem_st16(tbase + lane_off + 256u + 64u * k + (col0 + cc) / 2, op);
           }
         }
         tc::tmem_wait_st();
         tc::tc_fence_before();
-        tc::bar_sync(1, 256);
-        if (threadIdx.x == 64 && !sc.last[k]) tc::mbar_arrive(&op_ready[k]);
+        tc::bar_sync(bar_id, 256);
+        if (threadIdx.x == leader) {
+          if (!last) tc::mbar_arrive(&op_ready[k]);
+          tc::mbar_arrive(&empty[st]);
+        }
+      } else if (threadIdx.x == leader) {
+        tc::mbar_arrive(&empty[st]);
       }
-      if (!ok) break;
-      tc::bar_sync(1, 256);
-      if (threadIdx.x == 64) tc::mbar_arrive(&empty[st]);
       sc.advance();
       ++s;
     }

@@ -36,7 +36,7 @@ constexpr int kC = 64;
 constexpr int kKV = 0;             // [kh][K | V][64 rows][128 B]   32 KiB
 constexpr int kTT = 32768;         // [T gamma; T] 128 rows x 128 B 16 KiB; later D K
 constexpr int kScr = 49152;        // L, T float32 [64][65] each; later Wb^T, Ub^T operands
-constexpr int kLP = kC + 1;
+constexpr int kLP = kC + 4;  // row pitch of the float32 L and T (16-byte rows)
 constexpr int kSmemUsed = kScr + 2 * kC * kLP * 4;
 constexpr uint32_t kIdesc1 = tc::idesc_bf16_f32(128, 64, 0, 0);
 constexpr uint32_t kIdesc2 = tc::idesc_bf16_f32(128, 256, 0, 1);
@@ -147,21 +147,27 @@ __global__ void __launch_bounds__(128, 2)
   }
   ok = tc::bar_all(1, 128, ok);
   if (ok && tid < kC) {
-    // column c of T = (I + L)^{-1} diag(beta) by forward substitution
+    // column c of T = (I + L)^{-1} diag(beta) by forward substitution, fully unrolled
+    // so the column stays in registers; every thread runs the same schedule (entries
+    // above the diagonal come out as exact zeros), so the reads of L are broadcasts.
     const int c = tid;
-    for (int t = 0; t < c; ++t) Ts[t * kLP + c] = 0.0f;
-    for (int t = c; t < kC; ++t) {
+    float col[kC];
+#pragma unroll
+    for (int t = 0; t < kC; ++t) {
+      const float* Lrow = Ls + t * kLP;
       float a0 = (t == c) ? beta_s[t] : 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
-      int s = c;
-      for (; s + 3 < t; s += 4) {
-        a0 = fmaf(-Ls[t * kLP + s], Ts[s * kLP + c], a0);
-        a1 = fmaf(-Ls[t * kLP + s + 1], Ts[(s + 1) * kLP + c], a1);
-        a2 = fmaf(-Ls[t * kLP + s + 2], Ts[(s + 2) * kLP + c], a2);
-        a3 = fmaf(-Ls[t * kLP + s + 3], Ts[(s + 3) * kLP + c], a3);
+#pragma unroll
+      for (int s4 = 0; s4 < t; s4 += 4) {
+        const float4 l4 = *(const float4*)(Lrow + s4);
+        a0 = fmaf(-l4.x, col[s4], a0);
+        if (s4 + 1 < t) a1 = fmaf(-l4.y, col[s4 + 1], a1);
+        if (s4 + 2 < t) a2 = fmaf(-l4.z, col[s4 + 2], a2);
+        if (s4 + 3 < t) a3 = fmaf(-l4.w, col[s4 + 3], a3);
       }
-      for (; s < t; ++s) a0 = fmaf(-Ls[t * kLP + s], Ts[s * kLP + c], a0);
-      Ts[t * kLP + c] = (a0 + a1) + (a2 + a3);
+      col[t] = (a0 + a1) + (a2 + a3);
     }
+#pragma unroll
+    for (int t = 0; t < kC; ++t) Ts[t * kLP + c] = col[t];
   }
   ok = tc::bar_all(1, 128, ok);
   if (ok) {
