@@ -96,6 +96,15 @@ struct Sched {
   }
 };
 
+// One step of the merged schedule, published by the producer next to its stage.
+struct StepInfo {
+  int j;       // chunk index; -1 ends the schedule
+  int flags;   // bit k: chain k active; bit 2+k: first step of chain k; bit 4+k: last step
+  int p[2];    // index of this step in each chain's active list
+  float g[2];  // gates at this step
+  float gn[2]; // gates at each chain's next active step (0 if none)
+};
+
 __global__ void __launch_bounds__(kThreads, 1)
     compose_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       ComposeTcArgs a) {
@@ -103,12 +112,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* ring = smem;  // kStages x [A half0 | A half1 | B half0 | B half1]
   uint64_t* bars = (uint64_t*)(smem + kStages * kStageBytes);
-  uint64_t* full = bars;                 // [kStages]
-  uint64_t* empty = bars + kStages;      // [kStages]
+  uint64_t* full = bars;                    // [kStages]
+  uint64_t* empty = bars + kStages;         // [kStages]
   uint64_t* mma_done = bars + 2 * kStages;  // [2]
   uint64_t* op_ready = mma_done + 2;        // [2]
   uint64_t* final_bar = op_ready + 2;       // [1]
-  uint32_t* tmem_base_s = (uint32_t*)(final_bar + 1);
+  StepInfo* info = (StepInfo*)(final_bar + 1);  // [kStages]
+  uint32_t* tmem_base_s = (uint32_t*)(info + kStages);
   volatile int* abort_s = (volatile int*)(tmem_base_s + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -120,11 +130,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       tc::mbar_init(&full[s], 1);
-      tc::mbar_init(&empty[s], 3);  // MMA commit + one arrival per epilogue group
+      tc::mbar_init(&empty[s], 1 + 16);  // MMA commit + lane 0 of every epilogue warp
     }
     for (int k = 0; k < 2; ++k) {
       tc::mbar_init(&mma_done[k], 1);
-      tc::mbar_init(&op_ready[k], 1);
+      tc::mbar_init(&op_ready[k], 8);   // lane 0 of every warp of the chain's group
     }
     tc::mbar_init(final_bar, 1);
     *abort_s = 0;
@@ -141,17 +151,32 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc::tc_fence_after();
   const uint32_t tbase = *tmem_base_s;
 
-  Sched sc;
-  sc.init(a, bh, chains);
-
   if (warp == 0) {
-    // ---------------- TMA producer (lane 0) ----------------
+    // ---------------- TMA producer (lane 0): walks the merged lists ----------------
     if (lane == 0) {
+      Sched sc;
+      sc.init(a, bh, chains);
       int s = 0;
+      bool ok = true;
       while (sc.next()) {
         const int st = s % kStages;
-        if (s >= kStages && !tc::mbar_wait(&empty[st], ((s / kStages) - 1) & 1, abort_s)) break;
-        tc::mbar_arrive_expect_tx(&full[st], kStageBytes);
+        if (s >= kStages && !tc::mbar_wait(&empty[st], ((s / kStages) - 1) & 1, abort_s)) {
+          ok = false;
+          break;
+        }
+        StepInfo e;
+        e.j = sc.j;
+        e.flags = 0;
+        for (int k = 0; k < 2; ++k) {
+          e.flags |= (sc.act[k] ? 1 : 0) << k;
+          e.flags |= (sc.first[k] ? 1 : 0) << (2 + k);
+          e.flags |= (sc.last[k] ? 1 : 0) << (4 + k);
+          e.p[k] = sc.p[k];
+          e.g[k] = sc.gate[k];
+          e.gn[k] = sc.gnext[k];
+        }
+        info[st] = e;
+        tc::mbar_arrive_expect_tx(&full[st], kStageBytes);  // releases info[st]
         const int row = (int)(((long)bh * a.ab_chunk_stride + sc.j) * kD);
         uint8_t* dst = ring + st * kStageBytes;
         tc::tma_load_2d(dst, &tmA, 0, row, &full[st]);
@@ -160,6 +185,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::tma_load_2d(dst + 3 * kHalfBytes, &tmB, 64, row, &full[st]);
         sc.advance();
         ++s;
+      }
+      if (ok) {
+        // end marker: a stage phase with no data
+        const int st = s % kStages;
+        if (s < kStages || tc::mbar_wait(&empty[st], ((s / kStages) - 1) & 1, abort_s)) {
+          info[st].j = -1;
+          tc::mbar_arrive(&full[st]);
+        }
       }
       if (*abort_s) {
         // never leave the CTA with copies in flight
@@ -171,16 +204,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ---------------- MMA issuer (lane 0) ----------------
     if (lane == 0) {
-      int s = 0;
-      bool ok = true;
-      while (ok && sc.next()) {
+      for (int s = 0;; ++s) {
         const int st = s % kStages;
         if (!tc::mbar_wait(&full[st], (s / kStages) & 1, abort_s)) break;
+        const StepInfo e = info[st];
+        if (e.j < 0) break;
         tc::tc_fence_after();
         const uint32_t b_base = tc::smem_u32(ring + st * kStageBytes);
+        bool ok = true;
         for (int k = 0; k < 2; ++k) {
-          if (!sc.act[k] || sc.first[k]) continue;
-          if (!tc::mbar_wait(&op_ready[k], (sc.p[k] - 1) & 1, abort_s)) {
+          if (!((e.flags >> k) & 1) || ((e.flags >> (2 + k)) & 1)) continue;
+          if (!tc::mbar_wait(&op_ready[k], (e.p[k] - 1) & 1, abort_s)) {
             ok = false;
             break;
           }
@@ -196,8 +230,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!ok) break;
         tc::mma_commit(&empty[st]);
-        sc.advance();
-        ++s;
       }
       // all MMAs issued by this thread complete before the CTA frees tensor memory
       tc::mma_commit(final_bar);
@@ -208,7 +240,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------- epilogue: group k (8 warps, 256 threads, named barrier 1 + k) -------------
     const int k = (warp - 2) >> 3;
     const int bar_id = 1 + k;
-    const int leader = (2 + 8 * k) * 32;
     const int q = warp & 3;
     const int h = ((warp - 2) & 7) >> 2;
     const int v = 32 * q + lane;
@@ -218,35 +249,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     __nv_bfloat16* out_row =
         chain >= 0 ? a.S_in + ((long)bh * a.N + chain) * kD * kD + (long)v * kD + col0 : nullptr;
     // a chain with nothing active has S_in = 0
-    if (chain >= 0 && (k ? sc.cnt[1] : sc.cnt[0]) == 0)
+    if (chain >= 0 && a.act_cnt[(long)bh * a.N + chain] == 0)
       for (int e = 0; e < 8; ++e) ((uint4*)out_row)[e] = make_uint4(0u, 0u, 0u, 0u);
-    int s = 0;
-    bool ok = true;
-    while (ok && sc.next()) {
+    for (int s = 0;; ++s) {
       const int st = s % kStages;
-      ok = tc::bar_all(bar_id, 256, tc::mbar_wait(&full[st], (s / kStages) & 1, abort_s));
-      if (!ok) break;
-      if (k ? sc.act[1] : sc.act[0]) {
+      const bool w = tc::mbar_wait(&full[st], (s / kStages) & 1, abort_s);
+      const int jv = w ? ((volatile StepInfo*)info)[st].j : 0;
+      // one vote per step: stop at the end marker or on a timeout anywhere
+      if (tc::bar_any(bar_id, 256, !w || *abort_s != 0 || jv < 0)) break;
+      const StepInfo e = info[st];
+      const bool act = (e.flags >> k) & 1;
+      const bool last = (e.flags >> (4 + k)) & 1;
+      if (act) {
+        const bool first = (e.flags >> (2 + k)) & 1;
+        const float g = k ? e.g[1] : e.g[0];
+        const float gn = k ? e.gn[1] : e.gn[0];
+        const int pk = k ? e.p[1] : e.p[0];
+        const float keep = 1.0f - gn;
         // B_j[v][col0 .. col0+64) from the swizzled box
         const uint8_t* brow = ring + st * kStageBytes + 2 * kHalfBytes + h * kHalfBytes + v * 128;
         uint32_t bw[32];
 #pragma unroll
         for (int c8 = 0; c8 < 8; ++c8) {
-          const uint4 w = *(const uint4*)(brow + ((c8 ^ (v & 7)) << 4));
-          bw[4 * c8 + 0] = w.x;
-          bw[4 * c8 + 1] = w.y;
-          bw[4 * c8 + 2] = w.z;
-          bw[4 * c8 + 3] = w.w;
+          const uint4 w4 = *(const uint4*)(brow + ((c8 ^ (v & 7)) << 4));
+          bw[4 * c8 + 0] = w4.x;
+          bw[4 * c8 + 1] = w4.y;
+          bw[4 * c8 + 2] = w4.z;
+          bw[4 * c8 + 3] = w4.w;
         }
-        const bool first = k ? sc.first[1] : sc.first[0];
-        const bool last = k ? sc.last[1] : sc.last[0];
-        const float g = k ? sc.gate[1] : sc.gate[0];
-        const float gn = k ? sc.gnext[1] : sc.gnext[0];
-        const int pk = k ? sc.p[1] : sc.p[0];
-        const float keep = 1.0f - gn;
         if (!first) {
-          ok = tc::bar_all(bar_id, 256, tc::mbar_wait(&mma_done[k], (pk - 1) & 1, abort_s));
-          if (!ok) break;
+          tc::mbar_wait(&mma_done[k], (pk - 1) & 1, abort_s);
           tc::tc_fence_after();
         }
 #pragma unroll
@@ -258,32 +290,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::tmem_wait_ld();
           } else {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) d[e] = 0u;
+            for (int i = 0; i < 32; ++i) d[i] = 0u;
           }
           float x[32];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const uint32_t w = bw[cc / 2 + e];
-            tc::fma2(x[2 * e], x[2 * e + 1], g, g, tc::bf16lo(w), tc::bf16hi(w), __uint_as_float(d[2 * e]),
-                     __uint_as_float(d[2 * e + 1]));
+          for (int i = 0; i < 16; ++i) {
+            const uint32_t wb = bw[cc / 2 + i];
+            tc::fma2(x[2 * i], x[2 * i + 1], g, g, tc::bf16lo(wb), tc::bf16hi(wb), __uint_as_float(d[2 * i]),
+                     __uint_as_float(d[2 * i + 1]));
           }
           if (last) {
             uint4* out = (uint4*)(out_row + cc);
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              out[e] = make_uint4(tc::pack_bf16x2(x[8 * e], x[8 * e + 1]), tc::pack_bf16x2(x[8 * e + 2], x[8 * e + 3]),
-                                  tc::pack_bf16x2(x[8 * e + 4], x[8 * e + 5]),
-                                  tc::pack_bf16x2(x[8 * e + 6], x[8 * e + 7]));
+            for (int i = 0; i < 4; ++i)
+              out[i] = make_uint4(tc::pack_bf16x2(x[8 * i], x[8 * i + 1]), tc::pack_bf16x2(x[8 * i + 2], x[8 * i + 3]),
+                                  tc::pack_bf16x2(x[8 * i + 4], x[8 * i + 5]),
+                                  tc::pack_bf16x2(x[8 * i + 6], x[8 * i + 7]));
           } else {
             uint32_t op[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
+            for (int i = 0; i < 16; ++i) {
               float o0, o1, n0, n1;
-              tc::mul2(o0, o1, gn, gn, x[2 * e], x[2 * e + 1]);
-              tc::mul2(n0, n1, keep, keep, x[2 * e], x[2 * e + 1]);
-              op[e] = tc::pack_bf16x2(o0, o1);
-              d[2 * e] = __float_as_uint(n0);
-              d[2 * e + 1] = __float_as_uint(n1);
+              tc::mul2(o0, o1, gn, gn, x[2 * i], x[2 * i + 1]);
+              tc::mul2(n0, n1, keep, keep, x[2 * i], x[2 * i + 1]);
+              op[i] = tc::pack_bf16x2(o0, o1);
+              d[2 * i] = __float_as_uint(n0);
+              d[2 * i + 1] = __float_as_uint(n1);
             }
             tc::tmem_st32(d_addr, d);
             tc::tmem_st16(tbase + lane_off + 256u + 64u * k + (col0 + cc) / 2, op);
@@ -291,16 +323,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc::tmem_wait_st();
         tc::tc_fence_before();
-        tc::bar_sync(bar_id, 256);
-        if (threadIdx.x == leader) {
-          if (!last) tc::mbar_arrive(&op_ready[k]);
-          tc::mbar_arrive(&empty[st]);
-        }
-      } else if (threadIdx.x == leader) {
+      }
+      __syncwarp();
+      if (lane == 0) {
+        if (act && !last) tc::mbar_arrive(&op_ready[k]);
         tc::mbar_arrive(&empty[st]);
       }
-      sc.advance();
-      ++s;
     }
   }
   tc::tc_fence_before();
@@ -375,7 +403,7 @@ cudaError_t launch_compose_tc(const ComposeArgs& c, cudaStream_t s) {
   a.act_g = c.act_g;
   a.act_cnt = c.act_cnt;
   a.S_in = (__nv_bfloat16*)c.S_in;
-  const size_t smem = 1024 + kStages * kStageBytes + 256;
+  const size_t smem = 1024 + kStages * kStageBytes + 512;
   e = cudaFuncSetAttribute(compose_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int pairs = (c.N + 1) / 2;
