@@ -292,30 +292,29 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 32; ++i) d[i] = 0u;
           }
-          float x[32];
+          const float2 g2 = make_float2(g, g);
+          float2 x[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const uint32_t wb = bw[cc / 2 + i];
-            tc::fma2(x[2 * i], x[2 * i + 1], g, g, tc::bf16lo(wb), tc::bf16hi(wb), __uint_as_float(d[2 * i]),
-                     __uint_as_float(d[2 * i + 1]));
-          }
+          for (int i = 0; i < 16; ++i)
+            x[i] = tc::fma2(g2, tc::bf16x2_to_float2(bw[cc / 2 + i]),
+                            make_float2(__uint_as_float(d[2 * i]), __uint_as_float(d[2 * i + 1])));
           if (last) {
             uint4* out = (uint4*)(out_row + cc);
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-              out[i] = make_uint4(tc::pack_bf16x2(x[8 * i], x[8 * i + 1]), tc::pack_bf16x2(x[8 * i + 2], x[8 * i + 3]),
-                                  tc::pack_bf16x2(x[8 * i + 4], x[8 * i + 5]),
-                                  tc::pack_bf16x2(x[8 * i + 6], x[8 * i + 7]));
+              out[i] = make_uint4(tc::pack_bf16x2(x[4 * i].x, x[4 * i].y), tc::pack_bf16x2(x[4 * i + 1].x, x[4 * i + 1].y),
+                                  tc::pack_bf16x2(x[4 * i + 2].x, x[4 * i + 2].y),
+                                  tc::pack_bf16x2(x[4 * i + 3].x, x[4 * i + 3].y));
           } else {
+            const float2 gn2 = make_float2(gn, gn), keep2 = make_float2(keep, keep);
             uint32_t op[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              float o0, o1, n0, n1;
-              tc::mul2(o0, o1, gn, gn, x[2 * i], x[2 * i + 1]);
-              tc::mul2(n0, n1, keep, keep, x[2 * i], x[2 * i + 1]);
-              op[i] = tc::pack_bf16x2(o0, o1);
-              d[2 * i] = __float_as_uint(n0);
-              d[2 * i + 1] = __float_as_uint(n1);
+              const float2 o = tc::mul2(gn2, x[i]);
+              const float2 nn = tc::mul2(keep2, x[i]);
+              op[i] = tc::pack_bf16x2(o.x, o.y);
+              d[2 * i] = __float_as_uint(nn.x);
+              d[2 * i + 1] = __float_as_uint(nn.y);
             }
             tc::tmem_st32(d_addr, d);
             tc::tmem_st16(tbase + lane_off + 256u + 64u * k + (col0 + cc) / 2, op);
