@@ -78,7 +78,7 @@ float gate_scale(int d) { return (float)(1.0 / std::sqrt((double)d)); }
 
 // Prefill workspace layout.
 struct PrefillWs {
-  size_t rq, rk, act_idx, act_g, act_cnt, A, Bm, Wb, Ub, ell, S_in, dk, ut, total;
+  size_t rq, rk, act_idx, act_g, act_cnt, A, Bm, Wb, Ub, ell, S_in, total;
 };
 
 PrefillWs prefill_layout(const hla_config* c) {
@@ -103,10 +103,6 @@ PrefillWs prefill_layout(const hla_config* c) {
   w.Ub = take(B * H * N * C * d * 4);
   w.ell = take(B * H * N * C * 4);
   w.S_in = take(B * H * N * d * d * 4);
-  // tensor-core path: rank-C factors of B_j, (D K)_j [C][d] and Ub_j^T [d][C], bf16
-  const bool tc = c->dtype == HLA_BF16 && d == 128;
-  w.dk = take(tc ? B * H * N * C * d * 2 : 0);
-  w.ut = take(tc ? B * H * N * C * d * 2 : 0);
   w.total = off;
   return w;
 }
@@ -406,13 +402,7 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
           (long)cfg->T * cfg->H, 1, cfg->H};
   t.n_chunks = N;
   t.A = cache_out ? cache_out->A : (void*)(ws + w.A);
-  // the tensor-core composition uses B_j's factors, so B_j itself is only needed by
-  // the CUDA-core path or for the decode cache
-  t.Bm = cache_out ? cache_out->Bm : (tc_path ? nullptr : (void*)(ws + w.Bm));
-  if (tc_path) {
-    t.DK = ws + w.dk;
-    t.UT = ws + w.ut;
-  }
+  t.Bm = cache_out ? cache_out->Bm : (void*)(ws + w.Bm);
   t.ab_chunk_stride = cache_out ? cache_out->max_chunks : Nc;
   t.Wb = (float*)(ws + w.Wb);
   t.Ub = (float*)(ws + w.Ub);
@@ -437,8 +427,6 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
   c.act_g = act_g;
   c.act_cnt = act_cnt;
   c.S_in = (float*)(ws + w.S_in);
-  c.DK = t.DK;
-  c.UT = t.UT;
   {
     StageScope _sc(HLA_STAGE_COMPOSE, s, 1);
     if (tc_path)

@@ -46,8 +46,6 @@ struct TransArgs {
   float* ell;            // [B,H,N,C] fp32 or null
   const int32_t* close_m;   // decode close: per-b m_partial (before the step) or null
   const int32_t* close_n;   // decode close: per-b n_chunks or null
-  void* DK;                 // tensor-core path: D K factors [B,H,N,C,d] bf16 or null
-  void* UT;                 // tensor-core path: Ub^T factors [B,H,N,d,C] bf16 or null
 };
 
 struct ComposeArgs {
@@ -58,9 +56,7 @@ struct ComposeArgs {
   const int32_t* act_idx; // [B,H,N,N]
   const float* act_g;
   const int32_t* act_cnt; // [B,H,N]
-  float* S_in;            // [B,H,N,d,d] fp32 (bf16 on the tensor-core path)
-  const void* DK;         // tensor-core path: [B,H,N,C,d] bf16 (chunk stride N)
-  const void* UT;         // tensor-core path: [B,H,N,d,C] bf16
+  float* S_in;            // [B,H,N,d,d] fp32
 };
 
 struct ReadoutArgs {

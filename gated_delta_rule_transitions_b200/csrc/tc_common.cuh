@@ -83,6 +83,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Warp-cooperative wait: lane 0 polls (keeping shared-memory traffic off the tensor
+// core's operand reads), the other lanes wait at the warp barrier.  Returns lane 0's
+// result in every lane.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                               uint64_t limit_ns = 2000000000ull) {
+  int ok = 0;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, limit_ns) ? 1 : 0;
+  __syncwarp();  // orders the other lanes' later accesses after lane 0's acquire
+  return __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
+}
+
 // AND of `ok` over the `nthreads` threads that use named barrier `id` (all of them
 // must call it; it completes even when some pass false).
 __device__ __forceinline__ bool bar_all(int id, int nthreads, bool ok) {

@@ -53,8 +53,6 @@ struct TransTcArgs {
   __nv_bfloat16* Wb;                // [B,H,N,C,d] or null
   __nv_bfloat16* Ub;
   float* ell;                       // [B,H,N,C] or null
-  __nv_bfloat16* DK;                // [B,H,N,C,d] D K (row t) of complete chunks, or null
-  __nv_bfloat16* UT;                // [B,H,N,d,C] Ub^T (row v) of complete chunks, or null
 };
 
 __device__ __forceinline__ int swz(int row, int chunk) { return row * 128 + ((chunk ^ (row & 7)) << 4); }
@@ -227,16 +225,6 @@ __global__ void __launch_bounds__(128, 2)
 #pragma unroll
         for (int c8 = 0; c8 < 8; ++c8) dst[c8] = make_uint4(w[4 * c8], w[4 * c8 + 1], w[4 * c8 + 2], w[4 * c8 + 3]);
       }
-      if (!isW && a.UT != nullptr && n == kC) {
-        // Ub^T[v][t]: column t of the transposed factor (coalesced across t in a warp)
-        unsigned short* ut = (unsigned short*)a.UT + chunk * kD * kC + t;
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int v = 64 * half + 2 * e;
-          ut[(long)v * kC] = (unsigned short)(w[e] & 0xFFFFu);
-          ut[(long)(v + 1) * kC] = (unsigned short)(w[e] >> 16);
-        }
-      }
 #pragma unroll
       for (int c8 = 0; c8 < 8; ++c8)
         *(uint4*)(opT + half * 8192 + swz(t, c8)) = make_uint4(w[4 * c8], w[4 * c8 + 1], w[4 * c8 + 2], w[4 * c8 + 3]);
@@ -254,8 +242,6 @@ __global__ void __launch_bounds__(128, 2)
 #pragma unroll
           for (int e = 0; e < 4; ++e) w[e] = tc::pack_bf16x2(dt * tc::bf16lo(kk[e]), dt * tc::bf16hi(kk[e]));
           *(uint4*)(sm + kTT + half * 8192 + swz(t, c8)) = make_uint4(w[0], w[1], w[2], w[3]);
-          if (a.DK != nullptr && n == kC)
-            *(uint4*)(a.DK + (chunk * kC + t) * kD + 64 * half + 8 * c8) = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
     }
@@ -272,8 +258,7 @@ __global__ void __launch_bounds__(128, 2)
     for (int ks = 0; ks < kC / 16; ++ks) {
       const uint64_t bd = tc::sdesc_sw128(dbase + ks * 2048, 8192, 1024);
       tc::mma_ss(tm, tc::sdesc_sw128(wbase + ks * 2048, 8192, 1024), bd, kIdesc3, ks > 0 ? 1u : 0u);
-      if (a.Bm != nullptr)
-        tc::mma_ss(tm + 128, tc::sdesc_sw128(ubase + ks * 2048, 8192, 1024), bd, kIdesc3, ks > 0 ? 1u : 0u);
+      tc::mma_ss(tm + 128, tc::sdesc_sw128(ubase + ks * 2048, 8192, 1024), bd, kIdesc3, ks > 0 ? 1u : 0u);
     }
     tc::mma_commit(&bars[3]);
   }
@@ -283,7 +268,7 @@ __global__ void __launch_bounds__(128, 2)
     const int r = tid;
     const float gC = __expf(ell_s[kC - 1]);
     __nv_bfloat16* Arow = a.A + ((long)bh * a.ab_chunk_stride + i) * kD * kD + (long)r * kD;
-    __nv_bfloat16* Brow = a.Bm ? a.Bm + ((long)bh * a.ab_chunk_stride + i) * kD * kD + (long)r * kD : nullptr;
+    __nv_bfloat16* Brow = a.Bm + ((long)bh * a.ab_chunk_stride + i) * kD * kD + (long)r * kD;
 #pragma unroll
     for (int cc = 0; cc < kD; cc += 32) {
       uint32_t x[32], y[32];
@@ -300,12 +285,11 @@ __global__ void __launch_bounds__(128, 2)
         wb[e] = tc::pack_bf16x2(__uint_as_float(y[2 * e]), __uint_as_float(y[2 * e + 1]));
       }
       uint4* da = (uint4*)(Arow + cc);
+      uint4* db = (uint4*)(Brow + cc);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) da[e] = make_uint4(wa[4 * e], wa[4 * e + 1], wa[4 * e + 2], wa[4 * e + 3]);
-      if (a.Bm != nullptr) {
-        uint4* db = (uint4*)(Brow + cc);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) db[e] = make_uint4(wb[4 * e], wb[4 * e + 1], wb[4 * e + 2], wb[4 * e + 3]);
+      for (int e = 0; e < 4; ++e) {
+        da[e] = make_uint4(wa[4 * e], wa[4 * e + 1], wa[4 * e + 2], wa[4 * e + 3]);
+        db[e] = make_uint4(wb[4 * e], wb[4 * e + 1], wb[4 * e + 2], wb[4 * e + 3]);
       }
     }
   }
@@ -343,8 +327,6 @@ cudaError_t launch_transitions_tc(const TransArgs& t, cudaStream_t s) {
   a.Wb = (__nv_bfloat16*)t.Wb;
   a.Ub = (__nv_bfloat16*)t.Ub;
   a.ell = t.ell;
-  a.DK = (__nv_bfloat16*)t.DK;
-  a.UT = (__nv_bfloat16*)t.UT;
   // chunks beyond t.T (gdn_chunk_transitions limits T to whole chunks) are not launched
   const size_t smem = 1024 + kSmemUsed + 4 * 8 + 16 + 2 * kC * 4 + 16;
   e = cudaFuncSetAttribute(transitions_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
