@@ -12,6 +12,7 @@ from ._hla import (  # noqa: F401
     decode_workspace_bytes,
     gdn_chunk_transitions,
     hla_decode_step,
+    hla_decode_step_static,
     hla_device_status,
     hla_prefill,
     hla_profile_enable,

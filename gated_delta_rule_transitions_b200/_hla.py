@@ -66,6 +66,8 @@ _SIGS = {
                      ctypes.POINTER(HlaCache), _P, ctypes.c_size_t, _P], ctypes.c_int),
     "hla_decode_step": ([ctypes.POINTER(HlaConfig), ctypes.POINTER(HlaCache), _P, _P, _P, _P, _P, _P, _P, _P, _P,
                          ctypes.c_size_t, _P], ctypes.c_int),
+    "hla_decode_step_static": ([ctypes.POINTER(HlaConfig), ctypes.POINTER(HlaCache), _P, _P, _P, _P, _P, _P, _P,
+                                _P, _P], ctypes.c_int),
     "hla_device_status": ([ctypes.c_int32, ctypes.POINTER(ctypes.c_uint32)], ctypes.c_int),
     "hla_profile_enable": ([ctypes.c_int32], ctypes.c_int),
     "hla_profile_read": ([_P, _P, ctypes.c_int32], ctypes.c_int),
@@ -195,6 +197,14 @@ def hla_decode_step(cfg, cache: Cache, q, k, v, alpha, beta, o, q_route=None, k_
     _check(lib().hla_decode_step(ctypes.byref(cfg), ctypes.byref(cache.struct), _ptr(q), _ptr(k), _ptr(v),
                                  _ptr(alpha), _ptr(beta), _ptr(q_route), _ptr(k_route), _ptr(o),
                                  _ptr(workspace), workspace.numel(), _stream(stream)))
+    return o
+
+
+def hla_decode_step_static(cfg, cache: Cache, q, k, v, alpha, beta, o, q_route=None, k_route=None, stream=None):
+    """hla_decode_step with the library's fixed device scratch array: allocates nothing."""
+    _check(lib().hla_decode_step_static(ctypes.byref(cfg), ctypes.byref(cache.struct), _ptr(q), _ptr(k), _ptr(v),
+                                        _ptr(alpha), _ptr(beta), _ptr(q_route), _ptr(k_route), _ptr(o),
+                                        _stream(stream)))
     return o
 
 

@@ -544,6 +544,72 @@ hla_status hla_decode_step(const hla_config* cfg, hla_cache* cache, const void* 
   return HLA_OK;
 }
 
+// ---------------------------------------------------------------------------
+// Decode step with library-owned scratch.
+//
+// hla_decode_step wants the caller to hand it a device scratch block (the
+// per-head list of active chunks and their gates).  A caller that may not
+// allocate device memory at the point where it decodes -- a plug-in inside a
+// runtime that owns every byte through its own pool and forbids allocations by
+// its extensions, or a host thread that runs decode without an allocator in
+// reach -- uses hla_decode_step_static instead.  Its scratch is the fixed array
+// below: statically sized device memory of this library, looked up once per
+// device, never allocated or freed by any call.
+//
+// Every call on a device uses the same array.  Nothing in it must start at
+// zero (each decode kernel writes every entry it later reads), but two calls
+// whose kernels overlap in time -- on different streams, or from different
+// host threads -- write the same bytes and race: the caller serialises them.
+// ---------------------------------------------------------------------------
+namespace {
+constexpr size_t kStaticScratchBytes = HLA_DECODE_STATIC_SCRATCH_BYTES;
+constexpr int kStaticMaxDevices = 64;
+std::mutex g_static_mu;
+void* g_static_ptr[kStaticMaxDevices] = {};
+}  // namespace
+
+static __device__ __align__(256) unsigned char hla_static_scratch[kStaticScratchBytes];
+
+namespace {
+// Device address of hla_static_scratch on the current device.  The first call on
+// a device asks the runtime for the symbol's address (with that device current);
+// later calls reuse it.
+hla_status static_scratch_ptr(void** out) {
+  int dev = -1;
+  HLA_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  if (dev < 0 || dev >= kStaticMaxDevices)
+    return fail(HLA_ERR_UNSUPPORTED, "device ordinal %d beyond %d", dev, kStaticMaxDevices);
+  std::lock_guard<std::mutex> lk(g_static_mu);
+  if (g_static_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, hla_static_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(hla_static_scratch)");
+    if (p == nullptr || ((uintptr_t)p & 255u) != 0)
+      return fail(HLA_ERR_CUDA, "static scratch address %p is not 256-byte aligned", p);
+    g_static_ptr[dev] = p;
+  }
+  *out = g_static_ptr[dev];
+  return HLA_OK;
+}
+}  // namespace
+
+hla_status hla_decode_step_static(const hla_config* cfg, hla_cache* cache, const void* q, const void* k,
+                                  const void* v, const float* alpha, const float* beta, const void* q_route,
+                                  const void* k_route, void* o, hla_stream_t stream) {
+  g_msg[0] = 0;
+  HLA_TRY(check_cfg(cfg, false));
+  HLA_TRY(check_cache(cfg, cache));
+  const size_t need = hla_decode_workspace_bytes(cfg, cache->max_chunks);
+  if (need > kStaticScratchBytes)
+    return fail(HLA_ERR_WORKSPACE,
+                "decode scratch for B=%d H=%d max_chunks=%d is %zu bytes; the static array holds %zu "
+                "(B*H*max_chunks <= %zu); use hla_decode_step with a caller workspace",
+                cfg->B, cfg->H, cache->max_chunks, need, kStaticScratchBytes, kStaticScratchBytes / 8);
+  void* ws = nullptr;
+  HLA_TRY(static_scratch_ptr(&ws));
+  return hla_decode_step(cfg, cache, q, k, v, alpha, beta, q_route, k_route, o, ws, kStaticScratchBytes, stream);
+}
+
 hla_status hla_profile_enable(int32_t on) {
   g_msg[0] = 0;
   std::lock_guard<std::mutex> lk(g_prof_mu);

@@ -211,6 +211,28 @@ hla_status hla_decode_step(const hla_config* cfg, hla_cache* cache, const void* 
                            hla_stream_t stream);
 
 /*
+ * hla_decode_step_static -- hla_decode_step without a caller workspace.
+ * The pages have no counterpart to this call: it exists for callers that may not
+ * allocate device memory where they decode (a plug-in inside a runtime that owns
+ * all device memory through its own pool, or a thread with no allocator in
+ * reach).  Same arguments, layouts, semantics and errors as hla_decode_step, minus
+ * the workspace: the scratch is a fixed device array inside this library,
+ * HLA_DECODE_STATIC_SCRATCH_BYTES long, enough for B*H*max_chunks <= 2^20.  A
+ * larger cache is rejected with HLA_ERR_WORKSPACE before anything is launched.
+ * No call allocates or frees device memory.
+ * Set-up: the first call on a device (the current one) looks up the array's
+ * device address and keeps it; make that first call before any stream capture.
+ * Sharing: every call on a device writes the same array.  Nothing in it has to
+ * start at zero, but calls whose kernels may overlap in time (different streams
+ * or host threads) race on it; serialise them.
+ */
+#define HLA_DECODE_STATIC_SCRATCH_BYTES ((size_t)8 << 20)
+hla_status hla_decode_step_static(const hla_config* cfg, hla_cache* cache, const void* q,
+                                  const void* k, const void* v, const float* alpha,
+                                  const float* beta, const void* q_route,
+                                  const void* k_route, void* o, hla_stream_t stream);
+
+/*
  * Bounded device waits.  Kernels that wait on an mbarrier or a flag give up after
  * a fixed number of polls, record a code in a device-side error word and return.
  * hla_device_status synchronises the device, reads and (if clear != 0) resets that

@@ -143,3 +143,19 @@ def test_python_binding_refuses_cpu_tensors(hla):
     x = torch.zeros(1, 64, 1, 64)
     with pytest.raises(ValueError, match="CUDA"):
         hla.gdn_chunk_transitions(c, x, x, x[..., 0], x[..., 0], x, x)
+
+
+def test_static_decode_rejects_scratch_beyond_its_array(hla):
+    """hla_decode_step_static has B*H*max_chunks <= 2^20 entries of fixed scratch; a
+    larger cache is refused on the host (the fake aligned pointers are never read)."""
+    c = cfg(hla, B=64, H=16, T=1)
+    cache = hla.HlaCache()
+    cache.B, cache.H, cache.C, cache.d, cache.dtype = 64, 16, 64, 128, 1
+    cache.max_chunks = (1 << 20) // (64 * 16) + 1
+    for f in ("A", "Bm", "rk", "buf_k", "buf_v", "buf_qr", "buf_kr", "buf_alpha", "buf_beta", "n_chunks",
+              "m_partial"):
+        setattr(cache, f, 256)
+    P = ctypes.c_void_p(256)
+    st = hla.lib().hla_decode_step_static(ctypes.byref(c), ctypes.byref(cache), P, P, P, P, P, None, None, P,
+                                          None)
+    assert st == hla.HLA_ERR_WORKSPACE and "static array" in hla.last_error()
