@@ -43,6 +43,58 @@ FLOP_TRANSITION = 3 * 2 * 64 * 64 * 128 + 2 * 2 * 64 * 128 * 128
 FLOP_READOUT = 2 * 2 * 64 * 128 * 128 + 2 * 2 * 64 * 64 * 128
 
 
+def rank_env():
+    """(world, rank, local_rank) from the torchrun environment (1, 0, 0 alone)."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(values, device="cpu"):
+    """Element-wise maximum of per-rank timings (one all_reduce(MAX) when a process
+    group of more than one rank is up; the values themselves otherwise)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
+def whole_job_rate(units_per_rank, ms_max, world):
+    """Weak-scaling throughput: every rank runs an independent replica of the same
+    work, so the job processes world x units in the slowest rank's time."""
+    return units_per_rank * world / (ms_max * 1e-3)
+
+
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from the ncu
+# captures summarised under profiles/, keyed by the kernel and tagged with the SHA-256
+# prefix of the kernel's source files at capture time.  A figure is reported only
+# while those sources are unchanged.
+#   compose: full-size launch of the dense 0.8B-like prefill (compose_tc_prefill_0p8b.md)
+NCU_TRAFFIC = {
+    "compose": (2.0745e9, {"compose_tc.cu": "dd565710efa80768", "tc_common.cuh": "e25172df5d8aca96"}),
+}
+
+
+def ncu_traffic(kernel):
+    """The recorded traffic of `kernel` (bytes per launch), or None if there is no
+    capture or its sources have changed since."""
+    import hashlib
+    rec = NCU_TRAFFIC.get(kernel)
+    if rec is None:
+        return None
+    nbytes, files = rec
+    for name, tag in files.items():
+        path = os.path.join(ROOT, "gated_delta_rule_transitions_b200", "csrc", name)
+        try:
+            with open(path, "rb") as f:
+                if hashlib.sha256(f.read()).hexdigest()[:16] != tag:
+                    return None
+        except OSError:
+            return None
+    return nbytes
+
+
 def _peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -53,32 +105,76 @@ def _peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    """SM clocks, power and throttle reasons sampled during the timed region.
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    Reads NVML every 5 ms from a thread (read-only queries; no setting is changed),
+    on the NVML device whose PCI bus id matches the CUDA device; falls back to
+    polling nvidia-smi when NVML is unavailable."""
 
-    def __init__(self, index: int):
-        self.index = index
-        self.samples = []
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4))
+
+    def __init__(self, cuda_index: int):
+        self.cuda_index = cuda_index
+        self.samples = []  # (sm_mhz, max_mhz, power_w, reason_bits)
+        self.source = None
         self._stop = threading.Event()
         self._t = None
 
-    def _run(self):
+    def _nvml_handle(self):
+        """NVML handle of the CUDA device: matched by UUID, else by PCI bus id."""
+        import pynvml
+        pynvml.nvmlInit()
+        p = torch.cuda.get_device_properties(self.cuda_index)
+        uuid = str(getattr(p, "uuid", "")).lower().removeprefix("gpu-")
+        bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+        for i in range(pynvml.nvmlDeviceGetCount()):
+            h = pynvml.nvmlDeviceGetHandleByIndex(i)
+            u = pynvml.nvmlDeviceGetUUID(h)
+            u = (u.decode() if isinstance(u, bytes) else u).lower().removeprefix("gpu-")
+            b = pynvml.nvmlDeviceGetPciInfo(h).busId
+            b = (b.decode() if isinstance(b, bytes) else b).lower()
+            if (uuid and u == uuid) or b.endswith(bus[-12:]):
+                return pynvml, h
+        raise RuntimeError(f"no NVML device matches uuid {uuid} / bus {bus}")
+
+    def _run_nvml(self, nv, h):
+        mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
         while not self._stop.is_set():
             try:
-                out = subprocess.run(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((float(sm), float(mx), pw, int(rs)))
+            except Exception:
+                pass
+            self._stop.wait(0.005)
+
+    def _run_smi(self):
+        fields = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+                  "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_power_cap")
+        while not self._stop.is_set():
+            try:
+                out = subprocess.run(["nvidia-smi", "-i", str(self.cuda_index), f"--query-gpu={fields}",
                                       "--format=csv,noheader,nounits"], capture_output=True, text=True,
-                                     timeout=5).stdout.strip()
-                if out:
-                    self.samples.append([x.strip() for x in out.split(",")])
+                                     timeout=5).stdout.strip().split(",")
+                bits = 0
+                for (_, bit), flag in zip(self.REASONS, out[3:7]):
+                    bits |= bit if flag.strip() == "Active" else 0
+                self.samples.append((float(out[0]), float(out[1]), float(out[2]), bits))
             except Exception:
                 pass
             self._stop.wait(0.2)
 
     def __enter__(self):
-        self._t = threading.Thread(target=self._run, daemon=True)
+        try:
+            nv, h = self._nvml_handle()
+            self.source = "nvml"
+            self._t = threading.Thread(target=self._run_nvml, args=(nv, h), daemon=True)
+        except Exception as e:
+            self.source = f"nvidia-smi (nvml: {type(e).__name__}: {str(e)[:80]})"
+            self._t = threading.Thread(target=self._run_smi, daemon=True)
         self._t.start()
         return self
 
@@ -88,13 +184,12 @@ class ClockSampler:
 
     def summary(self):
         if not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        sm = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
-        mx = [float(s[2]) for s in self.samples if s[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for s in self.samples for i in range(4) if len(s) > 5 + i and s[5 + i] == "Active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(self.samples)}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        reasons = sorted({name for *_, bits in self.samples for name, bit in self.REASONS if bits & bit})
+        return {"sm_mhz": statistics.median(s[0] for s in self.samples),
+                "sm_max_mhz": max(s[1] for s in self.samples),
+                "power_w_max": round(max(s[2] for s in self.samples), 1),
+                "reasons": reasons, "samples": len(self.samples), "source": self.source}
 
 
 # ----------------------------------------------------------------------------------
@@ -146,9 +241,7 @@ def run_ours(args):
     import hla_synth as syn
 
     hla = pkg._hla
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_env()
     torch.cuda.set_device(local)
     if world > 1:
         import datetime
@@ -250,10 +343,7 @@ def run_ours(args):
     stages = hla.hla_profile_read(reset=True)
     pre_ms = sum(ev[2 * s][0].elapsed_time(ev[2 * s][1]) for s in range(args.steps)) / args.steps
     dec_ms = sum(ev[2 * s + 1][0].elapsed_time(ev[2 * s + 1][1]) for s in range(args.steps)) / args.steps
-    t = torch.tensor([pre_ms, dec_ms], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    pre_ms, dec_ms = float(t[0]), float(t[1])
+    pre_ms, dec_ms = max_over_ranks([pre_ms, dec_ms], device="cuda")
 
     # ---- end to end through the public API with host buffers ----
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(2)]
@@ -278,10 +368,7 @@ def run_ours(args):
         torch.cuda.synchronize()
         e2e_pre += e2e_ev[0][0].elapsed_time(e2e_ev[0][1]) / reps
         e2e_dec += e2e_ev[1][0].elapsed_time(e2e_ev[1][1]) / reps
-    t = torch.tensor([e2e_pre, e2e_dec], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    e2e_pre, e2e_dec = float(t[0]), float(t[1])
+    e2e_pre, e2e_dec = max_over_ranks([e2e_pre, e2e_dec], device="cuda")
     h2d_pre = sum(v.numel() * v.element_size() for v in host.values())
     d2h_pre = o.numel() * o.element_size()
     h2d_dec = sum(v.numel() * v.element_size() for v in toks_host[0].values())
@@ -300,11 +387,11 @@ def run_ours(args):
     dec_gbs = bytes_decode / (dmain_avg * 1e-3) / 1e9 if dmain_avg > 0 else None
     launches = sum(n for (_, n) in stages.values())
 
-    tokens_pre = wp.B * wp.T * world
-    tokens_dec = wd.B * world
+    tokens_pre = wp.B * wp.T
+    tokens_dec = wd.B
     out = {
         "metric": METRIC,
-        "value": tokens_pre / (pre_ms * 1e-3),
+        "value": whole_job_rate(tokens_pre, pre_ms, world),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -319,21 +406,23 @@ def run_ours(args):
                    "active_pairs": active_pairs, "parallelism": f"replicas x{world} (no data-path collective)",
                    "l2": "flushed before every timed phase (256 MiB write, untimed)"},
         "roofline": {"kernel": "compose", "bound": "tensor", "achieved": comp_tf, "peak": bf16_tf,
-                     "unit": "TFLOP/s", "frac": (comp_tf / bf16_tf) if comp_tf else None, "traffic": None,
+                     "unit": "TFLOP/s", "frac": (comp_tf / bf16_tf) if comp_tf else None,
+                     "traffic": ncu_traffic("compose"), "traffic_unit": "bytes per launch (ncu dram read+write)",
                      "peak_source": f"{peak_src} bf16 dense (burst)",
                      "algorithmic": f"{active_pairs} active pairs x 2 d^3 = {flops_compose:.4g} flop per launch",
                      "prefill_frac_of_peak": (flops_compose + N * wp.H * (FLOP_TRANSITION + FLOP_READOUT))
                      / (pre_ms * 1e-3) / 1e12 / bf16_tf},
-        "decode": {"value": tokens_dec / (dec_ms * 1e-3), "unit": "tokens/s", "ms_per_step": dec_ms,
+        "decode": {"value": whole_job_rate(tokens_dec, dec_ms, world), "unit": "tokens/s", "ms_per_step": dec_ms,
                    "roofline": {"kernel": "decode_main", "bound": "hbm", "achieved": dec_gbs, "peak": hbm_gbs,
                                 "unit": "GB/s", "frac": (dec_gbs / hbm_gbs) if dec_gbs else None,
-                                "traffic": None, "peak_source": f"{peak_src} HBM copy",
+                                "traffic": ncu_traffic("decode_main"), "traffic_unit": "bytes per launch (ncu dram read+write)",
+                                "peak_source": f"{peak_src} HBM copy",
                                 "algorithmic": f"{bytes_decode:.4g} bytes per launch (512 active A_j/B_j bf16 + "
                                                "key pools per sequence and head)"},
-                   "e2e": {"value": tokens_dec / (e2e_dec * 1e-3), "unit": "tokens/s",
+                   "e2e": {"value": whole_job_rate(tokens_dec, e2e_dec, world), "unit": "tokens/s",
                            "h2d_bytes_per_step": h2d_dec, "d2h_bytes_per_step": d2h_dec}},
         "stages_ms_per_step": {k: v[0] / args.steps for k, v in stages.items() if v[1]},
-        "e2e": {"value": tokens_pre / (e2e_pre * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d_pre,
+        "e2e": {"value": whole_job_rate(tokens_pre, e2e_pre, world), "unit": "tokens/s", "h2d_bytes_per_step": h2d_pre,
                 "d2h_bytes_per_step": d2h_pre},
         "gpu_launches": launches,
         "clocks": clocks.summary(),
@@ -404,8 +493,7 @@ def cpu_baseline(inp, wp, wd, ctx0, toks_host, torch):
 def run_reference(args):
     """The oracle as it stands, on the host cores, on bounded samples of the same
     workloads; rank 0 only."""
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
+    world, rank, _ = rank_env()
     if rank != 0:
         return
     import torch
