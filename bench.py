@@ -43,6 +43,13 @@ FLOP_TRANSITION = 3 * 2 * 64 * 64 * 128 + 2 * 2 * 64 * 128 * 128
 FLOP_READOUT = 2 * 2 * 64 * 128 * 128 + 2 * 2 * 64 * 64 * 128
 
 
+PREFILL_WORKLOADS = {
+    "dense": lambda syn: syn.PREFILL_0P8B,
+    "sparse": lambda syn: syn.SPARSE_LONG,
+    "gdn": lambda syn: syn.GDN_REDUCTION,
+}
+
+
 def rank_env():
     """(world, rank, local_rank) from the torchrun environment (1, 0, 0 alone)."""
     return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
@@ -124,6 +131,7 @@ class ClockSampler:
     def _nvml_handle(self):
         """NVML handle of the CUDA device: matched by UUID, else by PCI bus id."""
         import pynvml
+        import torch
         pynvml.nvmlInit()
         p = torch.cuda.get_device_properties(self.cuda_index)
         uuid = str(getattr(p, "uuid", "")).lower().removeprefix("gpu-")
@@ -250,14 +258,19 @@ def run_ours(args):
     stream = torch.cuda.current_stream()
 
     # ---- prefill workload (inputs resident in HBM) ----
-    wp = syn.PREFILL_0P8B
+    wp = PREFILL_WORKLOADS[args.prefill_workload](syn)
     if args.prefill_T:
-        wp = wp.with_(T=args.prefill_T, name=wp.name.replace("T16384", f"T{args.prefill_T}"))
-    inp = syn.make_gdn_inputs(wp)
-    qr, kr = syn.make_route_inputs(wp)
+        wp = wp.with_(T=args.prefill_T, name=f"{wp.name}_T{args.prefill_T}")
+    # the long sparse workload is generated on the device (5 x 1 GiB of inputs)
+    gen_dev = "cuda" if wp.B * wp.T * wp.H * wp.d > (1 << 28) else "cpu"
+    inp = syn.make_gdn_inputs(wp, device=gen_dev)
+    qr, kr = syn.make_route_inputs(wp, device=gen_dev)
     inp["q_route"], inp["k_route"] = qr, kr
-    host = {k: v.contiguous().pin_memory() for k, v in inp.items()}
+    inp = {k: v for k, v in inp.items() if v is not None}
+    host = {k: v.contiguous().cpu().pin_memory() for k, v in inp.items()}
     dev = {k: v.cuda() for k, v in host.items()}
+    del inp
+    inp = host
     pcfg = hla.make_config(wp.B, wp.H, wp.T, wp.C, wp.d, wp.dtype, wp.gate_mode, wp.tau, wp.bias, wp.thr)
     pws = torch.empty(hla.prefill_workspace_bytes(pcfg), dtype=torch.uint8, device="cuda")
     o = torch.empty_like(dev["q"])
@@ -267,7 +280,7 @@ def run_ours(args):
 
     def prefill():
         hla.hla_prefill(pcfg, dev["q"], dev["k"], dev["v"], dev["alpha"], dev["beta"], o,
-                        q_route=dev["q_route"], k_route=dev["k_route"], workspace=pws)
+                        q_route=dev.get("q_route"), k_route=dev.get("k_route"), workspace=pws)
 
     # ---- decode workload ----
     wd = syn.DECODE_32K
@@ -311,7 +324,7 @@ def run_ours(args):
 
     # active pairs of the prefill (for the algorithmic flop count)
     hla.hla_prefill(pcfg, dev["q"], dev["k"], dev["v"], dev["alpha"], dev["beta"], o,
-                    q_route=dev["q_route"], k_route=dev["k_route"], workspace=pws, active_cnt_out=acnt,
+                    q_route=dev.get("q_route"), k_route=dev.get("k_route"), workspace=pws, active_cnt_out=acnt,
                     active_idx_out=torch.empty((wp.B, wp.H, N, N), dtype=torch.int32, device="cuda"))
     torch.cuda.synchronize()
     active_pairs = int(acnt.sum().item())
@@ -376,7 +389,14 @@ def run_ours(args):
 
     # ---- roofline of the dominant kernels ----
     d = wp.d
-    flops_compose = active_pairs * 2.0 * d ** 3
+    if wp.gate_mode == "one":
+        # every gate one: the library composes by a prefix scan, N-1 steps per head
+        comp_units = wp.B * wp.H * max(N - 1, 0)
+        comp_what = f"{comp_units} scan steps (gates all one)"
+    else:
+        comp_units = active_pairs
+        comp_what = f"{active_pairs} active pairs"
+    flops_compose = comp_units * 2.0 * d ** 3
     comp_ms, comp_n = stages["compose"]
     comp_avg = comp_ms / max(comp_n, 1)
     comp_tf = flops_compose / (comp_avg * 1e-3) / 1e12 if comp_avg > 0 else None
@@ -409,8 +429,8 @@ def run_ours(args):
                      "unit": "TFLOP/s", "frac": (comp_tf / bf16_tf) if comp_tf else None,
                      "traffic": ncu_traffic("compose"), "traffic_unit": "bytes per launch (ncu dram read+write)",
                      "peak_source": f"{peak_src} bf16 dense (burst)",
-                     "algorithmic": f"{active_pairs} active pairs x 2 d^3 = {flops_compose:.4g} flop per launch",
-                     "prefill_frac_of_peak": (flops_compose + N * wp.H * (FLOP_TRANSITION + FLOP_READOUT))
+                     "algorithmic": f"{comp_what} x 2 d^3 = {flops_compose:.4g} flop per launch",
+                     "prefill_frac_of_peak": (flops_compose + N * wp.B * wp.H * (FLOP_TRANSITION + FLOP_READOUT))
                      / (pre_ms * 1e-3) / 1e12 / bf16_tf},
         "decode": {"value": whole_job_rate(tokens_dec, dec_ms, world), "unit": "tokens/s", "ms_per_step": dec_ms,
                    "roofline": {"kernel": "decode_main", "bound": "hbm", "achieved": dec_gbs, "peak": hbm_gbs,
@@ -538,7 +558,10 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     # smaller variants for profiling captures (the default is the full workload)
-    ap.add_argument("--prefill-T", type=int, default=None, help="prefill tokens (default 16384)")
+    ap.add_argument("--prefill-T", type=int, default=None, help="prefill tokens (default: the workload's)")
+    ap.add_argument("--prefill-workload", choices=sorted(PREFILL_WORKLOADS), default="dense",
+                    help="dense: the 0.8B-like layer (the metric's workload); sparse: B=1, H=32, T=131072 "
+                         "with planted gates; gdn: B=4, H=16, T=4096 with all gates one")
     ap.add_argument("--decode-B", type=int, default=None, help="decode sequences (default 64)")
     ap.add_argument("--decode-ctx", type=int, default=None, help="decode context tokens (default 32768)")
     ap.add_argument("--skip-decode", action="store_true")

@@ -53,6 +53,8 @@ def _compile(src: str, force: bool, extra: list[str]) -> str:
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"nvcc failed for {src}:\n{r.stdout}\n{r.stderr}")
+    if extra and r.stderr:
+        print(f"== {os.path.basename(src)}\n{r.stderr}", end="", flush=True)
     return obj
 
 

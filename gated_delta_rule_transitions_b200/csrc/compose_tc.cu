@@ -20,6 +20,10 @@
 // column half = ((warp - 2) % 8) / 4), so each chain's epilogue overlaps the other
 // chain's MMA.  Elementwise math uses packed float32 pairs.  All waits are bounded
 // (about 2 s, then a device error word is set and the CTA exits cleanly).
+//
+// Scan mode (every gate one, the native-GDN reduction): S_in(j+1) = S_in(j) A_j + B_j,
+// so one chain per head walks j = 0 .. N-2 once and stores every intermediate state;
+// the work is N-1 steps per head instead of N(N-1)/2.
 #include "common.cuh"
 #include "kernels.cuh"
 #include "tc_common.cuh"
@@ -105,6 +109,7 @@ struct StepInfo {
   float gn[2]; // gates at each chain's next active step (0 if none)
 };
 
+template <bool kScan>
 __global__ void __launch_bounds__(kThreads, 1)
     compose_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       ComposeTcArgs a) {
@@ -123,9 +128,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int pair = blockIdx.x / a.BH;
+  const int pair = kScan ? 0 : blockIdx.x / a.BH;
   const int bh = blockIdx.x % a.BH;
-  const int chains[2] = {a.N - 1 - 2 * pair, a.N - 2 - 2 * pair};
+  // scan mode: chain 0 is the head's running state (its S_in rows move with j), chain 1 idles
+  const int chains[2] = {kScan ? 0 : a.N - 1 - 2 * pair, kScan ? -1 : a.N - 2 - 2 * pair};
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -155,25 +161,37 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- TMA producer (lane 0): walks the merged lists ----------------
     if (lane == 0) {
       Sched sc;
-      sc.init(a, bh, chains);
+      if (!kScan) sc.init(a, bh, chains);
       int s = 0;
       bool ok = true;
-      while (sc.next()) {
+      while (kScan ? s < a.N - 1 : sc.next()) {
         const int st = s % kStages;
         if (s >= kStages && !tc::mbar_wait(&empty[st], ((s / kStages) - 1) & 1, abort_s)) {
           ok = false;
           break;
         }
         StepInfo e;
-        e.j = sc.j;
-        e.flags = 0;
-        for (int k = 0; k < 2; ++k) {
-          e.flags |= (sc.act[k] ? 1 : 0) << k;
-          e.flags |= (sc.first[k] ? 1 : 0) << (2 + k);
-          e.flags |= (sc.last[k] ? 1 : 0) << (4 + k);
-          e.p[k] = sc.p[k];
-          e.g[k] = sc.gate[k];
-          e.gn[k] = sc.gnext[k];
+        if (kScan) {
+          sc.j = s;
+          e.j = s;
+          e.flags = 1 | ((s == 0) ? 4 : 0) | ((s == a.N - 2) ? 16 : 0);
+          e.p[0] = s;
+          e.p[1] = 0;
+          e.g[0] = 1.0f;
+          e.g[1] = 0.0f;
+          e.gn[0] = (s == a.N - 2) ? 0.0f : 1.0f;
+          e.gn[1] = 0.0f;
+        } else {
+          e.j = sc.j;
+          e.flags = 0;
+          for (int k = 0; k < 2; ++k) {
+            e.flags |= (sc.act[k] ? 1 : 0) << k;
+            e.flags |= (sc.first[k] ? 1 : 0) << (2 + k);
+            e.flags |= (sc.last[k] ? 1 : 0) << (4 + k);
+            e.p[k] = sc.p[k];
+            e.g[k] = sc.gate[k];
+            e.gn[k] = sc.gnext[k];
+          }
         }
         info[st] = e;
         tc::mbar_arrive_expect_tx(&full[st], kStageBytes);  // releases info[st]
@@ -183,7 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::tma_load_2d(dst + kHalfBytes, &tmA, 64, row, &full[st]);
         tc::tma_load_2d(dst + 2 * kHalfBytes, &tmB, 0, row, &full[st]);
         tc::tma_load_2d(dst + 3 * kHalfBytes, &tmB, 64, row, &full[st]);
-        sc.advance();
+        if (!kScan) sc.advance();
         ++s;
       }
       if (ok) {
@@ -224,7 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int ks = 0; ks < kD / 16; ++ks) {
             const uint64_t bd = tc::sdesc_sw128(b_base + ks * 2048, kHalfBytes, 1024);
-            tc::mma_ts(d_t, a_t + 8u * ks, bd, kIdesc, 1u);
+            tc::mma_ts(d_t, a_t + 8u * ks, bd, kIdesc, (kScan && ks == 0) ? 0u : 1u);
           }
           tc::mma_commit(&mma_done[k]);
         }
@@ -248,8 +266,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int chain = k ? chains[1] : chains[0];
     __nv_bfloat16* out_row =
         chain >= 0 ? a.S_in + ((long)bh * a.N + chain) * kD * kD + (long)v * kD + col0 : nullptr;
-    // a chain with nothing active has S_in = 0
-    if (chain >= 0 && a.act_cnt[(long)bh * a.N + chain] == 0)
+    // a chain with nothing active has S_in = 0 (in scan mode: S_in(0))
+    if (chain >= 0 && (kScan || a.act_cnt[(long)bh * a.N + chain] == 0))
       for (int e = 0; e < 8; ++e) ((uint4*)out_row)[e] = make_uint4(0u, 0u, 0u, 0u);
     for (int s = 0;; ++s) {
       const int st = s % kStages;
@@ -298,14 +316,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 16; ++i)
             x[i] = tc::fma2(g2, tc::bf16x2_to_float2(bw[cc / 2 + i]),
                             make_float2(__uint_as_float(d[2 * i]), __uint_as_float(d[2 * i + 1])));
-          if (last) {
-            uint4* out = (uint4*)(out_row + cc);
+          if (kScan || last) {
+            // scan mode: this step's state is S_in(j + 1)
+            uint4* out = (uint4*)(out_row + (kScan ? (long)(e.j + 1) * kD * kD : 0) + cc);
 #pragma unroll
             for (int i = 0; i < 4; ++i)
               out[i] = make_uint4(tc::pack_bf16x2(x[4 * i].x, x[4 * i].y), tc::pack_bf16x2(x[4 * i + 1].x, x[4 * i + 1].y),
                                   tc::pack_bf16x2(x[4 * i + 2].x, x[4 * i + 2].y),
                                   tc::pack_bf16x2(x[4 * i + 3].x, x[4 * i + 3].y));
-          } else {
+          }
+          if (kScan && !last) {
+            // next operand bf16(S); the next product starts from zero, no state store
+            uint32_t op[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) op[i] = tc::pack_bf16x2(x[i].x, x[i].y);
+            tc::tmem_st16(tbase + lane_off + 256u + 64u * k + (col0 + cc) / 2, op);
+          } else if (!kScan && !last) {
             const float2 gn2 = make_float2(gn, gn), keep2 = make_float2(keep, keep);
             uint32_t op[16];
 #pragma unroll
@@ -384,7 +410,7 @@ cudaError_t make_tmap_rows128(CUtensorMap* m, const void* base, long rows) {
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-cudaError_t launch_compose_tc(const ComposeArgs& c, cudaStream_t s) {
+cudaError_t launch_compose_tc(const ComposeArgs& c, bool scan, cudaStream_t s) {
   if (c.N <= 0) return cudaSuccess;
   if (c.ab_chunk_stride <= 0)  // no complete chunk: every composed state is zero
     return cudaMemsetAsync(c.S_in, 0, (size_t)c.B * c.H * c.N * kD * kD * sizeof(__nv_bfloat16), s);
@@ -403,10 +429,16 @@ cudaError_t launch_compose_tc(const ComposeArgs& c, cudaStream_t s) {
   a.act_cnt = c.act_cnt;
   a.S_in = (__nv_bfloat16*)c.S_in;
   const size_t smem = 1024 + kStages * kStageBytes + 512;
-  e = cudaFuncSetAttribute(compose_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (scan) {
+    e = cudaFuncSetAttribute(compose_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    compose_tc_kernel<true><<<a.BH, kThreads, smem, s>>>(tmA, tmB, a);
+    return cudaGetLastError();
+  }
+  e = cudaFuncSetAttribute(compose_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int pairs = (c.N + 1) / 2;
-  compose_tc_kernel<<<pairs * a.BH, kThreads, smem, s>>>(tmA, tmB, a);
+  compose_tc_kernel<false><<<pairs * a.BH, kThreads, smem, s>>>(tmA, tmB, a);
   return cudaGetLastError();
 }
 

@@ -429,8 +429,10 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
   c.S_in = (float*)(ws + w.S_in);
   {
     StageScope _sc(HLA_STAGE_COMPOSE, s, 1);
+    // every gate one (and kept): the composition is a plain prefix scan over the chunks
+    const bool scan = cfg->gate_mode == HLA_GATES_ONE && cfg->skip_threshold <= 1.0f;
     if (tc_path)
-      HLA_CUDA(hla::launch_compose_tc(c, s), "compose (tensor core) launch");
+      HLA_CUDA(hla::launch_compose_tc(c, scan, s), "compose (tensor core) launch");
     else
       HLA_CUDA(hla::launch_compose(c, s), "compose launch");
   }

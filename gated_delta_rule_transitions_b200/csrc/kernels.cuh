@@ -111,7 +111,7 @@ cudaError_t launch_cache_fill(const DecodeArgs& c, const float* rk_ws, const voi
                               cudaStream_t s);
 cudaError_t read_error_word_decode(unsigned int* out, bool clear);
 cudaError_t read_error_word_compose_tc(unsigned int* out, bool clear);
-cudaError_t launch_compose_tc(const ComposeArgs& a, cudaStream_t s);
+cudaError_t launch_compose_tc(const ComposeArgs& a, bool scan, cudaStream_t s);
 cudaError_t launch_decode_stream(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_transitions_tc(const TransArgs& t, cudaStream_t s);
 cudaError_t launch_readout_tc(const ReadoutArgs& r, const void* S_in_bf16, const void* Wb_bf16, const void* Ub_bf16,

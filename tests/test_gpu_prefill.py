@@ -201,3 +201,37 @@ def test_full_size_prefill_sampled(hla):
         P.check_routing_exact(r, gates, aidx, acnt, 0, h)
         rows = np.concatenate([np.arange(64 * i, 64 * i + 64) for i in sample])
         assert P.rel_l2(P.np64(o[0, rows, h]), r.o[rows]) <= P.TOL_BF16_RELL2
+
+
+def test_full_size_gdn_reduction_sampled(hla):
+    """Native-GDN reduction at full size (B=4, H=16, T=4096, d=128, bf16, all gates
+    one): whole sequences of two (b, h) pairs against the sequential gated delta rule."""
+    w = syn.GDN_REDUCTION
+    inp = P.gpu_inputs(w)
+    o, gates, aidx, acnt = P.run_prefill(hla, w, inp)
+    assert torch.all(acnt[:, :, 1:] > 0)
+    for (b, h) in ((0, 0), (3, 11)):
+        ref, _ = ho.gdn_recurrent(P.np64(inp["q"][b, :, h]), P.np64(inp["k"][b, :, h]),
+                                  P.np64(inp["v"][b, :, h]), P.np64(inp["alpha"][b, :, h]),
+                                  P.np64(inp["beta"][b, :, h]))
+        assert P.rel_l2(P.np64(o[b, :, h]), ref) <= P.TOL_BF16_RELL2
+
+
+def test_full_size_sparse_prefill_sampled(hla):
+    """Long sparse prefill at full size (B=1, H=32, T=131072, 2048 chunks, bf16,
+    planted route inputs, threshold 0.05).  Inputs are generated on the device (the
+    oracle reads the sampled heads back); gates and active lists bit-exact on two
+    heads, sampled query chunks against the oracle, and the planted sparsity
+    (about 8 active earlier chunks per query chunk on average) is checked."""
+    w = syn.SPARSE_LONG
+    inp = syn.make_gdn_inputs(w, device="cuda")
+    inp["q_route"], inp["k_route"] = syn.make_route_inputs(w, device="cuda")
+    o, gates, aidx, acnt = P.run_prefill(hla, w, inp)
+    mean_active = float(acnt.double().mean())
+    assert 4.0 <= mean_active <= 12.0, mean_active
+    for h in (0, 21):
+        sample = [0, 1, 700, 1500, 2047]
+        r = P.oracle_prefill_head(w, inp, 0, h, query_chunks=sample)
+        P.check_routing_exact(r, gates, aidx, acnt, 0, h)
+        rows = np.concatenate([np.arange(64 * i, 64 * i + 64) for i in sample])
+        assert P.rel_l2(P.np64(o[0, rows, h]), r.o[rows]) <= P.TOL_BF16_RELL2
