@@ -149,13 +149,7 @@ class ClockSampler:
     def _run_nvml(self, nv, h):
         mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
         while not self._stop.is_set():
-            try:
-                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
-                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
-                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
-                self.samples.append((float(sm), float(mx), pw, int(rs)))
-            except Exception:
-                pass
+            self._sample_nvml(nv, h, mx)
             self._stop.wait(0.005)
 
     def _run_smi(self):
@@ -175,10 +169,20 @@ class ClockSampler:
                 pass
             self._stop.wait(0.2)
 
+    def _sample_nvml(self, nv, h, mx):
+        try:
+            sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+            pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+            rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+            self.samples.append((float(sm), float(mx), pw, int(rs)))
+        except Exception:
+            pass
+
     def __enter__(self):
         try:
             nv, h = self._nvml_handle()
             self.source = "nvml"
+            self._nv = (nv, h, nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
             self._t = threading.Thread(target=self._run_nvml, args=(nv, h), daemon=True)
         except Exception as e:
             self.source = f"nvidia-smi (nvml: {type(e).__name__}: {str(e)[:80]})"
@@ -187,12 +191,15 @@ class ClockSampler:
         return self
 
     def __exit__(self, *a):
+        if getattr(self, "_nv", None) is not None:
+            self._sample_nvml(*self._nv)   # at least one sample inside the region
         self._stop.set()
         self._t.join(timeout=10)
 
     def summary(self):
         if not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0,
+                    "source": self.source}
         reasons = sorted({name for *_, bits in self.samples for name, bit in self.REASONS if bits & bit})
         return {"sm_mhz": statistics.median(s[0] for s in self.samples),
                 "sm_max_mhz": max(s[1] for s in self.samples),

@@ -43,6 +43,7 @@ constexpr uint32_t kIdesc = tc::idesc_bf16_f32(128, 128, /*a_mn=*/0, /*b_mn=*/1)
 
 struct ComposeTcArgs {
   int BH, N;
+  int head_major;
   long ab_chunk_stride;
   const int32_t* act_idx;
   const float* act_g;
@@ -128,8 +129,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int pair = kScan ? 0 : blockIdx.x / a.BH;
-  const int bh = blockIdx.x % a.BH;
+  // Grid order.  Head-major (with skipping: short chains whose time is the A_j/B_j
+  // reads): the CTAs resident at one time share one head's A_j/B_j through L2.
+  // Interleaved heads (dense: long chains): the longest chains of every head go first.
+  const int npairs = (a.N + 1) / 2;
+  const int pair = kScan ? 0 : (a.head_major ? blockIdx.x % npairs : blockIdx.x / a.BH);
+  const int bh = kScan ? blockIdx.x : (a.head_major ? blockIdx.x / npairs : blockIdx.x % a.BH);
   // scan mode: chain 0 is the head's running state (its S_in rows move with j), chain 1 idles
   const int chains[2] = {kScan ? 0 : a.N - 1 - 2 * pair, kScan ? -1 : a.N - 2 - 2 * pair};
 
@@ -428,6 +433,7 @@ cudaError_t launch_compose_tc(const ComposeArgs& c, bool scan, cudaStream_t s) {
   a.act_g = c.act_g;
   a.act_cnt = c.act_cnt;
   a.S_in = (__nv_bfloat16*)c.S_in;
+  a.head_major = c.sparse ? 1 : 0;
   const size_t smem = 1024 + kStages * kStageBytes + 512;
   if (scan) {
     e = cudaFuncSetAttribute(compose_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -427,6 +427,7 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
   c.act_g = act_g;
   c.act_cnt = act_cnt;
   c.S_in = (float*)(ws + w.S_in);
+  c.sparse = cfg->skip_threshold > 0.0f;
   {
     StageScope _sc(HLA_STAGE_COMPOSE, s, 1);
     // every gate one (and kept): the composition is a plain prefix scan over the chunks

@@ -57,6 +57,7 @@ struct ComposeArgs {
   const float* act_g;
   const int32_t* act_cnt; // [B,H,N]
   float* S_in;            // [B,H,N,d,d] fp32
+  bool sparse;            // chunks may be skipped (threshold > 0)
 };
 
 struct ReadoutArgs {

@@ -1,6 +1,6 @@
 // Chunk transitions on tcgen05 tensor cores: bf16 operands, float32 accumulation and
-// float32 triangular solve.  d = 128, C = 64.  One CTA (4 warps) per chunk, two
-// CTAs per SM.
+// a float32 triangular inverse.  d = 128, C = 64.  Persistent CTAs of 4 warps, two per
+// SM, each walking chunks with a grid-wide stride.
 //
 // HLA summary page, "Methodology in Plain English" para. 1 (a chunk is summarised
 // exactly by one affine map S -> S A_c + B_c); chunkwise WY/UT form (the chunkwise WY
@@ -9,15 +9,19 @@
 //   L   = strictly-lower(diag(beta) (Gamma o K K^T)),  T = (I + L)^{-1} diag(beta)
 //   Wb  = T diag(gamma) K,  Ub = T V,  D = diag(gamma_C / gamma_t)
 //   A_c = gamma_C I - Wb^T D K,  B_c = Ub^T D K.
-// MMAs (M is always 128 by stacking):
+// Per chunk (M is always 128 by stacking):
+//   TMA   K, V tiles (bf16, 128-byte swizzle)
 //   MMA1  [K; V] (128 x 128) x K^T                  -> rows 0-63: K K^T   (64 cols)
-//   SIMT  L and the forward substitution for T (float32, shared memory)
+//   SIMT  L; U = (I + L)^{-1} by 16 x 16 blocks: forward substitution on the four
+//         diagonal blocks, then the off-diagonal blocks level by level,
+//         U_ij = -U_ii sum_{k=j}^{i-1} L_ik U_kj (float32, all 128 threads)
 //   MMA2  [T diag(gamma); T] (128 x 64) x [K | V]   -> rows 0-63: Wb, rows 64-127: Ub
 //   MMA3  Wb^T (128 x 64) x D K (64 x 128)          -> A_c (after gamma_C I - .)
 //   MMA4  Ub^T (128 x 64) x D K                     -> B_c
-// Wb, Ub (bf16) and l (float32) are also written for the read-out.  A final partial
-// chunk (n < C tokens) behaves as if padded with identity tokens (alpha = 1,
-// beta = 0): its extra rows of T, Wb and Ub are zero; its A/B are not written.
+// Wb, Ub (bf16) and l (float32) are also written for the read-out.  All tile outputs
+// leave through TMA stores from swizzled shared memory.  A final partial chunk
+// (n < C tokens) behaves as if padded with identity tokens (alpha = 1, beta = 0):
+// its extra rows of T, Wb and Ub are zero; its A/B are not written.
 #include "common.cuh"
 #include "kernels.cuh"
 #include "tc_common.cuh"
@@ -33,53 +37,96 @@ namespace {
 
 constexpr int kD = 128;
 constexpr int kC = 64;
-constexpr int kKV = 0;             // [kh][K | V][64 rows][128 B]   32 KiB
-constexpr int kTT = 32768;         // [T gamma; T] 128 rows x 128 B 16 KiB; later D K
-constexpr int kScr = 49152;        // L, T float32 [64][65] each; later Wb^T, Ub^T operands
-constexpr int kLP = kC + 4;  // row pitch of the float32 L and T (16-byte rows)
-constexpr int kSmemUsed = kScr + 2 * kC * kLP * 4;
+constexpr int kKV = 0;                        // [kh][K | V][64 rows][128 B] 32 KiB
+constexpr int kTT = 32768;                    // [T gamma; T] 16 KiB; then D K; then B staging (cols 0-63)
+constexpr int kScr = 49152;                   // L, U float32; then Wb/Ub operands; then A staging
+constexpr int kLP = kC + 4;                   // row pitch (floats) of L and U: 16-byte rows
+constexpr int kLU = kC * kLP * 4;             // bytes of one of L, U
+constexpr int kX = kScr + 2 * kLU;            // 16 KiB: L' (rows 16-63); then B staging (cols 64-127)
+constexpr int kXP = 52;                       // row pitch (floats) of L'
+constexpr int kSmall = kX + 16384;            // per-token scalars, barriers
+constexpr int kSmemUsed = kSmall + 4 * kC * 4 + 4 * 8 + 32;
+static_assert(kX % 1024 == 0 && 48 * kXP * 4 <= 16384, "shared-memory layout");
 constexpr uint32_t kIdesc1 = tc::idesc_bf16_f32(128, 64, 0, 0);
 constexpr uint32_t kIdesc2 = tc::idesc_bf16_f32(128, 256, 0, 1);
 constexpr uint32_t kIdesc3 = tc::idesc_bf16_f32(128, 128, 1, 1);
 
 struct TransTcArgs {
   int B, H, T, N;
+  long total;                       // B * H * N chunks
   long sb_a, sh_a, st_a;            // alpha/beta strides
   const float* alpha;
   const float* beta;
-  __nv_bfloat16* A;                 // [.., chunk_stride, d, d] or null
-  __nv_bfloat16* Bm;
+  bool has_ab;                      // A/B are written (complete chunks)
   long ab_chunk_stride;
-  __nv_bfloat16* Wb;                // [B,H,N,C,d] or null
-  __nv_bfloat16* Ub;
+  bool has_wu;                      // Wb/Ub are written
   float* ell;                       // [B,H,N,C] or null
 };
 
 __device__ __forceinline__ int swz(int row, int chunk) { return row * 128 + ((chunk ^ (row & 7)) << 4); }
 
+struct ChunkPos {
+  int i, b, h, t0, n;
+  long bh;
+};
+
+__device__ __forceinline__ ChunkPos chunk_pos(const TransTcArgs& a, long chunk) {
+  ChunkPos p;
+  p.i = (int)(chunk % a.N);
+  p.bh = chunk / a.N;
+  p.b = (int)(p.bh / a.H);
+  p.h = (int)(p.bh % a.H);
+  p.t0 = p.i * kC;
+  p.n = min(kC, a.T - p.t0);
+  return p;
+}
+
+__device__ __forceinline__ void load_kv(uint8_t* sm, const CUtensorMap* tmK, const CUtensorMap* tmV,
+                                        uint64_t* bar, const TransTcArgs& a, const ChunkPos& p) {
+  tc::mbar_arrive_expect_tx(bar, 4 * 8192);
+  const int y = p.b * a.T + p.t0;
+  for (int kh = 0; kh < 2; ++kh) {
+    tc::tma_load_2d(sm + kKV + kh * 16384, tmK, p.h * kD + 64 * kh, y, bar);
+    tc::tma_load_2d(sm + kKV + kh * 16384 + 8192, tmV, p.h * kD + 64 * kh, y, bar);
+  }
+}
+
+// alpha, beta of token `tid` of a chunk (identity token beyond n)
+__device__ __forceinline__ void load_ab(const TransTcArgs& a, const ChunkPos& p, int tid, float& al, float& be) {
+  if (tid < p.n) {
+    const long off = p.b * a.sb_a + p.h * a.sh_a + (long)(p.t0 + tid) * a.st_a;
+    al = a.alpha[off];
+    be = a.beta[off];
+  } else {
+    al = 1.0f;
+    be = 0.0f;
+  }
+}
+
+// Persistent: each CTA walks chunks blockIdx.x, blockIdx.x + gridDim.x, ...; the next
+// chunk's K/V tile and alpha/beta are fetched while the current one finishes.
 __global__ void __launch_bounds__(128, 2)
     transitions_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                          const __grid_constant__ CUtensorMap tmWb, const __grid_constant__ CUtensorMap tmUb,
+                          const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                           TransTcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint64_t* bars = (uint64_t*)(sm + kSmemUsed);  // tma, m1, m2, m3
+  float* Lsm = (float*)(sm + kScr);              // L, [C][kLP]
+  float* Usm = (float*)(sm + kScr + kLU);        // U = (I + L)^{-1}, [C][kLP]
+  float* Xsm = (float*)(sm + kX);                // L'_ik = U_ii L_ik, rows 16-63, [48][kXP]
+  float* ell_s = (float*)(sm + kSmall);          // l_t
+  float* beta_s = ell_s + kC;                    // beta_t
+  float* bg_s = beta_s + kC;                     // beta_t gamma_t
+  float* dk_s = bg_s + kC;                       // gamma_C / gamma_t
+  uint64_t* bars = (uint64_t*)(dk_s + kC);       // tma, mma1, mma2, mma34
   uint32_t* tmem_s = (uint32_t*)(bars + 4);
-  float* ell_s = (float*)(tmem_s + 4);           // [C]
-  float* beta_s = ell_s + kC;                    // [C]
-  float* wsum = beta_s + kC;                     // [2]
+  float* wsum = (float*)(tmem_s + 2);            // [2]
   volatile int* abort_s = (volatile int*)(wsum + 2);
-  float* Ls = (float*)(sm + kScr);               // [C][kLP]
-  float* Ts = Ls + kC * kLP;                     // [C][kLP]
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int i = blockIdx.x % a.N;
-  const int bh = blockIdx.x / a.N;
-  const int b = bh / a.H, h = bh % a.H;
-  const int t0 = i * kC;
-  const int n = min(kC, a.T - t0);
-  const long chunk = (long)bh * a.N + i;
 
   if (tid == 0) {
     for (int k = 0; k < 4; ++k) tc::mbar_init(&bars[k], 1);
@@ -87,211 +134,379 @@ __global__ void __launch_bounds__(128, 2)
     tc::mbar_fence_init();
     tc::fence_async_smem();
   }
-  if (warp == 0) tc::tmem_alloc(tmem_s, 256);
-  // l_t = cumulative log alpha (identity tokens beyond n)
-  float la = 0.0f;
-  if (tid < kC) {
-    const long off = b * a.sb_a + h * a.sh_a + (long)(t0 + tid) * a.st_a;
-    la = tid < n ? logf(a.alpha[off]) : 0.0f;
-    beta_s[tid] = tid < n ? a.beta[off] : 0.0f;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const float y = __shfl_up_sync(0xFFFFFFFFu, la, o);
-      if (lane >= o) la += y;
+  if (warp == 0 && lane == 0) {
+    tc::tma_prefetch_desc(&tmK);
+    tc::tma_prefetch_desc(&tmV);
+    if (a.has_wu) {
+      tc::tma_prefetch_desc(&tmWb);
+      tc::tma_prefetch_desc(&tmUb);
     }
-    if (lane == 31) wsum[warp] = la;
+    if (a.has_ab) {
+      tc::tma_prefetch_desc(&tmA);
+      tc::tma_prefetch_desc(&tmB);
+    }
   }
+  if (warp == 0) tc::tmem_alloc(tmem_s, 256);
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tm = *tmem_s;
-  if (tid < kC) {
-    if (warp == 1) la += wsum[0];
-    ell_s[tid] = la;
-    if (a.ell) a.ell[chunk * kC + tid] = la;
-  }
-  if (tid == 0) {
-    tc::mbar_arrive_expect_tx(&bars[0], 4 * 8192);
-    const int y = b * a.T + t0;
-    for (int kh = 0; kh < 2; ++kh) {
-      tc::tma_load_2d(sm + kKV + kh * 16384, &tmK, h * kD + 64 * kh, y, &bars[0]);
-      tc::tma_load_2d(sm + kKV + kh * 16384 + 8192, &tmV, h * kD + 64 * kh, y, &bars[0]);
-    }
-  }
-  bool ok = tc::bar_all(1, 128, tc::mbar_wait(&bars[0], 0, abort_s));
-  // MMA1: [K; V] K^T
-  if (ok && tid == 0) {
-    tc::tc_fence_after();
-    const uint32_t base = tc::smem_u32(sm + kKV);
-#pragma unroll
-    for (int ks = 0; ks < kD / 16; ++ks) {
-      const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-      tc::mma_ss(tm, tc::sdesc_sw128(base + off, 16, 1024), tc::sdesc_sw128(base + off, 16, 1024), kIdesc1,
-                 ks > 0 ? 1u : 0u);
-    }
-    tc::mma_commit(&bars[1]);
-  }
-  if (ok) ok = tc::bar_all(1, 128, tc::mbar_wait(&bars[1], 0, abort_s));
   const uint32_t lane_addr = tm + ((uint32_t)(32 * warp) << 16);
-  if (ok && tid < kC) {
-    // L row t
-    tc::tc_fence_after();
-    const int t = tid;
-    uint32_t g[64];
-    tc::tmem_ld32(lane_addr, *reinterpret_cast<uint32_t(*)[32]>(&g[0]));
-    tc::tmem_ld32(lane_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&g[32]));
-    tc::tmem_wait_ld();
-    const float bt = beta_s[t], lt = ell_s[t];
-#pragma unroll
-    for (int s = 0; s < kC; ++s) Ls[t * kLP + s] = s < t ? bt * __expf(lt - ell_s[s]) * __uint_as_float(g[s]) : 0.0f;
-  }
-  ok = tc::bar_all(1, 128, ok);
-  if (ok && tid < kC) {
-    // column c of T = (I + L)^{-1} diag(beta) by forward substitution, fully unrolled
-    // so the column stays in registers; every thread runs the same schedule (entries
-    // above the diagonal come out as exact zeros), so the reads of L are broadcasts.
-    const int c = tid;
-    float col[kC];
-#pragma unroll
-    for (int t = 0; t < kC; ++t) {
-      const float* Lrow = Ls + t * kLP;
-      float a0 = (t == c) ? beta_s[t] : 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
-#pragma unroll
-      for (int s4 = 0; s4 < t; s4 += 4) {
-        const float4 l4 = *(const float4*)(Lrow + s4);
-        a0 = fmaf(-l4.x, col[s4], a0);
-        if (s4 + 1 < t) a1 = fmaf(-l4.y, col[s4 + 1], a1);
-        if (s4 + 2 < t) a2 = fmaf(-l4.z, col[s4 + 2], a2);
-        if (s4 + 3 < t) a3 = fmaf(-l4.w, col[s4 + 3], a3);
-      }
-      col[t] = (a0 + a1) + (a2 + a3);
+
+  bool ok = true;
+  bool load_pending = false;  // thread 0: a K/V load was issued and not yet waited for
+  int load_parity = 0;
+  int it = 0, ph3 = 0;
+  float pa = 1.0f, pb = 0.0f;  // alpha, beta of token `tid` of the chunk to come
+  if (blockIdx.x < a.total) {
+    const ChunkPos p0 = chunk_pos(a, blockIdx.x);
+    if (tid == 0) {
+      load_kv(sm, &tmK, &tmV, &bars[0], a, p0);
+      load_pending = true;
+      load_parity = 0;
     }
-#pragma unroll
-    for (int t = 0; t < kC; ++t) Ts[t * kLP + c] = col[t];
+    if (tid < kC) load_ab(a, p0, tid, pa, pb);
   }
-  ok = tc::bar_all(1, 128, ok);
-  if (ok) {
-    // [T diag(gamma); T] as the K-major A operand (rows 0-63 scaled by gamma_s)
-    const int t = tid & (kC - 1);
-    const bool scaled = tid < kC;
+  for (long chunk = blockIdx.x; ok && chunk < a.total; chunk += gridDim.x, ++it) {
+    const ChunkPos P = chunk_pos(a, chunk);
+    const bool write_ab = (P.n == kC) && a.has_ab;
+    const long next = chunk + gridDim.x;
+
+    // ---- l_t = cumulative log alpha ----
+    float la = 0.0f;
+    if (tid < kC) {
+      la = logf(pa);
+      beta_s[tid] = pb;
 #pragma unroll
-    for (int c8 = 0; c8 < 8; ++c8) {
-      uint32_t w[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int s = c8 * 8 + 2 * e;
-        float x0 = Ts[t * kLP + s], x1 = Ts[t * kLP + s + 1];
-        if (scaled) {
-          x0 *= __expf(ell_s[s]);
-          x1 *= __expf(ell_s[s + 1]);
-        }
-        w[e] = tc::pack_bf16x2(x0, x1);
+      for (int o = 1; o < 32; o <<= 1) {
+        const float y = __shfl_up_sync(0xFFFFFFFFu, la, o);
+        if (lane >= o) la += y;
       }
-      *(uint4*)(sm + kTT + swz(tid, c8)) = make_uint4(w[0], w[1], w[2], w[3]);
+      if (lane == 31) wsum[warp] = la;
     }
-    tc::fence_async_smem();
-  }
-  ok = tc::bar_all(1, 128, ok);
-  // MMA2: [T gamma; T] x [K | V]  (N order: K c0-63, V v0-63, K c64-127, V v64-127)
-  if (ok && tid == 0) {
-    tc::tc_fence_after();
-    const uint32_t abase = tc::smem_u32(sm + kTT), bbase = tc::smem_u32(sm + kKV);
+    tc::bar_sync(1, 128);
+    if (tid < kC) {
+      if (warp == 1) la += wsum[0];
+      ell_s[tid] = la;
+      if (a.ell) a.ell[chunk * kC + tid] = la;
+    }
+    // the K/V tile has landed; the previous chunk's staged stores have left shared memory
+    bool got = true;
+    if (tid == 0) {
+      tc::bulk_wait_read_all();
+      got = tc::mbar_wait(&bars[0], it & 1, abort_s);
+      if (got) load_pending = false;
+    }
+    ok = tc::bar_all(1, 128, got);
+
+    // ---- MMA1: [K; V] K^T -> columns 0-63 (rows 0-63: K K^T) ----
+    if (ok && tid == 0) {
+      tc::tc_fence_after();
+      const uint32_t base = tc::smem_u32(sm + kKV);
 #pragma unroll
-    for (int ks = 0; ks < kC / 16; ++ks)
-      tc::mma_ss(tm, tc::sdesc_sw128(abase + ks * 32, 16, 1024), tc::sdesc_sw128(bbase + ks * 2048, 8192, 1024),
-                 kIdesc2, ks > 0 ? 1u : 0u);
-    tc::mma_commit(&bars[2]);
-  }
-  if (ok) ok = tc::bar_all(1, 128, tc::mbar_wait(&bars[2], 0, abort_s));
-  if (ok) {
-    tc::tc_fence_after();
-    // rows 0-63: Wb row t (cols 0-63 and 128-191); rows 64-127: Ub row t (64-127, 192-255)
-    const int t = tid & (kC - 1);
-    const bool isW = tid < kC;
-    uint8_t* opT = sm + kScr + (isW ? 0 : 16384);  // Wb^T / Ub^T operand, [half][64 rows t][128 B]
-    __nv_bfloat16* gout = isW ? a.Wb : a.Ub;
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      uint32_t x[64];
-      const uint32_t col = (isW ? 0 : 64) + 128 * half;
-      tc::tmem_ld32(lane_addr + col, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
-      tc::tmem_ld32(lane_addr + col + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
+      for (int ks = 0; ks < kD / 16; ++ks) {
+        const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+        tc::mma_ss(tm, tc::sdesc_sw128(base + off, 16, 1024), tc::sdesc_sw128(base + off, 16, 1024), kIdesc1,
+                   ks > 0 ? 1u : 0u);
+      }
+      tc::mma_commit(&bars[1]);
+    }
+    if (ok && tid >= kC) {
+      // per-token scales, while the MMA runs
+      const int s = tid - kC;
+      const float ls = ell_s[s];
+      bg_s[s] = beta_s[s] * __expf(ls);
+      dk_s[s] = __expf(ell_s[kC - 1] - ls);
+    }
+    {
+      const bool m1 = (ok && tid == 0) ? tc::mbar_wait(&bars[1], it & 1, abort_s) : true;
+      ok = tc::bar_all(1, 128, ok && m1);
+    }
+
+    // ---- L[t][s] = beta_t e^{l_t - l_s} (k_t . k_s) for s < t, else 0 ----
+    // warps 0-1 (the lanes of rows 0-63) spill beta_t (K K^T)[t][.]; then every thread
+    // applies the decay and the mask to half a row
+    if (ok && tid < kC) {
+      tc::tc_fence_after();
+      const int t = tid;
+      uint32_t g[64];
+      tc::tmem_ld32(lane_addr, *reinterpret_cast<uint32_t(*)[32]>(&g[0]));
+      tc::tmem_ld32(lane_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&g[32]));
       tc::tmem_wait_ld();
-      uint32_t w[32];
+      const float bt = beta_s[t];
+      float* Lrow = Lsm + t * kLP;
 #pragma unroll
-      for (int e = 0; e < 32; ++e) w[e] = tc::pack_bf16x2(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1]));
-      if (gout) {
-        uint4* dst = (uint4*)(gout + (chunk * kC + t) * kD + 64 * half);
+      for (int s4 = 0; s4 < kC; s4 += 4)
+        *(float4*)(Lrow + s4) = make_float4(bt * __uint_as_float(g[s4]), bt * __uint_as_float(g[s4 + 1]),
+                                            bt * __uint_as_float(g[s4 + 2]), bt * __uint_as_float(g[s4 + 3]));
+      tc::tc_fence_before();
+    }
+    ok = tc::bar_all(1, 128, ok);
+    if (ok) {
+      const int t = tid & (kC - 1), hs = tid >> 6;
+      const float lt = ell_s[t];
+      float* Lrow = Lsm + t * kLP;
 #pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) dst[c8] = make_uint4(w[4 * c8], w[4 * c8 + 1], w[4 * c8 + 2], w[4 * c8 + 3]);
+      for (int q = 0; q < 8; ++q) {
+        const int s4 = 32 * hs + 4 * q;
+        const float4 l4 = *(const float4*)(ell_s + s4);
+        const float4 g4 = *(const float4*)(Lrow + s4);
+        float4 v;
+        v.x = (s4 + 0 < t) ? __expf(lt - l4.x) * g4.x : 0.0f;
+        v.y = (s4 + 1 < t) ? __expf(lt - l4.y) * g4.y : 0.0f;
+        v.z = (s4 + 2 < t) ? __expf(lt - l4.z) * g4.z : 0.0f;
+        v.w = (s4 + 3 < t) ? __expf(lt - l4.w) * g4.w : 0.0f;
+        *(float4*)(Lrow + s4) = v;
+      }
+    }
+    ok = tc::bar_all(1, 128, ok);
+
+    // ---- U = (I + L)^{-1} by 16 x 16 blocks.  Diagonal blocks U_kk: forward
+    //      substitution, thread = (block k, column c) ----
+    if (ok && tid < kC) {
+      const int k = tid >> 4, c = tid & 15;
+      float x[16];
+#pragma unroll
+      for (int tl = 0; tl < 16; ++tl) {
+        const float* Lrow = Lsm + (16 * k + tl) * kLP + 16 * k;
+        float v = (tl == c) ? 1.0f : 0.0f;
+#pragma unroll
+        for (int sl = 0; sl < tl; ++sl) v = fmaf(-Lrow[sl], x[sl], v);
+        x[tl] = v;
       }
 #pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8)
-        *(uint4*)(opT + half * 8192 + swz(t, c8)) = make_uint4(w[4 * c8], w[4 * c8 + 1], w[4 * c8 + 2], w[4 * c8 + 3]);
+      for (int tl = 0; tl < 16; ++tl) Usm[(16 * k + tl) * kLP + 16 * k + c] = x[tl];
     }
-    if (isW) {
-      // D K row t: K row t scaled by gamma_C / gamma_t, into the old [T gamma; T] space
-      const float dt = __expf(ell_s[kC - 1] - ell_s[t]);
+    ok = tc::bar_all(1, 128, ok);
+    // Off-diagonal blocks.  With L'_ik = U_ii L_ik (k < i),  U_ij = -sum_{k=j}^{i-1} L'_ik U_kj,
+    // one level (i - j = 1, 2, 3) after the other.  Thread = (column c, rows tb and tb + 8).
+    const int cc16 = tid & 15, tb = tid >> 4;
+    if (ok) {
+#pragma unroll
+      for (int ib = 1; ib < 4; ++ib) {
+        float ua[16], ub[16];  // U_ii rows tb, tb + 8
+#pragma unroll
+        for (int u4 = 0; u4 < 16; u4 += 4) {
+          const float4 x0 = *(const float4*)(Usm + (16 * ib + tb) * kLP + 16 * ib + u4);
+          const float4 x1 = *(const float4*)(Usm + (16 * ib + tb + 8) * kLP + 16 * ib + u4);
+          ua[u4] = x0.x; ua[u4 + 1] = x0.y; ua[u4 + 2] = x0.z; ua[u4 + 3] = x0.w;
+          ub[u4] = x1.x; ub[u4 + 1] = x1.y; ub[u4 + 2] = x1.z; ub[u4 + 3] = x1.w;
+        }
+#pragma unroll
+        for (int mb = 0; mb < ib; ++mb) {
+          float s0 = 0.0f, s1 = 0.0f;
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const float l = Lsm[(16 * ib + u) * kLP + 16 * mb + cc16];
+            s0 = fmaf(ua[u], l, s0);
+            s1 = fmaf(ub[u], l, s1);
+          }
+          Xsm[(16 * ib - 16 + tb) * kXP + 16 * mb + cc16] = s0;
+          Xsm[(16 * ib - 16 + tb + 8) * kXP + 16 * mb + cc16] = s1;
+        }
+      }
+    }
+    ok = tc::bar_all(1, 128, ok);
+#pragma unroll
+    for (int lev = 1; lev < 4; ++lev) {
+      if (ok) {
+#pragma unroll
+        for (int jb = 0; jb + lev < 4; ++jb) {
+          const int ib = jb + lev;
+          const float* x0 = Xsm + (16 * ib - 16 + tb) * kXP;
+          const float* x1 = Xsm + (16 * ib - 16 + tb + 8) * kXP;
+          float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f, s3 = 0.0f;
+#pragma unroll
+          for (int s4 = 16 * jb; s4 < 16 * ib; s4 += 4) {
+            const float4 a4 = *(const float4*)(x0 + s4);
+            const float4 b4 = *(const float4*)(x1 + s4);
+            const float u0 = Usm[(s4 + 0) * kLP + 16 * jb + cc16];
+            const float u1 = Usm[(s4 + 1) * kLP + 16 * jb + cc16];
+            const float u2 = Usm[(s4 + 2) * kLP + 16 * jb + cc16];
+            const float u3 = Usm[(s4 + 3) * kLP + 16 * jb + cc16];
+            s0 = fmaf(a4.x, u0, fmaf(a4.y, u1, s0));
+            s1 = fmaf(a4.z, u2, fmaf(a4.w, u3, s1));
+            s2 = fmaf(b4.x, u0, fmaf(b4.y, u1, s2));
+            s3 = fmaf(b4.z, u2, fmaf(b4.w, u3, s3));
+          }
+          Usm[(16 * ib + tb) * kLP + 16 * jb + cc16] = -(s0 + s1);
+          Usm[(16 * ib + tb + 8) * kLP + 16 * jb + cc16] = -(s2 + s3);
+        }
+      }
+      ok = tc::bar_all(1, 128, ok);
+    }
+
+    // ---- operand [T diag(gamma); T] (bf16, K-major, 128 rows x 64), T = U diag(beta) ----
+    if (ok) {
+      const int r = tid, t = r & (kC - 1);
+      const float* scl = r < kC ? bg_s : beta_s;
+      const float* Urow = Usm + t * kLP;
+#pragma unroll
+      for (int c8 = 0; c8 < 8; ++c8) {
+        uint4 w = make_uint4(0u, 0u, 0u, 0u);
+        if ((c8 >> 1) <= (t >> 4)) {  // blocks above the diagonal are zero
+          const float4 u0 = *(const float4*)(Urow + 8 * c8);
+          const float4 u1 = *(const float4*)(Urow + 8 * c8 + 4);
+          const float4 s0 = *(const float4*)(scl + 8 * c8);
+          const float4 s1 = *(const float4*)(scl + 8 * c8 + 4);
+          w.x = tc::pack_bf16x2(u0.x * s0.x, u0.y * s0.y);
+          w.y = tc::pack_bf16x2(u0.z * s0.z, u0.w * s0.w);
+          w.z = tc::pack_bf16x2(u1.x * s1.x, u1.y * s1.y);
+          w.w = tc::pack_bf16x2(u1.z * s1.z, u1.w * s1.w);
+        }
+        *(uint4*)(sm + kTT + swz(r, c8)) = w;
+      }
+      tc::fence_async_smem();
+    }
+    ok = tc::bar_all(1, 128, ok);
+
+    // ---- MMA2: [T gamma; T] x [K | V]  (N order: K c0-63, V v0-63, K c64-127, V v64-127) ----
+    if (ok && tid == 0) {
+      tc::tc_fence_after();
+      const uint32_t abase = tc::smem_u32(sm + kTT), bbase = tc::smem_u32(sm + kKV);
+#pragma unroll
+      for (int ks = 0; ks < kC / 16; ++ks)
+        tc::mma_ss(tm, tc::sdesc_sw128(abase + ks * 32, 16, 1024), tc::sdesc_sw128(bbase + ks * 2048, 8192, 1024),
+                   kIdesc2, ks > 0 ? 1u : 0u);
+      tc::mma_commit(&bars[2]);
+    }
+    {
+      const bool m2 = (ok && tid == 0) ? tc::mbar_wait(&bars[2], it & 1, abort_s) : true;
+      ok = tc::bar_all(1, 128, ok && m2);
+    }
+
+    // ---- Wb (rows 0-63) and Ub (rows 64-127) to bf16 row-major swizzled tiles in Scr:
+    //      the MN-major A operands of MMA3/4 and the sources of their TMA stores;
+    //      D K (K row t scaled by gamma_C / gamma_t) into TT ----
+    if (ok) {
+      tc::tc_fence_after();
+      const int t = tid & (kC - 1);
+      const bool isW = tid < kC;
+      uint8_t* opT = sm + kScr + (isW ? 0 : 16384);  // [half][64 rows t][128 B]
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
+        uint32_t x[64];
+        const uint32_t col = (isW ? 0 : 64) + 128 * half;
+        tc::tmem_ld32(lane_addr + col, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
+        tc::tmem_ld32(lane_addr + col + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
+        tc::tmem_wait_ld();
 #pragma unroll
         for (int c8 = 0; c8 < 8; ++c8) {
-          const uint4 kw = *(const uint4*)(sm + kKV + half * 16384 + swz(t, c8));
-          const uint32_t kk[4] = {kw.x, kw.y, kw.z, kw.w};
-          uint32_t w[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) w[e] = tc::pack_bf16x2(dt * tc::bf16lo(kk[e]), dt * tc::bf16hi(kk[e]));
-          *(uint4*)(sm + kTT + half * 8192 + swz(t, c8)) = make_uint4(w[0], w[1], w[2], w[3]);
+          uint4 w;
+          w.x = tc::pack_bf16x2(__uint_as_float(x[8 * c8 + 0]), __uint_as_float(x[8 * c8 + 1]));
+          w.y = tc::pack_bf16x2(__uint_as_float(x[8 * c8 + 2]), __uint_as_float(x[8 * c8 + 3]));
+          w.z = tc::pack_bf16x2(__uint_as_float(x[8 * c8 + 4]), __uint_as_float(x[8 * c8 + 5]));
+          w.w = tc::pack_bf16x2(__uint_as_float(x[8 * c8 + 6]), __uint_as_float(x[8 * c8 + 7]));
+          *(uint4*)(opT + half * 8192 + swz(t, c8)) = w;
         }
       }
+      if (isW) {
+        const float dt = dk_s[t];
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+#pragma unroll
+          for (int c8 = 0; c8 < 8; ++c8) {
+            const uint4 kw = *(const uint4*)(sm + kKV + half * 16384 + swz(t, c8));
+            const uint32_t kk[4] = {kw.x, kw.y, kw.z, kw.w};
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) w[e] = tc::pack_bf16x2(dt * tc::bf16lo(kk[e]), dt * tc::bf16hi(kk[e]));
+            *(uint4*)(sm + kTT + half * 8192 + swz(t, c8)) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
+      tc::fence_async_smem();
+      tc::tc_fence_before();
     }
-    tc::fence_async_smem();
+    ok = tc::bar_all(1, 128, ok);
+    const bool mma34 = ok && write_ab;
+    if (ok && tid == 0) {
+      tc::tc_fence_after();
+      if (a.has_wu) {
+        const int y = (int)(chunk * kC);
+        tc::tma_store_2d(&tmWb, sm + kScr, 0, y);
+        tc::tma_store_2d(&tmWb, sm + kScr + 8192, 64, y);
+        tc::tma_store_2d(&tmUb, sm + kScr + 16384, 0, y);
+        tc::tma_store_2d(&tmUb, sm + kScr + 16384 + 8192, 64, y);
+        tc::bulk_commit();
+      }
+      // MMA3/4: Wb^T D K -> columns 0-127, Ub^T D K -> columns 128-255
+      if (mma34) {
+        const uint32_t wbase = tc::smem_u32(sm + kScr), ubase = wbase + 16384, dbase = tc::smem_u32(sm + kTT);
+#pragma unroll
+        for (int ks = 0; ks < kC / 16; ++ks) {
+          const uint64_t bd = tc::sdesc_sw128(dbase + ks * 2048, 8192, 1024);
+          tc::mma_ss(tm, tc::sdesc_sw128(wbase + ks * 2048, 8192, 1024), bd, kIdesc3, ks > 0 ? 1u : 0u);
+          tc::mma_ss(tm + 128, tc::sdesc_sw128(ubase + ks * 2048, 8192, 1024), bd, kIdesc3, ks > 0 ? 1u : 0u);
+        }
+        tc::mma_commit(&bars[3]);
+      }
+      // the K/V tile is no longer read (MMA2 done, D K built): fetch the next chunk's
+      if (next < a.total) {
+        load_kv(sm, &tmK, &tmV, &bars[0], a, chunk_pos(a, next));
+        load_pending = true;
+        load_parity = (it + 1) & 1;
+      }
+    }
+    if (ok && tid < kC && next < a.total) load_ab(a, chunk_pos(a, next), tid, pa, pb);
+    if (mma34) {
+      const bool m3 = tid == 0 ? tc::mbar_wait(&bars[3], ph3 & 1, abort_s) : true;
+      ++ph3;
+      if (tid == 0 && m3) tc::bulk_wait_read_all();  // the Wb/Ub stores have read Scr
+      ok = tc::bar_all(1, 128, m3);
+    }
+
+    // ---- A = gamma_C I - Wb^T D K and B = Ub^T D K (row r per thread) to bf16 swizzled
+    //      staging (A in Scr; B in TT and X), then TMA stores ----
+    if (mma34 && ok) {
+      tc::tc_fence_after();
+      const int r = tid;
+      const float gC = __expf(ell_s[kC - 1]);
+#pragma unroll
+      for (int cc = 0; cc < kD; cc += 32) {
+        uint32_t x[32], y[32];
+        tc::tmem_ld32(lane_addr + cc, x);
+        tc::tmem_ld32(lane_addr + 128 + cc, y);
+        tc::tmem_wait_ld();
+        const int half = cc >> 6;
+        uint8_t* bst = sm + (half ? kX : kTT);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int c8 = ((cc & 63) >> 3) + q;
+          uint32_t wa[4], wb[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = cc + 8 * q + 2 * e;
+            const float a0 = (r == c ? gC : 0.0f) - __uint_as_float(x[8 * q + 2 * e]);
+            const float a1 = (r == c + 1 ? gC : 0.0f) - __uint_as_float(x[8 * q + 2 * e + 1]);
+            wa[e] = tc::pack_bf16x2(a0, a1);
+            wb[e] = tc::pack_bf16x2(__uint_as_float(y[8 * q + 2 * e]), __uint_as_float(y[8 * q + 2 * e + 1]));
+          }
+          *(uint4*)(sm + kScr + half * 16384 + swz(r, c8)) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+          *(uint4*)(bst + swz(r, c8)) = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+        }
+      }
+      tc::fence_async_smem();
+      tc::tc_fence_before();
+      tc::bar_sync(1, 128);
+      if (tid == 0) {
+        const int y = (int)((P.bh * a.ab_chunk_stride + P.i) * kD);
+        tc::tma_store_2d(&tmA, sm + kScr, 0, y);
+        tc::tma_store_2d(&tmA, sm + kScr + 16384, 64, y);
+        tc::tma_store_2d(&tmB, sm + kTT, 0, y);
+        tc::tma_store_2d(&tmB, sm + kX, 64, y);
+        tc::bulk_commit();
+      }
+    }
+    // every reader of this chunk's shared and tensor memory is done
     tc::tc_fence_before();
+    ok = tc::bar_all(1, 128, ok);
   }
-  ok = tc::bar_all(1, 128, ok);
-  const bool write_ab = (n == kC) && a.A != nullptr;
-  // MMA3/4: Wb^T D K -> cols 0-127, Ub^T D K -> cols 128-255
-  if (ok && write_ab && tid == 0) {
-    tc::tc_fence_after();
-    const uint32_t wbase = tc::smem_u32(sm + kScr), ubase = wbase + 16384, dbase = tc::smem_u32(sm + kTT);
-#pragma unroll
-    for (int ks = 0; ks < kC / 16; ++ks) {
-      const uint64_t bd = tc::sdesc_sw128(dbase + ks * 2048, 8192, 1024);
-      tc::mma_ss(tm, tc::sdesc_sw128(wbase + ks * 2048, 8192, 1024), bd, kIdesc3, ks > 0 ? 1u : 0u);
-      tc::mma_ss(tm + 128, tc::sdesc_sw128(ubase + ks * 2048, 8192, 1024), bd, kIdesc3, ks > 0 ? 1u : 0u);
-    }
-    tc::mma_commit(&bars[3]);
-  }
-  if (ok && write_ab) ok = tc::bar_all(1, 128, tc::mbar_wait(&bars[3], 0, abort_s));
-  if (ok && write_ab) {
-    tc::tc_fence_after();
-    const int r = tid;
-    const float gC = __expf(ell_s[kC - 1]);
-    __nv_bfloat16* Arow = a.A + ((long)bh * a.ab_chunk_stride + i) * kD * kD + (long)r * kD;
-    __nv_bfloat16* Brow = a.Bm + ((long)bh * a.ab_chunk_stride + i) * kD * kD + (long)r * kD;
-#pragma unroll
-    for (int cc = 0; cc < kD; cc += 32) {
-      uint32_t x[32], y[32];
-      tc::tmem_ld32(lane_addr + cc, x);
-      tc::tmem_ld32(lane_addr + 128 + cc, y);
-      tc::tmem_wait_ld();
-      uint32_t wa[16], wb[16];
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const int c = cc + 2 * e;
-        const float a0 = (r == c ? gC : 0.0f) - __uint_as_float(x[2 * e]);
-        const float a1 = (r == c + 1 ? gC : 0.0f) - __uint_as_float(x[2 * e + 1]);
-        wa[e] = tc::pack_bf16x2(a0, a1);
-        wb[e] = tc::pack_bf16x2(__uint_as_float(y[2 * e]), __uint_as_float(y[2 * e + 1]));
-      }
-      uint4* da = (uint4*)(Arow + cc);
-      uint4* db = (uint4*)(Brow + cc);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        da[e] = make_uint4(wa[4 * e], wa[4 * e + 1], wa[4 * e + 2], wa[4 * e + 3]);
-        db[e] = make_uint4(wb[4 * e], wb[4 * e + 1], wb[4 * e + 2], wb[4 * e + 3]);
-      }
-    }
+
+  if (tid == 0) {
+    tc::bulk_wait_all();
+    // never leave the CTA with a copy in flight
+    if (load_pending) tc::mbar_wait(&bars[0], load_parity, nullptr, 200000000ull);
   }
   tc::tc_fence_before();
   __syncthreads();
@@ -307,31 +522,53 @@ cudaError_t launch_transitions_tc(const TransArgs& t, cudaStream_t s) {
   if (t.n_chunks <= 0) return cudaSuccess;
   const long HD = (long)t.H * kD;
   const long rows = (long)t.B * (t.in.sb / HD);  // B x tokens per sequence
-  CUtensorMap tk, tv;
+  const long total = (long)t.B * t.H * t.n_chunks;
+  const long ab_rows = (long)t.B * t.H * t.ab_chunk_stride * kD;
+  // tile coordinates are 32-bit
+  if (rows >= (1L << 31) || total * kC >= (1L << 31) || ab_rows >= (1L << 31)) return cudaErrorNotSupported;
+  CUtensorMap tk, tv, twb, tub, ta, tb;
   cudaError_t e = make_tmap_2d(&tk, t.in.k, HD, rows, HD * 2, 64, 64);
   if (e == cudaSuccess) e = make_tmap_2d(&tv, t.in.v, HD, rows, HD * 2, 64, 64);
+  // outputs that are not requested get a valid map that is never used
+  const void* wb = t.Wb ? (const void*)t.Wb : t.in.k;
+  const void* ub = t.Ub ? (const void*)t.Ub : t.in.k;
+  const bool has_ab = t.A != nullptr && t.Bm != nullptr && t.ab_chunk_stride > 0;
+  const void* ab = has_ab ? t.A : t.in.k;
+  const void* bb = has_ab ? t.Bm : t.in.k;
+  const long wu_rows = t.Wb ? total * kC : 64;
+  const long ab_map_rows = has_ab ? ab_rows : 128;
+  if (e == cudaSuccess) e = make_tmap_2d(&twb, wb, kD, wu_rows, kD * 2, 64, 64);
+  if (e == cudaSuccess) e = make_tmap_2d(&tub, ub, kD, wu_rows, kD * 2, 64, 64);
+  if (e == cudaSuccess) e = make_tmap_2d(&ta, ab, kD, ab_map_rows, kD * 2, 64, 128);
+  if (e == cudaSuccess) e = make_tmap_2d(&tb, bb, kD, ab_map_rows, kD * 2, 64, 128);
   if (e != cudaSuccess) return e;
   TransTcArgs a;
   a.B = t.B;
   a.H = t.H;
   a.T = (int)(t.in.sb / HD);  // tokens per sequence in the input layout
   a.N = t.n_chunks;
+  a.total = total;
   a.sb_a = t.in.ab;
   a.sh_a = t.in.ah;
   a.st_a = t.in.at;
   a.alpha = t.in.alpha;
   a.beta = t.in.beta;
-  a.A = (__nv_bfloat16*)t.A;
-  a.Bm = (__nv_bfloat16*)t.Bm;
+  a.has_ab = has_ab;
   a.ab_chunk_stride = t.ab_chunk_stride;
-  a.Wb = (__nv_bfloat16*)t.Wb;
-  a.Ub = (__nv_bfloat16*)t.Ub;
+  a.has_wu = t.Wb != nullptr && t.Ub != nullptr;
   a.ell = t.ell;
-  // chunks beyond t.T (gdn_chunk_transitions limits T to whole chunks) are not launched
-  const size_t smem = 1024 + kSmemUsed + 4 * 8 + 16 + 2 * kC * 4 + 16;
+  static int num_sms = 0;
+  if (num_sms == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || num_sms <= 0)
+      num_sms = 148;
+  }
+  const size_t smem = 1024 + kSmemUsed;
   e = cudaFuncSetAttribute(transitions_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  transitions_tc_kernel<<<(unsigned)(t.B * t.H * t.n_chunks), 128, smem, s>>>(tk, tv, a);
+  const long grid = total < 2L * num_sms ? total : 2L * num_sms;
+  transitions_tc_kernel<<<(unsigned)grid, 128, smem, s>>>(tk, tv, twb, tub, ta, tb, a);
   return cudaGetLastError();
 }
 
