@@ -15,9 +15,9 @@
 // chain: D_k <- (1 - g_next) S_new, Aop_k <- bf16(g_next S_new).  After a chain's
 // last active step S_new is written to S_in (float32, [v][c]).
 //
-// Warp roles: warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer, warps 2-9
-// epilogue of chain 0 and warps 10-17 epilogue of chain 1 (lane quarter = warp % 4,
-// column half = ((warp - 2) % 8) / 4), so each chain's epilogue overlaps the other
+// Warp roles: warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer, warps 2-17
+// epilogue (lane quarter = warp % 4, column quarter = (warp - 2) / 4).  The epilogue
+// warps finish each step chain by chain, so one chain's epilogue overlaps the other
 // chain's MMA.  Elementwise math uses packed float32 pairs.  All waits are bounded
 // (about 2 s, then a device error word is set and the CTA exits cleanly).
 //
@@ -145,7 +145,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int k = 0; k < 2; ++k) {
       tc::mbar_init(&mma_done[k], 1);
-      tc::mbar_init(&op_ready[k], 8);   // lane 0 of every warp of the chain's group
+      tc::mbar_init(&op_ready[k], 16);  // lane 0 of every epilogue warp
     }
     tc::mbar_init(final_bar, 1);
     *abort_s = 0;
@@ -260,105 +260,101 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else {
-    // ------------- epilogue: group k (8 warps, 256 threads, named barrier 1 + k) -------------
-    const int k = (warp - 2) >> 3;
-    const int bar_id = 1 + k;
+    // ------------- epilogue: all 16 warps (512 threads, named barrier 1) -------------
+    // Each step is finished chain by chain by every epilogue warp: warp w owns TMEM
+    // lane quarter q = w % 4 (rows v = 32 q + lane) and the column quarter
+    // [32 c4, 32 c4 + 32).  While the warps finish one chain, the tensor pipe runs the
+    // other chain's MMA.
     const int q = warp & 3;
-    const int h = ((warp - 2) & 7) >> 2;
+    const int c4 = (warp - 2) >> 2;
     const int v = 32 * q + lane;
-    const int col0 = 64 * h;
+    const int col0 = 32 * c4;
     const uint32_t lane_off = (uint32_t)(32 * q) << 16;
-    const int chain = k ? chains[1] : chains[0];
-    __nv_bfloat16* out_row =
-        chain >= 0 ? a.S_in + ((long)bh * a.N + chain) * kD * kD + (long)v * kD + col0 : nullptr;
-    // a chain with nothing active has S_in = 0 (in scan mode: S_in(0))
-    if (chain >= 0 && (kScan || a.act_cnt[(long)bh * a.N + chain] == 0))
-      for (int e = 0; e < 8; ++e) ((uint4*)out_row)[e] = make_uint4(0u, 0u, 0u, 0u);
+    __nv_bfloat16* out_row[2];
+    for (int k = 0; k < 2; ++k) {
+      const int chain = chains[k];
+      out_row[k] = chain >= 0 ? a.S_in + ((long)bh * a.N + chain) * kD * kD + (long)v * kD + col0 : nullptr;
+      // a chain with nothing active has S_in = 0 (in scan mode: S_in(0))
+      if (chain >= 0 && (kScan || a.act_cnt[(long)bh * a.N + chain] == 0))
+        for (int e = 0; e < 4; ++e) ((uint4*)out_row[k])[e] = make_uint4(0u, 0u, 0u, 0u);
+    }
     for (int s = 0;; ++s) {
       const int st = s % kStages;
       const bool w = tc::mbar_wait(&full[st], (s / kStages) & 1, abort_s);
       const int jv = w ? ((volatile StepInfo*)info)[st].j : 0;
       // one vote per step: stop at the end marker or on a timeout anywhere
-      if (tc::bar_any(bar_id, 256, !w || *abort_s != 0 || jv < 0)) break;
+      if (tc::bar_any(1, 512, !w || *abort_s != 0 || jv < 0)) break;
       const StepInfo e = info[st];
-      const bool act = (e.flags >> k) & 1;
-      const bool last = (e.flags >> (4 + k)) & 1;
-      if (act) {
+      // B_j[v][col0 .. col0+32) from the swizzled box (half col0 / 64, 16-byte chunks)
+      const uint8_t* brow = ring + st * kStageBytes + 2 * kHalfBytes + (col0 >> 6) * kHalfBytes + v * 128;
+      uint32_t bw[16];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int c8 = ((col0 & 63) >> 3) + c;
+        const uint4 w4 = *(const uint4*)(brow + ((c8 ^ (v & 7)) << 4));
+        bw[4 * c + 0] = w4.x;
+        bw[4 * c + 1] = w4.y;
+        bw[4 * c + 2] = w4.z;
+        bw[4 * c + 3] = w4.w;
+      }
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        if (!((e.flags >> k) & 1)) continue;
         const bool first = (e.flags >> (2 + k)) & 1;
+        const bool last = (e.flags >> (4 + k)) & 1;
         const float g = k ? e.g[1] : e.g[0];
         const float gn = k ? e.gn[1] : e.gn[0];
         const int pk = k ? e.p[1] : e.p[0];
-        const float keep = 1.0f - gn;
-        // B_j[v][col0 .. col0+64) from the swizzled box
-        const uint8_t* brow = ring + st * kStageBytes + 2 * kHalfBytes + h * kHalfBytes + v * 128;
-        uint32_t bw[32];
-#pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {
-          const uint4 w4 = *(const uint4*)(brow + ((c8 ^ (v & 7)) << 4));
-          bw[4 * c8 + 0] = w4.x;
-          bw[4 * c8 + 1] = w4.y;
-          bw[4 * c8 + 2] = w4.z;
-          bw[4 * c8 + 3] = w4.w;
-        }
+        const uint32_t d_addr = tbase + lane_off + 128u * k + col0;
+        uint32_t d[32];
         if (!first) {
           tc::mbar_wait(&mma_done[k], (pk - 1) & 1, abort_s);
           tc::tc_fence_after();
+          tc::tmem_ld32(d_addr, d);
+          tc::tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) d[i] = 0u;
         }
+        const float2 g2 = make_float2(g, g);
+        if (kScan || last) {
+          // the state after this step (scan mode: S_in(j + 1); else the chain's S_in)
+          uint4* out = (uint4*)(out_row[k] + (kScan ? (long)(e.j + 1) * kD * kD : 0));
+          uint32_t op[16];
 #pragma unroll
-        for (int cc = 0; cc < 64; cc += 32) {
-          const uint32_t d_addr = tbase + lane_off + 128u * k + col0 + cc;
-          uint32_t d[32];
-          if (!first) {
-            tc::tmem_ld32(d_addr, d);
-            tc::tmem_wait_ld();
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) d[i] = 0u;
+          for (int i = 0; i < 16; ++i) {
+            const float2 x = tc::fma2(g2, tc::bf16x2_to_float2(bw[i]),
+                                      make_float2(__uint_as_float(d[2 * i]), __uint_as_float(d[2 * i + 1])));
+            op[i] = tc::pack_bf16x2(x.x, x.y);
           }
-          const float2 g2 = make_float2(g, g);
-          float2 x[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            x[i] = tc::fma2(g2, tc::bf16x2_to_float2(bw[cc / 2 + i]),
-                            make_float2(__uint_as_float(d[2 * i]), __uint_as_float(d[2 * i + 1])));
-          if (kScan || last) {
-            // scan mode: this step's state is S_in(j + 1)
-            uint4* out = (uint4*)(out_row + (kScan ? (long)(e.j + 1) * kD * kD : 0) + cc);
+          for (int i = 0; i < 4; ++i) out[i] = make_uint4(op[4 * i], op[4 * i + 1], op[4 * i + 2], op[4 * i + 3]);
+          // scan mode: the same bf16(S) is the next operand; the next product starts from zero
+          if (kScan && !last) tc::tmem_st16(tbase + lane_off + 256u + 64u * k + col0 / 2, op);
+        } else {
+          const float keep = 1.0f - gn;
+          const float2 gn2 = make_float2(gn, gn), keep2 = make_float2(keep, keep);
+          uint32_t op[16];
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              out[i] = make_uint4(tc::pack_bf16x2(x[4 * i].x, x[4 * i].y), tc::pack_bf16x2(x[4 * i + 1].x, x[4 * i + 1].y),
-                                  tc::pack_bf16x2(x[4 * i + 2].x, x[4 * i + 2].y),
-                                  tc::pack_bf16x2(x[4 * i + 3].x, x[4 * i + 3].y));
+          for (int i = 0; i < 16; ++i) {
+            const float2 x = tc::fma2(g2, tc::bf16x2_to_float2(bw[i]),
+                                      make_float2(__uint_as_float(d[2 * i]), __uint_as_float(d[2 * i + 1])));
+            const float2 o = tc::mul2(gn2, x);
+            const float2 nn = tc::mul2(keep2, x);
+            op[i] = tc::pack_bf16x2(o.x, o.y);
+            d[2 * i] = __float_as_uint(nn.x);
+            d[2 * i + 1] = __float_as_uint(nn.y);
           }
-          if (kScan && !last) {
-            // next operand bf16(S); the next product starts from zero, no state store
-            uint32_t op[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) op[i] = tc::pack_bf16x2(x[i].x, x[i].y);
-            tc::tmem_st16(tbase + lane_off + 256u + 64u * k + (col0 + cc) / 2, op);
-          } else if (!kScan && !last) {
-            const float2 gn2 = make_float2(gn, gn), keep2 = make_float2(keep, keep);
-            uint32_t op[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float2 o = tc::mul2(gn2, x[i]);
-              const float2 nn = tc::mul2(keep2, x[i]);
-              op[i] = tc::pack_bf16x2(o.x, o.y);
-              d[2 * i] = __float_as_uint(nn.x);
-              d[2 * i + 1] = __float_as_uint(nn.y);
-            }
-            tc::tmem_st32(d_addr, d);
-            tc::tmem_st16(tbase + lane_off + 256u + 64u * k + (col0 + cc) / 2, op);
-          }
+          tc::tmem_st32(d_addr, d);
+          tc::tmem_st16(tbase + lane_off + 256u + 64u * k + col0 / 2, op);
         }
         tc::tmem_wait_st();
         tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0 && !last) tc::mbar_arrive(&op_ready[k]);
       }
       __syncwarp();
-      if (lane == 0) {
-        if (act && !last) tc::mbar_arrive(&op_ready[k]);
-        tc::mbar_arrive(&empty[st]);
-      }
+      if (lane == 0) tc::mbar_arrive(&empty[st]);
     }
   }
   tc::tc_fence_before();
