@@ -13,6 +13,7 @@ from ._hla import (  # noqa: F401
     gdn_chunk_transitions,
     hla_decode_step,
     hla_decode_step_static,
+    hla_check_bounded_wait,
     hla_device_status,
     hla_prefill,
     hla_profile_enable,

@@ -69,6 +69,7 @@ _SIGS = {
     "hla_decode_step_static": ([ctypes.POINTER(HlaConfig), ctypes.POINTER(HlaCache), _P, _P, _P, _P, _P, _P, _P,
                                 _P, _P], ctypes.c_int),
     "hla_device_status": ([ctypes.c_int32, ctypes.POINTER(ctypes.c_uint32)], ctypes.c_int),
+    "hla_check_bounded_wait": ([ctypes.c_uint32, ctypes.c_int32, _P], ctypes.c_int),
     "hla_profile_enable": ([ctypes.c_int32], ctypes.c_int),
     "hla_profile_read": ([_P, _P, ctypes.c_int32], ctypes.c_int),
 }
@@ -212,6 +213,11 @@ def hla_device_status(clear: bool = True):
     code = ctypes.c_uint32(0)
     st = lib().hla_device_status(1 if clear else 0, ctypes.byref(code))
     return st, int(code.value)
+
+
+def hla_check_bounded_wait(limit_us: int, complete: bool, stream=None):
+    """Enqueue the library's bounded-wait check (see include/hla.h)."""
+    _check(lib().hla_check_bounded_wait(int(limit_us), 1 if complete else 0, _stream(stream)))
 
 
 def hla_profile_enable(on: bool = True):

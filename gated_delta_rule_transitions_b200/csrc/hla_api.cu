@@ -642,6 +642,14 @@ hla_status hla_profile_read(float* ms_out, int32_t* launches_out, int32_t reset)
   return HLA_OK;
 }
 
+hla_status hla_check_bounded_wait(uint32_t limit_us, int32_t complete, hla_stream_t stream) {
+  g_msg[0] = 0;
+  if (limit_us < 1 || limit_us > 100000) return fail(HLA_ERR_INVALID_ARG, "limit_us must be in [1, 100000]");
+  HLA_CUDA(hla::launch_wait_check((uint64_t)limit_us * 1000ull, complete != 0, (cudaStream_t)stream),
+           "bounded-wait check launch");
+  return HLA_OK;
+}
+
 hla_status hla_device_status(int32_t clear, uint32_t* code_out) {
   g_msg[0] = 0;
   HLA_CUDA(cudaDeviceSynchronize(), "hla_device_status synchronize");
@@ -655,6 +663,8 @@ hla_status hla_device_status(int32_t clear, uint32_t* code_out) {
   HLA_CUDA(hla::read_error_word_transitions_tc(&w, clear != 0), "hla_device_status read");
   word |= w;
   HLA_CUDA(hla::read_error_word_readout_tc(&w, clear != 0), "hla_device_status read");
+  word |= w;
+  HLA_CUDA(hla::read_error_word_wait_check(&w, clear != 0), "hla_device_status read");
   word |= w;
   if (code_out) *code_out = word;
   if (word & (hla::kErrMbarTimeout | hla::kErrTmemAlloc))

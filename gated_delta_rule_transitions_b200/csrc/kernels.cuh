@@ -120,5 +120,7 @@ cudaError_t launch_readout_tc(const ReadoutArgs& r, const void* S_in_bf16, const
 cudaError_t read_error_word_transitions_tc(unsigned int* out, bool clear);
 cudaError_t read_error_word_readout_tc(unsigned int* out, bool clear);
 cudaError_t read_error_word_decode_stream(unsigned int* out, bool clear);
+cudaError_t read_error_word_wait_check(unsigned int* out, bool clear);
+cudaError_t launch_wait_check(uint64_t limit_ns, bool complete, cudaStream_t s);
 
 }  // namespace hla

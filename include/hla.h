@@ -242,6 +242,17 @@ hla_status hla_decode_step_static(const hla_config* cfg, hla_cache* cache, const
 hla_status hla_device_status(int32_t clear, uint32_t* code_out);
 
 /*
+ * Bounded-wait check (diagnostic).  Enqueues on stream one kernel that waits on an
+ * mbarrier with the library's bounded wait.  complete != 0: the barrier is
+ * completed before the wait, which returns at once.  complete == 0: nothing
+ * completes it, so the wait gives up after limit_us microseconds, records the
+ * timeout in the device error word and the kernel exits normally; the next
+ * hla_device_status returns HLA_ERR_TIMEOUT (code bit 0x1) and the context stays
+ * usable.  limit_us in [1, 100000].  Errors: INVALID_ARG, CUDA.
+ */
+hla_status hla_check_bounded_wait(uint32_t limit_us, int32_t complete, hla_stream_t stream);
+
+/*
  * Stage timing (tracing).  While enabled, hla_prefill and hla_decode_step record a
  * pair of CUDA events on the caller's stream around each stage below and count the
  * kernels each stage launches.  hla_profile_read synchronises the device, writes

@@ -159,3 +159,9 @@ def test_static_decode_rejects_scratch_beyond_its_array(hla):
     st = hla.lib().hla_decode_step_static(ctypes.byref(c), ctypes.byref(cache), P, P, P, P, P, None, None, P,
                                           None)
     assert st == hla.HLA_ERR_WORKSPACE and "static array" in hla.last_error()
+
+
+def test_bounded_wait_check_limit_checked_on_host(hla):
+    for bad in (0, 100001):
+        st = hla.lib().hla_check_bounded_wait(bad, 0, None)
+        assert st == hla.HLA_ERR_INVALID_ARG and "limit_us" in hla.last_error()

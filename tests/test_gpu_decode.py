@@ -108,3 +108,40 @@ def test_decode_cache_full_is_reported(hla):
     assert st == hla.HLA_ERR_WORKSPACE and code & 4
     st, code = hla.hla_device_status(clear=True)
     assert st == 0 and code == 0
+
+
+def test_full_size_decode_sampled(hla):
+    """The 32K decode step at full size (64 sequences x 32768-token contexts, 512
+    cached chunks per head, H=16, d=128, bf16, threshold 0.05): the cache is built
+    as bench.py builds it, one decode step runs over all sequences, and two
+    (sequence, head) outputs are compared with the oracle's decode head built from
+    the same context (definition form: forward composition over all 512 chunks)."""
+    import os
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+    w = syn.DECODE_32K
+    max_chunks = w.T // w.C + 1
+    cache, ctx = bench.build_decode_cache(hla, syn, torch, w, max_chunks, group=8)
+    try:
+        dcfg = hla.make_config(w.B, w.H, 1, w.C, w.d, w.dtype, w.gate_mode, w.tau, w.bias, w.thr)
+        tok = syn.make_decode_tokens(w, 1)[0]
+        g = {k: v.cuda().contiguous() for k, v in tok.items()}
+        o = torch.empty_like(g["q"])
+        hla.hla_decode_step(dcfg, cache, g["q"], g["k"], g["v"], g["alpha"], g["beta"], o)
+        torch.cuda.synchronize()
+        st, code = hla.hla_device_status()
+        assert st == hla.HLA_OK, code
+        n = cache.view("n_chunks", (w.B,), torch.int32).cpu()
+        m = cache.view("m_partial", (w.B,), torch.int32).cpu()
+        assert torch.all(n == w.T // w.C) and torch.all(m == 1)
+        for (b, h) in ((0, 0), (1, 9)):
+            f = lambda name: P.np64(ctx[name][b, :, h])
+            head = ho.HlaDecodeHead.from_prefill(f("q"), f("k"), f("v"), f("alpha"), f("beta"), w.C, w.tau,
+                                                 w.bias, w.thr, w.gate_mode)
+            ref = head.step(P.np64(tok["q"][b, h]), P.np64(tok["k"][b, h]), P.np64(tok["v"][b, h]),
+                            float(tok["alpha"][b, h]), float(tok["beta"][b, h]))
+            assert P.rel_l2(P.np64(o[b, h]), ref) <= P.TOL_BF16_RELL2
+    finally:
+        del cache
+        torch.cuda.empty_cache()
