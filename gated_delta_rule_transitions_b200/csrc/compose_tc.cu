@@ -44,6 +44,7 @@ constexpr uint32_t kIdesc = tc::idesc_bf16_f32(128, 128, /*a_mn=*/0, /*b_mn=*/1)
 struct ComposeTcArgs {
   int BH, N;
   int head_major;
+  const int32_t* order;  // [BH, N] query chunks in pairing order, or null (descending)
   long ab_chunk_stride;
   const int32_t* act_idx;
   const float* act_g;
@@ -110,6 +111,46 @@ struct StepInfo {
   float gn[2]; // gates at each chain's next active step (0 if none)
 };
 
+// Pairing order for the composition when chunks may be skipped.  Per (b, h) the query
+// chunks are sorted by their first active chunk, then the longer active list first,
+// then the later chunk first; consecutive entries are paired into one CTA.  Chunks
+// whose lists start at the same chunk share most of their active chunks, so one
+// A_j/B_j tile in the ring serves both chains.  Bitonic sort of 64-bit keys in
+// shared memory, P = power of two >= N <= 4096.
+__global__ void __launch_bounds__(1024) chain_order_kernel(const int32_t* __restrict__ act_idx,
+                                                           const int32_t* __restrict__ act_cnt, int N, int P,
+                                                           int32_t* __restrict__ order) {
+  extern __shared__ unsigned long long keys[];
+  const int bh = blockIdx.x;
+  for (int i = threadIdx.x; i < P; i += blockDim.x) {
+    unsigned long long k = ~0ull;
+    if (i < N) {
+      const long row = (long)bh * N + i;
+      const int cnt = act_cnt[row];
+      const int first = cnt > 0 ? act_idx[row * N] : N;
+      k = ((unsigned long long)first << 40) | ((unsigned long long)(N - cnt) << 20) | (unsigned long long)(N - 1 - i);
+    }
+    keys[i] = k;
+  }
+  __syncthreads();
+  for (int size = 2; size <= P; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int t = threadIdx.x; t < P / 2; t += blockDim.x) {
+        const int lo = 2 * stride * (t / stride) + (t % stride);
+        const int hi = lo + stride;
+        const bool up = (lo & size) == 0;
+        const unsigned long long x = keys[lo], y = keys[hi];
+        if ((x > y) == up) {
+          keys[lo] = y;
+          keys[hi] = x;
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = threadIdx.x; i < N; i += blockDim.x) order[(long)bh * N + i] = N - 1 - (int)(keys[i] & 0xFFFFFu);
+}
+
 template <bool kScan>
 __global__ void __launch_bounds__(kThreads, 1)
     compose_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -136,7 +177,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int pair = kScan ? 0 : (a.head_major ? blockIdx.x % npairs : blockIdx.x / a.BH);
   const int bh = kScan ? blockIdx.x : (a.head_major ? blockIdx.x / npairs : blockIdx.x % a.BH);
   // scan mode: chain 0 is the head's running state (its S_in rows move with j), chain 1 idles
-  const int chains[2] = {kScan ? 0 : a.N - 1 - 2 * pair, kScan ? -1 : a.N - 2 - 2 * pair};
+  int chains[2];
+  if (kScan) {
+    chains[0] = 0;
+    chains[1] = -1;
+  } else if (a.order != nullptr) {
+    // query chunks paired by the order kernel (shared active lists)
+    const int32_t* o = a.order + (long)bh * a.N;
+    chains[0] = o[2 * pair];
+    chains[1] = 2 * pair + 1 < a.N ? o[2 * pair + 1] : -1;
+  } else {
+    chains[0] = a.N - 1 - 2 * pair;
+    chains[1] = a.N - 2 - 2 * pair;
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -430,6 +483,18 @@ cudaError_t launch_compose_tc(const ComposeArgs& c, bool scan, cudaStream_t s) {
   a.act_cnt = c.act_cnt;
   a.S_in = (__nv_bfloat16*)c.S_in;
   a.head_major = c.sparse ? 1 : 0;
+  a.order = nullptr;
+  if (!scan && c.sparse && c.order != nullptr && c.N <= 4096) {
+    int P = 1;
+    while (P < c.N) P <<= 1;
+    const size_t osmem = (size_t)P * sizeof(unsigned long long);
+    e = cudaFuncSetAttribute(chain_order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)osmem);
+    if (e != cudaSuccess) return e;
+    chain_order_kernel<<<a.BH, 1024, osmem, s>>>(c.act_idx, c.act_cnt, c.N, P, c.order);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    a.order = c.order;
+  }
   const size_t smem = 1024 + kStages * kStageBytes + 512;
   if (scan) {
     e = cudaFuncSetAttribute(compose_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

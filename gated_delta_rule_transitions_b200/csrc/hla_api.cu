@@ -78,7 +78,7 @@ float gate_scale(int d) { return (float)(1.0 / std::sqrt((double)d)); }
 
 // Prefill workspace layout.
 struct PrefillWs {
-  size_t rq, rk, act_idx, act_g, act_cnt, A, Bm, Wb, Ub, ell, S_in, total;
+  size_t rq, rk, act_idx, act_g, act_cnt, order, A, Bm, Wb, Ub, ell, S_in, total;
 };
 
 PrefillWs prefill_layout(const hla_config* c) {
@@ -97,6 +97,7 @@ PrefillWs prefill_layout(const hla_config* c) {
   w.act_idx = take(B * H * N * N * 4);
   w.act_g = take(B * H * N * N * 4);
   w.act_cnt = take(B * H * N * 4);
+  w.order = take(B * H * N * 4);
   w.A = take(B * H * Nc * d * d * esize(c->dtype));
   w.Bm = take(B * H * Nc * d * d * esize(c->dtype));
   w.Wb = take(B * H * N * C * d * 4);
@@ -428,6 +429,7 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
   c.act_cnt = act_cnt;
   c.S_in = (float*)(ws + w.S_in);
   c.sparse = cfg->skip_threshold > 0.0f;
+  c.order = (int32_t*)(ws + w.order);
   {
     StageScope _sc(HLA_STAGE_COMPOSE, s, 1);
     // every gate one (and kept): the composition is a plain prefix scan over the chunks

@@ -58,6 +58,7 @@ struct ComposeArgs {
   const int32_t* act_cnt; // [B,H,N]
   float* S_in;            // [B,H,N,d,d] fp32
   bool sparse;            // chunks may be skipped (threshold > 0)
+  int32_t* order;         // [B,H,N] scratch for the pairing order (tensor-core path), or null
 };
 
 struct ReadoutArgs {
