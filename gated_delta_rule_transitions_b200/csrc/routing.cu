@@ -131,17 +131,35 @@ __global__ void __launch_bounds__(256) gates_tiled_kernel(GatesArgs a) {
   const route::Consts K = route::make_consts();
   const float* rq = a.rq + (size_t)bh * a.N * D;
   const float* rk = a.rk + (size_t)bh * a.N * D;
-  for (int e = tid; e < TI * D; e += 256) {
-    const int r = e / D, c = e - r * D;
-    rqT[c][r] = (i0 + r < a.N) ? rq[(size_t)(i0 + r) * D + c] : 0.0f;
+  // Tiles are channel-major with their float4 row groups XOR-swizzled by the channel
+  // (group g of channel c at slot g ^ (c % 16)): the fill below (one channel, four
+  // consecutive rows per thread, one 16-byte store) and the float4 reads of the dot
+  // products are both free of bank conflicts.
+  for (int e = tid; e < (TI / 4) * D; e += 256) {
+    const int g = e / D, c = e - g * D;
+    float4 v;
+    float* vp = &v.x;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + 4 * g + u;
+      vp[u] = i < a.N ? rq[(size_t)i * D + c] : 0.0f;
+    }
+    *(float4*)&rqT[c][(g ^ (c & 15)) << 2] = v;
   }
   if (tid < TI) cnt_s[tid] = 0;
   const int i_last = min(a.N, i0 + TI) - 1;
   for (int j0 = 0; j0 < i_last; j0 += TJ) {
     __syncthreads();
-    for (int e = tid; e < TJ * D; e += 256) {
-      const int r = e / D, c = e - r * D;
-      rkT[c][r] = (j0 + r < a.N) ? rk[(size_t)(j0 + r) * D + c] : 0.0f;
+    for (int e = tid; e < (TJ / 4) * D; e += 256) {
+      const int g = e / D, c = e - g * D;
+      float4 v;
+      float* vp = &v.x;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = j0 + 4 * g + u;
+        vp[u] = j < a.N ? rk[(size_t)j * D + c] : 0.0f;
+      }
+      *(float4*)&rkT[c][(g ^ (c & 15)) << 2] = v;
     }
     __syncthreads();
     float acc[4][4];
@@ -151,8 +169,8 @@ __global__ void __launch_bounds__(256) gates_tiled_kernel(GatesArgs a) {
       for (int w = 0; w < 4; ++w) acc[u][w] = 0.0f;
 #pragma unroll 4
     for (int c = 0; c < D; ++c) {
-      const float4 q4 = *(const float4*)&rqT[c][ty * 4];
-      const float4 k4 = *(const float4*)&rkT[c][tx * 4];
+      const float4 q4 = *(const float4*)&rqT[c][(ty ^ (c & 15)) << 2];
+      const float4 k4 = *(const float4*)&rkT[c][(tx ^ (c & 15)) << 2];
       const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
       const float kv[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
