@@ -183,6 +183,38 @@ class StageScope {
   bool on_ = false;
 };
 
+// ---- side stream ---------------------------------------------------------------
+// hla_prefill runs the routing stage (pools, gates, active lists) on a per-device
+// side stream, forked from and joined back to the caller's stream by events, so it
+// overlaps the chunk transitions: the two read only the caller's inputs and write
+// disjoint parts of the workspace.  Created on first use on each device.
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+constexpr int kMaxDevices = 64;
+std::mutex g_side_mu;
+SideStream g_side[kMaxDevices];
+
+hla_status side_stream(SideStream** out) {
+  int dev = -1;
+  HLA_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(HLA_ERR_UNSUPPORTED, "device ordinal %d beyond %d", dev, kMaxDevices);
+  SideStream& ss = g_side[dev];
+  if (ss.s == nullptr) {
+    cudaStream_t st = nullptr;
+    cudaEvent_t f = nullptr, j = nullptr;
+    HLA_CUDA(cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking), "side stream create");
+    HLA_CUDA(cudaEventCreateWithFlags(&f, cudaEventDisableTiming), "side stream event create");
+    HLA_CUDA(cudaEventCreateWithFlags(&j, cudaEventDisableTiming), "side stream event create");
+    ss.fork = f;
+    ss.join = j;
+    ss.s = st;
+  }
+  *out = &ss;
+  return HLA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -389,8 +421,16 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
   int32_t* act_idx = (int32_t*)(ws + w.act_idx);
   float* act_g = (float*)(ws + w.act_g);
   int32_t* act_cnt = (int32_t*)(ws + w.act_cnt);
+  // routing on the side stream, overlapping the transitions below; joined before the
+  // composition (the fork/join pair is enqueued under one lock)
+  std::unique_lock<std::mutex> side_lock(g_side_mu);
+  SideStream* side = nullptr;
+  HLA_TRY(side_stream(&side));
+  HLA_CUDA(cudaEventRecord(side->fork, s), "side stream fork");
+  HLA_CUDA(cudaStreamWaitEvent(side->s, side->fork, 0), "side stream fork");
   HLA_TRY(routing_impl(cfg, qr, kr, rq, (cfg->gate_mode == HLA_GATES_ROUTED || cache_out) ? rk : nullptr,
-                       user_gates, act_idx, act_g, act_cnt, gates_out, active_idx_out, active_cnt_out, s));
+                       user_gates, act_idx, act_g, act_cnt, gates_out, active_idx_out, active_cnt_out, side->s));
+  HLA_CUDA(cudaEventRecord(side->join, side->s), "side stream join");
   // transitions of every chunk (A/B of complete chunks into the cache or workspace)
   hla::TransArgs t{};
   t.B = cfg->B;
@@ -415,6 +455,8 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
     else
       HLA_CUDA(hla::launch_transitions(t, s), "transitions launch");
   }
+  HLA_CUDA(cudaStreamWaitEvent(s, side->join, 0), "side stream join");
+  side_lock.unlock();
   hla::ComposeArgs c{};
   c.B = cfg->B;
   c.H = cfg->H;
