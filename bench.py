@@ -80,7 +80,7 @@ def whole_job_rate(units_per_rank, ms_max, world):
 #   compose: full-size launch of the dense 0.8B-like prefill (compose_tc_prefill_0p8b.md)
 #   decode_main: see below
 NCU_TRAFFIC = {
-    "compose": (2.0406e9, {"compose_tc.cu": "fe94edd5ca26524f", "tc_common.cuh": "4e1419f23237b542"}),
+    "compose": (2.0436e9, {"compose_tc.cu": "9feae23bf70ea63b", "tc_common.cuh": "4e1419f23237b542"}),
     # decode_main: capture of a 4-sequence decode (64 of the 1024 (sequence, head)
     # streams), scaled by 16; per stream it equals the algorithmic bytes
     # (decode_stream_decode_32k.md)

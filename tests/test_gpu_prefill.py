@@ -82,6 +82,21 @@ def test_bf16_planted_sparse(hla):
         assert 0 < sum(kept) < sum(range(len(kept)))
 
 
+def test_bf16_planted_sparse_odd_chunks(hla):
+    """Skipping with an odd number of query chunks (one unpaired chain in the pairing
+    order), several sequences and heads, and a ragged last chunk."""
+    w = syn.SPARSE_LONG.with_(B=2, H=3, T=64 * 20 + 5, topics=5)
+    inp = P.gpu_inputs(w)
+    o, gates, aidx, acnt = P.run_prefill(hla, w, inp)
+    ref, res = _oracle_all(w, inp)
+    assert P.rel_l2(P.np64(o), ref) <= P.TOL_BF16_RELL2
+    skipped = 0
+    for (b, h), r in res.items():
+        P.check_routing_exact(r, gates, aidx, acnt, b, h)
+        skipped += sum(i - len(a) for i, a in enumerate(r.active))
+    assert skipped > 0
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_gates_one_is_native_gdn(hla, dtype):
     w = syn.GDN_REDUCTION.with_(B=2, H=2, T=64 * 4 + 9, dtype=dtype, d=64 if dtype == "f32" else 128)
