@@ -224,26 +224,12 @@ def build_decode_cache(hla, syn, torch, w, max_chunks, group=8):
     cache = hla.Cache(cfg, max_chunks)
     gcfg = hla.make_config(group, w.H, w.T, w.C, w.d, w.dtype, "zero", w.tau, w.bias, w.thr)
     ws = torch.empty(hla.prefill_workspace_bytes(gcfg), dtype=torch.uint8, device="cuda")
-    es = 2 if w.dtype == "bf16" else 4
-    per_b = {  # bytes per sequence of each buffer
-        "A": w.H * max_chunks * w.d * w.d * es, "Bm": w.H * max_chunks * w.d * w.d * es,
-        "rk": w.H * max_chunks * w.d * 4, "buf_k": w.H * w.C * w.d * es, "buf_v": w.H * w.C * w.d * es,
-        "buf_qr": w.H * w.C * w.d * es, "buf_kr": w.H * w.C * w.d * es, "buf_alpha": w.H * w.C * 4,
-        "buf_beta": w.H * w.C * 4, "n_chunks": 4, "m_partial": 4}
     first_ctx = None
     for b0 in range(0, w.B, group):
         ctx = syn.make_context_group(w, b0, group, device="cuda")
         if b0 == 0:
             first_ctx = {k: v[:2].clone() for k, v in ctx.items()}
-        sub = hla.HlaCache()
-        ctypes_fields = [f[0] for f in hla.HlaCache._fields_]
-        for f in ctypes_fields:
-            setattr(sub, f, getattr(cache.struct, f))
-        sub.B = group
-        for f, nb in per_b.items():
-            setattr(sub, f, getattr(cache.struct, f) + b0 * nb)
-        holder = type("SubCache", (), {})()
-        holder.struct = sub
+        holder = cache.slice(b0, group)
         o = torch.empty_like(ctx["q"])
         hla.hla_prefill(gcfg, ctx["q"], ctx["k"], ctx["v"], ctx["alpha"], ctx["beta"], o, cache=holder,
                         workspace=ws)

@@ -58,6 +58,8 @@ _SIGS = {
     "hla_cache_bytes": ([ctypes.POINTER(HlaConfig), ctypes.c_int32], ctypes.c_size_t),
     "hla_cache_init": ([ctypes.POINTER(HlaConfig), ctypes.c_int32, _P, ctypes.c_size_t, ctypes.POINTER(HlaCache), _P],
                        ctypes.c_int),
+    "hla_cache_slice": ([ctypes.POINTER(HlaCache), ctypes.c_int32, ctypes.c_int32, ctypes.POINTER(HlaCache)],
+                        ctypes.c_int),
     "hla_prefill_workspace_bytes": ([ctypes.POINTER(HlaConfig)], ctypes.c_size_t),
     "hla_decode_workspace_bytes": ([ctypes.POINTER(HlaConfig), ctypes.c_int32], ctypes.c_size_t),
     "gdn_chunk_transitions": ([ctypes.POINTER(HlaConfig), _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
@@ -142,6 +144,15 @@ def decode_workspace_bytes(cfg: HlaConfig, max_chunks: int) -> int:
     return int(lib().hla_decode_workspace_bytes(ctypes.byref(cfg), max_chunks))
 
 
+class CacheSlice:
+    """Sequences [b0, b0 + nb) of a Cache (see Cache.slice)."""
+
+    def __init__(self):
+        self.struct = HlaCache()
+        self.parent = None
+        self.max_chunks = 0
+
+
 class Cache:
     """A decode cache: one caller-owned device block plus the C struct of views."""
 
@@ -155,6 +166,14 @@ class Cache:
                                     ctypes.byref(self.struct), _stream(stream)))
         self.cfg = cfg
         self.max_chunks = max_chunks
+
+    def slice(self, b0: int, nb: int):
+        """The cache of sequences [b0, b0 + nb) (shares this cache's memory)."""
+        sub = CacheSlice()
+        sub.parent = self
+        sub.max_chunks = self.max_chunks
+        _check(lib().hla_cache_slice(ctypes.byref(self.struct), b0, nb, ctypes.byref(sub.struct)))
+        return sub
 
     def view(self, field: str, shape, dtype):
         """Torch view of one cache buffer (for tests and inspection)."""

@@ -141,9 +141,12 @@ hla_status check_cache(const hla_config* c, const hla_cache* k) {
   if (k->B != c->B || k->H != c->H || k->C != c->C || k->d != c->dk || k->dtype != c->dtype)
     return fail(HLA_ERR_INVALID_ARG, "cache was initialised for a different config");
   if (k->max_chunks <= 0) return fail(HLA_ERR_INVALID_ARG, "cache max_chunks must be positive");
-  const void* ps[] = {k->A, k->Bm, k->rk, k->buf_k, k->buf_v, k->buf_qr, k->buf_kr,
-                      k->buf_alpha, k->buf_beta, k->n_chunks, k->m_partial};
+  const void* ps[] = {k->A, k->Bm, k->rk, k->buf_k, k->buf_v, k->buf_qr, k->buf_kr, k->buf_alpha, k->buf_beta};
   for (const void* p : ps) HLA_TRY(need_ptr(p, "cache buffer"));
+  // the per-sequence counters are read and written as single int32 values, so a
+  // slice starting at any sequence is valid
+  for (const int32_t* p : {k->n_chunks, k->m_partial})
+    if (p == nullptr || ((uintptr_t)p & 3u) != 0) return fail(HLA_ERR_INVALID_ARG, "cache counters NULL or misaligned");
   return HLA_OK;
 }
 
@@ -257,6 +260,34 @@ hla_status hla_cache_init(const hla_config* cfg, int32_t max_chunks, void* mem, 
   c.m_partial = (int32_t*)(base + L.m);
   HLA_CUDA(cudaMemsetAsync(base + L.n, 0, L.total - L.n, (cudaStream_t)stream), "hla_cache_init memset");
   *out = c;
+  return HLA_OK;
+}
+
+hla_status hla_cache_slice(const hla_cache* cache, int32_t b0, int32_t nb, hla_cache* out) {
+  g_msg[0] = 0;
+  if (cache == nullptr || out == nullptr) return fail(HLA_ERR_INVALID_ARG, "cache and out must not be NULL");
+  if (cache->B <= 0 || cache->H <= 0 || cache->max_chunks <= 0 || cache->d <= 0 || cache->C <= 0)
+    return fail(HLA_ERR_INVALID_ARG, "cache is not initialised");
+  if (b0 < 0 || nb < 1 || (int64_t)b0 + nb > cache->B)
+    return fail(HLA_ERR_INVALID_ARG, "sequences [%d, %d) outside the cache's %d", b0, b0 + nb, cache->B);
+  // per-sequence bytes of each buffer (the layout of cache_layout, sequence-major)
+  const size_t H = cache->H, d = cache->d, C = cache->C, mc = cache->max_chunks;
+  const size_t es = esize(cache->dtype);
+  const size_t off = (size_t)b0;
+  hla_cache v = *cache;
+  v.B = nb;
+  v.A = (char*)cache->A + off * H * mc * d * d * es;
+  v.Bm = (char*)cache->Bm + off * H * mc * d * d * es;
+  v.rk = (float*)((char*)cache->rk + off * H * mc * d * 4);
+  v.buf_k = (char*)cache->buf_k + off * H * C * d * es;
+  v.buf_v = (char*)cache->buf_v + off * H * C * d * es;
+  v.buf_qr = (char*)cache->buf_qr + off * H * C * d * es;
+  v.buf_kr = (char*)cache->buf_kr + off * H * C * d * es;
+  v.buf_alpha = (float*)((char*)cache->buf_alpha + off * H * C * 4);
+  v.buf_beta = (float*)((char*)cache->buf_beta + off * H * C * 4);
+  v.n_chunks = cache->n_chunks + off;
+  v.m_partial = cache->m_partial + off;
+  *out = v;
   return HLA_OK;
 }
 

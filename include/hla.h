@@ -35,7 +35,8 @@
  *   - Every pointer argument named as device memory is a CUDA device pointer owned
  *     by the caller.  The library never allocates device memory: callers query
  *     the workspace and cache sizes and pass buffers in.
- *   - Every device pointer must be 16-byte aligned (HLA_ERR_INVALID_ARG otherwise).
+ *   - Every device pointer must be 16-byte aligned (HLA_ERR_INVALID_ARG otherwise),
+ *     except the cache's n_chunks / m_partial counters (4-byte aligned).
  *   - Layouts are dense row-major:
  *       q, k, v, q_route, k_route, o : [B, T, H, d]      (dtype)
  *       alpha, beta                   : [B, T, H]         float32, alpha in (0,1], beta in [0,1]
@@ -135,6 +136,13 @@ size_t hla_cache_bytes(const hla_config* cfg, int32_t max_chunks);
  * CUDA. */
 hla_status hla_cache_init(const hla_config* cfg, int32_t max_chunks, void* mem, size_t bytes,
                           hla_cache* out, hla_stream_t stream);
+
+/* View of sequences [b0, b0 + nb) of an initialised cache: *out gets B = nb and
+ * every pointer advanced to sequence b0 (the buffers are sequence-major).  Host
+ * only, nothing is launched.  Lets sequences of different prompt lengths be
+ * prefilled one at a time into one cache, after which hla_decode_step advances
+ * them together from their own positions.  Errors: INVALID_ARG. */
+hla_status hla_cache_slice(const hla_cache* cache, int32_t b0, int32_t nb, hla_cache* out);
 
 /* Workspace bytes that hla_prefill needs for cfg (0 for an unsupported config). */
 size_t hla_prefill_workspace_bytes(const hla_config* cfg);

@@ -165,3 +165,26 @@ def test_bounded_wait_check_limit_checked_on_host(hla):
     for bad in (0, 100001):
         st = hla.lib().hla_check_bounded_wait(bad, 0, None)
         assert st == hla.HLA_ERR_INVALID_ARG and "limit_us" in hla.last_error()
+
+
+def test_cache_slice_offsets_follow_the_sequence_major_layout(hla):
+    """hla_cache_slice advances every buffer by b0 sequences of the layout that
+    include/hla.h documents ([B, H, max_chunks, d, d] A/Bm, [B, H, max_chunks, d]
+    key pools, [B, H, C, d] / [B, H, C] open-chunk buffers, [B] counters)."""
+    c = hla.HlaCache()
+    c.B, c.H, c.C, c.d, c.dtype, c.max_chunks = 4, 2, 64, 128, 1, 3
+    fields = ("A", "Bm", "rk", "buf_k", "buf_v", "buf_qr", "buf_kr", "buf_alpha", "buf_beta", "n_chunks",
+              "m_partial")
+    for i, f in enumerate(fields):
+        setattr(c, f, (i + 1) << 32)
+    out = hla.HlaCache()
+    assert hla.lib().hla_cache_slice(ctypes.byref(c), 2, 2, ctypes.byref(out)) == hla.HLA_OK
+    per_seq = {"A": 2 * 3 * 128 * 128 * 2, "Bm": 2 * 3 * 128 * 128 * 2, "rk": 2 * 3 * 128 * 4,
+               "buf_k": 2 * 64 * 128 * 2, "buf_v": 2 * 64 * 128 * 2, "buf_qr": 2 * 64 * 128 * 2,
+               "buf_kr": 2 * 64 * 128 * 2, "buf_alpha": 2 * 64 * 4, "buf_beta": 2 * 64 * 4, "n_chunks": 4,
+               "m_partial": 4}
+    assert out.B == 2 and out.H == 2 and out.max_chunks == 3
+    for i, f in enumerate(fields):
+        assert getattr(out, f) == ((i + 1) << 32) + 2 * per_seq[f], f
+    for b0, nb in ((-1, 1), (0, 0), (3, 2), (4, 1)):
+        assert hla.lib().hla_cache_slice(ctypes.byref(c), b0, nb, ctypes.byref(out)) == hla.HLA_ERR_INVALID_ARG

@@ -93,6 +93,56 @@ def test_decode_chain_matches_oracle(hla, dtype, d, mode, thr, route):
             assert np.array_equal(rk[b, h, j].view(np.uint32), st_.rk[j].view(np.uint32))
 
 
+@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("f32", 64)])
+def test_decode_ragged_positions(hla, dtype, d):
+    """Sequences at different positions in one cache: each is prefilled on its own
+    (prompts of 202 and 370 tokens) into its slice of the cache, then chained decode
+    steps advance both together; they close chunks at different steps.  Every output
+    is compared with that sequence's oracle decode head."""
+    lens = [64 * 3 + 10, 64 * 5 + 50]
+    steps = 60
+    base = syn.DECODE_32K.with_(B=1, H=2, dtype=dtype, d=d, thr=0.05, bias=-0.5, route="spread")
+    cfg2 = hla.make_config(2, base.H, max(lens), 64, d, dtype, "routed", base.tau, base.bias, base.thr)
+    cache = hla.Cache(cfg2, max_chunks=8)
+    heads = {}
+    for b, T_b in enumerate(lens):
+        w = base.with_(T=T_b, seed=11 + b)
+        inp = P.gpu_inputs(w)
+        P.run_prefill(hla, w, inp, cache=cache.slice(b, 1))
+        for h in range(w.H):
+            f = lambda n: None if inp.get(n) is None else inp[n][0, :, h]
+            heads[(b, h)] = ho.HlaDecodeHead.from_prefill(
+                P.np64(f("q")), P.np64(f("k")), P.np64(f("v")), P.np64(f("alpha")), P.np64(f("beta")), 64,
+                w.tau, w.bias, w.thr, "routed", P.np32(f("q_route")), P.np32(f("k_route")))
+    dcfg = hla.make_config(2, base.H, 1, 64, d, dtype, "routed", base.tau, base.bias, base.thr)
+    toks = syn.make_decode_tokens(base.with_(B=2), steps)
+    routes = _route_tokens(2, base.H, d, steps, 91, syn.torch_dtype(base))
+    got, ref = [], []
+    for s_, tk in enumerate(toks):
+        g = {k: v.cuda().contiguous() for k, v in tk.items()}
+        qr, kr = routes[s_]
+        o = torch.empty_like(g["q"])
+        hla.hla_decode_step(dcfg, cache, g["q"], g["k"], g["v"], g["alpha"], g["beta"], o, q_route=qr.cuda(),
+                            k_route=kr.cuda())
+        torch.cuda.synchronize()
+        o = P.np64(o)
+        for (b, h), st_ in heads.items():
+            got.append(o[b, h])
+            ref.append(st_.step(P.np64(tk["q"][b, h]), P.np64(tk["k"][b, h]), P.np64(tk["v"][b, h]),
+                                float(tk["alpha"][b, h]), float(tk["beta"][b, h]), P.np32(qr[b, h]),
+                                P.np32(kr[b, h])))
+    got, ref = np.stack(got), np.stack(ref)
+    if dtype == "f32":
+        assert np.abs(got - ref).max() <= P.TOL_F32_MAXABS
+    else:
+        assert P.rel_l2(got, ref) <= P.TOL_BF16_RELL2
+    st, code = hla.hla_device_status()
+    assert st == 0 and code == 0
+    n = cache.view("n_chunks", (2,), torch.int32).cpu().tolist()
+    m = cache.view("m_partial", (2,), torch.int32).cpu().tolist()
+    assert n == [(T + steps) // 64 for T in lens] and m == [(T + steps) % 64 for T in lens]
+
+
 def test_decode_cache_full_is_reported(hla):
     w = syn.DECODE_32K.with_(B=1, H=1, T=64 * 2 + 63, dtype="f32", d=64)
     inp = P.gpu_inputs(w)
