@@ -216,13 +216,14 @@ class ClockSampler:
 # our arm
 # ----------------------------------------------------------------------------------
 
-def build_decode_cache(hla, syn, torch, w, max_chunks, group=8):
+def build_decode_cache(hla, syn, torch, w, max_chunks, group=8, cache_format="dense"):
     """Fill a decode cache for w.B sequences of w.T-token contexts through the public
     API: hla_prefill with every earlier-chunk weight 0 writes the cache (A/B/key pools
     do not depend on gates) without the quadratic composition."""
-    cfg = hla.make_config(w.B, w.H, w.T, w.C, w.d, w.dtype, "routed", w.tau, w.bias, w.thr)
+    cfg = hla.make_config(w.B, w.H, w.T, w.C, w.d, w.dtype, "routed", w.tau, w.bias, w.thr, cache_format=cache_format)
     cache = hla.Cache(cfg, max_chunks)
-    gcfg = hla.make_config(group, w.H, w.T, w.C, w.d, w.dtype, "zero", w.tau, w.bias, w.thr)
+    gcfg = hla.make_config(group, w.H, w.T, w.C, w.d, w.dtype, "zero", w.tau, w.bias, w.thr,
+                           cache_format=cache_format)
     ws = torch.empty(hla.prefill_workspace_bytes(gcfg), dtype=torch.uint8, device="cuda")
     first_ctx = None
     for b0 in range(0, w.B, group):
@@ -288,10 +289,14 @@ def run_ours(args):
         wd = wd.with_(B=B_, T=T_, name=f"decode_bf16_{B_}seq_ctx{T_}_H16_C64_d128_thr0.05")
     if args.skip_decode:
         wd = wd.with_(B=8, T=64 * 4, name="decode_skipped")
+    if args.decode_cache != "dense":
+        wd = wd.with_(name=f"{wd.name}_{args.decode_cache}_cache")
     max_chunks = wd.T // wd.C + 1
-    cache, ctx0 = build_decode_cache(hla, syn, torch, wd, max_chunks, group=min(8, wd.B))
+    cache, ctx0 = build_decode_cache(hla, syn, torch, wd, max_chunks, group=min(8, wd.B),
+                                     cache_format=args.decode_cache)
     torch.cuda.empty_cache()
-    dcfg = hla.make_config(wd.B, wd.H, 1, wd.C, wd.d, wd.dtype, wd.gate_mode, wd.tau, wd.bias, wd.thr)
+    dcfg = hla.make_config(wd.B, wd.H, 1, wd.C, wd.d, wd.dtype, wd.gate_mode, wd.tau, wd.bias, wd.thr,
+                           cache_format=args.decode_cache)
     dws = torch.empty(hla.decode_workspace_bytes(dcfg, max_chunks), dtype=torch.uint8, device="cuda")
     ntok = args.warmup + args.steps + 1
     toks_host = [{k: v.contiguous().pin_memory() for k, v in t.items()} for t in syn.make_decode_tokens(wd, ntok)]
@@ -399,7 +404,11 @@ def run_ours(args):
     comp_avg = comp_ms / max(comp_n, 1)
     comp_tf = flops_compose / (comp_avg * 1e-3) / 1e12 if comp_avg > 0 else None
     n_ctx = wd.T // wd.C
-    bytes_decode = wd.B * wd.H * (n_ctx * (2 * wd.d * wd.d * 2 + wd.d * 4))
+    if args.decode_cache == "factored":
+        per_chunk = 3 * wd.C * wd.d * 2 + (wd.C + 4) * 4   # K, Wb, Ub bf16 + scales
+    else:
+        per_chunk = 2 * wd.d * wd.d * 2                      # A, B bf16
+    bytes_decode = wd.B * wd.H * (n_ctx * (per_chunk + wd.d * 4))
     dmain_ms, dmain_n = stages["decode"]
     dmain_avg = dmain_ms / max(dmain_n, 1)
     dec_gbs = bytes_decode / (dmain_avg * 1e-3) / 1e9 if dmain_avg > 0 else None
@@ -433,10 +442,11 @@ def run_ours(args):
         "decode": {"value": whole_job_rate(tokens_dec, dec_ms, world), "unit": "tokens/s", "ms_per_step": dec_ms,
                    "roofline": {"kernel": "decode_main", "bound": "hbm", "achieved": dec_gbs, "peak": hbm_gbs,
                                 "unit": "GB/s", "frac": (dec_gbs / hbm_gbs) if dec_gbs else None,
-                                "traffic": ncu_traffic("decode_main"), "traffic_unit": "bytes per launch (ncu dram read+write)",
+                                "traffic": ncu_traffic("decode_main") if args.decode_cache == "dense" else None,
+                                "traffic_unit": "bytes per launch (ncu dram read+write)",
                                 "peak_source": f"{peak_src} HBM copy",
-                                "algorithmic": f"{bytes_decode:.4g} bytes per launch (512 active A_j/B_j bf16 + "
-                                               "key pools per sequence and head)"},
+                                "algorithmic": f"{bytes_decode:.4g} bytes per launch ({n_ctx} active chunks "
+                                               f"({args.decode_cache} cache) + key pools per sequence and head)"},
                    "e2e": {"value": whole_job_rate(tokens_dec, e2e_dec, world), "unit": "tokens/s",
                            "h2d_bytes_per_step": h2d_dec, "d2h_bytes_per_step": d2h_dec}},
         "stages_ms_per_step": {k: v[0] / args.steps for k, v in stages.items() if v[1]},
@@ -623,6 +633,8 @@ def main(argv=None):
     ap.add_argument("--decode-B", type=int, default=None, help="decode sequences (default 64)")
     ap.add_argument("--decode-ctx", type=int, default=None, help="decode context tokens (default 32768)")
     ap.add_argument("--skip-decode", action="store_true")
+    ap.add_argument("--decode-cache", choices=["dense", "factored"], default="dense",
+                    help="dense: A_j/B_j d x d (the metric's workload); factored: K_j, Wb_j, Ub_j per chunk")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

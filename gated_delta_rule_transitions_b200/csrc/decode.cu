@@ -227,6 +227,42 @@ __global__ void cache_fill_kernel(DecodeArgs c, FillArgs f) {
   }
 }
 
+// Prefill -> factored cache: K (from the input), Wb and Ub (bf16, from the
+// transition kernel's workspace output) and the scales of every complete chunk.
+// One CTA per (b, h, complete chunk), 16-byte copies.
+__global__ void __launch_bounds__(256) factor_fill_kernel(FactorFillArgs f) {
+  constexpr int C = 64, D = 128, PAD = C + 4;
+  const long chunk = blockIdx.x;
+  const int i = (int)(chunk % f.Nc);
+  const long bh = chunk / f.Nc;
+  const int b = (int)(bh / f.H), h = (int)(bh % f.H);
+  const uint4* wb = (const uint4*)f.Wb + (bh * f.N + i) * (C * D / 8);
+  const uint4* ub = (const uint4*)f.Ub + (bh * f.N + i) * (C * D / 8);
+  const long slot = bh * f.max_chunks + i;
+  uint4* kf = (uint4*)f.Kf + slot * (C * D / 8);
+  uint4* wf = (uint4*)f.Wf + slot * (C * D / 8);
+  uint4* uf = (uint4*)f.Uf + slot * (C * D / 8);
+  for (int e = threadIdx.x; e < C * D / 8; e += blockDim.x) {
+    const int t = e / (D / 8), c8 = e % (D / 8);
+    const long src = (((long)b * f.T + (long)i * C + t) * f.H + h) * (D / 8) + c8;
+    kf[e] = ((const uint4*)f.k)[src];
+    wf[e] = wb[e];
+    uf[e] = ub[e];
+  }
+  const float* ell = f.ell + (bh * f.N + i) * C;
+  float* dfo = f.df + slot * PAD;
+  const int tid = threadIdx.x;
+  if (tid < C) dfo[tid] = expf(ell[C - 1] - ell[tid]);
+  if (tid >= C && tid < PAD) dfo[tid] = tid == C ? expf(ell[C - 1]) : 0.0f;
+}
+
+cudaError_t launch_factor_fill(const FactorFillArgs& f, cudaStream_t s) {
+  const long blocks = (long)f.B * f.H * f.Nc;
+  if (blocks <= 0) return cudaSuccess;
+  factor_fill_kernel<<<(unsigned)blocks, 256, 0, s>>>(f);
+  return cudaGetLastError();
+}
+
 template <int D, typename Tio>
 static cudaError_t launch_main(const DecodeArgs& a, cudaStream_t s) {
   decode_main_kernel<D, Tio><<<a.B * a.H, D, 0, s>>>(a);
@@ -256,6 +292,10 @@ static cudaError_t launch_close(const DecodeArgs& a, cudaStream_t s) {
   t.n_chunks = 1;
   t.A = const_cast<void*>(a.A);
   t.Bm = const_cast<void*>(a.Bm);
+  t.Kf = a.Kf;  // factored cache: the transition kernel writes the factors instead of A/B
+  t.Wf = a.Wf;
+  t.Uf = a.Uf;
+  t.df = a.df;
   t.ab_chunk_stride = a.max_chunks;
   t.ab_chunk_offset = 0;
   t.close_m = a.m_partial;
@@ -271,6 +311,7 @@ static cudaError_t launch_close(const DecodeArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_decode_main(const DecodeArgs& a, cudaStream_t s) {
+  if (a.format == HLA_CACHE_FACTORED) return launch_decode_stream_factored(a, s);
   if (a.d == 128 && a.dtype == HLA_BF16) return launch_decode_stream(a, s);
   if (a.d == 128) return a.dtype == HLA_BF16 ? launch_main<128, __nv_bfloat16>(a, s) : launch_main<128, float>(a, s);
   return a.dtype == HLA_BF16 ? launch_main<64, __nv_bfloat16>(a, s) : launch_main<64, float>(a, s);

@@ -21,6 +21,8 @@ namespace hla {
 HLA_DEFINE_ERROR_WORD(decode_stream)
 
 cudaError_t make_tmap_rows128(CUtensorMap* m, const void* base, long rows);
+cudaError_t make_tmap_2d(CUtensorMap* m, const void* base, long inner, long rows, long row_stride_bytes,
+                         int box_inner, int box_rows);
 
 namespace {
 
@@ -40,6 +42,101 @@ __device__ __forceinline__ float blk_sum(float v, float* red) {
   return red[0] + red[1] + red[2] + red[3];
 }
 
+// Steps shared by the streaming kernels, run by the kCompute threads (thread = channel):
+// append the token to the open chunk, sweep the open chunk right to left (x = A_p q,
+// y0 = B_p q), pool the open chunk's route queries, gate every closed chunk and write
+// the ascending active list.  Returns the active count; x and y0 are this thread's.
+__device__ __forceinline__ int decode_prologue(const DecodeArgs& a, int bh, int n, int m, float* rq, float* red,
+                                             int* wcount, float& x, float& y0) {
+  const int tid = threadIdx.x;
+  const int C = a.C;
+  const int mp = m + 1;
+  int32_t* act_idx = a.act_idx + (long)bh * a.max_chunks;
+  float* act_g = a.act_g + (long)bh * a.max_chunks;
+  const long tok = (long)bh * kD + tid;
+  const long bslot = ((long)bh * C + m) * kD + tid;
+  const __nv_bfloat16* qr_in = (const __nv_bfloat16*)(a.q_route ? a.q_route : a.q);
+  const __nv_bfloat16* kr_in = (const __nv_bfloat16*)(a.k_route ? a.k_route : a.k);
+  ((__nv_bfloat16*)a.buf_k)[bslot] = ((const __nv_bfloat16*)a.k)[tok];
+  ((__nv_bfloat16*)a.buf_v)[bslot] = ((const __nv_bfloat16*)a.v)[tok];
+  ((__nv_bfloat16*)a.buf_qr)[bslot] = qr_in[tok];
+  ((__nv_bfloat16*)a.buf_kr)[bslot] = kr_in[tok];
+  if (tid == 0) {
+    a.buf_alpha[(long)bh * C + m] = a.alpha[bh];
+    a.buf_beta[(long)bh * C + m] = a.beta[bh];
+  }
+  tc::bar_sync(1, kCompute);
+  __threadfence_block();
+  const __nv_bfloat16* bk = (const __nv_bfloat16*)a.buf_k + (long)bh * C * kD;
+  const __nv_bfloat16* bv = (const __nv_bfloat16*)a.buf_v + (long)bh * C * kD;
+  // (1) open-chunk sweep
+  x = ldf((const __nv_bfloat16*)a.q + tok);
+  y0 = 0.0f;
+  for (int t = mp - 1; t >= 0; --t) {
+    const float kt = ldf(bk + (long)t * kD + tid);
+    const float c = blk_sum(kt * x, red);
+    const float bt = a.buf_beta[(long)bh * C + t];
+    const float at = a.buf_alpha[(long)bh * C + t];
+    y0 = fmaf(bt * c, ldf(bv + (long)t * kD + tid), y0);
+    x = at * (x - bt * c * kt);
+  }
+  // (2) gates and the ascending active list
+  int cnt = 0;
+  if (a.mode != HLA_GATES_ZERO && n > 0) {
+    const route::Consts K = route::make_consts();
+    if (a.mode == HLA_GATES_ROUTED) {
+      const __nv_bfloat16* bq = (const __nv_bfloat16*)a.buf_qr + (long)bh * C * kD + tid;
+      const float inv_tau = __fdiv_rn(1.0f, a.tau);
+      float mx = __fmul_rn(ldf(bq), inv_tau);
+      for (int t = 1; t < mp; ++t) mx = fmaxf(mx, __fmul_rn(ldf(bq + (long)t * kD), inv_tau));
+      float s = 0.0f;
+      for (int t = 0; t < mp; ++t)
+        s = __fadd_rn(s, route::rexp(__fsub_rn(__fmul_rn(ldf(bq + (long)t * kD), inv_tau), mx), K));
+      rq[tid] = __fmul_rn(a.tau, __fadd_rn(mx, route::rlog(__fdiv_rn(s, (float)mp), K)));
+      tc::bar_sync(1, kCompute);
+    }
+    const float* rk = a.rk + (long)bh * a.max_chunks * kD;
+    for (int jb = 0; jb < n; jb += kCompute) {
+      const int j = jb + tid;
+      float g = 1.0f;
+      bool keep = false;
+      if (j < n) {
+        if (a.mode == HLA_GATES_ROUTED) {
+          const float4* rkj = (const float4*)(rk + (long)j * kD);
+          float dot = 0.0f;
+          for (int c4 = 0; c4 < kD / 4; ++c4) {
+            const float4 r4 = rkj[c4];
+            dot = __fadd_rn(dot, __fmul_rn(rq[4 * c4 + 0], r4.x));
+            dot = __fadd_rn(dot, __fmul_rn(rq[4 * c4 + 1], r4.y));
+            dot = __fadd_rn(dot, __fmul_rn(rq[4 * c4 + 2], r4.z));
+            dot = __fadd_rn(dot, __fmul_rn(rq[4 * c4 + 3], r4.w));
+          }
+          g = route::gate_from_dot(dot, a.c_d, a.bias, K);
+        }
+        keep = a.thr <= 0.0f || g >= a.thr;
+      }
+      const unsigned int bal = __ballot_sync(0xFFFFFFFFu, keep);
+      const int w = tid >> 5;
+      if ((tid & 31) == 0) wcount[w] = __popc(bal);
+      tc::bar_sync(1, kCompute);
+      int before = 0, total = 0;
+#pragma unroll
+      for (int k2 = 0; k2 < 4; ++k2) {
+        if (k2 < w) before += wcount[k2];
+        total += wcount[k2];
+      }
+      if (keep) {
+        const int pos = cnt + before + __popc(bal & ((1u << (tid & 31)) - 1u));
+        act_idx[pos] = j;
+        act_g[pos] = g;
+      }
+      cnt += total;
+      tc::bar_sync(1, kCompute);
+    }
+  }
+  return cnt;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     decode_stream_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                          DecodeArgs a) {
@@ -57,10 +154,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int bh = blockIdx.x;
   const int b = bh / a.H;
   const int tid = threadIdx.x;
-  const int C = a.C;
   const int n = a.n_chunks[b];
   const int m = a.m_partial[b];
-  const int mp = m + 1;
   int32_t* act_idx = a.act_idx + (long)bh * a.max_chunks;
   float* act_g = a.act_g + (long)bh * a.max_chunks;
 
@@ -103,87 +198,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ---------------- compute (warps 0-3), thread = channel / row ----------------
+    float x, y0;
+    const int cnt = decode_prologue(a, bh, n, m, rq, red, wcount, x, y0);
     const long tok = (long)bh * kD + tid;
-    const long bslot = ((long)bh * C + m) * kD + tid;
-    const __nv_bfloat16* qr_in = (const __nv_bfloat16*)(a.q_route ? a.q_route : a.q);
-    const __nv_bfloat16* kr_in = (const __nv_bfloat16*)(a.k_route ? a.k_route : a.k);
-    ((__nv_bfloat16*)a.buf_k)[bslot] = ((const __nv_bfloat16*)a.k)[tok];
-    ((__nv_bfloat16*)a.buf_v)[bslot] = ((const __nv_bfloat16*)a.v)[tok];
-    ((__nv_bfloat16*)a.buf_qr)[bslot] = qr_in[tok];
-    ((__nv_bfloat16*)a.buf_kr)[bslot] = kr_in[tok];
-    if (tid == 0) {
-      a.buf_alpha[(long)bh * C + m] = a.alpha[bh];
-      a.buf_beta[(long)bh * C + m] = a.beta[bh];
-    }
-    tc::bar_sync(1, kCompute);
-    __threadfence_block();
-    const __nv_bfloat16* bk = (const __nv_bfloat16*)a.buf_k + (long)bh * C * kD;
-    const __nv_bfloat16* bv = (const __nv_bfloat16*)a.buf_v + (long)bh * C * kD;
-    // (1) open-chunk sweep
-    float x = ldf((const __nv_bfloat16*)a.q + tok);
-    float y0 = 0.0f;
-    for (int t = mp - 1; t >= 0; --t) {
-      const float kt = ldf(bk + (long)t * kD + tid);
-      const float c = blk_sum(kt * x, red);
-      const float bt = a.buf_beta[(long)bh * C + t];
-      const float at = a.buf_alpha[(long)bh * C + t];
-      y0 = fmaf(bt * c, ldf(bv + (long)t * kD + tid), y0);
-      x = at * (x - bt * c * kt);
-    }
-    // (2) gates and the ascending active list
-    int cnt = 0;
-    if (a.mode != HLA_GATES_ZERO && n > 0) {
-      const route::Consts K = route::make_consts();
-      if (a.mode == HLA_GATES_ROUTED) {
-        const __nv_bfloat16* bq = (const __nv_bfloat16*)a.buf_qr + (long)bh * C * kD + tid;
-        const float inv_tau = __fdiv_rn(1.0f, a.tau);
-        float mx = __fmul_rn(ldf(bq), inv_tau);
-        for (int t = 1; t < mp; ++t) mx = fmaxf(mx, __fmul_rn(ldf(bq + (long)t * kD), inv_tau));
-        float s = 0.0f;
-        for (int t = 0; t < mp; ++t)
-          s = __fadd_rn(s, route::rexp(__fsub_rn(__fmul_rn(ldf(bq + (long)t * kD), inv_tau), mx), K));
-        rq[tid] = __fmul_rn(a.tau, __fadd_rn(mx, route::rlog(__fdiv_rn(s, (float)mp), K)));
-        tc::bar_sync(1, kCompute);
-      }
-      const float* rk = a.rk + (long)bh * a.max_chunks * kD;
-      for (int jb = 0; jb < n; jb += kCompute) {
-        const int j = jb + tid;
-        float g = 1.0f;
-        bool keep = false;
-        if (j < n) {
-          if (a.mode == HLA_GATES_ROUTED) {
-            const float4* rkj = (const float4*)(rk + (long)j * kD);
-            float dot = 0.0f;
-            for (int c4 = 0; c4 < kD / 4; ++c4) {
-              const float4 r4 = rkj[c4];
-              dot = __fadd_rn(dot, __fmul_rn(rq[4 * c4 + 0], r4.x));
-              dot = __fadd_rn(dot, __fmul_rn(rq[4 * c4 + 1], r4.y));
-              dot = __fadd_rn(dot, __fmul_rn(rq[4 * c4 + 2], r4.z));
-              dot = __fadd_rn(dot, __fmul_rn(rq[4 * c4 + 3], r4.w));
-            }
-            g = route::gate_from_dot(dot, a.c_d, a.bias, K);
-          }
-          keep = a.thr <= 0.0f || g >= a.thr;
-        }
-        const unsigned int bal = __ballot_sync(0xFFFFFFFFu, keep);
-        const int w = tid >> 5;
-        if ((tid & 31) == 0) wcount[w] = __popc(bal);
-        tc::bar_sync(1, kCompute);
-        int before = 0, total = 0;
-#pragma unroll
-        for (int k2 = 0; k2 < 4; ++k2) {
-          if (k2 < w) before += wcount[k2];
-          total += wcount[k2];
-        }
-        if (keep) {
-          const int pos = cnt + before + __popc(bal & ((1u << (tid & 31)) - 1u));
-          act_idx[pos] = j;
-          act_g[pos] = g;
-        }
-        cnt += total;
-        tc::bar_sync(1, kCompute);
-      }
-    }
     if (tid == 0) *cnt_s = cnt;
     xs[tid] = x;
     __threadfence_block();
@@ -240,7 +257,181 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0 && *abort_s) report_device_error(kErrMbarTimeout);
 }
 
+// ---------------------------------------------------------------------------------
+// Factored cache.  A_j x = gamma_C x - Wb_j^T D_j (K_j x) and B_j x = Ub_j^T D_j (K_j x),
+// so per active chunk the stage holds K_j, Wb_j, Ub_j (64 x 128 bf16 each, 128-byte
+// swizzled 64-column boxes) and the scales (gamma_C / gamma_t, gamma_C): 48 KiB
+// instead of 64 KiB.  Phase 1: z_t = K_j[t] . x on pairs of threads (t = tid / 2, one
+// 64-column half each), z'_t = z_t gamma_C / gamma_t.  Phase 2: thread pairs own two
+// columns and split the 64 rows between them (rows with bit 2 clear / set, so the two
+// read disjoint banks): w = Wb^T z', u = Ub^T z'.  Then y += g u,
+// x <- (1 - g + g gamma_C) x - g w.
+constexpr int kFStages = 4;
+constexpr int kFTile = 64 * kD * 2;                 // 16 KiB: one 64 x 128 bf16 factor
+constexpr int kFScale = (64 + 4) * 4;               // scales of one chunk
+constexpr int kFStageBytes = 3 * kFTile + 1024;     // K, Wb, Ub, scales (1 KiB aligned)
+constexpr uint32_t kFTx = 3 * kFTile + kFScale;
+
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_stream_factored_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmW,
+                                  const __grid_constant__ CUtensorMap tmU, DecodeArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* ring = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint64_t* full = (uint64_t*)(ring + kFStages * kFStageBytes);
+  uint64_t* empty = full + kFStages;
+  float* xs = (float*)(empty + kFStages);    // [2][kD]
+  float* rq = xs + 2 * kD;                   // [kD]
+  float* zs = rq + kD;                       // [64]
+  float* red = zs + 64;                      // [4]
+  int* wcount = (int*)(red + 4);             // [4]
+  int* cnt_s = wcount + 4;                   // [1]
+  volatile int* abort_s = (volatile int*)(cnt_s + 1);
+
+  const int bh = blockIdx.x;
+  const int b = bh / a.H;
+  const int tid = threadIdx.x;
+  const int n = a.n_chunks[b];
+  const int m = a.m_partial[b];
+  const int32_t* act_idx = a.act_idx + (long)bh * a.max_chunks;
+  const float* act_g = a.act_g + (long)bh * a.max_chunks;
+
+  if (tid == 0) {
+    for (int s = 0; s < kFStages; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);
+    }
+    *abort_s = 0;
+    tc::mbar_fence_init();
+    tc::fence_async_smem();
+  }
+  __syncthreads();
+
+  if (tid >= kCompute) {
+    // ---------------- TMA producer (warp 4, lane 0) ----------------
+    tc::bar_sync(2, kThreads);
+    if (tid == kCompute) {
+      tc::tma_prefetch_desc(&tmK);
+      tc::tma_prefetch_desc(&tmW);
+      tc::tma_prefetch_desc(&tmU);
+      const int cnt = *cnt_s;
+      int s = 0;
+      for (int p = cnt - 1; p >= 0; --p, ++s) {
+        const int st = s % kFStages;
+        if (s >= kFStages && !tc::mbar_wait(&empty[st], ((s / kFStages) - 1) & 1, abort_s)) break;
+        const int j = act_idx[p];
+        const long slot = (long)bh * a.max_chunks + j;
+        const int row = (int)(slot * 64);
+        tc::mbar_arrive_expect_tx(&full[st], kFTx);
+        uint8_t* dst = ring + st * kFStageBytes;
+        tc::tma_load_2d(dst, &tmK, 0, row, &full[st]);
+        tc::tma_load_2d(dst + kFTile / 2, &tmK, 64, row, &full[st]);
+        tc::tma_load_2d(dst + kFTile, &tmW, 0, row, &full[st]);
+        tc::tma_load_2d(dst + kFTile + kFTile / 2, &tmW, 64, row, &full[st]);
+        tc::tma_load_2d(dst + 2 * kFTile, &tmU, 0, row, &full[st]);
+        tc::tma_load_2d(dst + 2 * kFTile + kFTile / 2, &tmU, 64, row, &full[st]);
+        tc::bulk_load_1d(dst + 3 * kFTile, a.df + slot * (64 + 4), kFScale, &full[st]);
+      }
+      if (*abort_s)
+        for (int t = max(0, s - kFStages); t < s; ++t)
+          tc::mbar_wait(&full[t % kFStages], (t / kFStages) & 1, nullptr, 200000000ull);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- compute (warps 0-3) ----------------
+    float x, y0;
+    const int cnt = decode_prologue(a, bh, n, m, rq, red, wcount, x, y0);
+    const long tok = (long)bh * kD + tid;
+    if (tid == 0) *cnt_s = cnt;
+    xs[tid] = x;
+    __threadfence_block();
+    tc::bar_sync(2, kThreads);  // releases the producer
+    const int pt = tid >> 1, ph = tid & 1;   // phase 1: row pt, column half ph
+    const int cp = tid >> 1, th = tid & 1;   // phase 2: columns 2cp, 2cp+1; row set th
+    const int cbox = (2 * cp) >> 6, c8 = ((2 * cp) & 63) >> 3, cw = ((2 * cp) & 7) * 2;
+    float y = 0.0f;
+    int cur = 0;
+    bool ok = true;
+    for (int p = cnt - 1, s = 0; p >= 0; --p, ++s) {
+      const int st = s % kFStages;
+      ok = tc::bar_all(1, kCompute, tc::mbar_wait(&full[st], (s / kFStages) & 1, abort_s));
+      if (!ok) break;
+      const uint8_t* stK = ring + st * kFStageBytes;
+      const uint8_t* stW = stK + kFTile;
+      const uint8_t* stU = stK + 2 * kFTile;
+      const float* dfs = (const float*)(stK + 3 * kFTile);
+      const float* xc = xs + cur * kD;
+      // phase 1: z'_t
+      {
+        const uint8_t* krow = stK + ph * (kFTile / 2) + pt * 128;
+        float z0 = 0.0f, z1 = 0.0f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const uint4 w = *(const uint4*)(krow + ((q ^ (pt & 7)) << 4));
+          const float4 x0 = *(const float4*)(xc + ph * 64 + q * 8);
+          const float4 x1 = *(const float4*)(xc + ph * 64 + q * 8 + 4);
+          z0 = fmaf(tc::bf16lo(w.x), x0.x, z0);
+          z1 = fmaf(tc::bf16hi(w.x), x0.y, z1);
+          z0 = fmaf(tc::bf16lo(w.y), x0.z, z0);
+          z1 = fmaf(tc::bf16hi(w.y), x0.w, z1);
+          z0 = fmaf(tc::bf16lo(w.z), x1.x, z0);
+          z1 = fmaf(tc::bf16hi(w.z), x1.y, z1);
+          z0 = fmaf(tc::bf16lo(w.w), x1.z, z0);
+          z1 = fmaf(tc::bf16hi(w.w), x1.w, z1);
+        }
+        float z = z0 + z1;
+        z += __shfl_xor_sync(0xFFFFFFFFu, z, 1);
+        if (ph == 0) zs[pt] = z * dfs[pt];
+      }
+      tc::bar_sync(1, kCompute);
+      // phase 2: w = Wb^T z', u = Ub^T z' for columns 2cp, 2cp+1 over this thread's rows
+      float w0 = 0.0f, w1 = 0.0f, u0 = 0.0f, u1 = 0.0f;
+#pragma unroll 8
+      for (int k = 0; k < 32; ++k) {
+        const int t = 8 * (k >> 2) + (k & 3) + 4 * th;
+        const int off = cbox * (kFTile / 2) + t * 128 + ((c8 ^ (t & 7)) << 4) + cw;
+        const uint32_t ww = *(const uint32_t*)(stW + off);
+        const uint32_t uu = *(const uint32_t*)(stU + off);
+        const float zt = zs[t];
+        w0 = fmaf(tc::bf16lo(ww), zt, w0);
+        w1 = fmaf(tc::bf16hi(ww), zt, w1);
+        u0 = fmaf(tc::bf16lo(uu), zt, u0);
+        u1 = fmaf(tc::bf16hi(uu), zt, u1);
+      }
+      w0 += __shfl_xor_sync(0xFFFFFFFFu, w0, 1);
+      w1 += __shfl_xor_sync(0xFFFFFFFFu, w1, 1);
+      u0 += __shfl_xor_sync(0xFFFFFFFFu, u0, 1);
+      u1 += __shfl_xor_sync(0xFFFFFFFFu, u1, 1);
+      // thread tid owns column tid = 2 cp + th
+      const float wc = th ? w1 : w0, uc = th ? u1 : u0;
+      const float g = act_g[p];
+      const float rho = (1.0f - g) + g * dfs[64];
+      y = fmaf(g, uc, y);
+      xs[(cur ^ 1) * kD + tid] = rho * xc[tid] - g * wc;
+      cur ^= 1;
+      tc::bar_sync(1, kCompute);
+      if (tid == 0) tc::mbar_arrive(&empty[st]);
+    }
+    stf((__nv_bfloat16*)a.o + tok, y + y0);
+  }
+  __syncthreads();
+  if (tid == 0 && *abort_s) report_device_error(kErrMbarTimeout);
+}
+
 }  // namespace
+
+cudaError_t launch_decode_stream_factored(const DecodeArgs& a, cudaStream_t s) {
+  const long rows = (long)a.B * a.H * a.max_chunks * 64;
+  CUtensorMap tmK, tmW, tmU;
+  cudaError_t e = make_tmap_2d(&tmK, a.Kf, kD, rows, kD * 2, 64, 64);
+  if (e == cudaSuccess) e = make_tmap_2d(&tmW, a.Wf, kD, rows, kD * 2, 64, 64);
+  if (e == cudaSuccess) e = make_tmap_2d(&tmU, a.Uf, kD, rows, kD * 2, 64, 64);
+  if (e != cudaSuccess) return e;
+  const size_t smem = 1024 + kFStages * kFStageBytes + 2 * kFStages * 8 + (4 * kD + 64 + 16) * 4;
+  e = cudaFuncSetAttribute(decode_stream_factored_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  decode_stream_factored_kernel<<<a.B * a.H, kThreads, smem, s>>>(tmK, tmW, tmU, a);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_decode_stream(const DecodeArgs& a, cudaStream_t s) {
   const long rows = (long)a.B * a.H * a.max_chunks * kD;

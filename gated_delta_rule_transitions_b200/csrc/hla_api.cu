@@ -43,6 +43,8 @@ hla_status check_cfg(const hla_config* c, bool need_T) {
   if (c->dtype != HLA_F32 && c->dtype != HLA_BF16) return fail(HLA_ERR_UNSUPPORTED, "dtype %d unsupported", c->dtype);
   if (c->gate_mode < HLA_GATES_ROUTED || c->gate_mode > HLA_GATES_USER)
     return fail(HLA_ERR_INVALID_ARG, "gate_mode %d invalid", c->gate_mode);
+  if (c->cache_format != HLA_CACHE_DENSE && c->cache_format != HLA_CACHE_FACTORED)
+    return fail(HLA_ERR_INVALID_ARG, "cache_format %d invalid", c->cache_format);
   if (!(c->tau > 0.0f) || !std::isfinite(c->tau)) return fail(HLA_ERR_INVALID_ARG, "tau must be finite and > 0");
   if (!std::isfinite(c->bias) || !std::isfinite(c->skip_threshold))
     return fail(HLA_ERR_INVALID_ARG, "bias and skip_threshold must be finite");
@@ -109,8 +111,12 @@ PrefillWs prefill_layout(const hla_config* c) {
 }
 
 struct CacheLayout {
-  size_t A, Bm, rk, bk, bv, bqr, bkr, balpha, bbeta, n, m, total;
+  size_t A, Bm, Kf, Wf, Uf, df, rk, bk, bv, bqr, bkr, balpha, bbeta, n, m, total;
 };
+
+// Scales stored per chunk in a factored cache: gamma_C / gamma_t for t < C, then
+// gamma_C, padded to a 16-byte multiple.
+inline size_t df_stride(size_t C) { return C + 4; }
 
 CacheLayout cache_layout(const hla_config* c, int32_t maxc) {
   CacheLayout L{};
@@ -121,8 +127,15 @@ CacheLayout cache_layout(const hla_config* c, int32_t maxc) {
     off = align256(off + bytes);
     return o;
   };
-  L.A = take(B * H * (size_t)maxc * d * d * es);
-  L.Bm = take(B * H * (size_t)maxc * d * d * es);
+  if (c->cache_format == HLA_CACHE_FACTORED) {
+    L.Kf = take(B * H * (size_t)maxc * C * d * es);
+    L.Wf = take(B * H * (size_t)maxc * C * d * es);
+    L.Uf = take(B * H * (size_t)maxc * C * d * es);
+    L.df = take(B * H * (size_t)maxc * df_stride(C) * 4);
+  } else {
+    L.A = take(B * H * (size_t)maxc * d * d * es);
+    L.Bm = take(B * H * (size_t)maxc * d * d * es);
+  }
   L.rk = take(B * H * (size_t)maxc * d * 4);
   L.bk = take(B * H * C * d * es);
   L.bv = take(B * H * C * d * es);
@@ -138,11 +151,19 @@ CacheLayout cache_layout(const hla_config* c, int32_t maxc) {
 
 hla_status check_cache(const hla_config* c, const hla_cache* k) {
   if (k == nullptr) return fail(HLA_ERR_INVALID_ARG, "cache is NULL");
-  if (k->B != c->B || k->H != c->H || k->C != c->C || k->d != c->dk || k->dtype != c->dtype)
+  if (k->B != c->B || k->H != c->H || k->C != c->C || k->d != c->dk || k->dtype != c->dtype ||
+      k->format != c->cache_format)
     return fail(HLA_ERR_INVALID_ARG, "cache was initialised for a different config");
   if (k->max_chunks <= 0) return fail(HLA_ERR_INVALID_ARG, "cache max_chunks must be positive");
-  const void* ps[] = {k->A, k->Bm, k->rk, k->buf_k, k->buf_v, k->buf_qr, k->buf_kr, k->buf_alpha, k->buf_beta};
+  const void* ps[] = {k->rk, k->buf_k, k->buf_v, k->buf_qr, k->buf_kr, k->buf_alpha, k->buf_beta};
   for (const void* p : ps) HLA_TRY(need_ptr(p, "cache buffer"));
+  if (k->format == HLA_CACHE_FACTORED) {
+    const void* fs[] = {k->Kf, k->Wf, k->Uf, k->df};
+    for (const void* p : fs) HLA_TRY(need_ptr(p, "cache factor buffer"));
+  } else {
+    HLA_TRY(need_ptr(k->A, "cache A"));
+    HLA_TRY(need_ptr(k->Bm, "cache B"));
+  }
   // the per-sequence counters are read and written as single int32 values, so a
   // slice starting at any sequence is valid
   for (const int32_t* p : {k->n_chunks, k->m_partial})
@@ -237,6 +258,8 @@ hla_status hla_cache_init(const hla_config* cfg, int32_t max_chunks, void* mem, 
   if (max_chunks <= 0) return fail(HLA_ERR_INVALID_ARG, "max_chunks must be positive");
   HLA_TRY(need_ptr(mem, "mem"));
   if (((uintptr_t)mem & 255u) != 0) return fail(HLA_ERR_INVALID_ARG, "cache memory must be 256-byte aligned");
+  if (cfg->cache_format == HLA_CACHE_FACTORED && !(cfg->dtype == HLA_BF16 && cfg->dk == 128))
+    return fail(HLA_ERR_UNSUPPORTED, "a factored cache needs bf16 and d = 128");
   const CacheLayout L = cache_layout(cfg, max_chunks);
   if (bytes < L.total) return fail(HLA_ERR_WORKSPACE, "cache block too small: %zu < %zu", bytes, L.total);
   char* base = (char*)mem;
@@ -247,8 +270,16 @@ hla_status hla_cache_init(const hla_config* cfg, int32_t max_chunks, void* mem, 
   c.C = cfg->C;
   c.d = cfg->dk;
   c.dtype = cfg->dtype;
-  c.A = base + L.A;
-  c.Bm = base + L.Bm;
+  c.format = cfg->cache_format;
+  if (cfg->cache_format == HLA_CACHE_FACTORED) {
+    c.Kf = base + L.Kf;
+    c.Wf = base + L.Wf;
+    c.Uf = base + L.Uf;
+    c.df = (float*)(base + L.df);
+  } else {
+    c.A = base + L.A;
+    c.Bm = base + L.Bm;
+  }
   c.rk = (float*)(base + L.rk);
   c.buf_k = base + L.bk;
   c.buf_v = base + L.bv;
@@ -276,8 +307,15 @@ hla_status hla_cache_slice(const hla_cache* cache, int32_t b0, int32_t nb, hla_c
   const size_t off = (size_t)b0;
   hla_cache v = *cache;
   v.B = nb;
-  v.A = (char*)cache->A + off * H * mc * d * d * es;
-  v.Bm = (char*)cache->Bm + off * H * mc * d * d * es;
+  if (cache->format == HLA_CACHE_FACTORED) {
+    v.Kf = (char*)cache->Kf + off * H * mc * C * d * es;
+    v.Wf = (char*)cache->Wf + off * H * mc * C * d * es;
+    v.Uf = (char*)cache->Uf + off * H * mc * C * d * es;
+    v.df = (float*)((char*)cache->df + off * H * mc * df_stride(C) * 4);
+  } else {
+    v.A = (char*)cache->A + off * H * mc * d * d * es;
+    v.Bm = (char*)cache->Bm + off * H * mc * d * d * es;
+  }
   v.rk = (float*)((char*)cache->rk + off * H * mc * d * 4);
   v.buf_k = (char*)cache->buf_k + off * H * C * d * es;
   v.buf_v = (char*)cache->buf_v + off * H * C * d * es;
@@ -473,9 +511,12 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
   t.in = {k, v, alpha, beta, (long)cfg->T * cfg->H * cfg->dk, cfg->dk, (long)cfg->H * cfg->dk,
           (long)cfg->T * cfg->H, 1, cfg->H};
   t.n_chunks = N;
-  t.A = cache_out ? cache_out->A : (void*)(ws + w.A);
-  t.Bm = cache_out ? cache_out->Bm : (void*)(ws + w.Bm);
-  t.ab_chunk_stride = cache_out ? cache_out->max_chunks : Nc;
+  // a dense cache takes A/B straight from the transitions; otherwise they go to the
+  // workspace (the composition reads them) and a factored cache gets the WY factors
+  const bool dense_out = cache_out != nullptr && cache_out->format == HLA_CACHE_DENSE;
+  t.A = dense_out ? cache_out->A : (void*)(ws + w.A);
+  t.Bm = dense_out ? cache_out->Bm : (void*)(ws + w.Bm);
+  t.ab_chunk_stride = dense_out ? cache_out->max_chunks : Nc;
   t.Wb = (float*)(ws + w.Wb);
   t.Ub = (float*)(ws + w.Ub);
   t.ell = (float*)(ws + w.ell);
@@ -551,8 +592,27 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
     dc.buf_beta = cache_out->buf_beta;
     dc.n_chunks = cache_out->n_chunks;
     dc.m_partial = cache_out->m_partial;
-    StageScope _sc(HLA_STAGE_CACHE, s, 1);
+    const bool factored = cache_out->format == HLA_CACHE_FACTORED;
+    StageScope _sc(HLA_STAGE_CACHE, s, factored ? 2 : 1);
     HLA_CUDA(hla::launch_cache_fill(dc, rk, qr, kr, k, v, alpha, beta, cfg->T, s), "cache fill launch");
+    if (factored && Nc > 0) {
+      hla::FactorFillArgs f{};
+      f.B = cfg->B;
+      f.H = cfg->H;
+      f.T = cfg->T;
+      f.N = N;
+      f.Nc = Nc;
+      f.max_chunks = cache_out->max_chunks;
+      f.k = k;
+      f.Wb = ws + w.Wb;
+      f.Ub = ws + w.Ub;
+      f.ell = (const float*)(ws + w.ell);
+      f.Kf = cache_out->Kf;
+      f.Wf = cache_out->Wf;
+      f.Uf = cache_out->Uf;
+      f.df = cache_out->df;
+      HLA_CUDA(hla::launch_factor_fill(f, s), "factor fill launch");
+    }
   }
   return HLA_OK;
 }
@@ -598,6 +658,11 @@ hla_status hla_decode_step(const hla_config* cfg, hla_cache* cache, const void* 
   a.o = o;
   a.A = cache->A;
   a.Bm = cache->Bm;
+  a.format = cache->format;
+  a.Kf = cache->Kf;
+  a.Wf = cache->Wf;
+  a.Uf = cache->Uf;
+  a.df = cache->df;
   a.rk = cache->rk;
   a.buf_k = cache->buf_k;
   a.buf_v = cache->buf_v;

@@ -46,6 +46,25 @@ struct TransArgs {
   float* ell;            // [B,H,N,C] fp32 or null
   const int32_t* close_m;   // decode close: per-b m_partial (before the step) or null
   const int32_t* close_n;   // decode close: per-b n_chunks or null
+  // decode close into a factored cache: K, Wb, Ub ([.., chunk_stride, C, d]) and the
+  // scales ([.., chunk_stride, C + 4]) of the closed chunk instead of A/B
+  void* Kf;
+  void* Wf;
+  void* Uf;
+  float* df;
+};
+
+// Prefill -> factored cache: the WY factors and scales of every complete chunk.
+struct FactorFillArgs {
+  int B, H, T, N, Nc, max_chunks;
+  const void* k;       // [B,T,H,d] bf16 (input keys)
+  const void* Wb;      // [B,H,N,C,d] bf16 (workspace)
+  const void* Ub;
+  const float* ell;    // [B,H,N,C]
+  void* Kf;            // [B,H,max_chunks,C,d] bf16
+  void* Wf;
+  void* Uf;
+  float* df;           // [B,H,max_chunks,C+4]
 };
 
 struct ComposeArgs {
@@ -86,6 +105,11 @@ struct DecodeArgs {
   // cache
   const void* A;
   const void* Bm;
+  int format;          // hla_cache_format
+  void* Kf;            // factored: [B,H,max_chunks,C,d]
+  void* Wf;
+  void* Uf;
+  float* df;           // factored: [B,H,max_chunks,C+4]
   float* rk;
   void* buf_k;
   void* buf_v;
@@ -116,6 +140,8 @@ cudaError_t read_error_word_compose_tc(unsigned int* out, bool clear);
 cudaError_t launch_compose_tc(const ComposeArgs& a, bool scan, cudaStream_t s);
 cudaError_t launch_decode_stream(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_transitions_tc(const TransArgs& t, cudaStream_t s);
+cudaError_t launch_factor_fill(const FactorFillArgs& f, cudaStream_t s);
+cudaError_t launch_decode_stream_factored(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_readout_tc(const ReadoutArgs& r, const void* S_in_bf16, const void* Wb_bf16, const void* Ub_bf16,
                               cudaStream_t s);
 cudaError_t read_error_word_transitions_tc(unsigned int* out, bool clear);

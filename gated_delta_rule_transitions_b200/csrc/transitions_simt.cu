@@ -123,6 +123,22 @@ __global__ void __launch_bounds__(256) transitions_simt_kernel(TransArgs a) {
     }
     if (tid < C) a.ell[(bhc * a.n_chunks + c) * C + tid] = ell[tid];
   }
+  if (complete && a.Kf != nullptr) {
+    // factored cache: K, Wb, Ub of the chunk and its scales gamma_C / gamma_t, gamma_C
+    const long slot = bhc * a.ab_chunk_stride + chunk_out + a.ab_chunk_offset;
+    Tio* Ko = (Tio*)a.Kf + slot * (long)C * D;
+    Tio* Wo = (Tio*)a.Wf + slot * (long)C * D;
+    Tio* Uo = (Tio*)a.Uf + slot * (long)C * D;
+    for (int idx = tid; idx < C * D; idx += blockDim.x) {
+      const int t = idx / D, cc = idx - t * D;
+      stf(Ko + idx, Ks[t * DP + cc]);
+      stf(Wo + idx, Wb[t * DP + cc]);
+      stf(Uo + idx, Ub[t * DP + cc]);
+    }
+    float* dfo = a.df + slot * (long)(C + 4);
+    if (tid < C) dfo[tid] = expf(ell[C - 1] - ell[tid]);
+    if (tid >= C && tid < C + 4) dfo[tid] = tid == C ? gam[C - 1] : 0.0f;
+  }
   if (!complete || a.A == nullptr) return;
   // D K (rows scaled by gamma_C / gamma_t)
   const float lC = ell[C - 1];

@@ -83,6 +83,15 @@ typedef enum {
   HLA_GATES_USER = 3    /* caller-given input-independent weights [B,H,N,N] (prefill) */
 } hla_gate_mode;
 
+/* Storage of the closed chunks' transitions in a decode cache. */
+typedef enum {
+  HLA_CACHE_DENSE = 0,    /* A_j, B_j as d x d matrices (2 d^2 elements per chunk)        */
+  HLA_CACHE_FACTORED = 1  /* the WY factors K_j, Wb_j, Ub_j (C x d each) and D_j, gamma_C:
+                             A_j = gamma_C I - Wb_j^T D_j K_j, B_j = Ub_j^T D_j K_j
+                             (3 C d elements; 25 % fewer bytes at C = 64, d = 128).
+                             bf16 with d = 128 only. */
+} hla_cache_format;
+
 typedef struct hla_config {
   int32_t B;              /* sequences                                          */
   int32_t H;              /* heads                                              */
@@ -91,6 +100,7 @@ typedef struct hla_config {
   int32_t dk, dv;         /* head dims, equal, 64 or 128                        */
   int32_t dtype;          /* hla_dtype                                          */
   int32_t gate_mode;      /* hla_gate_mode                                      */
+  int32_t cache_format;   /* hla_cache_format of the caches used with this config */
   float tau;              /* pooling temperature, > 0                           */
   float bias;             /* gate bias b                                        */
   float skip_threshold;   /* <= 0: nothing skipped                              */
@@ -100,6 +110,10 @@ typedef struct hla_config {
  * Decode cache of B sequences (all pointers are device memory carved out of one
  * caller-owned block by hla_cache_init):
  *   A, Bm        [B, H, max_chunks, d, d]  dtype  -- transitions of closed chunks
+ *                (HLA_CACHE_DENSE; NULL otherwise)
+ *   Kf, Wf, Uf   [B, H, max_chunks, C, d]  dtype  -- K_j, Wb_j, Ub_j of closed chunks
+ *   df           [B, H, max_chunks, C + 4] float32 -- gamma_C / gamma_t (t < C), then
+ *                gamma_C, then padding (HLA_CACHE_FACTORED; all NULL otherwise)
  *   rk           [B, H, max_chunks, d]     float32 -- key pools of closed chunks
  *   buf_k, buf_v, buf_qr, buf_kr  [B, H, C, d] dtype -- tokens of the open chunk
  *   buf_alpha, buf_beta           [B, H, C]  float32
@@ -111,8 +125,13 @@ typedef struct hla_config {
 typedef struct hla_cache {
   int32_t max_chunks;
   int32_t B, H, C, d, dtype;
+  int32_t format; /* hla_cache_format */
   void* A;
   void* Bm;
+  void* Kf;
+  void* Wf;
+  void* Uf;
+  float* df;
   float* rk;
   void* buf_k;
   void* buf_v;

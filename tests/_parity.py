@@ -37,10 +37,10 @@ def to_cuda(inp):
     return {k: (None if v is None else v.cuda().contiguous()) for k, v in inp.items()}
 
 
-def run_prefill(hla, w: syn.Workload, inp, user_gates=None, cache=None):
+def run_prefill(hla, w: syn.Workload, inp, user_gates=None, cache=None, cache_format="dense"):
     B, T, H, d = inp["q"].shape
     N = (T + w.C - 1) // w.C
-    cfg = hla.make_config(B, H, T, w.C, d, w.dtype, w.gate_mode, w.tau, w.bias, w.thr)
+    cfg = hla.make_config(B, H, T, w.C, d, w.dtype, w.gate_mode, w.tau, w.bias, w.thr, cache_format=cache_format)
     g = to_cuda(inp)
     o = torch.empty_like(g["q"])
     gates = torch.empty((B, H, N, N), dtype=torch.float32, device="cuda")

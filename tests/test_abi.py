@@ -188,3 +188,34 @@ def test_cache_slice_offsets_follow_the_sequence_major_layout(hla):
         assert getattr(out, f) == ((i + 1) << 32) + 2 * per_seq[f], f
     for b0, nb in ((-1, 1), (0, 0), (3, 2), (4, 1)):
         assert hla.lib().hla_cache_slice(ctypes.byref(c), b0, nb, ctypes.byref(out)) == hla.HLA_ERR_INVALID_ARG
+
+
+def test_factored_cache_sizes_and_slices(hla):
+    """A factored cache stores K_j, Wb_j, Ub_j (C x d each) and C + 4 float32 scales
+    per closed chunk instead of the two d x d matrices."""
+    dense = cfg(hla, B=2, H=3, T=1)
+    fact = cfg(hla, B=2, H=3, T=1, cache_format="factored")
+    mc = 5
+    per_chunk_dense = 2 * 128 * 128 * 2
+    per_chunk_fact = 3 * 64 * 128 * 2 + (64 + 4) * 4
+    diff = hla.cache_bytes(dense, mc) - hla.cache_bytes(fact, mc)
+    # the rest of the layout is identical; 256-byte alignment of 2 vs 4 sub-buffers
+    assert abs(diff - 2 * 3 * mc * (per_chunk_dense - per_chunk_fact)) <= 4 * 256
+    c = hla.HlaCache()
+    c.B, c.H, c.C, c.d, c.dtype, c.max_chunks, c.format = 4, 2, 64, 128, 1, 3, 1
+    for i, f in enumerate(("Kf", "Wf", "Uf", "df")):
+        setattr(c, f, (i + 1) << 32)
+    for f in ("rk", "buf_k", "buf_v", "buf_qr", "buf_kr", "buf_alpha", "buf_beta", "n_chunks", "m_partial"):
+        setattr(c, f, 1 << 40)
+    out = hla.HlaCache()
+    assert hla.lib().hla_cache_slice(ctypes.byref(c), 1, 2, ctypes.byref(out)) == hla.HLA_OK
+    assert out.Kf == (1 << 32) + 2 * 3 * 64 * 128 * 2
+    assert out.df == (4 << 32) + 2 * 3 * 68 * 4
+    assert not out.A and not out.Bm
+
+
+def test_factored_cache_needs_bf16_d128(hla):
+    c = cfg(hla, B=1, H=1, T=1, d=64, dtype="f32", cache_format="factored")
+    out = hla.HlaCache()
+    st = hla.lib().hla_cache_init(ctypes.byref(c), 4, ctypes.c_void_p(1 << 20), 1 << 30, ctypes.byref(out), None)
+    assert st == hla.HLA_ERR_UNSUPPORTED and "factored" in hla.last_error()

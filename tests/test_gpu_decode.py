@@ -93,8 +93,62 @@ def test_decode_chain_matches_oracle(hla, dtype, d, mode, thr, route):
             assert np.array_equal(rk[b, h, j].view(np.uint32), st_.rk[j].view(np.uint32))
 
 
-@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("f32", 64)])
-def test_decode_ragged_positions(hla, dtype, d):
+@pytest.mark.parametrize("mode,thr,route", [("routed", 0.05, False), ("routed", 0.4, True), ("one", 0.0, False)])
+def test_decode_factored_cache_matches_oracle(hla, mode, thr, route):
+    """Decode from a factored cache (K_j, Wb_j, Ub_j and the scales per closed chunk):
+    prefill hand-off, chained steps that close a chunk (the closing step writes the
+    new chunk's factors), outputs against the oracle and against the same steps on a
+    dense cache."""
+    T0 = 64 * 3 + 58
+    steps = 9
+    w = syn.DECODE_32K.with_(B=2, H=2, T=T0, gate_mode=mode, thr=thr,
+                             route="spread" if route else "default", bias=-0.5 if route else -2.0)
+    inp = P.gpu_inputs(w)
+    caches = {}
+    for fmt in ("factored", "dense"):
+        cfg = hla.make_config(w.B, w.H, T0, 64, 128, "bf16", mode, w.tau, w.bias, w.thr, cache_format=fmt)
+        caches[fmt] = hla.Cache(cfg, max_chunks=8)
+        P.run_prefill(hla, w.with_(), inp, cache=caches[fmt], cache_format=fmt)
+    toks = syn.make_decode_tokens(w, steps)
+    routes = _route_tokens(w.B, w.H, 128, steps, 77, torch.bfloat16) if route else [(None, None)] * steps
+    heads = {}
+    for b in range(w.B):
+        for h in range(w.H):
+            f = lambda n: None if inp.get(n) is None else inp[n][b, :, h]
+            heads[(b, h)] = ho.HlaDecodeHead.from_prefill(
+                P.np64(f("q")), P.np64(f("k")), P.np64(f("v")), P.np64(f("alpha")), P.np64(f("beta")), 64,
+                w.tau, w.bias, w.thr, mode,
+                None if f("q_route") is None else P.np32(f("q_route")),
+                None if f("k_route") is None else P.np32(f("k_route")))
+    got, dense, ref = [], [], []
+    for s_, tk in enumerate(toks):
+        g = {k: v.cuda().contiguous() for k, v in tk.items()}
+        qr, kr = routes[s_]
+        outs = {}
+        for fmt, cache in caches.items():
+            dcfg = hla.make_config(w.B, w.H, 1, 64, 128, "bf16", mode, w.tau, w.bias, w.thr, cache_format=fmt)
+            o = torch.empty_like(g["q"])
+            hla.hla_decode_step(dcfg, cache, g["q"], g["k"], g["v"], g["alpha"], g["beta"], o,
+                                q_route=None if qr is None else qr.cuda(), k_route=None if kr is None else kr.cuda())
+            outs[fmt] = o
+        torch.cuda.synchronize()
+        for (b, h), st_ in heads.items():
+            got.append(P.np64(outs["factored"][b, h]))
+            dense.append(P.np64(outs["dense"][b, h]))
+            ref.append(st_.step(P.np64(tk["q"][b, h]), P.np64(tk["k"][b, h]), P.np64(tk["v"][b, h]),
+                                float(tk["alpha"][b, h]), float(tk["beta"][b, h]),
+                                None if qr is None else P.np32(qr[b, h]), None if kr is None else P.np32(kr[b, h])))
+    got, dense, ref = np.stack(got), np.stack(dense), np.stack(ref)
+    assert P.rel_l2(got, ref) <= P.TOL_BF16_RELL2
+    assert P.rel_l2(got, dense) <= P.TOL_BF16_RELL2
+    st, code = hla.hla_device_status()
+    assert st == 0 and code == 0
+    n = caches["factored"].view("n_chunks", (w.B,), torch.int32).cpu().tolist()
+    assert n == [(T0 + steps) // 64] * w.B
+
+
+@pytest.mark.parametrize("dtype,d,fmt", [("bf16", 128, "dense"), ("f32", 64, "dense"), ("bf16", 128, "factored")])
+def test_decode_ragged_positions(hla, dtype, d, fmt):
     """Sequences at different positions in one cache: each is prefilled on its own
     (prompts of 202 and 370 tokens) into its slice of the cache, then chained decode
     steps advance both together; they close chunks at different steps.  Every output
@@ -102,19 +156,20 @@ def test_decode_ragged_positions(hla, dtype, d):
     lens = [64 * 3 + 10, 64 * 5 + 50]
     steps = 60
     base = syn.DECODE_32K.with_(B=1, H=2, dtype=dtype, d=d, thr=0.05, bias=-0.5, route="spread")
-    cfg2 = hla.make_config(2, base.H, max(lens), 64, d, dtype, "routed", base.tau, base.bias, base.thr)
+    cfg2 = hla.make_config(2, base.H, max(lens), 64, d, dtype, "routed", base.tau, base.bias, base.thr,
+                           cache_format=fmt)
     cache = hla.Cache(cfg2, max_chunks=8)
     heads = {}
     for b, T_b in enumerate(lens):
         w = base.with_(T=T_b, seed=11 + b)
         inp = P.gpu_inputs(w)
-        P.run_prefill(hla, w, inp, cache=cache.slice(b, 1))
+        P.run_prefill(hla, w, inp, cache=cache.slice(b, 1), cache_format=fmt)
         for h in range(w.H):
             f = lambda n: None if inp.get(n) is None else inp[n][0, :, h]
             heads[(b, h)] = ho.HlaDecodeHead.from_prefill(
                 P.np64(f("q")), P.np64(f("k")), P.np64(f("v")), P.np64(f("alpha")), P.np64(f("beta")), 64,
                 w.tau, w.bias, w.thr, "routed", P.np32(f("q_route")), P.np32(f("k_route")))
-    dcfg = hla.make_config(2, base.H, 1, 64, d, dtype, "routed", base.tau, base.bias, base.thr)
+    dcfg = hla.make_config(2, base.H, 1, 64, d, dtype, "routed", base.tau, base.bias, base.thr, cache_format=fmt)
     toks = syn.make_decode_tokens(base.with_(B=2), steps)
     routes = _route_tokens(2, base.H, d, steps, 91, syn.torch_dtype(base))
     got, ref = [], []
