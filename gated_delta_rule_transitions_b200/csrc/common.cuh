@@ -27,6 +27,21 @@ enum : unsigned int {
   kErrCacheFull = 4u,     // a decode step had to close a chunk into a full cache
 };
 
+// Streaming multiprocessors of the current device (read once per process; the
+// library runs on one kind of GPU).
+inline int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
+      n = v;
+    else
+      return 148;
+  }
+  return n;
+}
+
 #define HLA_DEFINE_ERROR_WORD(tu)                                                      \
   static __device__ unsigned int g_err_word;                                          \
   __device__ __forceinline__ void report_device_error(unsigned int code) {            \

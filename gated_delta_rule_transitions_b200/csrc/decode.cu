@@ -90,7 +90,7 @@ __global__ void __launch_bounds__(128) decode_main_kernel(DecodeArgs a) {
       for (int t = 1; t < mp; ++t) mx = fmaxf(mx, __fmul_rn(ldf(bq + (long)t * D), inv_tau));
       float s = 0.0f;
       for (int t = 0; t < mp; ++t)
-        s = __fadd_rn(s, route::rexp(__fsub_rn(__fmul_rn(ldf(bq + (long)t * D), inv_tau), mx), K));
+        s = __fadd_rn(s, route::rexp(route::pool_shift(ldf(bq + (long)t * D), inv_tau, mx), K));
       rq[tid] = __fmul_rn(a.tau, __fadd_rn(mx, route::rlog(__fdiv_rn(s, (float)mp), K)));
       __syncthreads();
     }
@@ -103,7 +103,7 @@ __global__ void __launch_bounds__(128) decode_main_kernel(DecodeArgs a) {
         if (a.mode == HLA_GATES_ROUTED) {
           const float* rkj = rk + (long)j * D;
           float dot = 0.0f;
-          for (int c = 0; c < D; ++c) dot = __fadd_rn(dot, __fmul_rn(rq[c], rkj[c]));
+          for (int c = 0; c < D; ++c) dot = route::dot_step(dot, rq[c], rkj[c]);
           g = route::gate_from_dot(dot, a.c_d, a.bias, K);
         }
         keep = a.thr <= 0.0f || g >= a.thr;
@@ -171,7 +171,7 @@ __global__ void decode_close_pool_kernel(DecodeArgs a) {
   for (int t = 1; t < a.C; ++t) mx = fmaxf(mx, __fmul_rn(ldf(bk + (long)t * D), inv_tau));
   float s = 0.0f;
   for (int t = 0; t < a.C; ++t)
-    s = __fadd_rn(s, route::rexp(__fsub_rn(__fmul_rn(ldf(bk + (long)t * D), inv_tau), mx), K));
+    s = __fadd_rn(s, route::rexp(route::pool_shift(ldf(bk + (long)t * D), inv_tau, mx), K));
   a.rk[((long)bh * a.max_chunks + n) * D + tid] =
       __fmul_rn(a.tau, __fadd_rn(mx, route::rlog(__fdiv_rn(s, (float)a.C), K)));
 }

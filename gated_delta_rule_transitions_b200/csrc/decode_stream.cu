@@ -91,7 +91,7 @@ __device__ __forceinline__ int decode_prologue(const DecodeArgs& a, int bh, int 
       for (int t = 1; t < mp; ++t) mx = fmaxf(mx, __fmul_rn(ldf(bq + (long)t * kD), inv_tau));
       float s = 0.0f;
       for (int t = 0; t < mp; ++t)
-        s = __fadd_rn(s, route::rexp(__fsub_rn(__fmul_rn(ldf(bq + (long)t * kD), inv_tau), mx), K));
+        s = __fadd_rn(s, route::rexp(route::pool_shift(ldf(bq + (long)t * kD), inv_tau, mx), K));
       rq[tid] = __fmul_rn(a.tau, __fadd_rn(mx, route::rlog(__fdiv_rn(s, (float)mp), K)));
       tc::bar_sync(1, kCompute);
     }
@@ -106,10 +106,10 @@ __device__ __forceinline__ int decode_prologue(const DecodeArgs& a, int bh, int 
           float dot = 0.0f;
           for (int c4 = 0; c4 < kD / 4; ++c4) {
             const float4 r4 = rkj[c4];
-            dot = __fadd_rn(dot, __fmul_rn(rq[4 * c4 + 0], r4.x));
-            dot = __fadd_rn(dot, __fmul_rn(rq[4 * c4 + 1], r4.y));
-            dot = __fadd_rn(dot, __fmul_rn(rq[4 * c4 + 2], r4.z));
-            dot = __fadd_rn(dot, __fmul_rn(rq[4 * c4 + 3], r4.w));
+            dot = route::dot_step(dot, rq[4 * c4 + 0], r4.x);
+            dot = route::dot_step(dot, rq[4 * c4 + 1], r4.y);
+            dot = route::dot_step(dot, rq[4 * c4 + 2], r4.z);
+            dot = route::dot_step(dot, rq[4 * c4 + 3], r4.w);
           }
           g = route::gate_from_dot(dot, a.c_d, a.bias, K);
         }

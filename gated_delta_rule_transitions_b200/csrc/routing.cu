@@ -1,5 +1,6 @@
 // Routing kernels: per-chunk log-mean-exp pools, gates and compacted active lists.
-// Built with -fmad=false; the recipe itself only uses __f*_rn intrinsics.
+// Built with -fmad=false; the recipe's products and sums are __f*_rn intrinsics or
+// explicit fused multiply-adds.
 #include "common.cuh"
 #include "kernels.cuh"
 #include "routing_recipe.cuh"
@@ -7,18 +8,99 @@
 namespace hla {
 
 // ---------------------------------------------------------------------------
-// Pools.  grid (N, B, 2), block 256.  blockIdx.z = 0 pools x0 into r0, 1 pools x1
-// into r1.  Threads stride over the H*d channels of one chunk; for a fixed token
-// the H*d channels are contiguous, so every token row is read coalesced, twice
-// (max pass, then sum pass; the second pass hits L2).
+// Pools.  grid (N, B, 2 * groups), 64 threads; blockIdx.z = tensor * groups + group,
+// a group is 128 consecutive channels of the H*d channel row and a thread owns two
+// adjacent channels of one chunk.  For a fixed token the H*d channels are
+// contiguous, so every token row is read coalesced.  bf16 inputs are read once
+// into registers (one bf16 pair per token); float32 inputs are read twice (the
+// second pass hits L1/L2).
+//   max:  multiplying by 1/tau > 0 is monotone under rounding, so
+//         max_t fl(x_t * (1/tau)) = fl((max_t x_t) * (1/tau)): one multiply per
+//         channel.
+//   sum:  s = sum_t exp(fma(x_t, 1/tau, -m)) in ascending t; the two channels
+//         of a thread go through packed float32 pairs.
 // out index: ((b*H + h)*out_chunk_stride + c)*d + ch.
 // ---------------------------------------------------------------------------
+
+namespace {
+// The recipe's e^x on a pair of values with packed float32 arithmetic
+// (sm_100; each lane of __ffma2_rn / __fadd2_rn / __fmul2_rn is rounded as its
+// scalar counterpart).  Every product that feeds a sum is a fused multiply-add in
+// the recipe itself, because the code generator contracts a packed multiply that
+// feeds a packed add; the product p * 2^n that the caller adds to its sum is exact,
+// so contracting it changes no bit.
+//   kInRange = true:  both inputs in [-86, 88] (the bits of route::rexp_core);
+//   kInRange = false: inputs <= 0, those below -86 give 0 (route::rexp_nonpos).
+template <bool kInRange>
+__device__ __forceinline__ float2 rexp2(float2 x, const route::Consts& k) {
+  const float2 xc = kInRange ? x : make_float2(fmaxf(x.x, -86.0f), fmaxf(x.y, -86.0f));
+  const float2 sum = __ffma2_rn(xc, make_float2(k.log2e, k.log2e), make_float2(route::kRoundMagic, route::kRoundMagic));
+  const float2 n = __fadd2_rn(sum, make_float2(-route::kRoundMagic, -route::kRoundMagic));
+  const float2 nn = make_float2(-n.x, -n.y);
+  const float2 r = __ffma2_rn(nn, make_float2(k.ln2_lo, k.ln2_lo), __ffma2_rn(nn, make_float2(k.ln2_hi, k.ln2_hi), xc));
+  float2 p = make_float2((float)(1.0 / 5040.0), (float)(1.0 / 5040.0));
+  p = __ffma2_rn(p, r, make_float2((float)(1.0 / 720.0), (float)(1.0 / 720.0)));
+  p = __ffma2_rn(p, r, make_float2((float)(1.0 / 120.0), (float)(1.0 / 120.0)));
+  p = __ffma2_rn(p, r, make_float2((float)(1.0 / 24.0), (float)(1.0 / 24.0)));
+  p = __ffma2_rn(p, r, make_float2((float)(1.0 / 6.0), (float)(1.0 / 6.0)));
+  p = __ffma2_rn(p, r, make_float2(0.5f, 0.5f));
+  p = __ffma2_rn(p, r, make_float2(1.0f, 1.0f));
+  p = __ffma2_rn(p, r, make_float2(1.0f, 1.0f));
+  const float2 sc = make_float2(__uint_as_float((__float_as_uint(sum.x) << 23) + route::kScaleOffset),
+                                __uint_as_float((__float_as_uint(sum.y) << 23) + route::kScaleOffset));
+  const float2 e = __fmul2_rn(p, sc);
+  if (kInRange) return e;
+  return make_float2(x.x < -86.0f ? 0.0f : e.x, x.y < -86.0f ? 0.0f : e.y);
+}
+
+// Lane-wise maximum / minimum of two bf16 pairs (exact).
+__device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t bf16x2_min(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("min.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// route::gate_from_dot on a pair of dot products: z = fma(dot, c_d, b), then
+// 1 / (1 + exp(-z)) with the exp's range checks (-z > 88 -> +inf, -z < -86 -> 0).
+__device__ __forceinline__ float2 gate2_from_dot(float2 dot, float c_d, float bias, const route::Consts& k) {
+  const float2 z = __ffma2_rn(dot, make_float2(c_d, c_d), make_float2(bias, bias));
+  const float2 x = make_float2(-z.x, -z.y);
+  const float2 xc = make_float2(fminf(fmaxf(x.x, -86.0f), 88.0f), fminf(fmaxf(x.y, -86.0f), 88.0f));
+  float2 e = rexp2<true>(xc, k);
+  e.x = x.x > 88.0f ? CUDART_INF_F : (x.x < -86.0f ? 0.0f : e.x);
+  e.y = x.y > 88.0f ? CUDART_INF_F : (x.y < -86.0f ? 0.0f : e.y);
+  const float2 den = __fadd2_rn(make_float2(1.0f, 1.0f), e);
+  return make_float2(__frcp_rn(den.x), __frcp_rn(den.y));
+}
+
+// s += exp(fma(x_t, inv_tau, -m)) over the staged bf16 pairs, ascending t.
+template <bool kInRange>
+__device__ __forceinline__ float2 pool_sum_bf16(const uint32_t (&w)[64], int n, float inv_tau, float m0, float m1,
+                                                const route::Consts& K) {
+  float2 s = make_float2(0.0f, 0.0f);
+#pragma unroll
+  for (int t = 0; t < 64; ++t)
+    if (t < n) {
+      const float2 u = __ffma2_rn(make_float2(__uint_as_float(w[t] << 16), __uint_as_float(w[t] & 0xFFFF0000u)),
+                                  make_float2(inv_tau, inv_tau), make_float2(-m0, -m1));
+      s = __fadd2_rn(s, rexp2<kInRange>(u, K));
+    }
+  return s;
+}
+}  // namespace
+
+constexpr int kPoolMaxC = 64;  // pool_sum_bf16 stages 64 tokens
+
 template <typename Tin>
 __global__ void __launch_bounds__(64) pool_kernel(const Tin* __restrict__ x0, const Tin* __restrict__ x1,
                                                   float* __restrict__ r0, float* __restrict__ r1, int T, int H,
                                                   int d, int C, int out_chunk_stride, float tau) {
-  // grid (N, B, 2 * groups): blockIdx.z = tensor * groups + group; a group is 128
-  // consecutive channels of the H*d channel row; thread = 2 adjacent channels.
+  constexpr bool kBf16 = sizeof(Tin) == 2;
   const int groups = (H * d + 127) / 128;
   const int c = blockIdx.x;
   const int b = blockIdx.y;
@@ -35,15 +117,48 @@ __global__ void __launch_bounds__(64) pool_kernel(const Tin* __restrict__ x0, co
   const int t0 = c * C;
   const int n = min(C, T - t0);
   const Tin* col = x + ((size_t)b * T + t0) * HD + ch0;
-  float m0 = __fmul_rn(ldf(col), inv_tau), m1 = __fmul_rn(ldf(col + 1), inv_tau);
-  for (int t = 1; t < n; ++t) {
-    m0 = fmaxf(m0, __fmul_rn(ldf(col + (size_t)t * HD), inv_tau));
-    m1 = fmaxf(m1, __fmul_rn(ldf(col + (size_t)t * HD + 1), inv_tau));
-  }
-  float s0 = 0.0f, s1 = 0.0f;
-  for (int t = 0; t < n; ++t) {
-    s0 = __fadd_rn(s0, route::rexp(__fsub_rn(__fmul_rn(ldf(col + (size_t)t * HD), inv_tau), m0), K));
-    s1 = __fadd_rn(s1, route::rexp(__fsub_rn(__fmul_rn(ldf(col + (size_t)t * HD + 1), inv_tau), m1), K));
+  float s0 = 0.0f, s1 = 0.0f, m0, m1;
+  if constexpr (kBf16) {
+    // H*d and ch0 are even, so each bf16 pair is one aligned 32-bit word
+    const uint32_t* colw = reinterpret_cast<const uint32_t*>(col);
+    const size_t stride = (size_t)HD / 2;
+    uint32_t w[kPoolMaxC];
+#pragma unroll
+    for (int t = 0; t < kPoolMaxC; ++t) w[t] = t < n ? __ldg(colw + t * stride) : 0u;
+    uint32_t hi = w[0], lo = w[0];
+#pragma unroll
+    for (int t = 1; t < kPoolMaxC; ++t)
+      if (t < n) {
+        hi = bf16x2_max(hi, w[t]);
+        lo = bf16x2_min(lo, w[t]);
+      }
+    m0 = __fmul_rn(__uint_as_float(hi << 16), inv_tau);
+    m1 = __fmul_rn(__uint_as_float(hi & 0xFFFF0000u), inv_tau);
+    // fma is monotone in x (1/tau > 0), so the smallest shifted value comes from the
+    // smallest input; when it is >= -86 no exp of the chunk needs the range checks
+    const bool in_range = __fmaf_rn(__uint_as_float(lo << 16), inv_tau, -m0) >= -86.0f &&
+                          __fmaf_rn(__uint_as_float(lo & 0xFFFF0000u), inv_tau, -m1) >= -86.0f;
+    const float2 ss = in_range ? pool_sum_bf16<true>(w, n, inv_tau, m0, m1, K)
+                               : pool_sum_bf16<false>(w, n, inv_tau, m0, m1, K);
+    s0 = ss.x;
+    s1 = ss.y;
+  } else {
+    const float2* colf = reinterpret_cast<const float2*>(col);
+    const size_t stride = (size_t)HD / 2;
+    float2 v = colf[0];
+    float a0 = v.x, a1 = v.y;
+    for (int t = 1; t < n; ++t) {
+      v = colf[t * stride];
+      a0 = fmaxf(a0, v.x);
+      a1 = fmaxf(a1, v.y);
+    }
+    m0 = __fmul_rn(a0, inv_tau);
+    m1 = __fmul_rn(a1, inv_tau);
+    for (int t = 0; t < n; ++t) {
+      v = colf[t * stride];
+      s0 = __fadd_rn(s0, route::rexp_nonpos(route::pool_shift(v.x, inv_tau, m0), K));
+      s1 = __fadd_rn(s1, route::rexp_nonpos(route::pool_shift(v.y, inv_tau, m1), K));
+    }
   }
   const float v0 = __fmul_rn(tau, __fadd_rn(m0, route::rlog(__fdiv_rn(s0, (float)n), K)));
   const float v1 = __fmul_rn(tau, __fadd_rn(m1, route::rlog(__fdiv_rn(s1, (float)n), K)));
@@ -79,7 +194,7 @@ __global__ void __launch_bounds__(256) gates_kernel(GatesArgs a) {
       if (a.mode == HLA_GATES_ROUTED) {
         const float* rkj = rk + (size_t)j * a.d;
         float dot = 0.0f;
-        for (int c = 0; c < a.d; ++c) dot = __fadd_rn(dot, __fmul_rn(rq[c], rkj[c]));
+        for (int c = 0; c < a.d; ++c) dot = route::dot_step(dot, rq[c], rkj[c]);
         g = route::gate_from_dot(dot, a.c_d, a.bias, K);
       } else if (a.mode == HLA_GATES_ONE) {
         g = 1.0f;
@@ -110,78 +225,125 @@ __global__ void __launch_bounds__(256) gates_kernel(GatesArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// Routed gates, tiled: one CTA per (64 query chunks, b, h).  Each thread computes a
-// 4 x 4 block of a 64 x 64 gate tile; every dot product still runs over channels in
-// ascending order with separately rounded products and sums, so the bits equal the
-// per-pair recipe.  Active chunks are compacted row by row in ascending j.
+// Routed gates, tiled: one CTA per (TI query chunks, b, h), 256 threads.  A thread
+// computes 4 rows x CPT columns of a TI x 64 gate tile (TI = 64: 4 x 4; TI = 16,
+// for grids too small to fill the GPU: 4 x 1).  Every dot product still runs over
+// channels in ascending order with separately rounded products and sums, so the
+// bits equal the per-pair recipe.  Active chunks are compacted row by row in
+// ascending j.
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, int TI>
 __global__ void __launch_bounds__(256) gates_tiled_kernel(GatesArgs a) {
-  constexpr int TI = 64, TJ = 64;
+  constexpr int TJ = 64;
+  constexpr int CPT = (TI * TJ) / (256 * 4);  // columns per thread
+  constexpr int NTX = TJ / CPT;               // threads along j
+  constexpr int QMASK = TI / 4 - 1;           // swizzle range of the rq tile
+  constexpr int FILL_Q = (TI / 4) * D / 256;  // float4 stores per thread, rq tile
+  constexpr int FILL_K = (TJ / 4) * D / 256;  // float4 stores per thread, rk tile
+  static_assert(CPT == 1 || CPT == 4, "tile shape");
+  static_assert(FILL_Q >= 1 && FILL_K >= 1, "tile shape");
   extern __shared__ float smf[];
   float(*rqT)[TI] = reinterpret_cast<float(*)[TI]>(smf);            // [D][TI] rq tile, channel-major
   float(*rkT)[TJ] = reinterpret_cast<float(*)[TJ]>(smf + D * TI);   // [D][TJ] rk tile, channel-major
-  float(*G)[TJ + 1] = reinterpret_cast<float(*)[TJ + 1]>(smf + 2 * D * TI);  // [TI][TJ+1]
-  int* cnt_s = reinterpret_cast<int*>(smf + 2 * D * TI + TI * (TJ + 1));     // [TI]
+  float(*G)[TJ + 1] = reinterpret_cast<float(*)[TJ + 1]>(smf + D * TI + D * TJ);  // [TI][TJ+1]
+  int* cnt_s = reinterpret_cast<int*>(smf + D * TI + D * TJ + TI * (TJ + 1));      // [TI]
   const int i0 = blockIdx.x * TI;
   const int bh = blockIdx.y;
   const int tid = threadIdx.x;
-  const int ty = tid >> 4, tx = tid & 15;
+  const int ty = tid / NTX, tx = tid % NTX;
   const int warp = tid >> 5, lane = tid & 31;
   const route::Consts K = route::make_consts();
   const float* rq = a.rq + (size_t)bh * a.N * D;
   const float* rk = a.rk + (size_t)bh * a.N * D;
   // Tiles are channel-major with their float4 row groups XOR-swizzled by the channel
-  // (group g of channel c at slot g ^ (c % 16)): the fill below (one channel, four
-  // consecutive rows per thread, one 16-byte store) and the float4 reads of the dot
-  // products are both free of bank conflicts.
-  for (int e = tid; e < (TI / 4) * D; e += 256) {
-    const int g = e / D, c = e - g * D;
-    float4 v;
-    float* vp = &v.x;
+  // (group g of channel c at slot g ^ (c % groups)): the fill below (one channel,
+  // four consecutive rows per thread, one 16-byte store) and the reads of the dot
+  // products are free of bank conflicts.  All loads of a fill are issued before its
+  // stores.
+  {
+    float4 v[FILL_Q];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int i = i0 + 4 * g + u;
-      vp[u] = i < a.N ? rq[(size_t)i * D + c] : 0.0f;
+    for (int f = 0; f < FILL_Q; ++f) {
+      const int e = tid + 256 * f;
+      const int g = e / D, c = e - g * D;
+      float* vp = &v[f].x;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + 4 * g + u;
+        vp[u] = i < a.N ? rq[(size_t)i * D + c] : 0.0f;
+      }
     }
-    *(float4*)&rqT[c][(g ^ (c & 15)) << 2] = v;
+#pragma unroll
+    for (int f = 0; f < FILL_Q; ++f) {
+      const int e = tid + 256 * f;
+      const int g = e / D, c = e - g * D;
+      *(float4*)&rqT[c][(g ^ (c & QMASK)) << 2] = v[f];
+    }
   }
   if (tid < TI) cnt_s[tid] = 0;
   const int i_last = min(a.N, i0 + TI) - 1;
-  for (int j0 = 0; j0 < i_last; j0 += TJ) {
-    __syncthreads();
-    for (int e = tid; e < (TJ / 4) * D; e += 256) {
+  // rk tiles are software-pipelined: the next tile's loads are in flight while the
+  // current tile is multiplied
+  float4 v[FILL_K];
+  auto load_rk = [&](int j0) {
+#pragma unroll
+    for (int f = 0; f < FILL_K; ++f) {
+      const int e = tid + 256 * f;
       const int g = e / D, c = e - g * D;
-      float4 v;
-      float* vp = &v.x;
+      float* vp = &v[f].x;
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int j = j0 + 4 * g + u;
         vp[u] = j < a.N ? rk[(size_t)j * D + c] : 0.0f;
       }
-      *(float4*)&rkT[c][(g ^ (c & 15)) << 2] = v;
+    }
+  };
+  if (i_last > 0) load_rk(0);
+  for (int j0 = 0; j0 < i_last; j0 += TJ) {
+    __syncthreads();  // the previous tile's readers are done
+#pragma unroll
+    for (int f = 0; f < FILL_K; ++f) {
+      const int e = tid + 256 * f;
+      const int g = e / D, c = e - g * D;
+      *(float4*)&rkT[c][(g ^ (c & 15)) << 2] = v[f];
     }
     __syncthreads();
-    float acc[4][4];
+    if (j0 + TJ < i_last) load_rk(j0 + TJ);
+    // accumulators of rows (2p, 2p + 1) and column w, packed as one float pair:
+    // each lane of a packed fused multiply-add is rounded on its own
+    float2 acc[2][CPT];
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
+    for (int u = 0; u < 2; ++u)
 #pragma unroll
-      for (int w = 0; w < 4; ++w) acc[u][w] = 0.0f;
+      for (int w = 0; w < CPT; ++w) acc[u][w] = make_float2(0.0f, 0.0f);
 #pragma unroll 4
     for (int c = 0; c < D; ++c) {
-      const float4 q4 = *(const float4*)&rqT[c][(ty ^ (c & 15)) << 2];
-      const float4 k4 = *(const float4*)&rkT[c][(tx ^ (c & 15)) << 2];
-      const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
-      const float kv[4] = {k4.x, k4.y, k4.z, k4.w};
+      const float4 q4 = *(const float4*)&rqT[c][(ty ^ (c & QMASK)) << 2];
+      const float2 qv[2] = {make_float2(q4.x, q4.y), make_float2(q4.z, q4.w)};
+      float kv[CPT];
+      if constexpr (CPT == 4) {
+        const float4 k4 = *(const float4*)&rkT[c][(tx ^ (c & 15)) << 2];
+        kv[0] = k4.x;
+        kv[1] = k4.y;
+        kv[2] = k4.z;
+        kv[3] = k4.w;
+      } else {
+        kv[0] = rkT[c][(((tx >> 2) ^ (c & 15)) << 2) | (tx & 3)];
+      }
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
+      for (int u = 0; u < 2; ++u)
 #pragma unroll
-        for (int w = 0; w < 4; ++w) acc[u][w] = __fadd_rn(acc[u][w], __fmul_rn(qv[u], kv[w]));
+        for (int w = 0; w < CPT; ++w)
+          acc[u][w] = __ffma2_rn(qv[u], make_float2(kv[w], kv[w]), acc[u][w]);
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
+    for (int u = 0; u < 2; ++u)
 #pragma unroll
-      for (int w = 0; w < 4; ++w) G[ty * 4 + u][tx * 4 + w] = route::gate_from_dot(acc[u][w], a.c_d, a.bias, K);
+      for (int w = 0; w < CPT; ++w) {
+        const float2 g = gate2_from_dot(acc[u][w], a.c_d, a.bias, K);
+        G[ty * 4 + 2 * u][tx * CPT + w] = g.x;
+        G[ty * 4 + 2 * u + 1][tx * CPT + w] = g.y;
+      }
     __syncthreads();
     // compaction: warp w handles rows w, w+8, ...
     for (int r = warp; r < TI; r += 8) {
@@ -231,11 +393,23 @@ __global__ void __launch_bounds__(256) gates_tiled_kernel(GatesArgs a) {
   }
 }
 
+template <int D, int TI>
+static cudaError_t launch_gates_tiled(const GatesArgs& a, cudaStream_t s) {
+  dim3 grid((a.N + TI - 1) / TI, a.B * a.H);
+  const size_t smem = (size_t)(D * TI + D * 64 + TI * 65 + TI) * 4;
+  cudaError_t e = cudaFuncSetAttribute(gates_tiled_kernel<D, TI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  gates_tiled_kernel<D, TI><<<grid, 256, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
 // ---------------------------------------------------------------------------
 // Launchers
 // ---------------------------------------------------------------------------
 cudaError_t launch_pools(const void* x0, const void* x1, float* r0, float* r1, int B, int T, int H, int d,
                          int C, int out_chunk_stride, float tau, int dtype, cudaStream_t s) {
+  if (C > kPoolMaxC) return cudaErrorInvalidValue;
   const int N = (T + C - 1) / C;
   const int groups = (H * d + 127) / 128;
   dim3 grid(N, B, 2 * groups);
@@ -250,19 +424,11 @@ cudaError_t launch_pools(const void* x0, const void* x1, float* r0, float* r1, i
 
 cudaError_t launch_gates(const GatesArgs& a, cudaStream_t s) {
   if (a.mode == HLA_GATES_ROUTED && (a.d == 128 || a.d == 64)) {
-    dim3 grid((a.N + 63) / 64, a.B * a.H);
-    const size_t smem = (size_t)(2 * a.d * 64 + 64 * 65 + 64) * 4;
-    cudaError_t e;
-    if (a.d == 128) {
-      e = cudaFuncSetAttribute(gates_tiled_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e != cudaSuccess) return e;
-      gates_tiled_kernel<128><<<grid, 256, smem, s>>>(a);
-    } else {
-      e = cudaFuncSetAttribute(gates_tiled_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e != cudaSuccess) return e;
-      gates_tiled_kernel<64><<<grid, 256, smem, s>>>(a);
-    }
-    return cudaGetLastError();
+    // 64-row tiles while they give two CTAs per SM or more, else 16-row tiles
+    const long tiles64 = (long)((a.N + 63) / 64) * a.B * a.H;
+    const bool small = tiles64 < 2L * num_sms();
+    if (a.d == 128) return small ? launch_gates_tiled<128, 16>(a, s) : launch_gates_tiled<128, 64>(a, s);
+    return small ? launch_gates_tiled<64, 16>(a, s) : launch_gates_tiled<64, 64>(a, s);
   }
   const long rows = (long)a.B * a.H * a.N;
   const int blocks = (int)((rows * 32 + 255) / 256);

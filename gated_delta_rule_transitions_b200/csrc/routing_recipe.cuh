@@ -4,21 +4,23 @@
 // Plain English": a sigmoid weight per historical chunk, thresholded without
 // renormalisation).  Gates decide which chunks are skipped, so this file fixes the
 // exact sequence of binary32 operations: only correctly rounded add, subtract,
-// multiply, divide (the __f*_rn intrinsics, which are never fused into FMA),
-// round-to-nearest-even to integer, and exact scaling by powers of two.
+// multiply, divide, fused multiply-add (fma: a*b + c rounded once) and exact
+// scaling by powers of two.  Products and sums written as separate operations use
+// the __f*_rn intrinsics, which are never fused.
 //
-//   exp:  n = rint(x * log2e);  r = (x - n*ln2_hi) - n*ln2_lo  (ln2_hi has 16
-//         significant bits so n*ln2_hi is exact);  p = Taylor series of e^r to r^7
-//         in Horner form (p = p*r + 1/k!);  result = p * 2^n.  x > 88 -> +inf,
-//         x < -86 -> 0.
+//   exp:  n = rint(x * log2e) of the exact product, as fma(x, log2e, 1.5 * 2^23)
+//         - 1.5 * 2^23;  r = fma(-n, ln2_lo, fma(-n, ln2_hi, x));
+//         p = Taylor series of e^r to r^7 in Horner form, p = fma(p, r, 1/k!);
+//         result = p * 2^n.  x > 88 -> +inf, x < -86 -> 0.
 //   log:  x = m 2^e with m in [sqrt(1/2), sqrt(2));  f = (m-1)/(m+1);
 //         log m = 2 (f + f^3 p(f^2)), p = odd-reciprocal series 1/3 .. 1/15 in
-//         Horner form;  result = e*ln2_hi + (log m + e*ln2_lo).
-//   pool: y_t = x_t * (1/tau); m = max y_t; s = sum_t exp(y_t - m) in ascending t;
-//         r = tau * (m + log(s / n)).
-//   gate: dot = sum_c rq[c]*rk[c] in ascending c (product and sum rounded
-//         separately); z = dot*c_d + b with c_d = 1/sqrt(d) rounded once from
-//         double;  g = 1 / (1 + exp(-z)).
+//         Horner form with separate products and sums;
+//         result = e*ln2_hi + (log m + e*ln2_lo).
+//   pool: inv = 1/tau; m = max_t (x_t * inv); s = sum_t exp(fma(x_t, inv, -m)) in
+//         ascending t;  r = tau * (m + log(s / n)).
+//   gate: dot = fma(rq[c], rk[c], dot) over ascending c from 0;
+//         z = fma(dot, c_d, b) with c_d = 1/sqrt(d) rounded once from double;
+//         g = 1 / (1 + exp(-z)).
 // All constants are derived from ln 2, 1/k! and 1/(2k+1), rounded once to binary32.
 #pragma once
 
@@ -45,22 +47,42 @@ __device__ __forceinline__ Consts make_consts() {
   return k;
 }
 
+// Round to nearest even of a product, |x * log2e| < 2^22: adding 1.5 * 2^23 inside
+// one fma puts the sum in [2^23, 2^24), where the spacing is 1, so the rounded sum is
+// 1.5 * 2^23 + rint(x * log2e) (ties go to the even integer, as 1.5 * 2^23 is even)
+// and the subtraction is exact.  The integer n sits in the low bits of the sum:
+// bits(sum) = 0x4B400000 + n.
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
+constexpr unsigned int kRoundMagicBits = 0x4B400000u;
+constexpr unsigned int kScaleOffset = (127u - kRoundMagicBits) << 23;  // 2^n = bits(sum) << 23 + this
+
+// e^x for -86 <= x <= 88 (no range checks).
+__device__ __forceinline__ float rexp_core(float x, const Consts& k) {
+  const float sum = __fmaf_rn(x, k.log2e, kRoundMagic);
+  const float n = __fsub_rn(sum, kRoundMagic);
+  const float r = __fmaf_rn(-n, k.ln2_lo, __fmaf_rn(-n, k.ln2_hi, x));
+  float p = (float)(1.0 / 5040.0);
+  p = __fmaf_rn(p, r, (float)(1.0 / 720.0));
+  p = __fmaf_rn(p, r, (float)(1.0 / 120.0));
+  p = __fmaf_rn(p, r, (float)(1.0 / 24.0));
+  p = __fmaf_rn(p, r, (float)(1.0 / 6.0));
+  p = __fmaf_rn(p, r, (float)(1.0 / 2.0));
+  p = __fmaf_rn(p, r, 1.0f);
+  p = __fmaf_rn(p, r, 1.0f);
+  const float scale = __uint_as_float((__float_as_uint(sum) << 23) + kScaleOffset);
+  return __fmul_rn(p, scale);
+}
+
 __device__ __forceinline__ float rexp(float x, const Consts& k) {
   if (x > 88.0f) return CUDART_INF_F;
   if (x < -86.0f) return 0.0f;
-  const float n = rintf(__fmul_rn(x, k.log2e));
-  const float r = __fsub_rn(__fsub_rn(x, __fmul_rn(n, k.ln2_hi)), __fmul_rn(n, k.ln2_lo));
-  float p = (float)(1.0 / 5040.0);
-  p = __fadd_rn(__fmul_rn(p, r), (float)(1.0 / 720.0));
-  p = __fadd_rn(__fmul_rn(p, r), (float)(1.0 / 120.0));
-  p = __fadd_rn(__fmul_rn(p, r), (float)(1.0 / 24.0));
-  p = __fadd_rn(__fmul_rn(p, r), (float)(1.0 / 6.0));
-  p = __fadd_rn(__fmul_rn(p, r), (float)(1.0 / 2.0));
-  p = __fadd_rn(__fmul_rn(p, r), 1.0f);
-  p = __fadd_rn(__fmul_rn(p, r), 1.0f);
-  const int ni = (int)n;
-  const float scale = __int_as_float((ni + 127) << 23);
-  return __fmul_rn(p, scale);
+  return rexp_core(x, k);
+}
+
+// e^x for x <= 0 (the pool's shifted values).
+__device__ __forceinline__ float rexp_nonpos(float x, const Consts& k) {
+  const float e = rexp_core(fmaxf(x, -86.0f), k);
+  return x < -86.0f ? 0.0f : e;
 }
 
 // Natural log of a positive normal binary32 value.
@@ -87,10 +109,16 @@ __device__ __forceinline__ float rlog(float x, const Consts& k) {
   return __fadd_rn(__fmul_rn(ef, k.ln2_hi), __fadd_rn(log_m, __fmul_rn(ef, k.ln2_lo)));
 }
 
+// The pool's shifted value fma(x, 1/tau, -m).
+__device__ __forceinline__ float pool_shift(float x, float inv_tau, float m) { return __fmaf_rn(x, inv_tau, -m); }
+
+// One step of the gate's dot product.
+__device__ __forceinline__ float dot_step(float acc, float a, float b) { return __fmaf_rn(a, b, acc); }
+
 // Sigmoid of the scaled score, from a finished dot product.
 __device__ __forceinline__ float gate_from_dot(float dot, float c_d, float bias, const Consts& k) {
-  const float z = __fadd_rn(__fmul_rn(dot, c_d), bias);
-  return __fdiv_rn(1.0f, __fadd_rn(1.0f, rexp(-z, k)));
+  const float z = __fmaf_rn(dot, c_d, bias);
+  return __frcp_rn(__fadd_rn(1.0f, rexp(-z, k)));  // 1/x correctly rounded, as 1.0f / x
 }
 
 }  // namespace route

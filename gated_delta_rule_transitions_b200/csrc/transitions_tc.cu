@@ -557,17 +557,10 @@ cudaError_t launch_transitions_tc(const TransArgs& t, cudaStream_t s) {
   a.ab_chunk_stride = t.ab_chunk_stride;
   a.has_wu = t.Wb != nullptr && t.Ub != nullptr;
   a.ell = t.ell;
-  static int num_sms = 0;
-  if (num_sms == 0) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || num_sms <= 0)
-      num_sms = 148;
-  }
   const size_t smem = 1024 + kSmemUsed;
   e = cudaFuncSetAttribute(transitions_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const long grid = total < 2L * num_sms ? total : 2L * num_sms;
+  const long grid = total < 2L * num_sms() ? total : 2L * num_sms();
   transitions_tc_kernel<<<(unsigned)grid, 128, smem, s>>>(tk, tv, twb, tub, ta, tb, a);
   return cudaGetLastError();
 }

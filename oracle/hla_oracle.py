@@ -138,10 +138,12 @@ def route_pools(x_route, C: int, tau: float):
     """Per-chunk log-mean-exp pools of one head's route tokens [T, d] -> [N, d] f32."""
     x = np.asarray(x_route, np.float32)
     T = x.shape[0]
-    out = []
-    for (a, b) in chunk_bounds(T, C):
-        out.append(rr.lme_pool32(x[a:b], tau))
-    return np.stack(out).astype(np.float32)
+    full = T // C
+    # complete chunks pooled side by side (each chunk on its own, same steps)
+    out = [rr.lme_pool32(x[:full * C].reshape(full, C, -1), tau)] if full else []
+    if T > full * C:
+        out.append(rr.lme_pool32(x[full * C:], tau)[None])
+    return np.concatenate(out).astype(np.float32)
 
 
 def gate_matrix(rq, rk, d: int, bias: float, mode: str = GATES_ROUTED, user=None):

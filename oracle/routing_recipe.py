@@ -22,19 +22,23 @@ Why a bit-level recipe
 ----------------------
 Gates decide which chunks are skipped, so the CPU and the GPU must take that
 decision on identical bits.  The recipe below uses only IEEE-754 binary32 operations
-that are correctly rounded (+, -, *, /, round-to-nearest-even to integer, exact
-scaling by powers of two).  There is no fused multiply-add anywhere in it, so every
-conforming implementation of the same sequence of operations produces the same bits.
+that are correctly rounded: +, -, *, /, the fused multiply-add ``fma(a, b, c)``
+(``a*b + c`` rounded once), and exact scaling by powers of two.  Every conforming
+implementation of the same sequence of operations therefore produces the same bits.
+``fma32`` below is that operation, emulated exactly with float64 arithmetic.
 ``exp`` and ``log`` are written here from their mathematical definitions:
 
-* ``exp32`` -- Cody & Waite argument reduction ``x = n*ln2 + r`` with ``ln 2`` split
-  into a 16-significant-bit head (so ``n*ln2_hi`` is exact for |n| < 256) and a tail,
-  then the degree-7 Taylor polynomial of ``e^r`` in Horner form, then exact scaling
-  by ``2^n``.  Inputs above 88 give +inf, inputs below -86 give 0 (so no subnormal
-  result is ever formed).
+* ``exp32`` -- Cody & Waite argument reduction ``x = n*ln2 + r``: ``n`` is the
+  integer nearest (ties to even) to the exact product ``x*log2e``; ``r`` is
+  ``fma(-n, ln2_lo, fma(-n, ln2_hi, x))`` with ``ln 2`` split into a
+  16-significant-bit head and a tail; then the degree-7 Taylor polynomial of
+  ``e^r`` in Horner form, one fma per step; then exact scaling by ``2^n``.  Inputs
+  above 88 give +inf, inputs below -86 give 0 (so no subnormal result is ever
+  formed).
 * ``log32`` -- split ``x = m * 2^e`` with ``m`` in [sqrt(1/2), sqrt(2)), then
-  ``log m = 2 atanh(f)``, ``f = (m-1)/(m+1)``, summed as the odd series up to f^15,
-  plus ``e*ln2`` (head exact, tail rounded).
+  ``log m = 2 atanh(f)``, ``f = (m-1)/(m+1)``, summed as the odd series up to f^15
+  with separately rounded products and sums, plus ``e*ln2`` (head exact, tail
+  rounded).
 
 Constants are derived below from the mathematics (``1/k!``, ``1/(2k+1)``, ``ln 2``),
 each rounded once to binary32.
@@ -77,14 +81,43 @@ def _f32(x):
     return np.asarray(x, dtype=np.float32)
 
 
+def fma32(a, b, c):
+    """Binary32 fused multiply-add, elementwise: the exact a*b + c rounded once to
+    nearest (ties to even).
+
+    The product of two binary32 values is exact in float64 (48 significant bits).
+    The float64 sum ``s`` is the float64 value nearest to the exact sum, and the
+    exact remainder ``e = (a*b + c) - s`` follows from the two-sum identity.  No
+    binary32 rounding boundary (a midpoint between neighbours) can lie strictly
+    between the exact sum and ``s``, so rounding ``s`` to binary32 is already correct
+    unless ``s`` sits exactly on a midpoint; there the exact sum is on the side given
+    by the sign of ``e`` (or on the midpoint itself when ``e`` is zero, where ties go
+    to the even neighbour, as the float64 -> binary32 conversion does).
+    """
+    a, b, c = np.broadcast_arrays(_f32(a), _f32(b), _f32(c))
+    p = a.astype(np.float64) * b.astype(np.float64)
+    c64 = c.astype(np.float64)
+    s = p + c64
+    bv = s - p
+    e = (p - (s - bv)) + (c64 - bv)
+    r = s.astype(np.float32)
+    d = s - r.astype(np.float64)
+    toward = np.where(d > 0, np.float32(np.inf), np.float32(-np.inf))
+    nb = np.nextafter(r, toward)
+    tie = (d != 0) & (s + s == r.astype(np.float64) + nb.astype(np.float64))
+    fix = tie & (e != 0) & (np.sign(e) == np.sign(d))
+    return np.where(fix, nb, r).astype(np.float32)
+
+
 def exp32(x):
     """e^x on binary32 arrays by the recipe above (elementwise, vectorised)."""
     x = _f32(x)
-    n = np.rint(x * LOG2E)  # round half to even, exact integer in float32
-    r = (x - n * LN2_HI) - n * LN2_LO
+    # nearest integer to the exact product (float64 holds it exactly)
+    n = np.rint(x.astype(np.float64) * np.float64(LOG2E)).astype(np.float32)
+    r = fma32(-n, LN2_LO, fma32(-n, LN2_HI, x))
     p = EXP_COEF[7]
     for c in EXP_COEF[6::-1]:
-        p = p * r + c  # two roundings: product, then sum
+        p = fma32(p, r, c)  # one rounding per step
     ni = np.clip(n, -126, 127).astype(np.int32)
     scale = ((ni + 127).astype(np.uint32) << np.uint32(23)).view(np.float32)
     out = (p * scale).astype(np.float32)
@@ -118,9 +151,9 @@ def lme_pool32(x, tau: float, n_tokens=None):
     """Per-channel log-mean-exp pool over axis -2 (tokens) of a binary32 array.
 
     ``x``: [..., n, d].  Returns [..., d].  Steps, in order:
-    inv_tau = 1/tau; y_t = x_t * inv_tau; m = max_t y_t;
-    s = sum over ascending t of exp32(y_t - m), one rounding per add, starting at 0;
-    r = tau * (m + log32(s / n)).
+    inv_tau = 1/tau; m = max_t (x_t * inv_tau);
+    s = sum over ascending t of exp32(fma(x_t, inv_tau, -m)), one rounding per add,
+    starting at 0;  r = tau * (m + log32(s / n)).
     """
     x = _f32(x)
     n = x.shape[-2] if n_tokens is None else n_tokens
@@ -132,7 +165,7 @@ def lme_pool32(x, tau: float, n_tokens=None):
         m = np.maximum(m, y[..., t, :])
     s = np.zeros_like(m)
     for t in range(n):
-        s = s + exp32(y[..., t, :] - m)
+        s = s + exp32(fma32(x[..., t, :], inv_tau, -m))
     mean = s / F32(n)
     return (tau32 * (m + log32(mean))).astype(np.float32)
 
@@ -143,21 +176,21 @@ def gate_scale(d: int) -> np.float32:
 
 
 def dot32(a, b):
-    """Sequential binary32 dot over the last axis: acc = 0; acc = acc + a[c]*b[c],
-    c ascending, product and sum each rounded (no fused multiply-add)."""
+    """Sequential binary32 dot over the last axis: acc = 0; acc = fma(a[c], b[c], acc),
+    c ascending (one rounding per step)."""
     a = _f32(a)
     b = _f32(b)
     a, b = np.broadcast_arrays(a, b)
     acc = np.zeros(a.shape[:-1], dtype=np.float32)
     for c in range(a.shape[-1]):
-        acc = acc + a[..., c] * b[..., c]
+        acc = fma32(a[..., c], b[..., c], acc)
     return acc
 
 
 def gate32(rq, rk, d: int, bias: float):
-    """g = 1 / (1 + exp32(-z)), z = dot32(rq, rk) * c_d + bias, all binary32."""
+    """g = 1 / (1 + exp32(-z)), z = fma(dot32(rq, rk), c_d, bias), all binary32."""
     dot = dot32(rq, rk)
-    z = dot * gate_scale(d) + F32(bias)
+    z = fma32(dot, gate_scale(d), F32(bias))
     return (F32(1.0) / (F32(1.0) + exp32(-z))).astype(np.float32)
 
 

@@ -204,6 +204,47 @@ def test_routing_bit_exact(hla, dtype, d, T):
             P.check_routing_exact(res, gates.cpu(), aidx.cpu(), acnt.cpu(), b, h)
 
 
+@pytest.mark.parametrize("d,H,T,tau,scale", [
+    # tau = 0.05 and large route values: pools whose shifted values fall below -86
+    # (the exp's zero branch) and scores whose exp overflows or underflows
+    (128, 3, 64 * 8 + 5, 0.05, 30.0),
+    # enough 64-row gate tiles to fill the GPU at d = 64 (the 64-row kernel)
+    (64, 37, 64 * 512, 1.0, 1.0),
+])
+def test_routing_bit_exact_ranges(hla, d, H, T, tau, scale):
+    gen = torch.Generator().manual_seed(123)
+    N = (T + 63) // 64
+    if scale > 1.0:
+        # chunks of route keys around +scale or -scale (alternating), queries around
+        # +scale: pooled scores of either sign and far beyond the exp's range
+        sign = torch.where(torch.arange(T) // 64 % 2 == 0, 1.0, -1.0)[None, :, None, None]
+        qr = (scale * (0.1 * torch.randn(1, T, H, d, generator=gen) + 1.0)).to(torch.bfloat16)
+        kr = (scale * (0.1 * torch.randn(1, T, H, d, generator=gen) + sign)).to(torch.bfloat16)
+    else:
+        qr = torch.randn(1, T, H, d, generator=gen).to(torch.bfloat16)
+        kr = torch.randn(1, T, H, d, generator=gen).to(torch.bfloat16)
+    bias, thr = -1.0, 0.3
+    cfg = hla.make_config(1, H, T, 64, d, "bf16", "routed", tau, bias, thr)
+    rq = torch.empty((1, H, N, d), device="cuda")
+    rk = torch.empty_like(rq)
+    gates = torch.empty((1, H, N, N), device="cuda")
+    aidx = torch.empty((1, H, N, N), dtype=torch.int32, device="cuda")
+    acnt = torch.empty((1, H, N), dtype=torch.int32, device="cuda")
+    hla.hla_routing(cfg, qr.cuda(), kr.cuda(), rq, rk, gates, aidx, acnt)
+    torch.cuda.synchronize()
+    for h in (0, H - 1):
+        rq_ref = ho.route_pools(P.np32(qr[0, :, h]), 64, tau)
+        rk_ref = ho.route_pools(P.np32(kr[0, :, h]), 64, tau)
+        assert np.array_equal(rq[0, h].cpu().numpy().view(np.uint32), rq_ref.view(np.uint32))
+        assert np.array_equal(rk[0, h].cpu().numpy().view(np.uint32), rk_ref.view(np.uint32))
+        G = ho.gate_matrix(rq_ref, rk_ref, d, bias)
+        if scale > 1.0:
+            low = np.tril(np.ones_like(G, dtype=bool), -1)
+            assert (G[low] == 0.0).any() and (G[low] == 1.0).any()  # both saturations reached
+        res = ho.HeadResult(o=None, gates=G, active=ho.active_lists(G, thr), rq=rq_ref, rk=rk_ref)
+        P.check_routing_exact(res, gates.cpu(), aidx.cpu(), acnt.cpu(), 0, h)
+
+
 def test_full_size_prefill_sampled(hla):
     """Dense 0.8B-like layer (T=16384, H=16, d=128, bf16): all gates bit-exact on
     two heads; sampled query chunks against the oracle."""

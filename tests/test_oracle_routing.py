@@ -8,6 +8,7 @@ limits, and the gate against a float64 sigmoid.  Source: HLA summary page,
 renormalisation).
 """
 import math
+from fractions import Fraction
 
 import numpy as np
 import pytest
@@ -122,7 +123,62 @@ def test_gate_saturation():
     assert rr.gate32(one * 0, one * 0, 4, 0.0) == np.float32(0.5)
 
 
-def test_dot32_is_sequential_single_rounding_sum():
+def _round_f32(fr: Fraction) -> np.float32:
+    """Nearest binary32 to an exact rational, ties to the even significand (brute
+    force over the neighbours of a close candidate)."""
+    c = np.float32(float(fr))
+    cands = [np.nextafter(c, np.float32(-np.inf)), c, np.nextafter(c, np.float32(np.inf))]
+    return min(cands, key=lambda v: (abs(Fraction(float(v)) - fr), int(np.array([v]).view(np.uint32)[0]) & 1))
+
+
+def _fma_exact(a, b, c) -> np.float32:
+    return _round_f32(Fraction(float(a)) * Fraction(float(b)) + Fraction(float(c)))
+
+
+def _midpoint_products(rng, count):
+    """Pairs (a, b) of binary32 values whose exact product is a midpoint between two
+    neighbouring binary32 values: (2m + 1) 2^k with 2m + 1 split into two factors
+    of at most 24 bits."""
+    out = []
+    while len(out) < count:
+        m = int(rng.integers(1 << 23, 1 << 24))
+        odd = 2 * m + 1
+        f = next((q for q in range(3, 5800, 2) if odd % q == 0), None)
+        if f is None or odd // f >= (1 << 24):
+            continue
+        ka, kb = int(rng.integers(-30, 0)), int(rng.integers(-30, 0))
+        out.append((np.float32(math.ldexp(f, ka)), np.float32(math.ldexp(odd // f, kb)), ka + kb))
+    return out
+
+
+def test_fma32_matches_exact_rounding():
+    rng = np.random.default_rng(11)
+    # random operands over a range of scales
+    n = 4000
+    a = (rng.standard_normal(n) * np.exp2(rng.integers(-20, 20, n))).astype(np.float32)
+    b = (rng.standard_normal(n) * np.exp2(rng.integers(-20, 20, n))).astype(np.float32)
+    c = (rng.standard_normal(n) * np.exp2(rng.integers(-40, 40, n))).astype(np.float32)
+    got = rr.fma32(a, b, c)
+    ref = np.array([_fma_exact(x, y, z) for x, y, z in zip(a, b, c)], np.float32)
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+    # products that sit exactly on a binary32 midpoint, plus addends far below the
+    # float64 resolution of the sum: rounding the float64 sum would tie to even,
+    # the single rounding of the exact sum goes the way of the addend's sign
+    cases = _midpoint_products(rng, 300)
+    a = np.array([x for x, _, _ in cases], np.float32)
+    b = np.array([y for _, y, _ in cases], np.float32)
+    c = np.array([np.float32(math.ldexp(float(rng.choice([-1.0, 1.0])) * (1 + float(rng.integers(0, 1 << 23)) / 2 ** 23),
+                                        k - 40)) for _, _, k in cases], np.float32)
+    c[::7] = 0.0  # exact ties: even significand
+    got = rr.fma32(a, b, c)
+    ref = np.array([_fma_exact(x, y, z) for x, y, z in zip(a, b, c)], np.float32)
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+    # the float64 sum rounded to binary32 really is wrong on about half of them
+    naive = (a.astype(np.float64) * b.astype(np.float64) + c.astype(np.float64)).astype(np.float32)
+    assert (naive != ref).sum() >= 60
+
+
+def test_dot32_is_sequential_fused_sum():
     # with exactly representable partial sums the sequential sum equals the exact one
     a = np.array([1.0, 2.0, 4.0, 8.0], np.float32)
     assert rr.dot32(a, a) == 85.0
@@ -130,6 +186,12 @@ def test_dot32_is_sequential_single_rounding_sum():
     a = np.array([2.0 ** 12, 1.0, 2.0 ** 12], np.float32)
     b = np.array([2.0 ** 12, 1.0, -(2.0 ** 12)], np.float32)
     assert rr.dot32(a, b) == 0.0
+    # each step is one fused rounding: (1 + 2^-12)^2 - (1 + 2^-11) = 2^-24 exactly,
+    # where a rounded product would give 0
+    u = np.float32(1 + 2.0 ** -12)
+    a = np.array([-(1 + 2.0 ** -11), u], np.float32)
+    b = np.array([1.0, u], np.float32)
+    assert rr.dot32(a, b) == np.float32(2.0 ** -24)
 
 
 def test_gate_matrix_masks_current_and_future():
