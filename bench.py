@@ -260,6 +260,8 @@ def run_ours(args):
     wp = PREFILL_WORKLOADS[args.prefill_workload](syn)
     if args.prefill_T:
         wp = wp.with_(T=args.prefill_T, name=f"{wp.name}_T{args.prefill_T}")
+    if args.chunk != wp.C:
+        wp = wp.with_(C=args.chunk, name=wp.name.replace("_C64_", f"_C{args.chunk}_"))
     # the long sparse workload is generated on the device (5 x 1 GiB of inputs)
     gen_dev = "cuda" if wp.B * wp.T * wp.H * wp.d > (1 << 28) else "cpu"
     inp = syn.make_gdn_inputs(wp, device=gen_dev)
@@ -291,6 +293,8 @@ def run_ours(args):
         wd = wd.with_(B=8, T=64 * 4, name="decode_skipped")
     if args.decode_cache != "dense":
         wd = wd.with_(name=f"{wd.name}_{args.decode_cache}_cache")
+    if args.chunk != wd.C:
+        wd = wd.with_(C=args.chunk, name=wd.name.replace("_C64_", f"_C{args.chunk}_"))
     max_chunks = wd.T // wd.C + 1
     cache, ctx0 = build_decode_cache(hla, syn, torch, wd, max_chunks, group=min(8, wd.B),
                                      cache_format=args.decode_cache)
@@ -400,6 +404,13 @@ def run_ours(args):
         comp_units = active_pairs
         comp_what = f"{active_pairs} active pairs"
     flops_compose = comp_units * 2.0 * d ** 3
+    # transitions and read-out per 64-token sub-chunk; at C > 64 also the merge of
+    # s = C / 64 sub-chunk transitions per complete chunk (2 (s - 1) products) and the
+    # advance of the composed state to the later sub-chunks (s - 1 products per chunk)
+    n_sub = (wp.T + 63) // 64
+    s_sub = wp.C // 64
+    flops_other = wp.B * wp.H * (n_sub * (FLOP_TRANSITION + FLOP_READOUT)
+                                 + (2 * (wp.T // wp.C) + N) * (s_sub - 1) * 2.0 * d ** 3)
     comp_ms, comp_n = stages["compose"]
     comp_avg = comp_ms / max(comp_n, 1)
     comp_tf = flops_compose / (comp_avg * 1e-3) / 1e12 if comp_avg > 0 else None
@@ -437,8 +448,7 @@ def run_ours(args):
                      "traffic": ncu_traffic("compose"), "traffic_unit": "bytes per launch (ncu dram read+write)",
                      "peak_source": f"{peak_src} bf16 dense (burst)",
                      "algorithmic": f"{comp_what} x 2 d^3 = {flops_compose:.4g} flop per launch",
-                     "prefill_frac_of_peak": (flops_compose + N * wp.B * wp.H * (FLOP_TRANSITION + FLOP_READOUT))
-                     / (pre_ms * 1e-3) / 1e12 / bf16_tf},
+                     "prefill_frac_of_peak": (flops_compose + flops_other) / (pre_ms * 1e-3) / 1e12 / bf16_tf},
         "decode": {"value": whole_job_rate(tokens_dec, dec_ms, world), "unit": "tokens/s", "ms_per_step": dec_ms,
                    "roofline": {"kernel": "decode_main", "bound": "hbm", "achieved": dec_gbs, "peak": hbm_gbs,
                                 "unit": "GB/s", "frac": (dec_gbs / hbm_gbs) if dec_gbs else None,
@@ -635,6 +645,8 @@ def main(argv=None):
     ap.add_argument("--skip-decode", action="store_true")
     ap.add_argument("--decode-cache", choices=["dense", "factored"], default="dense",
                     help="dense: A_j/B_j d x d (the metric's workload); factored: K_j, Wb_j, Ub_j per chunk")
+    ap.add_argument("--chunk", type=int, choices=[64, 128, 256], default=64,
+                    help="chunk size C of both workloads (the metric's workloads use 64)")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

@@ -81,7 +81,7 @@ _SIGS = {
     "hla_profile_read": ([_P, _P, ctypes.c_int32], ctypes.c_int),
 }
 
-STAGES = ("pools", "gates", "transitions", "compose", "readout", "cache", "decode", "decode_close")
+STAGES = ("pools", "gates", "transitions", "compose", "readout", "cache", "decode", "decode_close", "chain")
 
 # Every symbol that include/hla.h declares (checked by the CPU tests).
 EXPORTS = tuple(_SIGS)

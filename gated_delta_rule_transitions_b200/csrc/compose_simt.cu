@@ -5,7 +5,8 @@
 //   S <- 0;  for j in active(i), ascending:  S <- S + g_ij ((S A_j + B_j) - S)
 // and para. 4: a chunk whose weight fell below the threshold is the identity and is
 // not read at all (it is absent from the active list).  The result S_in(i) is
-// written as float32 [d_v][d_k] for the read-out.
+// written as float32 [d_v][d_k] for the read-out, into the slot of chunk i's first
+// 64-token sub-chunk.
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -63,7 +64,7 @@ __global__ void __launch_bounds__(256) compose_simt_kernel(ComposeArgs a) {
     }
     __syncthreads();
   }
-  float* out = a.S_in + row * (long)D * D;
+  float* out = a.S_in + (bh * a.n_slots + (long)i * a.slot_mult) * (long)D * D;
   for (int idx = tid; idx < D * D; idx += blockDim.x) {
     const int v = idx / D, cc = idx - v * D;
     out[idx] = S[v * DP + cc];

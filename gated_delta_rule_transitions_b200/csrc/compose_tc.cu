@@ -13,7 +13,7 @@
 // and the MMA operand Aop_k = bf16(g S) also lives in tensor memory.  The epilogue
 // warps then add g B_j[v][c], giving S_new, and prepare the next active step of that
 // chain: D_k <- (1 - g_next) S_new, Aop_k <- bf16(g_next S_new).  After a chain's
-// last active step S_new is written to S_in (float32, [v][c]).
+// last active step S_new is written to S_in (bf16, [v][c]).
 //
 // Warp roles: warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer, warps 2-17
 // epilogue (lane quarter = warp % 4, column quarter = (warp - 2) / 4).  The epilogue
@@ -49,7 +49,8 @@ struct ComposeTcArgs {
   const int32_t* act_idx;
   const float* act_g;
   const int32_t* act_cnt;
-  __nv_bfloat16* S_in;  // [B,H,N,d,d] bf16, row v, column c
+  __nv_bfloat16* S_in;  // [B,H,n_slots,d,d] bf16, row v, column c; S_in(i) in slot i * slot_mult
+  int slot_mult, n_slots;
 };
 
 // Walks the merged ascending active lists of the two chains.
@@ -326,7 +327,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     __nv_bfloat16* out_row[2];
     for (int k = 0; k < 2; ++k) {
       const int chain = chains[k];
-      out_row[k] = chain >= 0 ? a.S_in + ((long)bh * a.N + chain) * kD * kD + (long)v * kD + col0 : nullptr;
+      out_row[k] = chain >= 0 ? a.S_in + ((long)bh * a.n_slots + (long)chain * a.slot_mult) * kD * kD +
+                                    (long)v * kD + col0
+                              : nullptr;
       // a chain with nothing active has S_in = 0 (in scan mode: S_in(0))
       if (chain >= 0 && (kScan || a.act_cnt[(long)bh * a.N + chain] == 0))
         for (int e = 0; e < 4; ++e) ((uint4*)out_row[k])[e] = make_uint4(0u, 0u, 0u, 0u);
@@ -372,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float2 g2 = make_float2(g, g);
         if (kScan || last) {
           // the state after this step (scan mode: S_in(j + 1); else the chain's S_in)
-          uint4* out = (uint4*)(out_row[k] + (kScan ? (long)(e.j + 1) * kD * kD : 0));
+          uint4* out = (uint4*)(out_row[k] + (kScan ? (long)(e.j + 1) * a.slot_mult * kD * kD : 0));
           uint32_t op[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
@@ -467,7 +470,7 @@ cudaError_t make_tmap_rows128(CUtensorMap* m, const void* base, long rows) {
 cudaError_t launch_compose_tc(const ComposeArgs& c, bool scan, cudaStream_t s) {
   if (c.N <= 0) return cudaSuccess;
   if (c.ab_chunk_stride <= 0)  // no complete chunk: every composed state is zero
-    return cudaMemsetAsync(c.S_in, 0, (size_t)c.B * c.H * c.N * kD * kD * sizeof(__nv_bfloat16), s);
+    return cudaMemsetAsync(c.S_in, 0, (size_t)c.B * c.H * c.n_slots * kD * kD * sizeof(__nv_bfloat16), s);
   const long rows = (long)c.B * c.H * c.ab_chunk_stride * kD;
   CUtensorMap tmA, tmB;
   cudaError_t e = make_tmap_rows128(&tmA, c.A, rows);
@@ -482,6 +485,8 @@ cudaError_t launch_compose_tc(const ComposeArgs& c, bool scan, cudaStream_t s) {
   a.act_g = c.act_g;
   a.act_cnt = c.act_cnt;
   a.S_in = (__nv_bfloat16*)c.S_in;
+  a.slot_mult = c.slot_mult;
+  a.n_slots = c.n_slots;
   a.head_major = c.sparse ? 1 : 0;
   a.order = nullptr;
   if (!scan && c.sparse && c.order != nullptr && c.N <= 4096) {

@@ -300,8 +300,9 @@ static cudaError_t launch_close(const DecodeArgs& a, cudaStream_t s) {
   t.ab_chunk_offset = 0;
   t.close_m = a.m_partial;
   t.close_n = a.n_chunks;
-  // the transition kernel never writes past max_chunks; the pool kernel flags it
-  cudaError_t e = launch_transitions(t, s);
+  // the transition kernel never writes past max_chunks; the pool kernel flags it.
+  // Chunks longer than one 64-token WY tile close by the token rule (no workspace).
+  cudaError_t e = a.C > 64 ? launch_transitions_token(t, s) : launch_transitions(t, s);
   if (e != cudaSuccess) return e;
   decode_close_pool_kernel<D, Tio><<<a.B * a.H, D, 0, s>>>(a);
   e = cudaGetLastError();

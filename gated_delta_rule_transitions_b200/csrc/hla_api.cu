@@ -37,7 +37,8 @@ hla_status check_cfg(const hla_config* c, bool need_T) {
   if (c == nullptr) return fail(HLA_ERR_INVALID_ARG, "cfg is NULL");
   if (c->B <= 0 || c->H <= 0) return fail(HLA_ERR_INVALID_ARG, "B and H must be positive (B=%d H=%d)", c->B, c->H);
   if (need_T && c->T <= 0) return fail(HLA_ERR_INVALID_ARG, "T must be positive (T=%d)", c->T);
-  if (c->C != 64) return fail(HLA_ERR_UNSUPPORTED, "chunk size C=%d unsupported (64 only)", c->C);
+  if (c->C != 64 && c->C != 128 && c->C != 256)
+    return fail(HLA_ERR_UNSUPPORTED, "chunk size C=%d unsupported (64, 128, 256)", c->C);
   if (c->dk != c->dv) return fail(HLA_ERR_UNSUPPORTED, "dk != dv (%d, %d) unsupported", c->dk, c->dv);
   if (c->dk != 64 && c->dk != 128) return fail(HLA_ERR_UNSUPPORTED, "head dim %d unsupported (64, 128)", c->dk);
   if (c->dtype != HLA_F32 && c->dtype != HLA_BF16) return fail(HLA_ERR_UNSUPPORTED, "dtype %d unsupported", c->dtype);
@@ -78,9 +79,13 @@ hla_status opt_ptr(const void* p, const char* name) {
 
 float gate_scale(int d) { return (float)(1.0 / std::sqrt((double)d)); }
 
+// The WY solve and the intra-chunk read-out work on sub-chunks of kSub tokens; a
+// chunk of C tokens is C / kSub of them.
+constexpr int kSub = 64;
+
 // Prefill workspace layout.
 struct PrefillWs {
-  size_t rq, rk, act_idx, act_g, act_cnt, order, A, Bm, Wb, Ub, ell, S_in, total;
+  size_t rq, rk, act_idx, act_g, act_cnt, order, A, Bm, Asub, Bsub, Wb, Ub, ell, S_in, total;
 };
 
 PrefillWs prefill_layout(const hla_config* c) {
@@ -88,6 +93,8 @@ PrefillWs prefill_layout(const hla_config* c) {
   const size_t B = c->B, H = c->H, d = c->dk, C = c->C;
   const size_t N = (c->T + C - 1) / C;
   const size_t Nc = c->T / C;
+  const size_t Nsub = (c->T + kSub - 1) / kSub;
+  const size_t Nsub_c = c->T / kSub;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t o = off;
@@ -102,10 +109,14 @@ PrefillWs prefill_layout(const hla_config* c) {
   w.order = take(B * H * N * 4);
   w.A = take(B * H * Nc * d * d * esize(c->dtype));
   w.Bm = take(B * H * Nc * d * d * esize(c->dtype));
-  w.Wb = take(B * H * N * C * d * 4);
-  w.Ub = take(B * H * N * C * d * 4);
-  w.ell = take(B * H * N * C * 4);
-  w.S_in = take(B * H * N * d * d * 4);
+  if (C > kSub) {  // transitions of the complete sub-chunks, merged into A, Bm
+    w.Asub = take(B * H * Nsub_c * d * d * esize(c->dtype));
+    w.Bsub = take(B * H * Nsub_c * d * d * esize(c->dtype));
+  }
+  w.Wb = take(B * H * Nsub * kSub * d * 4);
+  w.Ub = take(B * H * Nsub * kSub * d * 4);
+  w.ell = take(B * H * Nsub * kSub * 4);
+  w.S_in = take(B * H * Nsub * d * d * 4);  // the state entering every sub-chunk
   w.total = off;
   return w;
 }
@@ -258,8 +269,8 @@ hla_status hla_cache_init(const hla_config* cfg, int32_t max_chunks, void* mem, 
   if (max_chunks <= 0) return fail(HLA_ERR_INVALID_ARG, "max_chunks must be positive");
   HLA_TRY(need_ptr(mem, "mem"));
   if (((uintptr_t)mem & 255u) != 0) return fail(HLA_ERR_INVALID_ARG, "cache memory must be 256-byte aligned");
-  if (cfg->cache_format == HLA_CACHE_FACTORED && !(cfg->dtype == HLA_BF16 && cfg->dk == 128))
-    return fail(HLA_ERR_UNSUPPORTED, "a factored cache needs bf16 and d = 128");
+  if (cfg->cache_format == HLA_CACHE_FACTORED && !(cfg->dtype == HLA_BF16 && cfg->dk == 128 && cfg->C == 64))
+    return fail(HLA_ERR_UNSUPPORTED, "a factored cache needs bf16, d = 128 and C = 64");
   const CacheLayout L = cache_layout(cfg, max_chunks);
   if (bytes < L.total) return fail(HLA_ERR_WORKSPACE, "cache block too small: %zu < %zu", bytes, L.total);
   char* base = (char*)mem;
@@ -365,7 +376,9 @@ hla_status gdn_chunk_transitions(const hla_config* cfg, const void* k, const voi
   t.A = A_out;
   t.Bm = B_out;
   t.ab_chunk_stride = Nc;
-  if (cfg->dtype == HLA_BF16 && cfg->dk == 128)
+  if (cfg->C > kSub)  // no workspace here for sub-chunk factors: the token rule per chunk
+    HLA_CUDA(hla::launch_transitions_token(t, (cudaStream_t)stream), "gdn_chunk_transitions (token rule) launch");
+  else if (cfg->dtype == HLA_BF16 && cfg->dk == 128)
     HLA_CUDA(hla::launch_transitions_tc(t, (cudaStream_t)stream), "gdn_chunk_transitions (tensor core) launch");
   else
     HLA_CUDA(hla::launch_transitions(t, (cudaStream_t)stream), "gdn_chunk_transitions launch");
@@ -500,23 +513,37 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
   HLA_TRY(routing_impl(cfg, qr, kr, rq, (cfg->gate_mode == HLA_GATES_ROUTED || cache_out) ? rk : nullptr,
                        user_gates, act_idx, act_g, act_cnt, gates_out, active_idx_out, active_cnt_out, side->s));
   HLA_CUDA(cudaEventRecord(side->join, side->s), "side stream join");
-  // transitions of every chunk (A/B of complete chunks into the cache or workspace)
+  // transitions of every 64-token sub-chunk (A/B of complete ones into the cache or
+  // workspace; at C > 64 into the workspace, merged per chunk below)
+  const int s_sub = cfg->C / kSub;
+  const int Nsub = (cfg->T + kSub - 1) / kSub;
+  const int Nsub_c = cfg->T / kSub;
   hla::TransArgs t{};
   t.B = cfg->B;
   t.H = cfg->H;
   t.T = cfg->T;
-  t.C = cfg->C;
+  t.C = kSub;
   t.d = cfg->dk;
   t.dtype = cfg->dtype;
   t.in = {k, v, alpha, beta, (long)cfg->T * cfg->H * cfg->dk, cfg->dk, (long)cfg->H * cfg->dk,
           (long)cfg->T * cfg->H, 1, cfg->H};
-  t.n_chunks = N;
-  // a dense cache takes A/B straight from the transitions; otherwise they go to the
-  // workspace (the composition reads them) and a factored cache gets the WY factors
+  t.n_chunks = Nsub;
+  // a dense cache takes A/B straight from the transitions (or the merge); otherwise
+  // they go to the workspace (the composition reads them) and a factored cache gets
+  // the WY factors
   const bool dense_out = cache_out != nullptr && cache_out->format == HLA_CACHE_DENSE;
-  t.A = dense_out ? cache_out->A : (void*)(ws + w.A);
-  t.Bm = dense_out ? cache_out->Bm : (void*)(ws + w.Bm);
-  t.ab_chunk_stride = dense_out ? cache_out->max_chunks : Nc;
+  void* A_chunk = dense_out ? cache_out->A : (void*)(ws + w.A);
+  void* B_chunk = dense_out ? cache_out->Bm : (void*)(ws + w.Bm);
+  const long chunk_stride = dense_out ? cache_out->max_chunks : Nc;
+  if (s_sub == 1) {
+    t.A = A_chunk;
+    t.Bm = B_chunk;
+    t.ab_chunk_stride = chunk_stride;
+  } else {
+    t.A = ws + w.Asub;
+    t.Bm = ws + w.Bsub;
+    t.ab_chunk_stride = Nsub_c;
+  }
   t.Wb = (float*)(ws + w.Wb);
   t.Ub = (float*)(ws + w.Ub);
   t.ell = (float*)(ws + w.ell);
@@ -527,6 +554,27 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
     else
       HLA_CUDA(hla::launch_transitions(t, s), "transitions launch");
   }
+  // chunks of C > 64 tokens: each chunk's transition from its sub-chunks' ones
+  hla::ChainArgs ch{};
+  ch.B = cfg->B;
+  ch.H = cfg->H;
+  ch.d = cfg->dk;
+  ch.dtype = cfg->dtype;
+  ch.s = s_sub;
+  ch.Asub = t.A;
+  ch.Bsub = t.Bm;
+  ch.sub_stride = Nsub_c;
+  ch.Nc = Nc;
+  ch.Aout = A_chunk;
+  ch.Bout = B_chunk;
+  ch.out_stride = chunk_stride;
+  ch.N = N;
+  ch.Nsub = Nsub;
+  ch.S = ws + w.S_in;
+  if (s_sub > 1 && Nc > 0) {
+    StageScope _sc(HLA_STAGE_CHAIN, s, 1);
+    HLA_CUDA(hla::launch_chain_merge(ch, s), "chunk merge launch");
+  }
   HLA_CUDA(cudaStreamWaitEvent(s, side->join, 0), "side stream join");
   side_lock.unlock();
   hla::ComposeArgs c{};
@@ -535,13 +583,15 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
   c.N = N;
   c.d = cfg->dk;
   c.dtype = cfg->dtype;
-  c.A = t.A;
-  c.Bm = t.Bm;
-  c.ab_chunk_stride = t.ab_chunk_stride;
+  c.A = A_chunk;
+  c.Bm = B_chunk;
+  c.ab_chunk_stride = Nc > 0 ? chunk_stride : 0;
   c.act_idx = act_idx;
   c.act_g = act_g;
   c.act_cnt = act_cnt;
   c.S_in = (float*)(ws + w.S_in);
+  c.slot_mult = s_sub;
+  c.n_slots = Nsub;
   c.sparse = cfg->skip_threshold > 0.0f;
   c.order = (int32_t*)(ws + w.order);
   {
@@ -553,12 +603,16 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
     else
       HLA_CUDA(hla::launch_compose(c, s), "compose launch");
   }
+  if (s_sub > 1 && Nsub > 1) {  // the state entering every later sub-chunk of each chunk
+    StageScope _sc(HLA_STAGE_CHAIN, s, 1);
+    HLA_CUDA(hla::launch_chain_advance(ch, s), "sub-chunk advance launch");
+  }
   hla::ReadoutArgs r{};
   r.B = cfg->B;
   r.H = cfg->H;
   r.T = cfg->T;
-  r.C = cfg->C;
-  r.N = N;
+  r.C = kSub;
+  r.N = Nsub;
   r.d = cfg->dk;
   r.dtype = cfg->dtype;
   r.q = q;
@@ -805,6 +859,8 @@ hla_status hla_device_status(int32_t clear, uint32_t* code_out) {
   HLA_CUDA(hla::read_error_word_readout_tc(&w, clear != 0), "hla_device_status read");
   word |= w;
   HLA_CUDA(hla::read_error_word_wait_check(&w, clear != 0), "hla_device_status read");
+  word |= w;
+  HLA_CUDA(hla::read_error_word_chain_tc(&w, clear != 0), "hla_device_status read");
   word |= w;
   if (code_out) *code_out = word;
   if (word & (hla::kErrMbarTimeout | hla::kErrTmemAlloc))

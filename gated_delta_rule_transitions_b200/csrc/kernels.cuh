@@ -75,9 +75,34 @@ struct ComposeArgs {
   const int32_t* act_idx; // [B,H,N,N]
   const float* act_g;
   const int32_t* act_cnt; // [B,H,N]
-  float* S_in;            // [B,H,N,d,d] fp32
+  float* S_in;            // [B,H,n_slots,d,d]: S_in(i) goes to slot i * slot_mult
+  int slot_mult;          // 64-token sub-chunks per chunk (1 at C = 64)
+  int n_slots;            // sub-chunks per (b,h)
   bool sparse;            // chunks may be skipped (threshold > 0)
   int32_t* order;         // [B,H,N] scratch for the pairing order (tensor-core path), or null
+};
+
+// Chunks of C = 64 s tokens (s > 1) are handled as s sub-chunks of 64 tokens.  The
+// affine chains below connect the two levels (all matrices d x d, row-major):
+//   merge    A_i = A_{is} A_{is+1} ... A_{is+s-1}
+//            B_i = (...((B_{is} A_{is+1} + B_{is+1}) A_{is+2} + B_{is+2}) ...)
+//            over the sub-chunk transitions of every complete chunk i;
+//   advance  S_(i,k) = S_(i,k-1) A_{is+k-1} + B_{is+k-1}, S_(i,0) = S_in(i), the state
+//            entering sub-chunk is+k, for every sub-chunk after the first of chunk i.
+struct ChainArgs {
+  int B, H, d, dtype;
+  int s;                 // sub-chunks per chunk (2 or 4)
+  const void* Asub;      // [B,H,sub_stride,d,d] (dtype): sub-chunk transitions
+  const void* Bsub;
+  long sub_stride;
+  // merge
+  int Nc;                // complete chunks per (b,h)
+  void* Aout;            // [B,H,out_stride,d,d] (dtype)
+  void* Bout;
+  long out_stride;
+  // advance
+  int N, Nsub;           // chunks and sub-chunks per (b,h)
+  void* S;               // [B,H,Nsub,d,d]: float32 (CUDA-core path) or bf16 (tensor-core path)
 };
 
 struct ReadoutArgs {
@@ -148,6 +173,12 @@ cudaError_t read_error_word_transitions_tc(unsigned int* out, bool clear);
 cudaError_t read_error_word_readout_tc(unsigned int* out, bool clear);
 cudaError_t read_error_word_decode_stream(unsigned int* out, bool clear);
 cudaError_t read_error_word_wait_check(unsigned int* out, bool clear);
+cudaError_t read_error_word_chain_tc(unsigned int* out, bool clear);
+cudaError_t launch_chain_merge(const ChainArgs& a, cudaStream_t s);
+cudaError_t launch_chain_advance(const ChainArgs& a, cudaStream_t s);
+// Transitions of chunks of a.C > 64 tokens by the token rule itself (CUDA cores);
+// same close_m / close_n semantics as launch_transitions.  Writes A/B only.
+cudaError_t launch_transitions_token(const TransArgs& a, cudaStream_t s);
 cudaError_t launch_wait_check(uint64_t limit_ns, bool complete, cudaStream_t s);
 
 }  // namespace hla

@@ -80,9 +80,8 @@ __device__ __forceinline__ float2 gate2_from_dot(float2 dot, float c_d, float bi
 
 // s += exp(fma(x_t, inv_tau, -m)) over the staged bf16 pairs, ascending t.
 template <bool kInRange>
-__device__ __forceinline__ float2 pool_sum_bf16(const uint32_t (&w)[64], int n, float inv_tau, float m0, float m1,
-                                                const route::Consts& K) {
-  float2 s = make_float2(0.0f, 0.0f);
+__device__ __forceinline__ float2 pool_sum_bf16(float2 s, const uint32_t (&w)[64], int n, float inv_tau, float m0,
+                                                float m1, const route::Consts& K) {
 #pragma unroll
   for (int t = 0; t < 64; ++t)
     if (t < n) {
@@ -94,7 +93,8 @@ __device__ __forceinline__ float2 pool_sum_bf16(const uint32_t (&w)[64], int n, 
 }
 }  // namespace
 
-constexpr int kPoolMaxC = 64;  // pool_sum_bf16 stages 64 tokens
+constexpr int kPoolSeg = 64;    // pool_sum_bf16 stages 64 tokens at a time
+constexpr int kPoolMaxC = 256;  // longer chunks are pooled segment by segment
 
 template <typename Tin>
 __global__ void __launch_bounds__(64) pool_kernel(const Tin* __restrict__ x0, const Tin* __restrict__ x1,
@@ -122,24 +122,47 @@ __global__ void __launch_bounds__(64) pool_kernel(const Tin* __restrict__ x0, co
     // H*d and ch0 are even, so each bf16 pair is one aligned 32-bit word
     const uint32_t* colw = reinterpret_cast<const uint32_t*>(col);
     const size_t stride = (size_t)HD / 2;
-    uint32_t w[kPoolMaxC];
+    uint32_t w[kPoolSeg];
 #pragma unroll
-    for (int t = 0; t < kPoolMaxC; ++t) w[t] = t < n ? __ldg(colw + t * stride) : 0u;
+    for (int t = 0; t < kPoolSeg; ++t) w[t] = t < n ? __ldg(colw + t * stride) : 0u;
     uint32_t hi = w[0], lo = w[0];
 #pragma unroll
-    for (int t = 1; t < kPoolMaxC; ++t)
+    for (int t = 1; t < kPoolSeg; ++t)
       if (t < n) {
         hi = bf16x2_max(hi, w[t]);
         lo = bf16x2_min(lo, w[t]);
       }
+    // chunks longer than one segment: the extremes over the remaining segments
+    for (int seg = kPoolSeg; seg < n; seg += kPoolSeg) {
+      const int ns = min(kPoolSeg, n - seg);
+#pragma unroll
+      for (int t = 0; t < kPoolSeg; ++t)
+        if (t < ns) {
+          const uint32_t x = __ldg(colw + (size_t)(seg + t) * stride);
+          hi = bf16x2_max(hi, x);
+          lo = bf16x2_min(lo, x);
+        }
+    }
     m0 = __fmul_rn(__uint_as_float(hi << 16), inv_tau);
     m1 = __fmul_rn(__uint_as_float(hi & 0xFFFF0000u), inv_tau);
     // fma is monotone in x (1/tau > 0), so the smallest shifted value comes from the
     // smallest input; when it is >= -86 no exp of the chunk needs the range checks
     const bool in_range = __fmaf_rn(__uint_as_float(lo << 16), inv_tau, -m0) >= -86.0f &&
                           __fmaf_rn(__uint_as_float(lo & 0xFFFF0000u), inv_tau, -m1) >= -86.0f;
-    const float2 ss = in_range ? pool_sum_bf16<true>(w, n, inv_tau, m0, m1, K)
-                               : pool_sum_bf16<false>(w, n, inv_tau, m0, m1, K);
+    float2 ss = make_float2(0.0f, 0.0f);
+    if (n <= kPoolSeg) {
+      ss = in_range ? pool_sum_bf16<true>(ss, w, n, inv_tau, m0, m1, K)
+                    : pool_sum_bf16<false>(ss, w, n, inv_tau, m0, m1, K);
+    } else {
+      // segment by segment, still in ascending t
+      for (int seg = 0; seg < n; seg += kPoolSeg) {
+        const int ns = min(kPoolSeg, n - seg);
+#pragma unroll
+        for (int t = 0; t < kPoolSeg; ++t) w[t] = t < ns ? __ldg(colw + (size_t)(seg + t) * stride) : 0u;
+        ss = in_range ? pool_sum_bf16<true>(ss, w, ns, inv_tau, m0, m1, K)
+                      : pool_sum_bf16<false>(ss, w, ns, inv_tau, m0, m1, K);
+      }
+    }
     s0 = ss.x;
     s1 = ss.y;
   } else {

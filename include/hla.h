@@ -23,9 +23,9 @@
  *   pools        r_c = tau * log(mean_t exp(x_t / tau)) per channel over chunk c's
  *                route tokens (route inputs default to q for r^q and k for r^k)
  *   gates        g_ij = sigmoid(<r^q_i, r^k_j> / sqrt(d) + bias), j < i, computed by
- *                a fixed binary32 recipe (no fused multiply-add, exp/log evaluated by
- *                a fixed polynomial scheme) so that gates and skip decisions are
- *                reproducible bit for bit
+ *                a fixed binary32 recipe (a fused multiply-add wherever a product
+ *                feeds a sum, exp/log evaluated by a fixed polynomial scheme) so
+ *                that gates and skip decisions are reproducible bit for bit
  *   skip         j is skipped for query chunk i iff skip_threshold > 0 and
  *                g_ij < skip_threshold (equality is kept)
  *   composition  S <- 0; for active j ascending: S <- S + g_ij ((S A_j + B_j) - S)
@@ -49,8 +49,14 @@
  *   - Calls are asynchronous on the given stream.  Argument checks run on the host
  *     before any launch; on error nothing is launched and hla_last_error() returns a
  *     message (thread-local).
- *   - Supported: C = 64; d_k = d_v in {64, 128}; dtype float32 or bf16; any T >= 1
- *     in prefill (a final partial chunk is read out and, with a cache, buffered).
+ *   - Supported: C in {64, 128, 256}; d_k = d_v in {64, 128}; dtype float32 or
+ *     bf16; any T >= 1 in prefill (a final partial chunk is read out and, with a
+ *     cache, buffered).  The pages' default chunk is 256 tokens ("Main Findings",
+ *     chunk-size ablation).  The WY solve and the intra-chunk read-out always work on
+ *     64-token sub-chunks; at C > 64 the sub-chunk transitions are merged into the
+ *     chunk's A_c, B_c (affine maps compose) and the composed state is carried to
+ *     each sub-chunk, so pools, gates, skipping, composition and the decode cache are
+ *     per chunk of C tokens.
  */
 #ifndef HLA_H_
 #define HLA_H_
@@ -89,14 +95,15 @@ typedef enum {
   HLA_CACHE_FACTORED = 1  /* the WY factors K_j, Wb_j, Ub_j (C x d each) and D_j, gamma_C:
                              A_j = gamma_C I - Wb_j^T D_j K_j, B_j = Ub_j^T D_j K_j
                              (3 C d elements; 25 % fewer bytes at C = 64, d = 128).
-                             bf16 with d = 128 only. */
+                             bf16 with d = 128 and C = 64 only (above C = 2d/3 the
+                             factors are larger than A_j, B_j). */
 } hla_cache_format;
 
 typedef struct hla_config {
   int32_t B;              /* sequences                                          */
   int32_t H;              /* heads                                              */
   int32_t T;              /* tokens per sequence (prefill, transitions)         */
-  int32_t C;              /* chunk size (64)                                    */
+  int32_t C;              /* chunk size (64, 128 or 256)                        */
   int32_t dk, dv;         /* head dims, equal, 64 or 128                        */
   int32_t dtype;          /* hla_dtype                                          */
   int32_t gate_mode;      /* hla_gate_mode                                      */
@@ -179,6 +186,10 @@ size_t hla_decode_workspace_bytes(const hla_config* cfg, int32_t max_chunks);
  * In:  k, v [B,T,H,d] dtype; alpha, beta [B,T,H] float32 (device).
  * Out: A_out [B,H,T/C,d,d], B_out [B,H,T/C,d,d] dtype (device); a final partial
  *      chunk has no output.  Errors: INVALID_ARG, UNSUPPORTED, CUDA.
+ * C = 64: the WY form above (tensor cores for bf16 with d = 128).  C > 64: this
+ * call has no workspace for sub-chunk factors, so each chunk runs the token rule
+ * row by row on CUDA cores (float32, exact in real arithmetic like the WY form);
+ * hla_prefill builds the same transitions from 64-token WY sub-chunks instead.
  */
 hla_status gdn_chunk_transitions(const hla_config* cfg, const void* k, const void* v,
                                  const float* alpha, const float* beta, void* A_out,
@@ -227,7 +238,8 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
  *      chunk's key pool; active chunks are applied by the equivalent right-to-left
  *      form  y += g_j B_j x; x <- (1-g_j) x + g_j A_j x  (j descending), which reads
  *      each active A_j/B_j once; when the open chunk reaches C tokens it is closed
- *      (its A/B/rk are appended).  Gate modes ROUTED, ONE and ZERO.
+ *      (its A/B/rk are appended; at C = 64 by the WY form, at C > 64 by the token
+ *      rule run row by row).  Gate modes ROUTED, ONE and ZERO.
  * workspace: device, >= hla_decode_workspace_bytes(cfg, cache->max_chunks).
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE (also: cache full), CUDA.
  */
@@ -296,7 +308,9 @@ typedef enum {
   HLA_STAGE_CACHE = 5,        /* prefill -> decode cache hand-off          */
   HLA_STAGE_DECODE = 6,       /* decode: sweep, gates, active chain        */
   HLA_STAGE_DECODE_CLOSE = 7, /* decode: closing full chunks, counters     */
-  HLA_STAGE_COUNT = 8
+  HLA_STAGE_CHAIN = 8,        /* C > 64: sub-chunk transitions merged per
+                                 chunk, states advanced to sub-chunks      */
+  HLA_STAGE_COUNT = 9
 } hla_stage;
 
 hla_status hla_profile_enable(int32_t on);

@@ -84,7 +84,8 @@ def test_prefill_workspace_grows_with_T(hla):
 
 
 @pytest.mark.parametrize("kw,status", [
-    (dict(C=32), 2), (dict(d=96), 2), (dict(T=0), 1), (dict(B=0), 1), (dict(tau=0.0), 1),
+    (dict(C=32), 2), (dict(C=96), 2), (dict(C=512), 2), (dict(d=96), 2), (dict(T=0), 1), (dict(B=0), 1),
+    (dict(tau=0.0), 1),
 ])
 def test_bad_config_rejected_on_host(hla, kw, status):
     c = cfg(hla, **kw)
@@ -219,3 +220,29 @@ def test_factored_cache_needs_bf16_d128(hla):
     out = hla.HlaCache()
     st = hla.lib().hla_cache_init(ctypes.byref(c), 4, ctypes.c_void_p(1 << 20), 1 << 30, ctypes.byref(out), None)
     assert st == hla.HLA_ERR_UNSUPPORTED and "factored" in hla.last_error()
+
+
+@pytest.mark.parametrize("C", [128, 256])
+def test_long_chunks_accepted(hla, C):
+    """Chunks of 128 and 256 tokens (the pages' default is 256): the prefill workspace
+    holds the gates of N = T / C chunks and the transitions of the T / 64 sub-chunks."""
+    T = 4096
+    c = cfg(hla, T=T, C=C)
+    ws = hla.prefill_workspace_bytes(c)
+    assert ws > 0
+    N, d = T // C, 128
+    # at least: A/B of the chunks and of the sub-chunks (bf16), the state entering
+    # every sub-chunk and the gate rows of the chunks
+    assert ws >= (N + T // 64) * 2 * d * d * 2 + (T // 64) * d * d * 4 + 2 * N * N * 4
+    assert hla.cache_bytes(c, 8) > 0
+    # the decode cache holds C-token buffers of the open chunk
+    c64 = cfg(hla, T=1, C=64)
+    cC = cfg(hla, T=1, C=C)
+    assert hla.cache_bytes(cC, 8) - hla.cache_bytes(c64, 8) >= 4 * (C - 64) * d * 2
+
+
+def test_factored_cache_needs_c64(hla):
+    c = cfg(hla, B=1, H=1, T=1, C=128, cache_format="factored")
+    out = hla.HlaCache()
+    st = hla.lib().hla_cache_init(ctypes.byref(c), 4, ctypes.c_void_p(1 << 20), 1 << 30, ctypes.byref(out), None)
+    assert st == hla.HLA_ERR_UNSUPPORTED and "C = 64" in hla.last_error()

@@ -54,6 +54,21 @@ def test_composition_law_two_chunks():
     assert np.abs(B - (B1 @ A2 + B2)).max() <= 1e-13
 
 
+def test_long_chunk_is_product_of_its_64_token_pieces():
+    # a chunk of 256 tokens acts as its four 64-token pieces applied in order:
+    # A = A1 A2 A3 A4 and B = ((B1 A2 + B2) A3 + B3) A4 + B4 (affine maps compose)
+    rng = np.random.default_rng(21)
+    _, k, v, a, b = _head(rng, 256, 10)
+    A, B = ho.chunk_transition(k, v, a, b)
+    Ap, Bp = np.eye(10), np.zeros((10, 10))
+    for p in range(4):
+        sl = slice(64 * p, 64 * p + 64)
+        Ai, Bi = ho.chunk_transition(k[sl], v[sl], a[sl], b[sl])
+        Ap, Bp = Ap @ Ai, Bp @ Ai + Bi
+    assert np.abs(A - Ap).max() <= 1e-13
+    assert np.abs(B - Bp).max() <= 1e-12
+
+
 def test_transition_contraction():
     # eigenvalues of I - beta k k^T lie in [1 - beta, 1] for unit k, so ||A_c||_2 <= gamma_C
     rng = np.random.default_rng(12)
@@ -92,11 +107,11 @@ def test_single_chunk_equals_gdn():
     assert np.abs(r.o - o).max() <= 1e-13
 
 
-@pytest.mark.parametrize("T", [64, 70])
-def test_gates_one_is_native_gdn(T):
+@pytest.mark.parametrize("T,C", [(64, 8), (70, 8), (600, 256), (300, 128)])
+def test_gates_one_is_native_gdn(T, C):
     rng = np.random.default_rng(16 + T)
     q, k, v, a, b = _head(rng, T, 12)
-    r = ho.hla_prefill_head(q, k, v, a, b, 8, gate_mode=ho.GATES_ONE)
+    r = ho.hla_prefill_head(q, k, v, a, b, C, gate_mode=ho.GATES_ONE)
     o, _ = ho.gdn_recurrent(q, k, v, a, b)
     assert np.abs(r.o - o).max() <= 1e-12
 
