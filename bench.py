@@ -336,6 +336,27 @@ def run_ours(args):
     torch.cuda.synchronize()
     active_pairs = int(acnt.sum().item())
 
+    # routing diagnostics (mass and effective support per query chunk) on the same
+    # gates, timed alone: it reads the lower triangle of the N x N gate rows
+    gates_full = torch.empty((wp.B, wp.H, N, N), dtype=torch.float32, device="cuda")
+    hla.hla_prefill(pcfg, dev["q"], dev["k"], dev["v"], dev["alpha"], dev["beta"], o,
+                    q_route=dev.get("q_route"), k_route=dev.get("k_route"), workspace=pws, gates_out=gates_full)
+    mass = torch.empty((wp.B, wp.H, N), dtype=torch.float32, device="cuda")
+    support = torch.empty_like(mass)
+    for _ in range(3):
+        hla.hla_gate_support(pcfg, gates_full, mass, support)
+    l2_flush()
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ev_s[0].record(stream)
+    for _ in range(20):
+        hla.hla_gate_support(pcfg, gates_full, mass, support)
+    ev_s[1].record(stream)
+    torch.cuda.synchronize()
+    support_us = ev_s[0].elapsed_time(ev_s[1]) / 20 * 1e3
+    diagnostics = {"gate_support_us": support_us, "gate_rows": wp.B * wp.H * N,
+                   "support_median": float(support.median().item()), "mass_median": float(mass.median().item())}
+    del gates_full
+
     hla.hla_profile_read(reset=True)
     hla.hla_profile_enable(True)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(4 * args.steps)]
@@ -462,6 +483,7 @@ def run_ours(args):
         "stages_ms_per_step": {k: v[0] / args.steps for k, v in stages.items() if v[1]},
         "e2e": {"value": whole_job_rate(tokens_pre, e2e_pre, world), "unit": "tokens/s", "h2d_bytes_per_step": h2d_pre,
                 "d2h_bytes_per_step": d2h_pre},
+        "diagnostics": diagnostics,
         "gpu_launches": launches,
         "clocks": clocks.summary(),
     }

@@ -69,6 +69,7 @@ _SIGS = {
     "hla_decode_workspace_bytes": ([ctypes.POINTER(HlaConfig), ctypes.c_int32], ctypes.c_size_t),
     "gdn_chunk_transitions": ([ctypes.POINTER(HlaConfig), _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
     "hla_routing": ([ctypes.POINTER(HlaConfig), _P, _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
+    "hla_gate_support": ([ctypes.POINTER(HlaConfig), _P, _P, _P, _P], ctypes.c_int),
     "hla_prefill": ([ctypes.POINTER(HlaConfig), _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                      ctypes.POINTER(HlaCache), _P, ctypes.c_size_t, _P], ctypes.c_int),
     "hla_decode_step": ([ctypes.POINTER(HlaConfig), ctypes.POINTER(HlaCache), _P, _P, _P, _P, _P, _P, _P, _P, _P,
@@ -200,6 +201,12 @@ def hla_routing(cfg, q_route, k_route, rq_out, rk_out, gates_out=None, active_id
                 active_cnt_out=None, stream=None):
     _check(lib().hla_routing(ctypes.byref(cfg), _ptr(q_route), _ptr(k_route), _ptr(rq_out), _ptr(rk_out),
                              _ptr(gates_out), _ptr(active_idx_out), _ptr(active_cnt_out), _stream(stream)))
+
+
+def hla_gate_support(cfg, gates, mass_out=None, support_out=None, stream=None):
+    """Routing mass and effective support per query chunk from a gate matrix."""
+    _check(lib().hla_gate_support(ctypes.byref(cfg), _ptr(gates), _ptr(mass_out), _ptr(support_out),
+                                  _stream(stream)))
 
 
 def hla_prefill(cfg, q, k, v, alpha, beta, o, q_route=None, k_route=None, user_gates=None, gates_out=None,

@@ -461,6 +461,23 @@ hla_status hla_routing(const hla_config* cfg, const void* q_route, const void* k
   return HLA_OK;
 }
 
+hla_status hla_gate_support(const hla_config* cfg, const float* gates, float* mass_out, float* support_out,
+                            hla_stream_t stream) {
+  g_msg[0] = 0;
+  HLA_TRY(check_cfg(cfg, true));
+  HLA_TRY(need_ptr(gates, "gates"));
+  HLA_TRY(opt_ptr(mass_out, "mass_out"));
+  HLA_TRY(opt_ptr(support_out, "support_out"));
+  if (mass_out == nullptr && support_out == nullptr)
+    return fail(HLA_ERR_INVALID_ARG, "mass_out and support_out are both NULL");
+  const int N = (cfg->T + cfg->C - 1) / cfg->C;
+  if ((double)cfg->B * cfg->H * N >= 2147483647.0) return fail(HLA_ERR_UNSUPPORTED, "too many gate rows");
+  HLA_CUDA(hla::launch_gate_support(gates, cfg->B, cfg->H, N, cfg->skip_threshold, mass_out, support_out,
+                                    (cudaStream_t)stream),
+           "gate support launch");
+  return HLA_OK;
+}
+
 hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, const void* v, const float* alpha,
                        const float* beta, const void* q_route, const void* k_route, const float* user_gates,
                        void* o, float* gates_out, int32_t* active_idx_out, int32_t* active_cnt_out,

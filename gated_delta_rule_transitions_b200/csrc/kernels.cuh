@@ -179,6 +179,8 @@ cudaError_t launch_chain_advance(const ChainArgs& a, cudaStream_t s);
 // Transitions of chunks of a.C > 64 tokens by the token rule itself (CUDA cores);
 // same close_m / close_n semantics as launch_transitions.  Writes A/B only.
 cudaError_t launch_transitions_token(const TransArgs& a, cudaStream_t s);
+cudaError_t launch_gate_support(const float* gates, int B, int H, int N, float thr, float* mass_out,
+                                float* support_out, cudaStream_t s);
 cudaError_t launch_wait_check(uint64_t limit_ns, bool complete, cudaStream_t s);
 
 }  // namespace hla

@@ -210,6 +210,22 @@ hla_status hla_routing(const hla_config* cfg, const void* q_route, const void* k
                        int32_t* active_idx_out, int32_t* active_cnt_out, hla_stream_t stream);
 
 /*
+ * hla_gate_support -- routing diagnostics ("Key Contributions" 3; "Methodology in
+ * Plain English" para. 4: a budget on the total routing mass and an order-2
+ * effective number, the inverse sum of squares, of the chunks a query accesses).
+ * For every query chunk i, over the chunks j < i kept by cfg->skip_threshold (all
+ * of them for a threshold <= 0):
+ *   mass_i = sum_j g_ij,   support_i = mass_i^2 / sum_j g_ij^2   (0 if none kept).
+ * In:  gates [B,H,N,N] float32 (device), N = ceil(T/C): a gate matrix as written by
+ *      hla_routing or hla_prefill (gates_out); only entries j < i are read.
+ * Out: mass_out, support_out [B,H,N] float32 (device); either may be NULL, not both.
+ * float32 sums (per-lane partial sums combined by a butterfly).
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA.
+ */
+hla_status hla_gate_support(const hla_config* cfg, const float* gates, float* mass_out, float* support_out,
+                            hla_stream_t stream);
+
+/*
  * hla_prefill -- HLA over a whole prompt (Key Contributions 3; Methodology paras. 1-4).
  * In:  q, k, v [B,T,H,d] dtype; alpha, beta [B,T,H] float32;
  *      q_route, k_route [B,T,H,d] dtype or NULL (NULL: q, k);

@@ -177,6 +177,28 @@ def active_lists(G, thr: float):
     return out
 
 
+def gate_support(G, thr: float):
+    """Routing mass and effective support per query chunk ("Key Contributions" 3 and
+    "Methodology in Plain English" para. 4: an order-2 effective number, the inverse
+    sum of squares, of the chunks a query accesses).
+
+    Over the chunks j < i that are kept (every one for thr <= 0, else G[i, j] >= thr):
+    mass_i = sum_j g_ij and support_i = mass_i^2 / sum_j g_ij^2 (0 with nothing
+    kept).  float64 sums of the binary32 gates.  Returns (mass [N], support [N])."""
+    G = np.asarray(G, np.float32)
+    N = G.shape[0]
+    mass = np.zeros(N)
+    support = np.zeros(N)
+    for i in range(N):
+        g = G[i, :i].astype(np.float64)
+        if thr > 0:
+            g = g[G[i, :i] >= np.float32(thr)]
+        m, q = g.sum(), (g * g).sum()
+        mass[i] = m
+        support[i] = m * m / q if q > 0 else 0.0
+    return mass, support
+
+
 # ----------------------------------------------------------------------------------
 # Prefill
 # ----------------------------------------------------------------------------------

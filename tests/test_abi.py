@@ -246,3 +246,12 @@ def test_factored_cache_needs_c64(hla):
     out = hla.HlaCache()
     st = hla.lib().hla_cache_init(ctypes.byref(c), 4, ctypes.c_void_p(1 << 20), 1 << 30, ctypes.byref(out), None)
     assert st == hla.HLA_ERR_UNSUPPORTED and "C = 64" in hla.last_error()
+
+
+def test_gate_support_needs_an_output(hla):
+    c = cfg(hla, T=256)
+    P = ctypes.c_void_p(0x100000)
+    st = hla.lib().hla_gate_support(ctypes.byref(c), P, None, None, None)
+    assert st == hla.HLA_ERR_INVALID_ARG and "both NULL" in hla.last_error()
+    st = hla.lib().hla_gate_support(ctypes.byref(c), None, P, P, None)
+    assert st == hla.HLA_ERR_INVALID_ARG and "gates is NULL" in hla.last_error()

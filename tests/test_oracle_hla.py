@@ -278,3 +278,43 @@ def test_decode_partial_chunk_sweep_closed_form():
         x = a[t] * (x - b[t] * k[t] * (k[t] @ x))
     assert np.abs(x - Ap @ qv).max() <= 1e-14
     assert np.abs(y0 - Bp @ qv).max() <= 1e-14
+
+
+# ---- effective support of the routing (order-2 effective number) ------------------
+
+def test_support_of_equal_gates_is_their_count():
+    # n kept gates of equal value g: (n g)^2 / (n g^2) = n, mass n g
+    G = np.zeros((6, 6), np.float32)
+    for i in range(6):
+        G[i, :i] = 0.375
+    mass, sup = ho.gate_support(G, 0.0)
+    assert sup.tolist() == [0.0, 1.0, 2.0, 3.0, 4.0, 5.0]
+    assert mass.tolist() == [0.375 * i for i in range(6)]
+
+
+def test_support_counts_only_kept_chunks_and_is_scale_free():
+    G = np.zeros((4, 4), np.float32)
+    G[3, :3] = [0.9, 0.02, 0.9]          # the middle chunk is below the threshold
+    G[2, :2] = [0.5, 0.0]
+    mass, sup = ho.gate_support(G, 0.05)
+    assert sup[3] == 2.0 and mass[3] == pytest.approx(1.8, abs=1e-7)
+    assert sup[2] == 1.0                  # one kept chunk
+    assert sup[1] == 0.0 and mass[1] == 0.0   # g = 0 < 0.05: nothing kept
+    _, sup_all = ho.gate_support(G, 0.0)
+    # without a threshold the small gate counts a little: 1.82^2 / (2 * 0.81 + 0.0004)
+    assert sup_all[3] == pytest.approx(1.82 ** 2 / (2 * 0.9 ** 2 + 0.02 ** 2), rel=1e-6)
+    _, sup_half = ho.gate_support(G * np.float32(0.5), 0.0)
+    assert np.allclose(sup_half, sup_all, rtol=1e-12)
+
+
+def test_support_lies_between_one_and_the_kept_count():
+    # Cauchy-Schwarz: (sum g)^2 <= n sum g^2, with equality for equal gates
+    rng = np.random.default_rng(31)
+    G = rng.uniform(0.0, 1.0, (40, 40)).astype(np.float32)
+    mass, sup = ho.gate_support(G, 0.3)
+    for i in range(40):
+        n = int((G[i, :i] >= np.float32(0.3)).sum())
+        if n == 0:
+            assert sup[i] == 0.0
+        else:
+            assert 1.0 - 1e-12 <= sup[i] <= n + 1e-12
