@@ -220,10 +220,11 @@ def build_decode_cache(hla, syn, torch, w, max_chunks, group=8, cache_format="de
     """Fill a decode cache for w.B sequences of w.T-token contexts through the public
     API: hla_prefill with every earlier-chunk weight 0 writes the cache (A/B/key pools
     do not depend on gates) without the quadratic composition."""
-    cfg = hla.make_config(w.B, w.H, w.T, w.C, w.d, w.dtype, "routed", w.tau, w.bias, w.thr, cache_format=cache_format)
+    cfg = hla.make_config(w.B, w.H, w.T, w.C, w.d, w.dtype, "routed", w.tau, w.bias, w.thr, cache_format=cache_format,
+                          pool_window=w.window)
     cache = hla.Cache(cfg, max_chunks)
     gcfg = hla.make_config(group, w.H, w.T, w.C, w.d, w.dtype, "zero", w.tau, w.bias, w.thr,
-                           cache_format=cache_format)
+                           cache_format=cache_format, pool_window=w.window)
     ws = torch.empty(hla.prefill_workspace_bytes(gcfg), dtype=torch.uint8, device="cuda")
     first_ctx = None
     for b0 in range(0, w.B, group):
@@ -262,6 +263,8 @@ def run_ours(args):
         wp = wp.with_(T=args.prefill_T, name=f"{wp.name}_T{args.prefill_T}")
     if args.chunk != wp.C:
         wp = wp.with_(C=args.chunk, name=wp.name.replace("_C64_", f"_C{args.chunk}_"))
+    if args.pool_window:
+        wp = wp.with_(window=args.pool_window, name=f"{wp.name}_window{args.pool_window}")
     # the long sparse workload is generated on the device (5 x 1 GiB of inputs)
     gen_dev = "cuda" if wp.B * wp.T * wp.H * wp.d > (1 << 28) else "cpu"
     inp = syn.make_gdn_inputs(wp, device=gen_dev)
@@ -272,7 +275,8 @@ def run_ours(args):
     dev = {k: v.cuda() for k, v in host.items()}
     del inp
     inp = host
-    pcfg = hla.make_config(wp.B, wp.H, wp.T, wp.C, wp.d, wp.dtype, wp.gate_mode, wp.tau, wp.bias, wp.thr)
+    pcfg = hla.make_config(wp.B, wp.H, wp.T, wp.C, wp.d, wp.dtype, wp.gate_mode, wp.tau, wp.bias, wp.thr,
+                           pool_window=wp.window)
     pws = torch.empty(hla.prefill_workspace_bytes(pcfg), dtype=torch.uint8, device="cuda")
     o = torch.empty_like(dev["q"])
     o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
@@ -295,12 +299,14 @@ def run_ours(args):
         wd = wd.with_(name=f"{wd.name}_{args.decode_cache}_cache")
     if args.chunk != wd.C:
         wd = wd.with_(C=args.chunk, name=wd.name.replace("_C64_", f"_C{args.chunk}_"))
+    if args.pool_window:
+        wd = wd.with_(window=args.pool_window, name=f"{wd.name}_window{args.pool_window}")
     max_chunks = wd.T // wd.C + 1
     cache, ctx0 = build_decode_cache(hla, syn, torch, wd, max_chunks, group=min(8, wd.B),
                                      cache_format=args.decode_cache)
     torch.cuda.empty_cache()
     dcfg = hla.make_config(wd.B, wd.H, 1, wd.C, wd.d, wd.dtype, wd.gate_mode, wd.tau, wd.bias, wd.thr,
-                           cache_format=args.decode_cache)
+                           cache_format=args.decode_cache, pool_window=wd.window)
     dws = torch.empty(hla.decode_workspace_bytes(dcfg, max_chunks), dtype=torch.uint8, device="cuda")
     ntok = args.warmup + args.steps + 1
     toks_host = [{k: v.contiguous().pin_memory() for k, v in t.items()} for t in syn.make_decode_tokens(wd, ntok)]
@@ -440,7 +446,8 @@ def run_ours(args):
         per_chunk = 3 * wd.C * wd.d * 2 + (wd.C + 4) * 4   # K, Wb, Ub bf16 + scales
     else:
         per_chunk = 2 * wd.d * wd.d * 2                      # A, B bf16
-    bytes_decode = wd.B * wd.H * (n_ctx * (per_chunk + wd.d * 4))
+    key_reps = wd.C // wd.window if wd.window else 1
+    bytes_decode = wd.B * wd.H * (n_ctx * (per_chunk + key_reps * wd.d * 4))
     dmain_ms, dmain_n = stages["decode"]
     dmain_avg = dmain_ms / max(dmain_n, 1)
     dec_gbs = bytes_decode / (dmain_avg * 1e-3) / 1e9 if dmain_avg > 0 else None
@@ -512,9 +519,9 @@ def _oracle_prefill_worker(job):
     """One (sequence, head) of the oracle prefill; returns its wall time (s)."""
     _limit_blas_threads()
     from oracle import hla_oracle as ho
-    arrays, params = job
+    arrays, params, window = job
     t0 = time.perf_counter()
-    ho.hla_prefill_head(*arrays[:5], *params, arrays[5], arrays[6])
+    ho.hla_prefill_head(*arrays[:5], *params, arrays[5], arrays[6], pool_window=window)
     return time.perf_counter() - t0
 
 
@@ -522,8 +529,8 @@ def _oracle_decode_worker(job):
     """Oracle decode head built from one context (untimed), then one timed step."""
     _limit_blas_threads()
     from oracle import hla_oracle as ho
-    ctx, params, tok = job
-    head = ho.HlaDecodeHead.from_prefill(*ctx, *params)
+    ctx, params, tok, window = job
+    head = ho.HlaDecodeHead.from_prefill(*ctx, *params, pool_window=window)
     t0 = time.perf_counter()
     head.step(*tok)
     return time.perf_counter() - t0
@@ -553,7 +560,7 @@ def _prefill_jobs(inp, wp, pairs):
     params = (wp.C, wp.tau, wp.bias, wp.thr, wp.gate_mode)
     return [((f("q", b, h, np.float64), f("k", b, h, np.float64), f("v", b, h, np.float64),
               f("alpha", b, h, np.float64), f("beta", b, h, np.float64),
-              f("q_route", b, h, np.float32), f("k_route", b, h, np.float32)), params) for (b, h) in pairs]
+              f("q_route", b, h, np.float32), f("k_route", b, h, np.float32)), params, wp.window) for (b, h) in pairs]
 
 
 def _decode_jobs(ctx, wd, tok, pairs):
@@ -563,7 +570,7 @@ def _decode_jobs(ctx, wd, tok, pairs):
         c = tuple(ctx[n][b, :, h].float().cpu().numpy().astype(np.float64) for n in ("q", "k", "v", "alpha", "beta"))
         t = (tok["q"][b, h].double().numpy(), tok["k"][b, h].double().numpy(), tok["v"][b, h].double().numpy(),
              float(tok["alpha"][b, h]), float(tok["beta"][b, h]))
-        jobs.append((c, params, t))
+        jobs.append((c, params, t, wd.window))
     return jobs
 
 
@@ -669,6 +676,8 @@ def main(argv=None):
                     help="dense: A_j/B_j d x d (the metric's workload); factored: K_j, Wb_j, Ub_j per chunk")
     ap.add_argument("--chunk", type=int, choices=[64, 128, 256], default=64,
                     help="chunk size C of both workloads (the metric's workloads use 64)")
+    ap.add_argument("--pool-window", type=int, default=0,
+                    help="key window representatives of this many tokens (0: one pool per chunk)")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

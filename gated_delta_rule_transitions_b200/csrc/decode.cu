@@ -38,7 +38,7 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
 // grid B*H, block D.  Thread = channel / row.
 template <int D, typename Tio>
 __global__ void __launch_bounds__(128) decode_main_kernel(DecodeArgs a) {
-  __shared__ float rq[D];
+  __shared__ __align__(16) float rq[D];
   __shared__ float xs[2][D];
   __shared__ float red[D / 32];
   __shared__ int wcount[D / 32];
@@ -94,13 +94,19 @@ __global__ void __launch_bounds__(128) decode_main_kernel(DecodeArgs a) {
       rq[tid] = __fmul_rn(a.tau, __fadd_rn(mx, route::rlog(__fdiv_rn(s, (float)mp), K)));
       __syncthreads();
     }
-    const float* rk = a.rk + (long)bh * a.max_chunks * D;
+    const int W = a.win > 0 ? a.win : 1;
+    const float* rk = a.rk + (long)bh * a.max_chunks * W * D;
     for (int jb = 0; jb < n; jb += D) {
       const int j = jb + tid;
       float g = 1.0f;
       bool keep = false;
       if (j < n) {
-        if (a.mode == HLA_GATES_ROUTED) {
+        if (a.mode == HLA_GATES_ROUTED && a.win > 0) {
+          // log-sum-exp over the closed chunk's window representatives
+          float t[kMaxWindows];
+          const float m = route::window_scores(rq, rk + (long)j * W * D, a.win, D, a.c_d, t);
+          g = route::gate_from_window_scores(t, a.win, m, a.bias, K);
+        } else if (a.mode == HLA_GATES_ROUTED) {
           const float* rkj = rk + (long)j * D;
           float dot = 0.0f;
           for (int c = 0; c < D; ++c) dot = route::dot_step(dot, rq[c], rkj[c]);
@@ -165,15 +171,20 @@ __global__ void decode_close_pool_kernel(DecodeArgs a) {
     return;
   }
   const route::Consts K = route::make_consts();
-  const Tio* bk = (const Tio*)a.buf_kr + (long)bh * a.C * D + tid;
   const float inv_tau = __fdiv_rn(1.0f, a.tau);
-  float mx = __fmul_rn(ldf(bk), inv_tau);
-  for (int t = 1; t < a.C; ++t) mx = fmaxf(mx, __fmul_rn(ldf(bk + (long)t * D), inv_tau));
-  float s = 0.0f;
-  for (int t = 0; t < a.C; ++t)
-    s = __fadd_rn(s, route::rexp(route::pool_shift(ldf(bk + (long)t * D), inv_tau, mx), K));
-  a.rk[((long)bh * a.max_chunks + n) * D + tid] =
-      __fmul_rn(a.tau, __fadd_rn(mx, route::rlog(__fdiv_rn(s, (float)a.C), K)));
+  // one pool over the chunk, or one per window of C / W tokens
+  const int W = a.win > 0 ? a.win : 1;
+  const int len = a.C / W;
+  for (int u = 0; u < W; ++u) {
+    const Tio* bk = (const Tio*)a.buf_kr + ((long)bh * a.C + (long)u * len) * D + tid;
+    float mx = __fmul_rn(ldf(bk), inv_tau);
+    for (int t = 1; t < len; ++t) mx = fmaxf(mx, __fmul_rn(ldf(bk + (long)t * D), inv_tau));
+    float s = 0.0f;
+    for (int t = 0; t < len; ++t)
+      s = __fadd_rn(s, route::rexp(route::pool_shift(ldf(bk + (long)t * D), inv_tau, mx), K));
+    a.rk[(((long)bh * a.max_chunks + n) * W + u) * D + tid] =
+        __fmul_rn(a.tau, __fadd_rn(mx, route::rlog(__fdiv_rn(s, (float)len), K)));
+  }
 }
 
 __global__ void decode_counters_kernel(int B, int C, int max_chunks, int32_t* n_chunks, int32_t* m_partial) {
@@ -193,7 +204,8 @@ __global__ void decode_counters_kernel(int B, int C, int max_chunks, int32_t* n_
 // sets the counters.  grid B*H, block 128.
 struct FillArgs {
   int B, H, T, C, d, N, max_chunks;
-  const float* rk_ws;  // [B,H,N,d]
+  int W;               // key representatives per chunk
+  const float* rk_ws;  // [B,H,N*W,d]
   const void *qr, *kr, *k, *v;  // [B,T,H,d]
   const float *alpha, *beta;    // [B,T,H]
 };
@@ -204,8 +216,8 @@ __global__ void cache_fill_kernel(DecodeArgs c, FillArgs f) {
   const int b = bh / f.H, h = bh % f.H;
   const int nc = f.T / f.C;
   const int m = f.T - nc * f.C;
-  for (long idx = threadIdx.x; idx < (long)nc * f.d; idx += blockDim.x)
-    c.rk[(long)bh * f.max_chunks * f.d + idx] = f.rk_ws[(long)bh * f.N * f.d + idx];
+  for (long idx = threadIdx.x; idx < (long)nc * f.W * f.d; idx += blockDim.x)
+    c.rk[(long)bh * f.max_chunks * f.W * f.d + idx] = f.rk_ws[(long)bh * f.N * f.W * f.d + idx];
   const long HD = (long)f.H * f.d;
   for (long idx = threadIdx.x; idx < (long)m * f.d; idx += blockDim.x) {
     const int t = (int)(idx / f.d), ch = (int)(idx - (long)t * f.d);
@@ -335,6 +347,7 @@ cudaError_t launch_cache_fill(const DecodeArgs& c, const float* rk_ws, const voi
   f.d = c.d;
   f.N = (T + c.C - 1) / c.C;
   f.max_chunks = c.max_chunks;
+  f.W = c.win > 0 ? c.win : 1;
   f.rk_ws = rk_ws;
   f.qr = q_route;
   f.kr = k_route;

@@ -95,13 +95,19 @@ __device__ __forceinline__ int decode_prologue(const DecodeArgs& a, int bh, int 
       rq[tid] = __fmul_rn(a.tau, __fadd_rn(mx, route::rlog(__fdiv_rn(s, (float)mp), K)));
       tc::bar_sync(1, kCompute);
     }
-    const float* rk = a.rk + (long)bh * a.max_chunks * kD;
+    const int W = a.win > 0 ? a.win : 1;
+    const float* rk = a.rk + (long)bh * a.max_chunks * W * kD;
     for (int jb = 0; jb < n; jb += kCompute) {
       const int j = jb + tid;
       float g = 1.0f;
       bool keep = false;
       if (j < n) {
-        if (a.mode == HLA_GATES_ROUTED) {
+        if (a.mode == HLA_GATES_ROUTED && a.win > 0) {
+          // log-sum-exp over the closed chunk's window representatives
+          float t[kMaxWindows];
+          const float m = route::window_scores(rq, rk + (long)j * W * kD, a.win, kD, a.c_d, t);
+          g = route::gate_from_window_scores(t, a.win, m, a.bias, K);
+        } else if (a.mode == HLA_GATES_ROUTED) {
           const float4* rkj = (const float4*)(rk + (long)j * kD);
           float dot = 0.0f;
           for (int c4 = 0; c4 < kD / 4; ++c4) {

@@ -46,6 +46,12 @@ hla_status check_cfg(const hla_config* c, bool need_T) {
     return fail(HLA_ERR_INVALID_ARG, "gate_mode %d invalid", c->gate_mode);
   if (c->cache_format != HLA_CACHE_DENSE && c->cache_format != HLA_CACHE_FACTORED)
     return fail(HLA_ERR_INVALID_ARG, "cache_format %d invalid", c->cache_format);
+  if (c->pool_window != 0) {
+    const int w = c->pool_window;
+    if (w < 8 || w >= c->C || c->C % w != 0 || c->C / w > hla::kMaxWindows)
+      return fail(HLA_ERR_UNSUPPORTED, "pool_window %d unsupported for C=%d (8 <= w < C, w | C, C / w <= %d)", w,
+                  c->C, hla::kMaxWindows);
+  }
   if (!(c->tau > 0.0f) || !std::isfinite(c->tau)) return fail(HLA_ERR_INVALID_ARG, "tau must be finite and > 0");
   if (!std::isfinite(c->bias) || !std::isfinite(c->skip_threshold))
     return fail(HLA_ERR_INVALID_ARG, "bias and skip_threshold must be finite");
@@ -79,6 +85,10 @@ hla_status opt_ptr(const void* p, const char* name) {
 
 float gate_scale(int d) { return (float)(1.0 / std::sqrt((double)d)); }
 
+// Window representatives per chunk (0: one pool per chunk) and key pools per chunk.
+int n_windows(const hla_config* c) { return c->pool_window > 0 ? c->C / c->pool_window : 0; }
+size_t key_reps(const hla_config* c) { return c->pool_window > 0 ? (size_t)(c->C / c->pool_window) : 1; }
+
 // The WY solve and the intra-chunk read-out work on sub-chunks of kSub tokens; a
 // chunk of C tokens is C / kSub of them.
 constexpr int kSub = 64;
@@ -102,7 +112,7 @@ PrefillWs prefill_layout(const hla_config* c) {
     return o;
   };
   w.rq = take(B * H * N * d * 4);
-  w.rk = take(B * H * N * d * 4);
+  w.rk = take(B * H * N * key_reps(c) * d * 4);
   w.act_idx = take(B * H * N * N * 4);
   w.act_g = take(B * H * N * N * 4);
   w.act_cnt = take(B * H * N * 4);
@@ -147,7 +157,7 @@ CacheLayout cache_layout(const hla_config* c, int32_t maxc) {
     L.A = take(B * H * (size_t)maxc * d * d * es);
     L.Bm = take(B * H * (size_t)maxc * d * d * es);
   }
-  L.rk = take(B * H * (size_t)maxc * d * 4);
+  L.rk = take(B * H * (size_t)maxc * key_reps(c) * d * 4);
   L.bk = take(B * H * C * d * es);
   L.bv = take(B * H * C * d * es);
   L.bqr = take(B * H * C * d * es);
@@ -163,7 +173,7 @@ CacheLayout cache_layout(const hla_config* c, int32_t maxc) {
 hla_status check_cache(const hla_config* c, const hla_cache* k) {
   if (k == nullptr) return fail(HLA_ERR_INVALID_ARG, "cache is NULL");
   if (k->B != c->B || k->H != c->H || k->C != c->C || k->d != c->dk || k->dtype != c->dtype ||
-      k->format != c->cache_format)
+      k->format != c->cache_format || k->pool_window != c->pool_window)
     return fail(HLA_ERR_INVALID_ARG, "cache was initialised for a different config");
   if (k->max_chunks <= 0) return fail(HLA_ERR_INVALID_ARG, "cache max_chunks must be positive");
   const void* ps[] = {k->rk, k->buf_k, k->buf_v, k->buf_qr, k->buf_kr, k->buf_alpha, k->buf_beta};
@@ -282,6 +292,7 @@ hla_status hla_cache_init(const hla_config* cfg, int32_t max_chunks, void* mem, 
   c.d = cfg->dk;
   c.dtype = cfg->dtype;
   c.format = cfg->cache_format;
+  c.pool_window = cfg->pool_window;
   if (cfg->cache_format == HLA_CACHE_FACTORED) {
     c.Kf = base + L.Kf;
     c.Wf = base + L.Wf;
@@ -327,7 +338,8 @@ hla_status hla_cache_slice(const hla_cache* cache, int32_t b0, int32_t nb, hla_c
     v.A = (char*)cache->A + off * H * mc * d * d * es;
     v.Bm = (char*)cache->Bm + off * H * mc * d * d * es;
   }
-  v.rk = (float*)((char*)cache->rk + off * H * mc * d * 4);
+  const size_t reps = cache->pool_window > 0 ? (size_t)(cache->C / cache->pool_window) : 1;
+  v.rk = (float*)((char*)cache->rk + off * H * mc * reps * d * 4);
   v.buf_k = (char*)cache->buf_k + off * H * C * d * es;
   v.buf_v = (char*)cache->buf_v + off * H * C * d * es;
   v.buf_qr = (char*)cache->buf_qr + off * H * C * d * es;
@@ -385,17 +397,37 @@ hla_status gdn_chunk_transitions(const hla_config* cfg, const void* k, const voi
   return HLA_OK;
 }
 
+// Query pools per chunk and key pools per chunk, or per window with window
+// representatives (window u of chunk j at row j * W + u).
+static hla_status launch_route_pools(const hla_config* cfg, const void* q_route, const void* k_route, float* rq,
+                                     float* rk, cudaStream_t s) {
+  const int N = (cfg->T + cfg->C - 1) / cfg->C;
+  if (cfg->pool_window == 0) {
+    HLA_CUDA(hla::launch_pools(q_route, k_route, rq, rk, cfg->B, cfg->T, cfg->H, cfg->dk, cfg->C, N, cfg->tau,
+                               cfg->dtype, s),
+             "pool launch");
+    return HLA_OK;
+  }
+  if (q_route != nullptr && rq != nullptr)
+    HLA_CUDA(hla::launch_pools(q_route, nullptr, rq, nullptr, cfg->B, cfg->T, cfg->H, cfg->dk, cfg->C, N, cfg->tau,
+                               cfg->dtype, s),
+             "query pool launch");
+  if (k_route != nullptr && rk != nullptr)
+    HLA_CUDA(hla::launch_pools(nullptr, k_route, nullptr, rk, cfg->B, cfg->T, cfg->H, cfg->dk, cfg->pool_window,
+                               N * n_windows(cfg), cfg->tau, cfg->dtype, s),
+             "window pool launch");
+  return HLA_OK;
+}
+
 static hla_status routing_impl(const hla_config* cfg, const void* q_route, const void* k_route, float* rq,
                                float* rk, const float* user_gates, int32_t* act_idx, float* act_g,
                                int32_t* act_cnt, float* gates_out, int32_t* active_idx_out,
                                int32_t* active_cnt_out, cudaStream_t s) {
   const int N = (cfg->T + cfg->C - 1) / cfg->C;
   if (cfg->gate_mode == HLA_GATES_ROUTED || rk != nullptr) {
-    StageScope _sc(HLA_STAGE_POOLS, s, 1);
-    HLA_CUDA(hla::launch_pools(cfg->gate_mode == HLA_GATES_ROUTED ? q_route : nullptr, k_route,
-                               cfg->gate_mode == HLA_GATES_ROUTED ? rq : nullptr, rk, cfg->B, cfg->T, cfg->H,
-                               cfg->dk, cfg->C, N, cfg->tau, cfg->dtype, s),
-             "pool launch");
+    const bool routed = cfg->gate_mode == HLA_GATES_ROUTED;
+    StageScope _sc(HLA_STAGE_POOLS, s, cfg->pool_window > 0 ? 2 : 1);
+    HLA_TRY(launch_route_pools(cfg, routed ? q_route : nullptr, k_route, routed ? rq : nullptr, rk, s));
   }
   hla::GatesArgs g{};
   g.B = cfg->B;
@@ -403,6 +435,7 @@ static hla_status routing_impl(const hla_config* cfg, const void* q_route, const
   g.N = N;
   g.d = cfg->dk;
   g.mode = cfg->gate_mode;
+  g.win = n_windows(cfg);
   g.c_d = gate_scale(cfg->dk);
   g.bias = cfg->bias;
   g.thr = cfg->skip_threshold;
@@ -439,15 +472,14 @@ hla_status hla_routing(const hla_config* cfg, const void* q_route, const void* k
     return fail(HLA_ERR_INVALID_ARG, "active_idx_out and active_cnt_out go together");
   const int N = (cfg->T + cfg->C - 1) / cfg->C;
   cudaStream_t s = (cudaStream_t)stream;
-  HLA_CUDA(hla::launch_pools(q_route, k_route, rq_out, rk_out, cfg->B, cfg->T, cfg->H, cfg->dk, cfg->C, N,
-                             cfg->tau, cfg->dtype, s),
-           "pool launch");
+  HLA_TRY(launch_route_pools(cfg, q_route, k_route, rq_out, rk_out, s));
   hla::GatesArgs g{};
   g.B = cfg->B;
   g.H = cfg->H;
   g.N = N;
   g.d = cfg->dk;
   g.mode = cfg->gate_mode;
+  g.win = n_windows(cfg);
   g.c_d = gate_scale(cfg->dk);
   g.bias = cfg->bias;
   g.thr = cfg->skip_threshold;
@@ -654,6 +686,7 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
     dc.d = cfg->dk;
     dc.dtype = cfg->dtype;
     dc.max_chunks = cache_out->max_chunks;
+    dc.win = n_windows(cfg);
     dc.rk = cache_out->rk;
     dc.buf_k = cache_out->buf_k;
     dc.buf_v = cache_out->buf_v;
@@ -715,6 +748,7 @@ hla_status hla_decode_step(const hla_config* cfg, hla_cache* cache, const void* 
   a.dtype = cfg->dtype;
   a.mode = cfg->gate_mode;
   a.max_chunks = cache->max_chunks;
+  a.win = n_windows(cfg);
   a.tau = cfg->tau;
   a.c_d = gate_scale(cfg->dk);
   a.bias = cfg->bias;

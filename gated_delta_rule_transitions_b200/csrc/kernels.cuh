@@ -6,11 +6,15 @@
 
 namespace hla {
 
+// Window representatives: at most this many per chunk (C / pool_window).
+constexpr int kMaxWindows = 16;
+
 struct GatesArgs {
   int B, H, N, d, mode;
+  int win;                  // key representatives per chunk with windows (0: one pool per chunk)
   float c_d, bias, thr;
   const float* rq;          // [B,H,N,d]
-  const float* rk;          // [B,H,N,d]
+  const float* rk;          // [B,H,N,d], or [B,H,N*win,d] with windows
   const float* user_gates;  // [B,H,N,N] (mode USER)
   int32_t* act_idx;         // [B,H,N,N] compacted ascending j
   float* act_g;             // [B,H,N,N] matching gates
@@ -118,6 +122,7 @@ struct ReadoutArgs {
 
 struct DecodeArgs {
   int B, H, C, d, dtype, mode, max_chunks;
+  int win;             // window pools per closed chunk (0: one pool per chunk)
   float tau, c_d, bias, thr;
   const void* q;   // [B,H,d]
   const void* k;
@@ -135,7 +140,7 @@ struct DecodeArgs {
   void* Wf;
   void* Uf;
   float* df;           // factored: [B,H,max_chunks,C+4]
-  float* rk;
+  float* rk;           // [B,H,max_chunks,max(win,1),d]
   void* buf_k;
   void* buf_v;
   void* buf_qr;

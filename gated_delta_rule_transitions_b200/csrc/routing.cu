@@ -206,7 +206,8 @@ __global__ void __launch_bounds__(256) gates_kernel(GatesArgs a) {
   const int bh = warp / a.N;
   const route::Consts K = route::make_consts();
   const float* rq = a.rq + ((size_t)bh * a.N + i) * a.d;
-  const float* rk = a.rk + (size_t)bh * a.N * a.d;
+  const int W = a.win > 0 ? a.win : 1;
+  const float* rk = a.rk + (size_t)bh * a.N * W * a.d;
   const size_t row = (size_t)warp * a.N;
   int cnt = 0;
   for (int jb = 0; jb < a.N; jb += 32) {
@@ -214,7 +215,12 @@ __global__ void __launch_bounds__(256) gates_kernel(GatesArgs a) {
     float g = 0.0f;
     const bool valid = j < i;
     if (valid) {
-      if (a.mode == HLA_GATES_ROUTED) {
+      if (a.mode == HLA_GATES_ROUTED && a.win > 0) {
+        // log-sum-exp over the key chunk's window representatives
+        float t[kMaxWindows];
+        const float m = route::window_scores(rq, rk + (size_t)j * W * a.d, a.win, a.d, a.c_d, t);
+        g = route::gate_from_window_scores(t, a.win, m, a.bias, K);
+      } else if (a.mode == HLA_GATES_ROUTED) {
         const float* rkj = rk + (size_t)j * a.d;
         float dot = 0.0f;
         for (int c = 0; c < a.d; ++c) dot = route::dot_step(dot, rq[c], rkj[c]);
@@ -446,7 +452,7 @@ cudaError_t launch_pools(const void* x0, const void* x1, float* r0, float* r1, i
 }
 
 cudaError_t launch_gates(const GatesArgs& a, cudaStream_t s) {
-  if (a.mode == HLA_GATES_ROUTED && (a.d == 128 || a.d == 64)) {
+  if (a.mode == HLA_GATES_ROUTED && a.win == 0 && (a.d == 128 || a.d == 64)) {
     // 64-row tiles while they give two CTAs per SM or more, else 16-row tiles
     const long tiles64 = (long)((a.N + 63) / 64) * a.B * a.H;
     const bool small = tiles64 < 2L * num_sms();

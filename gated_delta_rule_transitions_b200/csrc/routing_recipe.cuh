@@ -21,6 +21,9 @@
 //   gate: dot = fma(rq[c], rk[c], dot) over ascending c from 0;
 //         z = fma(dot, c_d, b) with c_d = 1/sqrt(d) rounded once from double;
 //         g = 1 / (1 + exp(-z)).
+//   windowed gate (W window representatives per key chunk): t_u = dot_u * c_d;
+//         m = max_u t_u; s = sum_u exp(t_u - m) ascending; z = (m + log s) + b;
+//         g = 1 / (1 + exp(-z)).
 // All constants are derived from ln 2, 1/k! and 1/(2k+1), rounded once to binary32.
 #pragma once
 
@@ -119,6 +122,54 @@ __device__ __forceinline__ float dot_step(float acc, float a, float b) { return 
 __device__ __forceinline__ float gate_from_dot(float dot, float c_d, float bias, const Consts& k) {
   const float z = __fmaf_rn(dot, c_d, bias);
   return __frcp_rn(__fadd_rn(1.0f, rexp(-z, k)));  // 1/x correctly rounded, as 1.0f / x
+}
+
+// Window scores of one key chunk: t_u = dot_u * c_d for u < W, where each dot_u is
+// the gate's fma chain over ascending channels from 0.  The W chains are independent
+// and advance together (four channels per step, 16-byte loads).  rq and rkj (W rows
+// of d floats) are 16-byte aligned, d a multiple of 4.  Returns m = max_u t_u.
+template <int kMax>
+__device__ __forceinline__ float window_scores(const float* rq, const float* rkj, int W, int d, float c_d,
+                                               float (&t)[kMax]) {
+  float acc[kMax];
+#pragma unroll
+  for (int u = 0; u < kMax; ++u) acc[u] = 0.0f;
+  for (int c = 0; c < d; c += 4) {
+    const float4 q4 = *(const float4*)(rq + c);
+#pragma unroll
+    for (int u = 0; u < kMax; ++u)
+      if (u < W) {
+        const float4 r4 = *(const float4*)(rkj + (long)u * d + c);
+        acc[u] = dot_step(acc[u], q4.x, r4.x);
+        acc[u] = dot_step(acc[u], q4.y, r4.y);
+        acc[u] = dot_step(acc[u], q4.z, r4.z);
+        acc[u] = dot_step(acc[u], q4.w, r4.w);
+      }
+  }
+  float m = -CUDART_INF_F;
+#pragma unroll
+  for (int u = 0; u < kMax; ++u) {
+    t[u] = 0.0f;
+    if (u < W) {
+      t[u] = __fmul_rn(acc[u], c_d);
+      m = fmaxf(m, t[u]);
+    }
+  }
+  return m;
+}
+
+// Sigmoid of a log-sum-exp over a chunk's W window scores t_u = dot_u * c_d (each
+// rounded once), m = max_u t_u:  s = sum_u exp(t_u - m) in ascending u from 0;
+// z = (m + log s) + b;  g = 1 / (1 + exp(-z)).
+template <int kMax>
+__device__ __forceinline__ float gate_from_window_scores(const float (&t)[kMax], int W, float m, float bias,
+                                                        const Consts& k) {
+  float s = 0.0f;
+#pragma unroll
+  for (int u = 0; u < kMax; ++u)
+    if (u < W) s = __fadd_rn(s, rexp_nonpos(__fsub_rn(t[u], m), k));
+  const float z = __fadd_rn(__fadd_rn(m, rlog(s, k)), bias);
+  return __frcp_rn(__fadd_rn(1.0f, rexp(-z, k)));
 }
 
 }  // namespace route

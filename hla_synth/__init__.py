@@ -51,6 +51,7 @@ class Workload:
     route: str = "default"      # default | spread | planted
     seed: int = 0
     topics: int = 128
+    window: int = 0             # key window representatives of `window` tokens (0: one per chunk)
 
     @property
     def N(self) -> int:

@@ -22,7 +22,9 @@
  *   chunk c      tokens cC .. cC+C-1 act as S -> S A_c + B_c (exact)
  *   pools        r_c = tau * log(mean_t exp(x_t / tau)) per channel over chunk c's
  *                route tokens (route inputs default to q for r^q and k for r^k)
- *   gates        g_ij = sigmoid(<r^q_i, r^k_j> / sqrt(d) + bias), j < i, computed by
+ *   gates        g_ij = sigmoid(<r^q_i, r^k_j> / sqrt(d) + bias), j < i (with window
+ *                representatives: a log-sum-exp over chunk j's windows, see
+ *                hla_config.pool_window), computed by
  *                a fixed binary32 recipe (a fused multiply-add wherever a product
  *                feeds a sum, exp/log evaluated by a fixed polynomial scheme) so
  *                that gates and skip decisions are reproducible bit for bit
@@ -111,6 +113,13 @@ typedef struct hla_config {
   float tau;              /* pooling temperature, > 0                           */
   float bias;             /* gate bias b                                        */
   float skip_threshold;   /* <= 0: nothing skipped                              */
+  int32_t pool_window;    /* 0: one key representative per chunk.  w > 0: the
+                             pages' window representatives -- chunk j's key side is
+                             W = C / w pools of w tokens each (w >= 8, w < C, w | C,
+                             W <= 16) and the gate takes a log-sum-exp over them:
+                             g_ij = sigmoid(log sum_u exp(<r^q_i, r^k_ju> / sqrt(d)) + b)
+                             ("Methodology in Plain English" para. 2; "Main
+                             Findings": window 32 by default)                   */
 } hla_config;
 
 /*
@@ -121,7 +130,8 @@ typedef struct hla_config {
  *   Kf, Wf, Uf   [B, H, max_chunks, C, d]  dtype  -- K_j, Wb_j, Ub_j of closed chunks
  *   df           [B, H, max_chunks, C + 4] float32 -- gamma_C / gamma_t (t < C), then
  *                gamma_C, then padding (HLA_CACHE_FACTORED; all NULL otherwise)
- *   rk           [B, H, max_chunks, d]     float32 -- key pools of closed chunks
+ *   rk           [B, H, max_chunks, W, d]  float32 -- key pools of closed chunks (W = 1,
+ *                or C / pool_window window pools)
  *   buf_k, buf_v, buf_qr, buf_kr  [B, H, C, d] dtype -- tokens of the open chunk
  *   buf_alpha, buf_beta           [B, H, C]  float32
  *   n_chunks     [B] int32 -- closed chunks per sequence
@@ -133,6 +143,7 @@ typedef struct hla_cache {
   int32_t max_chunks;
   int32_t B, H, C, d, dtype;
   int32_t format; /* hla_cache_format */
+  int32_t pool_window; /* key representatives per closed chunk: 1, or C / pool_window */
   void* A;
   void* Bm;
   void* Kf;
@@ -198,7 +209,8 @@ hla_status gdn_chunk_transitions(const hla_config* cfg, const void* k, const voi
 /*
  * hla_routing -- pools and gates only (Overview; Methodology paras. 2 and 4).
  * In:  q_route, k_route [B,T,H,d] dtype (device; NULL is not allowed here).
- * Out: rq_out, rk_out [B,H,N,d] float32 (required), N = ceil(T/C);
+ * Out: rq_out [B,H,N,d], rk_out [B,H,N*W,d] float32 (required), N = ceil(T/C), W = 1
+ *      or C / pool_window (window u of chunk j at row j*W + u; windows past T unset);
  *      gates_out [B,H,N,N] float32 raw gates for j < i, 0 elsewhere (may be NULL);
  *      active_idx_out [B,H,N,N] int32: entries 0..cnt-1 of row i are the active j
  *      in ascending order, the rest are -1 (may be NULL together with cnt);

@@ -146,11 +146,32 @@ def route_pools(x_route, C: int, tau: float):
     return np.concatenate(out).astype(np.float32)
 
 
+def window_pools(x_route, C: int, window: int, tau: float):
+    """Window representatives of one head's complete chunks: every chunk of C tokens
+    is split into W = C / window windows, each pooled on its own by the log-mean-exp
+    pool.  x_route [T, d] -> [T // C, W, d] f32."""
+    x = np.asarray(x_route, np.float32)
+    nc = x.shape[0] // C
+    W = C // window
+    if nc == 0:
+        return np.zeros((0, W, x.shape[1]), np.float32)
+    r = rr.lme_pool32(x[:nc * C].reshape(nc * W, window, -1), tau)
+    return r.reshape(nc, W, -1).astype(np.float32)
+
+
 def gate_matrix(rq, rk, d: int, bias: float, mode: str = GATES_ROUTED, user=None):
     """Raw gates G [N, N] (binary32) with G[i, j] meaningful for j < i, zero elsewhere
-    (the current chunk's own weight is 1 by definition and is not a gate)."""
+    (the current chunk's own weight is 1 by definition and is not a gate).  rk is
+    [N_k, d] (one representative per chunk) or [N_k, W, d] (window representatives,
+    combined by a log-sum-exp inside the sigmoid); N_k may be smaller than N when
+    only the complete chunks have key representatives."""
     N = rq.shape[0]
-    if mode == GATES_ROUTED:
+    if mode == GATES_ROUTED and np.ndim(rk) == 3:
+        G = np.zeros((N, N), np.float32)
+        nk = rk.shape[0]
+        if nk:
+            G[:, :nk] = rr.gate_matrix_window32(rq, rk, d, bias)
+    elif mode == GATES_ROUTED:
         G = rr.gate_matrix32(rq, rk, d, bias)
     elif mode == GATES_ONE:
         G = np.ones((N, N), np.float32)
@@ -227,8 +248,11 @@ class HeadResult:
 
 def hla_prefill_head(q, k, v, alpha, beta, C, tau=1.0, bias=0.0, thr=0.0,
                      gate_mode=GATES_ROUTED, q_route=None, k_route=None,
-                     user_gates=None, query_chunks=None, trans=None):
+                     user_gates=None, query_chunks=None, trans=None, pool_window=0):
     """HLA prefill for one (sequence, head).  q, k: [T, d_k]; v: [T, d_v].
+
+    ``pool_window`` > 0: each chunk's key side is represented by its C / pool_window
+    window pools and the gate takes a log-sum-exp over them (``gate_window32``).
 
     ``query_chunks``: if given, only those query chunks' outputs are computed (the rest
     of ``o`` is NaN) -- used for sampled checks at full size.  ``trans``: optional
@@ -246,7 +270,7 @@ def hla_prefill_head(q, k, v, alpha, beta, C, tau=1.0, bias=0.0, thr=0.0,
     qr = q if q_route is None else q_route
     kr = k if k_route is None else k_route
     rq = route_pools(qr, C, tau)
-    rk = route_pools(kr, C, tau)
+    rk = window_pools(kr, C, pool_window, tau) if pool_window else route_pools(kr, C, tau)
     G = gate_matrix(rq, rk, dk, bias, gate_mode, user_gates)
     act = active_lists(G, thr)
     n_complete = T // C
@@ -265,7 +289,7 @@ def hla_prefill_head(q, k, v, alpha, beta, C, tau=1.0, bias=0.0, thr=0.0,
 
 
 def hla_prefill(q, k, v, alpha, beta, C, tau=1.0, bias=0.0, thr=0.0,
-                gate_mode=GATES_ROUTED, q_route=None, k_route=None, user_gates=None):
+                gate_mode=GATES_ROUTED, q_route=None, k_route=None, user_gates=None, pool_window=0):
     """Batched prefill over [B, T, H, d] inputs (alpha, beta: [B, T, H];
     user_gates: [B, H, N, N]).  Returns (o [B, T, H, d_v], {(b, h): HeadResult})."""
     Bn, T, H, _ = np.shape(q)
@@ -279,7 +303,7 @@ def hla_prefill(q, k, v, alpha, beta, C, tau=1.0, bias=0.0, thr=0.0,
                 tau, bias, thr, gate_mode,
                 None if q_route is None else q_route[b, :, h],
                 None if k_route is None else k_route[b, :, h],
-                None if user_gates is None else user_gates[b, h])
+                None if user_gates is None else user_gates[b, h], pool_window=pool_window)
             o[b, :, h] = r.o
             res[(b, h)] = r
     return o, res
@@ -299,20 +323,21 @@ class HlaDecodeHead:
     rule over the buffered tokens from S_in.  When the partial chunk reaches C tokens
     it is closed: its transition and key pool are appended to the cache."""
 
-    def __init__(self, C, d_k, d_v, tau=1.0, bias=0.0, thr=0.0, gate_mode=GATES_ROUTED):
+    def __init__(self, C, d_k, d_v, tau=1.0, bias=0.0, thr=0.0, gate_mode=GATES_ROUTED, pool_window=0):
         self.C, self.dk, self.dv = C, d_k, d_v
         self.tau, self.bias, self.thr, self.mode = tau, bias, thr, gate_mode
+        self.window = pool_window
         self.trans = []       # [(A_j, B_j)] float64
-        self.rk = []          # [d] float32 pools
+        self.rk = []          # [d] float32 pools ([W, d] window pools with pool_window > 0)
         self.buf = []         # [(q, k, v, alpha, beta, q_route, k_route)]
 
     @classmethod
     def from_prefill(cls, q, k, v, alpha, beta, C, tau=1.0, bias=0.0, thr=0.0,
-                     gate_mode=GATES_ROUTED, q_route=None, k_route=None, trans=None):
+                     gate_mode=GATES_ROUTED, q_route=None, k_route=None, trans=None, pool_window=0):
         """Cache state after a prefill of one head's T tokens."""
         T, dk = np.shape(k)
         dv = np.shape(v)[1]
-        st = cls(C, dk, dv, tau, bias, thr, gate_mode)
+        st = cls(C, dk, dv, tau, bias, thr, gate_mode, pool_window)
         qr = q if q_route is None else q_route
         kr = k if k_route is None else k_route
         n = T // C
@@ -323,11 +348,16 @@ class HlaDecodeHead:
                                       alpha[c * C:(c + 1) * C], beta[c * C:(c + 1) * C])
                      for c in range(n)]
         st.trans = list(trans[:n])
-        st.rk = [rr.lme_pool32(np.asarray(kr[c * C:(c + 1) * C], np.float32), tau)
-                 for c in range(n)]
+        st.rk = [st._key_rep(np.asarray(kr[c * C:(c + 1) * C], np.float32)) for c in range(n)]
         for t in range(n * C, T):
             st.buf.append((q[t], k[t], v[t], alpha[t], beta[t], qr[t], kr[t]))
         return st
+
+    def _key_rep(self, krs):
+        """Key representative(s) of one closed chunk's C route keys."""
+        if self.window:
+            return window_pools(krs, self.C, self.window, self.tau)[0]
+        return rr.lme_pool32(krs, self.tau)
 
     def gates(self):
         """Raw binary32 gates of the partial chunk against all cached chunks."""
@@ -340,6 +370,8 @@ class HlaDecodeHead:
             return np.zeros(n, np.float32)
         qr = np.stack([np.asarray(b[5], np.float32) for b in self.buf])
         rq = rr.lme_pool32(qr, self.tau)
+        if self.window:
+            return rr.gate_window32(rq[None, :], np.stack(self.rk), self.dk, self.bias)
         return rr.gate32(rq[None, :], np.stack(self.rk), self.dk, self.bias)
 
     def active(self, g):
@@ -373,7 +405,7 @@ class HlaDecodeHead:
         be = np.array([float(b[4]) for b in self.buf])
         krs = np.stack([np.asarray(b[6], np.float32) for b in self.buf])
         self.trans.append(chunk_transition(ks, vs, al, be))
-        self.rk.append(rr.lme_pool32(krs, self.tau))
+        self.rk.append(self._key_rep(krs))
         self.buf = []
 
 

@@ -201,6 +201,31 @@ def gate_matrix32(rq, rk, d: int, bias: float):
     return gate32(rq[:, None, :], rk[None, :, :], d, bias)
 
 
+def gate_window32(rq, rkw, d: int, bias: float):
+    """Gate against a chunk summarised by W window representatives (the pages'
+    log-sum-exp over a chunk's representatives, then a sigmoid).  rq [..., d],
+    rkw [..., W, d].  Steps, all binary32:
+    t_u = dot32(rq, rk_u) * c_d (one rounding); m = max_u t_u;
+    s = sum over ascending u of exp32(t_u - m), one rounding per add, from 0;
+    z = (m + log32(s)) + bias (two roundings); g = 1 / (1 + exp32(-z))."""
+    rq = _f32(rq)
+    rkw = _f32(rkw)
+    t = (dot32(rq[..., None, :], rkw) * gate_scale(d)).astype(np.float32)
+    m = t.max(axis=-1)
+    s = np.zeros_like(m)
+    for u in range(t.shape[-1]):
+        s = (s + exp32((t[..., u] - m).astype(np.float32))).astype(np.float32)
+    z = ((m + log32(s)).astype(np.float32) + F32(bias)).astype(np.float32)
+    return (F32(1.0) / (F32(1.0) + exp32(-z))).astype(np.float32)
+
+
+def gate_matrix_window32(rq, rkw, d: int, bias: float):
+    """All pairs: rq [N_q, d], rkw [N_k, W, d] -> G [N_q, N_k] by gate_window32."""
+    rq = _f32(rq)
+    rkw = _f32(rkw)
+    return gate_window32(rq[:, None, :], rkw[None, :, :, :], d, bias)
+
+
 # ---- fp64 statements of the same quantities (to measure the recipe's own error) -----
 
 def lme_pool64(x, tau: float):
@@ -212,4 +237,14 @@ def gate64(rq, rk, d: int, bias: float):
     rq = np.asarray(rq, dtype=np.float64)
     rk = np.asarray(rk, dtype=np.float64)
     z = np.sum(rq * rk, axis=-1) / math.sqrt(d) + bias
+    return 1.0 / (1.0 + np.exp(-z))
+
+
+def gate_window64(rq, rkw, d: int, bias: float):
+    """sigmoid(log sum_u exp(<rq, rk_u> / sqrt(d)) + bias) in float64."""
+    rq = np.asarray(rq, dtype=np.float64)
+    rkw = np.asarray(rkw, dtype=np.float64)
+    t = np.sum(rq[..., None, :] * rkw, axis=-1) / math.sqrt(d)
+    m = t.max(axis=-1)
+    z = m + np.log(np.sum(np.exp(t - m[..., None]), axis=-1)) + bias
     return 1.0 / (1.0 + np.exp(-z))

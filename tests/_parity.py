@@ -40,7 +40,8 @@ def to_cuda(inp):
 def run_prefill(hla, w: syn.Workload, inp, user_gates=None, cache=None, cache_format="dense"):
     B, T, H, d = inp["q"].shape
     N = (T + w.C - 1) // w.C
-    cfg = hla.make_config(B, H, T, w.C, d, w.dtype, w.gate_mode, w.tau, w.bias, w.thr, cache_format=cache_format)
+    cfg = hla.make_config(B, H, T, w.C, d, w.dtype, w.gate_mode, w.tau, w.bias, w.thr, cache_format=cache_format,
+                          pool_window=w.window)
     g = to_cuda(inp)
     o = torch.empty_like(g["q"])
     gates = torch.empty((B, H, N, N), dtype=torch.float32, device="cuda")
@@ -62,7 +63,7 @@ def oracle_prefill_head(w: syn.Workload, inp, b, h, user_gates=None, query_chunk
         None if inp.get("q_route") is None else np32(inp["q_route"][b, :, h]),
         None if inp.get("k_route") is None else np32(inp["k_route"][b, :, h]),
         None if user_gates is None else user_gates[b, h].numpy(),
-        query_chunks=query_chunks)
+        query_chunks=query_chunks, pool_window=w.window)
 
 
 def check_routing_exact(res, gates, aidx, acnt, b, h):

@@ -255,3 +255,23 @@ def test_gate_support_needs_an_output(hla):
     assert st == hla.HLA_ERR_INVALID_ARG and "both NULL" in hla.last_error()
     st = hla.lib().hla_gate_support(ctypes.byref(c), None, P, P, None)
     assert st == hla.HLA_ERR_INVALID_ARG and "gates is NULL" in hla.last_error()
+
+
+@pytest.mark.parametrize("C,w,ok", [(64, 32, True), (64, 16, True), (256, 32, True), (256, 16, True),
+                                    (256, 8, False), (64, 64, False), (64, 4, False), (64, 48, False)])
+def test_pool_window_shapes(hla, C, w, ok):
+    """Window representatives: 8 <= w < C, w divides C, at most 16 windows per chunk."""
+    c = cfg(hla, T=1024, C=C, pool_window=w)
+    assert (hla.prefill_workspace_bytes(c) > 0) == ok
+    if not ok:
+        P = ctypes.c_void_p(0x100000)
+        assert hla.lib().gdn_chunk_transitions(ctypes.byref(c), P, P, P, P, P, P, None) == hla.HLA_ERR_UNSUPPORTED
+        assert "pool_window" in hla.last_error()
+
+
+def test_window_pools_enlarge_the_key_cache(hla):
+    d = 128
+    base = cfg(hla, T=1, C=256)
+    win = cfg(hla, T=1, C=256, pool_window=32)
+    per_chunk = lambda c: hla.cache_bytes(c, 101) - hla.cache_bytes(c, 100)
+    assert per_chunk(win) - per_chunk(base) == 7 * d * 4   # 8 window pools instead of one

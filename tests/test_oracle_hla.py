@@ -219,15 +219,15 @@ def _steps(rng, n, d):
     return out
 
 
-@pytest.mark.parametrize("T0", [16, 21])
-def test_decode_matches_prefill_of_extended_sequence(T0):
+@pytest.mark.parametrize("T0,window", [(16, 0), (21, 0), (21, 4), (19, 2)])
+def test_decode_matches_prefill_of_extended_sequence(T0, window):
     rng = np.random.default_rng(22 + T0)
     C, d = 8, 6
     q, k, v, a, b = _head(rng, T0, d)
     qr = rng.standard_normal((T0, d)) * 2
     kr = rng.standard_normal((T0, d)) * 2
     st = ho.HlaDecodeHead.from_prefill(q, k, v, a, b, C, bias=-0.5, thr=0.3,
-                                       q_route=qr, k_route=kr)
+                                       q_route=qr, k_route=kr, pool_window=window)
     toks = _steps(rng, 12, d)   # crosses a chunk boundary
     for s, (tq, tk, tv, ta, tb) in enumerate(toks):
         tqr = rng.standard_normal(d) * 2
@@ -237,7 +237,7 @@ def test_decode_matches_prefill_of_extended_sequence(T0):
         a = np.append(a, ta); b = np.append(b, tb)
         qr = np.vstack([qr, tqr]); kr = np.vstack([kr, tkr])
         ref = ho.hla_prefill_head(q, k, v, a, b, C, bias=-0.5, thr=0.3, q_route=qr,
-                                  k_route=kr, query_chunks=[(len(a) - 1) // C])
+                                  k_route=kr, query_chunks=[(len(a) - 1) // C], pool_window=window)
         assert np.abs(o - ref.o[-1]).max() <= 1e-12
     # closed chunks in the cache equal the literal transitions and pools
     n = len(a) // C
@@ -245,7 +245,12 @@ def test_decode_matches_prefill_of_extended_sequence(T0):
     A, B = ho.chunk_transition(k[(n - 1) * C:n * C], v[(n - 1) * C:n * C], a[(n - 1) * C:n * C],
                                b[(n - 1) * C:n * C])
     assert np.abs(st.trans[-1][0] - A).max() <= 1e-14
-    assert np.array_equal(st.rk[-1], rr.lme_pool32(kr[(n - 1) * C:n * C].astype(np.float32), 1.0))
+    last = kr[(n - 1) * C:n * C].astype(np.float32)
+    if window:
+        for u in range(C // window):
+            assert np.array_equal(st.rk[-1][u], rr.lme_pool32(last[u * window:(u + 1) * window], 1.0))
+    else:
+        assert np.array_equal(st.rk[-1], rr.lme_pool32(last, 1.0))
 
 
 def test_decode_backward_chain_equals_forward_composition():

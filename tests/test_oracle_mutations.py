@@ -60,6 +60,26 @@ def _bad_exp(x):
     return (np.exp(x.astype(np.float64)) * (1 + 3e-7)).astype(np.float32)
 
 
+def _window_gate_mean(rq, rkw, d, bias):
+    # a log-MEAN-exp over the windows instead of the log-sum-exp (drops log W)
+    rkw = np.asarray(rkw, np.float32)
+    t = (rr.dot32(np.asarray(rq, np.float32)[..., None, :], rkw) * rr.gate_scale(d)).astype(np.float32)
+    m = t.max(axis=-1)
+    s = np.zeros_like(m)
+    for u in range(t.shape[-1]):
+        s = (s + rr.exp32((t[..., u] - m).astype(np.float32))).astype(np.float32)
+    z = ((m + rr.log32(s / np.float32(t.shape[-1]))).astype(np.float32) + np.float32(bias)).astype(np.float32)
+    return (np.float32(1.0) / (np.float32(1.0) + rr.exp32(-z))).astype(np.float32)
+
+
+def _window_gate_max(rq, rkw, d, bias):
+    # the best window alone instead of the log-sum-exp
+    rkw = np.asarray(rkw, np.float32)
+    t = (rr.dot32(np.asarray(rq, np.float32)[..., None, :], rkw) * rr.gate_scale(d)).astype(np.float32)
+    z = (t.max(axis=-1) + np.float32(bias)).astype(np.float32)
+    return (np.float32(1.0) / (np.float32(1.0) + rr.exp32(-z))).astype(np.float32)
+
+
 def _run(fn, *args):
     try:
         fn(*args)
@@ -76,6 +96,8 @@ CASES = [
     ("compose_state", _ungated_b_compose, ho),
     ("lme_pool32", _mean_pool, rr),
     ("exp32", _bad_exp, rr),
+    ("gate_window32", _window_gate_mean, rr),
+    ("gate_window32", _window_gate_max, rr),
 ]
 
 
@@ -86,9 +108,11 @@ def test_planted_mistake_is_caught(monkeypatch, name, bad, mod):
         (th.test_wy_form_equals_literal_transition, 16, 12, 12),
         (th.test_exact_rational_brute_force, 8, 2, 2),
         (th.test_exact_rational_brute_force, 8, 4, 3),
-        (th.test_decode_matches_prefill_of_extended_sequence, 16),
+        (th.test_decode_matches_prefill_of_extended_sequence, 16, 0),
         (tr.test_lme_matches_float64_definition,),
         (tr.test_exp32_error_bound,),
+        (tr.test_window_gate_matches_float64_definition,),
+        (tr.test_window_gate_of_equal_windows_adds_log_count,),
     ]
     caught = [p[0].__name__ for p in pins if _run(*p)]
     assert caught, f"no pin caught the planted mistake in {name}"

@@ -211,3 +211,53 @@ def test_active_lists_threshold_semantics():
     assert [list(a) for a in act] == [[], [], [1], [1, 2]]   # equality is kept
     dense = ho.active_lists(G, 0.0)
     assert [list(a) for a in dense] == [[], [0], [0, 1], [0, 1, 2]]
+
+
+# ---- window representatives: log-sum-exp over a chunk's windows, then a sigmoid ----
+
+def test_window_gate_matches_float64_definition():
+    # the binary32 recipe against sigmoid(log sum_u exp(<rq, rk_u>/sqrt(d)) + b) in fp64
+    rng = np.random.default_rng(41)
+    d, W = 64, 8
+    rq = (rng.standard_normal((200, d)) * 0.8).astype(np.float32)
+    rkw = (rng.standard_normal((200, W, d)) * 0.8).astype(np.float32)
+    g32 = rr.gate_window32(rq, rkw, d, -2.0)
+    g64 = rr.gate_window64(rq, rkw, d, -2.0)
+    assert np.abs(g32.astype(np.float64) - g64).max() <= 2e-6
+
+
+def test_window_gate_of_equal_windows_adds_log_count():
+    # W equal representatives: log sum_u exp(t) = t + log W exactly
+    rng = np.random.default_rng(42)
+    d = 32
+    rq = rng.standard_normal(d).astype(np.float32)
+    r = rng.standard_normal(d).astype(np.float32)
+    for W in (2, 4, 8, 16):
+        g = rr.gate_window32(rq, np.tile(r, (W, 1)), d, 0.5)
+        t = float(np.dot(rq.astype(np.float64), r.astype(np.float64))) / np.sqrt(d)
+        ref = 1.0 / (1.0 + np.exp(-(t + np.log(W) + 0.5)))
+        assert abs(float(g) - ref) <= 2e-6
+
+
+def test_window_gate_follows_the_dominant_window():
+    # one window far above the others: the gate tends to the single-window gate of it
+    d = 16
+    rq = np.zeros(d, np.float32)
+    rq[3] = 8.0
+    rkw = np.zeros((4, d), np.float32)
+    rkw[2, 3] = 8.0                    # score 64 / 4 = 16; the rest score 0
+    g = float(rr.gate_window32(rq, rkw, d, -18.0))
+    ref = 1.0 / (1.0 + np.exp(-(16.0 + np.log1p(3 * np.exp(-16.0)) - 18.0)))
+    assert abs(g - ref) <= 1e-6
+    assert abs(g - 1.0 / (1.0 + np.exp(2.0))) <= 1e-5
+
+
+def test_window_pools_are_per_window_lme():
+    rng = np.random.default_rng(43)
+    x = rng.standard_normal((3 * 16 + 5, 4)).astype(np.float32)
+    r = ho.window_pools(x, 16, 4, 1.0)
+    assert r.shape == (3, 4, 4)          # complete chunks only
+    for c in range(3):
+        for u in range(4):
+            seg = x[16 * c + 4 * u:16 * c + 4 * u + 4]
+            assert np.array_equal(r[c, u], rr.lme_pool32(seg, 1.0))
