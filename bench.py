@@ -80,11 +80,11 @@ def whole_job_rate(units_per_rank, ms_max, world):
 #   compose: full-size launch of the dense 0.8B-like prefill (compose_tc_prefill_0p8b.md)
 #   decode_main: see below
 NCU_TRAFFIC = {
-    "compose": (2.0401e9, {"compose_tc.cu": "9feae23bf70ea63b", "tc_common.cuh": "c10beda371c1dd4b"}),
+    "compose": (2.0461e9, {"compose_tc.cu": "82d501993514b885", "tc_common.cuh": "c10beda371c1dd4b"}),
     # decode_main: capture of a 4-sequence decode (64 of the 1024 (sequence, head)
     # streams), scaled by 16; per stream it equals the algorithmic bytes
     # (decode_stream_decode_32k.md)
-    "decode_main": (3.4709e10, {"decode_stream.cu": "2dacede8d7508a41", "tc_common.cuh": "c10beda371c1dd4b"}),
+    "decode_main": (3.4693e10, {"decode_stream.cu": "eed338d0b2dada30", "tc_common.cuh": "c10beda371c1dd4b"}),
 }
 
 
