@@ -272,13 +272,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 // columns and split the 64 rows between them (rows with bit 2 clear / set, so the two
 // read disjoint banks): w = Wb^T z', u = Ub^T z'.  Then y += g u,
 // x <- (1 - g + g gamma_C) x - g w.
-constexpr int kFStages = 4;
+constexpr int kFStages = 2;  // two CTAs per SM: 4 stages of 49 KiB in flight per SM
 constexpr int kFTile = 64 * kD * 2;                 // 16 KiB: one 64 x 128 bf16 factor
 constexpr int kFScale = (64 + 4) * 4;               // scales of one chunk
 constexpr int kFStageBytes = 3 * kFTile + 1024;     // K, Wb, Ub, scales (1 KiB aligned)
 constexpr uint32_t kFTx = 3 * kFTile + kFScale;
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     decode_stream_factored_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmW,
                                   const __grid_constant__ CUtensorMap tmU, DecodeArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
