@@ -434,6 +434,131 @@ static cudaError_t launch_gates_tiled(const GatesArgs& a, cudaStream_t s) {
 }
 
 // ---------------------------------------------------------------------------
+// Routed gates with window representatives, tiled: one CTA per (TI query chunks,
+// b, h), 256 threads.  Key rows are the window pools (row j * W + u of chunk j);
+// a tile holds 64 of them, i.e. 64 / W chunks.  Per tile:
+//   1. TI x 64 window scores t = dot * c_d, each dot one fma chain over ascending
+//      channels (TI / 4 chains per thread, key row fixed per thread);
+//   2. one thread per (query chunk, key chunk) takes the log-sum-exp over its W
+//      scores in ascending u and the sigmoid (the recipe of gate_from_window_scores);
+//   3. warps compact each row's kept chunks in ascending j.
+// Query and key tiles are row-major with one float of padding per row, so the key
+// reads of a warp (32 different rows, one channel) fall in distinct banks.
+// ---------------------------------------------------------------------------
+template <int D, int TI>
+__global__ void __launch_bounds__(256) gates_window_tiled_kernel(GatesArgs a) {
+  constexpr int KR = 64;            // key rows (window pools) per tile
+  constexpr int DP = D + 1;
+  constexpr int CH = TI / 4;        // dot chains per thread
+  extern __shared__ float smf[];
+  float* rqS = smf;                         // [TI][DP]
+  float* rkS = rqS + TI * DP;               // [KR][DP]
+  float* Ts = rkS + KR * DP;                // [TI][KR]  scores
+  float* Gs = Ts + TI * KR;                 // [TI][KR]  gates of the tile's chunks
+  int* cnt_s = reinterpret_cast<int*>(Gs + TI * KR);  // [TI]
+  const int W = a.win;
+  const int JC = KR / W;                    // chunks per tile
+  const int i0 = blockIdx.x * TI;
+  const int bh = blockIdx.y;
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const route::Consts K = route::make_consts();
+  const float* rq = a.rq + (size_t)bh * a.N * D;
+  const float* rk = a.rk + (size_t)bh * a.N * W * D;
+  for (int e = tid; e < TI * D; e += 256) {
+    const int r = e / D, c = e - r * D;
+    rqS[r * DP + c] = i0 + r < a.N ? rq[(size_t)(i0 + r) * D + c] : 0.0f;
+  }
+  if (tid < TI) cnt_s[tid] = 0;
+  const int i_last = min(a.N, i0 + TI) - 1;
+  const int kr = tid & (KR - 1);            // key row of this thread
+  const int qb = (tid >> 6) * CH;           // first query row of this thread
+  for (int j0 = 0; j0 < i_last; j0 += JC) {
+    __syncthreads();  // the previous tile's readers are done
+    for (int e = tid; e < KR * D; e += 256) {
+      const int r = e / D, c = e - r * D;
+      const size_t row = (size_t)j0 * W + r;
+      rkS[r * DP + c] = row < (size_t)a.N * W ? rk[row * D + c] : 0.0f;
+    }
+    __syncthreads();
+    float acc[CH];
+#pragma unroll
+    for (int q = 0; q < CH; ++q) acc[q] = 0.0f;
+#pragma unroll 4
+    for (int c = 0; c < D; ++c) {
+      const float kv = rkS[kr * DP + c];
+#pragma unroll
+      for (int q = 0; q < CH; ++q) acc[q] = route::dot_step(acc[q], rqS[(qb + q) * DP + c], kv);
+    }
+#pragma unroll
+    for (int q = 0; q < CH; ++q) Ts[(qb + q) * KR + kr] = __fmul_rn(acc[q], a.c_d);
+    __syncthreads();
+    for (int e = tid; e < TI * JC; e += 256) {
+      const int r = e / JC, jj = e - r * JC;
+      const float* t = Ts + r * KR + jj * W;
+      float m = t[0];
+      for (int u = 1; u < W; ++u) m = fmaxf(m, t[u]);
+      float sum = 0.0f;
+      for (int u = 0; u < W; ++u) sum = __fadd_rn(sum, route::rexp_nonpos(__fsub_rn(t[u], m), K));
+      const float z = __fadd_rn(__fadd_rn(m, route::rlog(sum, K)), a.bias);
+      Gs[r * KR + jj] = __frcp_rn(__fadd_rn(1.0f, route::rexp(-z, K)));
+    }
+    __syncthreads();
+    // compaction: warp w handles rows w, w + 8, ...; lanes over the tile's chunks
+    for (int r = warp; r < TI; r += 8) {
+      const int i = i0 + r;
+      if (i >= a.N) continue;
+      const size_t row = ((size_t)bh * a.N + i) * a.N;
+      int cnt = cnt_s[r];
+      const int j = j0 + lane;
+      const bool valid = lane < JC && j < i;
+      const float g = lane < JC ? Gs[r * KR + lane] : 0.0f;
+      const bool keep = valid && (a.thr <= 0.0f || g >= a.thr);
+      const unsigned int bal = __ballot_sync(0xFFFFFFFFu, keep);
+      if (keep) {
+        const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
+        if (a.act_idx) a.act_idx[row + pos] = j;
+        if (a.act_g) a.act_g[row + pos] = g;
+      }
+      if (a.gates_out && lane < JC && j < a.N) a.gates_out[row + j] = valid ? g : 0.0f;
+      if (lane == 0) cnt_s[r] = cnt + __popc(bal);
+    }
+  }
+  __syncthreads();
+  // counts, zero gates beyond the computed tiles, padding and copies
+  for (int r = warp; r < TI; r += 8) {
+    const int i = i0 + r;
+    if (i >= a.N) continue;
+    const size_t row = ((size_t)bh * a.N + i) * a.N;
+    const int cnt = cnt_s[r];
+    if (lane == 0) {
+      if (a.act_cnt) a.act_cnt[(size_t)bh * a.N + i] = cnt;
+      if (a.active_cnt_out) a.active_cnt_out[(size_t)bh * a.N + i] = cnt;
+    }
+    const int jdone = (i_last > 0) ? ((i_last + JC - 1) / JC) * JC : 0;
+    if (a.gates_out)
+      for (int j = jdone + lane; j < a.N; j += 32) a.gates_out[row + j] = 0.0f;
+    if (a.pad_act_idx && a.act_idx)
+      for (int p = cnt + lane; p < a.N; p += 32) a.act_idx[row + p] = -1;
+    if (a.active_idx_out) {
+      __syncwarp();
+      for (int p = lane; p < a.N; p += 32) a.active_idx_out[row + p] = p < cnt ? a.act_idx[row + p] : -1;
+    }
+  }
+}
+
+template <int D, int TI>
+static cudaError_t launch_gates_window_tiled(const GatesArgs& a, cudaStream_t s) {
+  dim3 grid((a.N + TI - 1) / TI, a.B * a.H);
+  const size_t smem = (size_t)(TI * (D + 1) + 64 * (D + 1) + 2 * TI * 64 + TI) * 4;
+  cudaError_t e = cudaFuncSetAttribute(gates_window_tiled_kernel<D, TI>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  gates_window_tiled_kernel<D, TI><<<grid, 256, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
 // Launchers
 // ---------------------------------------------------------------------------
 cudaError_t launch_pools(const void* x0, const void* x1, float* r0, float* r1, int B, int T, int H, int d,
@@ -458,6 +583,14 @@ cudaError_t launch_gates(const GatesArgs& a, cudaStream_t s) {
     const bool small = tiles64 < 2L * num_sms();
     if (a.d == 128) return small ? launch_gates_tiled<128, 16>(a, s) : launch_gates_tiled<128, 64>(a, s);
     return small ? launch_gates_tiled<64, 16>(a, s) : launch_gates_tiled<64, 64>(a, s);
+  }
+  if (a.mode == HLA_GATES_ROUTED && a.win > 0 && 64 % a.win == 0 && (a.d == 128 || a.d == 64)) {
+    // 16 query chunks per CTA while that gives two CTAs per SM or more, else 4
+    const long tiles16 = (long)((a.N + 15) / 16) * a.B * a.H;
+    const bool small = tiles16 < 2L * num_sms();
+    if (a.d == 128)
+      return small ? launch_gates_window_tiled<128, 4>(a, s) : launch_gates_window_tiled<128, 16>(a, s);
+    return small ? launch_gates_window_tiled<64, 4>(a, s) : launch_gates_window_tiled<64, 16>(a, s);
   }
   const long rows = (long)a.B * a.H * a.N;
   const int blocks = (int)((rows * 32 + 255) / 256);
