@@ -221,10 +221,10 @@ def build_decode_cache(hla, syn, torch, w, max_chunks, group=8, cache_format="de
     API: hla_prefill with every earlier-chunk weight 0 writes the cache (A/B/key pools
     do not depend on gates) without the quadratic composition."""
     cfg = hla.make_config(w.B, w.H, w.T, w.C, w.d, w.dtype, "routed", w.tau, w.bias, w.thr, cache_format=cache_format,
-                          pool_window=w.window)
+                          pool_window=w.window, decay=w.decay)
     cache = hla.Cache(cfg, max_chunks)
     gcfg = hla.make_config(group, w.H, w.T, w.C, w.d, w.dtype, "zero", w.tau, w.bias, w.thr,
-                           cache_format=cache_format, pool_window=w.window)
+                           cache_format=cache_format, pool_window=w.window, decay=w.decay)
     ws = torch.empty(hla.prefill_workspace_bytes(gcfg), dtype=torch.uint8, device="cuda")
     first_ctx = None
     for b0 in range(0, w.B, group):
@@ -265,6 +265,8 @@ def run_ours(args):
         wp = wp.with_(C=args.chunk, name=wp.name.replace("_C64_", f"_C{args.chunk}_"))
     if args.pool_window:
         wp = wp.with_(window=args.pool_window, name=f"{wp.name}_window{args.pool_window}")
+    if args.decay != "scalar":
+        wp = wp.with_(decay=args.decay, name=f"{wp.name}_{args.decay}_decay")
     # the long sparse workload is generated on the device (5 x 1 GiB of inputs)
     gen_dev = "cuda" if wp.B * wp.T * wp.H * wp.d > (1 << 28) else "cpu"
     inp = syn.make_gdn_inputs(wp, device=gen_dev)
@@ -276,7 +278,7 @@ def run_ours(args):
     del inp
     inp = host
     pcfg = hla.make_config(wp.B, wp.H, wp.T, wp.C, wp.d, wp.dtype, wp.gate_mode, wp.tau, wp.bias, wp.thr,
-                           pool_window=wp.window)
+                           pool_window=wp.window, decay=wp.decay)
     pws = torch.empty(hla.prefill_workspace_bytes(pcfg), dtype=torch.uint8, device="cuda")
     o = torch.empty_like(dev["q"])
     o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
@@ -301,12 +303,14 @@ def run_ours(args):
         wd = wd.with_(C=args.chunk, name=wd.name.replace("_C64_", f"_C{args.chunk}_"))
     if args.pool_window:
         wd = wd.with_(window=args.pool_window, name=f"{wd.name}_window{args.pool_window}")
+    if args.decay != "scalar":
+        wd = wd.with_(decay=args.decay, name=f"{wd.name}_{args.decay}_decay")
     max_chunks = wd.T // wd.C + 1
     cache, ctx0 = build_decode_cache(hla, syn, torch, wd, max_chunks, group=min(8, wd.B),
                                      cache_format=args.decode_cache)
     torch.cuda.empty_cache()
     dcfg = hla.make_config(wd.B, wd.H, 1, wd.C, wd.d, wd.dtype, wd.gate_mode, wd.tau, wd.bias, wd.thr,
-                           cache_format=args.decode_cache, pool_window=wd.window)
+                           cache_format=args.decode_cache, pool_window=wd.window, decay=wd.decay)
     dws = torch.empty(hla.decode_workspace_bytes(dcfg, max_chunks), dtype=torch.uint8, device="cuda")
     ntok = args.warmup + args.steps + 1
     toks_host = [{k: v.contiguous().pin_memory() for k, v in t.items()} for t in syn.make_decode_tokens(wd, ntok)]
@@ -678,6 +682,8 @@ def main(argv=None):
                     help="chunk size C of both workloads (the metric's workloads use 64)")
     ap.add_argument("--pool-window", type=int, default=0,
                     help="key window representatives of this many tokens (0: one pool per chunk)")
+    ap.add_argument("--decay", choices=["scalar", "channel"], default="scalar",
+                    help="scalar: one decay per token (the metric's workloads); channel: one per key channel")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

@@ -29,19 +29,21 @@ HLA_CACHE_DENSE = 0
 HLA_CACHE_FACTORED = 1
 CACHE_FORMATS = {"dense": HLA_CACHE_DENSE, "factored": HLA_CACHE_FACTORED}
 GATE_MODES = {"routed": 0, "one": 1, "zero": 2, "user": 3}
+DECAY_MODES = {"scalar": 0, "channel": 1}
 
 
 class HlaConfig(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("T", ctypes.c_int32), ("C", ctypes.c_int32),
                 ("dk", ctypes.c_int32), ("dv", ctypes.c_int32), ("dtype", ctypes.c_int32),
                 ("gate_mode", ctypes.c_int32), ("cache_format", ctypes.c_int32), ("tau", ctypes.c_float),
-                ("bias", ctypes.c_float), ("skip_threshold", ctypes.c_float), ("pool_window", ctypes.c_int32)]
+                ("bias", ctypes.c_float), ("skip_threshold", ctypes.c_float), ("pool_window", ctypes.c_int32),
+                ("decay_mode", ctypes.c_int32)]
 
 
 class HlaCache(ctypes.Structure):
     _fields_ = [("max_chunks", ctypes.c_int32), ("B", ctypes.c_int32), ("H", ctypes.c_int32),
                 ("C", ctypes.c_int32), ("d", ctypes.c_int32), ("dtype", ctypes.c_int32),
-                ("format", ctypes.c_int32), ("pool_window", ctypes.c_int32),
+                ("format", ctypes.c_int32), ("pool_window", ctypes.c_int32), ("decay_mode", ctypes.c_int32),
                 ("A", ctypes.c_void_p), ("Bm", ctypes.c_void_p), ("Kf", ctypes.c_void_p), ("Wf", ctypes.c_void_p),
                 ("Uf", ctypes.c_void_p), ("df", ctypes.c_void_p), ("rk", ctypes.c_void_p),
                 ("buf_k", ctypes.c_void_p), ("buf_v", ctypes.c_void_p), ("buf_qr", ctypes.c_void_p),
@@ -114,11 +116,12 @@ def _check(status: int):
 
 
 def make_config(B, H, T, C=64, d=128, dtype="bf16", gate_mode="routed", tau=1.0, bias=0.0,
-                skip_threshold=0.0, cache_format="dense", pool_window=0) -> HlaConfig:
+                skip_threshold=0.0, cache_format="dense", pool_window=0, decay="scalar") -> HlaConfig:
     dt = {"bf16": HLA_BF16, "f32": HLA_F32, torch.bfloat16: HLA_BF16, torch.float32: HLA_F32}[dtype]
     gm = GATE_MODES[gate_mode] if isinstance(gate_mode, str) else int(gate_mode)
     cf = CACHE_FORMATS[cache_format] if isinstance(cache_format, str) else int(cache_format)
-    return HlaConfig(B, H, T, C, d, d, dt, gm, cf, tau, bias, skip_threshold, pool_window)
+    dm = DECAY_MODES[decay] if isinstance(decay, str) else int(decay)
+    return HlaConfig(B, H, T, C, d, d, dt, gm, cf, tau, bias, skip_threshold, pool_window, dm)
 
 
 def _ptr(t):

@@ -58,8 +58,9 @@ __global__ void __launch_bounds__(128) decode_main_kernel(DecodeArgs a) {
   ((Tio*)a.buf_v)[bslot] = ((const Tio*)a.v)[tok];
   ((Tio*)a.buf_qr)[bslot] = qr_in[tok];
   ((Tio*)a.buf_kr)[bslot] = kr_in[tok];
+  if (a.alpha_vec) a.buf_alpha[((long)bh * C + m) * D + tid] = a.alpha[(long)bh * D + tid];
   if (tid == 0) {
-    a.buf_alpha[(long)bh * C + m] = a.alpha[bh];
+    if (!a.alpha_vec) a.buf_alpha[(long)bh * C + m] = a.alpha[bh];
     a.buf_beta[(long)bh * C + m] = a.beta[bh];
   }
   __syncthreads();
@@ -72,7 +73,8 @@ __global__ void __launch_bounds__(128) decode_main_kernel(DecodeArgs a) {
     const float kt = ldf(bk + (long)t * D + tid);
     const float c = block_sum<D>(kt * x, red);
     const float bt = a.buf_beta[(long)bh * C + t];
-    const float at = a.buf_alpha[(long)bh * C + t];
+    // scalar decay, or this channel's decay
+    const float at = a.alpha_vec ? a.buf_alpha[((long)bh * C + t) * D + tid] : a.buf_alpha[(long)bh * C + t];
     y0 = fmaf(bt * c, ldf(bv + (long)t * D + tid), y0);
     x = at * (x - bt * c * kt);
   }
@@ -230,9 +232,14 @@ __global__ void cache_fill_kernel(DecodeArgs c, FillArgs f) {
   }
   for (int t = threadIdx.x; t < m; t += blockDim.x) {
     const long src = ((long)b * f.T + nc * f.C + t) * f.H + h;
-    c.buf_alpha[(long)bh * f.C + t] = f.alpha[src];
+    if (!c.alpha_vec) c.buf_alpha[(long)bh * f.C + t] = f.alpha[src];
     c.buf_beta[(long)bh * f.C + t] = f.beta[src];
   }
+  if (c.alpha_vec)  // channel-wise decay: alpha [B,T,H,d] into [B,H,C,d]
+    for (long idx = threadIdx.x; idx < (long)m * f.d; idx += blockDim.x) {
+      const int t = (int)(idx / f.d), ch = (int)(idx - (long)t * f.d);
+      c.buf_alpha[((long)bh * f.C + t) * f.d + ch] = f.alpha[(((long)b * f.T + nc * f.C + t) * f.H + h) * f.d + ch];
+    }
   if (h == 0 && threadIdx.x == 0) {
     c.n_chunks[b] = nc;
     c.m_partial[b] = m;
@@ -301,6 +308,12 @@ static cudaError_t launch_close(const DecodeArgs& a, cudaStream_t s) {
   t.in.ab = (long)a.H * a.C;
   t.in.ah = a.C;
   t.in.at = 1;
+  if (a.alpha_vec) {  // buf_alpha [B,H,C,d]: the alpha strides are those of beta times d
+    t.in.ab *= D;
+    t.in.ah *= D;
+    t.in.at *= D;
+    t.in.alpha_vec = 1;
+  }
   t.n_chunks = 1;
   t.A = const_cast<void*>(a.A);
   t.Bm = const_cast<void*>(a.Bm);
@@ -314,7 +327,7 @@ static cudaError_t launch_close(const DecodeArgs& a, cudaStream_t s) {
   t.close_n = a.n_chunks;
   // the transition kernel never writes past max_chunks; the pool kernel flags it.
   // Chunks longer than one 64-token WY tile close by the token rule (no workspace).
-  cudaError_t e = a.C > 64 ? launch_transitions_token(t, s) : launch_transitions(t, s);
+  cudaError_t e = (a.C > 64 || a.alpha_vec) ? launch_transitions_token(t, s) : launch_transitions(t, s);
   if (e != cudaSuccess) return e;
   decode_close_pool_kernel<D, Tio><<<a.B * a.H, D, 0, s>>>(a);
   e = cudaGetLastError();

@@ -61,8 +61,9 @@ __device__ __forceinline__ int decode_prologue(const DecodeArgs& a, int bh, int 
   ((__nv_bfloat16*)a.buf_v)[bslot] = ((const __nv_bfloat16*)a.v)[tok];
   ((__nv_bfloat16*)a.buf_qr)[bslot] = qr_in[tok];
   ((__nv_bfloat16*)a.buf_kr)[bslot] = kr_in[tok];
+  if (a.alpha_vec) a.buf_alpha[((long)bh * C + m) * kD + tid] = a.alpha[(long)bh * kD + tid];
   if (tid == 0) {
-    a.buf_alpha[(long)bh * C + m] = a.alpha[bh];
+    if (!a.alpha_vec) a.buf_alpha[(long)bh * C + m] = a.alpha[bh];
     a.buf_beta[(long)bh * C + m] = a.beta[bh];
   }
   tc::bar_sync(1, kCompute);
@@ -76,7 +77,8 @@ __device__ __forceinline__ int decode_prologue(const DecodeArgs& a, int bh, int 
     const float kt = ldf(bk + (long)t * kD + tid);
     const float c = blk_sum(kt * x, red);
     const float bt = a.buf_beta[(long)bh * C + t];
-    const float at = a.buf_alpha[(long)bh * C + t];
+    // scalar decay, or this channel's decay
+    const float at = a.alpha_vec ? a.buf_alpha[((long)bh * C + t) * kD + tid] : a.buf_alpha[(long)bh * C + t];
     y0 = fmaf(bt * c, ldf(bv + (long)t * kD + tid), y0);
     x = at * (x - bt * c * kt);
   }

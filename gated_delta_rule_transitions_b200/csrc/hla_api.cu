@@ -46,6 +46,10 @@ hla_status check_cfg(const hla_config* c, bool need_T) {
     return fail(HLA_ERR_INVALID_ARG, "gate_mode %d invalid", c->gate_mode);
   if (c->cache_format != HLA_CACHE_DENSE && c->cache_format != HLA_CACHE_FACTORED)
     return fail(HLA_ERR_INVALID_ARG, "cache_format %d invalid", c->cache_format);
+  if (c->decay_mode != HLA_DECAY_SCALAR && c->decay_mode != HLA_DECAY_CHANNEL)
+    return fail(HLA_ERR_INVALID_ARG, "decay_mode %d invalid", c->decay_mode);
+  if (c->decay_mode == HLA_DECAY_CHANNEL && c->cache_format == HLA_CACHE_FACTORED)
+    return fail(HLA_ERR_UNSUPPORTED, "a factored cache needs the scalar decay");
   if (c->pool_window != 0) {
     const int w = c->pool_window;
     if (w < 8 || w >= c->C || c->C % w != 0 || c->C / w > hla::kMaxWindows)
@@ -85,6 +89,23 @@ hla_status opt_ptr(const void* p, const char* name) {
 
 float gate_scale(int d) { return (float)(1.0 / std::sqrt((double)d)); }
 
+// Channel-wise decay (alpha with a trailing d_k axis).
+bool chan(const hla_config* c) { return c->decay_mode == HLA_DECAY_CHANNEL; }
+
+// Strides of the token-major alpha/beta view of [B,T,H] (scalar) or [B,T,H,d]
+// (channel-wise decay: alpha strides are beta's times d).
+void set_decay_view(hla::TokenView& in, const hla_config* c) {
+  in.ab = (long)c->T * c->H;
+  in.ah = 1;
+  in.at = c->H;
+  if (chan(c)) {
+    in.ab *= c->dk;
+    in.ah *= c->dk;
+    in.at *= c->dk;
+    in.alpha_vec = 1;
+  }
+}
+
 // Window representatives per chunk (0: one pool per chunk) and key pools per chunk.
 int n_windows(const hla_config* c) { return c->pool_window > 0 ? c->C / c->pool_window : 0; }
 size_t key_reps(const hla_config* c) { return c->pool_window > 0 ? (size_t)(c->C / c->pool_window) : 1; }
@@ -119,6 +140,11 @@ PrefillWs prefill_layout(const hla_config* c) {
   w.order = take(B * H * N * 4);
   w.A = take(B * H * Nc * d * d * esize(c->dtype));
   w.Bm = take(B * H * Nc * d * d * esize(c->dtype));
+  if (chan(c)) {  // token-rule transitions and read-out per chunk: no WY factors
+    w.S_in = take(B * H * N * d * d * 4);
+    w.total = off;
+    return w;
+  }
   if (C > kSub) {  // transitions of the complete sub-chunks, merged into A, Bm
     w.Asub = take(B * H * Nsub_c * d * d * esize(c->dtype));
     w.Bsub = take(B * H * Nsub_c * d * d * esize(c->dtype));
@@ -162,7 +188,7 @@ CacheLayout cache_layout(const hla_config* c, int32_t maxc) {
   L.bv = take(B * H * C * d * es);
   L.bqr = take(B * H * C * d * es);
   L.bkr = take(B * H * C * d * es);
-  L.balpha = take(B * H * C * 4);
+  L.balpha = take(B * H * C * (chan(c) ? d : 1) * 4);
   L.bbeta = take(B * H * C * 4);
   L.n = take(B * 4);
   L.m = take(B * 4);
@@ -173,7 +199,7 @@ CacheLayout cache_layout(const hla_config* c, int32_t maxc) {
 hla_status check_cache(const hla_config* c, const hla_cache* k) {
   if (k == nullptr) return fail(HLA_ERR_INVALID_ARG, "cache is NULL");
   if (k->B != c->B || k->H != c->H || k->C != c->C || k->d != c->dk || k->dtype != c->dtype ||
-      k->format != c->cache_format || k->pool_window != c->pool_window)
+      k->format != c->cache_format || k->pool_window != c->pool_window || k->decay_mode != c->decay_mode)
     return fail(HLA_ERR_INVALID_ARG, "cache was initialised for a different config");
   if (k->max_chunks <= 0) return fail(HLA_ERR_INVALID_ARG, "cache max_chunks must be positive");
   const void* ps[] = {k->rk, k->buf_k, k->buf_v, k->buf_qr, k->buf_kr, k->buf_alpha, k->buf_beta};
@@ -281,6 +307,8 @@ hla_status hla_cache_init(const hla_config* cfg, int32_t max_chunks, void* mem, 
   if (((uintptr_t)mem & 255u) != 0) return fail(HLA_ERR_INVALID_ARG, "cache memory must be 256-byte aligned");
   if (cfg->cache_format == HLA_CACHE_FACTORED && !(cfg->dtype == HLA_BF16 && cfg->dk == 128 && cfg->C == 64))
     return fail(HLA_ERR_UNSUPPORTED, "a factored cache needs bf16, d = 128 and C = 64");
+  if (cfg->cache_format == HLA_CACHE_FACTORED && chan(cfg))
+    return fail(HLA_ERR_UNSUPPORTED, "a factored cache needs the scalar decay");
   const CacheLayout L = cache_layout(cfg, max_chunks);
   if (bytes < L.total) return fail(HLA_ERR_WORKSPACE, "cache block too small: %zu < %zu", bytes, L.total);
   char* base = (char*)mem;
@@ -293,6 +321,7 @@ hla_status hla_cache_init(const hla_config* cfg, int32_t max_chunks, void* mem, 
   c.dtype = cfg->dtype;
   c.format = cfg->cache_format;
   c.pool_window = cfg->pool_window;
+  c.decay_mode = cfg->decay_mode;
   if (cfg->cache_format == HLA_CACHE_FACTORED) {
     c.Kf = base + L.Kf;
     c.Wf = base + L.Wf;
@@ -344,7 +373,8 @@ hla_status hla_cache_slice(const hla_cache* cache, int32_t b0, int32_t nb, hla_c
   v.buf_v = (char*)cache->buf_v + off * H * C * d * es;
   v.buf_qr = (char*)cache->buf_qr + off * H * C * d * es;
   v.buf_kr = (char*)cache->buf_kr + off * H * C * d * es;
-  v.buf_alpha = (float*)((char*)cache->buf_alpha + off * H * C * 4);
+  const size_t adim = cache->decay_mode == HLA_DECAY_CHANNEL ? d : 1;
+  v.buf_alpha = (float*)((char*)cache->buf_alpha + off * H * C * adim * 4);
   v.buf_beta = (float*)((char*)cache->buf_beta + off * H * C * 4);
   v.n_chunks = cache->n_chunks + off;
   v.m_partial = cache->m_partial + off;
@@ -384,11 +414,13 @@ hla_status gdn_chunk_transitions(const hla_config* cfg, const void* k, const voi
   t.dtype = cfg->dtype;
   t.in = {k, v, alpha, beta, (long)cfg->T * cfg->H * cfg->dk, cfg->dk, (long)cfg->H * cfg->dk,
           (long)cfg->T * cfg->H, 1, cfg->H};
+  set_decay_view(t.in, cfg);
   t.n_chunks = Nc;
   t.A = A_out;
   t.Bm = B_out;
   t.ab_chunk_stride = Nc;
-  if (cfg->C > kSub)  // no workspace here for sub-chunk factors: the token rule per chunk
+  // channel-wise decay, or no workspace here for sub-chunk factors: the token rule
+  if (cfg->C > kSub || chan(cfg))
     HLA_CUDA(hla::launch_transitions_token(t, (cudaStream_t)stream), "gdn_chunk_transitions (token rule) launch");
   else if (cfg->dtype == HLA_BF16 && cfg->dk == 128)
     HLA_CUDA(hla::launch_transitions_tc(t, (cudaStream_t)stream), "gdn_chunk_transitions (tensor core) launch");
@@ -564,18 +596,21 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
   HLA_CUDA(cudaEventRecord(side->join, side->s), "side stream join");
   // transitions of every 64-token sub-chunk (A/B of complete ones into the cache or
   // workspace; at C > 64 into the workspace, merged per chunk below)
-  const int s_sub = cfg->C / kSub;
-  const int Nsub = (cfg->T + kSub - 1) / kSub;
-  const int Nsub_c = cfg->T / kSub;
+  // Channel-wise decay: the token rule over whole chunks, no sub-chunks.
+  const bool chan_path = chan(cfg);
+  const int s_sub = chan_path ? 1 : cfg->C / kSub;
+  const int Nsub = chan_path ? N : (cfg->T + kSub - 1) / kSub;
+  const int Nsub_c = chan_path ? Nc : cfg->T / kSub;
   hla::TransArgs t{};
   t.B = cfg->B;
   t.H = cfg->H;
   t.T = cfg->T;
-  t.C = kSub;
+  t.C = chan_path ? cfg->C : kSub;
   t.d = cfg->dk;
   t.dtype = cfg->dtype;
   t.in = {k, v, alpha, beta, (long)cfg->T * cfg->H * cfg->dk, cfg->dk, (long)cfg->H * cfg->dk,
           (long)cfg->T * cfg->H, 1, cfg->H};
+  set_decay_view(t.in, cfg);
   t.n_chunks = Nsub;
   // a dense cache takes A/B straight from the transitions (or the merge); otherwise
   // they go to the workspace (the composition reads them) and a factored cache gets
@@ -593,12 +628,14 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
     t.Bm = ws + w.Bsub;
     t.ab_chunk_stride = Nsub_c;
   }
-  t.Wb = (float*)(ws + w.Wb);
-  t.Ub = (float*)(ws + w.Ub);
-  t.ell = (float*)(ws + w.ell);
+  t.Wb = chan_path ? nullptr : (float*)(ws + w.Wb);
+  t.Ub = chan_path ? nullptr : (float*)(ws + w.Ub);
+  t.ell = chan_path ? nullptr : (float*)(ws + w.ell);
   {
     StageScope _sc(HLA_STAGE_TRANSITIONS, s, 1);
-    if (tc_path)
+    if (chan_path)
+      HLA_CUDA(hla::launch_transitions_token(t, s), "transitions (token rule) launch");
+    else if (tc_path)
       HLA_CUDA(hla::launch_transitions_tc(t, s), "transitions (tensor core) launch");
     else
       HLA_CUDA(hla::launch_transitions(t, s), "transitions launch");
@@ -656,6 +693,23 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
     StageScope _sc(HLA_STAGE_CHAIN, s, 1);
     HLA_CUDA(hla::launch_chain_advance(ch, s), "sub-chunk advance launch");
   }
+  if (chan_path) {
+    hla::ReadoutTokenArgs rt{};
+    rt.B = cfg->B;
+    rt.H = cfg->H;
+    rt.T = cfg->T;
+    rt.C = cfg->C;
+    rt.N = N;
+    rt.d = cfg->dk;
+    rt.dtype = cfg->dtype;
+    rt.in = t.in;
+    rt.q = q;
+    rt.S_in = c.S_in;
+    rt.S_bf16 = tc_path;  // the tensor-core composition writes bf16 states
+    rt.o = o;
+    StageScope _sc(HLA_STAGE_READOUT, s, 1);
+    HLA_CUDA(hla::launch_readout_token(rt, s), "readout (token rule) launch");
+  }
   hla::ReadoutArgs r{};
   r.B = cfg->B;
   r.H = cfg->H;
@@ -671,7 +725,7 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
   r.Ub = t.Ub;
   r.ell = t.ell;
   r.o = o;
-  {
+  if (!chan_path) {
     StageScope _sc(HLA_STAGE_READOUT, s, 1);
     if (tc_path)
       HLA_CUDA(hla::launch_readout_tc(r, c.S_in, t.Wb, t.Ub, s), "readout (tensor core) launch");
@@ -687,6 +741,7 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
     dc.dtype = cfg->dtype;
     dc.max_chunks = cache_out->max_chunks;
     dc.win = n_windows(cfg);
+    dc.alpha_vec = chan_path ? 1 : 0;
     dc.rk = cache_out->rk;
     dc.buf_k = cache_out->buf_k;
     dc.buf_v = cache_out->buf_v;
@@ -749,6 +804,7 @@ hla_status hla_decode_step(const hla_config* cfg, hla_cache* cache, const void* 
   a.mode = cfg->gate_mode;
   a.max_chunks = cache->max_chunks;
   a.win = n_windows(cfg);
+  a.alpha_vec = chan(cfg) ? 1 : 0;
   a.tau = cfg->tau;
   a.c_d = gate_scale(cfg->dk);
   a.bias = cfg->bias;

@@ -35,6 +35,8 @@ struct TokenView {
   const float* beta;
   long sb, sh, st;   // k/v strides (elements)
   long ab, ah, at;   // alpha/beta strides (elements)
+  int alpha_vec;     // channel-wise decay: alpha (b, h, t, c) at b*ab + h*ah + t*at + c
+                     // and beta (b, h, t) at (b*ab + h*ah + t*at) / d
 };
 
 struct TransArgs {
@@ -109,6 +111,17 @@ struct ChainArgs {
   void* S;               // [B,H,Nsub,d,d]: float32 (CUDA-core path) or bf16 (tensor-core path)
 };
 
+// Intra-chunk read-out by the token rule (channel-wise decay): every chunk runs the
+// rule from its composed state S_in and emits o_t = S_t q_t.
+struct ReadoutTokenArgs {
+  int B, H, T, C, N, d, dtype;
+  TokenView in;            // k, v, alpha (channel-wise), beta
+  const void* q;           // [B,T,H,d], strides of in.k
+  const void* S_in;        // [B,H,N,d,d] ([v][c]); bf16 if S_bf16 else float32
+  bool S_bf16;
+  void* o;                 // [B,T,H,d]
+};
+
 struct ReadoutArgs {
   int B, H, T, C, N, d, dtype;
   const void* q;          // [B,T,H,d]
@@ -123,6 +136,7 @@ struct ReadoutArgs {
 struct DecodeArgs {
   int B, H, C, d, dtype, mode, max_chunks;
   int win;             // window pools per closed chunk (0: one pool per chunk)
+  int alpha_vec;       // channel-wise decay: alpha [B,H,d], buf_alpha [B,H,C,d]
   float tau, c_d, bias, thr;
   const void* q;   // [B,H,d]
   const void* k;
@@ -184,6 +198,7 @@ cudaError_t launch_chain_advance(const ChainArgs& a, cudaStream_t s);
 // Transitions of chunks of a.C > 64 tokens by the token rule itself (CUDA cores);
 // same close_m / close_n semantics as launch_transitions.  Writes A/B only.
 cudaError_t launch_transitions_token(const TransArgs& a, cudaStream_t s);
+cudaError_t launch_readout_token(const ReadoutTokenArgs& a, cudaStream_t s);
 cudaError_t launch_gate_support(const float* gates, int B, int H, int N, float thr, float* mass_out,
                                 float* support_out, cudaStream_t s);
 cudaError_t launch_wait_check(uint64_t limit_ns, bool complete, cudaStream_t s);

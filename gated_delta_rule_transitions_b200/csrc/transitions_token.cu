@@ -20,15 +20,22 @@ namespace hla {
 
 namespace {
 
-constexpr int kSeg = 64;
+// Tokens staged per step: 64 (keys only), 32 with channel-wise decay (keys and
+// decays), so the static shared memory stays at 32 KiB for d = 128.
+template <bool kChan>
+constexpr int seg_len() { return kChan ? 32 : 64; }
 
 // grid (chunks, H, 2 B): blockIdx.z & 1 selects the rows of A (0) or B (1).  Two
 // threads per row: thread (r, hf) keeps the row's elements 2 j + hf (interleaved, so
 // the pair reads adjacent shared-memory words) and the pair adds its dot products.
-template <int D, typename Tio>
+// kChan: channel-wise decay, the row is first scaled channel by channel,
+//   s <- s o alpha_t,  then  s <- s - (beta_t (s . k_t) - beta_t v_t[r]) k_t.
+template <int D, typename Tio, bool kChan>
 __global__ void __launch_bounds__(2 * D) transitions_token_kernel(TransArgs a) {
   constexpr int E = D / 2;
+  constexpr int kSeg = seg_len<kChan>();
   __shared__ float ks[kSeg][D];
+  __shared__ float as[kChan ? kSeg : 1][kChan ? D : 1];
   __shared__ float al[kSeg], be[kSeg];
   const int c = blockIdx.x;
   const int h = blockIdx.y;
@@ -57,23 +64,38 @@ __global__ void __launch_bounds__(2 * D) transitions_token_kernel(TransArgs a) {
     for (int idx = threadIdx.x; idx < kSeg * D; idx += 2 * D) {
       const int t = idx / D, cc = idx - t * D;
       ks[t][cc] = ldf(kin + (long)(s0 + t) * a.in.st + cc);
+      if constexpr (kChan) as[t][cc] = a.in.alpha[ab0 + (long)(s0 + t) * a.in.at + cc];
     }
     if (threadIdx.x < kSeg) {
-      al[threadIdx.x] = a.in.alpha[ab0 + (long)(s0 + threadIdx.x) * a.in.at];
-      be[threadIdx.x] = a.in.beta[ab0 + (long)(s0 + threadIdx.x) * a.in.at];
+      if constexpr (!kChan) al[threadIdx.x] = a.in.alpha[ab0 + (long)(s0 + threadIdx.x) * a.in.at];
+      // with channel-wise decay the alpha strides are those of beta times d
+      const long bdiv = kChan ? D : 1;
+      be[threadIdx.x] = a.in.beta[(ab0 + (long)(s0 + threadIdx.x) * a.in.at) / bdiv];
     }
     __syncthreads();
     for (int t = 0; t < kSeg; ++t) {
+      if constexpr (kChan) {
+#pragma unroll
+        for (int j = 0; j < E; ++j) x[j] *= as[t][2 * j + hf];
+      }
       float p[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // four partial sums for latency
 #pragma unroll
       for (int j = 0; j < E; ++j) p[j & 3] = fmaf(x[j], ks[t][2 * j + hf], p[j & 3]);
       float dot = (p[0] + p[1]) + (p[2] + p[3]);
       dot += __shfl_xor_sync(0xFFFFFFFFu, dot, 1);
-      const float at = al[t], bt = be[t];
-      float f = at * bt * dot;
-      if (rowsB) f -= bt * ldf(vin + (long)(s0 + t) * a.in.st + r);
+      const float bt = be[t];
+      if constexpr (kChan) {
+        float f = bt * dot;
+        if (rowsB) f -= bt * ldf(vin + (long)(s0 + t) * a.in.st + r);
 #pragma unroll
-      for (int j = 0; j < E; ++j) x[j] = fmaf(at, x[j], -f * ks[t][2 * j + hf]);
+        for (int j = 0; j < E; ++j) x[j] = fmaf(-f, ks[t][2 * j + hf], x[j]);
+      } else {
+        const float at = al[t];
+        float f = at * bt * dot;
+        if (rowsB) f -= bt * ldf(vin + (long)(s0 + t) * a.in.st + r);
+#pragma unroll
+        for (int j = 0; j < E; ++j) x[j] = fmaf(at, x[j], -f * ks[t][2 * j + hf]);
+      }
     }
   }
   const long bhc = (long)b * a.H + h;
@@ -86,14 +108,17 @@ __global__ void __launch_bounds__(2 * D) transitions_token_kernel(TransArgs a) {
 template <int D, typename Tio>
 cudaError_t launch_t(const TransArgs& a, int chunks, cudaStream_t s) {
   dim3 grid(chunks, a.H, 2 * a.B);
-  transitions_token_kernel<D, Tio><<<grid, 2 * D, 0, s>>>(a);
+  if (a.in.alpha_vec)
+    transitions_token_kernel<D, Tio, true><<<grid, 2 * D, 0, s>>>(a);
+  else
+    transitions_token_kernel<D, Tio, false><<<grid, 2 * D, 0, s>>>(a);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_transitions_token(const TransArgs& a, cudaStream_t s) {
-  if (a.C % kSeg != 0) return cudaErrorInvalidValue;
+  if (a.C % 64 != 0) return cudaErrorInvalidValue;
   const int chunks = a.close_m != nullptr ? 1 : a.n_chunks;
   if (chunks <= 0) return cudaSuccess;
   if (a.d == 128)

@@ -8,7 +8,8 @@ alpha, beta ``[B, T, H]`` float32.  Value distributions:
 
 * q, k ~ N(0, 1), then L2-normalised per token (unit keys keep I - beta k k^T a
   contraction); v ~ N(0, 1);
-* alpha_t = exp(-softplus(N(0,1) - 3)), beta_t = sigmoid(N(0,1));
+* alpha_t = exp(-softplus(N(0,1) - 3)), beta_t = sigmoid(N(0,1)); with channel-wise
+  decay alpha_t is a vector over the key channels, each entry drawn the same way;
 * bf16 workloads round q, k, v (and route inputs) to bf16 after normalisation
   (round to nearest even); alpha, beta stay float32.
 
@@ -52,6 +53,7 @@ class Workload:
     seed: int = 0
     topics: int = 128
     window: int = 0             # key window representatives of `window` tokens (0: one per chunk)
+    decay: str = "scalar"       # scalar (one alpha per token) | channel (one per key channel)
 
     @property
     def N(self) -> int:
@@ -85,7 +87,8 @@ def _l2n(x):
 
 def make_gdn_inputs(w: Workload, T: int | None = None, B: int | None = None, device="cpu",
                     seed: int | None = None):
-    """q, k, v [B,T,H,d] (workload dtype), alpha, beta [B,T,H] float32."""
+    """q, k, v [B,T,H,d] (workload dtype), alpha [B,T,H] (or [B,T,H,d] with channel-wise
+    decay) and beta [B,T,H] float32."""
     T = w.T if T is None else T
     B = w.B if B is None else B
     g = torch.Generator(device=device)
@@ -96,6 +99,8 @@ def make_gdn_inputs(w: Workload, T: int | None = None, B: int | None = None, dev
     v = torch.randn(shape, generator=g, device=device)
     a_raw = torch.randn((B, T, w.H), generator=g, device=device)
     b_raw = torch.randn((B, T, w.H), generator=g, device=device)
+    if w.decay == "channel":
+        a_raw = torch.randn((B, T, w.H, w.d), generator=g, device=device)
     alpha = torch.exp(-torch.nn.functional.softplus(a_raw - 3.0)).float()
     beta = torch.sigmoid(b_raw).float()
     dt = torch_dtype(w)
@@ -143,7 +148,8 @@ def make_user_gates(w: Workload, device="cpu", seed: int | None = None):
 
 
 def make_decode_tokens(w: Workload, steps: int, device="cpu", seed: int | None = None):
-    """Per-step new tokens: list of dicts with q, k, v [B,H,d], alpha, beta [B,H]."""
+    """Per-step new tokens: list of dicts with q, k, v [B,H,d], alpha [B,H] (or [B,H,d]
+    with channel-wise decay), beta [B,H]."""
     g = torch.Generator(device=device)
     g.manual_seed((w.seed if seed is None else seed) + 4242)
     dt = torch_dtype(w)
@@ -153,7 +159,8 @@ def make_decode_tokens(w: Workload, steps: int, device="cpu", seed: int | None =
         k = _l2n(torch.randn((w.B, w.H, w.d), generator=g, device=device))
         v = torch.randn((w.B, w.H, w.d), generator=g, device=device)
         a = torch.exp(-torch.nn.functional.softplus(
-            torch.randn((w.B, w.H), generator=g, device=device) - 3.0)).float()
+            torch.randn((w.B, w.H) + ((w.d,) if w.decay == "channel" else ()), generator=g, device=device)
+            - 3.0)).float()
         b = torch.sigmoid(torch.randn((w.B, w.H), generator=g, device=device)).float()
         out.append(dict(q=q.to(dt), k=k.to(dt), v=v.to(dt), alpha=a, beta=b))
     return out
@@ -172,6 +179,8 @@ def make_context_group(w: Workload, b0: int, nb: int, device="cuda"):
     v = torch.randn(shape, generator=g, device=device).to(dt)
     a_raw = torch.randn((nb, w.T, w.H), generator=g, device=device)
     b_raw = torch.randn((nb, w.T, w.H), generator=g, device=device)
+    if w.decay == "channel":
+        a_raw = torch.randn((nb, w.T, w.H, w.d), generator=g, device=device)
     alpha = torch.exp(-torch.nn.functional.softplus(a_raw - 3.0)).float()
     beta = torch.sigmoid(b_raw).float()
     return dict(q=q, k=k, v=v, alpha=alpha, beta=beta)

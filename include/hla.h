@@ -42,6 +42,7 @@
  *   - Layouts are dense row-major:
  *       q, k, v, q_route, k_route, o : [B, T, H, d]      (dtype)
  *       alpha, beta                   : [B, T, H]         float32, alpha in (0,1], beta in [0,1]
+ *                                       (alpha [B, T, H, d_k] with HLA_DECAY_CHANNEL)
  *       A_c                           : [d_k][d_k]; entry (r, c) multiplies column r
  *                                       of S into column c of S A
  *       B_c                           : [d_v][d_k]
@@ -91,6 +92,15 @@ typedef enum {
   HLA_GATES_USER = 3    /* caller-given input-independent weights [B,H,N,N] (prefill) */
 } hla_gate_mode;
 
+/* Decay of the token rule.  SCALAR: S_t = S_{t-1} alpha_t (I - beta_t k_t k_t^T) +
+ * beta_t v_t k_t^T (Gated DeltaNet).  CHANNEL: alpha_t is a vector over the d_k key
+ * channels, S_t = S_{t-1} Diag(alpha_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T (the
+ * KDA-style channel-wise decay named in the Gated DeltaNet-2 abstract on the HLA
+ * listing page); with equal channels it is the scalar rule.  In CHANNEL mode the
+ * chunk transitions and the intra-chunk read-out run the token rule row by row on
+ * CUDA cores (rows of S evolve independently); the composition is unchanged. */
+typedef enum { HLA_DECAY_SCALAR = 0, HLA_DECAY_CHANNEL = 1 } hla_decay_mode;
+
 /* Storage of the closed chunks' transitions in a decode cache. */
 typedef enum {
   HLA_CACHE_DENSE = 0,    /* A_j, B_j as d x d matrices (2 d^2 elements per chunk)        */
@@ -120,6 +130,8 @@ typedef struct hla_config {
                              g_ij = sigmoid(log sum_u exp(<r^q_i, r^k_ju> / sqrt(d)) + b)
                              ("Methodology in Plain English" para. 2; "Main
                              Findings": window 32 by default)                   */
+  int32_t decay_mode;     /* hla_decay_mode; CHANNEL takes alpha with a trailing
+                             d_k axis and no factored cache                    */
 } hla_config;
 
 /*
@@ -133,7 +145,7 @@ typedef struct hla_config {
  *   rk           [B, H, max_chunks, W, d]  float32 -- key pools of closed chunks (W = 1,
  *                or C / pool_window window pools)
  *   buf_k, buf_v, buf_qr, buf_kr  [B, H, C, d] dtype -- tokens of the open chunk
- *   buf_alpha, buf_beta           [B, H, C]  float32
+ *   buf_alpha, buf_beta           [B, H, C]  float32 (buf_alpha [B, H, C, d] if CHANNEL)
  *   n_chunks     [B] int32 -- closed chunks per sequence
  *   m_partial    [B] int32 -- tokens in the open chunk (0 .. C-1 between calls)
  * The cache is the resumable decode state ("Main Findings": per-chunk affine
@@ -144,6 +156,7 @@ typedef struct hla_cache {
   int32_t B, H, C, d, dtype;
   int32_t format; /* hla_cache_format */
   int32_t pool_window; /* key representatives per closed chunk: 1, or C / pool_window */
+  int32_t decay_mode;  /* hla_decay_mode (buf_alpha holds d_k values per token if CHANNEL) */
   void* A;
   void* Bm;
   void* Kf;
@@ -259,7 +272,8 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
 /*
  * hla_decode_step -- one new token per sequence (Key Contributions 3: dynamic
  * autoregressive decoding; Methodology para. 4: skipped chunks are not read).
- * In:  q, k, v [B,H,d] dtype; alpha, beta [B,H] float32; q_route, k_route [B,H,d]
+ * In:  q, k, v [B,H,d] dtype; alpha, beta [B,H] float32 (alpha [B,H,d] with channel-wise
+ *      decay); q_route, k_route [B,H,d]
  *      or NULL (q, k).  cache: initialised (by hla_prefill or empty).
  * Out: o [B,H,d] dtype.  The token is appended to the open chunk; the query pool
  *      runs over the open chunk's m tokens so far; gates against every closed

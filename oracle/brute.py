@@ -3,7 +3,8 @@
 TEST INFRASTRUCTURE ONLY (same import rule as the rest of ``oracle/``).
 
 Every per-token map is written out as an explicit matrix,
-  M_t = alpha_t (I - beta_t k_t k_t^T)   (d_k x d_k)
+  M_t = alpha_t (I - beta_t k_t k_t^T)   (d_k x d_k; Diag(alpha_t)(...) for a
+                                          channel-wise decay)
   N_t = beta_t v_t k_t^T                  (d_v x d_k)
 so that the token rule is S_t = S_{t-1} M_t + N_t (HLA summary page, "Methodology in
 Plain English": a matrix that decays and edits the old state plus an additive
@@ -60,12 +61,15 @@ def _mv(a, x, z):
 
 
 def token_matrices(k, v, alpha, beta, z, one):
-    """Per-token (M_t, N_t) as explicit nested lists."""
+    """Per-token (M_t, N_t) as explicit nested lists.  ``alpha`` is one number, or a
+    list over the key channels (channel-wise decay: M_t = Diag(alpha)(I - beta k k^T),
+    row r scaled by alpha[r])."""
     dk = len(k)
     M = _eye(dk, z, one)
     for r in range(dk):
+        a_r = alpha[r] if isinstance(alpha, (list, tuple)) else alpha
         for c in range(dk):
-            M[r][c] = alpha * (M[r][c] - beta * k[r] * k[c])
+            M[r][c] = a_r * (M[r][c] - beta * k[r] * k[c])
     N = [[beta * v[r] * k[c] for c in range(dk)] for r in range(len(v))]
     return M, N
 

@@ -58,15 +58,29 @@ GATES_USER = "user"
 # ----------------------------------------------------------------------------------
 
 def gdn_token_step(S, k, v, alpha, beta):
-    """One token of the gated delta rule: S alpha (I - beta k k^T) + beta v k^T."""
-    Sk = S @ k
-    return alpha * (S - beta * np.outer(Sk, k)) + beta * np.outer(v, k)
+    """One token of the gated delta rule: S Diag(alpha) (I - beta k k^T) + beta v k^T.
+
+    ``alpha`` is a scalar (Gated DeltaNet: S alpha (I - beta k k^T) + beta v k^T) or a
+    vector over the d_k key channels (channel-wise decay, the KDA-style decay named in
+    the Gated DeltaNet-2 abstract on the HLA listing page: the state's key channels
+    decay each at its own rate before the delta-rule edit)."""
+    if np.ndim(alpha) == 0:
+        Sk = S @ k
+        return alpha * (S - beta * np.outer(Sk, k)) + beta * np.outer(v, k)
+    Sa = S * np.asarray(alpha, np.float64)[None, :]
+    return Sa - beta * np.outer(Sa @ k, k) + beta * np.outer(v, k)
+
+
+def _alpha_of(a):
+    """A buffered decay as float (scalar) or float64 vector (channel-wise)."""
+    return float(a) if np.ndim(a) == 0 else np.asarray(a, np.float64)
 
 
 def gdn_recurrent(q, k, v, alpha, beta, S0=None):
     """Plain token-by-token gated delta rule for one head.
 
-    q, k: [T, d_k]; v: [T, d_v]; alpha, beta: [T].  Returns (o [T, d_v], S_T)."""
+    q, k: [T, d_k]; v: [T, d_v]; alpha: [T] or [T, d_k] (channel-wise); beta: [T].
+    Returns (o [T, d_v], S_T)."""
     q = np.asarray(q, np.float64)
     k = np.asarray(k, np.float64)
     v = np.asarray(v, np.float64)
@@ -392,7 +406,7 @@ class HlaDecodeHead:
             S = S + float(g[j]) * ((S @ A + B) - S)
         for (_q, _k, _v, _a, _b, _qr, _kr) in self.buf:
             S = gdn_token_step(S, np.asarray(_k, np.float64), np.asarray(_v, np.float64),
-                               float(_a), float(_b))
+                               _alpha_of(_a), float(_b))
         o = S @ np.asarray(q, np.float64)
         if len(self.buf) == self.C:
             self.close_chunk()
@@ -401,7 +415,7 @@ class HlaDecodeHead:
     def close_chunk(self):
         ks = np.stack([np.asarray(b[1], np.float64) for b in self.buf])
         vs = np.stack([np.asarray(b[2], np.float64) for b in self.buf])
-        al = np.array([float(b[3]) for b in self.buf])
+        al = np.array([_alpha_of(b[3]) for b in self.buf])
         be = np.array([float(b[4]) for b in self.buf])
         krs = np.stack([np.asarray(b[6], np.float32) for b in self.buf])
         self.trans.append(chunk_transition(ks, vs, al, be))

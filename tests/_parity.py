@@ -41,7 +41,7 @@ def run_prefill(hla, w: syn.Workload, inp, user_gates=None, cache=None, cache_fo
     B, T, H, d = inp["q"].shape
     N = (T + w.C - 1) // w.C
     cfg = hla.make_config(B, H, T, w.C, d, w.dtype, w.gate_mode, w.tau, w.bias, w.thr, cache_format=cache_format,
-                          pool_window=w.window)
+                          pool_window=w.window, decay=w.decay)
     g = to_cuda(inp)
     o = torch.empty_like(g["q"])
     gates = torch.empty((B, H, N, N), dtype=torch.float32, device="cuda")

@@ -275,3 +275,17 @@ def test_window_pools_enlarge_the_key_cache(hla):
     win = cfg(hla, T=1, C=256, pool_window=32)
     per_chunk = lambda c: hla.cache_bytes(c, 101) - hla.cache_bytes(c, 100)
     assert per_chunk(win) - per_chunk(base) == 7 * d * 4   # 8 window pools instead of one
+
+
+def test_decay_mode_checks(hla):
+    assert hla.prefill_workspace_bytes(cfg(hla, T=1024, decay="channel")) > 0
+    assert hla.prefill_workspace_bytes(cfg(hla, T=1024, decay=2)) == 0
+    # channel-wise decay keeps d decays per buffered token in the decode cache
+    d = 128
+    c1 = cfg(hla, T=1, C=64)
+    c2 = cfg(hla, T=1, C=64, decay="channel")
+    assert hla.cache_bytes(c2, 8) - hla.cache_bytes(c1, 8) >= 64 * (d - 1) * 4
+    out = hla.HlaCache()
+    c3 = cfg(hla, B=1, H=1, T=1, decay="channel", cache_format="factored")
+    st = hla.lib().hla_cache_init(ctypes.byref(c3), 4, ctypes.c_void_p(1 << 20), 1 << 30, ctypes.byref(out), None)
+    assert st == hla.HLA_ERR_UNSUPPORTED and "scalar decay" in hla.last_error()

@@ -1,0 +1,133 @@
+"""GPU parity with channel-wise decay (a decay per key channel, the KDA-style decay
+named in the Gated DeltaNet-2 abstract on the HLA listing page):
+  S_t = S_{t-1} Diag(alpha_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T.
+
+Transitions and the intra-chunk read-out run the token rule row by row on CUDA cores;
+the composition and the gates are those of the scalar path.  Bars as elsewhere:
+gates and lists bit-exact, outputs max-abs 1e-4 (float32) or relative L2 2e-2 (bf16)."""
+import numpy as np
+import pytest
+import torch
+
+import hla_synth as syn
+from oracle import hla_oracle as ho
+from tests import _parity as P
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def hla():
+    import gated_delta_rule_transitions_b200 as m
+    m.lib()
+    return m._hla
+
+
+def _check_prefill(hla, w):
+    inp = P.gpu_inputs(w)
+    assert inp["alpha"].dim() == 4
+    o, gates, aidx, acnt = P.run_prefill(hla, w, inp)
+    B, T, H, _ = inp["q"].shape
+    ref = np.zeros(tuple(inp["v"].shape))
+    for b in range(B):
+        for h in range(H):
+            r = P.oracle_prefill_head(w, inp, b, h)
+            ref[b, :, h] = r.o
+            P.check_routing_exact(r, gates, aidx, acnt, b, h)
+    got = P.np64(o)
+    if w.dtype == "f32":
+        assert np.abs(got - ref).max() <= P.TOL_F32_MAXABS
+    else:
+        assert P.rel_l2(got, ref) <= P.TOL_BF16_RELL2
+    st, code = hla.hla_device_status()
+    assert st == 0 and code == 0
+
+
+@pytest.mark.parametrize("C,T,thr", [(64, 64 * 6 + 21, 0.0), (256, 256 * 3 + 100, 0.3), (128, 128 * 4, 0.0)])
+def test_bf16_channel_decay_prefill(hla, C, T, thr):
+    _check_prefill(hla, syn.PREFILL_0P8B.with_(B=2, H=2, T=T, C=C, thr=thr, decay="channel"))
+
+
+def test_f32_channel_decay_prefill_planted(hla):
+    w = syn.SPARSE_LONG.with_(B=1, H=2, T=64 * 12 + 7, dtype="f32", d=64, topics=3, decay="channel")
+    _check_prefill(hla, w)
+
+
+@pytest.mark.parametrize("dtype,d", [("f32", 64), ("bf16", 128)])
+def test_channel_decay_gates_one_is_the_token_rule(hla, dtype, d):
+    w = syn.GDN_REDUCTION.with_(B=2, H=2, T=64 * 4 + 9, dtype=dtype, d=d, decay="channel")
+    inp = P.gpu_inputs(w)
+    o, *_ = P.run_prefill(hla, w, inp)
+    for b in range(2):
+        for h in range(2):
+            ref, _ = ho.gdn_recurrent(P.np64(inp["q"][b, :, h]), P.np64(inp["k"][b, :, h]),
+                                      P.np64(inp["v"][b, :, h]), P.np64(inp["alpha"][b, :, h]),
+                                      P.np64(inp["beta"][b, :, h]))
+            got = P.np64(o[b, :, h])
+            if dtype == "f32":
+                assert np.abs(got - ref).max() <= P.TOL_F32_MAXABS
+            else:
+                assert P.rel_l2(got, ref) <= P.TOL_BF16_RELL2
+
+
+def test_channel_decay_transitions(hla):
+    w = syn.TINY_F32.with_(B=1, H=2, T=64 * 3 + 5, decay="channel")
+    inp = P.gpu_inputs(w)
+    B, H, T, d = 1, 2, w.T, w.d
+    cfg = hla.make_config(B, H, T, 64, d, "f32", decay="channel")
+    g = P.to_cuda(inp)
+    A = torch.empty((B, H, T // 64, d, d), dtype=torch.float32, device="cuda")
+    Bm = torch.empty_like(A)
+    hla.gdn_chunk_transitions(cfg, g["k"], g["v"], g["alpha"], g["beta"], A, Bm)
+    torch.cuda.synchronize()
+    A, Bm = P.np64(A), P.np64(Bm)
+    for h in range(H):
+        for c in range(T // 64):
+            sl = slice(64 * c, 64 * c + 64)
+            Ar, Br = ho.chunk_transition(P.np64(inp["k"][0, sl, h]), P.np64(inp["v"][0, sl, h]),
+                                         P.np64(inp["alpha"][0, sl, h]), P.np64(inp["beta"][0, sl, h]))
+            assert np.abs(A[0, h, c] - Ar).max() <= P.TOL_F32_MAXABS
+            assert np.abs(Bm[0, h, c] - Br).max() <= P.TOL_F32_MAXABS
+
+
+@pytest.mark.parametrize("dtype,d,C,T0,steps", [
+    ("f32", 64, 64, 64 * 3 + 60, 7),      # CUDA-core decode, closes a chunk at step 4
+    ("bf16", 128, 64, 64 * 2 + 62, 5),    # TMA-streamed decode, closes at step 2
+    ("bf16", 128, 128, 128 + 126, 4),     # 128-token chunks
+])
+def test_channel_decay_decode(hla, dtype, d, C, T0, steps):
+    w = syn.DECODE_32K.with_(B=2, H=2, T=T0, C=C, dtype=dtype, d=d, thr=0.05, decay="channel")
+    inp = P.gpu_inputs(w)
+    maxc = T0 // C + 2
+    cfg = hla.make_config(w.B, w.H, T0, C, d, dtype, "routed", w.tau, w.bias, w.thr, decay="channel")
+    cache = hla.Cache(cfg, max_chunks=maxc)
+    P.run_prefill(hla, w, inp, cache=cache)
+    heads = {}
+    for b in range(w.B):
+        for h in range(w.H):
+            f = lambda n: inp[n][b, :, h]
+            heads[(b, h)] = ho.HlaDecodeHead.from_prefill(
+                P.np64(f("q")), P.np64(f("k")), P.np64(f("v")), P.np64(f("alpha")), P.np64(f("beta")), C,
+                w.tau, w.bias, w.thr)
+    dcfg = hla.make_config(w.B, w.H, 1, C, d, dtype, "routed", w.tau, w.bias, w.thr, decay="channel")
+    got, ref = [], []
+    for tk in syn.make_decode_tokens(w, steps):
+        assert tk["alpha"].shape == (w.B, w.H, d)
+        gt = {k: v.cuda().contiguous() for k, v in tk.items()}
+        o = torch.empty_like(gt["q"])
+        hla.hla_decode_step(dcfg, cache, gt["q"], gt["k"], gt["v"], gt["alpha"], gt["beta"], o)
+        torch.cuda.synchronize()
+        o = P.np64(o)
+        for (b, h), st in heads.items():
+            ref.append(st.step(P.np64(tk["q"][b, h]), P.np64(tk["k"][b, h]), P.np64(tk["v"][b, h]),
+                               P.np64(tk["alpha"][b, h]), float(tk["beta"][b, h])))
+            got.append(o[b, h])
+    got, ref = np.stack(got), np.stack(ref)
+    if dtype == "f32":
+        assert np.abs(got - ref).max() <= P.TOL_F32_MAXABS
+    else:
+        assert P.rel_l2(got, ref) <= P.TOL_BF16_RELL2
+    st, code = hla.hla_device_status()
+    assert st == 0 and code == 0
+    n = cache.view("n_chunks", (w.B,), torch.int32).cpu()
+    assert n.tolist() == [(T0 + steps) // C] * w.B

@@ -323,3 +323,59 @@ def test_support_lies_between_one_and_the_kept_count():
             assert sup[i] == 0.0
         else:
             assert 1.0 - 1e-12 <= sup[i] <= n + 1e-12
+
+
+# ---- channel-wise decay (KDA-style: S Diag(alpha_t)(I - beta k k^T) + beta v k^T) -----
+
+def _channel_alpha(rng, T, d):
+    return np.exp(-np.log1p(np.exp(rng.standard_normal((T, d)) - 3.0)))
+
+
+@pytest.mark.parametrize("T,C,d", [(8, 2, 2), (7, 4, 3)])
+def test_channel_decay_exact_rational_brute_force(T, C, d):
+    rng = np.random.default_rng(300 + T * C * d)
+    q, k, v, _, b = _head(rng, T, d)
+    a = _channel_alpha(rng, T, d)
+    N = (T + C - 1) // C
+    ug = np.tril(rng.uniform(0, 1, (N, N)), -1).astype(np.float32)
+    r = ho.hla_prefill_head(q, k, v, a, b, C, gate_mode=ho.GATES_USER, user_gates=ug)
+    F = lambda M: [[_frac(x) for x in row] for row in np.atleast_2d(M)]
+    ob = brute.hla_brute(F(q), F(k), F(v), F(a), [_frac(x) for x in b], C,
+                         [[_frac(x) for x in row] for row in ug], zero=Fraction(0), one=Fraction(1))
+    exact = np.array([[float(x) for x in row] for row in ob])
+    assert np.abs(r.o - exact).max() <= 1e-13
+
+
+def test_channel_decay_with_equal_channels_is_scalar_decay():
+    rng = np.random.default_rng(301)
+    q, k, v, a, b = _head(rng, 40, 6)
+    r1 = ho.hla_prefill_head(q, k, v, a, b, 8, bias=-1.0, thr=0.3)
+    r2 = ho.hla_prefill_head(q, k, v, np.repeat(a[:, None], 6, axis=1), b, 8, bias=-1.0, thr=0.3)
+    assert np.abs(r1.o - r2.o).max() <= 1e-12
+
+
+def test_channel_decay_without_edits_is_diagonal():
+    # beta = 0: no edit, so A_c = Diag(prod_t alpha_t) and B_c = 0
+    rng = np.random.default_rng(302)
+    _, k, v, _, _ = _head(rng, 9, 5)
+    a = _channel_alpha(rng, 9, 5)
+    A, B = ho.chunk_transition(k, v, a, np.zeros(9))
+    assert np.abs(A - np.diag(np.prod(a, axis=0))).max() <= 1e-15
+    assert np.abs(B).max() == 0.0
+
+
+def test_channel_decay_decode_matches_prefill():
+    rng = np.random.default_rng(303)
+    C, d, T0 = 8, 5, 13
+    q, k, v, _, b = _head(rng, T0, d)
+    a = _channel_alpha(rng, T0, d)
+    st = ho.HlaDecodeHead.from_prefill(q, k, v, a, b, C, bias=-0.5, thr=0.2)
+    for _ in range(6):   # closes chunk 1 at the third step
+        tq, tk, tv, _, tb = _head(rng, 1, d)
+        ta = _channel_alpha(rng, 1, d)
+        o = st.step(tq[0], tk[0], tv[0], ta[0], tb[0])
+        q = np.vstack([q, tq]); k = np.vstack([k, tk]); v = np.vstack([v, tv])
+        a = np.vstack([a, ta]); b = np.append(b, tb)
+        ref = ho.hla_prefill_head(q, k, v, a, b, C, bias=-0.5, thr=0.2, query_chunks=[(len(b) - 1) // C])
+        assert np.abs(o - ref.o[-1]).max() <= 1e-12
+    assert len(st.trans) == 2
