@@ -131,3 +131,18 @@ def test_channel_decay_decode(hla, dtype, d, C, T0, steps):
     assert st == 0 and code == 0
     n = cache.view("n_chunks", (w.B,), torch.int32).cpu()
     assert n.tolist() == [(T0 + steps) // C] * w.B
+
+
+def test_full_size_channel_decay_sampled(hla):
+    """Dense 0.8B-like layer at full size (T=16384, H=16, d=128, bf16) with a decay
+    per key channel: gates bit-exact on two heads, sampled query chunks against the
+    oracle."""
+    w = syn.PREFILL_0P8B.with_(decay="channel")
+    inp = P.gpu_inputs(w)
+    o, gates, aidx, acnt = P.run_prefill(hla, w, inp)
+    for h in (0, 9):
+        sample = [0, 1, 37, 128, 255]
+        r = P.oracle_prefill_head(w, inp, 0, h, query_chunks=sample)
+        P.check_routing_exact(r, gates, aidx, acnt, 0, h)
+        rows = np.concatenate([np.arange(64 * i, 64 * i + 64) for i in sample])
+        assert P.rel_l2(P.np64(o[0, rows, h]), r.o[rows]) <= P.TOL_BF16_RELL2

@@ -159,3 +159,18 @@ def test_decode_long_chunks(hla, dtype, d, C, T0, steps):
     for (b, h), st_ in heads.items():
         for j in range(len(st_.rk)):
             assert np.array_equal(rk[b, h, j].view(np.uint32), st_.rk[j].view(np.uint32))
+
+
+def test_full_size_c256_window32_sampled(hla):
+    """The pages' defaults at the dense 0.8B-like layer's full size (T=16384, H=16,
+    d=128, bf16, 256-token chunks, window-32 representatives): all gates and active
+    lists bit-exact on two heads; sampled query chunks against the oracle."""
+    w = syn.PREFILL_0P8B.with_(C=256, window=32)
+    inp = P.gpu_inputs(w)
+    o, gates, aidx, acnt = P.run_prefill(hla, w, inp)
+    for h in (0, 9):
+        sample = [0, 1, 17, 40, 63]
+        r = P.oracle_prefill_head(w, inp, 0, h, query_chunks=sample)
+        P.check_routing_exact(r, gates, aidx, acnt, 0, h)
+        rows = np.concatenate([np.arange(256 * i, 256 * i + 256) for i in sample])
+        assert P.rel_l2(P.np64(o[0, rows, h]), r.o[rows]) <= P.TOL_BF16_RELL2
