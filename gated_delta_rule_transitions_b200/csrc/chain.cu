@@ -77,155 +77,216 @@ __device__ __forceinline__ bool chain_job(const ChainArgs& a, long blk, int d, C
   return true;
 }
 
+// Tensor-core chains, persistent and pipelined.  One CTA per SM walks the jobs
+// blockIdx.x, blockIdx.x + gridDim.x, ... with three roles:
+//   warp 0       TMA producer: per job the starting matrix X0, then per step the
+//                right factor A_k and (B-chains, advance) B_k, into a 3-stage ring of
+//                64 KiB items that runs ahead across job boundaries;
+//   warp 1       TMEM allocation and the MMA issuer (one lane): step 0 multiplies X0
+//                straight from shared memory (SS form), later steps take the running
+//                product from tensor memory (TS form), D = X A_k into TMEM;
+//   warps 2-5    epilogue, one row v per thread: D + B_k (B_k rows read from the
+//                ring), rounded to bf16, written back as the next operand and, where
+//                the chain emits, to global memory.
+// Barriers: full/empty per stage (empty: the MMA's commit and the four epilogue
+// warps), mma_done per step, op_ready per step (the operand is written and D has
+// been read).  The epilogue releases a stage only after it has seen the step's
+// mma_done, so every commit of an earlier use of that stage has arrived before.
+// All waits are bounded.
+constexpr int kPStages = 3;
+constexpr int kPStage = 2 * kTile;  // X0 or A_k, then B_k: 64 KiB
+constexpr int kPThreads = 192;
+
 template <bool kAdvance>
-__global__ void __launch_bounds__(128) chain_tc_kernel(const __grid_constant__ CUtensorMap tmA, ChainArgs a) {
+__global__ void __launch_bounds__(kPThreads, 1)
+    chain_pipe_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                      const __grid_constant__ CUtensorMap tmX, ChainArgs a, long njobs) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint64_t* tma_bar = (uint64_t*)(sm + kMaxSteps * kTile);  // [kMaxSteps]
-  uint64_t* mma_bar = tma_bar + kMaxSteps;
-  uint64_t* fin_bar = mma_bar + 1;
+  uint8_t* ring = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint64_t* full = (uint64_t*)(ring + kPStages * kPStage);
+  uint64_t* empty = full + kPStages;
+  uint64_t* mma_done = empty + kPStages;
+  uint64_t* op_ready = mma_done + 1;
+  uint64_t* fin_bar = op_ready + 1;
   uint32_t* tmem_s = (uint32_t*)(fin_bar + 1);
   volatile int* abort_s = (volatile int*)(tmem_s + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  ChainJob jb;
-  if (!chain_job<kAdvance>(a, blockIdx.x, kD, jb)) return;  // uniform over the CTA
-  const __nv_bfloat16* xsrc = kAdvance ? (const __nv_bfloat16*)a.S
-                                       : (const __nv_bfloat16*)(jb.x_is_B ? a.Bsub : a.Asub);
-  __nv_bfloat16* odst = kAdvance ? (__nv_bfloat16*)a.S : (__nv_bfloat16*)(jb.x_is_B ? a.Bout : a.Aout);
-  const __nv_bfloat16* bsub = (const __nv_bfloat16*)a.Bsub;
-
-  const int tid = threadIdx.x;
-  const int warp = tid >> 5;
-  if (tid == 0) {
-    for (int k = 0; k < kMaxSteps; ++k) tc::mbar_init(&tma_bar[k], 1);
-    tc::mbar_init(mma_bar, 1);
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < kPStages; ++st) {
+      tc::mbar_init(&full[st], 1);
+      tc::mbar_init(&empty[st], 1 + 4);
+    }
+    tc::mbar_init(mma_done, 1);
+    tc::mbar_init(op_ready, 4);
     tc::mbar_init(fin_bar, 1);
     *abort_s = 0;
     tc::mbar_fence_init();
     tc::fence_async_smem();
   }
-  if (warp == 0) tc::tmem_alloc(tmem_s, 256);
+  if (warp == 1) tc::tmem_alloc(tmem_s, 256);
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
-  const uint32_t tm = *tmem_s;  // columns 0-127: D (float32); 128-191: X (bf16 pairs)
+  const uint32_t tm = *tmem_s;  // columns 0-127: D (float32); 128-191: operand (bf16 pairs)
 
-  if (tid == 0) {
-    tc::tma_prefetch_desc(&tmA);
-    for (int k = 0; k < jb.nsteps; ++k) {
-      tc::mbar_arrive_expect_tx(&tma_bar[k], kTile);
-      const int row = (int)((jb.sub0 + k) * kD);
-      tc::tma_load_2d(sm + k * kTile, &tmA, 0, row, &tma_bar[k]);
-      tc::tma_load_2d(sm + k * kTile + kHalf, &tmA, 64, row, &tma_bar[k]);
-    }
-  }
-  // X0 row v -> the operand columns (32 bf16 columns = 16 TMEM columns per store)
-  const int v = tid;
-  const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
-  // (the tcgen05 instructions order memory accesses around them, so every global
-  // load of a row is issued before the first of them)
-  {
-    const uint4* src = (const uint4*)(xsrc + jb.x0 + (long)v * kD);
-    uint4 xq[16];
-#pragma unroll
-    for (int e = 0; e < 16; ++e) xq[e] = src[e];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      uint32_t w[16];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        w[4 * e + 0] = xq[4 * c + e].x;
-        w[4 * e + 1] = xq[4 * c + e].y;
-        w[4 * e + 2] = xq[4 * c + e].z;
-        w[4 * e + 3] = xq[4 * c + e].w;
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      tc::tma_prefetch_desc(&tmA);
+      tc::tma_prefetch_desc(&tmB);
+      tc::tma_prefetch_desc(&tmX);
+      long s = 0;
+      bool ok = true;
+      for (long blk = blockIdx.x; blk < njobs && ok; blk += gridDim.x) {
+        ChainJob jb;
+        if (!chain_job<kAdvance>(a, blk, kD, jb)) continue;
+        const CUtensorMap* xmap = kAdvance ? &tmX : (jb.x_is_B ? &tmB : &tmA);
+        for (int item = 0; item <= jb.nsteps; ++item, ++s) {
+          const int st = (int)(s % kPStages);
+          if (s >= kPStages && !tc::mbar_wait(&empty[st], (uint32_t)((s / kPStages) - 1) & 1, abort_s)) {
+            ok = false;
+            break;
+          }
+          uint8_t* dst = ring + st * kPStage;
+          if (item == 0) {
+            const int row = (int)(jb.x0 / kD);  // X0 starts at row (matrix index) x 128
+            tc::mbar_arrive_expect_tx(&full[st], kTile);
+            tc::tma_load_2d(dst, xmap, 0, row, &full[st]);
+            tc::tma_load_2d(dst + kHalf, xmap, 64, row, &full[st]);
+          } else {
+            const int row = (int)((jb.sub0 + item - 1) * kD);
+            tc::mbar_arrive_expect_tx(&full[st], jb.addB ? 2 * kTile : kTile);
+            tc::tma_load_2d(dst, &tmA, 0, row, &full[st]);
+            tc::tma_load_2d(dst + kHalf, &tmA, 64, row, &full[st]);
+            if (jb.addB) {
+              tc::tma_load_2d(dst + kTile, &tmB, 0, row, &full[st]);
+              tc::tma_load_2d(dst + kTile + kHalf, &tmB, 64, row, &full[st]);
+            }
+          }
+        }
       }
-      tc::tmem_st16(tm + lane_off + 128u + 16u * c, w);
+      if (*abort_s)  // never leave the CTA with copies in flight
+        for (long t = s - kPStages > 0 ? s - kPStages : 0; t < s; ++t)
+          tc::mbar_wait(&full[t % kPStages], (uint32_t)(t / kPStages) & 1, nullptr, 200000000ull);
     }
-    tc::tmem_wait_st();
-  }
-  // row v of B for the next step, loaded while the product runs
-  uint4 bq[16];
-  const __nv_bfloat16* brow0 = bsub + jb.sub0 * kD * kD + (long)v * kD;
-  if (jb.addB) {
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      long s = 0, step = 0;
+      bool ok = true;
+      for (long blk = blockIdx.x; blk < njobs && ok; blk += gridDim.x) {
+        ChainJob jb;
+        if (!chain_job<kAdvance>(a, blk, kD, jb)) continue;
+        const int xs = (int)(s % kPStages);
+        if (!tc::mbar_wait(&full[xs], (uint32_t)(s / kPStages) & 1, abort_s)) break;
+        ++s;
+        for (int k = 0; k < jb.nsteps; ++k, ++s, ++step) {
+          const int st = (int)(s % kPStages);
+          if (!tc::mbar_wait(&full[st], (uint32_t)(s / kPStages) & 1, abort_s) ||
+              (step > 0 && !tc::mbar_wait(op_ready, (uint32_t)(step - 1) & 1, abort_s))) {
+            ok = false;
+            break;
+          }
+          tc::tc_fence_after();
+          const uint32_t b_base = tc::smem_u32(ring + st * kPStage);
+          if (k == 0) {
+            const uint32_t a_base = tc::smem_u32(ring + xs * kPStage);
 #pragma unroll
-    for (int e = 0; e < 16; ++e) bq[e] = ((const uint4*)brow0)[e];
+            for (int ks = 0; ks < kD / 16; ++ks) {
+              const uint64_t ad = tc::sdesc_sw128(a_base + (ks >> 2) * kHalf + (ks & 3) * 32, 16, 1024);
+              const uint64_t bd = tc::sdesc_sw128(b_base + ks * 2048, kHalf, 1024);
+              tc::mma_ss(tm, ad, bd, kIdesc, ks > 0 ? 1u : 0u);
+            }
+          } else {
+#pragma unroll
+            for (int ks = 0; ks < kD / 16; ++ks) {
+              const uint64_t bd = tc::sdesc_sw128(b_base + ks * 2048, kHalf, 1024);
+              tc::mma_ts(tm, tm + 128u + 8u * ks, bd, kIdesc, ks > 0 ? 1u : 0u);
+            }
+          }
+          tc::mma_commit(mma_done);
+          if (k == 0) tc::mma_commit(&empty[xs]);
+          tc::mma_commit(&empty[st]);
+        }
+      }
+      // every MMA issued by this thread completes before tensor memory is freed
+      tc::mma_commit(fin_bar);
+      tc::mbar_wait(fin_bar, 0, nullptr, 200000000ull);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue: warps 2-5, one row per thread ----------------
+    const int q = warp & 3;  // TMEM lane quarter of this warp
+    const int v = 32 * q + lane;
+    const uint32_t lane_off = (uint32_t)(32 * q) << 16;
+    const __nv_bfloat16* sbase = kAdvance ? (const __nv_bfloat16*)a.S : nullptr;
+    (void)sbase;
+    long s = 0, step = 0;
+    bool ok = true;
+    for (long blk = blockIdx.x; blk < njobs && ok; blk += gridDim.x) {
+      ChainJob jb;
+      if (!chain_job<kAdvance>(a, blk, kD, jb)) continue;
+      __nv_bfloat16* odst = kAdvance ? (__nv_bfloat16*)a.S : (__nv_bfloat16*)(jb.x_is_B ? a.Bout : a.Aout);
+      const int xs = (int)(s % kPStages);
+      ++s;
+      for (int k = 0; k < jb.nsteps; ++k, ++s, ++step) {
+        const int st = (int)(s % kPStages);
+        ok = tc::bar_all(1, 128, tc::mbar_wait(mma_done, (uint32_t)step & 1, abort_s) &&
+                                     tc::mbar_wait(&full[st], (uint32_t)(s / kPStages) & 1, abort_s));
+        if (!ok) break;
+        tc::tc_fence_after();
+        if (k == 0 && lane == 0) tc::mbar_arrive(&empty[xs]);  // X0 has been multiplied
+        const bool last = k + 1 == jb.nsteps;
+        const bool emit = kAdvance || last;
+        uint4* orow = emit ? (uint4*)(odst + jb.out0 + (kAdvance ? (long)k * kD * kD : 0) + (long)v * kD) : nullptr;
+        const uint8_t* bst = ring + st * kPStage + kTile;  // B_k of this step (two 64-column boxes)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t dr[32];
+          tc::tmem_ld32(tm + lane_off + 32u * c, dr);
+          tc::tmem_wait_ld();
+          uint32_t w[16];
+          if (jb.addB) {
+            const uint8_t* brow = bst + (c >> 1) * kHalf + v * 128;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int c8 = (c & 1) * 4 + e;
+              const uint4 bq = *(const uint4*)(brow + ((c8 ^ (v & 7)) << 4));
+              const uint32_t bw[4] = {bq.x, bq.y, bq.z, bq.w};
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const float2 bb = tc::bf16x2_to_float2(bw[u]);
+                const int i = 4 * e + u;
+                w[i] = tc::pack_bf16x2(__uint_as_float(dr[2 * i]) + bb.x, __uint_as_float(dr[2 * i + 1]) + bb.y);
+              }
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) w[i] = tc::pack_bf16x2(__uint_as_float(dr[2 * i]), __uint_as_float(dr[2 * i + 1]));
+          }
+          if (!last) tc::tmem_st16(tm + lane_off + 128u + 16u * c, w);
+          if (emit) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) orow[4 * c + e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+          }
+        }
+        if (!last) tc::tmem_wait_st();
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          tc::mbar_arrive(op_ready);   // operand written, D read
+          tc::mbar_arrive(&empty[st]);  // B_k read
+        }
+      }
+    }
   }
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
-
-  bool ok = true;
-  for (int k = 0; k < jb.nsteps; ++k) {
-    if (tid == 0 && tc::mbar_wait(&tma_bar[k], 0, abort_s)) {
-      tc::tc_fence_after();
-      const uint32_t b_base = tc::smem_u32(sm + k * kTile);
-#pragma unroll
-      for (int ks = 0; ks < kD / 16; ++ks) {
-        const uint64_t bd = tc::sdesc_sw128(b_base + ks * 2048, kHalf, 1024);
-        tc::mma_ts(tm, tm + 128u + 8u * ks, bd, kIdesc, ks > 0 ? 1u : 0u);
-      }
-      tc::mma_commit(mma_bar);
-    }
-    ok = tc::bar_all(1, 128, tc::mbar_wait(mma_bar, k & 1, abort_s));
-    if (!ok) break;
-    tc::tc_fence_after();
-    const bool last = k + 1 == jb.nsteps;
-    const bool emit = kAdvance || last;
-    uint4* orow = emit ? (uint4*)(odst + jb.out0 + (kAdvance ? (long)k * kD * kD : 0) + (long)v * kD) : nullptr;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      uint32_t dr[32];
-      tc::tmem_ld32(tm + lane_off + 32u * c, dr);
-      tc::tmem_wait_ld();
-      uint32_t w[16];
-      if (jb.addB) {
-        uint32_t bw[16];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          bw[4 * e + 0] = bq[4 * c + e].x;
-          bw[4 * e + 1] = bq[4 * c + e].y;
-          bw[4 * e + 2] = bq[4 * c + e].z;
-          bw[4 * e + 3] = bq[4 * c + e].w;
-        }
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float2 bb = tc::bf16x2_to_float2(bw[e]);
-          w[e] = tc::pack_bf16x2(__uint_as_float(dr[2 * e]) + bb.x, __uint_as_float(dr[2 * e + 1]) + bb.y);
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 16; ++e) w[e] = tc::pack_bf16x2(__uint_as_float(dr[2 * e]), __uint_as_float(dr[2 * e + 1]));
-      }
-      if (!last) tc::tmem_st16(tm + lane_off + 128u + 16u * c, w);
-      if (emit) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) orow[4 * c + e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
-      }
-    }
-    if (!last) {
-      tc::tmem_wait_st();
-      if (jb.addB) {  // the next step's row of B, in flight across the next product
-        const uint4* bn = (const uint4*)(brow0 + (long)(k + 1) * kD * kD);
-#pragma unroll
-        for (int e = 0; e < 16; ++e) bq[e] = bn[e];
-      }
-    }
-    tc::tc_fence_before();
-    __syncthreads();
-    tc::tc_fence_after();
-  }
-  if (tid == 0) {
-    if (!ok)  // never leave the CTA with copies in flight
-      for (int k = 0; k < jb.nsteps; ++k) tc::mbar_wait(&tma_bar[k], 0, nullptr, 200000000ull);
-    // every MMA issued by this thread completes before tensor memory is freed
-    tc::mma_commit(fin_bar);
-    tc::mbar_wait(fin_bar, 0, nullptr, 200000000ull);
-  }
-  tc::tc_fence_before();
-  __syncthreads();
-  tc::tc_fence_after();
-  if (warp == 0) tc::tmem_dealloc(tm, 256);
-  if (tid == 0 && *abort_s) report_device_error(kErrMbarTimeout);
+  if (warp == 1) tc::tmem_dealloc(tm, 256);
+  if (threadIdx.x == 0 && *abort_s) report_device_error(kErrMbarTimeout);
 }
 
 // CUDA-core chain: X (float32) in shared memory; each thread owns an R x R block of
@@ -295,17 +356,21 @@ cudaError_t launch_simt(const ChainArgs& a, long blocks, cudaStream_t s) {
 }
 
 template <bool kAdvance>
-cudaError_t launch_tc(const ChainArgs& a, long blocks, cudaStream_t s) {
+cudaError_t launch_tc(const ChainArgs& a, long jobs, cudaStream_t s) {
   // TMA row coordinates are 32-bit
   const long rows = (long)a.B * a.H * a.sub_stride * kD;
-  if (rows >= (1L << 31)) return cudaErrorInvalidValue;
-  CUtensorMap tmA;
+  const long srows = (long)a.B * a.H * a.Nsub * kD;
+  if (rows >= (1L << 31) || (kAdvance && srows >= (1L << 31))) return cudaErrorInvalidValue;
+  CUtensorMap tmA, tmB, tmX;
   cudaError_t e = make_tmap_rows128(&tmA, a.Asub, rows);
+  if (e == cudaSuccess) e = make_tmap_rows128(&tmB, a.Bsub, rows);
+  if (e == cudaSuccess) e = kAdvance ? make_tmap_rows128(&tmX, a.S, srows) : make_tmap_rows128(&tmX, a.Asub, rows);
   if (e != cudaSuccess) return e;
-  const size_t smem = 1024 + kMaxSteps * kTile + 64;
-  e = cudaFuncSetAttribute(chain_tc_kernel<kAdvance>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const size_t smem = 1024 + kPStages * kPStage + 128;
+  e = cudaFuncSetAttribute(chain_pipe_kernel<kAdvance>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  chain_tc_kernel<kAdvance><<<(unsigned)blocks, 128, smem, s>>>(tmA, a);
+  const long grid = jobs < num_sms() ? jobs : num_sms();
+  chain_pipe_kernel<kAdvance><<<(unsigned)grid, kPThreads, smem, s>>>(tmA, tmB, tmX, a, jobs);
   return cudaGetLastError();
 }
 
