@@ -11,12 +11,9 @@
 // WY solve and the intra-chunk read-out keep their 64-token tiles.  Merging costs
 // 2 (s - 1) d^3 multiply-adds per chunk, less than a WY solve over C tokens would.
 //
-// Tensor-core version (bf16, d = 128): one CTA of 4 warps per chain.  All s - 1
-// right-hand factors A_k arrive by TMA at once (128-byte swizzle, as compose_tc reads
-// them).  The running product X lives in tensor memory as the bf16 A operand of
-//   D = X A_k      (tcgen05.mma, M = N = K = 128, float32 accumulator in TMEM)
-// and each thread (one row) adds its row of B_k, rounds to bf16 and writes the next
-// operand back to tensor memory and, where the chain emits, to global memory.
+// Tensor-core version (bf16, d = 128): chain_pipe_kernel below, a persistent CTA per
+// SM with a TMA-fed ring; the running product X is the bf16 A operand of
+//   D = X A_k      (tcgen05.mma, M = N = K = 128, float32 accumulator in TMEM).
 // CUDA-core version (float32 arithmetic, any storage type, d = 64 or 128): one CTA
 // of 256 threads per chain, X in shared memory.
 #include "common.cuh"
@@ -221,8 +218,6 @@ __global__ void __launch_bounds__(kPThreads, 1)
     const int q = warp & 3;  // TMEM lane quarter of this warp
     const int v = 32 * q + lane;
     const uint32_t lane_off = (uint32_t)(32 * q) << 16;
-    const __nv_bfloat16* sbase = kAdvance ? (const __nv_bfloat16*)a.S : nullptr;
-    (void)sbase;
     long s = 0, step = 0;
     bool ok = true;
     for (long blk = blockIdx.x; blk < njobs && ok; blk += gridDim.x) {
