@@ -214,6 +214,7 @@ size_t hla_decode_workspace_bytes(const hla_config* cfg, int32_t max_chunks);
  * call has no workspace for sub-chunk factors, so each chunk runs the token rule
  * row by row on CUDA cores (float32, exact in real arithmetic like the WY form);
  * hla_prefill builds the same transitions from 64-token WY sub-chunks instead.
+ * HLA_DECAY_CHANNEL (alpha [B,T,H,d]): the token rule row by row at every C.
  */
 hla_status gdn_chunk_transitions(const hla_config* cfg, const void* k, const void* v,
                                  const float* alpha, const float* beta, void* A_out,
@@ -260,6 +261,10 @@ hla_status hla_gate_support(const hla_config* cfg, const float* gates, float* ma
  *      max_chunks >= T/C, filled with A/B/rk of every complete chunk, the final
  *      partial chunk's tokens and the counters.
  * workspace: device, >= hla_prefill_workspace_bytes(cfg), 256-byte aligned.
+ * Path: routing on a library side stream (forked from and joined back to `stream`
+ * by events) beside the chunk transitions; then the composition and the read-out.
+ * With HLA_DECAY_CHANNEL the transitions and the read-out run the token rule per
+ * chunk on CUDA cores.
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
  */
 hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, const void* v,
