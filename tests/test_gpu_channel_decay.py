@@ -146,3 +146,9 @@ def test_full_size_channel_decay_sampled(hla):
         P.check_routing_exact(r, gates, aidx, acnt, 0, h)
         rows = np.concatenate([np.arange(64 * i, 64 * i + 64) for i in sample])
         assert P.rel_l2(P.np64(o[0, rows, h]), r.o[rows]) <= P.TOL_BF16_RELL2
+
+
+def test_bf16_d64_channel_decay(hla):
+    """bf16 storage with d = 64 (CUDA-core composition, float32 states read by the
+    token-rule read-out)."""
+    _check_prefill(hla, syn.PREFILL_0P8B.with_(B=1, H=2, T=64 * 5 + 33, d=64, thr=0.2, decay="channel"))

@@ -137,3 +137,30 @@ def test_decode_window_gates(hla, dtype, d, C, window, T0, steps, fmt):
         assert len(st_.rk) == (T0 + steps) // C
         for j in range(len(st_.rk)):
             assert np.array_equal(rk[b, h, j].view(np.uint32), st_.rk[j].view(np.uint32))
+
+
+def test_window_gates_16_row_tiles(hla):
+    """Enough query chunks for the 16-row tiles of the windowed gate kernel (at least
+    two CTAs per SM): B=1, H=20, 256 chunks of 64 tokens, window 32.  Gates and
+    active lists bit-exact on two heads (the routing call alone)."""
+    w = syn.PREFILL_0P8B.with_(B=1, H=20, T=64 * 256, C=64, window=32, thr=0.3)
+    inp = P.gpu_inputs(w)
+    B, T, H, d = inp["q"].shape
+    N, W = w.N, w.C // w.window
+    assert (N // 16) * B * H >= 2 * 148
+    cfg = hla.make_config(B, H, T, w.C, d, w.dtype, "routed", w.tau, w.bias, w.thr, pool_window=w.window)
+    g = P.to_cuda(inp)
+    rq = torch.empty((B, H, N, d), dtype=torch.float32, device="cuda")
+    rk = torch.empty((B, H, N * W, d), dtype=torch.float32, device="cuda")
+    gates = torch.empty((B, H, N, N), dtype=torch.float32, device="cuda")
+    aidx = torch.empty((B, H, N, N), dtype=torch.int32, device="cuda")
+    acnt = torch.empty((B, H, N), dtype=torch.int32, device="cuda")
+    hla.hla_routing(cfg, g["q_route"], g["k_route"], rq, rk, gates_out=gates, active_idx_out=aidx,
+                    active_cnt_out=acnt)
+    torch.cuda.synchronize()
+    for h in (0, 13):
+        rqr = ho.route_pools(P.np32(inp["q_route"][0, :, h]), w.C, w.tau)
+        rkw = ho.window_pools(P.np32(inp["k_route"][0, :, h]), w.C, w.window, w.tau)
+        G = ho.gate_matrix(rqr, rkw, d, w.bias)
+        res = ho.HeadResult(o=None, gates=G, active=ho.active_lists(G, w.thr), rq=rqr, rk=rkw)
+        P.check_routing_exact(res, gates.cpu(), aidx.cpu(), acnt.cpu(), 0, h)
