@@ -572,8 +572,9 @@ def _decode_jobs(ctx, wd, tok, pairs):
     jobs = []
     for (b, h) in pairs:
         c = tuple(ctx[n][b, :, h].float().cpu().numpy().astype(np.float64) for n in ("q", "k", "v", "alpha", "beta"))
+        a_bh = tok["alpha"][b, h]
         t = (tok["q"][b, h].double().numpy(), tok["k"][b, h].double().numpy(), tok["v"][b, h].double().numpy(),
-             float(tok["alpha"][b, h]), float(tok["beta"][b, h]))
+             a_bh.double().numpy() if a_bh.dim() else float(a_bh), float(tok["beta"][b, h]))
         jobs.append((c, params, t, wd.window))
     return jobs
 

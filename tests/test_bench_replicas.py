@@ -83,3 +83,15 @@ def test_max_over_ranks_without_process_group_is_identity():
 def test_whole_job_rate_is_weak_scaling(world):
     # every rank processes 16384 tokens; the slowest rank took 4 ms
     assert bench.whole_job_rate(16384, 4.0, world) == pytest.approx(16384 * world / 4e-3)
+
+
+def test_oracle_baseline_jobs_take_every_variant():
+    """The CPU-baseline job builders of bench.py accept channel-wise decay and window
+    representatives (one tiny prefill and one decode step through the oracle)."""
+    import bench
+    import hla_synth as syn
+    for w in (syn.TINY_F32.with_(decay="channel", T=128), syn.TINY_F32.with_(window=16, T=128)):
+        inp = syn.make_gdn_inputs(w)
+        tok = syn.make_decode_tokens(w, 1)[0]
+        assert bench._oracle_prefill_worker(bench._prefill_jobs(inp, w, [(0, 1)])[0]) >= 0.0
+        assert bench._oracle_decode_worker(bench._decode_jobs(inp, w, tok, [(0, 0)])[0]) >= 0.0
