@@ -289,3 +289,31 @@ def test_decay_mode_checks(hla):
     c3 = cfg(hla, B=1, H=1, T=1, decay="channel", cache_format="factored")
     st = hla.lib().hla_cache_init(ctypes.byref(c3), 4, ctypes.c_void_p(1 << 20), 1 << 30, ctypes.byref(out), None)
     assert st == hla.HLA_ERR_UNSUPPORTED and "scalar decay" in hla.last_error()
+
+
+@pytest.mark.parametrize("window,decay", [(32, 0), (0, 1), (16, 1)])
+def test_cache_slice_offsets_with_windows_and_channel_decay(hla, window, decay):
+    """Window representatives keep C / w key pools per closed chunk and channel-wise
+    decay keeps d decays per buffered token; a slice advances those buffers by b0
+    sequences of the larger layouts (C = 64, d = 128, bf16)."""
+    c = hla.HlaCache()
+    c.B, c.H, c.C, c.d, c.dtype, c.max_chunks = 4, 2, 64, 128, 1, 3
+    c.pool_window, c.decay_mode = window, decay
+    fields = ("A", "Bm", "rk", "buf_k", "buf_v", "buf_qr", "buf_kr", "buf_alpha", "buf_beta", "n_chunks",
+              "m_partial")
+    for i, f in enumerate(fields):
+        setattr(c, f, (i + 1) << 32)
+    out = hla.HlaCache()
+    assert hla.lib().hla_cache_slice(ctypes.byref(c), 1, 3, ctypes.byref(out)) == hla.HLA_OK
+    reps = 64 // window if window else 1
+    adim = 128 if decay else 1
+    per_seq = {"A": 2 * 3 * 128 * 128 * 2, "Bm": 2 * 3 * 128 * 128 * 2, "rk": 2 * 3 * reps * 128 * 4,
+               "buf_k": 2 * 64 * 128 * 2, "buf_v": 2 * 64 * 128 * 2, "buf_qr": 2 * 64 * 128 * 2,
+               "buf_kr": 2 * 64 * 128 * 2, "buf_alpha": 2 * 64 * adim * 4, "buf_beta": 2 * 64 * 4,
+               "n_chunks": 4, "m_partial": 4}
+    for i, f in enumerate(fields):
+        assert getattr(out, f) == ((i + 1) << 32) + per_seq[f], f
+    # the cache block grows by exactly those buffers
+    base = hla.cache_bytes(cfg(hla, B=4, H=2, T=1, C=64), 3)
+    grown = hla.cache_bytes(cfg(hla, B=4, H=2, T=1, C=64, pool_window=window, decay=decay), 3)
+    assert grown - base >= 4 * (per_seq["rk"] - 2 * 3 * 128 * 4) + 4 * (per_seq["buf_alpha"] - 2 * 64 * 4)
