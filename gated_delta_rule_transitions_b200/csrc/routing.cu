@@ -97,7 +97,7 @@ constexpr int kPoolSeg = 64;    // pool_sum_bf16 stages 64 tokens at a time
 constexpr int kPoolMaxC = 256;  // longer chunks are pooled segment by segment
 
 template <typename Tin>
-__global__ void __launch_bounds__(64) pool_kernel(const Tin* __restrict__ x0, const Tin* __restrict__ x1,
+__global__ void __launch_bounds__(64, 12) pool_kernel(const Tin* __restrict__ x0, const Tin* __restrict__ x1,
                                                   float* __restrict__ r0, float* __restrict__ r1, int T, int H,
                                                   int d, int C, int out_chunk_stride, float tau) {
   constexpr bool kBf16 = sizeof(Tin) == 2;
