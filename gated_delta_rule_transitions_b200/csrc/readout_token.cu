@@ -9,9 +9,15 @@
 //   S_t = S_{t-1} Diag(alpha_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
 // and row r of S evolves on its own:
 //   s <- s o alpha_t;  s <- s - (beta_t (s . k_t) - beta_t v_t[r]) k_t;  o_t[r] = s . q_t.
-// One CTA per (chunk, head, sequence); a pair of threads keeps one row in registers
-// (interleaved channels 2j + hf); keys, queries and decays of 16 tokens at a time are
-// staged in shared memory.
+//
+// One CTA per (chunk, head, sequence) with 2 d threads.  A thread keeps two rows,
+// r0 = p and r1 = p + d/2, restricted to a quarter of the columns, in registers: the
+// columns 16 m + 4 g + u (u < 4) for its group index g = thread % 4.  So every
+// 16-byte shared-memory read of a key, decay or query is used for both rows, and the
+// four threads of a row pair read four adjacent 16-byte words (no bank conflict).
+// The dot products are summed over the four threads by two butterfly shuffles.
+// Keys, queries, decays and values of 16 tokens at a time are staged in shared
+// memory; the outputs of those tokens are gathered there and written row by row.
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -22,57 +28,119 @@ namespace {
 constexpr int kSeg = 16;
 
 template <int D, typename Tio, typename Ts>
-__global__ void __launch_bounds__(2 * D) readout_token_kernel(ReadoutTokenArgs a) {
-  constexpr int E = D / 2;
-  __shared__ float ks[kSeg][D];
-  __shared__ float qs[kSeg][D];
-  __shared__ float as[kSeg][D];
+__global__ void __launch_bounds__(2 * D, 2) readout_token_kernel(ReadoutTokenArgs a) {
+  constexpr int E = D / 4;   // columns per thread and row
+  constexpr int M = D / 16;  // 16-byte groups per thread and row
+  __shared__ __align__(16) float ks[kSeg][D];
+  __shared__ __align__(16) float qs[kSeg][D];
+  __shared__ __align__(16) float as[kSeg][D];
+  __shared__ float vs[kSeg][D];
+  __shared__ float os[kSeg][D];
   __shared__ float be[kSeg];
   const int i = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int r = threadIdx.x >> 1, hf = threadIdx.x & 1;
+  const int p = threadIdx.x >> 2, g = threadIdx.x & 3;
+  const int r0 = p, r1 = p + D / 2;
   const int t0 = i * a.C;
   const int n = min(a.C, a.T - t0);
   const long bh = (long)b * a.H + h;
-  const Ts* srow = (const Ts*)a.S_in + ((bh * a.N + i) * D + r) * (long)D + hf;
-  float x[E];
+  const Ts* S = (const Ts*)a.S_in + (bh * a.N + i) * (long)D * D;
+  float x0[E], x1[E];
 #pragma unroll
-  for (int j = 0; j < E; ++j) x[j] = ldf(srow + 2 * j);
+  for (int m = 0; m < M; ++m)
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int c = 16 * m + 4 * g + u;
+      x0[4 * m + u] = ldf(S + (long)r0 * D + c);
+      x1[4 * m + u] = ldf(S + (long)r1 * D + c);
+    }
   const long tok0 = b * a.in.sb + h * a.in.sh + (long)t0 * a.in.st;
   const Tio* kin = (const Tio*)a.in.k + tok0;
   const Tio* vin = (const Tio*)a.in.v + tok0;
   const Tio* qin = (const Tio*)a.q + tok0;
-  Tio* out = (Tio*)a.o + tok0 + r;
+  Tio* out = (Tio*)a.o + tok0;
   const long ab0 = b * a.in.ab + h * a.in.ah + (long)t0 * a.in.at;
   for (int s0 = 0; s0 < n; s0 += kSeg) {
     const int ns = min(kSeg, n - s0);
-    __syncthreads();
+    __syncthreads();  // the previous segment's staged inputs and outputs are consumed
     for (int idx = threadIdx.x; idx < ns * D; idx += 2 * D) {
       const int t = idx / D, cc = idx - t * D;
-      ks[t][cc] = ldf(kin + (long)(s0 + t) * a.in.st + cc);
-      qs[t][cc] = ldf(qin + (long)(s0 + t) * a.in.st + cc);
+      const long tk = (long)(s0 + t) * a.in.st + cc;
+      ks[t][cc] = ldf(kin + tk);
+      qs[t][cc] = ldf(qin + tk);
+      vs[t][cc] = ldf(vin + tk);
       as[t][cc] = a.in.alpha[ab0 + (long)(s0 + t) * a.in.at + cc];
     }
     // the alpha strides are those of beta times d
     if (threadIdx.x < ns) be[threadIdx.x] = a.in.beta[(ab0 + (long)(s0 + threadIdx.x) * a.in.at) / D];
     __syncthreads();
     for (int t = 0; t < ns; ++t) {
+      const float4* a4 = (const float4*)&as[t][4 * g];
+      const float4* k4 = (const float4*)&ks[t][4 * g];
+      const float4* q4 = (const float4*)&qs[t][4 * g];
+      float d0[2] = {0.0f, 0.0f}, d1[2] = {0.0f, 0.0f};
 #pragma unroll
-      for (int j = 0; j < E; ++j) x[j] *= as[t][2 * j + hf];
-      float p[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-      for (int j = 0; j < E; ++j) p[j & 3] = fmaf(x[j], ks[t][2 * j + hf], p[j & 3]);
-      float dot = (p[0] + p[1]) + (p[2] + p[3]);
-      dot += __shfl_xor_sync(0xFFFFFFFFu, dot, 1);
+      for (int m = 0; m < M; ++m) {
+        const float4 al = a4[4 * m];
+        const float4 kk = k4[4 * m];
+        x0[4 * m + 0] *= al.x;
+        x0[4 * m + 1] *= al.y;
+        x0[4 * m + 2] *= al.z;
+        x0[4 * m + 3] *= al.w;
+        x1[4 * m + 0] *= al.x;
+        x1[4 * m + 1] *= al.y;
+        x1[4 * m + 2] *= al.z;
+        x1[4 * m + 3] *= al.w;
+        d0[m & 1] = fmaf(x0[4 * m + 0], kk.x, d0[m & 1]);
+        d1[m & 1] = fmaf(x1[4 * m + 0], kk.x, d1[m & 1]);
+        d0[m & 1] = fmaf(x0[4 * m + 1], kk.y, d0[m & 1]);
+        d1[m & 1] = fmaf(x1[4 * m + 1], kk.y, d1[m & 1]);
+        d0[m & 1] = fmaf(x0[4 * m + 2], kk.z, d0[m & 1]);
+        d1[m & 1] = fmaf(x1[4 * m + 2], kk.z, d1[m & 1]);
+        d0[m & 1] = fmaf(x0[4 * m + 3], kk.w, d0[m & 1]);
+        d1[m & 1] = fmaf(x1[4 * m + 3], kk.w, d1[m & 1]);
+      }
+      float dot0 = d0[0] + d0[1], dot1 = d1[0] + d1[1];
+      dot0 += __shfl_xor_sync(0xFFFFFFFFu, dot0, 1);
+      dot1 += __shfl_xor_sync(0xFFFFFFFFu, dot1, 1);
+      dot0 += __shfl_xor_sync(0xFFFFFFFFu, dot0, 2);
+      dot1 += __shfl_xor_sync(0xFFFFFFFFu, dot1, 2);
       const float bt = be[t];
-      const float f = bt * dot - bt * ldf(vin + (long)(s0 + t) * a.in.st + r);
+      const float f0 = bt * dot0 - bt * vs[t][r0];
+      const float f1 = bt * dot1 - bt * vs[t][r1];
+      float y0[2] = {0.0f, 0.0f}, y1[2] = {0.0f, 0.0f};
 #pragma unroll
-      for (int j = 0; j < E; ++j) x[j] = fmaf(-f, ks[t][2 * j + hf], x[j]);
-      float o[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-      for (int j = 0; j < E; ++j) o[j & 3] = fmaf(x[j], qs[t][2 * j + hf], o[j & 3]);
-      float y = (o[0] + o[1]) + (o[2] + o[3]);
-      y += __shfl_xor_sync(0xFFFFFFFFu, y, 1);
-      if (hf == 0) stf(out + (long)(s0 + t) * a.in.st, y);
+      for (int m = 0; m < M; ++m) {
+        const float4 kk = k4[4 * m];
+        const float4 qq = q4[4 * m];
+        x0[4 * m + 0] = fmaf(-f0, kk.x, x0[4 * m + 0]);
+        x0[4 * m + 1] = fmaf(-f0, kk.y, x0[4 * m + 1]);
+        x0[4 * m + 2] = fmaf(-f0, kk.z, x0[4 * m + 2]);
+        x0[4 * m + 3] = fmaf(-f0, kk.w, x0[4 * m + 3]);
+        x1[4 * m + 0] = fmaf(-f1, kk.x, x1[4 * m + 0]);
+        x1[4 * m + 1] = fmaf(-f1, kk.y, x1[4 * m + 1]);
+        x1[4 * m + 2] = fmaf(-f1, kk.z, x1[4 * m + 2]);
+        x1[4 * m + 3] = fmaf(-f1, kk.w, x1[4 * m + 3]);
+        y0[m & 1] = fmaf(x0[4 * m + 0], qq.x, y0[m & 1]);
+        y1[m & 1] = fmaf(x1[4 * m + 0], qq.x, y1[m & 1]);
+        y0[m & 1] = fmaf(x0[4 * m + 1], qq.y, y0[m & 1]);
+        y1[m & 1] = fmaf(x1[4 * m + 1], qq.y, y1[m & 1]);
+        y0[m & 1] = fmaf(x0[4 * m + 2], qq.z, y0[m & 1]);
+        y1[m & 1] = fmaf(x1[4 * m + 2], qq.z, y1[m & 1]);
+        y0[m & 1] = fmaf(x0[4 * m + 3], qq.w, y0[m & 1]);
+        y1[m & 1] = fmaf(x1[4 * m + 3], qq.w, y1[m & 1]);
+      }
+      float o0 = y0[0] + y0[1], o1 = y1[0] + y1[1];
+      o0 += __shfl_xor_sync(0xFFFFFFFFu, o0, 1);
+      o1 += __shfl_xor_sync(0xFFFFFFFFu, o1, 1);
+      o0 += __shfl_xor_sync(0xFFFFFFFFu, o0, 2);
+      o1 += __shfl_xor_sync(0xFFFFFFFFu, o1, 2);
+      if (g == 0) os[t][r0] = o0;
+      if (g == 1) os[t][r1] = o1;
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < ns * D; idx += 2 * D) {
+      const int t = idx / D, cc = idx - t * D;
+      stf(out + (long)(s0 + t) * a.in.st + cc, os[t][cc]);
     }
   }
 }

@@ -7,11 +7,12 @@
 // over its tokens.  Row by row that is
 //   s <- alpha_t s - (alpha_t beta_t (s . k_t) - beta_t v_t[r]) k_t,
 // so every row of A_c (started at the unit row e_r, with no write) and of B_c
-// (started at zero) evolves on its own.  A pair of threads keeps one row in
-// registers; the CTA stages the keys of 64 tokens at a time in shared memory.
+// (started at zero) evolves on its own in registers; the CTA stages the tokens of a
+// segment in shared memory.
 //
-// Used where no workspace is at hand: the decode step closing a chunk of C > 64
-// tokens, and gdn_chunk_transitions at C > 64.  hla_prefill builds the same
+// Used for channel-wise decay (prefill and decode close) and where no workspace is
+// at hand: the decode step closing a chunk of C > 64 tokens, and
+// gdn_chunk_transitions at C > 64.  With a scalar decay hla_prefill builds the same
 // transitions from 64-token WY sub-chunks merged on the tensor cores.
 #include "common.cuh"
 #include "kernels.cuh"
@@ -20,30 +21,47 @@ namespace hla {
 
 namespace {
 
-// Tokens staged per step: 64 (keys only), 32 with channel-wise decay (keys and
-// decays), so the static shared memory stays at 32 KiB for d = 128.
+// Tokens staged per step: 32 (keys and values), 16 with channel-wise decay (keys,
+// decays and values).
 template <bool kChan>
-constexpr int seg_len() { return kChan ? 32 : 64; }
+constexpr int seg_len() { return kChan ? 16 : 32; }
 
-// grid (chunks, H, 2 B): blockIdx.z & 1 selects the rows of A (0) or B (1).  Two
-// threads per row: thread (r, hf) keeps the row's elements 2 j + hf (interleaved, so
-// the pair reads adjacent shared-memory words) and the pair adds its dot products.
+// Shared memory (floats): the staged tokens, reused at the end for the output rows
+// (d/2 rows at a time, row stride d + 16 so that the 16-byte stores of the eight
+// lanes of one phase fall in distinct banks).
+template <int D, bool kChan>
+constexpr int smem_floats() {
+  constexpr int stage = seg_len<kChan>() * D * (kChan ? 3 : 2);
+  constexpr int outp = (D / 2) * (D + 16);
+  return stage > outp ? stage : outp;
+}
+
+// grid (chunks, H, 2 B): blockIdx.z & 1 selects the rows of A (0) or B (1).  2 d
+// threads; a thread keeps rows r0 = p and r1 = p + d/2 restricted to the columns
+// 16 m + 4 g + u (u < 4) of its group index g = thread % 4, so every 16-byte
+// shared-memory read of a key or decay serves both rows and the four threads of a
+// row pair read four adjacent 16-byte words.  Two butterfly shuffles sum the dot
+// products over the four threads.
 // kChan: channel-wise decay, the row is first scaled channel by channel,
 //   s <- s o alpha_t,  then  s <- s - (beta_t (s . k_t) - beta_t v_t[r]) k_t.
 template <int D, typename Tio, bool kChan>
-__global__ void __launch_bounds__(2 * D) transitions_token_kernel(TransArgs a) {
-  constexpr int E = D / 2;
+__global__ void __launch_bounds__(2 * D, 2) transitions_token_kernel(TransArgs a) {
+  constexpr int E = D / 4;   // columns per thread and row
+  constexpr int M = D / 16;  // 16-byte groups per thread and row
   constexpr int kSeg = seg_len<kChan>();
-  __shared__ float ks[kSeg][D];
-  __shared__ float as[kChan ? kSeg : 1][kChan ? D : 1];
+  constexpr int kOutStride = D + 16;
+  __shared__ __align__(16) float sm[smem_floats<D, kChan>()];
   __shared__ float al[kSeg], be[kSeg];
+  float (*ks)[D] = (float (*)[D])sm;
+  float (*vs)[D] = (float (*)[D])(sm + kSeg * D);
+  float (*as)[D] = (float (*)[D])(sm + 2 * kSeg * D);  // kChan only
   const int c = blockIdx.x;
   const int h = blockIdx.y;
   const int b = blockIdx.z >> 1;
   const bool rowsB = (blockIdx.z & 1) != 0;
   const int C = a.C;
-  const int r = threadIdx.x >> 1;
-  const int hf = threadIdx.x & 1;
+  const int p = threadIdx.x >> 2, g = threadIdx.x & 3;
+  const int r0 = p, r1 = p + D / 2;
   long chunk_out = c;
   if (a.close_m != nullptr) {
     // decode close: only sequences whose open chunk becomes full this step
@@ -56,14 +74,21 @@ __global__ void __launch_bounds__(2 * D) transitions_token_kernel(TransArgs a) {
   const Tio* kin = (const Tio*)a.in.k + b * a.in.sb + h * a.in.sh + (long)t0 * a.in.st;
   const Tio* vin = (const Tio*)a.in.v + b * a.in.sb + h * a.in.sh + (long)t0 * a.in.st;
   const long ab0 = b * a.in.ab + h * a.in.ah + (long)t0 * a.in.at;
-  float x[E];
+  float x0[E], x1[E];
 #pragma unroll
-  for (int j = 0; j < E; ++j) x[j] = (!rowsB && 2 * j + hf == r) ? 1.0f : 0.0f;
+  for (int m = 0; m < M; ++m)
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int cc = 16 * m + 4 * g + u;
+      x0[4 * m + u] = (!rowsB && cc == r0) ? 1.0f : 0.0f;
+      x1[4 * m + u] = (!rowsB && cc == r1) ? 1.0f : 0.0f;
+    }
   for (int s0 = 0; s0 < C; s0 += kSeg) {
     __syncthreads();
     for (int idx = threadIdx.x; idx < kSeg * D; idx += 2 * D) {
       const int t = idx / D, cc = idx - t * D;
       ks[t][cc] = ldf(kin + (long)(s0 + t) * a.in.st + cc);
+      if (rowsB) vs[t][cc] = ldf(vin + (long)(s0 + t) * a.in.st + cc);
       if constexpr (kChan) as[t][cc] = a.in.alpha[ab0 + (long)(s0 + t) * a.in.at + cc];
     }
     if (threadIdx.x < kSeg) {
@@ -74,35 +99,100 @@ __global__ void __launch_bounds__(2 * D) transitions_token_kernel(TransArgs a) {
     }
     __syncthreads();
     for (int t = 0; t < kSeg; ++t) {
+      const float4* k4 = (const float4*)&ks[t][4 * g];
       if constexpr (kChan) {
+        const float4* a4 = (const float4*)&as[t][4 * g];
 #pragma unroll
-        for (int j = 0; j < E; ++j) x[j] *= as[t][2 * j + hf];
+        for (int m = 0; m < M; ++m) {
+          const float4 w = a4[4 * m];
+          x0[4 * m + 0] *= w.x;
+          x0[4 * m + 1] *= w.y;
+          x0[4 * m + 2] *= w.z;
+          x0[4 * m + 3] *= w.w;
+          x1[4 * m + 0] *= w.x;
+          x1[4 * m + 1] *= w.y;
+          x1[4 * m + 2] *= w.z;
+          x1[4 * m + 3] *= w.w;
+        }
       }
-      float p[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // four partial sums for latency
+      float d0[2] = {0.0f, 0.0f}, d1[2] = {0.0f, 0.0f};
 #pragma unroll
-      for (int j = 0; j < E; ++j) p[j & 3] = fmaf(x[j], ks[t][2 * j + hf], p[j & 3]);
-      float dot = (p[0] + p[1]) + (p[2] + p[3]);
-      dot += __shfl_xor_sync(0xFFFFFFFFu, dot, 1);
+      for (int m = 0; m < M; ++m) {
+        const float4 kk = k4[4 * m];
+        d0[m & 1] = fmaf(x0[4 * m + 0], kk.x, d0[m & 1]);
+        d1[m & 1] = fmaf(x1[4 * m + 0], kk.x, d1[m & 1]);
+        d0[m & 1] = fmaf(x0[4 * m + 1], kk.y, d0[m & 1]);
+        d1[m & 1] = fmaf(x1[4 * m + 1], kk.y, d1[m & 1]);
+        d0[m & 1] = fmaf(x0[4 * m + 2], kk.z, d0[m & 1]);
+        d1[m & 1] = fmaf(x1[4 * m + 2], kk.z, d1[m & 1]);
+        d0[m & 1] = fmaf(x0[4 * m + 3], kk.w, d0[m & 1]);
+        d1[m & 1] = fmaf(x1[4 * m + 3], kk.w, d1[m & 1]);
+      }
+      float dot0 = d0[0] + d0[1], dot1 = d1[0] + d1[1];
+      dot0 += __shfl_xor_sync(0xFFFFFFFFu, dot0, 1);
+      dot1 += __shfl_xor_sync(0xFFFFFFFFu, dot1, 1);
+      dot0 += __shfl_xor_sync(0xFFFFFFFFu, dot0, 2);
+      dot1 += __shfl_xor_sync(0xFFFFFFFFu, dot1, 2);
       const float bt = be[t];
       if constexpr (kChan) {
-        float f = bt * dot;
-        if (rowsB) f -= bt * ldf(vin + (long)(s0 + t) * a.in.st + r);
+        float f0 = bt * dot0, f1 = bt * dot1;
+        if (rowsB) {
+          f0 -= bt * vs[t][r0];
+          f1 -= bt * vs[t][r1];
+        }
 #pragma unroll
-        for (int j = 0; j < E; ++j) x[j] = fmaf(-f, ks[t][2 * j + hf], x[j]);
+        for (int m = 0; m < M; ++m) {
+          const float4 kk = k4[4 * m];
+          x0[4 * m + 0] = fmaf(-f0, kk.x, x0[4 * m + 0]);
+          x0[4 * m + 1] = fmaf(-f0, kk.y, x0[4 * m + 1]);
+          x0[4 * m + 2] = fmaf(-f0, kk.z, x0[4 * m + 2]);
+          x0[4 * m + 3] = fmaf(-f0, kk.w, x0[4 * m + 3]);
+          x1[4 * m + 0] = fmaf(-f1, kk.x, x1[4 * m + 0]);
+          x1[4 * m + 1] = fmaf(-f1, kk.y, x1[4 * m + 1]);
+          x1[4 * m + 2] = fmaf(-f1, kk.z, x1[4 * m + 2]);
+          x1[4 * m + 3] = fmaf(-f1, kk.w, x1[4 * m + 3]);
+        }
       } else {
         const float at = al[t];
-        float f = at * bt * dot;
-        if (rowsB) f -= bt * ldf(vin + (long)(s0 + t) * a.in.st + r);
+        float f0 = at * bt * dot0, f1 = at * bt * dot1;
+        if (rowsB) {
+          f0 -= bt * vs[t][r0];
+          f1 -= bt * vs[t][r1];
+        }
 #pragma unroll
-        for (int j = 0; j < E; ++j) x[j] = fmaf(at, x[j], -f * ks[t][2 * j + hf]);
+        for (int m = 0; m < M; ++m) {
+          const float4 kk = k4[4 * m];
+          x0[4 * m + 0] = fmaf(at, x0[4 * m + 0], -f0 * kk.x);
+          x0[4 * m + 1] = fmaf(at, x0[4 * m + 1], -f0 * kk.y);
+          x0[4 * m + 2] = fmaf(at, x0[4 * m + 2], -f0 * kk.z);
+          x0[4 * m + 3] = fmaf(at, x0[4 * m + 3], -f0 * kk.w);
+          x1[4 * m + 0] = fmaf(at, x1[4 * m + 0], -f1 * kk.x);
+          x1[4 * m + 1] = fmaf(at, x1[4 * m + 1], -f1 * kk.y);
+          x1[4 * m + 2] = fmaf(at, x1[4 * m + 2], -f1 * kk.z);
+          x1[4 * m + 3] = fmaf(at, x1[4 * m + 3], -f1 * kk.w);
+        }
       }
     }
   }
+  // the rows leave through shared memory, half of them at a time, so that the global
+  // writes run along rows
   const long bhc = (long)b * a.H + h;
-  Tio* out = (Tio*)(rowsB ? a.Bm : a.A) + (bhc * a.ab_chunk_stride + chunk_out + a.ab_chunk_offset) * (long)D * D +
-             (long)r * D + hf;
+  Tio* out = (Tio*)(rowsB ? a.Bm : a.A) + (bhc * a.ab_chunk_stride + chunk_out + a.ab_chunk_offset) * (long)D * D;
 #pragma unroll
-  for (int j = 0; j < E; ++j) stf(out + 2 * j, x[j]);
+  for (int half = 0; half < 2; ++half) {
+    __syncthreads();
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+      const float* x = half ? x1 : x0;
+      *(float4*)&sm[p * kOutStride + 16 * m + 4 * g] =
+          make_float4(x[4 * m + 0], x[4 * m + 1], x[4 * m + 2], x[4 * m + 3]);
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < (D / 2) * D; idx += 2 * D) {
+      const int rr = idx / D, cc = idx - rr * D;
+      stf(out + (long)(half * (D / 2) + rr) * D + cc, sm[rr * kOutStride + cc]);
+    }
+  }
 }
 
 template <int D, typename Tio>
