@@ -15,7 +15,8 @@
 // columns 16 m + 4 g + u (u < 4) for its group index g = thread % 4.  So every
 // 16-byte shared-memory read of a key, decay or query is used for both rows, and the
 // four threads of a row pair read four adjacent 16-byte words (no bank conflict).
-// The dot products are summed over the four threads by two butterfly shuffles.
+// The two rows advance together in packed float32 pairs (f32x2 arithmetic).  The
+// dot products are summed over the four threads by two butterfly shuffles.
 // Keys, queries, decays and values of 16 tokens at a time are staged in shared
 // memory; the outputs of those tokens are gathered there and written row by row.
 #include "common.cuh"
@@ -44,14 +45,15 @@ __global__ void __launch_bounds__(2 * D, 2) readout_token_kernel(ReadoutTokenArg
   const int n = min(a.C, a.T - t0);
   const long bh = (long)b * a.H + h;
   const Ts* S = (const Ts*)a.S_in + (bh * a.N + i) * (long)D * D;
-  float x0[E], x1[E];
+  // x[j] = (row r0, row r1) at column j: the two rows share every key, decay and
+  // query value, so each step is one packed float32 pair operation
+  float2 x[E];
 #pragma unroll
   for (int m = 0; m < M; ++m)
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int c = 16 * m + 4 * g + u;
-      x0[4 * m + u] = ldf(S + (long)r0 * D + c);
-      x1[4 * m + u] = ldf(S + (long)r1 * D + c);
+      x[4 * m + u] = make_float2(ldf(S + (long)r0 * D + c), ldf(S + (long)r1 * D + c));
     }
   const long tok0 = b * a.in.sb + h * a.in.sh + (long)t0 * a.in.st;
   const Tio* kin = (const Tio*)a.in.k + tok0;
@@ -77,59 +79,42 @@ __global__ void __launch_bounds__(2 * D, 2) readout_token_kernel(ReadoutTokenArg
       const float4* a4 = (const float4*)&as[t][4 * g];
       const float4* k4 = (const float4*)&ks[t][4 * g];
       const float4* q4 = (const float4*)&qs[t][4 * g];
-      float d0[2] = {0.0f, 0.0f}, d1[2] = {0.0f, 0.0f};
+      float2 d[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
 #pragma unroll
       for (int m = 0; m < M; ++m) {
         const float4 al = a4[4 * m];
         const float4 kk = k4[4 * m];
-        x0[4 * m + 0] *= al.x;
-        x0[4 * m + 1] *= al.y;
-        x0[4 * m + 2] *= al.z;
-        x0[4 * m + 3] *= al.w;
-        x1[4 * m + 0] *= al.x;
-        x1[4 * m + 1] *= al.y;
-        x1[4 * m + 2] *= al.z;
-        x1[4 * m + 3] *= al.w;
-        d0[m & 1] = fmaf(x0[4 * m + 0], kk.x, d0[m & 1]);
-        d1[m & 1] = fmaf(x1[4 * m + 0], kk.x, d1[m & 1]);
-        d0[m & 1] = fmaf(x0[4 * m + 1], kk.y, d0[m & 1]);
-        d1[m & 1] = fmaf(x1[4 * m + 1], kk.y, d1[m & 1]);
-        d0[m & 1] = fmaf(x0[4 * m + 2], kk.z, d0[m & 1]);
-        d1[m & 1] = fmaf(x1[4 * m + 2], kk.z, d1[m & 1]);
-        d0[m & 1] = fmaf(x0[4 * m + 3], kk.w, d0[m & 1]);
-        d1[m & 1] = fmaf(x1[4 * m + 3], kk.w, d1[m & 1]);
+        x[4 * m + 0] = __fmul2_rn(x[4 * m + 0], make_float2(al.x, al.x));
+        x[4 * m + 1] = __fmul2_rn(x[4 * m + 1], make_float2(al.y, al.y));
+        x[4 * m + 2] = __fmul2_rn(x[4 * m + 2], make_float2(al.z, al.z));
+        x[4 * m + 3] = __fmul2_rn(x[4 * m + 3], make_float2(al.w, al.w));
+        d[m & 1] = __ffma2_rn(x[4 * m + 0], make_float2(kk.x, kk.x), d[m & 1]);
+        d[m & 1] = __ffma2_rn(x[4 * m + 1], make_float2(kk.y, kk.y), d[m & 1]);
+        d[m & 1] = __ffma2_rn(x[4 * m + 2], make_float2(kk.z, kk.z), d[m & 1]);
+        d[m & 1] = __ffma2_rn(x[4 * m + 3], make_float2(kk.w, kk.w), d[m & 1]);
       }
-      float dot0 = d0[0] + d0[1], dot1 = d1[0] + d1[1];
+      float dot0 = d[0].x + d[1].x, dot1 = d[0].y + d[1].y;
       dot0 += __shfl_xor_sync(0xFFFFFFFFu, dot0, 1);
       dot1 += __shfl_xor_sync(0xFFFFFFFFu, dot1, 1);
       dot0 += __shfl_xor_sync(0xFFFFFFFFu, dot0, 2);
       dot1 += __shfl_xor_sync(0xFFFFFFFFu, dot1, 2);
       const float bt = be[t];
-      const float f0 = bt * dot0 - bt * vs[t][r0];
-      const float f1 = bt * dot1 - bt * vs[t][r1];
-      float y0[2] = {0.0f, 0.0f}, y1[2] = {0.0f, 0.0f};
+      const float2 nf = make_float2(-(bt * dot0 - bt * vs[t][r0]), -(bt * dot1 - bt * vs[t][r1]));
+      float2 y[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
 #pragma unroll
       for (int m = 0; m < M; ++m) {
         const float4 kk = k4[4 * m];
         const float4 qq = q4[4 * m];
-        x0[4 * m + 0] = fmaf(-f0, kk.x, x0[4 * m + 0]);
-        x0[4 * m + 1] = fmaf(-f0, kk.y, x0[4 * m + 1]);
-        x0[4 * m + 2] = fmaf(-f0, kk.z, x0[4 * m + 2]);
-        x0[4 * m + 3] = fmaf(-f0, kk.w, x0[4 * m + 3]);
-        x1[4 * m + 0] = fmaf(-f1, kk.x, x1[4 * m + 0]);
-        x1[4 * m + 1] = fmaf(-f1, kk.y, x1[4 * m + 1]);
-        x1[4 * m + 2] = fmaf(-f1, kk.z, x1[4 * m + 2]);
-        x1[4 * m + 3] = fmaf(-f1, kk.w, x1[4 * m + 3]);
-        y0[m & 1] = fmaf(x0[4 * m + 0], qq.x, y0[m & 1]);
-        y1[m & 1] = fmaf(x1[4 * m + 0], qq.x, y1[m & 1]);
-        y0[m & 1] = fmaf(x0[4 * m + 1], qq.y, y0[m & 1]);
-        y1[m & 1] = fmaf(x1[4 * m + 1], qq.y, y1[m & 1]);
-        y0[m & 1] = fmaf(x0[4 * m + 2], qq.z, y0[m & 1]);
-        y1[m & 1] = fmaf(x1[4 * m + 2], qq.z, y1[m & 1]);
-        y0[m & 1] = fmaf(x0[4 * m + 3], qq.w, y0[m & 1]);
-        y1[m & 1] = fmaf(x1[4 * m + 3], qq.w, y1[m & 1]);
+        x[4 * m + 0] = __ffma2_rn(nf, make_float2(kk.x, kk.x), x[4 * m + 0]);
+        x[4 * m + 1] = __ffma2_rn(nf, make_float2(kk.y, kk.y), x[4 * m + 1]);
+        x[4 * m + 2] = __ffma2_rn(nf, make_float2(kk.z, kk.z), x[4 * m + 2]);
+        x[4 * m + 3] = __ffma2_rn(nf, make_float2(kk.w, kk.w), x[4 * m + 3]);
+        y[m & 1] = __ffma2_rn(x[4 * m + 0], make_float2(qq.x, qq.x), y[m & 1]);
+        y[m & 1] = __ffma2_rn(x[4 * m + 1], make_float2(qq.y, qq.y), y[m & 1]);
+        y[m & 1] = __ffma2_rn(x[4 * m + 2], make_float2(qq.z, qq.z), y[m & 1]);
+        y[m & 1] = __ffma2_rn(x[4 * m + 3], make_float2(qq.w, qq.w), y[m & 1]);
       }
-      float o0 = y0[0] + y0[1], o1 = y1[0] + y1[1];
+      float o0 = y[0].x + y[1].x, o1 = y[0].y + y[1].y;
       o0 += __shfl_xor_sync(0xFFFFFFFFu, o0, 1);
       o1 += __shfl_xor_sync(0xFFFFFFFFu, o1, 1);
       o0 += __shfl_xor_sync(0xFFFFFFFFu, o0, 2);

@@ -40,8 +40,9 @@ constexpr int smem_floats() {
 // threads; a thread keeps rows r0 = p and r1 = p + d/2 restricted to the columns
 // 16 m + 4 g + u (u < 4) of its group index g = thread % 4, so every 16-byte
 // shared-memory read of a key or decay serves both rows and the four threads of a
-// row pair read four adjacent 16-byte words.  Two butterfly shuffles sum the dot
-// products over the four threads.
+// row pair read four adjacent 16-byte words; the two rows advance together in packed
+// float32 pairs (f32x2 arithmetic).  Two butterfly shuffles sum the dot products over
+// the four threads.
 // kChan: channel-wise decay, the row is first scaled channel by channel,
 //   s <- s o alpha_t,  then  s <- s - (beta_t (s . k_t) - beta_t v_t[r]) k_t.
 template <int D, typename Tio, bool kChan>
@@ -74,14 +75,14 @@ __global__ void __launch_bounds__(2 * D, 2) transitions_token_kernel(TransArgs a
   const Tio* kin = (const Tio*)a.in.k + b * a.in.sb + h * a.in.sh + (long)t0 * a.in.st;
   const Tio* vin = (const Tio*)a.in.v + b * a.in.sb + h * a.in.sh + (long)t0 * a.in.st;
   const long ab0 = b * a.in.ab + h * a.in.ah + (long)t0 * a.in.at;
-  float x0[E], x1[E];
+  // x[j] = (row r0, row r1) at column j: one packed float32 pair operation per step
+  float2 x[E];
 #pragma unroll
   for (int m = 0; m < M; ++m)
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int cc = 16 * m + 4 * g + u;
-      x0[4 * m + u] = (!rowsB && cc == r0) ? 1.0f : 0.0f;
-      x1[4 * m + u] = (!rowsB && cc == r1) ? 1.0f : 0.0f;
+      x[4 * m + u] = make_float2((!rowsB && cc == r0) ? 1.0f : 0.0f, (!rowsB && cc == r1) ? 1.0f : 0.0f);
     }
   for (int s0 = 0; s0 < C; s0 += kSeg) {
     __syncthreads();
@@ -105,30 +106,22 @@ __global__ void __launch_bounds__(2 * D, 2) transitions_token_kernel(TransArgs a
 #pragma unroll
         for (int m = 0; m < M; ++m) {
           const float4 w = a4[4 * m];
-          x0[4 * m + 0] *= w.x;
-          x0[4 * m + 1] *= w.y;
-          x0[4 * m + 2] *= w.z;
-          x0[4 * m + 3] *= w.w;
-          x1[4 * m + 0] *= w.x;
-          x1[4 * m + 1] *= w.y;
-          x1[4 * m + 2] *= w.z;
-          x1[4 * m + 3] *= w.w;
+          x[4 * m + 0] = __fmul2_rn(x[4 * m + 0], make_float2(w.x, w.x));
+          x[4 * m + 1] = __fmul2_rn(x[4 * m + 1], make_float2(w.y, w.y));
+          x[4 * m + 2] = __fmul2_rn(x[4 * m + 2], make_float2(w.z, w.z));
+          x[4 * m + 3] = __fmul2_rn(x[4 * m + 3], make_float2(w.w, w.w));
         }
       }
-      float d0[2] = {0.0f, 0.0f}, d1[2] = {0.0f, 0.0f};
+      float2 d[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
 #pragma unroll
       for (int m = 0; m < M; ++m) {
         const float4 kk = k4[4 * m];
-        d0[m & 1] = fmaf(x0[4 * m + 0], kk.x, d0[m & 1]);
-        d1[m & 1] = fmaf(x1[4 * m + 0], kk.x, d1[m & 1]);
-        d0[m & 1] = fmaf(x0[4 * m + 1], kk.y, d0[m & 1]);
-        d1[m & 1] = fmaf(x1[4 * m + 1], kk.y, d1[m & 1]);
-        d0[m & 1] = fmaf(x0[4 * m + 2], kk.z, d0[m & 1]);
-        d1[m & 1] = fmaf(x1[4 * m + 2], kk.z, d1[m & 1]);
-        d0[m & 1] = fmaf(x0[4 * m + 3], kk.w, d0[m & 1]);
-        d1[m & 1] = fmaf(x1[4 * m + 3], kk.w, d1[m & 1]);
+        d[m & 1] = __ffma2_rn(x[4 * m + 0], make_float2(kk.x, kk.x), d[m & 1]);
+        d[m & 1] = __ffma2_rn(x[4 * m + 1], make_float2(kk.y, kk.y), d[m & 1]);
+        d[m & 1] = __ffma2_rn(x[4 * m + 2], make_float2(kk.z, kk.z), d[m & 1]);
+        d[m & 1] = __ffma2_rn(x[4 * m + 3], make_float2(kk.w, kk.w), d[m & 1]);
       }
-      float dot0 = d0[0] + d0[1], dot1 = d1[0] + d1[1];
+      float dot0 = d[0].x + d[1].x, dot1 = d[0].y + d[1].y;
       dot0 += __shfl_xor_sync(0xFFFFFFFFu, dot0, 1);
       dot1 += __shfl_xor_sync(0xFFFFFFFFu, dot1, 1);
       dot0 += __shfl_xor_sync(0xFFFFFFFFu, dot0, 2);
@@ -140,17 +133,14 @@ __global__ void __launch_bounds__(2 * D, 2) transitions_token_kernel(TransArgs a
           f0 -= bt * vs[t][r0];
           f1 -= bt * vs[t][r1];
         }
+        const float2 nf = make_float2(-f0, -f1);
 #pragma unroll
         for (int m = 0; m < M; ++m) {
           const float4 kk = k4[4 * m];
-          x0[4 * m + 0] = fmaf(-f0, kk.x, x0[4 * m + 0]);
-          x0[4 * m + 1] = fmaf(-f0, kk.y, x0[4 * m + 1]);
-          x0[4 * m + 2] = fmaf(-f0, kk.z, x0[4 * m + 2]);
-          x0[4 * m + 3] = fmaf(-f0, kk.w, x0[4 * m + 3]);
-          x1[4 * m + 0] = fmaf(-f1, kk.x, x1[4 * m + 0]);
-          x1[4 * m + 1] = fmaf(-f1, kk.y, x1[4 * m + 1]);
-          x1[4 * m + 2] = fmaf(-f1, kk.z, x1[4 * m + 2]);
-          x1[4 * m + 3] = fmaf(-f1, kk.w, x1[4 * m + 3]);
+          x[4 * m + 0] = __ffma2_rn(nf, make_float2(kk.x, kk.x), x[4 * m + 0]);
+          x[4 * m + 1] = __ffma2_rn(nf, make_float2(kk.y, kk.y), x[4 * m + 1]);
+          x[4 * m + 2] = __ffma2_rn(nf, make_float2(kk.z, kk.z), x[4 * m + 2]);
+          x[4 * m + 3] = __ffma2_rn(nf, make_float2(kk.w, kk.w), x[4 * m + 3]);
         }
       } else {
         const float at = al[t];
@@ -159,17 +149,14 @@ __global__ void __launch_bounds__(2 * D, 2) transitions_token_kernel(TransArgs a
           f0 -= bt * vs[t][r0];
           f1 -= bt * vs[t][r1];
         }
+        const float2 nf = make_float2(-f0, -f1), at2 = make_float2(at, at);
 #pragma unroll
         for (int m = 0; m < M; ++m) {
           const float4 kk = k4[4 * m];
-          x0[4 * m + 0] = fmaf(at, x0[4 * m + 0], -f0 * kk.x);
-          x0[4 * m + 1] = fmaf(at, x0[4 * m + 1], -f0 * kk.y);
-          x0[4 * m + 2] = fmaf(at, x0[4 * m + 2], -f0 * kk.z);
-          x0[4 * m + 3] = fmaf(at, x0[4 * m + 3], -f0 * kk.w);
-          x1[4 * m + 0] = fmaf(at, x1[4 * m + 0], -f1 * kk.x);
-          x1[4 * m + 1] = fmaf(at, x1[4 * m + 1], -f1 * kk.y);
-          x1[4 * m + 2] = fmaf(at, x1[4 * m + 2], -f1 * kk.z);
-          x1[4 * m + 3] = fmaf(at, x1[4 * m + 3], -f1 * kk.w);
+          x[4 * m + 0] = __ffma2_rn(at2, x[4 * m + 0], __fmul2_rn(nf, make_float2(kk.x, kk.x)));
+          x[4 * m + 1] = __ffma2_rn(at2, x[4 * m + 1], __fmul2_rn(nf, make_float2(kk.y, kk.y)));
+          x[4 * m + 2] = __ffma2_rn(at2, x[4 * m + 2], __fmul2_rn(nf, make_float2(kk.z, kk.z)));
+          x[4 * m + 3] = __ffma2_rn(at2, x[4 * m + 3], __fmul2_rn(nf, make_float2(kk.w, kk.w)));
         }
       }
     }
@@ -182,11 +169,10 @@ __global__ void __launch_bounds__(2 * D, 2) transitions_token_kernel(TransArgs a
   for (int half = 0; half < 2; ++half) {
     __syncthreads();
 #pragma unroll
-    for (int m = 0; m < M; ++m) {
-      const float* x = half ? x1 : x0;
+    for (int m = 0; m < M; ++m)
       *(float4*)&sm[p * kOutStride + 16 * m + 4 * g] =
-          make_float4(x[4 * m + 0], x[4 * m + 1], x[4 * m + 2], x[4 * m + 3]);
-    }
+          half ? make_float4(x[4 * m + 0].y, x[4 * m + 1].y, x[4 * m + 2].y, x[4 * m + 3].y)
+               : make_float4(x[4 * m + 0].x, x[4 * m + 1].x, x[4 * m + 2].x, x[4 * m + 3].x);
     __syncthreads();
     for (int idx = threadIdx.x; idx < (D / 2) * D; idx += 2 * D) {
       const int rr = idx / D, cc = idx - rr * D;
