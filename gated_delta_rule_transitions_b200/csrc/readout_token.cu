@@ -10,17 +10,17 @@
 // and row r of S evolves on its own:
 //   s <- s o alpha_t;  s <- s - (beta_t (s . k_t) - beta_t v_t[r]) k_t;  o_t[r] = s . q_t.
 //
-// One CTA per (chunk, head, sequence) with 2 d threads.  A thread keeps two rows,
-// r0 = p and r1 = p + d/2, restricted to a quarter of the columns, in registers: the
-// columns 16 m + 4 g + u (u < 4) for its group index g = thread % 4.  So every
-// 16-byte shared-memory read of a key, decay or query is used for both rows, and the
-// four threads of a row pair read four adjacent 16-byte words (no bank conflict).
-// The two rows advance together in packed float32 pairs (f32x2 arithmetic).  The
-// dot products are summed over the four threads by two butterfly shuffles.
-// Keys, queries, decays and values of 16 tokens at a time are staged in shared
-// memory; the outputs of those tokens are gathered there and written row by row.
+// One CTA per (chunk, head, sequence) with 2 d threads in groups of 8; each thread
+// keeps its group's four rows of S on an eighth of the columns (token_rows.cuh): every
+// 16-byte shared-memory read of a key, decay or query feeds four rows, the rows
+// advance in packed float32 pairs, and a reduce-scatter / all-gather over the group
+// forms the per-row dot products.  The keys of the current token stay in registers
+// between the dot product and the update.  Keys, queries, decays and values of 16
+// tokens at a time are staged in shared memory; the outputs of those tokens are
+// gathered there and written row by row.
 #include "common.cuh"
 #include "kernels.cuh"
+#include "token_rows.cuh"
 
 namespace hla {
 
@@ -30,8 +30,10 @@ constexpr int kSeg = 16;
 
 template <int D, typename Tio, typename Ts>
 __global__ void __launch_bounds__(2 * D, 2) readout_token_kernel(ReadoutTokenArgs a) {
-  constexpr int E = D / 4;   // columns per thread and row
-  constexpr int M = D / 16;  // 16-byte groups per thread and row
+  using namespace token_rows;
+  constexpr int E = D / 8;   // columns per thread
+  constexpr int M = D / 32;  // 16-byte groups per thread
+  constexpr int G = D / 4;   // row groups: rows p, p + G, p + 2G, p + 3G
   __shared__ __align__(16) float ks[kSeg][D];
   __shared__ __align__(16) float qs[kSeg][D];
   __shared__ __align__(16) float as[kSeg][D];
@@ -39,21 +41,21 @@ __global__ void __launch_bounds__(2 * D, 2) readout_token_kernel(ReadoutTokenArg
   __shared__ float os[kSeg][D];
   __shared__ float be[kSeg];
   const int i = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int p = threadIdx.x >> 2, g = threadIdx.x & 3;
-  const int r0 = p, r1 = p + D / 2;
+  const int p = threadIdx.x >> 3, g = threadIdx.x & 7;
+  const int rown = p + G * owned_row(g);
   const int t0 = i * a.C;
   const int n = min(a.C, a.T - t0);
   const long bh = (long)b * a.H + h;
   const Ts* S = (const Ts*)a.S_in + (bh * a.N + i) * (long)D * D;
-  // x[j] = (row r0, row r1) at column j: the two rows share every key, decay and
-  // query value, so each step is one packed float32 pair operation
-  float2 x[E];
+  // x01[j] = (rows p, p + G) and x23[j] = (rows p + 2G, p + 3G) at column j
+  float2 x01[E], x23[E];
 #pragma unroll
   for (int m = 0; m < M; ++m)
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const int c = 16 * m + 4 * g + u;
-      x[4 * m + u] = make_float2(ldf(S + (long)r0 * D + c), ldf(S + (long)r1 * D + c));
+      const long c = 32 * m + 4 * g + u;
+      x01[4 * m + u] = make_float2(ldf(S + (long)p * D + c), ldf(S + (long)(p + G) * D + c));
+      x23[4 * m + u] = make_float2(ldf(S + (long)(p + 2 * G) * D + c), ldf(S + (long)(p + 3 * G) * D + c));
     }
   const long tok0 = b * a.in.sb + h * a.in.sh + (long)t0 * a.in.st;
   const Tio* kin = (const Tio*)a.in.k + tok0;
@@ -79,48 +81,47 @@ __global__ void __launch_bounds__(2 * D, 2) readout_token_kernel(ReadoutTokenArg
       const float4* a4 = (const float4*)&as[t][4 * g];
       const float4* k4 = (const float4*)&ks[t][4 * g];
       const float4* q4 = (const float4*)&qs[t][4 * g];
-      float2 d[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
+      float kr[E];
+      float2 d01[2] = {dup(0.0f), dup(0.0f)}, d23[2] = {dup(0.0f), dup(0.0f)};
 #pragma unroll
       for (int m = 0; m < M; ++m) {
-        const float4 al = a4[4 * m];
-        const float4 kk = k4[4 * m];
-        x[4 * m + 0] = __fmul2_rn(x[4 * m + 0], make_float2(al.x, al.x));
-        x[4 * m + 1] = __fmul2_rn(x[4 * m + 1], make_float2(al.y, al.y));
-        x[4 * m + 2] = __fmul2_rn(x[4 * m + 2], make_float2(al.z, al.z));
-        x[4 * m + 3] = __fmul2_rn(x[4 * m + 3], make_float2(al.w, al.w));
-        d[m & 1] = __ffma2_rn(x[4 * m + 0], make_float2(kk.x, kk.x), d[m & 1]);
-        d[m & 1] = __ffma2_rn(x[4 * m + 1], make_float2(kk.y, kk.y), d[m & 1]);
-        d[m & 1] = __ffma2_rn(x[4 * m + 2], make_float2(kk.z, kk.z), d[m & 1]);
-        d[m & 1] = __ffma2_rn(x[4 * m + 3], make_float2(kk.w, kk.w), d[m & 1]);
+        const float4 al = a4[8 * m];
+        const float4 kk = k4[8 * m];
+        const float alv[4] = {al.x, al.y, al.z, al.w};
+        kr[4 * m + 0] = kk.x;
+        kr[4 * m + 1] = kk.y;
+        kr[4 * m + 2] = kk.z;
+        kr[4 * m + 3] = kk.w;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int j = 4 * m + u;
+          x01[j] = __fmul2_rn(x01[j], dup(alv[u]));
+          x23[j] = __fmul2_rn(x23[j], dup(alv[u]));
+          d01[u & 1] = __ffma2_rn(x01[j], dup(kr[j]), d01[u & 1]);
+          d23[u & 1] = __ffma2_rn(x23[j], dup(kr[j]), d23[u & 1]);
+        }
       }
-      float dot0 = d[0].x + d[1].x, dot1 = d[0].y + d[1].y;
-      dot0 += __shfl_xor_sync(0xFFFFFFFFu, dot0, 1);
-      dot1 += __shfl_xor_sync(0xFFFFFFFFu, dot1, 1);
-      dot0 += __shfl_xor_sync(0xFFFFFFFFu, dot0, 2);
-      dot1 += __shfl_xor_sync(0xFFFFFFFFu, dot1, 2);
+      const float dot = rs_sum4(add2(d01[0], d01[1]), add2(d23[0], d23[1]), g);
       const float bt = be[t];
-      const float2 nf = make_float2(-(bt * dot0 - bt * vs[t][r0]), -(bt * dot1 - bt * vs[t][r1]));
-      float2 y[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
+      float2 f01, f23;
+      ag_rows4(bt * dot - bt * vs[t][rown], g, f01, f23);
+      const float2 n01 = make_float2(-f01.x, -f01.y), n23 = make_float2(-f23.x, -f23.y);
+      float2 y01[2] = {dup(0.0f), dup(0.0f)}, y23[2] = {dup(0.0f), dup(0.0f)};
 #pragma unroll
       for (int m = 0; m < M; ++m) {
-        const float4 kk = k4[4 * m];
-        const float4 qq = q4[4 * m];
-        x[4 * m + 0] = __ffma2_rn(nf, make_float2(kk.x, kk.x), x[4 * m + 0]);
-        x[4 * m + 1] = __ffma2_rn(nf, make_float2(kk.y, kk.y), x[4 * m + 1]);
-        x[4 * m + 2] = __ffma2_rn(nf, make_float2(kk.z, kk.z), x[4 * m + 2]);
-        x[4 * m + 3] = __ffma2_rn(nf, make_float2(kk.w, kk.w), x[4 * m + 3]);
-        y[m & 1] = __ffma2_rn(x[4 * m + 0], make_float2(qq.x, qq.x), y[m & 1]);
-        y[m & 1] = __ffma2_rn(x[4 * m + 1], make_float2(qq.y, qq.y), y[m & 1]);
-        y[m & 1] = __ffma2_rn(x[4 * m + 2], make_float2(qq.z, qq.z), y[m & 1]);
-        y[m & 1] = __ffma2_rn(x[4 * m + 3], make_float2(qq.w, qq.w), y[m & 1]);
+        const float4 qq = q4[8 * m];
+        const float qv[4] = {qq.x, qq.y, qq.z, qq.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int j = 4 * m + u;
+          x01[j] = __ffma2_rn(n01, dup(kr[j]), x01[j]);
+          x23[j] = __ffma2_rn(n23, dup(kr[j]), x23[j]);
+          y01[u & 1] = __ffma2_rn(x01[j], dup(qv[u]), y01[u & 1]);
+          y23[u & 1] = __ffma2_rn(x23[j], dup(qv[u]), y23[u & 1]);
+        }
       }
-      float o0 = y[0].x + y[1].x, o1 = y[0].y + y[1].y;
-      o0 += __shfl_xor_sync(0xFFFFFFFFu, o0, 1);
-      o1 += __shfl_xor_sync(0xFFFFFFFFu, o1, 1);
-      o0 += __shfl_xor_sync(0xFFFFFFFFu, o0, 2);
-      o1 += __shfl_xor_sync(0xFFFFFFFFu, o1, 2);
-      if (g == 0) os[t][r0] = o0;
-      if (g == 1) os[t][r1] = o1;
+      const float y = rs_sum4(add2(y01[0], y01[1]), add2(y23[0], y23[1]), g);
+      if ((g & 1) == 0) os[t][rown] = y;
     }
     __syncthreads();
     for (int idx = threadIdx.x; idx < ns * D; idx += 2 * D) {

@@ -16,6 +16,7 @@
 // transitions from 64-token WY sub-chunks merged on the tensor cores.
 #include "common.cuh"
 #include "kernels.cuh"
+#include "token_rows.cuh"
 
 namespace hla {
 
@@ -27,30 +28,28 @@ template <bool kChan>
 constexpr int seg_len() { return kChan ? 16 : 32; }
 
 // Shared memory (floats): the staged tokens, reused at the end for the output rows
-// (d/2 rows at a time, row stride d + 16 so that the 16-byte stores of the eight
-// lanes of one phase fall in distinct banks).
+// (d/4 rows at a time).
 template <int D, bool kChan>
 constexpr int smem_floats() {
   constexpr int stage = seg_len<kChan>() * D * (kChan ? 3 : 2);
-  constexpr int outp = (D / 2) * (D + 16);
+  constexpr int outp = (D / 4) * D;
   return stage > outp ? stage : outp;
 }
 
 // grid (chunks, H, 2 B): blockIdx.z & 1 selects the rows of A (0) or B (1).  2 d
-// threads; a thread keeps rows r0 = p and r1 = p + d/2 restricted to the columns
-// 16 m + 4 g + u (u < 4) of its group index g = thread % 4, so every 16-byte
-// shared-memory read of a key or decay serves both rows and the four threads of a
-// row pair read four adjacent 16-byte words; the two rows advance together in packed
-// float32 pairs (f32x2 arithmetic).  Two butterfly shuffles sum the dot products over
-// the four threads.
+// threads in groups of 8; each thread keeps its group's four rows on an eighth of the
+// columns (token_rows.cuh), so every 16-byte shared-memory read of a key or decay
+// feeds four rows, and the keys of the current token stay in registers between the
+// dot product and the update.  The rows advance in packed float32 pairs.
 // kChan: channel-wise decay, the row is first scaled channel by channel,
 //   s <- s o alpha_t,  then  s <- s - (beta_t (s . k_t) - beta_t v_t[r]) k_t.
 template <int D, typename Tio, bool kChan>
 __global__ void __launch_bounds__(2 * D, 2) transitions_token_kernel(TransArgs a) {
-  constexpr int E = D / 4;   // columns per thread and row
-  constexpr int M = D / 16;  // 16-byte groups per thread and row
+  using namespace token_rows;
+  constexpr int E = D / 8;   // columns per thread
+  constexpr int M = D / 32;  // 16-byte groups per thread
+  constexpr int G = D / 4;   // row groups: rows p, p + G, p + 2G, p + 3G
   constexpr int kSeg = seg_len<kChan>();
-  constexpr int kOutStride = D + 16;
   __shared__ __align__(16) float sm[smem_floats<D, kChan>()];
   __shared__ float al[kSeg], be[kSeg];
   float (*ks)[D] = (float (*)[D])sm;
@@ -61,8 +60,8 @@ __global__ void __launch_bounds__(2 * D, 2) transitions_token_kernel(TransArgs a
   const int b = blockIdx.z >> 1;
   const bool rowsB = (blockIdx.z & 1) != 0;
   const int C = a.C;
-  const int p = threadIdx.x >> 2, g = threadIdx.x & 3;
-  const int r0 = p, r1 = p + D / 2;
+  const int p = threadIdx.x >> 3, g = threadIdx.x & 7;
+  const int rown = p + G * owned_row(g);
   long chunk_out = c;
   if (a.close_m != nullptr) {
     // decode close: only sequences whose open chunk becomes full this step
@@ -75,14 +74,17 @@ __global__ void __launch_bounds__(2 * D, 2) transitions_token_kernel(TransArgs a
   const Tio* kin = (const Tio*)a.in.k + b * a.in.sb + h * a.in.sh + (long)t0 * a.in.st;
   const Tio* vin = (const Tio*)a.in.v + b * a.in.sb + h * a.in.sh + (long)t0 * a.in.st;
   const long ab0 = b * a.in.ab + h * a.in.ah + (long)t0 * a.in.at;
-  // x[j] = (row r0, row r1) at column j: one packed float32 pair operation per step
-  float2 x[E];
+  // x01[j] = (rows p, p + G) and x23[j] = (rows p + 2G, p + 3G) at column j
+  float2 x01[E], x23[E];
 #pragma unroll
   for (int m = 0; m < M; ++m)
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const int cc = 16 * m + 4 * g + u;
-      x[4 * m + u] = make_float2((!rowsB && cc == r0) ? 1.0f : 0.0f, (!rowsB && cc == r1) ? 1.0f : 0.0f);
+      const int cc = 32 * m + 4 * g + u;
+      const bool unit = !rowsB && cc % G == p;  // rows of A start at the unit row
+      const int q = cc / G;                     // which of the four rows is row cc
+      x01[4 * m + u] = make_float2(unit && q == 0 ? 1.0f : 0.0f, unit && q == 1 ? 1.0f : 0.0f);
+      x23[4 * m + u] = make_float2(unit && q == 2 ? 1.0f : 0.0f, unit && q == 3 ? 1.0f : 0.0f);
     }
   for (int s0 = 0; s0 < C; s0 += kSeg) {
     __syncthreads();
@@ -101,82 +103,82 @@ __global__ void __launch_bounds__(2 * D, 2) transitions_token_kernel(TransArgs a
     __syncthreads();
     for (int t = 0; t < kSeg; ++t) {
       const float4* k4 = (const float4*)&ks[t][4 * g];
+      float kr[E];
+#pragma unroll
+      for (int m = 0; m < M; ++m) {
+        const float4 kk = k4[8 * m];
+        kr[4 * m + 0] = kk.x;
+        kr[4 * m + 1] = kk.y;
+        kr[4 * m + 2] = kk.z;
+        kr[4 * m + 3] = kk.w;
+      }
       if constexpr (kChan) {
         const float4* a4 = (const float4*)&as[t][4 * g];
 #pragma unroll
         for (int m = 0; m < M; ++m) {
-          const float4 w = a4[4 * m];
-          x[4 * m + 0] = __fmul2_rn(x[4 * m + 0], make_float2(w.x, w.x));
-          x[4 * m + 1] = __fmul2_rn(x[4 * m + 1], make_float2(w.y, w.y));
-          x[4 * m + 2] = __fmul2_rn(x[4 * m + 2], make_float2(w.z, w.z));
-          x[4 * m + 3] = __fmul2_rn(x[4 * m + 3], make_float2(w.w, w.w));
+          const float4 w = a4[8 * m];
+          const float wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            x01[4 * m + u] = __fmul2_rn(x01[4 * m + u], dup(wv[u]));
+            x23[4 * m + u] = __fmul2_rn(x23[4 * m + u], dup(wv[u]));
+          }
         }
       }
-      float2 d[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
+      float2 d01[2] = {dup(0.0f), dup(0.0f)}, d23[2] = {dup(0.0f), dup(0.0f)};
 #pragma unroll
-      for (int m = 0; m < M; ++m) {
-        const float4 kk = k4[4 * m];
-        d[m & 1] = __ffma2_rn(x[4 * m + 0], make_float2(kk.x, kk.x), d[m & 1]);
-        d[m & 1] = __ffma2_rn(x[4 * m + 1], make_float2(kk.y, kk.y), d[m & 1]);
-        d[m & 1] = __ffma2_rn(x[4 * m + 2], make_float2(kk.z, kk.z), d[m & 1]);
-        d[m & 1] = __ffma2_rn(x[4 * m + 3], make_float2(kk.w, kk.w), d[m & 1]);
+      for (int j = 0; j < E; ++j) {
+        d01[j & 1] = __ffma2_rn(x01[j], dup(kr[j]), d01[j & 1]);
+        d23[j & 1] = __ffma2_rn(x23[j], dup(kr[j]), d23[j & 1]);
       }
-      float dot0 = d[0].x + d[1].x, dot1 = d[0].y + d[1].y;
-      dot0 += __shfl_xor_sync(0xFFFFFFFFu, dot0, 1);
-      dot1 += __shfl_xor_sync(0xFFFFFFFFu, dot1, 1);
-      dot0 += __shfl_xor_sync(0xFFFFFFFFu, dot0, 2);
-      dot1 += __shfl_xor_sync(0xFFFFFFFFu, dot1, 2);
+      const float dot = rs_sum4(add2(d01[0], d01[1]), add2(d23[0], d23[1]), g);
       const float bt = be[t];
+      float f;
+      if constexpr (kChan)
+        f = bt * dot;
+      else
+        f = al[t] * bt * dot;
+      if (rowsB) f -= bt * vs[t][rown];
+      float2 f01, f23;
+      ag_rows4(f, g, f01, f23);
+      const float2 n01 = make_float2(-f01.x, -f01.y), n23 = make_float2(-f23.x, -f23.y);
       if constexpr (kChan) {
-        float f0 = bt * dot0, f1 = bt * dot1;
-        if (rowsB) {
-          f0 -= bt * vs[t][r0];
-          f1 -= bt * vs[t][r1];
-        }
-        const float2 nf = make_float2(-f0, -f1);
 #pragma unroll
-        for (int m = 0; m < M; ++m) {
-          const float4 kk = k4[4 * m];
-          x[4 * m + 0] = __ffma2_rn(nf, make_float2(kk.x, kk.x), x[4 * m + 0]);
-          x[4 * m + 1] = __ffma2_rn(nf, make_float2(kk.y, kk.y), x[4 * m + 1]);
-          x[4 * m + 2] = __ffma2_rn(nf, make_float2(kk.z, kk.z), x[4 * m + 2]);
-          x[4 * m + 3] = __ffma2_rn(nf, make_float2(kk.w, kk.w), x[4 * m + 3]);
+        for (int j = 0; j < E; ++j) {
+          x01[j] = __ffma2_rn(n01, dup(kr[j]), x01[j]);
+          x23[j] = __ffma2_rn(n23, dup(kr[j]), x23[j]);
         }
       } else {
-        const float at = al[t];
-        float f0 = at * bt * dot0, f1 = at * bt * dot1;
-        if (rowsB) {
-          f0 -= bt * vs[t][r0];
-          f1 -= bt * vs[t][r1];
-        }
-        const float2 nf = make_float2(-f0, -f1), at2 = make_float2(at, at);
+        const float2 at2 = dup(al[t]);
 #pragma unroll
-        for (int m = 0; m < M; ++m) {
-          const float4 kk = k4[4 * m];
-          x[4 * m + 0] = __ffma2_rn(at2, x[4 * m + 0], __fmul2_rn(nf, make_float2(kk.x, kk.x)));
-          x[4 * m + 1] = __ffma2_rn(at2, x[4 * m + 1], __fmul2_rn(nf, make_float2(kk.y, kk.y)));
-          x[4 * m + 2] = __ffma2_rn(at2, x[4 * m + 2], __fmul2_rn(nf, make_float2(kk.z, kk.z)));
-          x[4 * m + 3] = __ffma2_rn(at2, x[4 * m + 3], __fmul2_rn(nf, make_float2(kk.w, kk.w)));
+        for (int j = 0; j < E; ++j) {
+          x01[j] = __ffma2_rn(at2, x01[j], __fmul2_rn(n01, dup(kr[j])));
+          x23[j] = __ffma2_rn(at2, x23[j], __fmul2_rn(n23, dup(kr[j])));
         }
       }
     }
   }
-  // the rows leave through shared memory, half of them at a time, so that the global
-  // writes run along rows
+  // the rows leave through shared memory, a quarter of them at a time, so that the
+  // global writes run along rows
   const long bhc = (long)b * a.H + h;
   Tio* out = (Tio*)(rowsB ? a.Bm : a.A) + (bhc * a.ab_chunk_stride + chunk_out + a.ab_chunk_offset) * (long)D * D;
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {
+  for (int q = 0; q < 4; ++q) {
     __syncthreads();
 #pragma unroll
-    for (int m = 0; m < M; ++m)
-      *(float4*)&sm[p * kOutStride + 16 * m + 4 * g] =
-          half ? make_float4(x[4 * m + 0].y, x[4 * m + 1].y, x[4 * m + 2].y, x[4 * m + 3].y)
-               : make_float4(x[4 * m + 0].x, x[4 * m + 1].x, x[4 * m + 2].x, x[4 * m + 3].x);
+    for (int m = 0; m < M; ++m) {
+      float w[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float2 v2 = q < 2 ? x01[4 * m + u] : x23[4 * m + u];
+        w[u] = (q & 1) ? v2.y : v2.x;
+      }
+      *(float4*)&sm[p * D + 32 * m + 4 * g] = make_float4(w[0], w[1], w[2], w[3]);
+    }
     __syncthreads();
-    for (int idx = threadIdx.x; idx < (D / 2) * D; idx += 2 * D) {
+    for (int idx = threadIdx.x; idx < G * D; idx += 2 * D) {
       const int rr = idx / D, cc = idx - rr * D;
-      stf(out + (long)(half * (D / 2) + rr) * D + cc, sm[rr * kOutStride + cc]);
+      stf(out + (long)(q * G + rr) * D + cc, sm[rr * D + cc]);
     }
   }
 }
