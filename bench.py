@@ -73,19 +73,23 @@ def whole_job_rate(units_per_rank, ms_max, world):
     return units_per_rank * world / (ms_max * 1e-3)
 
 
-# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from the ncu
-# captures summarised under profiles/, keyed by the kernel and tagged with the SHA-256
-# prefix of the kernel's source files at capture time.  A figure is reported only
-# while those sources are unchanged.
-#   compose: full-size launch of the dense 0.8B-like prefill (compose_tc_prefill_0p8b.md)
-#   decode_main: see below
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu
+# capture of each kernel, keyed by the kernel and tagged with the SHA-256 prefix of
+# the kernel's source files at capture time.  A figure is reported only while those
+# sources are unchanged.
+#   compose: one full-size launch on the dense 0.8B-like prefill
+#   decode_main: a 4-sequence decode (64 of the 1024 (sequence, head) streams of the
+#     32K-context step), scaled by 16; per stream it equals the algorithmic bytes
 NCU_TRAFFIC = {
     "compose": (2.0461e9, {"compose_tc.cu": "82d501993514b885", "tc_common.cuh": "c10beda371c1dd4b"}),
-    # decode_main: capture of a 4-sequence decode (64 of the 1024 (sequence, head)
-    # streams), scaled by 16; per stream it equals the algorithmic bytes
-    # (decode_stream_decode_32k.md)
     "decode_main": (3.4694e10, {"decode_stream.cu": "6aebf8bbbdfe238d", "tc_common.cuh": "c10beda371c1dd4b"}),
 }
+
+# Datasheet figures of one B200, reported beside the measured denominators: dense
+# bf16 tensor throughput 2.25 PFLOP/s (without 2:4 sparsity) and HBM3e bandwidth of
+# about 8 TB/s (7.7 TB/s in the HGX configuration).
+DATASHEET_BF16_TFLOPS = 2250.0
+DATASHEET_HBM_GBS = 8000.0
 
 
 def ncu_traffic(kernel):
@@ -108,11 +112,17 @@ def ncu_traffic(kernel):
 
 
 def _peaks():
+    """(HBM GB/s, bf16 burst TFLOP/s, bf16 sustained TFLOP/s, source).  The measured
+    copy bandwidth and cuBLAS bf16 throughput of this GPU pool when the measurement
+    file is present; otherwise an earlier measurement on the same pool, labelled
+    "fallback" in the output line and announced on stderr."""
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             p = json.load(f)
         return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]), "measured"
-    except Exception:
+    except Exception as e:
+        print(f"bench.py: no measured peaks ({type(e).__name__}); using the fallback figures 6650 GB/s and "
+              f"1590 / 1400 TFLOP/s, labelled 'fallback'", file=sys.stderr)
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
@@ -479,6 +489,9 @@ def run_ours(args):
                      "unit": "TFLOP/s", "frac": (comp_tf / bf16_tf) if comp_tf else None,
                      "traffic": ncu_traffic("compose"), "traffic_unit": "bytes per launch (ncu dram read+write)",
                      "peak_source": f"{peak_src} bf16 dense (burst)",
+                     "datasheet": {"peak": DATASHEET_BF16_TFLOPS,
+                                   "frac": (comp_tf / DATASHEET_BF16_TFLOPS) if comp_tf else None,
+                                   "source": "B200 datasheet, dense bf16"},
                      "algorithmic": f"{comp_what} x 2 d^3 = {flops_compose:.4g} flop per launch",
                      "prefill_frac_of_peak": (flops_compose + flops_other) / (pre_ms * 1e-3) / 1e12 / bf16_tf},
         "decode": {"value": whole_job_rate(tokens_dec, dec_ms, world), "unit": "tokens/s", "ms_per_step": dec_ms,
@@ -487,6 +500,9 @@ def run_ours(args):
                                 "traffic": ncu_traffic("decode_main") if args.decode_cache == "dense" else None,
                                 "traffic_unit": "bytes per launch (ncu dram read+write)",
                                 "peak_source": f"{peak_src} HBM copy",
+                                "datasheet": {"peak": DATASHEET_HBM_GBS,
+                                              "frac": (dec_gbs / DATASHEET_HBM_GBS) if dec_gbs else None,
+                                              "source": "B200 datasheet HBM3e (about 8 TB/s)"},
                                 "algorithmic": f"{bytes_decode:.4g} bytes per launch ({n_ctx} active chunks "
                                                f"({args.decode_cache} cache) + key pools per sequence and head)"},
                    "e2e": {"value": whole_job_rate(tokens_dec, e2e_dec, world), "unit": "tokens/s",

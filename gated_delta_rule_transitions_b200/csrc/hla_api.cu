@@ -7,6 +7,8 @@
 #include <mutex>
 #include <vector>
 
+#include <cuda.h>
+
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -254,24 +256,79 @@ class StageScope {
   bool on_ = false;
 };
 
+// ---- CUDA context identity ----------------------------------------------------------
+// Streams, events and symbol addresses belong to the CUDA context that was current
+// when they were made.  The library keeps such handles per device and remembers the
+// unique id of the context they belong to; a call made under another context (a
+// non-primary one, or the primary context recreated after cudaDeviceReset) makes
+// new ones.  The id comes from the driver API through the runtime's entry-point
+// query, so the library does not link against the driver library.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Id of the context current on this thread; 0 if none is current or the driver
+// does not provide the calls.
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = (CtxGetCurrentFn)p;
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = (CtxGetIdFn)p;
+  });
+  if (get_current == nullptr || get_id == nullptr) return 0;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  unsigned long long id = 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
 // ---- side stream ---------------------------------------------------------------
 // hla_prefill runs the routing stage (pools, gates, active lists) on a per-device
 // side stream, forked from and joined back to the caller's stream by events, so it
 // overlaps the chunk transitions: the two read only the caller's inputs and write
-// disjoint parts of the workspace.  Created on first use on each device.
+// disjoint parts of the workspace.  Created on first use on each device (and again
+// when the current context is not the one it was made in).  One lock covers every
+// device's side stream: concurrent hla_prefill calls, on any streams, enqueue their
+// routing one after another through it.
 struct SideStream {
   cudaStream_t s = nullptr;
   cudaEvent_t fork = nullptr, join = nullptr;
+  unsigned long long ctx_id = 0;
 };
 constexpr int kMaxDevices = 64;
 std::mutex g_side_mu;
 SideStream g_side[kMaxDevices];
+
+// Makes `s` wait for the routing enqueued on the side stream.  Armed once the
+// side stream has forked from `s`; an error return before the regular join runs
+// it, so the caller's stream (or a capture on it) never holds an unjoined fork.
+struct SideJoin {
+  cudaStream_t side = nullptr, s = nullptr;
+  cudaEvent_t join = nullptr;
+  bool armed = false;
+  ~SideJoin() {
+    if (!armed) return;
+    cudaEventRecord(join, side);
+    cudaStreamWaitEvent(s, join, 0);
+  }
+};
 
 hla_status side_stream(SideStream** out) {
   int dev = -1;
   HLA_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
   if (dev < 0 || dev >= kMaxDevices) return fail(HLA_ERR_UNSUPPORTED, "device ordinal %d beyond %d", dev, kMaxDevices);
   SideStream& ss = g_side[dev];
+  // handles of another context are dropped, not destroyed (that context may be gone)
+  if (ss.s != nullptr && ss.ctx_id != current_context_id()) ss = SideStream{};
   if (ss.s == nullptr) {
     cudaStream_t st = nullptr;
     cudaEvent_t f = nullptr, j = nullptr;
@@ -281,6 +338,7 @@ hla_status side_stream(SideStream** out) {
     ss.fork = f;
     ss.join = j;
     ss.s = st;
+    ss.ctx_id = current_context_id();
   }
   *out = &ss;
   return HLA_OK;
@@ -591,6 +649,11 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
   HLA_TRY(side_stream(&side));
   HLA_CUDA(cudaEventRecord(side->fork, s), "side stream fork");
   HLA_CUDA(cudaStreamWaitEvent(side->s, side->fork, 0), "side stream fork");
+  SideJoin side_join;
+  side_join.side = side->s;
+  side_join.s = s;
+  side_join.join = side->join;
+  side_join.armed = true;
   HLA_TRY(routing_impl(cfg, qr, kr, rq, (cfg->gate_mode == HLA_GATES_ROUTED || cache_out) ? rk : nullptr,
                        user_gates, act_idx, act_g, act_cnt, gates_out, active_idx_out, active_cnt_out, side->s));
   HLA_CUDA(cudaEventRecord(side->join, side->s), "side stream join");
@@ -661,6 +724,7 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
     StageScope _sc(HLA_STAGE_CHAIN, s, 1);
     HLA_CUDA(hla::launch_chain_merge(ch, s), "chunk merge launch");
   }
+  side_join.armed = false;
   HLA_CUDA(cudaStreamWaitEvent(s, side->join, 0), "side stream join");
   side_lock.unlock();
   hla::ComposeArgs c{};
@@ -870,6 +934,7 @@ constexpr size_t kStaticScratchBytes = HLA_DECODE_STATIC_SCRATCH_BYTES;
 constexpr int kStaticMaxDevices = 64;
 std::mutex g_static_mu;
 void* g_static_ptr[kStaticMaxDevices] = {};
+unsigned long long g_static_ctx[kStaticMaxDevices] = {};
 }  // namespace
 
 static __device__ __align__(256) unsigned char hla_static_scratch[kStaticScratchBytes];
@@ -877,20 +942,25 @@ static __device__ __align__(256) unsigned char hla_static_scratch[kStaticScratch
 namespace {
 // Device address of hla_static_scratch on the current device.  The first call on
 // a device asks the runtime for the symbol's address (with that device current);
-// later calls reuse it.
+// later calls reuse it while the same CUDA context is current.  A different
+// context -- a non-primary one, or the primary context recreated after
+// cudaDeviceReset -- has its own copy of the array, so the address is looked up
+// again.
 hla_status static_scratch_ptr(void** out) {
   int dev = -1;
   HLA_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
   if (dev < 0 || dev >= kStaticMaxDevices)
     return fail(HLA_ERR_UNSUPPORTED, "device ordinal %d beyond %d", dev, kStaticMaxDevices);
   std::lock_guard<std::mutex> lk(g_static_mu);
-  if (g_static_ptr[dev] == nullptr) {
+  const unsigned long long ctx = current_context_id();
+  if (g_static_ptr[dev] == nullptr || ctx == 0 || ctx != g_static_ctx[dev]) {
     void* p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, hla_static_scratch);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(hla_static_scratch)");
     if (p == nullptr || ((uintptr_t)p & 255u) != 0)
       return fail(HLA_ERR_CUDA, "static scratch address %p is not 256-byte aligned", p);
     g_static_ptr[dev] = p;
+    g_static_ctx[dev] = current_context_id();  // the lookup makes the context current if none was
   }
   *out = g_static_ptr[dev];
   return HLA_OK;

@@ -263,6 +263,11 @@ hla_status hla_gate_support(const hla_config* cfg, const float* gates, float* ma
  * workspace: device, >= hla_prefill_workspace_bytes(cfg), 256-byte aligned.
  * Path: routing on a library side stream (forked from and joined back to `stream`
  * by events) beside the chunk transitions; then the composition and the read-out.
+ * The side stream is one per device, made on the first call (and again when a
+ * different CUDA context is current), and one process-wide lock is held while a
+ * call enqueues its fork, routing and join: concurrent calls on different streams
+ * are correct, but their routing stages run one after another on that stream.
+ * Every return after the fork, an error included, leaves `stream` joined to it.
  * With HLA_DECAY_CHANNEL the transitions and the read-out run the token rule per
  * chunk on CUDA cores.
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
@@ -308,6 +313,10 @@ hla_status hla_decode_step(const hla_config* cfg, hla_cache* cache, const void* 
  * No call allocates or frees device memory.
  * Set-up: the first call on a device (the current one) looks up the array's
  * device address and keeps it; make that first call before any stream capture.
+ * The address belongs to the CUDA context current at that call.  A call under a
+ * different context (a non-primary context, or the primary context recreated by
+ * cudaDeviceReset) looks it up again, which is again a set-up call: make it
+ * outside stream capture too.
  * Sharing: every call on a device writes the same array.  Nothing in it has to
  * start at zero, but calls whose kernels may overlap in time (different streams
  * or host threads) race on it; serialise them.

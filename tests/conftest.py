@@ -25,3 +25,22 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Worst parity error each test reached against its bar (max-abs on the float32
+    path, per-(sequence, head) relative L2 on the bf16 path)."""
+    try:
+        from tests import _parity as P
+    except Exception:  # pragma: no cover
+        return
+    if not P.MARGINS:
+        return
+    worst = {}
+    for test, what, kind, err, bar in P.MARGINS:
+        key = (test, what, kind)
+        if key not in worst or err / bar > worst[key][0] / worst[key][1]:
+            worst[key] = (err, bar)
+    terminalreporter.section("parity margins (worst per test; error / bar)")
+    for (test, what, kind), (err, bar) in sorted(worst.items()):
+        terminalreporter.write_line(f"{err:10.3e} / {bar:.0e}  {kind:16s} {what:28s} {test}")

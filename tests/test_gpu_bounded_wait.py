@@ -43,6 +43,6 @@ def test_expired_wait_is_reported_and_context_stays_usable(hla):
     o, gates, aidx, acnt = P.run_prefill(hla, w, inp)
     for h in range(w.H):
         r = P.oracle_prefill_head(w, inp, 0, h)
-        assert np.abs(P.np64(o[0, :, h]) - r.o).max() <= P.TOL_F32_MAXABS
+        P.check_f32(P.np64(o[0, :, h]), r.o)
     st, code = hla.hla_device_status(clear=True)
     assert st == hla.HLA_OK

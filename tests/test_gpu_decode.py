@@ -78,9 +78,9 @@ def test_decode_chain_matches_oracle(hla, dtype, d, mode, thr, route):
     got = np.stack([e[0] for e in errs])
     ref = np.stack([e[1] for e in errs])
     if dtype == "f32":
-        assert np.abs(got - ref).max() <= P.TOL_F32_MAXABS
+        P.check_f32(got, ref)
     else:
-        assert P.rel_l2(got, ref) <= P.TOL_BF16_RELL2
+        P.check_bf16(got, ref, layout="steps", nh=len(heads))
     st, code = hla.hla_device_status()
     assert st == 0 and code == 0
     # counters and the closed chunk's key pool
@@ -139,8 +139,8 @@ def test_decode_factored_cache_matches_oracle(hla, mode, thr, route):
                                 float(tk["alpha"][b, h]), float(tk["beta"][b, h]),
                                 None if qr is None else P.np32(qr[b, h]), None if kr is None else P.np32(kr[b, h])))
     got, dense, ref = np.stack(got), np.stack(dense), np.stack(ref)
-    assert P.rel_l2(got, ref) <= P.TOL_BF16_RELL2
-    assert P.rel_l2(got, dense) <= P.TOL_BF16_RELL2
+    P.check_bf16(got, ref, layout="steps", nh=len(heads))
+    P.check_bf16(got, dense, "factored vs dense cache", layout="steps", nh=len(heads))
     st, code = hla.hla_device_status()
     assert st == 0 and code == 0
     n = caches["factored"].view("n_chunks", (w.B,), torch.int32).cpu().tolist()
@@ -188,9 +188,9 @@ def test_decode_ragged_positions(hla, dtype, d, fmt):
                                 P.np32(kr[b, h])))
     got, ref = np.stack(got), np.stack(ref)
     if dtype == "f32":
-        assert np.abs(got - ref).max() <= P.TOL_F32_MAXABS
+        P.check_f32(got, ref)
     else:
-        assert P.rel_l2(got, ref) <= P.TOL_BF16_RELL2
+        P.check_bf16(got, ref, layout="steps", nh=len(heads))
     st, code = hla.hla_device_status()
     assert st == 0 and code == 0
     n = cache.view("n_chunks", (2,), torch.int32).cpu().tolist()
@@ -246,7 +246,7 @@ def test_full_size_decode_sampled(hla):
                                                  w.bias, w.thr, w.gate_mode)
             ref = head.step(P.np64(tok["q"][b, h]), P.np64(tok["k"][b, h]), P.np64(tok["v"][b, h]),
                             float(tok["alpha"][b, h]), float(tok["beta"][b, h]))
-            assert P.rel_l2(P.np64(o[b, h]), ref) <= P.TOL_BF16_RELL2
+            P.check_bf16(P.np64(o[b, h]), ref)
     finally:
         del cache
         torch.cuda.empty_cache()

@@ -37,9 +37,9 @@ def _check_prefill(hla, w, tol_f32=True):
             P.check_routing_exact(r, gates, aidx, acnt, b, h)
     got = P.np64(o)
     if w.dtype == "f32":
-        assert np.abs(got - ref).max() <= P.TOL_F32_MAXABS
+        P.check_f32(got, ref)
     else:
-        assert P.rel_l2(got, ref) <= P.TOL_BF16_RELL2
+        P.check_bf16(got, ref, layout="bthd")
     st, code = hla.hla_device_status()
     assert st == 0 and code == 0
 
@@ -81,9 +81,9 @@ def test_gates_one_is_native_gdn(hla, dtype, C):
                                       P.np64(inp["beta"][b, :, h]))
             got = P.np64(o[b, :, h])
             if dtype == "f32":
-                assert np.abs(got - ref).max() <= P.TOL_F32_MAXABS
+                P.check_f32(got, ref)
             else:
-                assert P.rel_l2(got, ref) <= P.TOL_BF16_RELL2
+                P.check_bf16(got, ref)
 
 
 @pytest.mark.parametrize("dtype,d,C", [("f32", 64, 128), ("bf16", 128, 256)])
@@ -105,11 +105,11 @@ def test_gdn_chunk_transitions_long(hla, dtype, d, C):
             Ar, Br = ho.chunk_transition(P.np64(inp["k"][0, sl, h]), P.np64(inp["v"][0, sl, h]),
                                          P.np64(inp["alpha"][0, sl, h]), P.np64(inp["beta"][0, sl, h]))
             if dtype == "f32":
-                assert np.abs(A[0, h, c] - Ar).max() <= P.TOL_F32_MAXABS
-                assert np.abs(Bm[0, h, c] - Br).max() <= P.TOL_F32_MAXABS
+                P.check_f32(A[0, h, c], Ar)
+                P.check_f32(Bm[0, h, c], Br)
             else:
-                assert P.rel_l2(A[0, h, c], Ar) <= 1e-2
-                assert P.rel_l2(Bm[0, h, c], Br) <= 1e-2
+                P.check_bf16(A[0, h, c], Ar, "transition", tol=1e-2)
+                P.check_bf16(Bm[0, h, c], Br, "transition", tol=1e-2)
 
 
 @pytest.mark.parametrize("dtype,d,C,T0,steps", [
@@ -147,9 +147,9 @@ def test_decode_long_chunks(hla, dtype, d, C, T0, steps):
             got.append(o[b, h])
     got, ref = np.stack(got), np.stack(ref)
     if dtype == "f32":
-        assert np.abs(got - ref).max() <= P.TOL_F32_MAXABS
+        P.check_f32(got, ref)
     else:
-        assert P.rel_l2(got, ref) <= P.TOL_BF16_RELL2
+        P.check_bf16(got, ref, layout="steps", nh=len(heads))
     st, code = hla.hla_device_status()
     assert st == 0 and code == 0
     n = cache.view("n_chunks", (w.B,), torch.int32).cpu()
@@ -173,4 +173,4 @@ def test_full_size_c256_window32_sampled(hla):
         r = P.oracle_prefill_head(w, inp, 0, h, query_chunks=sample)
         P.check_routing_exact(r, gates, aidx, acnt, 0, h)
         rows = np.concatenate([np.arange(256 * i, 256 * i + 256) for i in sample])
-        assert P.rel_l2(P.np64(o[0, rows, h]), r.o[rows]) <= P.TOL_BF16_RELL2
+        P.check_bf16(P.np64(o[0, rows, h]), r.o[rows])

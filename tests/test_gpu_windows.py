@@ -34,9 +34,9 @@ def _check_prefill(hla, w):
             P.check_routing_exact(r, gates, aidx, acnt, b, h)
     got = P.np64(o)
     if w.dtype == "f32":
-        assert np.abs(got - ref).max() <= P.TOL_F32_MAXABS
+        P.check_f32(got, ref)
     else:
-        assert P.rel_l2(got, ref) <= P.TOL_BF16_RELL2
+        P.check_bf16(got, ref, layout="bthd")
     st, code = hla.hla_device_status()
     assert st == 0 and code == 0
     return gates
@@ -126,9 +126,9 @@ def test_decode_window_gates(hla, dtype, d, C, window, T0, steps, fmt):
             got.append(o[b, h])
     got, ref = np.stack(got), np.stack(ref)
     if dtype == "f32":
-        assert np.abs(got - ref).max() <= P.TOL_F32_MAXABS
+        P.check_f32(got, ref)
     else:
-        assert P.rel_l2(got, ref) <= P.TOL_BF16_RELL2
+        P.check_bf16(got, ref, layout="steps", nh=len(heads))
     st, code = hla.hla_device_status()
     assert st == 0 and code == 0
     W = C // window

@@ -5,7 +5,8 @@ Two caches start from the same prefill (the second is a byte copy of the first);
 each then takes the same two decode tokens, one entry point per cache.  The first
 token fills the open chunk, so that step also closes it into the cache; the second
 opens the next chunk.  Outputs must agree within the parity tolerances, and the
-cache counters exactly.  The file is named to be collected last, and it also
+cache counters exactly; around the second static call the device's free memory and
+torch's allocated bytes must not move.  The file is named to be collected last, and it also
 passes alone in a fresh process (the first call on the device does the set-up)."""
 import pytest
 import torch
@@ -43,7 +44,7 @@ def test_static_scratch_decode_matches_workspace_decode(hla, dtype, d, mode, thr
     dcfg = hla.make_config(w.B, w.H, 1, 64, d, dtype, mode, w.tau, w.bias, w.thr)
     toks = syn.make_decode_tokens(w, 2)
     gen = torch.Generator().manual_seed(5)
-    for tk in toks:
+    for step, tk in enumerate(toks):
         g = {k: v.cuda().contiguous() for k, v in tk.items()}
         qr = kr = None
         if route:
@@ -54,14 +55,21 @@ def test_static_scratch_decode_matches_workspace_decode(hla, dtype, d, mode, thr
         o_st = torch.empty_like(g["q"])
         hla.hla_decode_step(dcfg, ref_cache, g["q"], g["k"], g["v"], g["alpha"], g["beta"], o_ref,
                             q_route=qr, k_route=kr)
+        torch.cuda.synchronize()
+        before = (torch.cuda.memory_allocated(), torch.cuda.mem_get_info()[0])
         hla.hla_decode_step_static(dcfg, st_cache, g["q"], g["k"], g["v"], g["alpha"], g["beta"], o_st,
                                    q_route=qr, k_route=kr)
         torch.cuda.synchronize()
+        after = (torch.cuda.memory_allocated(), torch.cuda.mem_get_info()[0])
+        if step > 0:
+            # past the set-up of the first call in this process: no device memory
+            # taken by torch's allocator or by any other allocation on the device
+            assert after == before, (before, after)
         a, b = P.np64(o_st), P.np64(o_ref)
         if dtype == "f32":
-            assert abs(a - b).max() <= P.TOL_F32_MAXABS
+            P.check_f32(a, b, "static vs workspace decode")
         else:
-            assert P.rel_l2(a, b) <= P.TOL_BF16_RELL2
+            P.check_bf16(a, b, "static vs workspace decode", layout="bhd")
     for field in ("n_chunks", "m_partial"):
         got = st_cache.view(field, (w.B,), torch.int32).cpu()
         ref = ref_cache.view(field, (w.B,), torch.int32).cpu()
