@@ -244,11 +244,110 @@ def build_decode_cache(hla, syn, torch, w, max_chunks, group=8, cache_format="de
         holder = cache.slice(b0, group)
         o = torch.empty_like(ctx["q"])
         hla.hla_prefill(gcfg, ctx["q"], ctx["k"], ctx["v"], ctx["alpha"], ctx["beta"], o, cache=holder,
-                        workspace=ws)
+                        q_route=ctx.get("q_route"), k_route=ctx.get("k_route"), workspace=ws)
         del ctx, o
     torch.cuda.synchronize()
     del ws
     return cache, first_ctx
+
+
+def _stage_avg(stages, name):
+    ms, n = stages.get(name, (0.0, 0))
+    return ms / n if n else None
+
+
+def measure_decode_planted(hla, syn, torch, stream, l2_flush, steps, warmup):
+    """The planted 32K decode step (the step of the 32K decode with planted route
+    inputs: about 4 of the 512 cached chunks active per (sequence, head)).  Timed on
+    its own after the main loop: `steps` steps with CUDA events on the launching
+    stream, the L2 flushed (untimed) before each.  The active chunks are counted on
+    the first warm-up step from its decode workspace, pre-filled with a sentinel:
+    the entries the kernel writes are exactly the active ones."""
+    wd = syn.DECODE_32K_PLANTED
+    max_chunks = wd.T // wd.C + 1
+    cache, _ = build_decode_cache(hla, syn, torch, wd, max_chunks, group=8)
+    dcfg = hla.make_config(wd.B, wd.H, 1, wd.C, wd.d, wd.dtype, wd.gate_mode, wd.tau, wd.bias, wd.thr)
+    nbytes = hla.decode_workspace_bytes(dcfg, max_chunks)
+    dws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    toks = [{k: v.cuda() for k, v in t.items()} for t in syn.make_decode_tokens(wd, warmup + steps)]
+    n = wd.B * wd.H * max_chunks
+    od = torch.empty_like(toks[0]["q"])
+    active = None
+    for i in range(warmup):
+        t = toks[i]
+        if i == 0:
+            dws.view(torch.int32).fill_(-7)
+        hla.hla_decode_step(dcfg, cache, t["q"], t["k"], t["v"], t["alpha"], t["beta"], od, q_route=t["q_route"],
+                            k_route=t["k_route"], workspace=dws)
+        if i == 0:
+            active = (dws.view(torch.int32)[:n] != -7).view(wd.B, wd.H, max_chunks).sum(-1).cpu()
+        l2_flush()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    hla.hla_profile_read(reset=True)
+    hla.hla_profile_enable(True)
+    for s_ in range(steps):
+        t = toks[warmup + s_]
+        ev[s_][0].record(stream)
+        hla.hla_decode_step(dcfg, cache, t["q"], t["k"], t["v"], t["alpha"], t["beta"], od, q_route=t["q_route"],
+                            k_route=t["k_route"], workspace=dws)
+        ev[s_][1].record(stream)
+        l2_flush()
+    torch.cuda.synchronize()
+    hla.hla_profile_enable(False)
+    stages = hla.hla_profile_read(reset=True)
+    ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+    n_ctx = wd.T // wd.C
+    per_chunk = 2 * wd.d * wd.d * 2
+    act_total = int(active.sum())
+    nbytes_alg = act_total * per_chunk + wd.B * wd.H * n_ctx * wd.d * 4
+    kern = _stage_avg(stages, "decode")
+    del cache, dws
+    torch.cuda.empty_cache()
+    return wd, ms, kern, act_total, nbytes_alg, stages
+
+
+def measure_sparse_prefill(hla, syn, torch, stream, l2_flush, steps, warmup):
+    """The long sparse prefill (B=1, H=32, T=131072, C=64, d=128, bf16, planted
+    route inputs, threshold 0.05), timed on its own after the main loop: `steps`
+    prefills with CUDA events on the launching stream, the L2 flushed (untimed)
+    before each.  Inputs are generated on the device (5 x 1 GiB)."""
+    wp = syn.SPARSE_LONG
+    inp = syn.make_gdn_inputs(wp, device="cuda")
+    inp["q_route"], inp["k_route"] = syn.make_route_inputs(wp, device="cuda")
+    cfg = hla.make_config(wp.B, wp.H, wp.T, wp.C, wp.d, wp.dtype, wp.gate_mode, wp.tau, wp.bias, wp.thr)
+    ws = torch.empty(hla.prefill_workspace_bytes(cfg), dtype=torch.uint8, device="cuda")
+    o = torch.empty_like(inp["q"])
+    N = wp.N
+    acnt = torch.empty((wp.B, wp.H, N), dtype=torch.int32, device="cuda")
+
+    def run(**kw):
+        hla.hla_prefill(cfg, inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], o, q_route=inp["q_route"],
+                        k_route=inp["k_route"], workspace=ws, **kw)
+
+    for _ in range(warmup):
+        run()
+        l2_flush()
+    run(active_cnt_out=acnt, active_idx_out=torch.empty((wp.B, wp.H, N, N), dtype=torch.int32, device="cuda"))
+    torch.cuda.synchronize()
+    pairs = int(acnt.sum().item())
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    hla.hla_profile_read(reset=True)
+    hla.hla_profile_enable(True)
+    for s_ in range(steps):
+        l2_flush()
+        ev[s_][0].record(stream)
+        run()
+        ev[s_][1].record(stream)
+    torch.cuda.synchronize()
+    hla.hla_profile_enable(False)
+    stages = hla.hla_profile_read(reset=True)
+    ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+    # the CPU oracle's sample: the first 16384 tokens of four heads
+    sample = {k: inp[k][:, :16384, :4].cpu() for k in ("q", "k", "v", "alpha", "beta", "q_route", "k_route")}
+    del inp, ws, o
+    torch.cuda.empty_cache()
+    return wp, ms, pairs, stages, sample
 
 
 def run_ours(args):
@@ -514,8 +613,56 @@ def run_ours(args):
         "gpu_launches": launches,
         "clocks": clocks.summary(),
     }
+    sparse_sample = None
+    if not args.no_extra_lines:
+        del cache, dws
+        torch.cuda.empty_cache()
+        # the planted 32K decode: about 4 active chunks per (sequence, head)
+        wdp, ms_dp, kern_dp, act_dp, bytes_dp, st_dp = measure_decode_planted(
+            hla, syn, torch, stream, l2_flush, args.steps, args.warmup)
+        ms_dp, kern_dp = max_over_ranks([ms_dp, kern_dp or 0.0], device="cuda")
+        gbs_dp = bytes_dp / (kern_dp * 1e-3) / 1e9 if kern_dp > 0 else None
+        out["decode_sparse"] = {
+            "workload": wdp.name, "value": whole_job_rate(wdp.B, ms_dp, world), "unit": "tokens/s",
+            "ms_per_step": ms_dp, "active_chunks_mean": act_dp / (wdp.B * wdp.H),
+            "roofline": {"kernel": "decode_main", "bound": "hbm", "achieved": gbs_dp, "peak": hbm_gbs,
+                         "unit": "GB/s", "frac": (gbs_dp / hbm_gbs) if gbs_dp else None,
+                         "peak_source": f"{peak_src} HBM copy",
+                         "datasheet": {"peak": DATASHEET_HBM_GBS,
+                                       "frac": (gbs_dp / DATASHEET_HBM_GBS) if gbs_dp else None},
+                         "algorithmic": f"{bytes_dp:.4g} bytes per launch ({act_dp} active A_j/B_j of 64 KiB, "
+                                        f"counted on the first warm-up step, + all {wdp.T // wdp.C} key pools of "
+                                        f"512 B per sequence and head)", "traffic": None},
+            "stages_ms_per_step": {k: v[0] / args.steps for k, v in st_dp.items() if v[1]}}
+        # the long sparse prefill (B=1, H=32, T=131072, planted, threshold 0.05)
+        wsp, ms_sp, pairs_sp, st_sp, sparse_sample = measure_sparse_prefill(
+            hla, syn, torch, stream, l2_flush, args.steps, args.warmup)
+        (ms_sp,) = max_over_ranks([ms_sp], device="cuda")
+        bthd = wsp.B * wsp.T * wsp.H * wsp.d
+        n_sub = wsp.T // 64
+        flops_sp = pairs_sp * 2.0 * wsp.d ** 3 + wsp.B * wsp.H * n_sub * (FLOP_TRANSITION + FLOP_READOUT)
+        ab_bytes = wsp.B * wsp.H * (wsp.T // wsp.C) * 2 * wsp.d * wsp.d * 2
+        bytes_sp = 6 * bthd * 2 + 2 * ab_bytes   # q, k, v, route inputs in, o out; A/B written once, read once
+        tf_sp = flops_sp / (ms_sp * 1e-3) / 1e12
+        gbs_sp = bytes_sp / (ms_sp * 1e-3) / 1e9
+        comp_sp = _stage_avg(st_sp, "compose")
+        out["sparse_prefill"] = {
+            "workload": wsp.name, "value": whole_job_rate(wsp.B * wsp.T, ms_sp, world), "unit": "tokens/s",
+            "ms": ms_sp, "active_pairs": pairs_sp,
+            "roofline_tensor": {"achieved": tf_sp, "peak": bf16_tf, "unit": "TFLOP/s", "frac": tf_sp / bf16_tf,
+                                "peak_source": f"{peak_src} bf16 dense (burst)",
+                                "datasheet": {"peak": DATASHEET_BF16_TFLOPS, "frac": tf_sp / DATASHEET_BF16_TFLOPS},
+                                "algorithmic": f"{flops_sp:.4g} flop per prefill ({pairs_sp} active pairs x 2 d^3 "
+                                               f"+ transitions and read-out of {n_sub} chunks per head)"},
+            "roofline_hbm": {"achieved": gbs_sp, "peak": hbm_gbs, "unit": "GB/s", "frac": gbs_sp / hbm_gbs,
+                             "peak_source": f"{peak_src} HBM copy",
+                             "datasheet": {"peak": DATASHEET_HBM_GBS, "frac": gbs_sp / DATASHEET_HBM_GBS},
+                             "algorithmic": f"{bytes_sp:.4g} bytes per prefill (q, k, v, two route inputs read "
+                                            f"and o written once; every A_c/B_c written once and read once)"},
+            "compose_tflops": (pairs_sp * 2.0 * wsp.d ** 3 / (comp_sp * 1e-3) / 1e12) if comp_sp else None,
+            "stages_ms_per_step": {k: v[0] / args.steps for k, v in st_sp.items() if v[1]}}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(inp, wp, wd, ctx0, toks_host, torch)
+        out["cpu_baseline"] = cpu_baseline(inp, wp, wd, ctx0, toks_host, torch, sparse_sample)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -554,6 +701,38 @@ def _oracle_decode_worker(job):
     t0 = time.perf_counter()
     head.step(*tok)
     return time.perf_counter() - t0
+
+
+_REASSOC_TRANS = None
+
+
+def _oracle_decode_reassoc_worker(job):
+    """The decode read-out of `pairs` (sequence, head) pairs in the oracle's
+    reassociated mat-vec form (decode_output_backward) over every cached chunk;
+    returns the wall time (s).  The cached transitions are seeded random matrices
+    of the cache's shape (the work does not depend on their values), made once per
+    worker outside the timed region."""
+    global _REASSOC_TRANS
+    _limit_blas_threads()
+    from oracle import hla_oracle as ho
+    pairs, n_chunks, d, seed = job
+    if _REASSOC_TRANS is None or len(_REASSOC_TRANS) != n_chunks:
+        rng = np.random.default_rng(seed)
+        _REASSOC_TRANS = [(rng.standard_normal((d, d)) / d, rng.standard_normal((d, d)) / d) for _ in range(n_chunks)]
+    rng = np.random.default_rng(seed + 1)
+    g = rng.uniform(0.05, 0.2, n_chunks)
+    x = rng.standard_normal(d)
+    y0 = np.zeros(d)
+    active = list(range(n_chunks))
+    t0 = time.perf_counter()
+    for _ in range(pairs):
+        ho.decode_output_backward(_REASSOC_TRANS, g, active, x, y0)
+    return time.perf_counter() - t0
+
+
+def _oracle_sparse_head_worker(job):
+    """One head of the long sparse prefill by the oracle; returns its wall time (s)."""
+    return _oracle_prefill_worker(job)
 
 
 class OraclePool:
@@ -606,10 +785,11 @@ def _cpu_model():
     return "unknown CPU"
 
 
-def cpu_baseline(inp, wp, wd, ctx0, toks_host, torch):
+def cpu_baseline(inp, wp, wd, ctx0, toks_host, torch, sparse_sample=None):
     """The oracle on the host cores: the full prefill (every (sequence, head) of the
-    prompt, one per worker process) and one decode step of a sample of (sequence,
-    head) pairs."""
+    prompt, one per worker process), one decode step of a sample of (sequence,
+    head) pairs in the definition form, the whole decode step in the reassociated
+    mat-vec form, and (given its sample) four heads of the long sparse prefill."""
     pairs_p = [(b, h) for b in range(wp.B) for h in range(wp.H)]
     pairs_d = [(b, h) for b in range(min(2, wd.B)) for h in range(8)]
     pool = OraclePool(max(len(pairs_p), len(pairs_d)))
@@ -618,15 +798,43 @@ def cpu_baseline(inp, wp, wd, ctx0, toks_host, torch):
         pool.map(_oracle_prefill_worker, _prefill_jobs(inp, wp, pairs_p))
         tp = time.perf_counter() - t0
         td = pool.map(_oracle_decode_worker, _decode_jobs(ctx0, wd, toks_host[0], pairs_d))
+        # the whole decode step (all B x H pairs) in the reassociated form, split over the workers
+        n_pairs = wd.B * wd.H
+        per = [n_pairs // pool.n + (1 if i < n_pairs % pool.n else 0) for i in range(pool.n)]
+        # each worker times its own share (its set-up of the cached matrices excluded);
+        # the step takes as long as the slowest share
+        tr = max(pool.map(_oracle_decode_reassoc_worker, [(p_, wd.T // wd.C, wd.d, 11) for p_ in per]))
+        sparse = None
+        if sparse_sample is not None:
+            import hla_synth as syn
+            ws_ = syn.SPARSE_LONG
+            nh, ts_ = sparse_sample["q"].shape[2], sparse_sample["q"].shape[1]
+            ts = pool.map(_oracle_sparse_head_worker,
+                          _prefill_jobs(sparse_sample, ws_.with_(T=ts_), [(0, h) for h in range(nh)]))
+            # head-tokens per second on `cores` workers, extrapolated linearly to the whole
+            # prompt (the token rule dominates the oracle's time on this sparse workload)
+            rate = pool.n * ts_ / max(ts)
+            sparse = {"value": rate * ws_.T / (ws_.H * ws_.T), "unit": "tokens/s", "kind": "oracle",
+                      "sample": f"the first {ts_} tokens of {nh} of the {ws_.H} heads, one per worker (slowest "
+                                f"{max(ts):.1f} s); tokens/s of the whole prompt on {pool.n} workers, scaled "
+                                f"linearly in tokens and heads"}
     finally:
         pool.close()
     td_mean = statistics.mean(td)
-    return {"value": wp.B * wp.T / tp, "unit": "tokens/s", "cores": pool.n, "kind": "oracle",
+    res = {"value": wp.B * wp.T / tp, "unit": "tokens/s", "cores": pool.n, "kind": "oracle",
             "sample": f"prefill: the whole prompt ({wp.B * wp.H} (sequence, head) pairs of T={wp.T}, "
                       f"{tp:.1f} s wall on {pool.n} worker processes); decode: one step of {len(pairs_d)} "
                       f"(sequence, head) pairs of the 32K context ({td_mean:.3f} s each), tokens/s = cores / "
                       f"(H x time per pair); {_cpu_model()}",
-            "decode": {"value": pool.n / (wd.H * td_mean), "unit": "tokens/s"}}
+            "decode": {"value": pool.n / (wd.H * td_mean), "unit": "tokens/s"},
+            "decode_reassociated": {"value": wd.B / tr, "unit": "tokens/s", "kind": "oracle (reassociated mat-vec form)",
+                                    "sample": f"the whole step: {wd.B * wd.H} (sequence, head) pairs x "
+                                              f"{wd.T // wd.C} cached chunks by decode_output_backward on "
+                                              f"{pool.n} workers (slowest share {tr:.2f} s); cached "
+                                              f"transitions are seeded matrices of the cache's shape"}}
+    if sparse is not None:
+        res["sparse_prefill"] = sparse
+    return res
 
 
 def run_reference(args):
@@ -685,6 +893,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra-lines", action="store_true",
+                    help="skip the planted 32K decode and the long sparse prefill (timed after the main loop)")
     # smaller variants for profiling captures (the default is the full workload)
     ap.add_argument("--prefill-T", type=int, default=None, help="prefill tokens (default: the workload's)")
     ap.add_argument("--prefill-workload", choices=sorted(PREFILL_WORKLOADS), default="dense",

@@ -221,7 +221,7 @@ def hla_prefill(cfg, q, k, v, alpha, beta, o, q_route=None, k_route=None, user_g
                              _ptr(q_route), _ptr(k_route), _ptr(user_gates), _ptr(o), _ptr(gates_out),
                              _ptr(active_idx_out), _ptr(active_cnt_out),
                              ctypes.byref(cache.struct) if cache is not None else None,
-                             _ptr(workspace), workspace.numel(), _stream(stream)))
+                             _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
     return o
 
 
@@ -232,7 +232,7 @@ def hla_decode_step(cfg, cache: Cache, q, k, v, alpha, beta, o, q_route=None, k_
                                 device=q.device)
     _check(lib().hla_decode_step(ctypes.byref(cfg), ctypes.byref(cache.struct), _ptr(q), _ptr(k), _ptr(v),
                                  _ptr(alpha), _ptr(beta), _ptr(q_route), _ptr(k_route), _ptr(o),
-                                 _ptr(workspace), workspace.numel(), _stream(stream)))
+                                 _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
     return o
 
 

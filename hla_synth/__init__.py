@@ -73,8 +73,13 @@ DECODE_32K = Workload("decode_bf16_64seq_ctx32768_H16_C64_d128_thr0.05", 64, 16,
                       1.0, -2.0, 0.05, seed=3)
 SPARSE_LONG = Workload("sparse_prefill_bf16_B1_H32_T131072_C64_d128_thr0.05", 1, 32, 131072, 64, 128,
                        "bf16", 1.0, -4.0, 0.05, route="planted", seed=5)
+# The decode step of DECODE_32K with planted route inputs (the recipe of SPARSE_LONG):
+# the open chunk matches about 512 / 128 = 4 of the 512 cached chunks.
+DECODE_32K_PLANTED = Workload("decode_bf16_64seq_ctx32768_H16_C64_d128_thr0.05_planted", 64, 16, 32768, 64, 128,
+                              "bf16", 1.0, -4.0, 0.05, route="planted", seed=4)
 
-WORKLOADS = {w.name: w for w in (TINY_F32, GDN_REDUCTION, PREFILL_0P8B, DECODE_32K, SPARSE_LONG)}
+WORKLOADS = {w.name: w for w in (TINY_F32, GDN_REDUCTION, PREFILL_0P8B, DECODE_32K, SPARSE_LONG,
+                                 DECODE_32K_PLANTED)}
 
 
 def torch_dtype(w: Workload):
@@ -149,7 +154,8 @@ def make_user_gates(w: Workload, device="cpu", seed: int | None = None):
 
 def make_decode_tokens(w: Workload, steps: int, device="cpu", seed: int | None = None):
     """Per-step new tokens: list of dicts with q, k, v [B,H,d], alpha [B,H] (or [B,H,d]
-    with channel-wise decay), beta [B,H]."""
+    with channel-wise decay), beta [B,H].  With planted route inputs each dict also
+    holds q_route, k_route [B,H,d] (see ``make_decode_route_tokens``)."""
     g = torch.Generator(device=device)
     g.manual_seed((w.seed if seed is None else seed) + 4242)
     dt = torch_dtype(w)
@@ -163,13 +169,44 @@ def make_decode_tokens(w: Workload, steps: int, device="cpu", seed: int | None =
             - 3.0)).float()
         b = torch.sigmoid(torch.randn((w.B, w.H), generator=g, device=device)).float()
         out.append(dict(q=q.to(dt), k=k.to(dt), v=v.to(dt), alpha=a, beta=b))
+    if w.route == "planted":
+        for tok, (qr, kr) in zip(out, make_decode_route_tokens(w, steps, device=device, seed=seed)):
+            tok["q_route"], tok["k_route"] = qr, kr
+    return out
+
+
+def make_decode_route_tokens(w: Workload, steps: int, device="cpu", seed: int | None = None):
+    """Planted route inputs of the decode tokens that follow a w.T-token context:
+    list of (q_route, k_route) [B,H,d].  Token t of the decode (position w.T + t)
+    belongs to chunk (w.T + t) // C; each such chunk gets a topic c ~ U{0..topics-1}
+    per (sequence, head), and its route tokens are s e_c + 0.1 N(0, I) (s = 9.51),
+    the recipe of ``make_route_inputs``."""
+    assert w.route == "planted", w.route
+    g = torch.Generator(device=device)
+    g.manual_seed((w.seed if seed is None else seed) + 2718281)
+    dt = torch_dtype(w)
+    s = 9.51
+    first = w.T // w.C
+    n_chunks = (w.T + steps - 1) // w.C - first + 1
+    topic = torch.randint(0, w.topics, (n_chunks, w.B, w.H), generator=g, device=device)
+    onehot = torch.nn.functional.one_hot(topic, w.d).float() * s   # [n_chunks, B, H, d]
+    out = []
+    for t in range(steps):
+        c = (w.T + t) // w.C - first
+        pair = []
+        for _ in range(2):
+            eps = torch.randn((w.B, w.H, w.d), generator=g, device=device) * 0.1
+            pair.append((onehot[c] + eps).to(dt))
+        out.append((pair[0], pair[1]))
     return out
 
 
 def make_context_group(w: Workload, b0: int, nb: int, device="cuda"):
     """Decode context (prompt) of sequences b0 .. b0+nb-1, generated on ``device``
     with a generator seeded by (seed, b0): q, k, v [nb, T, H, d], alpha, beta
-    [nb, T, H].  Used to build large decode caches group by group."""
+    [nb, T, H]; with spread or planted route inputs also q_route, k_route
+    [nb, T, H, d] (``make_route_inputs`` seeded by (seed, b0)).  Used to build large
+    decode caches group by group."""
     g = torch.Generator(device=device)
     g.manual_seed(w.seed * 1000003 + b0)
     shape = (nb, w.T, w.H, w.d)
@@ -183,4 +220,7 @@ def make_context_group(w: Workload, b0: int, nb: int, device="cuda"):
         a_raw = torch.randn((nb, w.T, w.H, w.d), generator=g, device=device)
     alpha = torch.exp(-torch.nn.functional.softplus(a_raw - 3.0)).float()
     beta = torch.sigmoid(b_raw).float()
-    return dict(q=q, k=k, v=v, alpha=alpha, beta=beta)
+    out = dict(q=q, k=k, v=v, alpha=alpha, beta=beta)
+    if w.route != "default":
+        out["q_route"], out["k_route"] = make_route_inputs(w, B=nb, device=device, seed=w.seed * 1000003 + b0 + 17)
+    return out

@@ -250,3 +250,57 @@ def test_full_size_decode_sampled(hla):
     finally:
         del cache
         torch.cuda.empty_cache()
+
+
+def test_full_size_planted_decode_sampled(hla):
+    """The planted 32K decode step at full size (64 sequences x 32768-token contexts,
+    H=16, d=128, bf16, bias -4, threshold 0.05, planted route inputs: the open chunk
+    matches about 4 of the 512 cached chunks).  The step's active lists are read
+    from the decode workspace (pre-filled with a sentinel, so the entries the kernel
+    wrote are exactly the active ones) and must equal the oracle's, with bit-exact
+    gates; sampled (sequence, head) outputs are compared with the oracle's decode
+    head built from the same context (forward composition over the active chunks)."""
+    import os
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+    w = syn.DECODE_32K_PLANTED
+    max_chunks = w.T // w.C + 1
+    cache, ctx = bench.build_decode_cache(hla, syn, torch, w, max_chunks, group=8)
+    try:
+        dcfg = hla.make_config(w.B, w.H, 1, w.C, w.d, w.dtype, w.gate_mode, w.tau, w.bias, w.thr)
+        tok = syn.make_decode_tokens(w, 1)[0]
+        g = {k: v.cuda().contiguous() for k, v in tok.items()}
+        o = torch.empty_like(g["q"])
+        nbytes = hla.decode_workspace_bytes(dcfg, max_chunks)
+        ws = torch.full((nbytes // 4,), -7, dtype=torch.int32, device="cuda")
+        hla.hla_decode_step(dcfg, cache, g["q"], g["k"], g["v"], g["alpha"], g["beta"], o,
+                            q_route=g["q_route"], k_route=g["k_route"], workspace=ws)
+        torch.cuda.synchronize()
+        st, code = hla.hla_device_status()
+        assert st == hla.HLA_OK, code
+        n = w.B * w.H * max_chunks
+        g_off = ((n * 4 + 255) // 256) * 256 // 4
+        idx = ws[:n].view(w.B, w.H, max_chunks).cpu()
+        gts = ws[g_off:g_off + n].view(torch.float32).view(w.B, w.H, max_chunks).cpu()
+        counts = (idx != -7).sum(-1)
+        assert 1.0 <= counts.float().mean() <= 12.0, counts.float().mean()
+        for (b, h) in ((0, 0), (1, 9), (0, 15)):
+            f = lambda name: P.np64(ctx[name][b, :, h])
+            r32 = lambda name: P.np32(ctx[name][b, :, h])
+            head = ho.HlaDecodeHead.from_prefill(f("q"), f("k"), f("v"), f("alpha"), f("beta"), w.C, w.tau,
+                                                 w.bias, w.thr, w.gate_mode, r32("q_route"), r32("k_route"))
+            ref = head.step(P.np64(tok["q"][b, h]), P.np64(tok["k"][b, h]), P.np64(tok["v"][b, h]),
+                            float(tok["alpha"][b, h]), float(tok["beta"][b, h]),
+                            P.np32(tok["q_route"][b, h]), P.np32(tok["k_route"][b, h]))
+            P.check_bf16(P.np64(o[b, h]), ref, "planted decode output")
+            # the oracle's gates of this step: its open chunk now holds the new token
+            g_ref = head.gates()
+            act_ref = head.active(g_ref)
+            c = int(counts[b, h])
+            assert idx[b, h, :c].tolist() == [int(j) for j in act_ref]
+            assert np.array_equal(gts[b, h, :c].numpy().view(np.uint32),
+                                  np.asarray(g_ref[act_ref], np.float32).view(np.uint32))
+    finally:
+        del cache
+        torch.cuda.empty_cache()
