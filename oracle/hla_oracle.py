@@ -139,6 +139,58 @@ def chunk_transition_wy(k, v, alpha, beta):
     return A, B, Wb, Ub, ell
 
 
+def chunk_transition_wy_channel(k, v, alpha, beta):
+    """(A, B) of one chunk under channel-wise decay (alpha [n, d_k]) through the
+    chunkwise WY/UT form with the decays folded into the keys.
+
+    With l_t = sum_{s<=t} log alpha_s (a vector over key channels), gamma_t = exp(l_t):
+    the state after token t from S_0 is S_0 Diag(gamma_t) + sum_{s<=t} u_s (k_s o
+    gamma_t / gamma_s)^T with u_t = beta_t (v_t - S_{t-1} Diag(alpha_t) k_t).  Writing
+    kt_t = gamma_t o k_t and kh_s = k_s / gamma_s, the coupling of u_t to u_s (s < t) is
+    beta_t (kt_t . kh_s), so
+      L = strictly-lower part of diag(beta) Kt Kh^T
+      T = (I + L)^{-1} diag(beta)
+      Wb = T Kt,  Ub = T V,  Kc = rows k_s o gamma_n / gamma_s
+      A = Diag(gamma_n) - Wb^T Kc,  B = Ub^T Kc.
+    With equal channels it is ``chunk_transition_wy``.  The entries of Kt Kh^T are
+    formed here as sum_c k_t[c] k_s[c] exp(l_t[c] - l_s[c]) (every factor at most 1 for
+    s < t).  Returns (A, B, Wb, Ub, l) with l [n, d_k]."""
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    alpha = np.asarray(alpha, np.float64)
+    beta = np.asarray(beta, np.float64)
+    n, dk = k.shape
+    ell = np.cumsum(np.log(alpha), axis=0)             # [n, d_k]
+    gamma = np.exp(ell)
+    # [t, s, c] = gamma_t / gamma_s for s < t, else 0
+    lower = np.tri(n, n, -1)[:, :, None] > 0
+    ratio = np.exp(np.where(lower, ell[:, None, :] - ell[None, :, :], -np.inf))
+    L = beta[:, None] * np.einsum("tc,sc,tsc->ts", k, k, ratio)
+    T = np.linalg.solve(np.eye(n) + L, np.diag(beta))
+    Wb = T @ (gamma * k)
+    Ub = T @ v
+    Kc = np.exp(ell[-1][None, :] - ell) * k
+    A = np.diag(gamma[-1]) - Wb.T @ Kc
+    B = Ub.T @ Kc
+    return A, B, Wb, Ub, ell
+
+
+def chunk_readout_wy_channel(q, k, Wb, Ub, ell, S0):
+    """Outputs of one chunk from its incoming state S0 under channel-wise decay, in
+    the WY form (the form a tensor-core read-out uses): with qt_t = gamma_t o q_t,
+      O = Qt S0^T + tril(Qt Kh^T) (Ub - Wb S0^T)     (diagonal included),
+    where (Qt Kh^T)_ts = sum_c q_t[c] k_s[c] exp(l_t[c] - l_s[c]).  Returns O [n, d_v]."""
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    n = q.shape[0]
+    gamma = np.exp(ell)
+    lower = np.tri(n, n, 0)[:, :, None] > 0
+    ratio = np.exp(np.where(lower, ell[:, None, :] - ell[None, :, :], -np.inf))
+    P = np.einsum("tc,sc,tsc->ts", q, k, ratio)
+    U = Ub - Wb @ np.asarray(S0, np.float64).T
+    return (gamma * q) @ np.asarray(S0, np.float64).T + P @ U
+
+
 # ----------------------------------------------------------------------------------
 # Routing (binary32 recipe)
 # ----------------------------------------------------------------------------------

@@ -379,3 +379,39 @@ def test_channel_decay_decode_matches_prefill():
         ref = ho.hla_prefill_head(q, k, v, a, b, C, bias=-0.5, thr=0.2, query_chunks=[(len(b) - 1) // C])
         assert np.abs(o - ref.o[-1]).max() <= 1e-12
     assert len(st.trans) == 2
+
+
+@pytest.mark.parametrize("n,d,dv", [(8, 5, 6), (16, 12, 12), (64, 128, 128)])
+def test_channel_wy_form_equals_literal_transition(n, d, dv):
+    """The chunkwise WY form with the decays folded into the keys (kt = gamma o k,
+    kh = k / gamma) reaches the token rule's (A, B) with a decay per key channel."""
+    rng = np.random.default_rng(100 + n + d)
+    _, k, v, _, b = _head(rng, n, d, dv)
+    a = _channel_alpha(rng, n, d)
+    A, B = ho.chunk_transition(k, v, a, b)
+    A2, B2, Wb, Ub, ell = ho.chunk_transition_wy_channel(k, v, a, b)
+    assert np.abs(A - A2).max() <= 1e-12
+    assert np.abs(B - B2).max() <= 1e-12
+
+
+def test_channel_wy_form_with_equal_channels_is_the_scalar_wy_form():
+    rng = np.random.default_rng(7)
+    _, k, v, a, b = _head(rng, 16, 8)
+    A1, B1, W1, U1, _ = ho.chunk_transition_wy(k, v, a, b)
+    A2, B2, W2, U2, _ = ho.chunk_transition_wy_channel(k, v, np.repeat(a[:, None], 8, axis=1), b)
+    for x, y in ((A1, A2), (B1, B2), (W1, W2), (U1, U2)):
+        assert np.abs(x - y).max() <= 1e-13
+
+
+@pytest.mark.parametrize("n,d", [(8, 5), (64, 32)])
+def test_channel_wy_readout_equals_token_rule(n, d):
+    """O = Qt S0^T + tril(Qt Kh^T)(Ub - Wb S0^T) equals the token rule run from S0
+    with a decay per key channel, output o_t = S_t q_t."""
+    rng = np.random.default_rng(200 + n)
+    q, k, v, _, b = _head(rng, n, d)
+    a = _channel_alpha(rng, n, d)
+    S0 = rng.standard_normal((d, d))
+    o, _ = ho.gdn_recurrent(q, k, v, a, b, S0=S0)
+    _, _, Wb, Ub, ell = ho.chunk_transition_wy_channel(k, v, a, b)
+    O = ho.chunk_readout_wy_channel(q, k, Wb, Ub, ell, S0)
+    assert np.abs(O - o).max() <= 1e-12
