@@ -8,9 +8,19 @@
 // y0 = B_p q), pool the open chunk's route queries, gate every closed chunk, then
 //   for active j descending:  y += g_j B_j x;  x <- (1-g_j) x + g_j A_j x
 // and o = y + y0.  The chain is bound by HBM: each active chunk costs 64 KiB of bf16
-// and 4 d^2 flops.  One CTA per (sequence, head): warps 0-3 compute (thread = row r),
-// warp 4 issues TMA loads of A_j and B_j (128-byte swizzle, 64-column boxes) into a
-// 3-stage ring, so about two chunks are in flight per SM while one is consumed.
+// and 4 d^2 flops.  One CTA per (sequence, head), two CTAs per SM: warps 0-3 compute
+// (thread = row r), warp 4 issues TMA loads of A_j and B_j (128-byte swizzle, 64-column
+// boxes) into a ring of three 32 KiB units, so about three chunks are in flight per SM.
+//
+// With routed gates and one key pool per chunk, the gate prologue reads every closed
+// chunk's pool (512 B each; 256 KiB per (sequence, head) at 512 chunks -- as many
+// bytes as four active chunks).  Those pools go through the same ring first: pieces
+// of 64 pools (32 KiB, four 32-column boxes of float32 with the 128-byte swizzle),
+// issued by the producer while the compute warps sweep the open chunk, so the
+// pools stream from HBM as fast as the A_j/B_j tiles do.  Each pool is scored by one
+// thread from shared memory (the swizzle keeps its 16-byte reads conflict-free).
+#include <cstring>
+
 #include "common.cuh"
 #include "kernels.cuh"
 #include "routing_recipe.cuh"
@@ -26,10 +36,34 @@ cudaError_t make_tmap_2d(CUtensorMap* m, const void* base, long inner, long rows
 
 namespace {
 
+typedef CUresult (*EncodeTiledFnF32)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                     const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                     CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// Float32 tensor map over `rows` rows of 128 values (the key pools of a cache), box
+// 32 values (128 bytes) x box_rows rows, 128-byte swizzle.
+cudaError_t make_tmap_pools(CUtensorMap* m, const float* base, long rows, int box_rows) {
+  static EncodeTiledFnF32 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFnF32)p;
+  }
+  if (fn == nullptr) return cudaErrorNotSupported;
+  cuuint64_t dims[2] = {128, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {128 * 4};
+  cuuint32_t box[2] = {32, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 constexpr int kD = 128;
-constexpr int kStages = 3;
 constexpr int kHalf = kD * 64 * 2;       // 16 KiB: one 64-column box of a 128x128 bf16 matrix
-constexpr int kStageBytes = 4 * kHalf;   // A_j and B_j
 constexpr int kCompute = 128;
 constexpr int kThreads = kCompute + 32;
 
@@ -46,8 +80,9 @@ __device__ __forceinline__ float blk_sum(float v, float* red) {
 // append the token to the open chunk, sweep the open chunk right to left (x = A_p q,
 // y0 = B_p q), pool the open chunk's route queries, gate every closed chunk and write
 // the ascending active list.  Returns the active count; x and y0 are this thread's.
+// With gates_here false the routed gates are left to the caller (rq is written).
 __device__ __forceinline__ int decode_prologue(const DecodeArgs& a, int bh, int n, int m, float* rq, float* red,
-                                             int* wcount, float& x, float& y0) {
+                                             int* wcount, float& x, float& y0, bool gates_here = true) {
   const int tid = threadIdx.x;
   const int C = a.C;
   const int mp = m + 1;
@@ -97,6 +132,7 @@ __device__ __forceinline__ int decode_prologue(const DecodeArgs& a, int bh, int 
       rq[tid] = __fmul_rn(a.tau, __fadd_rn(mx, route::rlog(__fdiv_rn(s, (float)mp), K)));
       tc::bar_sync(1, kCompute);
     }
+    if (!gates_here) return 0;
     const int W = a.win > 0 ? a.win : 1;
     const float* rk = a.rk + (long)bh * a.max_chunks * W * kD;
     for (int jb = 0; jb < n; jb += kCompute) {
@@ -145,14 +181,23 @@ __device__ __forceinline__ int decode_prologue(const DecodeArgs& a, int bh, int 
   return cnt;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+// The dense-cache kernel runs two CTAs per SM.  Its ring holds three units of 32 KiB:
+// a unit is one 64-column half of A_j together with the same half of B_j (the two
+// passes of the mat-vec chain), or one piece of 64 key pools (four 32-column boxes of
+// float32).  The producer issues the pool pieces, then two units per active chunk; the
+// compute warps release a unit as soon as its pass is done.
+constexpr int kUnit = 2 * kHalf;                    // 32 KiB
+constexpr int kUnits = 3;
+constexpr int kPoolRows = kUnit / (kD * 4);          // 64 key pools of 512 B per unit
+
+__global__ void __launch_bounds__(kThreads, 2)
     decode_stream_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                         DecodeArgs a) {
+                         const __grid_constant__ CUtensorMap tmR, DecodeArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* ring = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint64_t* full = (uint64_t*)(ring + kStages * kStageBytes);
-  uint64_t* empty = full + kStages;
-  float* xs = (float*)(empty + kStages);     // [2][kD]
+  uint64_t* full = (uint64_t*)(ring + kUnits * kUnit);
+  uint64_t* empty = full + kUnits;
+  float* xs = (float*)(empty + kUnits);      // [2][kD]
   float* rq = xs + 2 * kD;                   // [kD]
   float* red = rq + kD;                      // [4]
   int* wcount = (int*)(red + 4);             // [4]
@@ -166,11 +211,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int m = a.m_partial[b];
   int32_t* act_idx = a.act_idx + (long)bh * a.max_chunks;
   float* act_g = a.act_g + (long)bh * a.max_chunks;
+  // routed gates with one pool per chunk: the pools stream through the ring first
+  const bool stream_pools = a.mode == HLA_GATES_ROUTED && a.win == 0 && n > 0;
+  const int npieces = stream_pools ? (n + kPoolRows - 1) / kPoolRows : 0;
 
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      tc::mbar_init(&full[s], 1);
-      tc::mbar_init(&empty[s], 1);
+    for (int u = 0; u < kUnits; ++u) {
+      tc::mbar_init(&full[u], 1);
+      tc::mbar_init(&empty[u], 1);
     }
     *abort_s = 0;
     tc::mbar_fence_init();
@@ -180,56 +228,136 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid >= kCompute) {
     // ---------------- TMA producer (warp 4, lane 0) ----------------
-    // waits for the active list, then streams A_j / B_j for j descending
-    tc::bar_sync(2, kThreads);
+    // key pool pieces (routed gates); then, once the active list is known, two units
+    // per active chunk for j descending.  Units are numbered across both phases.
+    int u = 0;
     if (tid == kCompute) {
       tc::tma_prefetch_desc(&tmA);
       tc::tma_prefetch_desc(&tmB);
-      const int cnt = *cnt_s;
-      int s = 0;
-      for (int p = cnt - 1; p >= 0; --p, ++s) {
-        const int st = s % kStages;
-        if (s >= kStages && !tc::mbar_wait(&empty[st], ((s / kStages) - 1) & 1, abort_s)) break;
+      if (stream_pools) tc::tma_prefetch_desc(&tmR);
+      for (int pc = 0; pc < npieces; ++pc, ++u) {
+        const int st = u % kUnits;
+        if (u >= kUnits && !tc::mbar_wait(&empty[st], ((u / kUnits) - 1) & 1, abort_s)) break;
+        const int row = (int)((long)bh * a.max_chunks + (long)pc * kPoolRows);
+        tc::mbar_arrive_expect_tx(&full[st], kUnit);
+        uint8_t* dst = ring + st * kUnit;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) tc::tma_load_2d(dst + q4 * (kUnit / 4), &tmR, 32 * q4, row, &full[st]);
+      }
+    }
+    tc::bar_sync(2, kThreads);
+    if (tid == kCompute) {
+      const int cnt = *abort_s ? 0 : *cnt_s;
+      bool go = true;
+      for (int p = cnt - 1; go && p >= 0; --p) {
         const int j = act_idx[p];
         const int row = (int)(((long)bh * a.max_chunks + j) * kD);
-        tc::mbar_arrive_expect_tx(&full[st], kStageBytes);
-        uint8_t* dst = ring + st * kStageBytes;
-        tc::tma_load_2d(dst, &tmA, 0, row, &full[st]);
-        tc::tma_load_2d(dst + kHalf, &tmA, 64, row, &full[st]);
-        tc::tma_load_2d(dst + 2 * kHalf, &tmB, 0, row, &full[st]);
-        tc::tma_load_2d(dst + 3 * kHalf, &tmB, 64, row, &full[st]);
+        for (int hh = 0; hh < 2; ++hh, ++u) {
+          const int st = u % kUnits;
+          if (u >= kUnits && !tc::mbar_wait(&empty[st], ((u / kUnits) - 1) & 1, abort_s)) {
+            go = false;
+            break;
+          }
+          tc::mbar_arrive_expect_tx(&full[st], kUnit);
+          uint8_t* dst = ring + st * kUnit;
+          tc::tma_load_2d(dst, &tmA, 64 * hh, row, &full[st]);
+          tc::tma_load_2d(dst + kHalf, &tmB, 64 * hh, row, &full[st]);
+        }
       }
       if (*abort_s)
-        for (int t = max(0, s - kStages); t < s; ++t)
-          tc::mbar_wait(&full[t % kStages], (t / kStages) & 1, nullptr, 200000000ull);
+        for (int t = max(0, u - kUnits); t < u; ++t)
+          tc::mbar_wait(&full[t % kUnits], (t / kUnits) & 1, nullptr, 200000000ull);
     }
     __syncwarp();
   } else {
     // ---------------- compute (warps 0-3), thread = channel / row ----------------
     float x, y0;
-    const int cnt = decode_prologue(a, bh, n, m, rq, red, wcount, x, y0);
+    int cnt = decode_prologue(a, bh, n, m, rq, red, wcount, x, y0, !stream_pools);
+    bool ok = true;
+    int u = 0;
+    if (stream_pools) {
+      // gates of the closed chunks from the pool pieces in the ring, two pieces a
+      // round: threads 0-63 score the first piece's pools, threads 64-127 the second's
+      // (one fma chain over ascending channels per pool, as the recipe fixes); the
+      // block then compacts the kept chunks in ascending j
+      const route::Consts K = route::make_consts();
+      const int half = tid >> 6, r = tid & 63;
+      for (int pc0 = 0; pc0 < npieces; pc0 += 2) {
+        const bool two = pc0 + 1 < npieces;
+        bool got = tc::mbar_wait(&full[u % kUnits], (u / kUnits) & 1, abort_s);
+        if (two) got = got && tc::mbar_wait(&full[(u + 1) % kUnits], ((u + 1) / kUnits) & 1, abort_s);
+        ok = tc::bar_all(1, kCompute, got);
+        if (!ok) break;
+        const int mine = u + half;
+        const int j = (pc0 + half) * kPoolRows + r;
+        float dot = 0.0f;
+        if (half == 0 || two) {
+          const uint8_t* piece = ring + (mine % kUnits) * kUnit;
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const uint8_t* rowp = piece + q4 * (kUnit / 4) + r * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const float4 r4 = *(const float4*)(rowp + ((c ^ (r & 7)) << 4));
+              const int c0 = 32 * q4 + 4 * c;
+              dot = route::dot_step(dot, rq[c0 + 0], r4.x);
+              dot = route::dot_step(dot, rq[c0 + 1], r4.y);
+              dot = route::dot_step(dot, rq[c0 + 2], r4.z);
+              dot = route::dot_step(dot, rq[c0 + 3], r4.w);
+            }
+          }
+        }
+        float g = 0.0f;
+        bool keep = false;
+        if (j < n) {
+          g = route::gate_from_dot(dot, a.c_d, a.bias, K);
+          keep = a.thr <= 0.0f || g >= a.thr;
+        }
+        const unsigned int bal = __ballot_sync(0xFFFFFFFFu, keep);
+        const int w = tid >> 5;
+        if ((tid & 31) == 0) wcount[w] = __popc(bal);
+        tc::bar_sync(1, kCompute);  // also: every thread has read this round's pieces
+        if (tid == 0) {
+          tc::mbar_arrive(&empty[u % kUnits]);
+          if (two) tc::mbar_arrive(&empty[(u + 1) % kUnits]);
+        }
+        u += two ? 2 : 1;
+        int before = 0, total = 0;
+#pragma unroll
+        for (int k2 = 0; k2 < 4; ++k2) {
+          if (k2 < w) before += wcount[k2];
+          total += wcount[k2];
+        }
+        if (keep) {
+          const int pos = cnt + before + __popc(bal & ((1u << (tid & 31)) - 1u));
+          act_idx[pos] = j;
+          act_g[pos] = g;
+        }
+        cnt += total;
+        tc::bar_sync(1, kCompute);
+      }
+      if (!ok) cnt = 0;
+    }
     const long tok = (long)bh * kD + tid;
     if (tid == 0) *cnt_s = cnt;
     xs[tid] = x;
     __threadfence_block();
     tc::bar_sync(2, kThreads);  // releases the producer
-    // (3) active chain, descending j
+    // (3) active chain, descending j: two units per chunk (column halves of A_j, B_j)
     float y = 0.0f;
     int cur = 0;
-    bool ok = true;
-    for (int p = cnt - 1, s = 0; p >= 0; --p, ++s) {
-      const int st = s % kStages;
-      ok = tc::bar_all(1, kCompute, tc::mbar_wait(&full[st], (s / kStages) & 1, abort_s));
-      if (!ok) break;
-      const uint8_t* stA = ring + st * kStageBytes;
-      const uint8_t* stB = stA + 2 * kHalf;
+    for (int p = cnt - 1; ok && p >= 0; --p) {
       const float* xc = xs + cur * kD;
       float ax0 = 0.f, ax1 = 0.f, bx0 = 0.f, bx1 = 0.f;
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
+      for (int hh = 0; hh < 2; ++hh, ++u) {
+        const int st = u % kUnits;
+        ok = tc::bar_all(1, kCompute, tc::mbar_wait(&full[st], (u / kUnits) & 1, abort_s));
+        if (!ok) break;
+        const uint8_t* stA = ring + st * kUnit;
+        const uint8_t* stB = stA + kHalf;
 #pragma unroll
         for (int c8 = 0; c8 < 8; ++c8) {
-          const int off = hh * kHalf + tid * 128 + ((c8 ^ (tid & 7)) << 4);
+          const int off = tid * 128 + ((c8 ^ (tid & 7)) << 4);
           const uint4 wa = *(const uint4*)(stA + off);
           const uint4 wb = *(const uint4*)(stB + off);
           const float4 x0 = *(const float4*)(xc + hh * 64 + c8 * 8);
@@ -251,13 +379,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           bx0 = fmaf(tc::bf16lo(wb.w), x1.z, bx0);
           bx1 = fmaf(tc::bf16hi(wb.w), x1.w, bx1);
         }
+        if (hh == 0) {
+          // every thread has read this unit: hand it back to the producer
+          tc::bar_sync(1, kCompute);
+          if (tid == 0) tc::mbar_arrive(&empty[st]);
+        } else {
+          const float g = act_g[p];
+          y = fmaf(g, bx0 + bx1, y);
+          xs[(cur ^ 1) * kD + tid] = (1.0f - g) * xc[tid] + g * (ax0 + ax1);
+          cur ^= 1;
+          tc::bar_sync(1, kCompute);
+          if (tid == 0) tc::mbar_arrive(&empty[st]);
+        }
       }
-      const float g = act_g[p];
-      y = fmaf(g, bx0 + bx1, y);
-      xs[(cur ^ 1) * kD + tid] = (1.0f - g) * xc[tid] + g * (ax0 + ax1);
-      cur ^= 1;
-      tc::bar_sync(1, kCompute);
-      if (tid == 0) tc::mbar_arrive(&empty[st]);
     }
     stf((__nv_bfloat16*)a.o + tok, y + y0);
   }
@@ -448,10 +582,17 @@ cudaError_t launch_decode_stream(const DecodeArgs& a, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   e = make_tmap_rows128(&tmB, a.Bm, rows);
   if (e != cudaSuccess) return e;
-  const size_t smem = 1024 + kStages * kStageBytes + 2 * kStages * 8 + (4 * kD + 16) * 4;
+  // key pools (one per chunk; with window representatives the kernel reads them directly)
+  CUtensorMap tmR;
+  std::memset(&tmR, 0, sizeof(tmR));
+  if (a.mode == HLA_GATES_ROUTED && a.win == 0) {
+    e = make_tmap_pools(&tmR, a.rk, (long)a.B * a.H * a.max_chunks, kPoolRows);
+    if (e != cudaSuccess) return e;
+  }
+  const size_t smem = 1024 + kUnits * kUnit + 2 * kUnits * 8 + (4 * kD + 16) * 4;
   e = cudaFuncSetAttribute(decode_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  decode_stream_kernel<<<a.B * a.H, kThreads, smem, s>>>(tmA, tmB, a);
+  decode_stream_kernel<<<a.B * a.H, kThreads, smem, s>>>(tmA, tmB, tmR, a);
   return cudaGetLastError();
 }
 
