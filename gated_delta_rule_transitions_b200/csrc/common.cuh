@@ -25,6 +25,7 @@ enum : unsigned int {
   kErrMbarTimeout = 1u,   // an mbarrier wait gave up
   kErrTmemAlloc = 2u,     // tensor-memory allocation could not be satisfied
   kErrCacheFull = 4u,     // a decode step had to close a chunk into a full cache
+  kErrDecayRange = 8u,    // a channel's decay over one sub-chunk left the tensor-core range
 };
 
 // Streaming multiprocessors of the current device (read once per process; the

@@ -80,9 +80,12 @@ __device__ __forceinline__ float blk_sum(float v, float* red) {
 // append the token to the open chunk, sweep the open chunk right to left (x = A_p q,
 // y0 = B_p q), pool the open chunk's route queries, gate every closed chunk and write
 // the ascending active list.  Returns the active count; x and y0 are this thread's.
-// With gates_here false the routed gates are left to the caller (rq is written).
+// The flags leave steps to the caller: gates_here false -- the routed gates (rq is
+// written); do_append / do_sweep / do_pool false -- the append, the sweep (x = y0 = 0)
+// or the query pool.
 __device__ __forceinline__ int decode_prologue(const DecodeArgs& a, int bh, int n, int m, float* rq, float* red,
-                                             int* wcount, float& x, float& y0, bool gates_here = true) {
+                                             int* wcount, float& x, float& y0, bool gates_here = true,
+                                             bool do_append = true, bool do_sweep = true, bool do_pool = true) {
   const int tid = threadIdx.x;
   const int C = a.C;
   const int mp = m + 1;
@@ -90,25 +93,27 @@ __device__ __forceinline__ int decode_prologue(const DecodeArgs& a, int bh, int 
   float* act_g = a.act_g + (long)bh * a.max_chunks;
   const long tok = (long)bh * kD + tid;
   const long bslot = ((long)bh * C + m) * kD + tid;
-  const __nv_bfloat16* qr_in = (const __nv_bfloat16*)(a.q_route ? a.q_route : a.q);
-  const __nv_bfloat16* kr_in = (const __nv_bfloat16*)(a.k_route ? a.k_route : a.k);
-  ((__nv_bfloat16*)a.buf_k)[bslot] = ((const __nv_bfloat16*)a.k)[tok];
-  ((__nv_bfloat16*)a.buf_v)[bslot] = ((const __nv_bfloat16*)a.v)[tok];
-  ((__nv_bfloat16*)a.buf_qr)[bslot] = qr_in[tok];
-  ((__nv_bfloat16*)a.buf_kr)[bslot] = kr_in[tok];
-  if (a.alpha_vec) a.buf_alpha[((long)bh * C + m) * kD + tid] = a.alpha[(long)bh * kD + tid];
-  if (tid == 0) {
-    if (!a.alpha_vec) a.buf_alpha[(long)bh * C + m] = a.alpha[bh];
-    a.buf_beta[(long)bh * C + m] = a.beta[bh];
+  if (do_append) {
+    const __nv_bfloat16* qr_in = (const __nv_bfloat16*)(a.q_route ? a.q_route : a.q);
+    const __nv_bfloat16* kr_in = (const __nv_bfloat16*)(a.k_route ? a.k_route : a.k);
+    ((__nv_bfloat16*)a.buf_k)[bslot] = ((const __nv_bfloat16*)a.k)[tok];
+    ((__nv_bfloat16*)a.buf_v)[bslot] = ((const __nv_bfloat16*)a.v)[tok];
+    ((__nv_bfloat16*)a.buf_qr)[bslot] = qr_in[tok];
+    ((__nv_bfloat16*)a.buf_kr)[bslot] = kr_in[tok];
+    if (a.alpha_vec) a.buf_alpha[((long)bh * C + m) * kD + tid] = a.alpha[(long)bh * kD + tid];
+    if (tid == 0) {
+      if (!a.alpha_vec) a.buf_alpha[(long)bh * C + m] = a.alpha[bh];
+      a.buf_beta[(long)bh * C + m] = a.beta[bh];
+    }
+    tc::bar_sync(1, kCompute);
+    __threadfence_block();
   }
-  tc::bar_sync(1, kCompute);
-  __threadfence_block();
   const __nv_bfloat16* bk = (const __nv_bfloat16*)a.buf_k + (long)bh * C * kD;
   const __nv_bfloat16* bv = (const __nv_bfloat16*)a.buf_v + (long)bh * C * kD;
   // (1) open-chunk sweep
-  x = ldf((const __nv_bfloat16*)a.q + tok);
+  x = do_sweep ? ldf((const __nv_bfloat16*)a.q + tok) : 0.0f;
   y0 = 0.0f;
-  for (int t = mp - 1; t >= 0; --t) {
+  for (int t = do_sweep ? mp - 1 : -1; t >= 0; --t) {
     const float kt = ldf(bk + (long)t * kD + tid);
     const float c = blk_sum(kt * x, red);
     const float bt = a.buf_beta[(long)bh * C + t];
@@ -119,9 +124,9 @@ __device__ __forceinline__ int decode_prologue(const DecodeArgs& a, int bh, int 
   }
   // (2) gates and the ascending active list
   int cnt = 0;
-  if (a.mode != HLA_GATES_ZERO && n > 0) {
+  if (a.mode != HLA_GATES_ZERO && n > 0 && (do_pool || gates_here)) {
     const route::Consts K = route::make_consts();
-    if (a.mode == HLA_GATES_ROUTED) {
+    if (a.mode == HLA_GATES_ROUTED && do_pool) {
       const __nv_bfloat16* bq = (const __nv_bfloat16*)a.buf_qr + (long)bh * C * kD + tid;
       const float inv_tau = __fdiv_rn(1.0f, a.tau);
       float mx = __fmul_rn(ldf(bq), inv_tau);
@@ -181,28 +186,38 @@ __device__ __forceinline__ int decode_prologue(const DecodeArgs& a, int bh, int 
   return cnt;
 }
 
-// The dense-cache kernel runs two CTAs per SM.  Its ring holds three units of 32 KiB:
-// a unit is one 64-column half of A_j together with the same half of B_j (the two
-// passes of the mat-vec chain), or one piece of 64 key pools (four 32-column boxes of
-// float32).  The producer issues the pool pieces, then two units per active chunk; the
-// compute warps release a unit as soon as its pass is done.
+// Dense cache (bf16, d = 128): two kernels per decode step.
+//
+// decode_gates_kernel -- one CTA per (sequence, head), three CTAs per SM: appends the
+// token to the open chunk, pools the open chunk's route queries, scores every closed
+// chunk's key pool and writes the ascending active list and its length.  With routed
+// gates and one pool per chunk the pools stream in by TMA in pieces of 64 pools
+// (32 KiB, four 32-column boxes of float32 with the 128-byte swizzle) through a ring
+// of two pieces; threads 0-63 score the first piece of a round and threads 64-127 the
+// second (one fma chain over ascending channels per pool, the recipe's order; the
+// swizzle keeps the 16-byte reads conflict-free).  Every (sequence, head) is gated at
+// once across the GPU, and the 512 B per closed chunk stream at full bandwidth.
+//
+// decode_stream_kernel -- one CTA per (sequence, head), two CTAs per SM: the producer
+// reads the list's length and streams the active chunks at once, j descending, two
+// 32 KiB units each (a 64-column half of A_j with the same half of B_j) through a ring
+// of three units, while the compute warps sweep the open chunk; then the chain, a unit
+// handed back to the producer as soon as its pass is done.
 constexpr int kUnit = 2 * kHalf;                    // 32 KiB
 constexpr int kUnits = 3;
-constexpr int kPoolRows = kUnit / (kD * 4);          // 64 key pools of 512 B per unit
+constexpr int kPoolRows = kUnit / (kD * 4);          // 64 key pools of 512 B per piece
+constexpr int kGPieces = 2;                          // ring of the gate kernel
 
-__global__ void __launch_bounds__(kThreads, 2)
-    decode_stream_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                         const __grid_constant__ CUtensorMap tmR, DecodeArgs a) {
+__global__ void __launch_bounds__(kThreads, 3)
+    decode_gates_kernel(const __grid_constant__ CUtensorMap tmR, DecodeArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* ring = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint64_t* full = (uint64_t*)(ring + kUnits * kUnit);
-  uint64_t* empty = full + kUnits;
-  float* xs = (float*)(empty + kUnits);      // [2][kD]
-  float* rq = xs + 2 * kD;                   // [kD]
+  uint64_t* full = (uint64_t*)(ring + kGPieces * kUnit);
+  uint64_t* empty = full + kGPieces;
+  float* rq = (float*)(empty + kGPieces);    // [kD]
   float* red = rq + kD;                      // [4]
   int* wcount = (int*)(red + 4);             // [4]
-  int* cnt_s = wcount + 4;                   // [1]
-  volatile int* abort_s = (volatile int*)(cnt_s + 1);
+  volatile int* abort_s = (volatile int*)(wcount + 4);
 
   const int bh = blockIdx.x;
   const int b = bh / a.H;
@@ -211,12 +226,11 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int m = a.m_partial[b];
   int32_t* act_idx = a.act_idx + (long)bh * a.max_chunks;
   float* act_g = a.act_g + (long)bh * a.max_chunks;
-  // routed gates with one pool per chunk: the pools stream through the ring first
   const bool stream_pools = a.mode == HLA_GATES_ROUTED && a.win == 0 && n > 0;
   const int npieces = stream_pools ? (n + kPoolRows - 1) / kPoolRows : 0;
 
   if (tid == 0) {
-    for (int u = 0; u < kUnits; ++u) {
+    for (int u = 0; u < kGPieces; ++u) {
       tc::mbar_init(&full[u], 1);
       tc::mbar_init(&empty[u], 1);
     }
@@ -227,72 +241,45 @@ __global__ void __launch_bounds__(kThreads, 2)
   __syncthreads();
 
   if (tid >= kCompute) {
-    // ---------------- TMA producer (warp 4, lane 0) ----------------
-    // key pool pieces (routed gates); then, once the active list is known, two units
-    // per active chunk for j descending.  Units are numbered across both phases.
-    int u = 0;
-    if (tid == kCompute) {
-      tc::tma_prefetch_desc(&tmA);
-      tc::tma_prefetch_desc(&tmB);
-      if (stream_pools) tc::tma_prefetch_desc(&tmR);
-      for (int pc = 0; pc < npieces; ++pc, ++u) {
-        const int st = u % kUnits;
-        if (u >= kUnits && !tc::mbar_wait(&empty[st], ((u / kUnits) - 1) & 1, abort_s)) break;
-        const int row = (int)((long)bh * a.max_chunks + (long)pc * kPoolRows);
+    // ---------------- TMA producer (warp 4, lane 0): the key pool pieces ----------------
+    if (tid == kCompute && npieces > 0) {
+      tc::tma_prefetch_desc(&tmR);
+      int u = 0;
+      for (; u < npieces; ++u) {
+        const int st = u % kGPieces;
+        if (u >= kGPieces && !tc::mbar_wait(&empty[st], ((u / kGPieces) - 1) & 1, abort_s)) break;
+        const int row = (int)((long)bh * a.max_chunks + (long)u * kPoolRows);
         tc::mbar_arrive_expect_tx(&full[st], kUnit);
         uint8_t* dst = ring + st * kUnit;
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) tc::tma_load_2d(dst + q4 * (kUnit / 4), &tmR, 32 * q4, row, &full[st]);
       }
-    }
-    tc::bar_sync(2, kThreads);
-    if (tid == kCompute) {
-      const int cnt = *abort_s ? 0 : *cnt_s;
-      bool go = true;
-      for (int p = cnt - 1; go && p >= 0; --p) {
-        const int j = act_idx[p];
-        const int row = (int)(((long)bh * a.max_chunks + j) * kD);
-        for (int hh = 0; hh < 2; ++hh, ++u) {
-          const int st = u % kUnits;
-          if (u >= kUnits && !tc::mbar_wait(&empty[st], ((u / kUnits) - 1) & 1, abort_s)) {
-            go = false;
-            break;
-          }
-          tc::mbar_arrive_expect_tx(&full[st], kUnit);
-          uint8_t* dst = ring + st * kUnit;
-          tc::tma_load_2d(dst, &tmA, 64 * hh, row, &full[st]);
-          tc::tma_load_2d(dst + kHalf, &tmB, 64 * hh, row, &full[st]);
-        }
-      }
       if (*abort_s)
-        for (int t = max(0, u - kUnits); t < u; ++t)
-          tc::mbar_wait(&full[t % kUnits], (t / kUnits) & 1, nullptr, 200000000ull);
+        for (int t = max(0, u - kGPieces); t < u; ++t)
+          tc::mbar_wait(&full[t % kGPieces], (t / kGPieces) & 1, nullptr, 200000000ull);
     }
     __syncwarp();
   } else {
-    // ---------------- compute (warps 0-3), thread = channel / row ----------------
+    // ---------------- compute (warps 0-3), thread = channel ----------------
     float x, y0;
-    int cnt = decode_prologue(a, bh, n, m, rq, red, wcount, x, y0, !stream_pools);
+    // append, query pool, and (without streamed pools) the gates
+    int cnt = decode_prologue(a, bh, n, m, rq, red, wcount, x, y0, !stream_pools, true, false, true);
     bool ok = true;
-    int u = 0;
     if (stream_pools) {
-      // gates of the closed chunks from the pool pieces in the ring, two pieces a
-      // round: threads 0-63 score the first piece's pools, threads 64-127 the second's
-      // (one fma chain over ascending channels per pool, as the recipe fixes); the
-      // block then compacts the kept chunks in ascending j
       const route::Consts K = route::make_consts();
       const int half = tid >> 6, r = tid & 63;
+      int u = 0;
       for (int pc0 = 0; pc0 < npieces; pc0 += 2) {
         const bool two = pc0 + 1 < npieces;
-        bool got = tc::mbar_wait(&full[u % kUnits], (u / kUnits) & 1, abort_s);
-        if (two) got = got && tc::mbar_wait(&full[(u + 1) % kUnits], ((u + 1) / kUnits) & 1, abort_s);
+        bool got = tc::mbar_wait(&full[u % kGPieces], (u / kGPieces) & 1, abort_s);
+        if (two) got = got && tc::mbar_wait(&full[(u + 1) % kGPieces], ((u + 1) / kGPieces) & 1, abort_s);
         ok = tc::bar_all(1, kCompute, got);
         if (!ok) break;
         const int mine = u + half;
         const int j = (pc0 + half) * kPoolRows + r;
         float dot = 0.0f;
         if (half == 0 || two) {
-          const uint8_t* piece = ring + (mine % kUnits) * kUnit;
+          const uint8_t* piece = ring + (mine % kGPieces) * kUnit;
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) {
             const uint8_t* rowp = piece + q4 * (kUnit / 4) + r * 128;
@@ -318,8 +305,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         if ((tid & 31) == 0) wcount[w] = __popc(bal);
         tc::bar_sync(1, kCompute);  // also: every thread has read this round's pieces
         if (tid == 0) {
-          tc::mbar_arrive(&empty[u % kUnits]);
-          if (two) tc::mbar_arrive(&empty[(u + 1) % kUnits]);
+          tc::mbar_arrive(&empty[u % kGPieces]);
+          if (two) tc::mbar_arrive(&empty[(u + 1) % kGPieces]);
         }
         u += two ? 2 : 1;
         int before = 0, total = 0;
@@ -336,16 +323,84 @@ __global__ void __launch_bounds__(kThreads, 2)
         cnt += total;
         tc::bar_sync(1, kCompute);
       }
-      if (!ok) cnt = 0;
     }
+    if (tid == 0) a.act_cnt[bh] = ok ? cnt : 0;
+  }
+  __syncthreads();
+  if (tid == 0 && *abort_s) report_device_error(kErrMbarTimeout);
+}
+
+__global__ void __launch_bounds__(kThreads, 2)
+    decode_stream_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                         DecodeArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* ring = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint64_t* full = (uint64_t*)(ring + kUnits * kUnit);
+  uint64_t* empty = full + kUnits;
+  float* xs = (float*)(empty + kUnits);      // [2][kD]
+  float* rq = xs + 2 * kD;                   // [kD] (not used: the gates are done)
+  float* red = rq + kD;                      // [4]
+  int* wcount = (int*)(red + 4);             // [4]
+  volatile int* abort_s = (volatile int*)(wcount + 4);
+
+  const int bh = blockIdx.x;
+  const int b = bh / a.H;
+  const int tid = threadIdx.x;
+  const int n = a.n_chunks[b];
+  const int m = a.m_partial[b];
+  const int32_t* act_idx = a.act_idx + (long)bh * a.max_chunks;
+  const float* act_g = a.act_g + (long)bh * a.max_chunks;
+  const int cnt = a.act_cnt[bh];
+
+  if (tid == 0) {
+    for (int u = 0; u < kUnits; ++u) {
+      tc::mbar_init(&full[u], 1);
+      tc::mbar_init(&empty[u], 1);
+    }
+    *abort_s = 0;
+    tc::mbar_fence_init();
+    tc::fence_async_smem();
+  }
+  __syncthreads();
+
+  if (tid >= kCompute) {
+    // ---------------- TMA producer (warp 4, lane 0): two units per active chunk ----------------
+    if (tid == kCompute && cnt > 0) {
+      tc::tma_prefetch_desc(&tmA);
+      tc::tma_prefetch_desc(&tmB);
+      int u = 0;
+      bool go = true;
+      for (int p = cnt - 1; go && p >= 0; --p) {
+        const int j = act_idx[p];
+        const int row = (int)(((long)bh * a.max_chunks + j) * kD);
+        for (int hh = 0; hh < 2; ++hh, ++u) {
+          const int st = u % kUnits;
+          if (u >= kUnits && !tc::mbar_wait(&empty[st], ((u / kUnits) - 1) & 1, abort_s)) {
+            go = false;
+            break;
+          }
+          tc::mbar_arrive_expect_tx(&full[st], kUnit);
+          uint8_t* dst = ring + st * kUnit;
+          tc::tma_load_2d(dst, &tmA, 64 * hh, row, &full[st]);
+          tc::tma_load_2d(dst + kHalf, &tmB, 64 * hh, row, &full[st]);
+        }
+      }
+      if (*abort_s)
+        for (int t = max(0, u - kUnits); t < u; ++t)
+          tc::mbar_wait(&full[t % kUnits], (t / kUnits) & 1, nullptr, 200000000ull);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- compute (warps 0-3), thread = channel / row ----------------
+    float x, y0;
+    decode_prologue(a, bh, n, m, rq, red, wcount, x, y0, false, false, true, false);  // the sweep only
     const long tok = (long)bh * kD + tid;
-    if (tid == 0) *cnt_s = cnt;
     xs[tid] = x;
-    __threadfence_block();
-    tc::bar_sync(2, kThreads);  // releases the producer
-    // (3) active chain, descending j: two units per chunk (column halves of A_j, B_j)
+    tc::bar_sync(1, kCompute);
+    // active chain, descending j: two units per chunk (column halves of A_j, B_j)
     float y = 0.0f;
-    int cur = 0;
+    int cur = 0, u = 0;
+    bool ok = true;
     for (int p = cnt - 1; ok && p >= 0; --p) {
       const float* xc = xs + cur * kD;
       float ax0 = 0.f, ax1 = 0.f, bx0 = 0.f, bx1 = 0.f;
@@ -582,17 +637,23 @@ cudaError_t launch_decode_stream(const DecodeArgs& a, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   e = make_tmap_rows128(&tmB, a.Bm, rows);
   if (e != cudaSuccess) return e;
-  // key pools (one per chunk; with window representatives the kernel reads them directly)
+  // key pools (one per chunk; with window representatives the gates read them directly)
   CUtensorMap tmR;
   std::memset(&tmR, 0, sizeof(tmR));
   if (a.mode == HLA_GATES_ROUTED && a.win == 0) {
     e = make_tmap_pools(&tmR, a.rk, (long)a.B * a.H * a.max_chunks, kPoolRows);
     if (e != cudaSuccess) return e;
   }
+  const size_t gsmem = 1024 + kGPieces * kUnit + 2 * kGPieces * 8 + (kD + 16) * 4;
+  e = cudaFuncSetAttribute(decode_gates_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gsmem);
+  if (e != cudaSuccess) return e;
+  decode_gates_kernel<<<a.B * a.H, kThreads, gsmem, s>>>(tmR, a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
   const size_t smem = 1024 + kUnits * kUnit + 2 * kUnits * 8 + (4 * kD + 16) * 4;
   e = cudaFuncSetAttribute(decode_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  decode_stream_kernel<<<a.B * a.H, kThreads, smem, s>>>(tmA, tmB, tmR, a);
+  decode_stream_kernel<<<a.B * a.H, kThreads, smem, s>>>(tmA, tmB, a);
   return cudaGetLastError();
 }
 

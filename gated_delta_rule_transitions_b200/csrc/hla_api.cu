@@ -118,8 +118,15 @@ constexpr int kSub = 64;
 
 // Prefill workspace layout.
 struct PrefillWs {
-  size_t rq, rk, act_idx, act_g, act_cnt, order, A, Bm, Asub, Bsub, Wb, Ub, ell, S_in, total;
+  size_t rq, rk, act_idx, act_g, act_cnt, order, A, Bm, Asub, Bsub, Wb, Ub, ell, S_in;
+  size_t Kt, Kh, Kc, Qt, gC;  // channel-wise decay on the tensor cores: prepared operands
+  size_t total;
 };
+
+// Channel-wise decay runs on the tensor cores for bf16 with d = 128 (the decays folded
+// into the keys and queries per 64-token sub-chunk), else by the token rule on CUDA
+// cores.
+bool chan_tc(const hla_config* c) { return chan(c) && c->dtype == HLA_BF16 && c->dk == 128; }
 
 PrefillWs prefill_layout(const hla_config* c) {
   PrefillWs w{};
@@ -142,10 +149,17 @@ PrefillWs prefill_layout(const hla_config* c) {
   w.order = take(B * H * N * 4);
   w.A = take(B * H * Nc * d * d * esize(c->dtype));
   w.Bm = take(B * H * Nc * d * d * esize(c->dtype));
-  if (chan(c)) {  // token-rule transitions and read-out per chunk: no WY factors
+  if (chan(c) && !chan_tc(c)) {  // token-rule transitions and read-out per chunk: no WY factors
     w.S_in = take(B * H * N * d * d * 4);
     w.total = off;
     return w;
+  }
+  if (chan_tc(c)) {  // Kt, Kh, Kc, Qt [B,H,Nsub,64,d] bf16 and gamma_C [B,H,Nsub,d] float32
+    w.Kt = take(B * H * Nsub * kSub * d * 2);
+    w.Kh = take(B * H * Nsub * kSub * d * 2);
+    w.Kc = take(B * H * Nsub * kSub * d * 2);
+    w.Qt = take(B * H * Nsub * kSub * d * 2);
+    w.gC = take(B * H * Nsub * d * 4);
   }
   if (C > kSub) {  // transitions of the complete sub-chunks, merged into A, Bm
     w.Asub = take(B * H * Nsub_c * d * d * esize(c->dtype));
@@ -448,7 +462,8 @@ size_t hla_prefill_workspace_bytes(const hla_config* cfg) {
 size_t hla_decode_workspace_bytes(const hla_config* cfg, int32_t max_chunks) {
   if (check_cfg(cfg, false) != HLA_OK || max_chunks <= 0) return 0;
   const size_t n = (size_t)cfg->B * cfg->H * max_chunks;
-  return align256(n * 4) + align256(n * 4);
+  // active lists and gates [B,H,max_chunks], then one list length per (sequence, head)
+  return align256(n * 4) + align256(n * 4) + align256((size_t)cfg->B * cfg->H * 4);
 }
 
 hla_status gdn_chunk_transitions(const hla_config* cfg, const void* k, const void* v, const float* alpha,
@@ -659,8 +674,11 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
   HLA_CUDA(cudaEventRecord(side->join, side->s), "side stream join");
   // transitions of every 64-token sub-chunk (A/B of complete ones into the cache or
   // workspace; at C > 64 into the workspace, merged per chunk below)
-  // Channel-wise decay: the token rule over whole chunks, no sub-chunks.
-  const bool chan_path = chan(cfg);
+  // Channel-wise decay: the token rule over whole chunks, no sub-chunks (float32, or
+  // d = 64); bf16 with d = 128 takes the tensor-core path below with the decays folded
+  // into prepared keys and queries (chan_tc_path).
+  const bool chan_path = chan(cfg) && !chan_tc(cfg);
+  const bool chan_tc_path = chan_tc(cfg);
   const int s_sub = chan_path ? 1 : cfg->C / kSub;
   const int Nsub = chan_path ? N : (cfg->T + kSub - 1) / kSub;
   const int Nsub_c = chan_path ? Nc : cfg->T / kSub;
@@ -693,15 +711,40 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
   }
   t.Wb = chan_path ? nullptr : (float*)(ws + w.Wb);
   t.Ub = chan_path ? nullptr : (float*)(ws + w.Ub);
-  t.ell = chan_path ? nullptr : (float*)(ws + w.ell);
+  t.ell = (chan_path || chan_tc_path) ? nullptr : (float*)(ws + w.ell);
+  hla::ChanOperands ops{};
+  if (chan_tc_path) {
+    ops.Kt = ws + w.Kt;
+    ops.Kh = ws + w.Kh;
+    ops.Kc = ws + w.Kc;
+    ops.Qt = ws + w.Qt;
+    ops.gC = (const float*)(ws + w.gC);
+  }
   {
-    StageScope _sc(HLA_STAGE_TRANSITIONS, s, 1);
-    if (chan_path)
+    StageScope _sc(HLA_STAGE_TRANSITIONS, s, chan_tc_path ? 2 : 1);
+    if (chan_tc_path) {
+      hla::ChanPrepArgs pa{};
+      pa.B = cfg->B;
+      pa.H = cfg->H;
+      pa.T = cfg->T;
+      pa.Nsub = Nsub;
+      pa.k = k;
+      pa.q = q;
+      pa.alpha = alpha;
+      pa.Kt = ws + w.Kt;
+      pa.Kh = ws + w.Kh;
+      pa.Kc = ws + w.Kc;
+      pa.Qt = ws + w.Qt;
+      pa.gC = (float*)(ws + w.gC);
+      HLA_CUDA(hla::launch_chan_prep(pa, s), "channel-decay operand launch");
+      HLA_CUDA(hla::launch_transitions_tc(t, s, &ops), "transitions (tensor core, channel decay) launch");
+    } else if (chan_path) {
       HLA_CUDA(hla::launch_transitions_token(t, s), "transitions (token rule) launch");
-    else if (tc_path)
+    } else if (tc_path) {
       HLA_CUDA(hla::launch_transitions_tc(t, s), "transitions (tensor core) launch");
-    else
+    } else {
       HLA_CUDA(hla::launch_transitions(t, s), "transitions launch");
+    }
   }
   // chunks of C > 64 tokens: each chunk's transition from its sub-chunks' ones
   hla::ChainArgs ch{};
@@ -792,7 +835,8 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
   if (!chan_path) {
     StageScope _sc(HLA_STAGE_READOUT, s, 1);
     if (tc_path)
-      HLA_CUDA(hla::launch_readout_tc(r, c.S_in, t.Wb, t.Ub, s), "readout (tensor core) launch");
+      HLA_CUDA(hla::launch_readout_tc(r, c.S_in, t.Wb, t.Ub, s, chan_tc_path ? &ops : nullptr),
+               "readout (tensor core) launch");
     else
       HLA_CUDA(hla::launch_readout(r, s), "readout launch");
   }
@@ -805,7 +849,7 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
     dc.dtype = cfg->dtype;
     dc.max_chunks = cache_out->max_chunks;
     dc.win = n_windows(cfg);
-    dc.alpha_vec = chan_path ? 1 : 0;
+    dc.alpha_vec = chan(cfg) ? 1 : 0;
     dc.rk = cache_out->rk;
     dc.buf_k = cache_out->buf_k;
     dc.buf_v = cache_out->buf_v;
@@ -900,9 +944,12 @@ hla_status hla_decode_step(const hla_config* cfg, hla_cache* cache, const void* 
   const size_t n = (size_t)cfg->B * cfg->H * cache->max_chunks;
   a.act_idx = (int32_t*)workspace;
   a.act_g = (float*)((char*)workspace + align256(n * 4));
+  a.act_cnt = (int32_t*)((char*)workspace + 2 * align256(n * 4));
   cudaStream_t s = (cudaStream_t)stream;
   {
-    StageScope _sc(HLA_STAGE_DECODE, s, 1);
+    // the dense bf16 cache with d = 128 gates in one kernel and streams in another
+    const bool two = cache->format == HLA_CACHE_DENSE && cfg->dtype == HLA_BF16 && cfg->dk == 128;
+    StageScope _sc(HLA_STAGE_DECODE, s, two ? 2 : 1);
     HLA_CUDA(hla::launch_decode_main(a, s), "decode launch");
   }
   {
@@ -977,8 +1024,9 @@ hla_status hla_decode_step_static(const hla_config* cfg, hla_cache* cache, const
   if (need > kStaticScratchBytes)
     return fail(HLA_ERR_WORKSPACE,
                 "decode scratch for B=%d H=%d max_chunks=%d is %zu bytes; the static array holds %zu "
-                "(B*H*max_chunks <= %zu); use hla_decode_step with a caller workspace",
-                cfg->B, cfg->H, cache->max_chunks, need, kStaticScratchBytes, kStaticScratchBytes / 8);
+                "(8 B per (sequence, head, chunk) and 4 B per (sequence, head), each part rounded up to "
+                "256 B); use hla_decode_step with a caller workspace",
+                cfg->B, cfg->H, cache->max_chunks, need, kStaticScratchBytes);
   void* ws = nullptr;
   HLA_TRY(static_scratch_ptr(&ws));
   return hla_decode_step(cfg, cache, q, k, v, alpha, beta, q_route, k_route, o, ws, kStaticScratchBytes, stream);
@@ -1039,10 +1087,17 @@ hla_status hla_device_status(int32_t clear, uint32_t* code_out) {
   word |= w;
   HLA_CUDA(hla::read_error_word_chain_tc(&w, clear != 0), "hla_device_status read");
   word |= w;
+  HLA_CUDA(hla::read_error_word_chan_prep(&w, clear != 0), "hla_device_status read");
+  word |= w;
   if (code_out) *code_out = word;
   if (word & (hla::kErrMbarTimeout | hla::kErrTmemAlloc))
     return fail(HLA_ERR_TIMEOUT, "a bounded device wait expired (code 0x%x)", word);
   if (word & hla::kErrCacheFull) return fail(HLA_ERR_WORKSPACE, "a decode step found the cache full (code 0x%x)", word);
+  if (word & hla::kErrDecayRange)
+    return fail(HLA_ERR_UNSUPPORTED,
+                "a channel decayed below e^-80 within one 64-token sub-chunk: outside the range of the "
+                "tensor-core channel-decay path (code 0x%x)",
+                word);
   return HLA_OK;
 }
 

@@ -122,6 +122,31 @@ struct ReadoutTokenArgs {
   void* o;                 // [B,T,H,d]
 };
 
+// Channel-wise decay on the tensor cores: per 64-token sub-chunk the decays folded
+// into the keys and queries (chan_prep.cu).  Every operand is [B,H,Nsub,64,128] bf16
+// (row t of sub-chunk n at ((b*H + h)*Nsub + n)*64 + t); gC is [B,H,Nsub,128] float32.
+struct ChanPrepArgs {
+  int B, H, T, Nsub;
+  const void* k;        // [B,T,H,128] bf16
+  const void* q;
+  const float* alpha;   // [B,T,H,128]
+  void* Kt;             // k o gamma_t
+  void* Kh;             // k / gamma_t
+  void* Kc;             // k o gamma_C / gamma_t
+  void* Qt;             // q o gamma_t
+  float* gC;            // gamma_C (the sub-chunk's whole decay per channel)
+};
+
+// Operands of the tensor-core transition / read-out kernels under channel-wise decay
+// (null for the scalar decay).
+struct ChanOperands {
+  const void* Kt;
+  const void* Kh;
+  const void* Kc;
+  const void* Qt;
+  const float* gC;
+};
+
 struct ReadoutArgs {
   int B, H, T, C, N, d, dtype;
   const void* q;          // [B,T,H,d]
@@ -166,6 +191,7 @@ struct DecodeArgs {
   // workspace
   int32_t* act_idx;  // [B,H,max_chunks]
   float* act_g;      // [B,H,max_chunks]
+  int32_t* act_cnt;  // [B,H]: length of each active list (dense-cache streaming kernels)
 };
 
 cudaError_t launch_pools(const void* x0, const void* x1, float* r0, float* r1, int B, int T, int H, int d,
@@ -183,16 +209,18 @@ cudaError_t read_error_word_decode(unsigned int* out, bool clear);
 cudaError_t read_error_word_compose_tc(unsigned int* out, bool clear);
 cudaError_t launch_compose_tc(const ComposeArgs& a, bool scan, cudaStream_t s);
 cudaError_t launch_decode_stream(const DecodeArgs& a, cudaStream_t s);
-cudaError_t launch_transitions_tc(const TransArgs& t, cudaStream_t s);
+cudaError_t launch_transitions_tc(const TransArgs& t, cudaStream_t s, const ChanOperands* chan = nullptr);
 cudaError_t launch_factor_fill(const FactorFillArgs& f, cudaStream_t s);
 cudaError_t launch_decode_stream_factored(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_readout_tc(const ReadoutArgs& r, const void* S_in_bf16, const void* Wb_bf16, const void* Ub_bf16,
-                              cudaStream_t s);
+                              cudaStream_t s, const ChanOperands* chan = nullptr);
 cudaError_t read_error_word_transitions_tc(unsigned int* out, bool clear);
 cudaError_t read_error_word_readout_tc(unsigned int* out, bool clear);
 cudaError_t read_error_word_decode_stream(unsigned int* out, bool clear);
 cudaError_t read_error_word_wait_check(unsigned int* out, bool clear);
 cudaError_t read_error_word_chain_tc(unsigned int* out, bool clear);
+cudaError_t read_error_word_chan_prep(unsigned int* out, bool clear);
+cudaError_t launch_chan_prep(const ChanPrepArgs& a, cudaStream_t s);
 cudaError_t launch_chain_merge(const ChainArgs& a, cudaStream_t s);
 cudaError_t launch_chain_advance(const ChainArgs& a, cudaStream_t s);
 // Transitions of chunks of a.C > 64 tokens by the token rule itself (CUDA cores);

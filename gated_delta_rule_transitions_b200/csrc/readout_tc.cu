@@ -13,6 +13,11 @@
 //   MMA2  P (128 x 64) x X (64 x 128)  ->  D2 (TMEM)
 //   epilogue 2: o_t = gamma_t (Q S_in^T)_t + D2_t, rows t < tokens in the chunk.
 // Operands come in by TMA with 128-byte swizzle; P and X reuse the [Q; Wb] buffer.
+//
+// Channel-wise decay (kChan): with Qt = Q o gamma and Kh = K / gamma per channel
+// (chan_prep.cu) the read-out is O = Qt S_in^T + tril(Qt Kh^T) (Ub - Wb S_in^T): the
+// same two MMAs with Qt in place of Q and Kh in place of K, no exp in P and no gamma
+// row scaling at the end.
 #include "common.cuh"
 #include "kernels.cuh"
 #include "tc_common.cuh"
@@ -46,6 +51,7 @@ struct ReadoutTcArgs {
 
 __device__ __forceinline__ int swz(int row, int chunk) { return row * 128 + ((chunk ^ (row & 7)) << 4); }
 
+template <bool kChan>
 __global__ void __launch_bounds__(128, 2)
     readout_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmU,
@@ -72,7 +78,7 @@ __global__ void __launch_bounds__(128, 2)
     tc::mbar_fence_init();
     tc::fence_async_smem();
   }
-  if (tid < kC) ell_s[tid] = a.ell[chunk * kC + tid];
+  if (!kChan && tid < kC) ell_s[tid] = a.ell[chunk * kC + tid];
   if (warp == 0) tc::tmem_alloc(tmem_s, 256);
   tc::tc_fence_before();
   __syncthreads();
@@ -85,10 +91,12 @@ __global__ void __launch_bounds__(128, 2)
     const int yw = (int)(chunk * kC);
     const int ys = (int)(chunk * kD);
     for (int kh = 0; kh < 2; ++kh) {
-      tc::tma_load_2d(sm + kA1 + kh * 16384, &tmQ, h * kD + 64 * kh, yq, &bars[0]);
+      // kChan: Qt and Kh are [chunk x 64 rows, 128] like Wb
+      tc::tma_load_2d(sm + kA1 + kh * 16384, &tmQ, kChan ? 64 * kh : h * kD + 64 * kh, kChan ? yw : yq, &bars[0]);
       tc::tma_load_2d(sm + kA1 + kh * 16384 + 8192, &tmW, 64 * kh, yw, &bars[0]);
       tc::tma_load_2d(sm + kB1 + kh * 24576, &tmS, 64 * kh, ys, &bars[0]);
-      tc::tma_load_2d(sm + kB1 + kh * 24576 + 16384, &tmK, h * kD + 64 * kh, yq, &bars[0]);
+      tc::tma_load_2d(sm + kB1 + kh * 24576 + 16384, &tmK, kChan ? 64 * kh : h * kD + 64 * kh, kChan ? yw : yq,
+                      &bars[0]);
       tc::tma_load_2d(sm + kU + kh * 8192, &tmU, 64 * kh, yw, &bars[0]);
     }
   }
@@ -115,15 +123,18 @@ __global__ void __launch_bounds__(128, 2)
       tc::tmem_ld32(lane_addr + 128, *reinterpret_cast<uint32_t(*)[32]>(&qk[0]));
       tc::tmem_ld32(lane_addr + 160, *reinterpret_cast<uint32_t(*)[32]>(&qk[32]));
       tc::tmem_wait_ld();
-      const float lt = ell_s[t];
+      const float lt = kChan ? 0.0f : ell_s[t];
 #pragma unroll
       for (int c8 = 0; c8 < 8; ++c8) {
         uint32_t w[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int s0 = c8 * 8 + 2 * e;
-          const float p0 = s0 <= t ? __expf(lt - ell_s[s0]) * __uint_as_float(qk[s0]) : 0.0f;
-          const float p1 = s0 + 1 <= t ? __expf(lt - ell_s[s0 + 1]) * __uint_as_float(qk[s0 + 1]) : 0.0f;
+          // kChan: Qt Kh^T is already decayed
+          const float d0 = kChan ? 1.0f : __expf(lt - ell_s[s0]);
+          const float d1 = kChan ? 1.0f : __expf(lt - ell_s[s0 + 1]);
+          const float p0 = s0 <= t ? d0 * __uint_as_float(qk[s0]) : 0.0f;
+          const float p1 = s0 + 1 <= t ? d1 * __uint_as_float(qk[s0 + 1]) : 0.0f;
           w[e] = tc::pack_bf16x2(p0, p1);
         }
         *(uint4*)(sm + kP + swz(t, c8)) = make_uint4(w[0], w[1], w[2], w[3]);
@@ -174,7 +185,7 @@ __global__ void __launch_bounds__(128, 2)
     tc::tc_fence_after();
     const int t = tid;
     const uint32_t lane_addr = tm + ((uint32_t)(32 * warp) << 16);
-    const float gt = __expf(ell_s[t]);
+    const float gt = kChan ? 1.0f : __expf(ell_s[t]);
     __nv_bfloat16* orow = a.o + (((long)b * a.T + t0 + t) * a.H + h) * kD;
 #pragma unroll
     for (int cc = 0; cc < kD; cc += 32) {
@@ -204,15 +215,22 @@ __global__ void __launch_bounds__(128, 2)
 }  // namespace
 
 // Readout for bf16, d = 128: q, k [B,T,H,d]; Wb, Ub bf16 [B,H,N,C,d]; S_in bf16
-// [B,H,N,d,d] ([v][c]); ell float [B,H,N,C]; o bf16 [B,T,H,d].
+// [B,H,N,d,d] ([v][c]); ell float [B,H,N,C]; o bf16 [B,T,H,d].  With `chan` the
+// prepared Qt and Kh ([B,H,N,C,d] bf16) take the places of q and k.
 cudaError_t launch_readout_tc(const ReadoutArgs& r, const void* S_in_bf16, const void* Wb_bf16,
-                              const void* Ub_bf16, cudaStream_t s) {
+                              const void* Ub_bf16, cudaStream_t s, const ChanOperands* chan) {
   if (r.N <= 0) return cudaSuccess;
   const long HD = (long)r.H * kD;
   const long BHN = (long)r.B * r.H * r.N;
   CUtensorMap tq, tk, tw, tu, ts;
-  cudaError_t e = make_tmap_2d(&tq, r.q, HD, (long)r.B * r.T, HD * 2, 64, 64);
-  if (e == cudaSuccess) e = make_tmap_2d(&tk, r.k, HD, (long)r.B * r.T, HD * 2, 64, 64);
+  cudaError_t e = cudaSuccess;
+  if (chan != nullptr) {
+    e = make_tmap_2d(&tq, chan->Qt, kD, BHN * kC, kD * 2, 64, 64);
+    if (e == cudaSuccess) e = make_tmap_2d(&tk, chan->Kh, kD, BHN * kC, kD * 2, 64, 64);
+  } else {
+    e = make_tmap_2d(&tq, r.q, HD, (long)r.B * r.T, HD * 2, 64, 64);
+    if (e == cudaSuccess) e = make_tmap_2d(&tk, r.k, HD, (long)r.B * r.T, HD * 2, 64, 64);
+  }
   if (e == cudaSuccess) e = make_tmap_2d(&tw, Wb_bf16, kD, BHN * kC, kD * 2, 64, 64);
   if (e == cudaSuccess) e = make_tmap_2d(&tu, Ub_bf16, kD, BHN * kC, kD * 2, 64, 64);
   if (e == cudaSuccess) e = make_tmap_2d(&ts, S_in_bf16, kD, BHN * kD, kD * 2, 64, 128);
@@ -225,9 +243,15 @@ cudaError_t launch_readout_tc(const ReadoutArgs& r, const void* S_in_bf16, const
   a.ell = r.ell;
   a.o = (__nv_bfloat16*)r.o;
   const size_t smem = 1024 + kSmemUsed + 3 * 8 + 16 + kC * 4 + 16;
-  e = cudaFuncSetAttribute(readout_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (chan != nullptr) {
+    e = cudaFuncSetAttribute(readout_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    readout_tc_kernel<true><<<(unsigned)BHN, 128, smem, s>>>(tq, tk, tw, tu, ts, a);
+    return cudaGetLastError();
+  }
+  e = cudaFuncSetAttribute(readout_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  readout_tc_kernel<<<(unsigned)BHN, 128, smem, s>>>(tq, tk, tw, tu, ts, a);
+  readout_tc_kernel<false><<<(unsigned)BHN, 128, smem, s>>>(tq, tk, tw, tu, ts, a);
   return cudaGetLastError();
 }
 

@@ -22,6 +22,13 @@
 // leave through TMA stores from swizzled shared memory.  A final partial chunk
 // (n < C tokens) behaves as if padded with identity tokens (alpha = 1, beta = 0):
 // its extra rows of T, Wb and Ub are zero; its A/B are not written.
+//
+// Channel-wise decay (kChan): the decays come folded into the keys (chan_prep.cu:
+// Kt = K o gamma, Kh = K / gamma, Kc = K o gamma_C / gamma, per channel), so
+//   MMA1  [Kt; V] x Kh^T  -> rows 0-63: Kt Kh^T, already decayed (L needs no exp)
+//   MMA2  [T; T] x [Kt | V]  (T without a gamma row scaling)
+//   MMA3/4 take Kc (loaded by TMA) in place of D K, and A = Diag(gamma_C) - Wb^T Kc.
+// Kh is loaded into the T-operand buffer before MMA1, Kc into it after MMA2.
 #include "common.cuh"
 #include "kernels.cuh"
 #include "tc_common.cuh"
@@ -45,7 +52,8 @@ constexpr int kLU = kC * kLP * 4;             // bytes of one of L, U
 constexpr int kX = kScr + 2 * kLU;            // 16 KiB: L' (rows 16-63); then B staging (cols 64-127)
 constexpr int kXP = 52;                       // row pitch (floats) of L'
 constexpr int kSmall = kX + 16384;            // per-token scalars, barriers
-constexpr int kSmemUsed = kSmall + 4 * kC * 4 + 4 * 8 + 32;
+constexpr int kBars = 6;                      // tma, mma1, mma2, mma34, Kh, Kc
+constexpr int kSmemUsed = kSmall + 4 * kC * 4 + kBars * 8 + 32;
 static_assert(kX % 1024 == 0 && 48 * kXP * 4 <= 16384, "shared-memory layout");
 constexpr uint32_t kIdesc1 = tc::idesc_bf16_f32(128, 64, 0, 0);
 constexpr uint32_t kIdesc2 = tc::idesc_bf16_f32(128, 256, 0, 1);
@@ -54,13 +62,15 @@ constexpr uint32_t kIdesc3 = tc::idesc_bf16_f32(128, 128, 1, 1);
 struct TransTcArgs {
   int B, H, T, N;
   long total;                       // B * H * N chunks
-  long sb_a, sh_a, st_a;            // alpha/beta strides
+  long sb_a, sh_a, st_a;            // alpha strides (scalar decay)
+  long sb_b, sh_b, st_b;            // beta strides
   const float* alpha;
   const float* beta;
   bool has_ab;                      // A/B are written (complete chunks)
   long ab_chunk_stride;
   bool has_wu;                      // Wb/Ub are written
   float* ell;                       // [B,H,N,C] or null
+  const float* gC;                  // channel-wise decay: gamma_C [total, d]
 };
 
 __device__ __forceinline__ int swz(int row, int chunk) { return row * 128 + ((chunk ^ (row & 7)) << 4); }
@@ -81,22 +91,34 @@ __device__ __forceinline__ ChunkPos chunk_pos(const TransTcArgs& a, long chunk) 
   return p;
 }
 
+// The K (kChan: Kt, rows chunk * 64 + t of the prepared operand) and V tiles of a chunk.
+template <bool kChan>
 __device__ __forceinline__ void load_kv(uint8_t* sm, const CUtensorMap* tmK, const CUtensorMap* tmV,
-                                        uint64_t* bar, const TransTcArgs& a, const ChunkPos& p) {
+                                        uint64_t* bar, const TransTcArgs& a, const ChunkPos& p, long chunk) {
   tc::mbar_arrive_expect_tx(bar, 4 * 8192);
   const int y = p.b * a.T + p.t0;
   for (int kh = 0; kh < 2; ++kh) {
-    tc::tma_load_2d(sm + kKV + kh * 16384, tmK, p.h * kD + 64 * kh, y, bar);
+    if (kChan)
+      tc::tma_load_2d(sm + kKV + kh * 16384, tmK, 64 * kh, (int)(chunk * kC), bar);
+    else
+      tc::tma_load_2d(sm + kKV + kh * 16384, tmK, p.h * kD + 64 * kh, y, bar);
     tc::tma_load_2d(sm + kKV + kh * 16384 + 8192, tmV, p.h * kD + 64 * kh, y, bar);
   }
 }
 
-// alpha, beta of token `tid` of a chunk (identity token beyond n)
+// A 64 x 128 prepared operand (Kh or Kc) of a chunk into the T-operand buffer.
+__device__ __forceinline__ void load_tt(uint8_t* sm, const CUtensorMap* tm, uint64_t* bar, long chunk) {
+  tc::mbar_arrive_expect_tx(bar, 2 * 8192);
+  for (int kh = 0; kh < 2; ++kh) tc::tma_load_2d(sm + kTT + kh * 8192, tm, 64 * kh, (int)(chunk * kC), bar);
+}
+
+// alpha, beta of token `tid` of a chunk (identity token beyond n); with a decay per
+// channel only beta (the decays are in the prepared operands)
+template <bool kChan>
 __device__ __forceinline__ void load_ab(const TransTcArgs& a, const ChunkPos& p, int tid, float& al, float& be) {
   if (tid < p.n) {
-    const long off = p.b * a.sb_a + p.h * a.sh_a + (long)(p.t0 + tid) * a.st_a;
-    al = a.alpha[off];
-    be = a.beta[off];
+    al = kChan ? 1.0f : a.alpha[p.b * a.sb_a + p.h * a.sh_a + (long)(p.t0 + tid) * a.st_a];
+    be = a.beta[p.b * a.sb_b + p.h * a.sh_b + (long)(p.t0 + tid) * a.st_b];
   } else {
     al = 1.0f;
     be = 0.0f;
@@ -105,10 +127,12 @@ __device__ __forceinline__ void load_ab(const TransTcArgs& a, const ChunkPos& p,
 
 // Persistent: each CTA walks chunks blockIdx.x, blockIdx.x + gridDim.x, ...; the next
 // chunk's K/V tile and alpha/beta are fetched while the current one finishes.
+template <bool kChan>
 __global__ void __launch_bounds__(128, 2)
     transitions_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                           const __grid_constant__ CUtensorMap tmWb, const __grid_constant__ CUtensorMap tmUb,
                           const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                          const __grid_constant__ CUtensorMap tmKh, const __grid_constant__ CUtensorMap tmKc,
                           TransTcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -119,8 +143,8 @@ __global__ void __launch_bounds__(128, 2)
   float* beta_s = ell_s + kC;                    // beta_t
   float* bg_s = beta_s + kC;                     // beta_t gamma_t
   float* dk_s = bg_s + kC;                       // gamma_C / gamma_t
-  uint64_t* bars = (uint64_t*)(dk_s + kC);       // tma, mma1, mma2, mma34
-  uint32_t* tmem_s = (uint32_t*)(bars + 4);
+  uint64_t* bars = (uint64_t*)(dk_s + kC);       // tma, mma1, mma2, mma34, Kh, Kc
+  uint32_t* tmem_s = (uint32_t*)(bars + kBars);
   float* wsum = (float*)(tmem_s + 2);            // [2]
   volatile int* abort_s = (volatile int*)(wsum + 2);
 
@@ -129,7 +153,7 @@ __global__ void __launch_bounds__(128, 2)
   const int lane = tid & 31;
 
   if (tid == 0) {
-    for (int k = 0; k < 4; ++k) tc::mbar_init(&bars[k], 1);
+    for (int k = 0; k < kBars; ++k) tc::mbar_init(&bars[k], 1);
     *abort_s = 0;
     tc::mbar_fence_init();
     tc::fence_async_smem();
@@ -145,6 +169,10 @@ __global__ void __launch_bounds__(128, 2)
       tc::tma_prefetch_desc(&tmA);
       tc::tma_prefetch_desc(&tmB);
     }
+    if (kChan) {
+      tc::tma_prefetch_desc(&tmKh);
+      tc::tma_prefetch_desc(&tmKc);
+    }
   }
   if (warp == 0) tc::tmem_alloc(tmem_s, 256);
   tc::tc_fence_before();
@@ -156,62 +184,78 @@ __global__ void __launch_bounds__(128, 2)
   bool ok = true;
   bool load_pending = false;  // thread 0: a K/V load was issued and not yet waited for
   int load_parity = 0;
-  int it = 0, ph3 = 0;
+  int it = 0, ph3 = 0, ph5 = 0;
+  bool kh_pending = false, kc_pending = false;  // thread 0 (kChan): a Kh / Kc load in flight
   float pa = 1.0f, pb = 0.0f;  // alpha, beta of token `tid` of the chunk to come
   if (blockIdx.x < a.total) {
     const ChunkPos p0 = chunk_pos(a, blockIdx.x);
     if (tid == 0) {
-      load_kv(sm, &tmK, &tmV, &bars[0], a, p0);
+      load_kv<kChan>(sm, &tmK, &tmV, &bars[0], a, p0, blockIdx.x);
       load_pending = true;
       load_parity = 0;
     }
-    if (tid < kC) load_ab(a, p0, tid, pa, pb);
+    if (tid < kC) load_ab<kChan>(a, p0, tid, pa, pb);
   }
   for (long chunk = blockIdx.x; ok && chunk < a.total; chunk += gridDim.x, ++it) {
     const ChunkPos P = chunk_pos(a, chunk);
     const bool write_ab = (P.n == kC) && a.has_ab;
     const long next = chunk + gridDim.x;
 
-    // ---- l_t = cumulative log alpha ----
+    // ---- l_t = cumulative log alpha (a decay per channel: only beta) ----
     float la = 0.0f;
     if (tid < kC) {
-      la = logf(pa);
       beta_s[tid] = pb;
+      if (!kChan) {
+        la = logf(pa);
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const float y = __shfl_up_sync(0xFFFFFFFFu, la, o);
-        if (lane >= o) la += y;
+        for (int o = 1; o < 32; o <<= 1) {
+          const float y = __shfl_up_sync(0xFFFFFFFFu, la, o);
+          if (lane >= o) la += y;
+        }
+        if (lane == 31) wsum[warp] = la;
       }
-      if (lane == 31) wsum[warp] = la;
+    }
+    if (kChan && tid == 0) {
+      // Kh into the T-operand buffer, once the previous chunk's staged stores have
+      // read it
+      tc::bulk_wait_read_all();
+      load_tt(sm, &tmKh, &bars[4], chunk);
+      kh_pending = true;
     }
     tc::bar_sync(1, 128);
-    if (tid < kC) {
+    if (!kChan && tid < kC) {
       if (warp == 1) la += wsum[0];
       ell_s[tid] = la;
       if (a.ell) a.ell[chunk * kC + tid] = la;
     }
-    // the K/V tile has landed; the previous chunk's staged stores have left shared memory
+    // the K/V tile has landed (the previous chunk's staged stores may still be reading
+    // shared memory: they are waited for before the L rows are written)
     bool got = true;
     if (tid == 0) {
-      tc::bulk_wait_read_all();
       got = tc::mbar_wait(&bars[0], it & 1, abort_s);
       if (got) load_pending = false;
+      if (kChan && got) {
+        got = tc::mbar_wait(&bars[4], it & 1, abort_s);
+        if (got) kh_pending = false;
+      }
     }
     ok = tc::bar_all(1, 128, got);
 
-    // ---- MMA1: [K; V] K^T -> columns 0-63 (rows 0-63: K K^T) ----
+    // ---- MMA1: [K; V] K^T -> columns 0-63 (rows 0-63: K K^T; kChan: [Kt; V] Kh^T) ----
     if (ok && tid == 0) {
       tc::tc_fence_after();
       const uint32_t base = tc::smem_u32(sm + kKV);
+      const uint32_t bbase = tc::smem_u32(sm + (kChan ? kTT : kKV));
 #pragma unroll
       for (int ks = 0; ks < kD / 16; ++ks) {
         const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-        tc::mma_ss(tm, tc::sdesc_sw128(base + off, 16, 1024), tc::sdesc_sw128(base + off, 16, 1024), kIdesc1,
+        const uint32_t boff = kChan ? (ks >> 2) * 8192 + (ks & 3) * 32 : off;
+        tc::mma_ss(tm, tc::sdesc_sw128(base + off, 16, 1024), tc::sdesc_sw128(bbase + boff, 16, 1024), kIdesc1,
                    ks > 0 ? 1u : 0u);
       }
       tc::mma_commit(&bars[1]);
     }
-    if (ok && tid >= kC) {
+    if (!kChan && ok && tid >= kC) {
       // per-token scales, while the MMA runs
       const int s = tid - kC;
       const float ls = ell_s[s];
@@ -219,13 +263,19 @@ __global__ void __launch_bounds__(128, 2)
       dk_s[s] = __expf(ell_s[kC - 1] - ls);
     }
     {
-      const bool m1 = (ok && tid == 0) ? tc::mbar_wait(&bars[1], it & 1, abort_s) : true;
+      // MMA1 is done and the previous chunk's staged stores have read shared memory
+      bool m1 = true;
+      if (ok && tid == 0) {
+        m1 = tc::mbar_wait(&bars[1], it & 1, abort_s);
+        tc::bulk_wait_read_all();
+      }
       ok = tc::bar_all(1, 128, ok && m1);
     }
 
     // ---- L[t][s] = beta_t e^{l_t - l_s} (k_t . k_s) for s < t, else 0 ----
     // warps 0-1 (the lanes of rows 0-63) spill beta_t (K K^T)[t][.]; then every thread
-    // applies the decay and the mask to half a row
+    // applies the decay and the mask to half a row (the exponentials spread over all
+    // four sub-partitions)
     if (ok && tid < kC) {
       tc::tc_fence_after();
       const int t = tid;
@@ -235,14 +285,24 @@ __global__ void __launch_bounds__(128, 2)
       tc::tmem_wait_ld();
       const float bt = beta_s[t];
       float* Lrow = Lsm + t * kLP;
+      if (kChan) {
+        // the decays are in Kt Kh^T already: mask the strictly lower part
 #pragma unroll
-      for (int s4 = 0; s4 < kC; s4 += 4)
-        *(float4*)(Lrow + s4) = make_float4(bt * __uint_as_float(g[s4]), bt * __uint_as_float(g[s4 + 1]),
-                                            bt * __uint_as_float(g[s4 + 2]), bt * __uint_as_float(g[s4 + 3]));
+        for (int s4 = 0; s4 < kC; s4 += 4)
+          *(float4*)(Lrow + s4) = make_float4(s4 + 0 < t ? bt * __uint_as_float(g[s4 + 0]) : 0.0f,
+                                              s4 + 1 < t ? bt * __uint_as_float(g[s4 + 1]) : 0.0f,
+                                              s4 + 2 < t ? bt * __uint_as_float(g[s4 + 2]) : 0.0f,
+                                              s4 + 3 < t ? bt * __uint_as_float(g[s4 + 3]) : 0.0f);
+      } else {
+#pragma unroll
+        for (int s4 = 0; s4 < kC; s4 += 4)
+          *(float4*)(Lrow + s4) = make_float4(bt * __uint_as_float(g[s4]), bt * __uint_as_float(g[s4 + 1]),
+                                              bt * __uint_as_float(g[s4 + 2]), bt * __uint_as_float(g[s4 + 3]));
+      }
       tc::tc_fence_before();
     }
     ok = tc::bar_all(1, 128, ok);
-    if (ok) {
+    if (!kChan && ok) {
       const int t = tid & (kC - 1), hs = tid >> 6;
       const float lt = ell_s[t];
       float* Lrow = Lsm + t * kLP;
@@ -339,7 +399,7 @@ __global__ void __launch_bounds__(128, 2)
     // ---- operand [T diag(gamma); T] (bf16, K-major, 128 rows x 64), T = U diag(beta) ----
     if (ok) {
       const int r = tid, t = r & (kC - 1);
-      const float* scl = r < kC ? bg_s : beta_s;
+      const float* scl = (!kChan && r < kC) ? bg_s : beta_s;
       const float* Urow = Usm + t * kLP;
 #pragma unroll
       for (int c8 = 0; c8 < 8; ++c8) {
@@ -372,6 +432,11 @@ __global__ void __launch_bounds__(128, 2)
     }
     {
       const bool m2 = (ok && tid == 0) ? tc::mbar_wait(&bars[2], it & 1, abort_s) : true;
+      // kChan: the T operand has been read; Kc takes its buffer for MMA3/4
+      if (kChan && ok && m2 && tid == 0 && write_ab) {
+        load_tt(sm, &tmKc, &bars[5], chunk);
+        kc_pending = true;
+      }
       ok = tc::bar_all(1, 128, ok && m2);
     }
 
@@ -400,7 +465,7 @@ __global__ void __launch_bounds__(128, 2)
           *(uint4*)(opT + half * 8192 + swz(t, c8)) = w;
         }
       }
-      if (isW) {
+      if (!kChan && isW) {
         const float dt = dk_s[t];
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
@@ -430,8 +495,17 @@ __global__ void __launch_bounds__(128, 2)
         tc::tma_store_2d(&tmUb, sm + kScr + 16384 + 8192, 64, y);
         tc::bulk_commit();
       }
-      // MMA3/4: Wb^T D K -> columns 0-127, Ub^T D K -> columns 128-255
-      if (mma34) {
+      // kChan: Kc has landed in the T-operand buffer
+      bool kc_ok = true;
+      if (kChan && kc_pending) {
+        kc_ok = tc::mbar_wait(&bars[5], ph5 & 1, abort_s);
+        if (kc_ok) {
+          kc_pending = false;
+          ++ph5;
+        }
+      }
+      // MMA3/4: Wb^T D K -> columns 0-127, Ub^T D K -> columns 128-255 (kChan: Kc for D K)
+      if (mma34 && kc_ok) {
         const uint32_t wbase = tc::smem_u32(sm + kScr), ubase = wbase + 16384, dbase = tc::smem_u32(sm + kTT);
 #pragma unroll
         for (int ks = 0; ks < kC / 16; ++ks) {
@@ -443,12 +517,12 @@ __global__ void __launch_bounds__(128, 2)
       }
       // the K/V tile is no longer read (MMA2 done, D K built): fetch the next chunk's
       if (next < a.total) {
-        load_kv(sm, &tmK, &tmV, &bars[0], a, chunk_pos(a, next));
+        load_kv<kChan>(sm, &tmK, &tmV, &bars[0], a, chunk_pos(a, next), next);
         load_pending = true;
         load_parity = (it + 1) & 1;
       }
     }
-    if (ok && tid < kC && next < a.total) load_ab(a, chunk_pos(a, next), tid, pa, pb);
+    if (ok && tid < kC && next < a.total) load_ab<kChan>(a, chunk_pos(a, next), tid, pa, pb);
     if (mma34) {
       const bool m3 = tid == 0 ? tc::mbar_wait(&bars[3], ph3 & 1, abort_s) : true;
       ++ph3;
@@ -461,7 +535,7 @@ __global__ void __launch_bounds__(128, 2)
     if (mma34 && ok) {
       tc::tc_fence_after();
       const int r = tid;
-      const float gC = __expf(ell_s[kC - 1]);
+      const float gC = kChan ? a.gC[chunk * kD + r] : __expf(ell_s[kC - 1]);
 #pragma unroll
       for (int cc = 0; cc < kD; cc += 32) {
         uint32_t x[32], y[32];
@@ -507,6 +581,8 @@ __global__ void __launch_bounds__(128, 2)
     tc::bulk_wait_all();
     // never leave the CTA with a copy in flight
     if (load_pending) tc::mbar_wait(&bars[0], load_parity, nullptr, 200000000ull);
+    if (kh_pending) tc::mbar_wait(&bars[4], it & 1, nullptr, 200000000ull);
+    if (kc_pending) tc::mbar_wait(&bars[5], ph5 & 1, nullptr, 200000000ull);
   }
   tc::tc_fence_before();
   __syncthreads();
@@ -517,8 +593,9 @@ __global__ void __launch_bounds__(128, 2)
 
 }  // namespace
 
-// Transitions for bf16, d = 128 over [B,T,H,d] inputs (k, v) and [B,T,H] alpha/beta.
-cudaError_t launch_transitions_tc(const TransArgs& t, cudaStream_t s) {
+// Transitions for bf16, d = 128 over [B,T,H,d] inputs (k, v) and [B,T,H] alpha/beta;
+// with `chan` (channel-wise decay) over the prepared operands of every sub-chunk.
+cudaError_t launch_transitions_tc(const TransArgs& t, cudaStream_t s, const ChanOperands* chan) {
   if (t.n_chunks <= 0) return cudaSuccess;
   const long HD = (long)t.H * kD;
   const long rows = (long)t.B * (t.in.sb / HD);  // B x tokens per sequence
@@ -526,8 +603,18 @@ cudaError_t launch_transitions_tc(const TransArgs& t, cudaStream_t s) {
   const long ab_rows = (long)t.B * t.H * t.ab_chunk_stride * kD;
   // tile coordinates are 32-bit
   if (rows >= (1L << 31) || total * kC >= (1L << 31) || ab_rows >= (1L << 31)) return cudaErrorNotSupported;
-  CUtensorMap tk, tv, twb, tub, ta, tb;
-  cudaError_t e = make_tmap_2d(&tk, t.in.k, HD, rows, HD * 2, 64, 64);
+  CUtensorMap tk, tv, twb, tub, ta, tb, tkh, tkc;
+  cudaError_t e = cudaSuccess;
+  if (chan != nullptr) {
+    // Kt, Kh, Kc: [total chunks x 64 rows, 128] bf16
+    e = make_tmap_2d(&tk, chan->Kt, kD, total * kC, kD * 2, 64, 64);
+    if (e == cudaSuccess) e = make_tmap_2d(&tkh, chan->Kh, kD, total * kC, kD * 2, 64, 64);
+    if (e == cudaSuccess) e = make_tmap_2d(&tkc, chan->Kc, kD, total * kC, kD * 2, 64, 64);
+  } else {
+    e = make_tmap_2d(&tk, t.in.k, HD, rows, HD * 2, 64, 64);
+    tkh = tk;  // not used
+    tkc = tk;
+  }
   if (e == cudaSuccess) e = make_tmap_2d(&tv, t.in.v, HD, rows, HD * 2, 64, 64);
   // outputs that are not requested get a valid map that is never used
   const void* wb = t.Wb ? (const void*)t.Wb : t.in.k;
@@ -551,17 +638,29 @@ cudaError_t launch_transitions_tc(const TransArgs& t, cudaStream_t s) {
   a.sb_a = t.in.ab;
   a.sh_a = t.in.ah;
   a.st_a = t.in.at;
+  // beta is [B,T,H]; with a decay per channel the alpha strides carry a factor d
+  const long bdiv = t.in.alpha_vec ? kD : 1;
+  a.sb_b = t.in.ab / bdiv;
+  a.sh_b = t.in.ah / bdiv;
+  a.st_b = t.in.at / bdiv;
   a.alpha = t.in.alpha;
   a.beta = t.in.beta;
   a.has_ab = has_ab;
   a.ab_chunk_stride = t.ab_chunk_stride;
   a.has_wu = t.Wb != nullptr && t.Ub != nullptr;
-  a.ell = t.ell;
+  a.ell = chan != nullptr ? nullptr : t.ell;
+  a.gC = chan != nullptr ? chan->gC : nullptr;
   const size_t smem = 1024 + kSmemUsed;
-  e = cudaFuncSetAttribute(transitions_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
   const long grid = total < 2L * num_sms() ? total : 2L * num_sms();
-  transitions_tc_kernel<<<(unsigned)grid, 128, smem, s>>>(tk, tv, twb, tub, ta, tb, a);
+  if (chan != nullptr) {
+    e = cudaFuncSetAttribute(transitions_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    transitions_tc_kernel<true><<<(unsigned)grid, 128, smem, s>>>(tk, tv, twb, tub, ta, tb, tkh, tkc, a);
+    return cudaGetLastError();
+  }
+  e = cudaFuncSetAttribute(transitions_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  transitions_tc_kernel<false><<<(unsigned)grid, 128, smem, s>>>(tk, tv, twb, tub, ta, tb, tkh, tkc, a);
   return cudaGetLastError();
 }
 

@@ -268,8 +268,14 @@ hla_status hla_gate_support(const hla_config* cfg, const float* gates, float* ma
  * call enqueues its fork, routing and join: concurrent calls on different streams
  * are correct, but their routing stages run one after another on that stream.
  * Every return after the fork, an error included, leaves `stream` joined to it.
- * With HLA_DECAY_CHANNEL the transitions and the read-out run the token rule per
- * chunk on CUDA cores.
+ * With HLA_DECAY_CHANNEL and bf16, d = 128, the transitions and the read-out run on
+ * the tensor cores with the decays folded into prepared keys and queries per 64-token
+ * sub-chunk (k o gamma_t, k / gamma_t, k o gamma_C / gamma_t, q o gamma_t with
+ * gamma_t the decay accumulated since the sub-chunk's first token, per channel).
+ * Their range: in every channel the decay over one sub-chunk must stay above e^-80
+ * (k / gamma_t stays finite); a prefill that leaves it records code 0x8, reported by
+ * hla_device_status.  With float32 or d = 64 they run the token rule per chunk on CUDA
+ * cores (no such limit).
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
  */
 hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, const void* v,
@@ -292,7 +298,9 @@ hla_status hla_prefill(const hla_config* cfg, const void* q, const void* k, cons
  *      each active A_j/B_j once; when the open chunk reaches C tokens it is closed
  *      (its A/B/rk are appended; at C = 64 by the WY form, at C > 64 by the token
  *      rule run row by row).  Gate modes ROUTED, ONE and ZERO.
- * workspace: device, >= hla_decode_workspace_bytes(cfg, cache->max_chunks).
+ * workspace: device, >= hla_decode_workspace_bytes(cfg, cache->max_chunks): the
+ *      active lists and gates ([B,H,max_chunks] int32 and float32) and one list length
+ *      per (sequence, head), each part rounded up to 256 bytes.
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE (also: cache full), CUDA.
  */
 hla_status hla_decode_step(const hla_config* cfg, hla_cache* cache, const void* q,
@@ -308,8 +316,10 @@ hla_status hla_decode_step(const hla_config* cfg, hla_cache* cache, const void* 
  * all device memory through its own pool, or a thread with no allocator in
  * reach).  Same arguments, layouts, semantics and errors as hla_decode_step, minus
  * the workspace: the scratch is a fixed device array inside this library,
- * HLA_DECODE_STATIC_SCRATCH_BYTES long, enough for B*H*max_chunks <= 2^20.  A
- * larger cache is rejected with HLA_ERR_WORKSPACE before anything is launched.
+ * HLA_DECODE_STATIC_SCRATCH_BYTES long: it holds hla_decode_workspace_bytes(cfg,
+ * max_chunks) when 8 B per (sequence, head, chunk) plus 4 B per (sequence, head), each
+ * part rounded up to 256 B, fit in it (for example B*H = 1024 with max_chunks = 1023).
+ * A larger cache is rejected with HLA_ERR_WORKSPACE before anything is launched.
  * No call allocates or frees device memory.
  * Set-up: the first call on a device (the current one) looks up the array's
  * device address and keeps it; make that first call before any stream capture.
@@ -331,8 +341,11 @@ hla_status hla_decode_step_static(const hla_config* cfg, hla_cache* cache, const
  * Bounded device waits.  Kernels that wait on an mbarrier or a flag give up after
  * a fixed number of polls, record a code in a device-side error word and return.
  * hla_device_status synchronises the device, reads and (if clear != 0) resets that
- * word; it returns HLA_ERR_TIMEOUT if a wait expired since the last reset, else
- * HLA_OK (or HLA_ERR_CUDA).  *code_out (may be NULL) receives the raw word.
+ * word; it returns HLA_ERR_TIMEOUT if a wait expired since the last reset (code bit
+ * 0x1, or 0x2 for a tensor-memory allocation), HLA_ERR_WORKSPACE if a decode step
+ * found its cache full (0x4), HLA_ERR_UNSUPPORTED if a prefill with a decay per
+ * channel left the tensor-core range described at hla_prefill (0x8), else HLA_OK (or
+ * HLA_ERR_CUDA).  *code_out (may be NULL) receives the raw word.
  */
 hla_status hla_device_status(int32_t clear, uint32_t* code_out);
 

@@ -74,7 +74,8 @@ def test_decode_workspace_and_cache_sizes(hla):
     nb = hla.cache_bytes(c, 512)
     assert nb >= 64 * 16 * 512 * 2 * 128 * 128 * 2
     assert nb < 64 * 16 * 512 * 2 * 128 * 128 * 2 * 1.02
-    assert hla.decode_workspace_bytes(c, 512) == 2 * 64 * 16 * 512 * 4
+    # active lists and gates per (sequence, head, chunk), one list length per (sequence, head)
+    assert hla.decode_workspace_bytes(c, 512) == 2 * 64 * 16 * 512 * 4 + 64 * 16 * 4
 
 
 def test_prefill_workspace_grows_with_T(hla):
@@ -147,8 +148,9 @@ def test_python_binding_refuses_cpu_tensors(hla):
 
 
 def test_static_decode_rejects_scratch_beyond_its_array(hla):
-    """hla_decode_step_static has B*H*max_chunks <= 2^20 entries of fixed scratch; a
-    larger cache is refused on the host (the fake aligned pointers are never read)."""
+    """hla_decode_step_static has 8 MiB of fixed scratch (8 B per sequence, head and
+    cached chunk, plus 4 B per sequence and head); a larger cache is refused on the
+    host (the fake aligned pointers are never read)."""
     c = cfg(hla, B=64, H=16, T=1)
     cache = hla.HlaCache()
     cache.B, cache.H, cache.C, cache.d, cache.dtype = 64, 16, 64, 128, 1

@@ -2,9 +2,12 @@
 named in the Gated DeltaNet-2 abstract on the HLA listing page):
   S_t = S_{t-1} Diag(alpha_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T.
 
-Transitions and the intra-chunk read-out run the token rule row by row on CUDA cores;
-the composition and the gates are those of the scalar path.  Bars as elsewhere:
-gates and lists bit-exact, outputs max-abs 1e-4 (float32) or relative L2 2e-2 (bf16)."""
+With bf16 and d = 128 the prefill runs on the tensor cores (the decays folded into
+prepared keys and queries per 64-token sub-chunk); with float32 or d = 64, and in
+gdn_chunk_transitions and the decode close, the transitions and read-out run the token
+rule row by row on CUDA cores.  The composition and the gates are those of the scalar
+path.  Bars as elsewhere: gates and lists bit-exact, outputs max-abs 1e-4 (float32) or
+relative L2 2e-2 (bf16) per head; bf16 transitions relative L2 1e-2 per matrix."""
 import numpy as np
 import pytest
 import torch
@@ -164,3 +167,28 @@ def test_bf16_d64_channel_decay(hla):
     """bf16 storage with d = 64 (CUDA-core composition, float32 states read by the
     token-rule read-out)."""
     _check_prefill(hla, syn.PREFILL_0P8B.with_(B=1, H=2, T=64 * 5 + 33, d=64, thr=0.2, decay="channel"))
+
+
+@pytest.mark.parametrize("C,T", [(64, 64 * 5 + 7), (256, 256 * 2 + 64 + 3)])
+def test_channel_decay_tensor_core_cache_transitions(hla, C, T):
+    """The A_c, B_c that a bf16, d = 128 prefill with a decay per channel writes into a
+    dense cache (tensor-core transitions of the 64-token sub-chunks, merged at C > 64),
+    chunk by chunk against the oracle's literal token-rule transition."""
+    w = syn.PREFILL_0P8B.with_(B=1, H=2, T=T, C=C, decay="channel")
+    inp = P.gpu_inputs(w)
+    cfg = hla.make_config(1, 2, T, C, 128, "bf16", "routed", w.tau, w.bias, w.thr, decay="channel")
+    cache = hla.Cache(cfg, max_chunks=T // C + 1)
+    P.run_prefill(hla, w, inp, cache=cache)
+    st, code = hla.hla_device_status()
+    assert st == 0 and code == 0
+    n = T // C
+    # the closed chunks' slots only (the slot after them has not been written)
+    A = P.np64(cache.view("A", (1, 2, n + 1, 128, 128), torch.bfloat16)[:, :, :n])
+    Bm = P.np64(cache.view("Bm", (1, 2, n + 1, 128, 128), torch.bfloat16)[:, :, :n])
+    for h in range(2):
+        for c in range(n):
+            sl = slice(C * c, C * c + C)
+            Ar, Br = ho.chunk_transition(P.np64(inp["k"][0, sl, h]), P.np64(inp["v"][0, sl, h]),
+                                         P.np64(inp["alpha"][0, sl, h]), P.np64(inp["beta"][0, sl, h]))
+            P.check_bf16(A[0, h, c], Ar, "transition", tol=1e-2)
+            P.check_bf16(Bm[0, h, c], Br, "transition", tol=1e-2)
