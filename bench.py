@@ -9,7 +9,8 @@ One step is one pass of the hot path over synthetic inputs already resident in H
     transitions, gated composition, read-out;
   * one decode step of 64 sequences with 32768-token contexts (512 cached A_j/B_j
     per head, H=16, d=128, bf16, bias -2, threshold 0.05: every chunk active).
-The L2 cache is flushed (256 MiB write, untimed) before each timed phase.  Each
+The L2 cache is flushed before each timed phase (a 256 MiB write, then a 256 MiB read so
+that the write's dirty lines go back to HBM outside the timed region; untimed).  Each
 phase is timed with CUDA events on the launching stream; per-stage times come from
 the library's own event pairs (hla_profile_*), on the same stream.
 
@@ -251,9 +252,10 @@ def build_decode_cache(hla, syn, torch, w, max_chunks, group=8, cache_format="de
     return cache, first_ctx
 
 
-def _stage_avg(stages, name):
+def _stage_avg(stages, name, calls):
+    """Device milliseconds of one stage per call (a stage may launch several kernels)."""
     ms, n = stages.get(name, (0.0, 0))
-    return ms / n if n else None
+    return ms / calls if n and calls else None
 
 
 def measure_decode_planted(hla, syn, torch, stream, l2_flush, steps, warmup):
@@ -301,7 +303,7 @@ def measure_decode_planted(hla, syn, torch, stream, l2_flush, steps, warmup):
     per_chunk = 2 * wd.d * wd.d * 2
     act_total = int(active.sum())
     nbytes_alg = act_total * per_chunk + wd.B * wd.H * n_ctx * wd.d * 4
-    kern = _stage_avg(stages, "decode")
+    kern = _stage_avg(stages, "decode", steps)
     del cache, dws
     torch.cuda.empty_cache()
     return wd, ms, kern, act_total, nbytes_alg, stages
@@ -434,9 +436,14 @@ def run_ours(args):
         hla.hla_decode_step(dcfg, cache, t["q"], t["k"], t["v"], t["alpha"], t["beta"], od, workspace=dws)
 
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush_read = torch.ones(L2_FLUSH_BYTES // 8, dtype=torch.int64, device="cuda")
 
     def l2_flush():
+        # write a buffer larger than L2, then read another: the dirty lines of the write
+        # go back to HBM here, outside the timed region, and the next phase starts with
+        # a cache of clean, unrelated lines
         flush.zero_()
+        flush_read.sum()
 
     for _ in range(max(args.warmup, 0)):
         prefill()
@@ -551,8 +558,7 @@ def run_ours(args):
     s_sub = wp.C // 64
     flops_other = wp.B * wp.H * (n_sub * (FLOP_TRANSITION + FLOP_READOUT)
                                  + (2 * (wp.T // wp.C) + N) * (s_sub - 1) * 2.0 * d ** 3)
-    comp_ms, comp_n = stages["compose"]
-    comp_avg = comp_ms / max(comp_n, 1)
+    comp_avg = _stage_avg(stages, "compose", args.steps) or 0.0
     comp_tf = flops_compose / (comp_avg * 1e-3) / 1e12 if comp_avg > 0 else None
     n_ctx = wd.T // wd.C
     if args.decode_cache == "factored":
@@ -561,8 +567,7 @@ def run_ours(args):
         per_chunk = 2 * wd.d * wd.d * 2                      # A, B bf16
     key_reps = wd.C // wd.window if wd.window else 1
     bytes_decode = wd.B * wd.H * (n_ctx * (per_chunk + key_reps * wd.d * 4))
-    dmain_ms, dmain_n = stages["decode"]
-    dmain_avg = dmain_ms / max(dmain_n, 1)
+    dmain_avg = _stage_avg(stages, "decode", args.steps) or 0.0
     dec_gbs = bytes_decode / (dmain_avg * 1e-3) / 1e9 if dmain_avg > 0 else None
     launches = sum(n for (_, n) in stages.values())
 
@@ -583,7 +588,8 @@ def run_ours(args):
         "data": "synthetic (seeded; shapes and distributions of the HLA workloads; no dataset)",
         "config": {"workload": wp.name, "decode_workload": wd.name, "prefill_ms": pre_ms, "decode_ms": dec_ms,
                    "active_pairs": active_pairs, "parallelism": f"replicas x{world} (no data-path collective)",
-                   "l2": "flushed before every timed phase (256 MiB write, untimed)"},
+                   "l2": "flushed before every timed phase (256 MiB write, then a 256 MiB read that "
+                         "leaves only clean lines; untimed)"},
         "roofline": {"kernel": "compose", "bound": "tensor", "achieved": comp_tf, "peak": bf16_tf,
                      "unit": "TFLOP/s", "frac": (comp_tf / bf16_tf) if comp_tf else None,
                      "traffic": ncu_traffic("compose"), "traffic_unit": "bytes per launch (ncu dram read+write)",
@@ -594,7 +600,7 @@ def run_ours(args):
                      "algorithmic": f"{comp_what} x 2 d^3 = {flops_compose:.4g} flop per launch",
                      "prefill_frac_of_peak": (flops_compose + flops_other) / (pre_ms * 1e-3) / 1e12 / bf16_tf},
         "decode": {"value": whole_job_rate(tokens_dec, dec_ms, world), "unit": "tokens/s", "ms_per_step": dec_ms,
-                   "roofline": {"kernel": "decode_main", "bound": "hbm", "achieved": dec_gbs, "peak": hbm_gbs,
+                   "roofline": {"kernel": "decode (gate and stream kernels of the step)", "bound": "hbm", "achieved": dec_gbs, "peak": hbm_gbs,
                                 "unit": "GB/s", "frac": (dec_gbs / hbm_gbs) if dec_gbs else None,
                                 "traffic": ncu_traffic("decode_main") if args.decode_cache == "dense" else None,
                                 "traffic_unit": "bytes per launch (ncu dram read+write)",
@@ -625,7 +631,7 @@ def run_ours(args):
         out["decode_sparse"] = {
             "workload": wdp.name, "value": whole_job_rate(wdp.B, ms_dp, world), "unit": "tokens/s",
             "ms_per_step": ms_dp, "active_chunks_mean": act_dp / (wdp.B * wdp.H),
-            "roofline": {"kernel": "decode_main", "bound": "hbm", "achieved": gbs_dp, "peak": hbm_gbs,
+            "roofline": {"kernel": "decode (gate and stream kernels of the step)", "bound": "hbm", "achieved": gbs_dp, "peak": hbm_gbs,
                          "unit": "GB/s", "frac": (gbs_dp / hbm_gbs) if gbs_dp else None,
                          "peak_source": f"{peak_src} HBM copy",
                          "datasheet": {"peak": DATASHEET_HBM_GBS,
@@ -645,7 +651,7 @@ def run_ours(args):
         bytes_sp = 6 * bthd * 2 + 2 * ab_bytes   # q, k, v, route inputs in, o out; A/B written once, read once
         tf_sp = flops_sp / (ms_sp * 1e-3) / 1e12
         gbs_sp = bytes_sp / (ms_sp * 1e-3) / 1e9
-        comp_sp = _stage_avg(st_sp, "compose")
+        comp_sp = _stage_avg(st_sp, "compose", args.steps)
         out["sparse_prefill"] = {
             "workload": wsp.name, "value": whole_job_rate(wsp.B * wsp.T, ms_sp, world), "unit": "tokens/s",
             "ms": ms_sp, "active_pairs": pairs_sp,

@@ -23,6 +23,8 @@ namespace hla {
 // ---------------------------------------------------------------------------
 
 namespace {
+constexpr int kPoolBlock = 16;  // tokens read per step by the pools
+
 // The recipe's e^x on a pair of values with packed float32 arithmetic
 // (sm_100; each lane of __ffma2_rn / __fadd2_rn / __fmul2_rn is rounded as its
 // scalar counterpart).  Every product that feeds a sum is a fused multiply-add in
@@ -78,13 +80,17 @@ __device__ __forceinline__ float2 gate2_from_dot(float2 dot, float c_d, float bi
   return make_float2(__frcp_rn(den.x), __frcp_rn(den.y));
 }
 
-// s += exp(fma(x_t, inv_tau, -m)) over the staged bf16 pairs, ascending t.
+// s += exp(fma(x_t, inv_tau, -m)) over the bf16 pairs of tokens t0 .. t0+15 (t < n),
+// ascending t, read again from global memory (L1 / L2 hits: the first pass read them).
 template <bool kInRange>
-__device__ __forceinline__ float2 pool_sum_bf16(float2 s, const uint32_t (&w)[64], int n, float inv_tau, float m0,
-                                                float m1, const route::Consts& K) {
+__device__ __forceinline__ float2 pool_sum_bf16(float2 s, const uint32_t* colw, size_t stride, int t0, int n,
+                                                float inv_tau, float m0, float m1, const route::Consts& K) {
+  uint32_t w[kPoolBlock];
 #pragma unroll
-  for (int t = 0; t < 64; ++t)
-    if (t < n) {
+  for (int t = 0; t < kPoolBlock; ++t) w[t] = t0 + t < n ? __ldg(colw + (size_t)(t0 + t) * stride) : 0u;
+#pragma unroll
+  for (int t = 0; t < kPoolBlock; ++t)
+    if (t0 + t < n) {
       const float2 u = __ffma2_rn(make_float2(__uint_as_float(w[t] << 16), __uint_as_float(w[t] & 0xFFFF0000u)),
                                   make_float2(inv_tau, inv_tau), make_float2(-m0, -m1));
       s = __fadd2_rn(s, rexp2<kInRange>(u, K));
@@ -93,11 +99,10 @@ __device__ __forceinline__ float2 pool_sum_bf16(float2 s, const uint32_t (&w)[64
 }
 }  // namespace
 
-constexpr int kPoolSeg = 64;    // pool_sum_bf16 stages 64 tokens at a time
-constexpr int kPoolMaxC = 256;  // longer chunks are pooled segment by segment
+constexpr int kPoolMaxC = 256;  // longest chunk (or window) pooled
 
 template <typename Tin>
-__global__ void __launch_bounds__(64, 12) pool_kernel(const Tin* __restrict__ x0, const Tin* __restrict__ x1,
+__global__ void __launch_bounds__(64, 16) pool_kernel(const Tin* __restrict__ x0, const Tin* __restrict__ x1,
                                                   float* __restrict__ r0, float* __restrict__ r1, int T, int H,
                                                   int d, int C, int out_chunk_stride, float tau) {
   constexpr bool kBf16 = sizeof(Tin) == 2;
@@ -119,29 +124,21 @@ __global__ void __launch_bounds__(64, 12) pool_kernel(const Tin* __restrict__ x0
   const Tin* col = x + ((size_t)b * T + t0) * HD + ch0;
   float s0 = 0.0f, s1 = 0.0f, m0, m1;
   if constexpr (kBf16) {
-    // H*d and ch0 are even, so each bf16 pair is one aligned 32-bit word
+    // H*d and ch0 are even, so each bf16 pair is one aligned 32-bit word.  Two passes
+    // over the chunk, 16 tokens at a time (few registers, so the pools can share the
+    // SMs with a concurrent kernel): the extremes, then the sum of exponentials.
     const uint32_t* colw = reinterpret_cast<const uint32_t*>(col);
     const size_t stride = (size_t)HD / 2;
-    uint32_t w[kPoolSeg];
+    uint32_t hi = __ldg(colw), lo = hi;
+    for (int t0 = 0; t0 < n; t0 += kPoolBlock) {
+      uint32_t w[kPoolBlock];
 #pragma unroll
-    for (int t = 0; t < kPoolSeg; ++t) w[t] = t < n ? __ldg(colw + t * stride) : 0u;
-    uint32_t hi = w[0], lo = w[0];
+      for (int t = 0; t < kPoolBlock; ++t) w[t] = t0 + t < n ? __ldg(colw + (size_t)(t0 + t) * stride) : hi;
 #pragma unroll
-    for (int t = 1; t < kPoolSeg; ++t)
-      if (t < n) {
+      for (int t = 0; t < kPoolBlock; ++t) {
         hi = bf16x2_max(hi, w[t]);
         lo = bf16x2_min(lo, w[t]);
       }
-    // chunks longer than one segment: the extremes over the remaining segments
-    for (int seg = kPoolSeg; seg < n; seg += kPoolSeg) {
-      const int ns = min(kPoolSeg, n - seg);
-#pragma unroll
-      for (int t = 0; t < kPoolSeg; ++t)
-        if (t < ns) {
-          const uint32_t x = __ldg(colw + (size_t)(seg + t) * stride);
-          hi = bf16x2_max(hi, x);
-          lo = bf16x2_min(lo, x);
-        }
     }
     m0 = __fmul_rn(__uint_as_float(hi << 16), inv_tau);
     m1 = __fmul_rn(__uint_as_float(hi & 0xFFFF0000u), inv_tau);
@@ -150,19 +147,9 @@ __global__ void __launch_bounds__(64, 12) pool_kernel(const Tin* __restrict__ x0
     const bool in_range = __fmaf_rn(__uint_as_float(lo << 16), inv_tau, -m0) >= -86.0f &&
                           __fmaf_rn(__uint_as_float(lo & 0xFFFF0000u), inv_tau, -m1) >= -86.0f;
     float2 ss = make_float2(0.0f, 0.0f);
-    if (n <= kPoolSeg) {
-      ss = in_range ? pool_sum_bf16<true>(ss, w, n, inv_tau, m0, m1, K)
-                    : pool_sum_bf16<false>(ss, w, n, inv_tau, m0, m1, K);
-    } else {
-      // segment by segment, still in ascending t
-      for (int seg = 0; seg < n; seg += kPoolSeg) {
-        const int ns = min(kPoolSeg, n - seg);
-#pragma unroll
-        for (int t = 0; t < kPoolSeg; ++t) w[t] = t < ns ? __ldg(colw + (size_t)(seg + t) * stride) : 0u;
-        ss = in_range ? pool_sum_bf16<true>(ss, w, ns, inv_tau, m0, m1, K)
-                      : pool_sum_bf16<false>(ss, w, ns, inv_tau, m0, m1, K);
-      }
-    }
+    for (int t0 = 0; t0 < n; t0 += kPoolBlock)
+      ss = in_range ? pool_sum_bf16<true>(ss, colw, stride, t0, n, inv_tau, m0, m1, K)
+                    : pool_sum_bf16<false>(ss, colw, stride, t0, n, inv_tau, m0, m1, K);
     s0 = ss.x;
     s1 = ss.y;
   } else {
