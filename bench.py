@@ -83,7 +83,10 @@ def whole_job_rate(units_per_rank, ms_max, world):
 #     32K-context step), scaled by 16; per stream it equals the algorithmic bytes
 NCU_TRAFFIC = {
     "compose": (2.0461e9, {"compose_tc.cu": "82d501993514b885", "tc_common.cuh": "c10beda371c1dd4b"}),
-    "decode_main": (3.4694e10, {"decode_stream.cu": "6aebf8bbbdfe238d", "tc_common.cuh": "c10beda371c1dd4b"}),
+    # gate + stream kernels of one step, captured on 4 (dense) and 8 (planted) of the
+    # 64 sequences and scaled by the sequence count (the traffic is per sequence)
+    "decode_main": (3.4638e10, {"decode_stream.cu": "983ccd7e646f1584", "tc_common.cuh": "c10beda371c1dd4b"}),
+    "decode_planted": (5.447e8, {"decode_stream.cu": "983ccd7e646f1584", "tc_common.cuh": "c10beda371c1dd4b"}),
 }
 
 # Datasheet figures of one B200, reported beside the measured denominators: dense
@@ -401,11 +404,12 @@ def run_ours(args):
                         q_route=dev.get("q_route"), k_route=dev.get("k_route"), workspace=pws)
 
     # ---- decode workload ----
-    wd = syn.DECODE_32K
+    wd = syn.DECODE_32K_PLANTED if args.decode_workload == "planted" else syn.DECODE_32K
     if args.decode_B or args.decode_ctx:
         B_ = args.decode_B or wd.B
         T_ = args.decode_ctx or wd.T
-        wd = wd.with_(B=B_, T=T_, name=f"decode_bf16_{B_}seq_ctx{T_}_H16_C64_d128_thr0.05")
+        wd = wd.with_(B=B_, T=T_, name=f"decode_bf16_{B_}seq_ctx{T_}_H16_C64_d128_thr0.05"
+                                       + ("_planted" if args.decode_workload == "planted" else ""))
     if args.skip_decode:
         wd = wd.with_(B=8, T=64 * 4, name="decode_skipped")
     if args.decode_cache != "dense":
@@ -433,7 +437,8 @@ def run_ours(args):
     def decode():
         t = toks[step_idx[0]]
         step_idx[0] += 1
-        hla.hla_decode_step(dcfg, cache, t["q"], t["k"], t["v"], t["alpha"], t["beta"], od, workspace=dws)
+        hla.hla_decode_step(dcfg, cache, t["q"], t["k"], t["v"], t["alpha"], t["beta"], od,
+                            q_route=t.get("q_route"), k_route=t.get("k_route"), workspace=dws)
 
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     flush_read = torch.ones(L2_FLUSH_BYTES // 8, dtype=torch.int64, device="cuda")
@@ -529,7 +534,8 @@ def run_ours(args):
         t_, th = toks[-1], toks_host[-1]
         for k in t_:
             t_[k].copy_(th[k], non_blocking=True)
-        hla.hla_decode_step(dcfg, cache, t_["q"], t_["k"], t_["v"], t_["alpha"], t_["beta"], od, workspace=dws)
+        hla.hla_decode_step(dcfg, cache, t_["q"], t_["k"], t_["v"], t_["alpha"], t_["beta"], od,
+                            q_route=t_.get("q_route"), k_route=t_.get("k_route"), workspace=dws)
         od_host.copy_(od, non_blocking=True)
         e2e_ev[1][1].record(stream)
         torch.cuda.synchronize()
@@ -569,6 +575,8 @@ def run_ours(args):
     bytes_decode = wd.B * wd.H * (n_ctx * (per_chunk + key_reps * wd.d * 4))
     dmain_avg = _stage_avg(stages, "decode", args.steps) or 0.0
     dec_gbs = bytes_decode / (dmain_avg * 1e-3) / 1e9 if dmain_avg > 0 else None
+    if args.decode_workload == "planted":
+        dec_gbs = None  # the active chunks are counted by the planted extra line only
     launches = sum(n for (_, n) in stages.values())
 
     tokens_pre = wp.B * wp.T
@@ -603,7 +611,7 @@ def run_ours(args):
                    "roofline": {"kernel": "decode (gate and stream kernels of the step)", "bound": "hbm", "achieved": dec_gbs, "peak": hbm_gbs,
                                 "unit": "GB/s", "frac": (dec_gbs / hbm_gbs) if dec_gbs else None,
                                 "traffic": ncu_traffic("decode_main") if args.decode_cache == "dense" else None,
-                                "traffic_unit": "bytes per launch (ncu dram read+write)",
+                                "traffic_unit": "bytes per step (ncu dram read+write, gate and stream kernels)",
                                 "peak_source": f"{peak_src} HBM copy",
                                 "datasheet": {"peak": DATASHEET_HBM_GBS,
                                               "frac": (dec_gbs / DATASHEET_HBM_GBS) if dec_gbs else None,
@@ -638,7 +646,8 @@ def run_ours(args):
                                        "frac": (gbs_dp / DATASHEET_HBM_GBS) if gbs_dp else None},
                          "algorithmic": f"{bytes_dp:.4g} bytes per launch ({act_dp} active A_j/B_j of 64 KiB, "
                                         f"counted on the first warm-up step, + all {wdp.T // wdp.C} key pools of "
-                                        f"512 B per sequence and head)", "traffic": None},
+                                        f"512 B per sequence and head)", "traffic": ncu_traffic("decode_planted"),
+                         "traffic_unit": "bytes per step (ncu dram read+write, gate and stream kernels)"},
             "stages_ms_per_step": {k: v[0] / args.steps for k, v in st_dp.items() if v[1]}}
         # the long sparse prefill (B=1, H=32, T=131072, planted, threshold 0.05)
         wsp, ms_sp, pairs_sp, st_sp, sparse_sample = measure_sparse_prefill(
@@ -909,6 +918,9 @@ def main(argv=None):
     ap.add_argument("--decode-B", type=int, default=None, help="decode sequences (default 64)")
     ap.add_argument("--decode-ctx", type=int, default=None, help="decode context tokens (default 32768)")
     ap.add_argument("--skip-decode", action="store_true")
+    ap.add_argument("--decode-workload", choices=["dense", "planted"], default="dense",
+                    help="main decode line: every cached chunk active (dense) or the planted routes "
+                         "(about 4 active chunks per sequence and head)")
     ap.add_argument("--decode-cache", choices=["dense", "factored"], default="dense",
                     help="dense: A_j/B_j d x d (the metric's workload); factored: K_j, Wb_j, Ub_j per chunk")
     ap.add_argument("--chunk", type=int, choices=[64, 128, 256], default=64,

@@ -1,5 +1,5 @@
 // Chunk transitions on tcgen05 tensor cores: bf16 operands, float32 accumulation and
-// a float32 triangular inverse.  d = 128, C = 64.  Persistent CTAs of 4 warps, two per
+// a blocked triangular inverse.  d = 128, C = 64.  Persistent CTAs of 4 warps, two per
 // SM, each walking chunks with a grid-wide stride.
 //
 // HLA summary page, "Methodology in Plain English" para. 1 (a chunk is summarised
@@ -12,9 +12,10 @@
 // Per chunk (M is always 128 by stacking):
 //   TMA   K, V tiles (bf16, 128-byte swizzle)
 //   MMA1  [K; V] (128 x 128) x K^T                  -> rows 0-63: K K^T   (64 cols)
-//   SIMT  L; U = (I + L)^{-1} by 16 x 16 blocks: forward substitution on the four
-//         diagonal blocks, then the off-diagonal blocks level by level,
-//         U_ij = -U_ii sum_{k=j}^{i-1} L_ik U_kj (float32, all 128 threads)
+//   SIMT  L; U = (I + L)^{-1} by 16 x 16 blocks: float32 forward substitution on the
+//         four diagonal blocks, then the off-diagonal blocks level by level,
+//         U_ij = -sum_{k=j}^{i-1} (U_ii L_ik) U_kj, as warp-level tensor-core products
+//         (mma.sync, tf32 inputs, float32 accumulation)
 //   MMA2  [T diag(gamma); T] (128 x 64) x [K | V]   -> rows 0-63: Wb, rows 64-127: Ub
 //   MMA3  Wb^T (128 x 64) x D K (64 x 128)          -> A_c (after gamma_C I - .)
 //   MMA4  Ub^T (128 x 64) x D K                     -> B_c
@@ -74,6 +75,53 @@ struct TransTcArgs {
 };
 
 __device__ __forceinline__ int swz(int row, int chunk) { return row * 128 + ((chunk ^ (row & 7)) << 4); }
+
+#ifndef HLA_TRANS_WARP_MMA
+#define HLA_TRANS_WARP_MMA 1
+#endif
+// Off-diagonal blocks of the inverse on warp-level tensor-core products (tf32
+// inputs, float32 accumulation) instead of CUDA-core dot products.
+constexpr bool kWarpMma = HLA_TRANS_WARP_MMA != 0;
+
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+
+// d += a b on one 16 x 8 x 8 tile (PTX fragment layout of mma.m16n8k8 with tf32:
+// g = lane / 4, q = lane % 4; a: (g, q), (g + 8, q), (g, q + 4), (g + 8, q + 4);
+// b: (k = q, n = g), (k = q + 4, n = g); d: (g, 2q), (g, 2q + 1), (g + 8, 2q), (g + 8, 2q + 1)).
+__device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// acc (16 x 8) = A (16 x KD, row pitch pa floats) times B (KD x 8, row pitch pb), both
+// float32 in shared memory; the warp's lanes hold acc in the layout above.
+template <int KD>
+__device__ __forceinline__ void warp_mma_rows16(float (&acc)[4], const float* A, int pa, const float* B, int pb,
+                                                int lane) {
+  const int g = lane >> 2, q = lane & 3;
+  acc[0] = acc[1] = acc[2] = acc[3] = 0.0f;
+#pragma unroll
+  for (int k0 = 0; k0 < KD; k0 += 8) {
+    const uint32_t af[4] = {to_tf32(A[g * pa + k0 + q]), to_tf32(A[(g + 8) * pa + k0 + q]),
+                            to_tf32(A[g * pa + k0 + q + 4]), to_tf32(A[(g + 8) * pa + k0 + q + 4])};
+    const uint32_t bf[2] = {to_tf32(B[(k0 + q) * pb + g]), to_tf32(B[(k0 + q + 4) * pb + g])};
+    mma_tf32_16x8x8(acc, af, bf);
+  }
+}
+
+// Stores s * acc at D (16 x 8, row pitch pd).
+__device__ __forceinline__ void warp_store_rows16(float* D, int pd, const float (&acc)[4], float s, int lane) {
+  const int g = lane >> 2, q = lane & 3;
+  *(float2*)(D + g * pd + 2 * q) = make_float2(s * acc[0], s * acc[1]);
+  *(float2*)(D + (g + 8) * pd + 2 * q) = make_float2(s * acc[2], s * acc[3]);
+}
 
 struct ChunkPos {
   int i, b, h, t0, n;
@@ -339,9 +387,57 @@ __global__ void __launch_bounds__(128, 2)
     }
     ok = tc::bar_all(1, 128, ok);
     // Off-diagonal blocks.  With L'_ik = U_ii L_ik (k < i),  U_ij = -sum_{k=j}^{i-1} L'_ik U_kj,
-    // one level (i - j = 1, 2, 3) after the other.  Thread = (column c, rows tb and tb + 8).
+    // one level (i - j = 1, 2, 3) after the other.
+    if (kWarpMma) {
+      // warp-level products: a unit is one 16 x 8 half (column half nh) of a block
+      if (ok) {
+        // L'_ik for (i, k) = (1,0) (2,0) (2,1) (3,0) (3,1) (3,2): 12 units, 3 per warp
+#pragma unroll
+        for (int r = 0; r < 3; ++r) {
+          const int u = warp + 4 * r, blk = u >> 1, nh = u & 1;
+          const int ib = blk < 1 ? 1 : (blk < 3 ? 2 : 3);
+          const int kb = blk - (ib * (ib - 1)) / 2;
+          float acc[4];
+          warp_mma_rows16<16>(acc, Usm + 16 * ib * kLP + 16 * ib, kLP, Lsm + 16 * ib * kLP + 16 * kb + 8 * nh, kLP,
+                              lane);
+          warp_store_rows16(Xsm + (16 * ib - 16) * kXP + 16 * kb + 8 * nh, kXP, acc, 1.0f, lane);
+        }
+      }
+      ok = tc::bar_all(1, 128, ok);
+      if (ok) {
+        // level 1: U_{j+1,j} = -L'_{j+1,j} U_jj, j = 0, 1, 2 (6 units)
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const int u = warp + 4 * r;
+          if (u < 6) {
+            const int jb = u >> 1, nh = u & 1;
+            float acc[4];
+            warp_mma_rows16<16>(acc, Xsm + 16 * jb * kXP + 16 * jb, kXP, Usm + 16 * jb * kLP + 16 * jb + 8 * nh, kLP,
+                                lane);
+            warp_store_rows16(Usm + 16 * (jb + 1) * kLP + 16 * jb + 8 * nh, kLP, acc, -1.0f, lane);
+          }
+        }
+      }
+      ok = tc::bar_all(1, 128, ok);
+      if (ok) {
+        // level 2: U_{j+2,j} = -(L'_{j+2,j} U_jj + L'_{j+2,j+1} U_{j+1,j}), j = 0, 1 (4 units)
+        const int jb = warp >> 1, nh = warp & 1;
+        float acc[4];
+        warp_mma_rows16<32>(acc, Xsm + 16 * (jb + 1) * kXP + 16 * jb, kXP, Usm + 16 * jb * kLP + 16 * jb + 8 * nh,
+                            kLP, lane);
+        warp_store_rows16(Usm + 16 * (jb + 2) * kLP + 16 * jb + 8 * nh, kLP, acc, -1.0f, lane);
+      }
+      ok = tc::bar_all(1, 128, ok);
+      if (ok && warp < 2) {
+        // level 3: U_30 = -(L'_30 U_00 + L'_31 U_10 + L'_32 U_20) (2 units)
+        float acc[4];
+        warp_mma_rows16<48>(acc, Xsm + 32 * kXP, kXP, Usm + 8 * warp, kLP, lane);
+        warp_store_rows16(Usm + 48 * kLP + 8 * warp, kLP, acc, -1.0f, lane);
+      }
+      ok = tc::bar_all(1, 128, ok);
+    }
     const int cc16 = tid & 15, tb = tid >> 4;
-    if (ok) {
+    if (!kWarpMma && ok) {
 #pragma unroll
       for (int ib = 1; ib < 4; ++ib) {
         float ua[16], ub[16];  // U_ii rows tb, tb + 8
@@ -366,9 +462,9 @@ __global__ void __launch_bounds__(128, 2)
         }
       }
     }
-    ok = tc::bar_all(1, 128, ok);
+    if (!kWarpMma) ok = tc::bar_all(1, 128, ok);
 #pragma unroll
-    for (int lev = 1; lev < 4; ++lev) {
+    for (int lev = 1; lev < 4 && !kWarpMma; ++lev) {
       if (ok) {
 #pragma unroll
         for (int jb = 0; jb + lev < 4; ++jb) {
