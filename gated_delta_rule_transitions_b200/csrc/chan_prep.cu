@@ -22,9 +22,12 @@
 // overflow it; the kernel then records kErrDecayRange (hla_device_status reports it)
 // and that prefill's outputs are not valid.
 //
-// One CTA per (sub-chunk, b, h), thread = channel.  Tokens past the end of the
-// sequence (a final partial sub-chunk) are identity tokens: alpha = 1, and their
-// rows of Kt, Kh, Kc and Qt are zero.
+// One CTA per (sub-chunk, b, h) of 128 threads: thread = (token half, channel pair),
+// so that every access moves two adjacent channels (float2 decays, bf16 pairs).  The
+// cumulative sums run in ascending token order (the second half continues from the
+// first half's total).  Tokens past the end of the sequence (a final partial
+// sub-chunk) are identity tokens: alpha = 1, and their rows of Kt, Kh, Kc and Qt are
+// zero.
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -35,47 +38,92 @@ HLA_DEFINE_ERROR_WORD(chan_prep)
 namespace {
 
 constexpr int kSub = 64;
+constexpr int kHalf = kSub / 2;
 constexpr int kD = 128;
 
-__global__ void __launch_bounds__(kD) chan_prep_kernel(ChanPrepArgs a) {
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+__global__ void __launch_bounds__(128) chan_prep_kernel(ChanPrepArgs a) {
+  __shared__ float2 tot_s[2][kD / 2];
   const int sub = blockIdx.x;
   const int bh = blockIdx.y;
   const int b = bh / a.H, h = bh - b * a.H;
-  const int c = threadIdx.x;
+  const int cp = threadIdx.x & (kD / 2 - 1);  // channels 2 cp, 2 cp + 1
+  const int half = threadIdx.x >> 6;          // tokens kHalf * half ...
   const int t0 = sub * kSub;
   const int n = min(kSub, a.T - t0);
   const long HD = (long)a.H * kD;
-  const long row0 = ((long)b * a.T + t0) * HD + (long)h * kD + c;  // (b, t0, h, c) of [B,T,H,d]
-  // pass 1: l_t per channel (identity tokens past the end: log alpha = 0)
-  float ell[kSub];
-  float acc = 0.0f;
+  const long e0 = ((long)b * a.T + t0) * HD + (long)h * kD + 2 * cp;  // (b, t0, h, 2 cp) of [B,T,H,d]
+  // pass 1: log alpha of this thread's tokens (identity tokens past the end: 0) ...
+  const float2* alpha2 = reinterpret_cast<const float2*>(a.alpha);
+  float2 ell[kHalf];
 #pragma unroll
-  for (int t = 0; t < kSub; ++t) {
-    if (t < n) acc += __logf(a.alpha[row0 + (long)t * HD]);
-    ell[t] = acc;
-  }
-  const long chunk = (long)bh * a.Nsub + sub;
-  a.gC[chunk * kD + c] = __expf(acc);
-  if (-acc > 80.0f && n > 0) report_device_error(kErrDecayRange);
-  // pass 2: the four operands, row t of each at (chunk * 64 + t) * 128 + c
-  const __nv_bfloat16* k = (const __nv_bfloat16*)a.k;
-  const __nv_bfloat16* q = (const __nv_bfloat16*)a.q;
-  __nv_bfloat16* Kt = (__nv_bfloat16*)a.Kt + chunk * kSub * kD + c;
-  __nv_bfloat16* Kh = (__nv_bfloat16*)a.Kh + chunk * kSub * kD + c;
-  __nv_bfloat16* Kc = (__nv_bfloat16*)a.Kc + chunk * kSub * kD + c;
-  __nv_bfloat16* Qt = (__nv_bfloat16*)a.Qt + chunk * kSub * kD + c;
-#pragma unroll
-  for (int t = 0; t < kSub; ++t) {
-    float kv = 0.0f, qv = 0.0f;
+  for (int u = 0; u < kHalf; ++u) {
+    const int t = kHalf * half + u;
+    ell[u] = make_float2(0.0f, 0.0f);
     if (t < n) {
-      kv = __bfloat162float(k[row0 + (long)t * HD]);
-      qv = __bfloat162float(q[row0 + (long)t * HD]);
+      const float2 al = alpha2[(e0 + (long)t * HD) >> 1];
+      ell[u] = make_float2(__logf(al.x), __logf(al.y));
     }
-    const float e = __expf(ell[t]);
-    Kt[t * kD] = __float2bfloat16_rn(kv * e);
-    Kh[t * kD] = __float2bfloat16_rn(kv * __expf(-ell[t]));
-    Kc[t * kD] = __float2bfloat16_rn(kv * __expf(acc - ell[t]));
-    Qt[t * kD] = __float2bfloat16_rn(qv * e);
+  }
+  // ... then l_t, the running sums over the sub-chunk in ascending t
+  float2 acc = make_float2(0.0f, 0.0f);
+  if (half == 0) {
+#pragma unroll
+    for (int u = 0; u < kHalf; ++u) {
+      acc.x += ell[u].x;
+      acc.y += ell[u].y;
+      ell[u] = acc;
+    }
+    tot_s[0][cp] = acc;
+  }
+  __syncthreads();
+  if (half == 1) {
+    acc = tot_s[0][cp];
+#pragma unroll
+    for (int u = 0; u < kHalf; ++u) {
+      acc.x += ell[u].x;
+      acc.y += ell[u].y;
+      ell[u] = acc;
+    }
+    tot_s[1][cp] = acc;
+  }
+  __syncthreads();
+  acc = tot_s[1][cp];  // l_C
+  const long chunk = (long)bh * a.Nsub + sub;
+  if (half == 1) {
+    *reinterpret_cast<float2*>(a.gC + chunk * kD + 2 * cp) = make_float2(__expf(acc.x), __expf(acc.y));
+    if ((-acc.x > 80.0f || -acc.y > 80.0f) && n > 0) report_device_error(kErrDecayRange);
+  }
+  // pass 2: the four operands, row t of each at (chunk * 64 + t) * 128 + c
+  const uint32_t* k2 = reinterpret_cast<const uint32_t*>(a.k);
+  const uint32_t* q2 = reinterpret_cast<const uint32_t*>(a.q);
+  const long o0 = (chunk * kSub) * (kD / 2) + cp;  // 32-bit word of (chunk row 0, channel pair cp)
+  uint32_t* Kt = reinterpret_cast<uint32_t*>(a.Kt) + o0;
+  uint32_t* Kh = reinterpret_cast<uint32_t*>(a.Kh) + o0;
+  uint32_t* Kc = reinterpret_cast<uint32_t*>(a.Kc) + o0;
+  uint32_t* Qt = reinterpret_cast<uint32_t*>(a.Qt) + o0;
+#pragma unroll
+  for (int u = 0; u < kHalf; ++u) {
+    const int t = kHalf * half + u;
+    float k0 = 0.0f, k1 = 0.0f, q0 = 0.0f, q1 = 0.0f;
+    if (t < n) {
+      const uint32_t kw = k2[(e0 + (long)t * HD) >> 1];
+      const uint32_t qw = q2[(e0 + (long)t * HD) >> 1];
+      k0 = __uint_as_float(kw << 16);
+      k1 = __uint_as_float(kw & 0xFFFF0000u);
+      q0 = __uint_as_float(qw << 16);
+      q1 = __uint_as_float(qw & 0xFFFF0000u);
+    }
+    const float ex = __expf(ell[u].x), ey = __expf(ell[u].y);
+    const long row = (long)t * (kD / 2);
+    Kt[row] = bf16x2_bits(k0 * ex, k1 * ey);
+    Kh[row] = bf16x2_bits(k0 * __expf(-ell[u].x), k1 * __expf(-ell[u].y));
+    Kc[row] = bf16x2_bits(k0 * __expf(acc.x - ell[u].x), k1 * __expf(acc.y - ell[u].y));
+    Qt[row] = bf16x2_bits(q0 * ex, q1 * ey);
   }
 }
 

@@ -1,6 +1,8 @@
 // Routing kernels: per-chunk log-mean-exp pools, gates and compacted active lists.
 // Built with -fmad=false; the recipe's products and sums are __f*_rn intrinsics or
 // explicit fused multiply-adds.
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.cuh"
 #include "routing_recipe.cuh"
@@ -180,6 +182,113 @@ __global__ void __launch_bounds__(64, 16) pool_kernel(const Tin* __restrict__ x0
 }
 
 // ---------------------------------------------------------------------------
+// Pools of bf16 inputs with chunks of up to 64 tokens, staged through shared memory.
+// A unit is (tensor, b, chunk, group of 64 channels): a tile of n <= 64 token rows of
+// 128 bytes.  Each warp walks units with a grid-wide stride and keeps two tile
+// buffers: the next unit's rows are in flight (16-byte cp.async, one 128-byte row
+// per 8 lanes) while the current one is reduced, lane = two adjacent channels.  The
+// arithmetic, and so every bit, is that of pool_kernel.
+// ---------------------------------------------------------------------------
+constexpr int kTileWarps = 4;
+constexpr int kTileRows = 64;
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+struct PoolTileArgs {
+  const __nv_bfloat16* x[2];
+  float* r[2];
+  int B, T, H, d, C, N, out_chunk_stride, groups;
+  long units;
+  float tau;
+};
+
+__device__ __forceinline__ void pool_tile_fetch(const PoolTileArgs& a, long u, uint32_t buf, int lane, int& n) {
+  const int g = (int)(u % a.groups);
+  long r = u / a.groups;
+  const int c = (int)(r % a.N);
+  r /= a.N;
+  const int b = (int)(r % a.B);
+  const int which = (int)(r / a.B);
+  const int t0 = c * a.C;
+  n = min(a.C, a.T - t0);
+  const long HD = (long)a.H * a.d;
+  const __nv_bfloat16* x = which == 0 ? a.x[0] : a.x[1];
+  const char* src = (const char*)(x + ((long)b * a.T + t0) * HD + g * 64) + (lane & 7) * 16;
+  for (int t = lane >> 3; t < n; t += 4) cp_async16(buf + t * 128 + (lane & 7) * 16, src + (long)t * HD * 2);
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(32 * kTileWarps) pool_tile_kernel(PoolTileArgs a) {
+  extern __shared__ __align__(16) uint8_t pool_sm[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t base = (uint32_t)__cvta_generic_to_shared(pool_sm) + warp * 2 * kTileRows * 128;
+  const uint32_t* words = reinterpret_cast<const uint32_t*>(pool_sm + warp * 2 * kTileRows * 128);
+  const long stride = (long)gridDim.x * kTileWarps;
+  long u = (long)blockIdx.x * kTileWarps + warp;
+  if (u >= a.units) return;
+  const route::Consts K = route::make_consts();
+  const float inv_tau = __fdiv_rn(1.0f, a.tau);
+  int n_cur = 0, n_next = 0;
+  pool_tile_fetch(a, u, base, lane, n_cur);
+  for (int k = 0; u < a.units; u += stride, ++k) {
+    const int cur = k & 1;
+    const bool more = u + stride < a.units;
+    if (more) {
+      pool_tile_fetch(a, u + stride, base + (cur ^ 1) * kTileRows * 128, lane, n_next);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+    }
+    __syncwarp();
+    const uint32_t* w = words + cur * kTileRows * 32 + lane;
+    const int n = n_cur;
+    uint32_t hi = w[0], lo = hi;
+    for (int t = 1; t < n; ++t) {
+      hi = bf16x2_max(hi, w[t * 32]);
+      lo = bf16x2_min(lo, w[t * 32]);
+    }
+    const float m0 = __fmul_rn(__uint_as_float(hi << 16), inv_tau);
+    const float m1 = __fmul_rn(__uint_as_float(hi & 0xFFFF0000u), inv_tau);
+    const bool in_range = __fmaf_rn(__uint_as_float(lo << 16), inv_tau, -m0) >= -86.0f &&
+                          __fmaf_rn(__uint_as_float(lo & 0xFFFF0000u), inv_tau, -m1) >= -86.0f;
+    float2 s = make_float2(0.0f, 0.0f);
+    if (in_range) {
+#pragma unroll 8
+      for (int t = 0; t < n; ++t) {
+        const uint32_t x = w[t * 32];
+        const float2 v = __ffma2_rn(make_float2(__uint_as_float(x << 16), __uint_as_float(x & 0xFFFF0000u)),
+                                    make_float2(inv_tau, inv_tau), make_float2(-m0, -m1));
+        s = __fadd2_rn(s, rexp2<true>(v, K));
+      }
+    } else {
+#pragma unroll 8
+      for (int t = 0; t < n; ++t) {
+        const uint32_t x = w[t * 32];
+        const float2 v = __ffma2_rn(make_float2(__uint_as_float(x << 16), __uint_as_float(x & 0xFFFF0000u)),
+                                    make_float2(inv_tau, inv_tau), make_float2(-m0, -m1));
+        s = __fadd2_rn(s, rexp2<false>(v, K));
+      }
+    }
+    __syncwarp();  // every lane has read the buffer before the next fetch refills it
+    const float v0 = __fmul_rn(a.tau, __fadd_rn(m0, route::rlog(__fdiv_rn(s.x, (float)n), K)));
+    const float v1 = __fmul_rn(a.tau, __fadd_rn(m1, route::rlog(__fdiv_rn(s.y, (float)n), K)));
+    const int g = (int)(u % a.groups);
+    long r = u / a.groups;
+    const int c = (int)(r % a.N);
+    r /= a.N;
+    const int b = (int)(r % a.B);
+    const int which = (int)(r / a.B);
+    const int ch = g * 64 + 2 * lane;
+    const int h = ch / a.d, cc = ch - h * a.d;
+    float* out = which == 0 ? a.r[0] : a.r[1];
+    *reinterpret_cast<float2*>(out + (((long)b * a.H + h) * a.out_chunk_stride + c) * a.d + cc) = make_float2(v0, v1);
+    n_cur = n_next;
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Gates + active lists.  One warp per query-chunk row (b, h, i).  Lane j' handles
 // j = jb + lane; the dot product runs over channels in ascending order.  Active j
 // (ascending) are compacted with a warp ballot.
@@ -244,7 +353,7 @@ __global__ void __launch_bounds__(256) gates_kernel(GatesArgs a) {
 // Routed gates, tiled: one CTA per (TI query chunks, b, h), 256 threads.  A thread
 // computes 4 rows x CPT columns of a TI x 64 gate tile (TI = 64: 4 x 4; TI = 16,
 // for grids too small to fill the GPU: 4 x 1).  Every dot product still runs over
-// channels in ascending order with separately rounded products and sums, so the
+// channels in ascending order, one fused multiply-add per channel, so the
 // bits equal the per-pair recipe.  Active chunks are compacted row by row in
 // ascending j.
 // ---------------------------------------------------------------------------
@@ -263,8 +372,12 @@ __global__ void __launch_bounds__(256) gates_tiled_kernel(GatesArgs a) {
   float(*rkT)[TJ] = reinterpret_cast<float(*)[TJ]>(smf + D * TI);   // [D][TJ] rk tile, channel-major
   float(*G)[TJ + 1] = reinterpret_cast<float(*)[TJ + 1]>(smf + D * TI + D * TJ);  // [TI][TJ+1]
   int* cnt_s = reinterpret_cast<int*>(smf + D * TI + D * TJ + TI * (TJ + 1));      // [TI]
-  const int i0 = blockIdx.x * TI;
-  const int bh = blockIdx.y;
+  // 1-D grid in descending row-tile order over all heads: the CTAs with the most key
+  // tiles (the last query chunks) start first, the short ones fill the tail
+  const int nrt = (a.N + TI - 1) / TI;
+  const int BHn = a.B * a.H;
+  const int i0 = (nrt - 1 - (int)(blockIdx.x / BHn)) * TI;
+  const int bh = (int)(blockIdx.x % BHn);
   const int tid = threadIdx.x;
   const int ty = tid / NTX, tx = tid % NTX;
   const int warp = tid >> 5, lane = tid & 31;
@@ -411,7 +524,7 @@ __global__ void __launch_bounds__(256) gates_tiled_kernel(GatesArgs a) {
 
 template <int D, int TI>
 static cudaError_t launch_gates_tiled(const GatesArgs& a, cudaStream_t s) {
-  dim3 grid((a.N + TI - 1) / TI, a.B * a.H);
+  const unsigned grid = (unsigned)(((a.N + TI - 1) / TI) * a.B * a.H);
   const size_t smem = (size_t)(D * TI + D * 64 + TI * 65 + TI) * 4;
   cudaError_t e = cudaFuncSetAttribute(gates_tiled_kernel<D, TI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
@@ -552,6 +665,34 @@ cudaError_t launch_pools(const void* x0, const void* x1, float* r0, float* r1, i
                          int C, int out_chunk_stride, float tau, int dtype, cudaStream_t s) {
   if (C > kPoolMaxC) return cudaErrorInvalidValue;
   const int N = (T + C - 1) / C;
+  if (dtype == HLA_BF16 && C <= kTileRows && (H * d) % 64 == 0 && (x0 != nullptr) == (r0 != nullptr) &&
+      (x1 != nullptr) == (r1 != nullptr)) {
+    PoolTileArgs a{};
+    const int nt = (x0 != nullptr) + (x1 != nullptr);
+    if (nt == 0) return cudaSuccess;
+    // the present tensors first
+    a.x[0] = (const __nv_bfloat16*)(x0 ? x0 : x1);
+    a.r[0] = x0 ? r0 : r1;
+    a.x[1] = (const __nv_bfloat16*)x1;
+    a.r[1] = r1;
+    a.B = B;
+    a.T = T;
+    a.H = H;
+    a.d = d;
+    a.C = C;
+    a.N = N;
+    a.out_chunk_stride = out_chunk_stride;
+    a.groups = H * d / 64;
+    a.units = (long)nt * B * N * a.groups;
+    a.tau = tau;
+    const int smem = kTileWarps * 2 * kTileRows * 128;
+    cudaError_t e = cudaFuncSetAttribute(pool_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    const long want = (a.units + kTileWarps - 1) / kTileWarps;
+    const int blocks = (int)std::min<long>(want, 3L * num_sms());
+    pool_tile_kernel<<<blocks, 32 * kTileWarps, smem, s>>>(a);
+    return cudaGetLastError();
+  }
   const int groups = (H * d + 127) / 128;
   dim3 grid(N, B, 2 * groups);
   if (dtype == HLA_BF16)

@@ -54,7 +54,7 @@ constexpr int kX = kScr + 2 * kLU;            // 16 KiB: L' (rows 16-63); then B
 constexpr int kXP = 52;                       // row pitch (floats) of L'
 constexpr int kSmall = kX + 16384;            // per-token scalars, barriers
 constexpr int kBars = 6;                      // tma, mma1, mma2, mma34, Kh, Kc
-constexpr int kSmemUsed = kSmall + 4 * kC * 4 + kBars * 8 + 32;
+constexpr int kSmemUsed = kSmall + 6 * kC * 4 + kBars * 8 + 48;
 static_assert(kX % 1024 == 0 && 48 * kXP * 4 <= 16384, "shared-memory layout");
 constexpr uint32_t kIdesc1 = tc::idesc_bf16_f32(128, 64, 0, 0);
 constexpr uint32_t kIdesc2 = tc::idesc_bf16_f32(128, 256, 0, 1);
@@ -82,6 +82,15 @@ __device__ __forceinline__ int swz(int row, int chunk) { return row * 128 + ((ch
 // Off-diagonal blocks of the inverse on warp-level tensor-core products (tf32
 // inputs, float32 accumulation) instead of CUDA-core dot products.
 constexpr bool kWarpMma = HLA_TRANS_WARP_MMA != 0;
+
+#ifndef HLA_TRANS_DECAY_PRODUCT
+#define HLA_TRANS_DECAY_PRODUCT 1
+#endif
+// Scalar decay: the pair decays e^{l_t - l_s} of L as e^{l_t} e^{-l_s} (two per-token
+// exponentials instead of one per pair) when every |l_t| of the chunk is at most 80,
+// so that both factors stay normal float32 numbers; else one exponential per pair.
+constexpr bool kDecayProduct = HLA_TRANS_DECAY_PRODUCT != 0;
+constexpr float kProductRange = 80.0f;
 
 __device__ __forceinline__ uint32_t to_tf32(float x) {
   uint32_t r;
@@ -191,10 +200,13 @@ __global__ void __launch_bounds__(128, 2)
   float* beta_s = ell_s + kC;                    // beta_t
   float* bg_s = beta_s + kC;                     // beta_t gamma_t
   float* dk_s = bg_s + kC;                       // gamma_C / gamma_t
-  uint64_t* bars = (uint64_t*)(dk_s + kC);       // tma, mma1, mma2, mma34, Kh, Kc
+  float* gam_s = dk_s + kC;                      // e^{l_t}
+  float* igam_s = gam_s + kC;                    // e^{-l_t}
+  uint64_t* bars = (uint64_t*)(igam_s + kC);     // tma, mma1, mma2, mma34, Kh, Kc
   uint32_t* tmem_s = (uint32_t*)(bars + kBars);
   float* wsum = (float*)(tmem_s + 2);            // [2]
-  volatile int* abort_s = (volatile int*)(wsum + 2);
+  uint32_t* lmax_s = (uint32_t*)(wsum + 2);      // [2] largest |l_t| bits of each half chunk
+  volatile int* abort_s = (volatile int*)(lmax_s + 2);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -275,6 +287,11 @@ __global__ void __launch_bounds__(128, 2)
       if (warp == 1) la += wsum[0];
       ell_s[tid] = la;
       if (a.ell) a.ell[chunk * kC + tid] = la;
+      if (kDecayProduct) {
+        // |l| >= 0, so its bits order like the values (a NaN compares above every bound)
+        const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(fabsf(la)));
+        if (lane == 0) lmax_s[warp] = m;
+      }
     }
     // the K/V tile has landed (the previous chunk's staged stores may still be reading
     // shared memory: they are waited for before the L rows are written)
@@ -307,8 +324,13 @@ __global__ void __launch_bounds__(128, 2)
       // per-token scales, while the MMA runs
       const int s = tid - kC;
       const float ls = ell_s[s];
-      bg_s[s] = beta_s[s] * __expf(ls);
+      const float e = __expf(ls);
+      bg_s[s] = beta_s[s] * e;
       dk_s[s] = __expf(ell_s[kC - 1] - ls);
+      if (kDecayProduct) {
+        gam_s[s] = e;
+        igam_s[s] = __expf(-ls);
+      }
     }
     {
       // MMA1 is done and the previous chunk's staged stores have read shared memory
@@ -350,7 +372,24 @@ __global__ void __launch_bounds__(128, 2)
       tc::tc_fence_before();
     }
     ok = tc::bar_all(1, 128, ok);
-    if (!kChan && ok) {
+    const bool product = kDecayProduct && max(lmax_s[0], lmax_s[1]) <= __float_as_uint(kProductRange);
+    if (!kChan && ok && product) {
+      const int t = tid & (kC - 1), hs = tid >> 6;
+      const float gt = gam_s[t];
+      float* Lrow = Lsm + t * kLP;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const int s4 = 32 * hs + 4 * q;
+        const float4 i4 = *(const float4*)(igam_s + s4);
+        const float4 g4 = *(const float4*)(Lrow + s4);
+        float4 v;
+        v.x = (s4 + 0 < t) ? (gt * i4.x) * g4.x : 0.0f;
+        v.y = (s4 + 1 < t) ? (gt * i4.y) * g4.y : 0.0f;
+        v.z = (s4 + 2 < t) ? (gt * i4.z) * g4.z : 0.0f;
+        v.w = (s4 + 3 < t) ? (gt * i4.w) * g4.w : 0.0f;
+        *(float4*)(Lrow + s4) = v;
+      }
+    } else if (!kChan && ok) {
       const int t = tid & (kC - 1), hs = tid >> 6;
       const float lt = ell_s[t];
       float* Lrow = Lsm + t * kLP;

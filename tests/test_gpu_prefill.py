@@ -176,6 +176,44 @@ def test_gdn_chunk_transitions(hla, dtype, d):
                     P.check_bf16(Bm[b, h, c], Br, "transition", tol=1e-2)
 
 
+def test_gdn_chunk_transitions_strong_decay(hla):
+    """Chunks whose accumulated decay exceeds e^80 (the pair decays then come from one
+    exponential per pair, not from per-token factors) next to weakly decaying ones.
+    Where the chunk's decay is beyond e^-60, A_c is of the order of gamma_C, at the
+    bottom of the float32 / bf16 range, so A_c is checked in absolute terms there and
+    B_c (of order one: the last tokens' keys barely decay) relatively."""
+    w = syn.TINY_F32.with_(dtype="bf16", d=128, B=1, H=2, T=64 * 4)
+    inp = P.gpu_inputs(w)
+    gen = torch.Generator().manual_seed(77)
+    # log alpha per chunk: about -0.05 (weak), -2 (|l| reaches about 128), -1.3 (about
+    # 83 at the end of the chunk), and -40 on a single token of an otherwise weak chunk
+    la = torch.empty(1, w.T, 2)
+    la[:, 0:64] = -0.05
+    la[:, 64:128] = -2.0
+    la[:, 128:192] = -1.3
+    la[:, 192:256] = -0.05
+    la[:, 224] = -40.0
+    la = la * (1.0 + 0.1 * torch.rand(la.shape, generator=gen))
+    inp["alpha"] = torch.exp(la).float().contiguous()
+    cfg = hla.make_config(1, 2, w.T, 64, 128, "bf16")
+    g = P.to_cuda(inp)
+    A = torch.empty((1, 2, w.T // 64, 128, 128), dtype=torch.bfloat16, device="cuda")
+    Bm = torch.empty_like(A)
+    hla.gdn_chunk_transitions(cfg, g["k"], g["v"], g["alpha"], g["beta"], A, Bm)
+    torch.cuda.synchronize()
+    A, Bm = P.np64(A), P.np64(Bm)
+    for h in range(2):
+        for c in range(w.T // 64):
+            sl = slice(64 * c, 64 * c + 64)
+            Ar, Br = ho.chunk_transition(P.np64(inp["k"][0, sl, h]), P.np64(inp["v"][0, sl, h]),
+                                         P.np64(inp["alpha"][0, sl, h]), P.np64(inp["beta"][0, sl, h]))
+            if -np.log(P.np64(inp["alpha"][0, sl, h])).sum() > 60.0:
+                assert np.abs(A[0, h, c]).max() <= 1e-20 and np.abs(Ar).max() <= 1e-20
+            else:
+                P.check_bf16(A[0, h, c], Ar, "transition", tol=1e-2)
+            P.check_bf16(Bm[0, h, c], Br, "transition", tol=1e-2)
+
+
 @pytest.mark.parametrize("dtype,d,T", [("f32", 64, 64 * 7 + 3), ("bf16", 128, 64 * 9)])
 def test_routing_bit_exact(hla, dtype, d, T):
     w = syn.PREFILL_0P8B.with_(B=2, H=3, T=T, dtype=dtype, d=d, thr=0.3)
@@ -210,6 +248,8 @@ def test_routing_bit_exact(hla, dtype, d, T):
     (128, 3, 64 * 8 + 5, 0.05, 30.0),
     # enough 64-row gate tiles to fill the GPU at d = 64 (the 64-row kernel)
     (64, 37, 64 * 512, 1.0, 1.0),
+    # several pool tiles per warp of the staged pool kernel, ending in a partial chunk
+    (128, 4, 64 * 1000 + 17, 1.0, 1.0),
 ])
 def test_routing_bit_exact_ranges(hla, d, H, T, tau, scale):
     gen = torch.Generator().manual_seed(123)
