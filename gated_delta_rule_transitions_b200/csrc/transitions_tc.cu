@@ -125,6 +125,37 @@ __device__ __forceinline__ void warp_mma_rows16(float (&acc)[4], const float* A,
   }
 }
 
+// 32 lanes x 16 columns of 32-bit from tensor memory.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+// Waits for this thread's tensor-memory loads; the registers of the last two loads are
+// operands, so no use of them is scheduled before the wait.
+__device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&x)[16], uint32_t (&y)[16]) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(x[0]), "+r"(x[1]), "+r"(x[2]), "+r"(x[3]), "+r"(x[4]), "+r"(x[5]), "+r"(x[6]), "+r"(x[7]),
+        "+r"(x[8]), "+r"(x[9]), "+r"(x[10]), "+r"(x[11]), "+r"(x[12]), "+r"(x[13]), "+r"(x[14]), "+r"(x[15]),
+        "+r"(y[0]), "+r"(y[1]), "+r"(y[2]), "+r"(y[3]), "+r"(y[4]), "+r"(y[5]), "+r"(y[6]), "+r"(y[7]),
+        "+r"(y[8]), "+r"(y[9]), "+r"(y[10]), "+r"(y[11]), "+r"(y[12]), "+r"(y[13]), "+r"(y[14]), "+r"(y[15])
+      :
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&x)[16]) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(x[0]), "+r"(x[1]), "+r"(x[2]), "+r"(x[3]), "+r"(x[4]), "+r"(x[5]), "+r"(x[6]), "+r"(x[7]),
+        "+r"(x[8]), "+r"(x[9]), "+r"(x[10]), "+r"(x[11]), "+r"(x[12]), "+r"(x[13]), "+r"(x[14]), "+r"(x[15])
+      :
+      : "memory");
+}
+
 // Stores s * acc at D (16 x 8, row pitch pd).
 __device__ __forceinline__ void warp_store_rows16(float* D, int pd, const float (&acc)[4], float s, int lane) {
   const int g = lane >> 2, q = lane & 3;
@@ -146,6 +177,30 @@ __device__ __forceinline__ ChunkPos chunk_pos(const TransTcArgs& a, long chunk) 
   p.t0 = p.i * kC;
   p.n = min(kC, a.T - p.t0);
   return p;
+}
+
+// The position `stride` = qN * N + rN chunks after p (the persistent loop's step),
+// without 64-bit divisions: the chunk index wraps into the next (b, h) at most once
+// beyond the qN whole heads, and (b, h) is stepped from p's.
+__device__ __forceinline__ ChunkPos step_pos(const TransTcArgs& a, const ChunkPos& p, int qN, int rN) {
+  ChunkPos n;
+  n.i = p.i + rN;
+  int dbh = qN;
+  if (n.i >= a.N) {
+    n.i -= a.N;
+    ++dbh;
+  }
+  n.bh = p.bh + dbh;
+  n.h = p.h + dbh;
+  n.b = p.b;
+  if (n.h >= a.H) {
+    const int q = n.h / a.H;
+    n.b += q;
+    n.h -= q * a.H;
+  }
+  n.t0 = n.i * kC;
+  n.n = min(kC, a.T - n.t0);
+  return n;
 }
 
 // The K (kChan: Kt, rows chunk * 64 + t of the prepared operand) and V tiles of a chunk.
@@ -247,17 +302,20 @@ __global__ void __launch_bounds__(128, 2)
   int it = 0, ph3 = 0, ph5 = 0;
   bool kh_pending = false, kc_pending = false;  // thread 0 (kChan): a Kh / Kc load in flight
   float pa = 1.0f, pb = 0.0f;  // alpha, beta of token `tid` of the chunk to come
+  // this CTA's chunk and the one after it (the loop steps both by gridDim.x)
+  const int qN = (int)(gridDim.x / (unsigned)a.N), rN = (int)(gridDim.x % (unsigned)a.N);
+  ChunkPos P = chunk_pos(a, blockIdx.x);
+  ChunkPos Pn = P;
   if (blockIdx.x < a.total) {
-    const ChunkPos p0 = chunk_pos(a, blockIdx.x);
     if (tid == 0) {
-      load_kv<kChan>(sm, &tmK, &tmV, &bars[0], a, p0, blockIdx.x);
+      load_kv<kChan>(sm, &tmK, &tmV, &bars[0], a, P, blockIdx.x);
       load_pending = true;
       load_parity = 0;
     }
-    if (tid < kC) load_ab<kChan>(a, p0, tid, pa, pb);
+    if (tid < kC) load_ab<kChan>(a, P, tid, pa, pb);
   }
-  for (long chunk = blockIdx.x; ok && chunk < a.total; chunk += gridDim.x, ++it) {
-    const ChunkPos P = chunk_pos(a, chunk);
+  for (long chunk = blockIdx.x; ok && chunk < a.total; chunk += gridDim.x, ++it, P = Pn) {
+    Pn = step_pos(a, P, qN, rN);  // position of `next`
     const bool write_ab = (P.n == kC) && a.has_ab;
     const long next = chunk + gridDim.x;
 
@@ -583,37 +641,44 @@ __global__ void __launch_bounds__(128, 2)
       const int t = tid & (kC - 1);
       const bool isW = tid < kC;
       uint8_t* opT = sm + kScr + (isW ? 0 : 16384);  // [half][64 rows t][128 B]
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t x[64];
-        const uint32_t col = (isW ? 0 : 64) + 128 * half;
-        tc::tmem_ld32(lane_addr + col, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
-        tc::tmem_ld32(lane_addr + col + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
-        tc::tmem_wait_ld();
+      // the row's 128 columns (K half 0: 0-63, half 1: 128-191; V at +64) in pieces of 16;
+      // the next piece's tensor-memory load is in flight while one is converted and
+      // stored, and the first one while D K is built
+      const uint32_t col0 = isW ? 0 : 64;
+      uint32_t x[2][16];
+      tmem_ld16(lane_addr + col0, x[0]);
+      if (!kChan) {
+        // D K: row t, columns 64 half .. 64 half + 63 (warps 0-1 the first half, 2-3 the second)
+        const float dt = dk_s[t];
+        const int half = tid >> 6;
 #pragma unroll
         for (int c8 = 0; c8 < 8; ++c8) {
-          uint4 w;
-          w.x = tc::pack_bf16x2(__uint_as_float(x[8 * c8 + 0]), __uint_as_float(x[8 * c8 + 1]));
-          w.y = tc::pack_bf16x2(__uint_as_float(x[8 * c8 + 2]), __uint_as_float(x[8 * c8 + 3]));
-          w.z = tc::pack_bf16x2(__uint_as_float(x[8 * c8 + 4]), __uint_as_float(x[8 * c8 + 5]));
-          w.w = tc::pack_bf16x2(__uint_as_float(x[8 * c8 + 6]), __uint_as_float(x[8 * c8 + 7]));
-          *(uint4*)(opT + half * 8192 + swz(t, c8)) = w;
+          const uint4 kw = *(const uint4*)(sm + kKV + half * 16384 + swz(t, c8));
+          const uint32_t kk[4] = {kw.x, kw.y, kw.z, kw.w};
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) w[e] = tc::pack_bf16x2(dt * tc::bf16lo(kk[e]), dt * tc::bf16hi(kk[e]));
+          *(uint4*)(sm + kTT + half * 8192 + swz(t, c8)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
-      if (!kChan && isW) {
-        const float dt = dk_s[t];
+      tmem_wait_ld_regs(x[0]);
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
+      for (int pc = 0; pc < 8; ++pc) {
+        const int cur = pc & 1;
+        if (pc + 1 < 8)
+          tmem_ld16(lane_addr + col0 + 128 * ((pc + 1) >> 2) + 16 * ((pc + 1) & 3), x[cur ^ 1]);
+        const int half = pc >> 2;
 #pragma unroll
-          for (int c8 = 0; c8 < 8; ++c8) {
-            const uint4 kw = *(const uint4*)(sm + kKV + half * 16384 + swz(t, c8));
-            const uint32_t kk[4] = {kw.x, kw.y, kw.z, kw.w};
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) w[e] = tc::pack_bf16x2(dt * tc::bf16lo(kk[e]), dt * tc::bf16hi(kk[e]));
-            *(uint4*)(sm + kTT + half * 8192 + swz(t, c8)) = make_uint4(w[0], w[1], w[2], w[3]);
-          }
+        for (int c = 0; c < 2; ++c) {
+          const int c8 = 2 * (pc & 3) + c;
+          uint4 w;
+          w.x = tc::pack_bf16x2(__uint_as_float(x[cur][8 * c + 0]), __uint_as_float(x[cur][8 * c + 1]));
+          w.y = tc::pack_bf16x2(__uint_as_float(x[cur][8 * c + 2]), __uint_as_float(x[cur][8 * c + 3]));
+          w.z = tc::pack_bf16x2(__uint_as_float(x[cur][8 * c + 4]), __uint_as_float(x[cur][8 * c + 5]));
+          w.w = tc::pack_bf16x2(__uint_as_float(x[cur][8 * c + 6]), __uint_as_float(x[cur][8 * c + 7]));
+          *(uint4*)(opT + half * 8192 + swz(t, c8)) = w;
         }
+        if (pc + 1 < 8) tmem_wait_ld_regs(x[cur ^ 1]);
       }
       tc::fence_async_smem();
       tc::tc_fence_before();
@@ -622,14 +687,6 @@ __global__ void __launch_bounds__(128, 2)
     const bool mma34 = ok && write_ab;
     if (ok && tid == 0) {
       tc::tc_fence_after();
-      if (a.has_wu) {
-        const int y = (int)(chunk * kC);
-        tc::tma_store_2d(&tmWb, sm + kScr, 0, y);
-        tc::tma_store_2d(&tmWb, sm + kScr + 8192, 64, y);
-        tc::tma_store_2d(&tmUb, sm + kScr + 16384, 0, y);
-        tc::tma_store_2d(&tmUb, sm + kScr + 16384 + 8192, 64, y);
-        tc::bulk_commit();
-      }
       // kChan: Kc has landed in the T-operand buffer
       bool kc_ok = true;
       if (kChan && kc_pending) {
@@ -650,14 +707,23 @@ __global__ void __launch_bounds__(128, 2)
         }
         tc::mma_commit(&bars[3]);
       }
+      // Wb/Ub leave from the same tiles MMA3/4 read (both only read them)
+      if (a.has_wu) {
+        const int y = (int)(chunk * kC);
+        tc::tma_store_2d(&tmWb, sm + kScr, 0, y);
+        tc::tma_store_2d(&tmWb, sm + kScr + 8192, 64, y);
+        tc::tma_store_2d(&tmUb, sm + kScr + 16384, 0, y);
+        tc::tma_store_2d(&tmUb, sm + kScr + 16384 + 8192, 64, y);
+        tc::bulk_commit();
+      }
       // the K/V tile is no longer read (MMA2 done, D K built): fetch the next chunk's
       if (next < a.total) {
-        load_kv<kChan>(sm, &tmK, &tmV, &bars[0], a, chunk_pos(a, next), next);
+        load_kv<kChan>(sm, &tmK, &tmV, &bars[0], a, Pn, next);
         load_pending = true;
         load_parity = (it + 1) & 1;
       }
     }
-    if (ok && tid < kC && next < a.total) load_ab<kChan>(a, chunk_pos(a, next), tid, pa, pb);
+    if (ok && tid < kC && next < a.total) load_ab<kChan>(a, Pn, tid, pa, pb);
     if (mma34) {
       const bool m3 = tid == 0 ? tc::mbar_wait(&bars[3], ph3 & 1, abort_s) : true;
       ++ph3;
@@ -671,29 +737,39 @@ __global__ void __launch_bounds__(128, 2)
       tc::tc_fence_after();
       const int r = tid;
       const float gC = kChan ? a.gC[chunk * kD + r] : __expf(ell_s[kC - 1]);
+      // 16 columns at a time; the next 16 columns' tensor-memory loads are in flight
+      // while the current ones are converted and stored
+      uint32_t x[2][16], y[2][16];
+      tmem_ld16(lane_addr, x[0]);
+      tmem_ld16(lane_addr + 128, y[0]);
+      tmem_wait_ld_regs(x[0], y[0]);
 #pragma unroll
-      for (int cc = 0; cc < kD; cc += 32) {
-        uint32_t x[32], y[32];
-        tc::tmem_ld32(lane_addr + cc, x);
-        tc::tmem_ld32(lane_addr + 128 + cc, y);
-        tc::tmem_wait_ld();
+      for (int k = 0; k < kD / 16; ++k) {
+        const int cur = k & 1;
+        if (k + 1 < kD / 16) {
+          tmem_ld16(lane_addr + 16 * (k + 1), x[cur ^ 1]);
+          tmem_ld16(lane_addr + 128 + 16 * (k + 1), y[cur ^ 1]);
+        }
+        const int cc = 16 * k;
         const int half = cc >> 6;
         uint8_t* bst = sm + (half ? kX : kTT);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < 2; ++q) {
           const int c8 = ((cc & 63) >> 3) + q;
           uint32_t wa[4], wb[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int c = cc + 8 * q + 2 * e;
-            const float a0 = (r == c ? gC : 0.0f) - __uint_as_float(x[8 * q + 2 * e]);
-            const float a1 = (r == c + 1 ? gC : 0.0f) - __uint_as_float(x[8 * q + 2 * e + 1]);
+            const float a0 = (r == c ? gC : 0.0f) - __uint_as_float(x[cur][8 * q + 2 * e]);
+            const float a1 = (r == c + 1 ? gC : 0.0f) - __uint_as_float(x[cur][8 * q + 2 * e + 1]);
             wa[e] = tc::pack_bf16x2(a0, a1);
-            wb[e] = tc::pack_bf16x2(__uint_as_float(y[8 * q + 2 * e]), __uint_as_float(y[8 * q + 2 * e + 1]));
+            wb[e] = tc::pack_bf16x2(__uint_as_float(y[cur][8 * q + 2 * e]),
+                                    __uint_as_float(y[cur][8 * q + 2 * e + 1]));
           }
           *(uint4*)(sm + kScr + half * 16384 + swz(r, c8)) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
           *(uint4*)(bst + swz(r, c8)) = make_uint4(wb[0], wb[1], wb[2], wb[3]);
         }
+        if (k + 1 < kD / 16) tmem_wait_ld_regs(x[cur ^ 1], y[cur ^ 1]);
       }
       tc::fence_async_smem();
       tc::tc_fence_before();
