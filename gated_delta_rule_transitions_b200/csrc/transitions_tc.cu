@@ -76,13 +76,6 @@ struct TransTcArgs {
 
 __device__ __forceinline__ int swz(int row, int chunk) { return row * 128 + ((chunk ^ (row & 7)) << 4); }
 
-#ifndef HLA_TRANS_WARP_MMA
-#define HLA_TRANS_WARP_MMA 1
-#endif
-// Off-diagonal blocks of the inverse on warp-level tensor-core products (tf32
-// inputs, float32 accumulation) instead of CUDA-core dot products.
-constexpr bool kWarpMma = HLA_TRANS_WARP_MMA != 0;
-
 #ifndef HLA_TRANS_DECAY_PRODUCT
 #define HLA_TRANS_DECAY_PRODUCT 1
 #endif
@@ -485,8 +478,9 @@ __global__ void __launch_bounds__(128, 2)
     ok = tc::bar_all(1, 128, ok);
     // Off-diagonal blocks.  With L'_ik = U_ii L_ik (k < i),  U_ij = -sum_{k=j}^{i-1} L'_ik U_kj,
     // one level (i - j = 1, 2, 3) after the other.
-    if (kWarpMma) {
-      // warp-level products: a unit is one 16 x 8 half (column half nh) of a block
+    {
+      // warp-level products (tf32 inputs, float32 accumulation): a unit is one 16 x 8
+      // half (column half nh) of a block
       if (ok) {
         // L'_ik for (i, k) = (1,0) (2,0) (2,1) (3,0) (3,1) (3,2): 12 units, 3 per warp
 #pragma unroll
@@ -530,61 +524,6 @@ __global__ void __launch_bounds__(128, 2)
         float acc[4];
         warp_mma_rows16<48>(acc, Xsm + 32 * kXP, kXP, Usm + 8 * warp, kLP, lane);
         warp_store_rows16(Usm + 48 * kLP + 8 * warp, kLP, acc, -1.0f, lane);
-      }
-      ok = tc::bar_all(1, 128, ok);
-    }
-    const int cc16 = tid & 15, tb = tid >> 4;
-    if (!kWarpMma && ok) {
-#pragma unroll
-      for (int ib = 1; ib < 4; ++ib) {
-        float ua[16], ub[16];  // U_ii rows tb, tb + 8
-#pragma unroll
-        for (int u4 = 0; u4 < 16; u4 += 4) {
-          const float4 x0 = *(const float4*)(Usm + (16 * ib + tb) * kLP + 16 * ib + u4);
-          const float4 x1 = *(const float4*)(Usm + (16 * ib + tb + 8) * kLP + 16 * ib + u4);
-          ua[u4] = x0.x; ua[u4 + 1] = x0.y; ua[u4 + 2] = x0.z; ua[u4 + 3] = x0.w;
-          ub[u4] = x1.x; ub[u4 + 1] = x1.y; ub[u4 + 2] = x1.z; ub[u4 + 3] = x1.w;
-        }
-#pragma unroll
-        for (int mb = 0; mb < ib; ++mb) {
-          float s0 = 0.0f, s1 = 0.0f;
-#pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            const float l = Lsm[(16 * ib + u) * kLP + 16 * mb + cc16];
-            s0 = fmaf(ua[u], l, s0);
-            s1 = fmaf(ub[u], l, s1);
-          }
-          Xsm[(16 * ib - 16 + tb) * kXP + 16 * mb + cc16] = s0;
-          Xsm[(16 * ib - 16 + tb + 8) * kXP + 16 * mb + cc16] = s1;
-        }
-      }
-    }
-    if (!kWarpMma) ok = tc::bar_all(1, 128, ok);
-#pragma unroll
-    for (int lev = 1; lev < 4 && !kWarpMma; ++lev) {
-      if (ok) {
-#pragma unroll
-        for (int jb = 0; jb + lev < 4; ++jb) {
-          const int ib = jb + lev;
-          const float* x0 = Xsm + (16 * ib - 16 + tb) * kXP;
-          const float* x1 = Xsm + (16 * ib - 16 + tb + 8) * kXP;
-          float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f, s3 = 0.0f;
-#pragma unroll
-          for (int s4 = 16 * jb; s4 < 16 * ib; s4 += 4) {
-            const float4 a4 = *(const float4*)(x0 + s4);
-            const float4 b4 = *(const float4*)(x1 + s4);
-            const float u0 = Usm[(s4 + 0) * kLP + 16 * jb + cc16];
-            const float u1 = Usm[(s4 + 1) * kLP + 16 * jb + cc16];
-            const float u2 = Usm[(s4 + 2) * kLP + 16 * jb + cc16];
-            const float u3 = Usm[(s4 + 3) * kLP + 16 * jb + cc16];
-            s0 = fmaf(a4.x, u0, fmaf(a4.y, u1, s0));
-            s1 = fmaf(a4.z, u2, fmaf(a4.w, u3, s1));
-            s2 = fmaf(b4.x, u0, fmaf(b4.y, u1, s2));
-            s3 = fmaf(b4.z, u2, fmaf(b4.w, u3, s3));
-          }
-          Usm[(16 * ib + tb) * kLP + 16 * jb + cc16] = -(s0 + s1);
-          Usm[(16 * ib + tb + 8) * kLP + 16 * jb + cc16] = -(s2 + s3);
-        }
       }
       ok = tc::bar_all(1, 128, ok);
     }
