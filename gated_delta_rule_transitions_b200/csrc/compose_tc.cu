@@ -53,7 +53,18 @@ struct ComposeTcArgs {
   int slot_mult, n_slots;
 };
 
-// Walks the merged ascending active lists of the two chains.
+#ifndef HLA_COMPOSE_LIST_PREFETCH
+#define HLA_COMPOSE_LIST_PREFETCH 1
+#endif
+constexpr bool kListPrefetch = HLA_COMPOSE_LIST_PREFETCH != 0;
+
+__device__ __forceinline__ void prefetch_l1(const void* p) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
+}
+
+// Walks the merged ascending active lists of the two chains.  The list entries are
+// read one step at a time by one thread; with kListPrefetch the lines 32 entries
+// ahead are requested into L1 as the walk goes, so that each step's reads hit L1.
 struct Sched {
   const int32_t* idx[2];
   const float* g[2];
@@ -74,6 +85,15 @@ struct Sched {
         idx[k] = a.act_idx + row * a.N;
         g[k] = a.act_g + row * a.N;
         cnt[k] = a.act_cnt[row];
+        if (kListPrefetch) {
+          // the first two lines of each list (entries 0-63 that exist)
+          prefetch_l1(idx[k]);
+          prefetch_l1(g[k]);
+          if (cnt[k] > 32) {
+            prefetch_l1(idx[k] + 32);
+            prefetch_l1(g[k] + 32);
+          }
+        }
       } else {
         idx[k] = nullptr;
         g[k] = nullptr;
@@ -99,7 +119,14 @@ struct Sched {
   }
   __device__ void advance() {
     for (int k = 0; k < 2; ++k)
-      if (act[k]) ++p[k];
+      if (act[k]) {
+        ++p[k];
+        // one 128-byte line holds 32 entries: entering a line, ask for the one after it
+        if (kListPrefetch && (p[k] & 31) == 0 && p[k] + 32 < cnt[k]) {
+          prefetch_l1(idx[k] + p[k] + 32);
+          prefetch_l1(g[k] + p[k] + 32);
+        }
+      }
   }
 };
 
