@@ -328,11 +328,17 @@ __global__ void __launch_bounds__(kThreads, 3)
   }
   __syncthreads();
   if (tid == 0 && *abort_s) report_device_error(kErrMbarTimeout);
+  // the stream kernel, launched as this grid's programmatic dependent, may start its
+  // CTAs now (it waits for this grid's completion before reading anything)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 __global__ void __launch_bounds__(kThreads, 2)
     decode_stream_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                          DecodeArgs a) {
+  // launched as the gate kernel's programmatic dependent: everything below reads its
+  // results (or the step's appended token), so wait for that grid to complete first
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* ring = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint64_t* full = (uint64_t*)(ring + kUnits * kUnit);
@@ -653,7 +659,20 @@ cudaError_t launch_decode_stream(const DecodeArgs& a, cudaStream_t s) {
   const size_t smem = 1024 + kUnits * kUnit + 2 * kUnits * 8 + (4 * kD + 16) * 4;
   e = cudaFuncSetAttribute(decode_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  decode_stream_kernel<<<a.B * a.H, kThreads, smem, s>>>(tmA, tmB, a);
+  // programmatic dependent launch: the stream CTAs are scheduled while the gate grid
+  // drains and wait (griddepcontrol.wait) for it to complete
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.B * a.H);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, decode_stream_kernel, tmA, tmB, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
