@@ -85,8 +85,8 @@ NCU_TRAFFIC = {
     "compose": (2.0470e9, {"compose_tc.cu": "4b50659baac7102a", "tc_common.cuh": "c10beda371c1dd4b"}),
     # gate + stream kernels of one step, captured on 4 (dense) and 8 (planted) of the
     # 64 sequences and scaled by the sequence count (the traffic is per sequence)
-    "decode_main": (3.4638e10, {"decode_stream.cu": "983ccd7e646f1584", "tc_common.cuh": "c10beda371c1dd4b"}),
-    "decode_planted": (5.447e8, {"decode_stream.cu": "983ccd7e646f1584", "tc_common.cuh": "c10beda371c1dd4b"}),
+    "decode_main": (3.4638e10, {"decode_stream.cu": "8916b84931f22b4f", "tc_common.cuh": "c10beda371c1dd4b"}),
+    "decode_planted": (5.447e8, {"decode_stream.cu": "8916b84931f22b4f", "tc_common.cuh": "c10beda371c1dd4b"}),
 }
 
 # Datasheet figures of one B200, reported beside the measured denominators: dense
