@@ -176,6 +176,29 @@ def test_gdn_chunk_transitions(hla, dtype, d):
                     P.check_bf16(Bm[b, h, c], Br, "transition", tol=1e-2)
 
 
+def test_gdn_chunk_transitions_many_heads(hla):
+    """More chunks than persistent CTAs with few chunks per head (N = 3, 150 heads):
+    every CTA steps through several (b, h) positions, wrapping across sequences."""
+    w = syn.TINY_F32.with_(dtype="bf16", d=128, B=3, H=50, T=64 * 2 + 5)
+    inp = P.gpu_inputs(w)
+    B, H, T = 3, 50, w.T
+    cfg = hla.make_config(B, H, T, 64, 128, "bf16")
+    g = P.to_cuda(inp)
+    A = torch.empty((B, H, T // 64, 128, 128), dtype=torch.bfloat16, device="cuda")
+    Bm = torch.empty_like(A)
+    hla.gdn_chunk_transitions(cfg, g["k"], g["v"], g["alpha"], g["beta"], A, Bm)
+    torch.cuda.synchronize()
+    A, Bm = P.np64(A), P.np64(Bm)
+    for b in range(B):
+        for h in (0, 1, 17, H - 1):
+            for c in range(T // 64):
+                sl = slice(64 * c, 64 * c + 64)
+                Ar, Br = ho.chunk_transition(P.np64(inp["k"][b, sl, h]), P.np64(inp["v"][b, sl, h]),
+                                             P.np64(inp["alpha"][b, sl, h]), P.np64(inp["beta"][b, sl, h]))
+                P.check_bf16(A[b, h, c], Ar, "transition", tol=1e-2)
+                P.check_bf16(Bm[b, h, c], Br, "transition", tol=1e-2)
+
+
 def test_gdn_chunk_transitions_strong_decay(hla):
     """Chunks whose accumulated decay exceeds e^80 (the pair decays then come from one
     exponential per pair, not from per-token factors) next to weakly decaying ones.
