@@ -162,7 +162,7 @@ __global__ void __launch_bounds__(128) decode_main_kernel(DecodeArgs a) {
 // Key pool of the closing chunk into the cache (only sequences whose open chunk
 // becomes full this step).  grid B*H, block D.
 template <int D, typename Tio>
-__global__ void decode_close_pool_kernel(DecodeArgs a) {
+__device__ __forceinline__ void close_pool(const DecodeArgs& a) {
   const int bh = blockIdx.x;
   const int b = bh / a.H;
   const int tid = threadIdx.x;
@@ -189,7 +189,20 @@ __global__ void decode_close_pool_kernel(DecodeArgs a) {
   }
 }
 
+// Launched as the closing transition's programmatic dependent: the two read the same
+// open-chunk rows and counters and write disjoint outputs, so they may overlap.  Every
+// CTA waits for the transition grid before it exits, so this grid completes after it;
+// the counters kernel (this grid's dependent) waits for this grid alone.
+template <int D, typename Tio>
+__global__ void decode_close_pool_kernel(DecodeArgs a) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  close_pool<D, Tio>(a);
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 __global__ void decode_counters_kernel(int B, int C, int max_chunks, int32_t* n_chunks, int32_t* m_partial) {
+  // the pool kernel (and through it the closing transition) read the counters
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b >= B) return;
   const int m = m_partial[b] + 1;
@@ -329,10 +342,22 @@ static cudaError_t launch_close(const DecodeArgs& a, cudaStream_t s) {
   // Chunks longer than one 64-token WY tile close by the token rule (no workspace).
   cudaError_t e = (a.C > 64 || a.alpha_vec) ? launch_transitions_token(t, s) : launch_transitions(t, s);
   if (e != cudaSuccess) return e;
-  decode_close_pool_kernel<D, Tio><<<a.B * a.H, D, 0, s>>>(a);
-  e = cudaGetLastError();
+  // the pool and counters kernels are programmatic dependents of the kernel before each
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.B * a.H);
+  cfg.blockDim = dim3(D);
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, decode_close_pool_kernel<D, Tio>, a);
   if (e != cudaSuccess) return e;
-  decode_counters_kernel<<<(a.B + 127) / 128, 128, 0, s>>>(a.B, a.C, a.max_chunks, a.n_chunks, a.m_partial);
+  cfg.gridDim = dim3((a.B + 127) / 128);
+  cfg.blockDim = dim3(128);
+  e = cudaLaunchKernelEx(&cfg, decode_counters_kernel, a.B, a.C, a.max_chunks, a.n_chunks, a.m_partial);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

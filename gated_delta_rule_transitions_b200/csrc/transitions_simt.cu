@@ -20,6 +20,9 @@ namespace hla {
 
 template <int D, typename Tio>
 __global__ void __launch_bounds__(256) transitions_simt_kernel(TransArgs a) {
+  // a programmatic dependent launched after this grid (the decode close's pool kernel)
+  // may be scheduled at once; it waits for this grid before it completes
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   constexpr int C = 64;
   constexpr int DP = D + 1;
   constexpr int CP = C + 1;

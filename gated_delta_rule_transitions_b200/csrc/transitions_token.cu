@@ -45,6 +45,9 @@ constexpr int smem_floats() {
 //   s <- s o alpha_t,  then  s <- s - (beta_t (s . k_t) - beta_t v_t[r]) k_t.
 template <int D, typename Tio, bool kChan>
 __global__ void __launch_bounds__(2 * D, 2) transitions_token_kernel(TransArgs a) {
+  // a programmatic dependent launched after this grid (the decode close's pool kernel)
+  // may be scheduled at once; it waits for this grid before it completes
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   using namespace token_rows;
   constexpr int E = D / 8;   // columns per thread
   constexpr int M = D / 32;  // 16-byte groups per thread
