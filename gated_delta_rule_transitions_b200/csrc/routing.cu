@@ -123,6 +123,9 @@ __global__ void __launch_bounds__(64, 16) pool_kernel(const Tin* __restrict__ x0
   const float inv_tau = __fdiv_rn(1.0f, tau);
   const int t0 = c * C;
   const int n = min(C, T - t0);
+  // window representatives of a final partial chunk may start past the sequence: such
+  // windows are never read (only complete chunks are keys), so nothing is pooled
+  if (n <= 0) return;
   const Tin* col = x + ((size_t)b * T + t0) * HD + ch0;
   float s0 = 0.0f, s1 = 0.0f, m0, m1;
   if constexpr (kBf16) {
@@ -244,6 +247,11 @@ __global__ void __launch_bounds__(32 * kTileWarps) pool_tile_kernel(PoolTileArgs
     __syncwarp();
     const uint32_t* w = words + cur * kTileRows * 32 + lane;
     const int n = n_cur;
+    if (n <= 0) {
+      // a window past the end of the sequence (a final partial chunk): never read
+      n_cur = n_next;
+      continue;
+    }
     uint32_t hi = w[0], lo = hi;
     for (int t = 1; t < n; ++t) {
       hi = bf16x2_max(hi, w[t * 32]);
